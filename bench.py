@@ -1,0 +1,450 @@
+"""Benchmark: one DSA decode layer-step at the native 1,048,576-token context.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path (lightning indexer over every cached
+key -> top-2048 selection -> sparse GQA4 attention with sink -> split combine)
+for batch 1, one query token, context 1,048,576, on synthetic seeded inputs.
+Each rank runs its own replica of the workload (the steps are independent
+problems: weak scaling, no data-path collective); ``value`` is the tokens all
+ranks decoded divided by the slowest rank's device time.
+
+L2 is flushed (256 MB write) between timed steps, outside the timed events.
+Per-stage CUDA events recorded by the library itself give the indexer's
+duration for the roofline.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA layer-step µs & tok/s at 1M ctx; indexer HBM GB/s vs B200 peak"
+WORKLOAD = "ctx_1m"
+L_CTX = 1048576
+TOP_K = 2048
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+INDEXER_SRC = os.path.join(ROOT, "local_attention_decode_b200", "csrc", "indexer.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "indexer_ctx_1m_traffic.json")
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def indexer_bytes(L: int, T: int) -> int:
+    """Algorithmic bytes of one indexer launch for one sequence: every visible
+    key read once (128 B of e4m3 codes + 4 B scale), one fp32 score written per
+    (query token, key), and the query block (T x (2 KiB codes + 128 B of
+    scales and weights))."""
+    return L * (128 + 4) + T * L * 4 + T * (16 * 128 + 16 * 8)
+
+
+def gathered_bytes(T: int, top_k: int, G: int = 4) -> int:
+    """Backbone K/V bytes gathered by the sparse attention: top_k rows of G heads x (192 + 128) bf16."""
+    return T * top_k * G * (192 + 128) * 2
+
+
+def recorded_traffic():
+    """DRAM bytes per indexer launch from the committed ncu summary, if it was
+    taken on the current indexer source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        sha = hashlib.sha256(open(INDEXER_SRC, "rb").read()).hexdigest()
+        if d.get("indexer_cu_sha256") == sha:
+            return int(d["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.002)
+
+    def start(self):
+        if self.nv is not None:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.nv is not None:
+            self._stop.set()
+            if self._t:
+                self._t.join()
+            self._sample()
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------- multi-rank helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def throughput(tokens_per_rank_step: int, steps: int, world: int, slowest_s: float) -> float:
+    """Whole-job tokens per second: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / slowest_s
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import local_attention_decode_b200 as dsa
+    from workloads import CONFIGS, make_decode_workload
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS[WORKLOAD]
+    wl = make_decode_workload(device=dev, **cfg)
+    B, T = wl.B, wl.T
+    L = wl.layout.seq_lens[0]
+    sm_scale = 1.0 / math.sqrt(192)
+    kv = dsa.KV(k=wl.K, v=wl.V, index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G,
+                seq_stride=wl.layout.seq_stride, num_rows=wl.layout.num_rows)
+    O = torch.empty((B, T, 64, 128), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((B, T, TOP_K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, T), dtype=torch.int32, device=dev)
+    ws = dsa.alloc_workspace(dsa.OP_LAYER, B, T, L, TOP_K, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)   # materialise the handle
+        return evs
+
+    def step(events=None):
+        dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, L, TOP_K, wl.sink, sm_scale, O,
+                             None, idx, cnt, ws, stage_events=events)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st, _ = dsa.dsa_check_device_status(ws)
+    if st != dsa.DSA_OK:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    K = args.steps
+    stage = [new_events(5) for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for i in range(K):
+        flush.zero_()
+        step(stage[i])
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clocks = sampler.stop()
+
+    step_ms = [stage[i][0].elapsed_time(stage[i][4]) for i in range(K)]
+    idx_ms = [stage[i][0].elapsed_time(stage[i][1]) for i in range(K)]
+    topk_ms = [stage[i][1].elapsed_time(stage[i][2]) for i in range(K)]
+    attn_ms = [stage[i][2].elapsed_time(stage[i][3]) for i in range(K)]
+    comb_ms = [stage[i][3].elapsed_time(stage[i][4]) for i in range(K)]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, dev)
+    st, _ = dsa.dsa_check_device_status(ws)
+    if st != dsa.DSA_OK:
+        raise RuntimeError(f"device status {st} after the timed steps")
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush)
+
+    tokens = B * T
+    value = throughput(tokens, K, world, total_s)
+    peak, peak_kind = measured_peaks()
+    idx_avg_s = sum(idx_ms) / K / 1e3
+    ib = indexer_bytes(L, T)
+    achieved = ib / idx_avg_s / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_s * 1e3 / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
+        "data": "synthetic",
+        "config": {
+            "workload": "ctx_1m: DSA decode layer-step, batch 1, 1 query token at position 1,048,575, "
+                        "context 1,048,576, top-2048, 64 Q heads / 4 KV heads (GQA4), qk 192, v 128, sink",
+            "batch": B, "query_tokens": T, "context": L, "top_k": TOP_K, "seed": cfg["seed"],
+            "needles": cfg["n_needles"], "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (256 MB write outside the timed events)",
+        },
+        "us_per_layer_step": total_s * 1e6 / K,
+        "stage_us_median": {
+            "indexer": statistics.median(idx_ms) * 1e3, "topk": statistics.median(topk_ms) * 1e3,
+            "attention": statistics.median(attn_ms) * 1e3, "combine": statistics.median(comb_ms) * 1e3,
+        },
+        "layer_step_byte_roofline_us": {
+            "bytes": ib + gathered_bytes(T, TOP_K),
+            "at_measured_peak": (ib + gathered_bytes(T, TOP_K)) / (peak * 1e9) * 1e6,
+            "at_8TBps_nominal": (ib + gathered_bytes(T, TOP_K)) / (NOMINAL_HBM_GBS * 1e9) * 1e6,
+        },
+        "roofline": {
+            "kernel": "indexer_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+            "frac_of_8TBps_nominal": achieved / NOMINAL_HBM_GBS,
+            "traffic": recorded_traffic(), "algorithmic_bytes_per_launch": ib,
+            "avg_launch_us": idx_avg_s * 1e6,
+        },
+        "e2e": e2e,
+        "gpu_launches": 4 * K,
+        "clocks": clocks,
+    }
+    return line
+
+
+def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
+    """Same metric through the public API with host buffers: per step the new
+    token's inputs (index query + scales + weights, backbone query, position,
+    and its index-key / K / V cache row) go host -> device from pinned memory,
+    the layer-step runs, and the output and selection come back to the host."""
+    B, T = wl.B, wl.T
+    L = wl.layout.seq_lens[0]
+    row = L - 1
+    h_q8 = wl.q8.cpu().pin_memory()
+    h_qs = wl.q_scale.cpu().pin_memory()
+    h_w = wl.w.cpu().pin_memory()
+    h_Q = wl.Q.cpu().pin_memory()
+    h_pos = wl.q_pos.cpu().pin_memory()
+    h_k8 = wl.k8[row].cpu().pin_memory()
+    h_ks = wl.k_scale[row:row + 1].cpu().pin_memory()
+    h_K = wl.K[row].cpu().pin_memory()
+    h_V = wl.V[row].cpu().pin_memory()
+    d_q8, d_qs, d_w = torch.empty_like(wl.q8), torch.empty_like(wl.q_scale), torch.empty_like(wl.w)
+    d_Q, d_pos = torch.empty_like(wl.Q), torch.empty_like(wl.q_pos)
+    O = torch.empty((B, T, 64, 128), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((B, T, TOP_K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, T), dtype=torch.int32, device=dev)
+    h_O = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    h_idx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    h_in = [h_q8, h_qs, h_w, h_Q, h_pos, h_k8, h_ks, h_K, h_V]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_O.numel() * h_O.element_size() + h_idx.numel() * h_idx.element_size()
+
+    def step():
+        d_q8.copy_(h_q8, non_blocking=True)
+        d_qs.copy_(h_qs, non_blocking=True)
+        d_w.copy_(h_w, non_blocking=True)
+        d_Q.copy_(h_Q, non_blocking=True)
+        d_pos.copy_(h_pos, non_blocking=True)
+        wl.k8[row].copy_(h_k8, non_blocking=True)
+        wl.k_scale[row:row + 1].copy_(h_ks, non_blocking=True)
+        wl.K[row].copy_(h_K, non_blocking=True)
+        wl.V[row].copy_(h_V, non_blocking=True)
+        dsa.dsa_layer_decode(d_q8, d_qs, d_w, d_Q, kv, d_pos, L, TOP_K, wl.sink, sm_scale, O, None, idx, cnt, ws)
+        h_O.copy_(O, non_blocking=True)
+        h_idx.copy_(idx, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
+    import torch.distributed as dist
+    world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
+    return {"value": throughput(B * T, K, world, total_s), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K}
+
+
+# ------------------------------------------------------- CPU oracle timing
+def oracle_sample(n_keys: int, seed: int = 2):
+    """Time the CPU oracle on a contiguous sample of n_keys keys of the 1M
+    workload's recipe (indexer + top-k over the sample, attention over 2,048
+    keys) and scale the indexer and selection linearly to 1,048,576 keys.
+    Returns (seconds per full layer-step, seconds measured)."""
+    import numpy as np
+    import oracle
+    from workloads import bits16, make_decode_workload
+    wl = make_decode_workload(seed=seed, seq_lens=[max(n_keys, TOP_K)], T=1, n_needles=4, needle_mode="zipf")
+    n = wl.layout.seq_lens[0]
+    t0 = time.perf_counter()
+    s = oracle.indexer_scores(wl.q8[0].numpy(), wl.q_scale[0].numpy(), wl.w[0].numpy(), wl.k8.numpy(),
+                              wl.k_scale.numpy(), wl.q_pos[0].numpy())
+    sel, c = oracle.topk(s[0], TOP_K)
+    t1 = time.perf_counter()
+    sel = sel[:c] if c else np.arange(min(n, TOP_K), dtype=np.int32)
+    oracle.gqa_attention(bits16(wl.Q[0, 0]), bits16(wl.K), bits16(wl.V), sel, wl.sink.numpy(),
+                         1.0 / math.sqrt(192))
+    t2 = time.perf_counter()
+    full = (t1 - t0) * (L_CTX / n) + (t2 - t1)
+    return full, t2 - t0
+
+
+def cpu_baseline_line(target_s: float = 15.0):
+    n = 16384
+    full, spent = oracle_sample(n)
+    # grow the sample toward the target CPU time
+    per_key = max(1e-7, (spent - 0.3) / n)
+    n2 = int(min(L_CTX, max(n, (target_s - spent) / per_key)))
+    if n2 > n:
+        full, spent2 = oracle_sample(n2)
+        n, spent = n2, spent + spent2
+    return {"value": 1.0 / full, "unit": "tok/s", "cores": 1, "kind": "oracle",
+            "sample": f"one layer-step of the ctx_1m recipe on the first {n} keys (indexer + top-2048 over them, "
+                      f"attention over 2,048 keys), indexer and selection time scaled by {L_CTX}/{n}; "
+                      f"single-threaded C oracle in double; {spent:.1f} s of CPU"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    budget_s = 150.0
+    steps = args.steps + args.warmup
+    per_step = budget_s / max(1, steps)
+    n = int(max(TOP_K, min(65536, per_step / 1.1e-4)))
+    times = []
+    for i in range(steps):
+        full, _ = oracle_sample(n)
+        if i >= args.warmup:
+            times.append(full)
+    total = sum(times)
+    value = len(times) / total
+    cores = 1
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "ctx_1m: DSA decode layer-step, batch 1, 1 query token, context 1,048,576, "
+                               "top-2048, GQA4, sink", "context": L_CTX, "top_k": TOP_K},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the CPU oracle on the first {n} keys of the ctx_1m recipe, "
+                                   f"indexer and selection scaled by {L_CTX}/{n}"},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local_rank = dist_env()
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1:
+                line["cpu_baseline"] = cpu_baseline_line()
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

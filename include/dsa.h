@@ -1,0 +1,215 @@
+/*
+ * dsa.h -- C ABI of libdsa: the decode step of a DeepSeek-Sparse-Attention
+ * (DSA) layer and of a sliding-window (SWA) layer, for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources: the explainer page "Naive-N0.5-Flash: no
+ * full-attention layers, and a runtime built by AI"):
+ *   - property table: 16 index heads x 128, one shared index-key head in
+ *     fp8_e4m3; top 2,048 keys per DSA query; SWA window 128; 64 query heads,
+ *     qk head dim 192, v head dim 128; 4 KV heads on DSA layers (GQA4), 8 on
+ *     SWA layers (GQA8); native context 1,048,576.
+ *   - "Inside a DSA layer: the lightning indexer": every visible key gets one
+ *     score, relu(q_h . k) per index head combined by a per-head weight; the
+ *     main heads attend only to the top-scoring 2,048 keys; the SWA heads carry
+ *     a sink column in the softmax.
+ *   - "What 'no full-attention layers' means": SWA masks keys with
+ *     query_offset - key_offset >= window; DSA takes the first top_k entries
+ *     of an argsort of the scores (ties toward the lower position, "How much
+ *     of this did AI actually build?").
+ *
+ * Conventions shared by every call
+ *   - All pointers named as device pointers must point to device (or managed)
+ *     memory of the current CUDA device.  The caller owns every buffer; the
+ *     library allocates nothing.  Scratch memory is the caller's workspace
+ *     (`ws`, `ws_bytes`); `dsa_workspace_size` gives the size each call needs.
+ *     A workspace must be zero when first used (`dsa_workspace_init`); the
+ *     calls leave it zeroed again when they finish.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream).  Host-side argument checks return before anything is
+ *     enqueued.  Device-side checks (positions out of range, a bounded wait
+ *     that ran out) set a status word in the workspace instead of faulting;
+ *     read it with `dsa_check_device_status`.
+ *   - Return value: DSA_OK or a DSA_ERR_* code; `dsa_last_error()` gives a
+ *     thread-local message for the last failing call on this thread.  No C++
+ *     exception crosses this boundary.
+ *   - Calls that use the same workspace must not overlap in time.
+ *   - Positions are 0-based int32.  Query (b, t) sits at position
+ *     q_pos[b*T + t] and sees keys 0..q_pos[b*T + t] of its sequence.
+ *
+ * Tensor layouts (row-major, innermost last; "rows" are KV-cache rows, see
+ * dsa_kv_t):
+ *   q8       uint8 (e4m3 codes) [B][T][16][128]   index queries
+ *   q_scale  float [B][T][16]                      index-query scales (> 0)
+ *   w        float [B][T][16]                      index-head weights
+ *   Q        bf16  [B][T][64][192]                 backbone queries
+ *   O        bf16  [B][T][64][128]                 attention output
+ *   lse      float [B][T][64]                      optional: natural-log
+ *            sum-exp of the logits including the sink, log(sum_i e^{s_i} + e^{sink})
+ *   scores   float [B][T][scores_stride]           indexer output
+ *   idx      int32 [B][T][top_k]                   selected positions, -1 padded
+ *   count    int32 [B][T]                          number of valid entries of idx
+ *   sink     float [64]                            optional per-head sink logits
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define DSA_OK                      0
+#define DSA_ERR_INVALID_ARG         1  /* null pointer, negative size, bad stride ... */
+#define DSA_ERR_UNSUPPORTED_SHAPE   2  /* head dims, T, top_k, page size outside what is built */
+#define DSA_ERR_WORKSPACE_TOO_SMALL 3
+#define DSA_ERR_CUDA                4  /* a CUDA runtime call failed; see dsa_last_error() */
+#define DSA_ERR_DEVICE_TIMEOUT      5  /* a bounded device-side wait ran out */
+#define DSA_ERR_DEVICE_BAD_INDEX    6  /* a device-side position/page index was out of range */
+
+/* Compile-time model dimensions (property table of the explainer page). */
+#define DSA_INDEX_HEADS 16
+#define DSA_INDEX_DIM   128
+#define DSA_Q_HEADS     64
+#define DSA_QK_DIM      192
+#define DSA_V_DIM       128
+#define DSA_MAX_TOPK    2048   /* largest top_k the selection kernel supports */
+#define DSA_MAX_T       16     /* query tokens per sequence per decode call */
+
+/* Operation ids for dsa_workspace_size. */
+#define DSA_OP_INDEXER     0
+#define DSA_OP_TOPK        1
+#define DSA_OP_SPARSE_ATTN 2
+#define DSA_OP_SWA_ATTN    3
+#define DSA_OP_LAYER       4
+
+/*
+ * KV-cache description.  One "row" holds one position of one sequence:
+ *   k            bf16  [rows][num_kv_heads][192]   backbone keys (post-RoPE)
+ *   v            bf16  [rows][num_kv_heads][128]   backbone values
+ *   index_k      uint8 [rows][128]                 e4m3 index keys
+ *   index_k_scale float [rows]                     per-row index-key scales (> 0)
+ * The row of position `pos` of sequence `b` is
+ *   contiguous (block_table == NULL): b * seq_stride + pos, pos < seq_stride
+ *   paged:  block_table[b * max_pages + pos / page_size] * page_size + pos % page_size,
+ *           pos / page_size < max_pages; page ids < num_rows / page_size.
+ * `num_rows` is the number of rows the buffers hold (bounds every access).
+ * Unused members may be NULL (e.g. index_k for the attention calls, k / v
+ * for the indexer).  All device pointers must be 16-byte aligned.
+ */
+typedef struct dsa_kv {
+    const void    *k;
+    const void    *v;
+    const void    *index_k;
+    const float   *index_k_scale;
+    int32_t        num_kv_heads;   /* G: 4 on DSA layers, 8 on SWA layers (any divisor of 64 up to 16 heads per group) */
+    int32_t        page_size;      /* paged only: rows per page, a multiple of 16 dividing 128 or a multiple of 128 */
+    int64_t        seq_stride;     /* contiguous only: rows reserved per sequence */
+    int64_t        num_rows;       /* rows held by the buffers */
+    const int32_t *block_table;    /* device int32 [B][max_pages], or NULL for contiguous */
+    int32_t        max_pages;      /* row stride of block_table */
+    int32_t        reserved;
+} dsa_kv_t;
+
+/* Thread-local message describing the last error returned on this thread. */
+const char *dsa_last_error(void);
+
+/* Writes the compiled dims {16, 128, 64, 192, 128, DSA_MAX_TOPK, DSA_MAX_T}
+ * to dims[0..n) (n <= 7) and returns DSA_OK. */
+int dsa_get_dims(int32_t *dims, int n);
+
+/* Workspace bytes that operation `op` (DSA_OP_*) needs for a call with B
+ * sequences, T query tokens each, contexts of at most Lmax positions and the
+ * given top_k (window for DSA_OP_SWA_ATTN).  Writes *bytes and returns DSA_OK,
+ * or an error for unsupported arguments. */
+int dsa_workspace_size(int op, int B, int T, int64_t Lmax, int top_k, size_t *bytes);
+
+/* Zeroes a workspace (cudaMemsetAsync on `stream`). */
+int dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then reads and clears the device status word held in
+ * the workspace.  *status receives DSA_OK, DSA_ERR_DEVICE_TIMEOUT or
+ * DSA_ERR_DEVICE_BAD_INDEX (a bitwise OR of 1 << code for each kind seen is
+ * returned in *flags if flags is not NULL).  After a device error the
+ * workspace must be re-initialised with dsa_workspace_init. */
+int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags);
+
+/*
+ * dsa_indexer_scores -- lightning-indexer scores of every visible key
+ * ("Inside a DSA layer: the lightning indexer"):
+ *   scores[b][t][s] = sum_h w[b][t][h] * max(0, q_scale[b][t][h] * index_k_scale[row(b,s)]
+ *                                             * <q8[b][t][h][:], index_k[row(b,s)][:]>)
+ * for 0 <= s <= q_pos[b][t]; the entries q_pos[b][t] < s <= max_t q_pos[b][t]
+ * are written as -infinity; entries beyond are not touched.
+ * e4m3 products, fp32 accumulation on the tensor cores.  Needs scores_stride
+ * >= Lmax >= max q_pos + 1, T <= DSA_MAX_T, q_scale and index_k_scale > 0.
+ */
+int dsa_indexer_scores(const void *q8, const float *q_scale, const float *w,
+                       const dsa_kv_t *kv, const int32_t *q_pos, int B, int T,
+                       int64_t Lmax, float *scores, int64_t scores_stride,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_topk_select -- for each query (b, t): the min(top_k, n) positions among
+ * 0..n-1 (n = q_pos[b][t] + 1) with the largest scores, equal scores broken
+ * toward the lower position, -0.0 equal to +0.0 ("What 'no full-attention
+ * layers' means": argsort(...)[:, :top_k]).  idx[b][t][:] receives the
+ * selected positions in increasing position order, padded with -1;
+ * count[b][t] = min(top_k, n).  Scores must not be NaN.  1 <= top_k <=
+ * DSA_MAX_TOPK.
+ */
+int dsa_topk_select(const float *scores, int64_t scores_stride, const int32_t *q_pos,
+                    int B, int T, int64_t Lmax, int top_k, int32_t *idx, int32_t *count,
+                    void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * sparse_gqa_attn_decode -- softmax attention of each query head over the
+ * selected key positions only ("Inside a DSA layer": the main heads gather
+ * and attend to the selected K/V), grouped-query with contiguous head groups
+ * (head h reads KV head h / (64 / G)), and an optional per-head sink logit in
+ * the denominator:
+ *   s_i = sm_scale * Q[h] . K[row(b, idx_i)][g]
+ *   O[h] = sum_i e^{s_i} V[row(b, idx_i)][g] / (sum_i e^{s_i} + e^{sink[h]})
+ * idx [B][T][top_k] (first count[b][t] entries used; each must satisfy
+ * 0 <= idx <= q_pos is NOT required, only 0 <= idx < capacity of the
+ * sequence).  sink may be NULL (no sink term); lse may be NULL.
+ * A query with count == 0 and no sink gets O = 0 and lse = -inf.
+ */
+int sparse_gqa_attn_decode(const void *Q, const dsa_kv_t *kv, const int32_t *idx,
+                           const int32_t *count, int B, int T, int top_k,
+                           const float *sink, float sm_scale, void *O, float *lse,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * swa_attn_decode -- the same attention over the implicit contiguous key set
+ * {max(0, p - window + 1) .. p}, p = q_pos[b][t] ("What 'no full-attention
+ * layers' means": keys with query_offset - key_offset >= window are masked).
+ * 1 <= window <= DSA_MAX_TOPK.
+ */
+int swa_attn_decode(const void *Q, const dsa_kv_t *kv, const int32_t *q_pos, int B, int T,
+                    int window, const float *sink, float sm_scale, void *O, float *lse,
+                    void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_layer_decode -- one DSA decode layer-step: dsa_indexer_scores, then
+ * dsa_topk_select, then sparse_gqa_attn_decode, enqueued back to back on
+ * `stream` with the scores and the selection kept in the workspace.
+ * idx_out (int32 [B][T][top_k]) and count_out (int32 [B][T]) are optional
+ * copies of the selection (NULL = not wanted).
+ * stage_events: NULL, or an array of 5 cudaEvent_t recorded on `stream`
+ * before the indexer, before the selection, before the attention, before the
+ * combine and at the end (for per-stage timing).
+ */
+int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const void *Q,
+                     const dsa_kv_t *kv, const int32_t *q_pos, int B, int T, int64_t Lmax,
+                     int top_k, const float *sink, float sm_scale, void *O, float *lse,
+                     int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
+                     void *stream, void *const *stage_events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

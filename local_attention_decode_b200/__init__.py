@@ -1,0 +1,234 @@
+"""Python binding of libdsa: DSA / SWA decode layer-step kernels for B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libdsa.so`` (built from ``csrc/`` for sm_100a, C ABI in
+``include/dsa.h``).  PyTorch provides device memory and streams.  There is no
+fallback path: if the library is missing, importing this package fails.
+
+Function names match the C entry points.  Tensors must be CUDA tensors of the
+documented dtype and shape, contiguous, on the current device; the calls are
+enqueued on the current torch stream (or ``stream=``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libdsa.so is not built: run `python -c 'import __graft_entry__ as g; g.build()'` "
+        "or `python local_attention_decode_b200/_build.py` first")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status codes and constants (include/dsa.h)
+DSA_OK = 0
+DSA_ERR_INVALID_ARG = 1
+DSA_ERR_UNSUPPORTED_SHAPE = 2
+DSA_ERR_WORKSPACE_TOO_SMALL = 3
+DSA_ERR_CUDA = 4
+DSA_ERR_DEVICE_TIMEOUT = 5
+DSA_ERR_DEVICE_BAD_INDEX = 6
+OP_INDEXER, OP_TOPK, OP_SPARSE_ATTN, OP_SWA_ATTN, OP_LAYER = range(5)
+
+EXPORTED = ("dsa_last_error", "dsa_get_dims", "dsa_workspace_size", "dsa_workspace_init",
+            "dsa_check_device_status", "dsa_indexer_scores", "dsa_topk_select",
+            "sparse_gqa_attn_decode", "swa_attn_decode", "dsa_layer_decode")
+
+
+class DSAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libdsa error {code}: {msg}")
+        self.code = code
+
+
+class dsa_kv_t(ctypes.Structure):
+    _fields_ = [
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("index_k", ctypes.c_void_p),
+        ("index_k_scale", ctypes.c_void_p),
+        ("num_kv_heads", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("seq_stride", ctypes.c_int64),
+        ("num_rows", ctypes.c_int64),
+        ("block_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+P = ctypes.c_void_p
+I32, I64, SZ, F32 = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_lib.dsa_last_error.restype = ctypes.c_char_p
+_lib.dsa_last_error.argtypes = []
+_lib.dsa_get_dims.argtypes = [P, I32]
+_lib.dsa_workspace_size.argtypes = [I32, I32, I32, I64, I32, ctypes.POINTER(ctypes.c_size_t)]
+_lib.dsa_workspace_init.argtypes = [P, SZ, P]
+_lib.dsa_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_uint32)]
+_lib.dsa_indexer_scores.argtypes = [P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I64, P, I64, P, SZ, P]
+_lib.dsa_topk_select.argtypes = [P, I64, P, I32, I32, I64, I32, P, P, P, SZ, P]
+_lib.sparse_gqa_attn_decode.argtypes = [P, ctypes.POINTER(dsa_kv_t), P, P, I32, I32, I32, P, F32, P, P, P, SZ, P]
+_lib.swa_attn_decode.argtypes = [P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I32, P, F32, P, P, P, SZ, P]
+_lib.dsa_layer_decode.argtypes = [P, P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I64, I32, P, F32, P, P, P, P,
+                                  P, SZ, P, P]
+for _name in EXPORTED[1:]:
+    getattr(_lib, _name).restype = ctypes.c_int
+
+
+def _check(rc: int):
+    if rc != DSA_OK:
+        raise DSAError(rc, _lib.dsa_last_error().decode(errors="replace"))
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def get_dims():
+    dims = (ctypes.c_int32 * 7)()
+    _check(_lib.dsa_get_dims(ctypes.cast(dims, P), 7))
+    return list(dims)
+
+
+def workspace_size(op: int, B: int, T: int, Lmax: int, top_k: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.dsa_workspace_size(op, B, T, Lmax, top_k, ctypes.byref(out)))
+    return out.value
+
+
+def alloc_workspace(op: int, B: int, T: int, Lmax: int, top_k: int, device=None) -> torch.Tensor:
+    """A zeroed workspace (uint8, 256-byte aligned by the caching allocator)."""
+    n = workspace_size(op, B, T, Lmax, top_k)
+    ws = torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def dsa_workspace_init(ws: torch.Tensor, stream=None):
+    _check(_lib.dsa_workspace_init(_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def dsa_check_device_status(ws: torch.Tensor, stream=None):
+    """(status, flags) of the device status word; synchronises the stream."""
+    st = ctypes.c_int(0)
+    fl = ctypes.c_uint32(0)
+    _check(_lib.dsa_check_device_status(_ptr(ws, torch.uint8, "ws"), _stream(stream), ctypes.byref(st),
+                                        ctypes.byref(fl)))
+    return st.value, fl.value
+
+
+class KV:
+    """KV-cache description (dsa_kv_t) over caller-owned tensors.
+
+    k [rows, G, 192] bf16, v [rows, G, 128] bf16, index_k [rows, 128] uint8 (e4m3
+    codes), index_k_scale [rows] f32; contiguous layout with ``seq_stride`` rows
+    per sequence, or paged with ``block_table`` [B, max_pages] int32 and
+    ``page_size``.
+    """
+
+    def __init__(self, *, k=None, v=None, index_k=None, index_k_scale=None, num_kv_heads=None,
+                 seq_stride=0, block_table=None, page_size=0, num_rows=None):
+        self._keep = (k, v, index_k, index_k_scale, block_table)
+        rows = None
+        for t in (index_k, k, v, index_k_scale):
+            if t is not None:
+                rows = t.shape[0]
+                break
+        if num_rows is None:
+            num_rows = rows
+        if num_kv_heads is None:
+            num_kv_heads = k.shape[1] if k is not None else 0
+        s = dsa_kv_t()
+        s.k = _ptr(k, torch.bfloat16, "k") if k is not None else None
+        s.v = _ptr(v, torch.bfloat16, "v") if v is not None else None
+        s.index_k = _ptr(index_k, torch.uint8, "index_k") if index_k is not None else None
+        s.index_k_scale = _ptr(index_k_scale, torch.float32, "index_k_scale") if index_k_scale is not None else None
+        s.num_kv_heads = int(num_kv_heads)
+        s.page_size = int(page_size)
+        s.seq_stride = int(seq_stride)
+        s.num_rows = int(num_rows)
+        s.block_table = _ptr(block_table, torch.int32, "block_table") if block_table is not None else None
+        s.max_pages = int(block_table.shape[1]) if block_table is not None else 0
+        s.reserved = 0
+        self.struct = s
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def _bt(t: torch.Tensor, trailing: Sequence[int], name: str):
+    if tuple(t.shape[2:]) != tuple(trailing):
+        raise ValueError(f"{name}: expected [B, T, {', '.join(map(str, trailing))}], got {tuple(t.shape)}")
+    return t.shape[0], t.shape[1]
+
+
+def dsa_indexer_scores(q8, q_scale, w, kv: KV, q_pos, Lmax: int, scores, ws, stream=None):
+    B, T = _bt(q8, (16, 128), "q8")
+    _check(_lib.dsa_indexer_scores(_ptr(q8, torch.uint8, "q8"), _ptr(q_scale, torch.float32, "q_scale"),
+                                   _ptr(w, torch.float32, "w"), kv.ref, _ptr(q_pos, torch.int32, "q_pos"), B, T,
+                                   int(Lmax), _ptr(scores, torch.float32, "scores"), scores.shape[-1],
+                                   _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def dsa_topk_select(scores, q_pos, Lmax: int, top_k: int, idx, count, ws, stream=None):
+    B, T = q_pos.shape
+    _check(_lib.dsa_topk_select(_ptr(scores, torch.float32, "scores"), scores.shape[-1],
+                                _ptr(q_pos, torch.int32, "q_pos"), B, T, int(Lmax), int(top_k),
+                                _ptr(idx, torch.int32, "idx"), _ptr(count, torch.int32, "count"),
+                                _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def sparse_gqa_attn_decode(Q, kv: KV, idx, count, top_k: int, sink, sm_scale: float, O, lse=None, ws=None,
+                           stream=None):
+    B, T = _bt(Q, (64, 192), "Q")
+    _check(_lib.sparse_gqa_attn_decode(_ptr(Q, torch.bfloat16, "Q"), kv.ref, _ptr(idx, torch.int32, "idx"),
+                                       _ptr(count, torch.int32, "count"), B, T, int(top_k),
+                                       _ptr(sink, torch.float32, "sink"), float(sm_scale),
+                                       _ptr(O, torch.bfloat16, "O"), _ptr(lse, torch.float32, "lse"),
+                                       _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def swa_attn_decode(Q, kv: KV, q_pos, window: int, sink, sm_scale: float, O, lse=None, ws=None, stream=None):
+    B, T = _bt(Q, (64, 192), "Q")
+    _check(_lib.swa_attn_decode(_ptr(Q, torch.bfloat16, "Q"), kv.ref, _ptr(q_pos, torch.int32, "q_pos"), B, T,
+                                int(window), _ptr(sink, torch.float32, "sink"), float(sm_scale),
+                                _ptr(O, torch.bfloat16, "O"), _ptr(lse, torch.float32, "lse"),
+                                _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def dsa_layer_decode(q8, q_scale, w, Q, kv: KV, q_pos, Lmax: int, top_k: int, sink, sm_scale: float, O, lse=None,
+                     idx_out=None, count_out=None, ws=None, stream=None, stage_events=None):
+    B, T = _bt(q8, (16, 128), "q8")
+    ev = None
+    if stage_events is not None:
+        arr = (ctypes.c_void_p * 5)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
+                                      for e in stage_events])
+        ev = ctypes.cast(arr, P)
+    _check(_lib.dsa_layer_decode(_ptr(q8, torch.uint8, "q8"), _ptr(q_scale, torch.float32, "q_scale"),
+                                 _ptr(w, torch.float32, "w"), _ptr(Q, torch.bfloat16, "Q"), kv.ref,
+                                 _ptr(q_pos, torch.int32, "q_pos"), B, T, int(Lmax), int(top_k),
+                                 _ptr(sink, torch.float32, "sink"), float(sm_scale), _ptr(O, torch.bfloat16, "O"),
+                                 _ptr(lse, torch.float32, "lse"), _ptr(idx_out, torch.int32, "idx_out"),
+                                 _ptr(count_out, torch.int32, "count_out"), _ptr(ws, torch.uint8, "ws"),
+                                 ws.numel(), _stream(stream), ev))

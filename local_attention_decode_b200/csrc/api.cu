@@ -1,0 +1,351 @@
+// api.cu -- the C ABI of libdsa (declared in include/dsa.h): argument checks,
+// workspace layout, and the launch sequences of each entry point.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+
+static thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+const DeviceInfo &device_info() {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        static DeviceInfo none;
+        return none;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo &d = cache[dev];
+    if (d.device != dev) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess) {
+            d.num_sms = prop.multiProcessorCount;
+            d.smem_optin = prop.sharedMemPerBlockOptin;
+            d.device = dev;
+        }
+    }
+    return d;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ----------------------------------------------------------- argument checks
+static int check_common(int B, int T) {
+    if (B < 1 || B > 1024) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "B=%d outside [1, 1024]", B);
+    if (T < 1 || T > DSA_MAX_T) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "T=%d outside [1, %d]", T, DSA_MAX_T);
+    return DSA_OK;
+}
+
+static int check_kv_layout(const dsa_kv_t *kv) {
+    if (!kv) return fail(DSA_ERR_INVALID_ARG, "kv is NULL");
+    if (kv->num_rows < 1 || kv->num_rows >= (int64_t(1) << 31))
+        return fail(DSA_ERR_UNSUPPORTED_SHAPE, "kv.num_rows=%lld outside [1, 2^31)", (long long)kv->num_rows);
+    if (kv->block_table) {
+        const int ps = kv->page_size;
+        bool ok = ps >= 16 && ((ps <= 128 && 128 % ps == 0 && ps % 16 == 0) || (ps % 128 == 0));
+        if (!ok) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "page_size=%d: need 16/32/64/128 or a multiple of 128", ps);
+        if (kv->max_pages < 1) return fail(DSA_ERR_INVALID_ARG, "max_pages=%d < 1", kv->max_pages);
+        if (kv->num_rows % ps) return fail(DSA_ERR_INVALID_ARG, "num_rows is not a multiple of page_size");
+    } else {
+        if (kv->seq_stride < 1) return fail(DSA_ERR_INVALID_ARG, "seq_stride=%lld < 1", (long long)kv->seq_stride);
+    }
+    return DSA_OK;
+}
+
+static int check_kv_backbone(const dsa_kv_t *kv) {
+    int rc = check_kv_layout(kv);
+    if (rc) return rc;
+    if (!kv->k || !kv->v) return fail(DSA_ERR_INVALID_ARG, "kv.k / kv.v is NULL");
+    if (!aligned16(kv->k) || !aligned16(kv->v)) return fail(DSA_ERR_INVALID_ARG, "kv.k / kv.v not 16-byte aligned");
+    const int G = kv->num_kv_heads;
+    if (G < 1 || DSA_Q_HEADS % G || DSA_Q_HEADS / G > 16)
+        return fail(DSA_ERR_UNSUPPORTED_SHAPE, "num_kv_heads=%d: need a divisor of 64 with at most 16 heads per group", G);
+    return DSA_OK;
+}
+
+static int check_kv_index(const dsa_kv_t *kv) {
+    int rc = check_kv_layout(kv);
+    if (rc) return rc;
+    if (!kv->index_k || !kv->index_k_scale) return fail(DSA_ERR_INVALID_ARG, "kv.index_k / index_k_scale is NULL");
+    if (!aligned16(kv->index_k) || !aligned16(kv->index_k_scale))
+        return fail(DSA_ERR_INVALID_ARG, "kv.index_k / index_k_scale not 16-byte aligned");
+    return DSA_OK;
+}
+
+// ------------------------------------------------------------ workspace plan
+struct WsPlan {
+    size_t status = 0, scores = 0, idx = 0, count = 0, topk = 0, part_o = 0, part_ml = 0, total = 0;
+    TopkPlan tp;
+};
+
+static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan *w) {
+    size_t off = kStatusBytes;
+    w->status = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off = align_up(off + bytes, 256);
+        return at;
+    };
+    switch (op) {
+        case DSA_OP_INDEXER:
+            break;
+        case DSA_OP_TOPK: {
+            int rc = plan_topk(B, T, Lmax, top_k, &w->tp);
+            if (rc) return rc;
+            w->topk = take(w->tp.scratch_bytes);
+            break;
+        }
+        case DSA_OP_SPARSE_ATTN:
+        case DSA_OP_SWA_ATTN: {
+            const int splits = (top_k + kAttnChunk - 1) / kAttnChunk;
+            const size_t rows = (size_t)B * T * DSA_Q_HEADS * splits;
+            w->part_o = take(rows * DSA_V_DIM * 4);
+            w->part_ml = take(rows * 2 * 4);
+            break;
+        }
+        case DSA_OP_LAYER: {
+            int rc = plan_topk(B, T, Lmax, top_k, &w->tp);
+            if (rc) return rc;
+            w->scores = take((size_t)B * T * Lmax * 4);
+            w->idx = take((size_t)B * T * top_k * 4);
+            w->count = take((size_t)B * T * 4);
+            w->topk = take(w->tp.scratch_bytes);
+            const int splits = (top_k + kAttnChunk - 1) / kAttnChunk;
+            const size_t rows = (size_t)B * T * DSA_Q_HEADS * splits;
+            w->part_o = take(rows * DSA_V_DIM * 4);
+            w->part_ml = take(rows * 2 * 4);
+            break;
+        }
+        default:
+            return fail(DSA_ERR_INVALID_ARG, "unknown op %d", op);
+    }
+    w->total = off;
+    return DSA_OK;
+}
+
+static int check_ws(void *ws, size_t ws_bytes, const WsPlan &w) {
+    if (!ws) return fail(DSA_ERR_INVALID_ARG, "workspace is NULL");
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(DSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    if (ws_bytes < w.total)
+        return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, w.total);
+    return DSA_OK;
+}
+
+template <class T>
+static T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+static int record(void *const *events, int i, cudaStream_t s) {
+    if (!events || !events[i]) return DSA_OK;
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e, "cudaEventRecord");
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char *dsa_last_error(void) { return g_err; }
+
+int dsa_get_dims(int32_t *dims, int n) {
+    if (!dims || n < 0 || n > 7) return fail(DSA_ERR_INVALID_ARG, "dims / n");
+    const int32_t v[7] = {DSA_INDEX_HEADS, DSA_INDEX_DIM, DSA_Q_HEADS, DSA_QK_DIM, DSA_V_DIM, DSA_MAX_TOPK, DSA_MAX_T};
+    for (int i = 0; i < n; ++i) dims[i] = v[i];
+    return DSA_OK;
+}
+
+int dsa_workspace_size(int op, int B, int T, int64_t Lmax, int top_k, size_t *bytes) {
+    if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
+    if (op != DSA_OP_INDEXER && (top_k < 1 || top_k > DSA_MAX_TOPK))
+        return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k/window=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
+    WsPlan w;
+    rc = plan_workspace(op, B, T, Lmax, top_k, &w);
+    if (rc) return rc;
+    *bytes = w.total;
+    return DSA_OK;
+}
+
+int dsa_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws) return fail(DSA_ERR_INVALID_ARG, "workspace is NULL");
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e, "cudaMemsetAsync(workspace)");
+}
+
+int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags) {
+    if (!ws || !status) return fail(DSA_ERR_INVALID_ARG, "ws / status is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(&word, ws, 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && word) e = cudaMemset(ws, 0, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (flags) *flags = word;
+    *status = (word & (1u << DSA_ERR_DEVICE_TIMEOUT))     ? DSA_ERR_DEVICE_TIMEOUT
+              : (word & (1u << DSA_ERR_DEVICE_BAD_INDEX)) ? DSA_ERR_DEVICE_BAD_INDEX
+                                                          : DSA_OK;
+    return DSA_OK;
+}
+
+int dsa_indexer_scores(const void *q8, const float *q_scale, const float *w, const dsa_kv_t *kv,
+                       const int32_t *q_pos, int B, int T, int64_t Lmax, float *scores, int64_t scores_stride,
+                       void *ws, size_t ws_bytes, void *stream) {
+    if (!q8 || !q_scale || !w || !q_pos || !scores) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(q8)) return fail(DSA_ERR_INVALID_ARG, "q8 not 16-byte aligned");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (rc = check_kv_index(kv); rc) return rc;
+    if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
+    if (scores_stride < Lmax) return fail(DSA_ERR_INVALID_ARG, "scores_stride < Lmax");
+    WsPlan wp;
+    if (rc = plan_workspace(DSA_OP_INDEXER, B, T, Lmax, 1, &wp); rc) return rc;
+    if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
+    IndexerArgs a{static_cast<const uint8_t *>(q8), q_scale, w, kv, q_pos, B, T, Lmax, scores, scores_stride,
+                  at<uint32_t>(ws, wp.status)};
+    return launch_indexer(a, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk_select(const float *scores, int64_t scores_stride, const int32_t *q_pos, int B, int T, int64_t Lmax,
+                    int top_k, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes, void *stream) {
+    if (!scores || !q_pos || !idx || !count) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
+    if (scores_stride < Lmax) return fail(DSA_ERR_INVALID_ARG, "scores_stride < Lmax");
+    if (top_k < 1 || top_k > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
+    WsPlan wp;
+    if (rc = plan_workspace(DSA_OP_TOPK, B, T, Lmax, top_k, &wp); rc) return rc;
+    if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
+    return launch_topk(wp.tp, scores, scores_stride, q_pos, top_k, idx, count, at<uint32_t>(ws, wp.topk),
+                       at<uint32_t>(ws, wp.status), static_cast<cudaStream_t>(stream));
+}
+
+static int attention_common(const void *Q, const dsa_kv_t *kv, const int32_t *idx, const int32_t *count,
+                            const int32_t *q_pos, int window, int B, int T, int max_keys, const float *sink,
+                            float sm_scale, void *O, float *lse, void *ws, size_t ws_bytes, void *stream, int op) {
+    if (!Q || !O) return fail(DSA_ERR_INVALID_ARG, "Q / O is NULL");
+    if (!aligned16(Q) || !aligned16(O)) return fail(DSA_ERR_INVALID_ARG, "Q / O not 16-byte aligned");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (rc = check_kv_backbone(kv); rc) return rc;
+    if (max_keys < 1 || max_keys > DSA_MAX_TOPK)
+        return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k/window=%d outside [1, %d]", max_keys, DSA_MAX_TOPK);
+    if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+    WsPlan wp;
+    if (rc = plan_workspace(op, B, T, 1, max_keys, &wp); rc) return rc;
+    if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
+    AttnArgs a;
+    a.Q = static_cast<const __nv_bfloat16 *>(Q);
+    a.kv = kv;
+    a.idx = idx;
+    a.count = count;
+    a.idx_stride = max_keys;
+    a.q_pos = q_pos;
+    a.window = window;
+    a.B = B;
+    a.T = T;
+    a.max_keys = max_keys;
+    a.sink = sink;
+    a.sm_scale = sm_scale;
+    a.O = static_cast<__nv_bfloat16 *>(O);
+    a.lse = lse;
+    a.part_o = at<float>(ws, wp.part_o);
+    a.part_ml = at<float>(ws, wp.part_ml);
+    a.status = at<uint32_t>(ws, wp.status);
+    return launch_attention(a, static_cast<cudaStream_t>(stream));
+}
+
+int sparse_gqa_attn_decode(const void *Q, const dsa_kv_t *kv, const int32_t *idx, const int32_t *count, int B, int T,
+                           int top_k, const float *sink, float sm_scale, void *O, float *lse, void *ws,
+                           size_t ws_bytes, void *stream) {
+    if (!idx || !count) return fail(DSA_ERR_INVALID_ARG, "idx / count is NULL");
+    return attention_common(Q, kv, idx, count, nullptr, 0, B, T, top_k, sink, sm_scale, O, lse, ws, ws_bytes, stream,
+                            DSA_OP_SPARSE_ATTN);
+}
+
+int swa_attn_decode(const void *Q, const dsa_kv_t *kv, const int32_t *q_pos, int B, int T, int window,
+                    const float *sink, float sm_scale, void *O, float *lse, void *ws, size_t ws_bytes, void *stream) {
+    if (!q_pos) return fail(DSA_ERR_INVALID_ARG, "q_pos is NULL");
+    return attention_common(Q, kv, nullptr, nullptr, q_pos, window, B, T, window, sink, sm_scale, O, lse, ws, ws_bytes,
+                            stream, DSA_OP_SWA_ATTN);
+}
+
+int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+                     const int32_t *q_pos, int B, int T, int64_t Lmax, int top_k, const float *sink, float sm_scale,
+                     void *O, float *lse, int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
+                     void *stream, void *const *stage_events) {
+    if (!q8 || !q_scale || !w || !Q || !q_pos || !O) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(q8) || !aligned16(Q) || !aligned16(O)) return fail(DSA_ERR_INVALID_ARG, "q8 / Q / O not 16-byte aligned");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (rc = check_kv_index(kv); rc) return rc;
+    if (rc = check_kv_backbone(kv); rc) return rc;
+    if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
+    if (top_k < 1 || top_k > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
+    if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+    WsPlan wp;
+    if (rc = plan_workspace(DSA_OP_LAYER, B, T, Lmax, top_k, &wp); rc) return rc;
+    if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *status = at<uint32_t>(ws, wp.status);
+    float *scores = at<float>(ws, wp.scores);
+    int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, wp.idx);
+    int32_t *count = count_out ? count_out : at<int32_t>(ws, wp.count);
+
+    if (rc = record(stage_events, 0, s); rc) return rc;
+    IndexerArgs ia{static_cast<const uint8_t *>(q8), q_scale, w, kv, q_pos, B, T, Lmax, scores, Lmax, status};
+    if (rc = launch_indexer(ia, s); rc) return rc;
+    if (rc = record(stage_events, 1, s); rc) return rc;
+    if (rc = launch_topk(wp.tp, scores, Lmax, q_pos, top_k, idx, count, at<uint32_t>(ws, wp.topk), status, s); rc)
+        return rc;
+    if (rc = record(stage_events, 2, s); rc) return rc;
+    AttnArgs a;
+    a.Q = static_cast<const __nv_bfloat16 *>(Q);
+    a.kv = kv;
+    a.idx = idx;
+    a.count = count;
+    a.idx_stride = top_k;
+    a.q_pos = nullptr;
+    a.window = 0;
+    a.B = B;
+    a.T = T;
+    a.max_keys = top_k;
+    a.sink = sink;
+    a.sm_scale = sm_scale;
+    a.O = static_cast<__nv_bfloat16 *>(O);
+    a.lse = lse;
+    a.part_o = at<float>(ws, wp.part_o);
+    a.part_ml = at<float>(ws, wp.part_ml);
+    a.status = status;
+    a.mid_event = stage_events ? stage_events[3] : nullptr;
+    if (rc = launch_attention(a, s); rc) return rc;
+    if (rc = record(stage_events, 4, s); rc) return rc;
+    return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,293 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Sizes span several 128-key tiles with ragged tails, contiguous and paged
+caches, 1 and 4 query tokens, and the 1,048,576-token context (sampled where
+the oracle cannot do the whole thing).  Tolerances are in tests/parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():   # collected on CPU machines, skipped there by the marker filter
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import oracle  # noqa: E402
+import local_attention_decode_b200 as dsa  # noqa: E402
+from workloads import CONFIGS, bits16, make_decode_workload, logical_rows, ragged_batch_lengths  # noqa: E402
+from parity import (kv_for, assert_scores_close, assert_attn_close, oracle_scores,  # noqa: E402
+                    oracle_attention_rows, selection_is_valid)
+
+DEV = "cuda"
+SM = 1.0 / math.sqrt(192)
+
+
+def run_indexer(wl, Lmax=None):
+    Lmax = Lmax or int(wl.q_pos.max()) + 1
+    scores = torch.full((wl.B, wl.T, Lmax), float("nan"), device=DEV)
+    ws = dsa.alloc_workspace(dsa.OP_INDEXER, wl.B, wl.T, Lmax, 1)
+    dsa.dsa_indexer_scores(wl.q8, wl.q_scale, wl.w, kv_for(wl, with_backbone=False), wl.q_pos, Lmax, scores, ws)
+    st, _ = dsa.dsa_check_device_status(ws)
+    assert st == dsa.DSA_OK
+    return scores
+
+
+def run_topk(scores, q_pos, top_k):
+    B, T, Lmax = scores.shape
+    idx = torch.full((B, T, top_k), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((B, T), -7, dtype=torch.int32, device=DEV)
+    ws = dsa.alloc_workspace(dsa.OP_TOPK, B, T, Lmax, top_k)
+    dsa.dsa_topk_select(scores, q_pos, Lmax, top_k, idx, cnt, ws)
+    st, _ = dsa.dsa_check_device_status(ws)
+    assert st == dsa.DSA_OK
+    # the workspace is left zeroed for the next call
+    assert int(ws.count_nonzero()) == 0
+    return idx, cnt
+
+
+# ------------------------------------------------------------------ indexer
+@pytest.mark.parametrize("case", [
+    dict(seq_lens=[8192], T=1),                 # the tiny decode workload
+    dict(seq_lens=[3001], T=4),                 # ragged tail, speculative block
+    dict(seq_lens=[1, 127, 128, 129, 700], T=1),  # degenerate and boundary lengths
+    dict(seq_lens=[5000, 300, 2000], T=2, page_size=64),   # paged, ragged
+    dict(seq_lens=[1000, 4100], T=1, page_size=16),
+    dict(seq_lens=[3000, 1500], T=3, page_size=256),
+])
+def test_indexer_matches_oracle(case):
+    wl = make_decode_workload(seed=11, device=DEV, n_needles=4, **case)
+    scores = run_indexer(wl).cpu().numpy()
+    for b in range(wl.B):
+        ref = oracle_scores(wl, b)
+        assert_scores_close(scores[b, :, :ref.shape[1]], ref)
+
+
+def test_indexer_t16_and_many_sequences():
+    wl = make_decode_workload(seed=12, seq_lens=[700] * 3, T=16, device=DEV)
+    scores = run_indexer(wl).cpu().numpy()
+    for b in range(wl.B):
+        ref = oracle_scores(wl, b)
+        assert_scores_close(scores[b], ref)
+    lens = [int(x) for x in np.random.default_rng(0).integers(1, 600, 100)]
+    wl = make_decode_workload(seed=13, seq_lens=lens, T=1, device=DEV, page_size=64)
+    scores = run_indexer(wl).cpu().numpy()
+    for b in range(0, wl.B, 7):
+        ref = oracle_scores(wl, b)
+        assert_scores_close(scores[b, :, :ref.shape[1]], ref)
+
+
+# -------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("n,k", [(1, 2048), (2047, 2048), (2048, 2048), (2049, 2048), (5000, 2048),
+                                 (70000, 2048), (70000, 1), (300000, 2048), (1048576, 2048)])
+def test_topk_bit_exact_against_oracle(n, k):
+    g = torch.Generator(device=DEV).manual_seed(n + k)
+    scores = torch.rand((1, 1, n), generator=g, device=DEV) * 10
+    q_pos = torch.tensor([[n - 1]], dtype=torch.int32, device=DEV)
+    idx, cnt = run_topk(scores, q_pos, k)
+    ref_idx, ref_cnt = oracle.topk(scores[0, 0].cpu().numpy(), k)
+    assert int(cnt) == ref_cnt
+    got = idx[0, 0].cpu().numpy()
+    assert np.all(got[ref_cnt:] == -1)
+    assert np.all(np.diff(got[:ref_cnt]) > 0)              # increasing position order
+    assert np.array_equal(got[:ref_cnt], np.sort(ref_idx[:ref_cnt]))
+
+
+@pytest.mark.parametrize("kind", ["all_equal", "few_values", "signed_zero", "negative", "heavy_ties_long"])
+def test_topk_ties(kind):
+    n, k = (200000, 2048) if kind == "heavy_ties_long" else (9000, 2048)
+    g = torch.Generator(device=DEV).manual_seed(7)
+    if kind == "all_equal":
+        s = torch.full((n,), 3.25, device=DEV)
+    elif kind == "few_values":
+        s = torch.randint(0, 5, (n,), generator=g, device=DEV).float()
+    elif kind == "signed_zero":
+        s = torch.where(torch.rand(n, generator=g, device=DEV) < 0.5, torch.tensor(-0.0, device=DEV),
+                        torch.tensor(0.0, device=DEV))
+        s[::97] = 1.0
+    elif kind == "negative":
+        s = -torch.rand(n, generator=g, device=DEV) - 1
+    else:
+        s = torch.randint(0, 3, (n,), generator=g, device=DEV).float()
+    scores = s.view(1, 1, n).contiguous()
+    q_pos = torch.tensor([[n - 1]], dtype=torch.int32, device=DEV)
+    idx, cnt = run_topk(scores, q_pos, k)
+    ref_idx, ref_cnt = oracle.topk(s.cpu().numpy(), k)
+    assert int(cnt) == ref_cnt
+    assert np.array_equal(idx[0, 0, :ref_cnt].cpu().numpy(), np.sort(ref_idx[:ref_cnt]))
+
+
+def test_topk_many_rows_ragged():
+    B, T, L = 6, 4, 40000
+    g = torch.Generator(device=DEV).manual_seed(3)
+    scores = torch.randn((B, T, L), generator=g, device=DEV)
+    q_pos = torch.randint(0, L, (B, T), generator=g, device=DEV, dtype=torch.int32)
+    q_pos[0, 0] = 0
+    q_pos[1, 1] = 2047
+    q_pos[2, 2] = L - 1
+    idx, cnt = run_topk(scores, q_pos, 2048)
+    sc = scores.cpu().numpy()
+    for b in range(B):
+        for t in range(T):
+            n = int(q_pos[b, t]) + 1
+            ref_idx, ref_cnt = oracle.topk(sc[b, t, :n], 2048)
+            assert int(cnt[b, t]) == ref_cnt
+            assert np.array_equal(idx[b, t, :ref_cnt].cpu().numpy(), np.sort(ref_idx[:ref_cnt]))
+            assert np.all(idx[b, t, ref_cnt:].cpu().numpy() == -1)
+
+
+# ---------------------------------------------------------------- attention
+def _sparse_case(seed, seq_len, T, count_list, G=4, qk_std=None, page_size=0, sink=True):
+    wl = make_decode_workload(seed=seed, seq_lens=[seq_len], T=T, G=G, device=DEV, qk_std=qk_std,
+                              page_size=page_size)
+    rng = np.random.default_rng(seed)
+    top_k = 2048
+    idx = np.full((1, T, top_k), -1, np.int32)
+    cnt = np.zeros((1, T), np.int32)
+    for t, c in enumerate(count_list):
+        idx[0, t, :c] = rng.choice(seq_len, c, replace=False)
+        cnt[0, t] = c
+    idx_t = torch.from_numpy(idx).to(DEV)
+    cnt_t = torch.from_numpy(cnt).to(DEV)
+    O = torch.empty((1, T, 64, 128), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((1, T, 64), dtype=torch.float32, device=DEV)
+    ws = dsa.alloc_workspace(dsa.OP_SPARSE_ATTN, 1, T, 1, top_k)
+    sk = wl.sink if sink else None
+    dsa.sparse_gqa_attn_decode(wl.Q, kv_for(wl, with_index=False), idx_t, cnt_t, top_k, sk, SM, O, lse, ws)
+    st, _ = dsa.dsa_check_device_status(ws)
+    assert st == dsa.DSA_OK
+    for t in range(T):
+        ref_o, ref_l = oracle_attention_rows(wl, 0, t, idx[0, t, :cnt[0, t]], sk, SM)
+        assert_attn_close(O[0, t], ref_o, lse[0, t], ref_l)
+
+
+@pytest.mark.parametrize("counts", [[2048], [1], [0], [2047, 64, 65, 1000]])
+def test_sparse_attention_matches_oracle(counts):
+    _sparse_case(20 + len(counts), 10000, len(counts), counts)
+
+
+def test_sparse_attention_peaked_and_paged():
+    _sparse_case(31, 7000, 2, [2048, 333], qk_std=1.0, page_size=64)
+    _sparse_case(32, 7000, 1, [2048], qk_std=1.0, sink=False)
+
+
+@pytest.mark.parametrize("G", [4, 8, 16])
+def test_sparse_attention_other_group_sizes(G):
+    _sparse_case(40 + G, 3000, 1, [1500], G=G)
+
+
+@pytest.mark.parametrize("seq_lens,T,page_size", [([8192], 1, 0), ([100], 1, 0), ([1], 1, 0),
+                                                  ([300, 129, 5000], 2, 64)])
+def test_swa_attention_matches_oracle(seq_lens, T, page_size):
+    wl = make_decode_workload(seed=50, seq_lens=seq_lens, T=T, G=8, device=DEV, page_size=page_size)
+    O = torch.empty((wl.B, T, 64, 128), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((wl.B, T, 64), dtype=torch.float32, device=DEV)
+    ws = dsa.alloc_workspace(dsa.OP_SWA_ATTN, wl.B, T, 1, 128)
+    dsa.swa_attn_decode(wl.Q, kv_for(wl, with_index=False), wl.q_pos, 128, wl.sink, SM, O, lse, ws)
+    for b in range(wl.B):
+        for t in range(T):
+            p = int(wl.q_pos[b, t])
+            win = oracle.swa_indices(p, 128)
+            ref_o, ref_l = oracle_attention_rows(wl, b, t, win, wl.sink, SM)
+            assert_attn_close(O[b, t], ref_o, lse[b, t], ref_l)
+
+
+# -------------------------------------------------------- fused layer-step
+def run_layer(wl, top_k=2048, sink=True, events=None):
+    Lmax = int(wl.q_pos.max()) + 1
+    O = torch.empty((wl.B, wl.T, 64, 128), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((wl.B, wl.T, 64), dtype=torch.float32, device=DEV)
+    idx = torch.empty((wl.B, wl.T, top_k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((wl.B, wl.T), dtype=torch.int32, device=DEV)
+    ws = dsa.alloc_workspace(dsa.OP_LAYER, wl.B, wl.T, Lmax, top_k)
+    dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv_for(wl), wl.q_pos, Lmax, top_k,
+                         wl.sink if sink else None, SM, O, lse, idx, cnt, ws)
+    st, _ = dsa.dsa_check_device_status(ws)
+    assert st == dsa.DSA_OK
+    return O, lse, idx, cnt
+
+
+def _check_layer(wl, O, lse, idx, cnt, top_k=2048, full_oracle=True):
+    for b in range(wl.B):
+        ref_scores = oracle_scores(wl, b) if full_oracle else None
+        for t in range(wl.T):
+            n = int(wl.q_pos[b, t]) + 1
+            c = int(cnt[b, t])
+            assert c == min(n, top_k)
+            sel = idx[b, t, :c].cpu().numpy()
+            assert np.all(idx[b, t, c:].cpu().numpy() == -1)
+            if ref_scores is not None:
+                assert selection_is_valid(sel, ref_scores[t, :n].astype(np.float64), top_k)
+                ref_idx, _ = oracle.topk(ref_scores[t, :n], top_k)
+                # same set unless scores tie within rounding at the threshold
+                diff = len(set(ref_idx[:c].tolist()) ^ set(sel.tolist()))
+                assert diff <= 8, f"selection differs from the oracle's in {diff} positions"
+            ref_o, ref_l = oracle_attention_rows(wl, b, t, sel, wl.sink, SM)
+            assert_attn_close(O[b, t], ref_o, lse[b, t], ref_l)
+
+
+@pytest.mark.parametrize("name", ["tiny_8k", "verify_64k_t4"])
+def test_layer_decode_matches_oracle(name):
+    wl = make_decode_workload(device=DEV, **CONFIGS[name])
+    O, lse, idx, cnt = run_layer(wl)
+    _check_layer(wl, O, lse, idx, cnt)
+    # planted needles rank in the oracle's top-2048 and are selected
+    sel = set(idx[0, 0].cpu().numpy().tolist())
+    assert set(wl.needles[0].tolist()) <= sel
+
+
+def test_layer_decode_short_contexts_and_pages():
+    wl = make_decode_workload(seed=60, seq_lens=[1, 900, 2048, 2049, 4000], T=2, device=DEV, page_size=64,
+                              n_needles=2)
+    O, lse, idx, cnt = run_layer(wl)
+    _check_layer(wl, O, lse, idx, cnt)
+
+
+def test_layer_decode_is_deterministic():
+    wl = make_decode_workload(device=DEV, **CONFIGS["verify_64k_t4"])
+    a = run_layer(wl)
+    b = run_layer(wl)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8) if x.dtype == torch.bfloat16 else x,
+                           y.view(torch.uint8) if y.dtype == torch.bfloat16 else y)
+
+
+def test_layer_decode_1m_context_sampled():
+    """Native 1,048,576-token context: scores at sampled positions and every
+    needle against the oracle; the selection bit-exact against the oracle's
+    top-k over the GPU scores; attention against the oracle over the selection."""
+    wl = make_decode_workload(device=DEV, **CONFIGS["ctx_1m"])
+    L = wl.layout.seq_lens[0]
+    scores = run_indexer(wl)
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([rng.choice(L, 8192, replace=False), wl.needles[0].numpy(),
+                                       np.arange(L - 300, L)]))
+    rows = torch.from_numpy(sample).to(DEV)
+    ref = oracle.indexer_scores(wl.q8[0].cpu().numpy(), wl.q_scale[0].cpu().numpy(), wl.w[0].cpu().numpy(),
+                                wl.k8[rows].cpu().numpy(), wl.k_scale[rows].cpu().numpy(),
+                                np.array([len(sample) - 1], np.int32))
+    assert_scores_close(scores[0][:, rows].cpu().numpy(), ref)
+    O, lse, idx, cnt = run_layer(wl)
+    gpu_scores = scores[0, 0].cpu().numpy()
+    ref_idx, ref_cnt = oracle.topk(gpu_scores, 2048)
+    assert int(cnt[0, 0]) == 2048
+    assert np.array_equal(idx[0, 0].cpu().numpy(), np.sort(ref_idx))
+    ref_o, ref_l = oracle_attention_rows(wl, 0, 0, idx[0, 0].cpu().numpy(), wl.sink, SM)
+    assert_attn_close(O[0, 0], ref_o, lse[0, 0], ref_l)
+
+
+def test_bad_positions_are_flagged_not_faulted():
+    wl = make_decode_workload(seed=70, seq_lens=[1000], T=1, device=DEV)
+    idx = torch.full((1, 1, 2048), -1, dtype=torch.int32, device=DEV)
+    idx[0, 0, :3] = torch.tensor([5, 999999, -3], dtype=torch.int32)
+    cnt = torch.tensor([[3]], dtype=torch.int32, device=DEV)
+    O = torch.empty((1, 1, 64, 128), dtype=torch.bfloat16, device=DEV)
+    ws = dsa.alloc_workspace(dsa.OP_SPARSE_ATTN, 1, 1, 1, 2048)
+    dsa.sparse_gqa_attn_decode(wl.Q, kv_for(wl, with_index=False), idx, cnt, 2048, wl.sink, SM, O, None, ws)
+    st, flags = dsa.dsa_check_device_status(ws)
+    assert st == dsa.DSA_ERR_DEVICE_BAD_INDEX and flags == (1 << dsa.DSA_ERR_DEVICE_BAD_INDEX)
+    ref_o, _ = oracle_attention_rows(wl, 0, 0, np.array([5]), wl.sink, SM)   # bad entries are skipped
+    assert_attn_close(O[0, 0], ref_o)
+    assert dsa.dsa_check_device_status(ws)[0] == dsa.DSA_OK   # reading clears the word

@@ -129,11 +129,11 @@ def _needle_positions(g: torch.Generator, L: int, n: int, mode: str) -> torch.Te
         return torch.randperm(L, generator=g)[:n].sort().values
     if mode == "zipf":
         # distance from the end r in [1, L] with P(r) ~ 1/r; duplicates resampled
+        # continuous inverse CDF of P(r) ~ 1/r on [1, L]: r = L^u
         chosen = set()
-        H = math.log(L) + 0.5772156649
         while len(chosen) < n:
             u = torch.rand(4 * n, generator=g, dtype=torch.float64)
-            r = torch.exp(u * H).floor().clamp(1, L).long()
+            r = torch.exp(u * math.log(L)).floor().clamp(1, L).long()
             for v in r.tolist():
                 if len(chosen) < n:
                     chosen.add(L - v)
