@@ -40,6 +40,16 @@ INDEXER_SRC = os.path.join(ROOT, "local_attention_decode_b200", "csrc", "indexer
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "indexer_ctx_1m_traffic.json")
 
 
+WORKLOAD_DESC = {
+    "ctx_1m": "ctx_1m: DSA decode layer-step, batch 1, 1 query token at position 1,048,575, context 1,048,576, "
+              "top-2048, 64 Q heads / 4 KV heads (GQA4), qk 192, v 128, sink, 256 Zipf needles",
+    "verify_64k_t4": "verify_64k_t4: DSA decode layer-step, batch 1, 4 query tokens (speculative verify block) at "
+                     "positions 65,532..65,535, context 65,536, top-2048, GQA4, sink, 64 needles",
+    "tiny_8k": "tiny_8k: DSA decode layer-step, batch 1, 1 query token, context 8,192, top-2048, GQA4, sink, "
+               "16 needles",
+}
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -171,7 +181,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = CONFIGS[WORKLOAD]
+    cfg = CONFIGS[args.workload]
     wl = make_decode_workload(device=dev, **cfg)
     B, T = wl.B, wl.T
     L = wl.layout.seq_lens[0]
@@ -250,8 +260,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
         "data": "synthetic",
         "config": {
-            "workload": "ctx_1m: DSA decode layer-step, batch 1, 1 query token at position 1,048,575, "
-                        "context 1,048,576, top-2048, 64 Q heads / 4 KV heads (GQA4), qk 192, v 128, sink",
+            "workload": WORKLOAD_DESC[args.workload],
             "batch": B, "query_tokens": T, "context": L, "top_k": TOP_K, "seed": cfg["seed"],
             "needles": cfg["n_needles"], "parallelism": f"replicas x{world}",
             "l2": "flushed between steps (256 MB write outside the timed events)",
@@ -417,6 +426,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m"], default=WORKLOAD,
+                    help="decode workload recipe (workloads.CONFIGS); the headline metric is on ctx_1m")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -438,7 +449,7 @@ def main():
     try:
         line = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            if world == 1:
+            if world == 1 and args.workload == WORKLOAD:
                 line["cpu_baseline"] = cpu_baseline_line()
             print(json.dumps(line), flush=True)
     finally:

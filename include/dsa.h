@@ -97,7 +97,8 @@ extern "C" {
  *           pos / page_size < max_pages; page ids < num_rows / page_size.
  * `num_rows` is the number of rows the buffers hold (bounds every access).
  * Unused members may be NULL (e.g. index_k for the attention calls, k / v
- * for the indexer).  All device pointers must be 16-byte aligned.
+ * for the indexer).  All device pointers must be 16-byte aligned.  The
+ * indexer calls with B > 1 on a contiguous cache need seq_stride % 16 == 0.
  */
 typedef struct dsa_kv {
     const void    *k;

@@ -92,6 +92,17 @@ static int check_kv_index(const dsa_kv_t *kv) {
     return DSA_OK;
 }
 
+// The indexer's tensor copies start at row b * seq_stride of a contiguous
+// cache; the fp32 scale copy needs that row to be a multiple of 4, so batched
+// contiguous caches need seq_stride % 16 == 0 (paged caches start every copy
+// at a page boundary).
+static int check_index_stride(const dsa_kv_t *kv, int B) {
+    if (!kv->block_table && B > 1 && kv->seq_stride % 16 != 0)
+        return fail(DSA_ERR_UNSUPPORTED_SHAPE, "contiguous index cache with B > 1 needs seq_stride %% 16 == 0 (got %lld)",
+                    (long long)kv->seq_stride);
+    return DSA_OK;
+}
+
 // ------------------------------------------------------------ workspace plan
 struct WsPlan {
     size_t status = 0, scores = 0, idx = 0, count = 0, topk = 0, part_o = 0, part_ml = 0, total = 0;
@@ -220,6 +231,7 @@ int dsa_indexer_scores(const void *q8, const float *q_scale, const float *w, con
     int rc = check_common(B, T);
     if (rc) return rc;
     if (rc = check_kv_index(kv); rc) return rc;
+    if (rc = check_index_stride(kv, B); rc) return rc;
     if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
     if (scores_stride < Lmax) return fail(DSA_ERR_INVALID_ARG, "scores_stride < Lmax");
     WsPlan wp;
@@ -304,6 +316,7 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
     int rc = check_common(B, T);
     if (rc) return rc;
     if (rc = check_kv_index(kv); rc) return rc;
+    if (rc = check_index_stride(kv, B); rc) return rc;
     if (rc = check_kv_backbone(kv); rc) return rc;
     if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
     if (top_k < 1 || top_k > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);

@@ -292,6 +292,8 @@ gather_attn_kernel(const Params p) {
 }
 
 // One warp per (query, head): merge the splits and the sink, normalise.
+// Lane j holds split j's (max, sum); the O partials are read with all loads of
+// a group independent of one another.  splits <= 32.
 __global__ void __launch_bounds__(128)
 combine_kernel(const float *part_o, const float *part_ml, int rows, int splits, const float *sink, int T,
                __nv_bfloat16 *O, float *lse) {
@@ -299,19 +301,34 @@ combine_kernel(const float *part_o, const float *part_ml, int rows, int splits, 
     if (gw >= rows) return;
     const int h = gw % DSA_Q_HEADS;
     const float *ml = part_ml + (int64_t)gw * splits * 2;
-    float M = sink ? sink[h] * kLog2e : -INFINITY;
-    for (int j = 0; j < splits; ++j) M = fmaxf(M, ml[2 * j]);
-    float L = 0.f;
+    const float mj = lane < splits ? ml[2 * lane] : -INFINITY;
+    const float lj = lane < splits ? ml[2 * lane + 1] : 0.f;
+    const float sk = sink ? __ldg(sink + h) * kLog2e : -INFINITY;
+    float M = fmaxf(mj, sk);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wj = (mj == -INFINITY) ? 0.f : exp2f(mj - M);
+    float L = lj * wj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (sink && M != -INFINITY) L += exp2f(sk - M);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-        if (sink) L = exp2f(sink[h] * kLog2e - M);
-        for (int j = 0; j < splits; ++j) {
-            const float mj = ml[2 * j];
-            if (mj == -INFINITY) continue;
-            const float wgt = exp2f(mj - M);
-            L += ml[2 * j + 1] * wgt;
-            float4 v = *reinterpret_cast<const float4 *>(part_o + ((int64_t)gw * splits + j) * DSA_V_DIM + lane * 4);
-            acc.x += v.x * wgt; acc.y += v.y * wgt; acc.z += v.z * wgt; acc.w += v.w * wgt;
+    const float *po = part_o + (int64_t)gw * splits * DSA_V_DIM + lane * 4;
+    for (int j0 = 0; j0 < splits; j0 += 8) {
+        float4 v[8];
+        float w[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int j = j0 + u;
+            w[u] = __shfl_sync(0xffffffffu, wj, j & 31);
+            v[u] = (j < splits && w[u] != 0.f) ? *reinterpret_cast<const float4 *>(po + (int64_t)j * DSA_V_DIM)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (j0 + u < splits && w[u] != 0.f) {
+                acc.x += v[u].x * w[u]; acc.y += v[u].y * w[u]; acc.z += v[u].z * w[u]; acc.w += v[u].w * w[u];
+            }
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;

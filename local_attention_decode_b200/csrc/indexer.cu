@@ -35,6 +35,13 @@ constexpr int kTile = 128;            // keys per tile = UMMA M
 constexpr int kKeyBytes = DSA_INDEX_DIM;  // 128 e4m3 codes per key
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
+constexpr int kKsStageBytes = 1024;   // key-scale slots of one stage
+
+// Byte offset, inside a stage's key-scale area, of the scale of tile row r.
+__host__ __device__ __forceinline__ int ks_slot_offset(int r, int R) {
+    const int slot = (R * 4 + 127) & ~127;
+    return (r / R) * slot + (r % R) * 4;
+}
 
 struct Params {
     const float *q_scale;
@@ -65,7 +72,9 @@ struct __align__(8) Bars {
 // Shared memory carve-up (base aligned to 1024 bytes):
 //   [0, S*16K)                    key tiles
 //   [S*16K, S*(16K + 2K*T))       query tiles
-//   then S*512 B                  key scales
+//   then S*1 KB                   key scales: one 128-byte aligned slot per TMA
+//                                 box (tensor copies need 128-byte aligned
+//                                 shared destinations), R*4 bytes used per slot
 //   then Bars, tmem address, per-sequence tables, per-warp epilogue constants
 struct Layout {
     uint32_t k_off, q_off, ks_off, bar_off, tmem_off, len_off, tile_off, epi_off, total;
@@ -73,7 +82,7 @@ struct Layout {
         k_off = 0;
         q_off = k_off + S * kTile * kKeyBytes;
         ks_off = q_off + S * 16 * T * kKeyBytes;
-        bar_off = ks_off + S * kTile * 4;
+        bar_off = ks_off + S * kKsStageBytes;
         tmem_off = bar_off + (uint32_t)sizeof(Bars);
         len_off = (tmem_off + 16 + 15) & ~15u;
         tile_off = len_off + 4 * (B + 1);
@@ -205,7 +214,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 if (i >= S && !mbar_wait(&bars->empty[s], ((i / S) & 1) ^ 1, p.status)) { alive = false; break; }
                 mbar_arrive_expect_tx(&bars->full[s], stage_tx);
                 uint8_t *kdst = smem + lay.k_off + s * kTile * kKeyBytes;
-                float *ksdst = reinterpret_cast<float *>(smem + lay.ks_off + s * kTile * 4);
+                uint8_t *ksdst = smem + lay.ks_off + s * kKsStageBytes;
                 tma_load_2d(smem + lay.q_off + s * N * kKeyBytes, &tmap_q, &bars->full[s], 0, b * T * 16);
                 const int R = p.rows_per_load;
                 for (int j = 0; j < kTile / R; ++j) {
@@ -217,7 +226,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                         if (!ok) { flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX); row = 0; }
                     }
                     tma_load_2d(kdst + j * R * kKeyBytes, &tmap_k, &bars->full[s], 0, (int32_t)row);
-                    tma_load_1d(ksdst + j * R, &tmap_ks, &bars->full[s], (int32_t)row);
+                    tma_load_1d(ksdst + ks_slot_offset(j * R, R), &tmap_ks, &bars->full[s], (int32_t)row);
                 }
                 ++issued;
                 if (++ti * kTile >= seq_len[b]) {   // next non-empty sequence
@@ -275,7 +284,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                       mbar_wait(&bars->full[s], (i / S) & 1, p.status);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
-            const float ks = reinterpret_cast<const float *>(smem + lay.ks_off + s * kTile * 4)[row_in_tile];
+            const float ks = *reinterpret_cast<const float *>(smem + lay.ks_off + s * kKsStageBytes +
+                                                              ks_slot_offset(row_in_tile, p.rows_per_load));
             const int64_t pos = (int64_t)ti * kTile + row_in_tile;
             const int len = seq_len[b];
             float *out = p.scores + (int64_t)b * T * p.scores_stride + pos;
@@ -322,15 +332,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-static int make_map(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
-                    const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz) {
+static int make_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
+                    const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz) {
     auto enc = get_encode();
     if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     uint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, dt, rank, const_cast<void *>(base), dims, strides_bytes, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    uint64_t no_strides[1] = {0};   // rank-1 maps take no strides; pass a valid pointer anyway
+    CUresult r = enc(map, dt, rank, const_cast<void *>(base), dims, strides_bytes ? strides_bytes : no_strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(DSA_ERR_INVALID_ARG, "tensor map encoding failed (CUresult %d)", (int)r);
+    if (r != CUDA_SUCCESS)
+        return fail(DSA_ERR_INVALID_ARG,
+                    "tensor map encoding failed for %s (CUresult %d; base %p, dims %llu x %llu, box %u x %u)", what,
+                    (int)r, base, (unsigned long long)dims[0], (unsigned long long)(rank > 1 ? dims[1] : 1),
+                    box[0], rank > 1 ? box[1] : 1u);
     return DSA_OK;
 }
 
@@ -350,14 +365,14 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream) {
         uint64_t dims[2] = {(uint64_t)kKeyBytes, (uint64_t)kv->num_rows};
         uint64_t strides[1] = {(uint64_t)kKeyBytes};
         uint32_t box[2] = {(uint32_t)kKeyBytes, (uint32_t)R};
-        int rc = make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->index_k, dims, strides, box,
+        int rc = make_map("index keys", &tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->index_k, dims, strides, box,
                           CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }
     {
         uint64_t dims[1] = {(uint64_t)kv->num_rows};
         uint32_t box[1] = {(uint32_t)R};
-        int rc = make_map(&tks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, kv->index_k_scale, dims, nullptr, box,
+        int rc = make_map("index key scales", &tks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, kv->index_k_scale, dims, nullptr, box,
                           CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc) return rc;
     }
@@ -365,7 +380,7 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream) {
         uint64_t dims[2] = {(uint64_t)kKeyBytes, (uint64_t)a.B * T * 16};
         uint64_t strides[1] = {(uint64_t)kKeyBytes};
         uint32_t box[2] = {(uint32_t)kKeyBytes, (uint32_t)N};
-        int rc = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q8, dims, strides, box,
+        int rc = make_map("index queries", &tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q8, dims, strides, box,
                           CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }

@@ -31,6 +31,7 @@ constexpr int kThreads = 512;
 constexpr int kBins = 2048;                 // largest digit: 11 bits
 constexpr int kMinChunk = 4096;             // keys per CTA below which a row is not split further
 constexpr int kMaxCacheKeys = 40 * 1024;    // 160 KB of cached keys per CTA
+constexpr int kUnroll = 8;                  // independent loads in flight per thread
 
 // Per-row scratch (u32 words), used only when C > 1.
 constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kCnt = 5120;
@@ -161,11 +162,37 @@ topk_kernel(const Params p) {
     const bool cached = len <= p.cache_keys;
     uint32_t *rs = C > 1 ? p.scratch + (int64_t)row * p.scratch_row_words : nullptr;
 
+    auto key_at = [&](int64_t j) -> uint32_t { return cached ? cache[j] : float_order_key(__ldg(src + lo + j)); };
+    // Visits keys j = base + u * kThreads + tid in batches of kUnroll per
+    // thread, all loads of a batch issued before any is used.
+    auto for_each_key = [&](auto &&fn) {
+        for (int64_t base = 0; base < len; base += (int64_t)kUnroll * kThreads) {
+            uint32_t kk[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t j = base + u * kThreads + threadIdx.x;
+                kk[u] = j < len ? key_at(j) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) fn(base + u * kThreads + threadIdx.x, kk[u]);
+        }
+    };
     if (cached) {
-        for (int64_t j = threadIdx.x; j < len; j += kThreads) cache[j] = float_order_key(__ldg(src + lo + j));
+        for (int64_t base = 0; base < len; base += (int64_t)kUnroll * kThreads) {
+            float v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t j = base + u * kThreads + threadIdx.x;
+                v[u] = j < len ? __ldg(src + lo + j) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t j = base + u * kThreads + threadIdx.x;
+                if (j < len) cache[j] = float_order_key(v[u]);
+            }
+        }
         __syncthreads();
     }
-    auto key_at = [&](int64_t j) -> uint32_t { return cached ? cache[j] : float_order_key(__ldg(src + lo + j)); };
 
     // ---- three digit rounds
     uint32_t prefix = 0, mask = 0, Krem = (uint32_t)K;
@@ -177,14 +204,12 @@ topk_kernel(const Params p) {
         for (int j = threadIdx.x; j < nb; j += kThreads) sh->hist[j] = 0;
         __syncthreads();
         // warp-aggregated increments: lanes that hit the same bin add once
-        for (int64_t base = 0; base < len; base += kThreads) {
-            const int64_t j = base + threadIdx.x;
-            uint32_t k = j < len ? key_at(j) : 0u;
+        for_each_key([&](int64_t j, uint32_t k) {
             bool active = j < len && (k & mask) == prefix;
             uint32_t bin = active ? (k >> sh_) & (nb - 1) : 0xFFFFFFFFu;
             uint32_t peers = __match_any_sync(0xffffffffu, bin);
             if (active && lane_id() == __ffs(peers) - 1) atomicAdd(&sh->hist[bin], (uint32_t)__popc(peers));
-        }
+        });
         __syncthreads();
         if (C > 1) {
             uint32_t *g = rs + hoff[r];
@@ -205,11 +230,10 @@ topk_kernel(const Params p) {
 
     // ---- per-CTA counts of keys > T* and == T*
     uint32_t gt = 0, eq = 0;
-    for (int64_t j = threadIdx.x; j < len; j += kThreads) {
-        uint32_t k = key_at(j);
-        gt += k > Tstar;
-        eq += k == Tstar;
-    }
+    for_each_key([&](int64_t j, uint32_t k) {
+        gt += j < len && k > Tstar;
+        eq += j < len && k == Tstar;
+    });
     uint32_t tot_gt, tot_eq;
     block_scan(gt, sh->warp_tmp, &tot_gt);
     block_scan(eq, sh->warp_tmp, &tot_eq);
@@ -271,12 +295,14 @@ topk_kernel(const Params p) {
     }
     if (c == 0 && threadIdx.x == 0) p.count[row] = K;
 
-    if (C > 1) {   // last CTA of the row out resets the barrier words
+    if (C > 1) {   // the last CTA of the row out clears the counts and the barrier words
         __syncthreads();
         if (threadIdx.x == 0) {
             uint32_t *bar = rs + kCnt + 2 * C;
+            __threadfence();
             uint32_t done = atomicAdd(bar + 1, 1u);
             if (done == (uint32_t)C - 1) {
+                for (int j = 0; j < 2 * C; ++j) rs[kCnt + j] = 0;
                 atomicExch(bar, 0u);
                 atomicExch(bar + 1, 0u);
             }

@@ -239,7 +239,7 @@ def test_layer_decode_matches_oracle(name):
 
 
 def test_layer_decode_short_contexts_and_pages():
-    wl = make_decode_workload(seed=60, seq_lens=[1, 900, 2048, 2049, 4000], T=2, device=DEV, page_size=64,
+    wl = make_decode_workload(seed=60, seq_lens=[2, 900, 2048, 2049, 4000], T=2, device=DEV, page_size=64,
                               n_needles=2)
     O, lse, idx, cnt = run_layer(wl)
     _check_layer(wl, O, lse, idx, cnt)

@@ -80,7 +80,7 @@ def make_layout(seq_lens, page_size: int = 0, seed: int = 0, device="cpu") -> KV
     seq_lens = [int(x) for x in seq_lens]
     B = len(seq_lens)
     if page_size <= 0:
-        stride = max(seq_lens)
+        stride = max(seq_lens) if B == 1 else -(-max(seq_lens) // 128) * 128
         return KVLayout(seq_lens=seq_lens, seq_stride=stride, num_rows=B * stride)
     pages = [math.ceil(L / page_size) for L in seq_lens]
     total = sum(pages)
