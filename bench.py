@@ -9,7 +9,9 @@ Each rank runs its own replica of the workload (the steps are independent
 problems: weak scaling, no data-path collective); ``value`` is the tokens all
 ranks decoded divided by the slowest rank's device time.
 
-L2 is flushed (256 MB write) between timed steps, outside the timed events.
+L2 is flushed between timed steps, outside the timed events: a 256 MB write
+evicts everything, then a 256 MB read retires the dirty lines, so each step
+starts cold and clean.
 Per-stage CUDA events recorded by the library itself give the indexer's
 duration for the roofline.  ``--impl reference`` times the CPU oracle on a
 bounded sample of the same workload instead (rank 0 only).
@@ -143,6 +145,23 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+class L2Flush:
+    """Leaves L2 cold and clean between timed steps: write a 256 MB buffer (evicts
+    everything), then read another 256 MB buffer so the write-backs of the dirty
+    lines happen here, not inside the next timed step."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        self.out.copy_(self.r.sum())
+
+
 # ------------------------------------------------------- multi-rank helpers
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -192,7 +211,7 @@ def run_ours(args, rank, world, local_rank):
     idx = torch.empty((B, T, TOP_K), dtype=torch.int32, device=dev)
     cnt = torch.empty((B, T), dtype=torch.int32, device=dev)
     ws = dsa.alloc_workspace(dsa.OP_LAYER, B, T, L, TOP_K, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def new_events(n):
@@ -206,7 +225,7 @@ def run_ours(args, rank, world, local_rank):
                              None, idx, cnt, ws, stage_events=events)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize(dev)
     st, _ = dsa.dsa_check_device_status(ws)
@@ -221,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     sampler.start()
     for i in range(K):
-        flush.zero_()
+        flush()
         step(stage[i])
     torch.cuda.synchronize(dev)
     barrier(dev)
@@ -263,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
             "workload": WORKLOAD_DESC[args.workload],
             "batch": B, "query_tokens": T, "context": L, "top_k": TOP_K, "seed": cfg["seed"],
             "needles": cfg["n_needles"], "parallelism": f"replicas x{world}",
-            "l2": "flushed between steps (256 MB write outside the timed events)",
+            "l2": "flushed between steps outside the timed events (256 MB write, then 256 MB read so no dirty lines remain)",
         },
         "us_per_layer_step": total_s * 1e6 / K,
         "stage_us_median": {
@@ -332,7 +351,7 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
         h_idx.copy_(idx, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize(dev)
     K = args.steps
@@ -340,7 +359,7 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
     barrier(dev)
     torch.cuda.synchronize(dev)
     for i in range(K):
-        flush.zero_()
+        flush()
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)

@@ -9,16 +9,18 @@
 // the kernel takes the raw e4m3 dot products from the tensor cores and applies
 // the scales in the epilogue: I = ks * sum_h (w_h qs_h) * relu(dot_h).
 //
-// Design (one persistent CTA per SM, warp-specialised):
+// Design (persistent, two CTAs per SM, warp-specialised):
 //   warp 0  TMA producer: per 128-key tile, loads the e4m3 key tile
 //           [128 x 128 B] (128-byte swizzle), the 128 fp32 key scales and the
 //           query's index heads [16T x 128 B] into one pipeline stage.
 //   warp 1  MMA issuer: D[128 keys x 16T] += K_tile[128 x 32] * Q^T[32 x 16T]
 //           with tcgen05.mma kind::f8f6f4 (four K=32 steps), fp32 accumulators
-//           in TMEM, two accumulator buffers so the epilogue of tile i
-//           overlaps the MMA of tile i + 1.
-//   warps 2-5 epilogue: tcgen05.ld of one key row per thread, ReLU, per-head
-//           weighting, key scale, causal mask, coalesced fp32 store.
+//           in TMEM, one accumulator per epilogue group so the epilogue of
+//           tile i overlaps the MMA of tile i + 1.
+//   warps 2-9 epilogue, two groups of four warps (one per TMEM lane quarter),
+//           each group with its own accumulator and every other tile:
+//           tcgen05.ld of one key row per thread, ReLU, per-head weighting, key
+//           scale, causal mask, coalesced fp32 store.
 // Each CTA owns a contiguous range of the (sequence, tile) list, so the HBM
 // stream of every SM is sequential.
 #include <algorithm>
@@ -33,8 +35,15 @@ namespace indexer {
 
 constexpr int kTile = 128;            // keys per tile = UMMA M
 constexpr int kKeyBytes = DSA_INDEX_DIM;  // 128 e4m3 codes per key
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
+constexpr int kMaxGroups = 2;         // epilogue groups (4 warps each), one TMEM accumulator per group
+constexpr int kThreads = 64 + 128 * kMaxGroups;
+// Two CTAs share each SM: a single CTA's TMA pipeline does not reach the
+// per-SM share of HBM bandwidth on its own (measured: 0.65 us per 16 KB tile
+// with one pipeline per SM, twice the throughput with two).  Each CTA keeps
+// its shared memory under half an SM and its TMEM under 256 columns.
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxTmemCols = 512 / kCtasPerSm;
+constexpr int kEpiWarps = 4;          // warps per epilogue group (one per TMEM lane quarter)
 constexpr int kKsStageBytes = 1024;   // key-scale slots of one stage
 
 // Byte offset, inside a stage's key-scale area, of the scale of tile row r.
@@ -59,13 +68,14 @@ struct Params {
     uint32_t *status;
     int stages;
     int rows_per_load;   // R: rows per TMA box (128, or the page size when pages are smaller)
+    int groups;          // epilogue groups in use (1..kMaxGroups)
 };
 
 struct __align__(8) Bars {
     uint64_t full[8];
     uint64_t empty[8];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t tfull[kMaxGroups];
+    uint64_t tempty[kMaxGroups];
     uint64_t mma_done;
 };
 
@@ -90,7 +100,7 @@ struct Layout {
         epi_off = tile_off + 4 * (B + 1);
         epi_off = (epi_off + 15) & ~15u;
         // per epilogue warp: 16*T coefficients + T positions
-        total = epi_off + kEpiWarps * (16 * T + T) * 4;
+        total = epi_off + kMaxGroups * kEpiWarps * (16 * T + T) * 4;
     }
 };
 
@@ -104,7 +114,7 @@ __device__ __forceinline__ int64_t row_of(const Params &p, int b, int64_t pos, b
     return row;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
                const __grid_constant__ CUtensorMap tmap_q, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -161,15 +171,16 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     const int n_tiles = per + ((int)blockIdx.x < rem ? 1 : 0);
     if (n_tiles == 0) return;   // uniform across the CTA
 
-    // --- barriers and TMEM
+    // --- barriers and TMEM (one N-column fp32 accumulator per epilogue group)
+    const int GE = p.groups;
     uint32_t tmem_cols = 32;
-    while (tmem_cols < (uint32_t)(2 * N)) tmem_cols <<= 1;
+    while (tmem_cols < (uint32_t)(GE * N)) tmem_cols <<= 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1 + kEpiWarps);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < GE; ++a) {
             mbar_init(&bars->tfull[a], 1);
             mbar_init(&bars->tempty[a], kEpiWarps);
         }
@@ -243,9 +254,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_e4m3_f32(kTile, N);
             for (int i = 0; i < n_tiles; ++i) {
-                const int s = i % S, a = i & 1;
+                const int s = i % S, a = i % GE;
                 if (!mbar_wait(&bars->full[s], (i / S) & 1, p.status)) break;
-                if (i >= 2 && !mbar_wait(&bars->tempty[a], ((i >> 1) & 1) ^ 1, p.status)) break;
+                if (i >= GE && !mbar_wait(&bars->tempty[a], ((i / GE) & 1) ^ 1, p.status)) break;
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(smem + lay.k_off + s * kTile * kKeyBytes);
                 const uint32_t b_addr = smem_u32(smem + lay.q_off + s * N * kKeyBytes);
@@ -262,16 +273,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;                  // 0..3
+        // group e (warps 2+4e .. 5+4e) takes tiles e, e + GE, e + 2 GE, ... into accumulator e
+        const int ew = warp - 2;                  // 0..15
+        const int a = ew / kEpiWarps;             // group == accumulator
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int row_in_tile = quarter * 32 + lane;
         float *coef = reinterpret_cast<float *>(smem + lay.epi_off) + ew * (17 * T);
         int32_t *qp = reinterpret_cast<int32_t *>(coef + 16 * T);
-        int b, ti;
-        locate(t_begin, b, ti);
         int cur_b = -1;
-        for (int i = 0; i < n_tiles; ++i) {
-            const int s = i % S, a = i & 1;
+        for (int i = a; i < n_tiles && a < GE; i += GE) {
+            const int s = i % S;
+            int b, ti;
+            locate(t_begin + i, b, ti);
             if (b != cur_b) {   // per-sequence constants: w * q_scale and query positions
                 __syncwarp();
                 for (int j = lane; j < 16 * T; j += 32)
@@ -280,7 +293,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 __syncwarp();
                 cur_b = b;
             }
-            bool ok = mbar_wait(&bars->tfull[a], (i >> 1) & 1, p.status) &&
+            bool ok = mbar_wait(&bars->tfull[a], (i / GE) & 1, p.status) &&
                       mbar_wait(&bars->full[s], (i / S) & 1, p.status);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
@@ -302,10 +315,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             if (lane == 0) {
                 mbar_arrive(&bars->tempty[a]);
                 mbar_arrive(&bars->empty[s]);
-            }
-            if (++ti * kTile >= seq_len[b]) {
-                ti = 0;
-                do { ++b; } while (b < B && seq_len[b] == 0);
             }
         }
     }
@@ -385,8 +394,8 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream) {
         if (rc) return rc;
     }
 
-    // stages: as many as fit next to the tables (2..8)
-    const size_t budget = dev.smem_optin - 1024;
+    // stages: as many as fit next to the tables (2..8) in half an SM's shared memory
+    const size_t budget = std::min<size_t>(dev.smem_optin, 228 * 1024 / kCtasPerSm - 1024) - 1024;
     int S = 8;
     while (S > 2 && Layout(S, T, a.B).total > budget) --S;
     Layout lay(S, T, a.B);
@@ -410,9 +419,10 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream) {
     p.status = a.status;
     p.stages = S;
     p.rows_per_load = R;
+    p.groups = std::max(1, std::min(kMaxGroups, kMaxTmemCols / N));
 
     const int64_t max_tiles = (int64_t)a.B * ((a.Lmax + kTile - 1) / kTile);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(dev.num_sms, max_tiles));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)dev.num_sms * kCtasPerSm, max_tiles));
 
     cudaError_t e = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer)");
