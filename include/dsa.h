@@ -209,6 +209,36 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
                      int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
                      void *stream, void *const *stage_events);
 
+/*
+ * dsa_topk_select_noalloc -- the selection of dsa_topk_select for callers
+ * that cannot allocate device memory and so cannot provide a workspace: a
+ * framework that owns every device allocation and refuses new ones after it
+ * starts, a latency-critical loop that must never reach the allocator, a
+ * plug-in handed only its input and output buffers.  (The pages have no
+ * counterpart; this is an interface convenience of this library.)
+ *
+ * Same arguments and results as dsa_topk_select, without ws / ws_bytes.  The
+ * scratch is a 2 MiB array in device memory declared by the library itself;
+ * every GPU that loads the library holds it until the process exits.  A call
+ * whose scratch need exceeds it returns DSA_ERR_UNSUPPORTED_SHAPE with a
+ * message (use dsa_topk_select with a workspace then); on a 148-SM B200 the
+ * largest need is about 1.6 MB (74 query rows split two CTAs each), so every
+ * shape dsa_topk_select accepts fits.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents; each call clears the part that must start at zero
+ *     (cudaMemsetAsync on `stream`) before its kernel.  Calls that may overlap
+ *     on the GPU (different streams, or concurrent host threads) race on the
+ *     array: serialise them.
+ *   - Device-side status (bad positions, a bounded wait running out) is
+ *     recorded in the array but not reported by this entry point.
+ */
+int dsa_topk_select_noalloc(const float *scores, int64_t scores_stride, const int32_t *q_pos, int B, int T,
+                            int64_t Lmax, int top_k, int32_t *idx, int32_t *count, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,7 +39,7 @@ OP_INDEXER, OP_TOPK, OP_SPARSE_ATTN, OP_SWA_ATTN, OP_LAYER = range(5)
 
 EXPORTED = ("dsa_last_error", "dsa_get_dims", "dsa_workspace_size", "dsa_workspace_init",
             "dsa_check_device_status", "dsa_indexer_scores", "dsa_topk_select",
-            "sparse_gqa_attn_decode", "swa_attn_decode", "dsa_layer_decode")
+            "sparse_gqa_attn_decode", "swa_attn_decode", "dsa_layer_decode", "dsa_topk_select_noalloc")
 
 
 class DSAError(RuntimeError):
@@ -76,6 +76,7 @@ _lib.dsa_indexer_scores.argtypes = [P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I
 _lib.dsa_topk_select.argtypes = [P, I64, P, I32, I32, I64, I32, P, P, P, SZ, P]
 _lib.sparse_gqa_attn_decode.argtypes = [P, ctypes.POINTER(dsa_kv_t), P, P, I32, I32, I32, P, F32, P, P, P, SZ, P]
 _lib.swa_attn_decode.argtypes = [P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I32, P, F32, P, P, P, SZ, P]
+_lib.dsa_topk_select_noalloc.argtypes = [P, I64, P, I32, I32, I64, I32, P, P, P]
 _lib.dsa_layer_decode.argtypes = [P, P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I64, I32, P, F32, P, P, P, P,
                                   P, SZ, P, P]
 for _name in EXPORTED[1:]:
@@ -197,6 +198,16 @@ def dsa_topk_select(scores, q_pos, Lmax: int, top_k: int, idx, count, ws, stream
                                 _ptr(q_pos, torch.int32, "q_pos"), B, T, int(Lmax), int(top_k),
                                 _ptr(idx, torch.int32, "idx"), _ptr(count, torch.int32, "count"),
                                 _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
+def dsa_topk_select_noalloc(scores, q_pos, Lmax: int, top_k: int, idx, count, stream=None):
+    """dsa_topk_select without a workspace: the library's own 2 MiB device
+    scratch is used (see include/dsa.h for who needs this and its limits)."""
+    B, T = q_pos.shape
+    _check(_lib.dsa_topk_select_noalloc(_ptr(scores, torch.float32, "scores"), scores.shape[-1],
+                                        _ptr(q_pos, torch.int32, "q_pos"), B, T, int(Lmax), int(top_k),
+                                        _ptr(idx, torch.int32, "idx"), _ptr(count, torch.int32, "count"),
+                                        _stream(stream)))
 
 
 def sparse_gqa_attn_decode(Q, kv: KV, idx, count, top_k: int, sink, sm_scale: float, O, lse=None, ws=None,
