@@ -38,8 +38,9 @@ L_CTX = 1048576
 TOP_K = 2048
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-INDEXER_SRC = os.path.join(ROOT, "local_attention_decode_b200", "csrc", "indexer.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "indexer_ctx_1m_traffic.json")
+CSRC = os.path.join(ROOT, "local_attention_decode_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_ctx_1m.json")
+FUSED_MAX_ROWS = 16   # dsa_layer_decode runs as one fused kernel for B * T <= 16
 
 
 WORKLOAD_DESC = {
@@ -74,15 +75,24 @@ def gathered_bytes(T: int, top_k: int, G: int = 4) -> int:
     return T * top_k * G * (192 + 128) * 2
 
 
-def recorded_traffic():
-    """DRAM bytes per indexer launch from the committed ncu summary, if it was
-    taken on the current indexer source; else None."""
+def kernel_sources_sha() -> str:
+    """Hash of the CUDA sources the timed kernels are built from."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(CSRC, name), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on the current kernel sources; else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
-        sha = hashlib.sha256(open(INDEXER_SRC, "rb").read()).hexdigest()
-        if d.get("indexer_cu_sha256") == sha:
-            return int(d["traffic_bytes_per_launch"])
+        if d.get("sources_sha256") == kernel_sources_sha() and kernel in d.get("kernels", {}):
+            return int(d["kernels"][kernel]["dram_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -255,6 +265,25 @@ def run_ours(args, rank, world, local_rank):
     st, _ = dsa.dsa_check_device_status(ws)
     if st != dsa.DSA_OK:
         raise RuntimeError(f"device status {st} after the timed steps")
+    fused = B * T <= FUSED_MAX_ROWS
+
+    # the indexer on its own (dsa_indexer_scores), same inputs, for its HBM rate
+    idx_ws = dsa.alloc_workspace(dsa.OP_INDEXER, B, T, L, 1, device=dev)
+    scores = torch.empty((B, T, L), dtype=torch.float32, device=dev)
+    ikv = dsa.KV(index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G, seq_stride=wl.layout.seq_stride,
+                 num_rows=wl.layout.num_rows)
+    K2 = min(K, 200)
+    iev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
+    for i in range(3 + K2):
+        flush()
+        if i >= 3:
+            iev[i - 3][0].record(stream)
+        dsa.dsa_indexer_scores(wl.q8, wl.q_scale, wl.w, ikv, wl.q_pos, L, scores, idx_ws)
+        if i >= 3:
+            iev[i - 3][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ind_ms = [a.elapsed_time(b) for a, b in iev]
+    del scores
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush)
@@ -262,9 +291,14 @@ def run_ours(args, rank, world, local_rank):
     tokens = B * T
     value = throughput(tokens, K, world, total_s)
     peak, peak_kind = measured_peaks()
-    idx_avg_s = sum(idx_ms) / K / 1e3
     ib = indexer_bytes(L, T)
-    achieved = ib / idx_avg_s / 1e9
+    layer_bytes = ib + gathered_bytes(T, TOP_K)
+    ind_avg_s = sum(ind_ms) / K2 / 1e3
+    if fused:   # one kernel does the whole step: its roofline is the whole step's bytes
+        kern, kern_bytes, kern_avg_s = "dsa_layer_fused_kernel", layer_bytes, total_s / K
+    else:
+        kern, kern_bytes, kern_avg_s = "indexer_kernel", ib, sum(idx_ms) / K / 1e3
+    achieved = kern_bytes / kern_avg_s / 1e9
     line = {
         "metric": METRIC,
         "value": value,
@@ -285,9 +319,15 @@ def run_ours(args, rank, world, local_rank):
             "l2": "flushed between steps outside the timed events (256 MB write, then 256 MB read so no dirty lines remain)",
         },
         "us_per_layer_step": total_s * 1e6 / K,
-        "stage_us_median": {
+        "path": "one fused cooperative kernel" if fused else "four kernels",
+        "stage_us_median": ({"fused_layer_step": statistics.median(step_ms) * 1e3} if fused else {
             "indexer": statistics.median(idx_ms) * 1e3, "topk": statistics.median(topk_ms) * 1e3,
             "attention": statistics.median(attn_ms) * 1e3, "combine": statistics.median(comb_ms) * 1e3,
+        }),
+        "indexer_standalone": {
+            "us_median": statistics.median(ind_ms) * 1e3, "us_mean": ind_avg_s * 1e6, "bytes": ib,
+            "GBps": ib / ind_avg_s / 1e9, "frac_of_measured_peak": ib / ind_avg_s / 1e9 / peak,
+            "frac_of_8TBps_nominal": ib / ind_avg_s / 1e9 / NOMINAL_HBM_GBS,
         },
         "layer_step_byte_roofline_us": {
             "bytes": ib + gathered_bytes(T, TOP_K),
@@ -295,14 +335,14 @@ def run_ours(args, rank, world, local_rank):
             "at_8TBps_nominal": (ib + gathered_bytes(T, TOP_K)) / (NOMINAL_HBM_GBS * 1e9) * 1e6,
         },
         "roofline": {
-            "kernel": "indexer_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+            "kernel": kern, "bound": "hbm", "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
             "frac_of_8TBps_nominal": achieved / NOMINAL_HBM_GBS,
-            "traffic": recorded_traffic(), "algorithmic_bytes_per_launch": ib,
-            "avg_launch_us": idx_avg_s * 1e6,
+            "traffic": recorded_traffic(kern), "algorithmic_bytes_per_launch": kern_bytes,
+            "avg_launch_us": kern_avg_s * 1e6,
         },
         "e2e": e2e,
-        "gpu_launches": 4 * K,
+        "gpu_launches": (1 if fused else 4) * K,
         "clocks": clocks,
     }
     return line

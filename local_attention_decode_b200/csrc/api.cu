@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -107,6 +108,7 @@ static int check_index_stride(const dsa_kv_t *kv, int B) {
 struct WsPlan {
     size_t status = 0, scores = 0, idx = 0, count = 0, topk = 0, part_o = 0, part_ml = 0, total = 0;
     TopkPlan tp;
+    FusedPlan fp;
 };
 
 static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan *w) {
@@ -137,10 +139,11 @@ static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan 
         case DSA_OP_LAYER: {
             int rc = plan_topk(B, T, Lmax, top_k, &w->tp);
             if (rc) return rc;
+            if ((rc = plan_fused(B, T, Lmax, top_k, &w->fp))) return rc;
             w->scores = take((size_t)B * T * Lmax * 4);
             w->idx = take((size_t)B * T * top_k * 4);
             w->count = take((size_t)B * T * 4);
-            w->topk = take(w->tp.scratch_bytes);
+            w->topk = take(std::max(w->tp.scratch_bytes, w->fp.ok ? w->fp.scratch_bytes : 0));
             const int splits = (top_k + kAttnChunk - 1) / kAttnChunk;
             const size_t rows = (size_t)B * T * DSA_Q_HEADS * splits;
             w->part_o = take(rows * DSA_V_DIM * 4);
@@ -332,6 +335,35 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
 
     if (rc = record(stage_events, 0, s); rc) return rc;
     IndexerArgs ia{static_cast<const uint8_t *>(q8), q_scale, w, kv, q_pos, B, T, Lmax, scores, Lmax, status};
+    if (wp.fp.ok) {
+        // one cooperative launch for the whole layer-step
+        AttnArgs a;
+        a.Q = static_cast<const __nv_bfloat16 *>(Q);
+        a.kv = kv;
+        a.idx = idx;
+        a.count = count;
+        a.idx_stride = top_k;
+        a.q_pos = nullptr;
+        a.window = 0;
+        a.B = B;
+        a.T = T;
+        a.max_keys = top_k;
+        a.sink = sink;
+        a.sm_scale = sm_scale;
+        a.O = static_cast<__nv_bfloat16 *>(O);
+        a.lse = lse;
+        a.part_o = at<float>(ws, wp.part_o);
+        a.part_ml = at<float>(ws, wp.part_ml);
+        a.status = status;
+        rc = launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s);
+        if (rc == DSA_OK) {
+            for (int i = 1; i <= 4; ++i)
+                if (rc = record(stage_events, i, s); rc) return rc;
+            return DSA_OK;
+        }
+        if (rc != DSA_ERR_UNSUPPORTED_SHAPE) return rc;
+        // the fused kernel does not fit this shape: run the separate kernels
+    }
     if (rc = launch_indexer(ia, s); rc) return rc;
     if (rc = record(stage_events, 1, s); rc) return rc;
     if (rc = launch_topk(wp.tp, scores, Lmax, q_pos, top_k, idx, count, at<uint32_t>(ws, wp.topk), status, s); rc)

@@ -1,344 +1,27 @@
-// attention.cu -- split-KV gather attention for decode, with a per-head sink.
-//
-// For each query head h of query (b, t), over a key set S (the selected
-// top-k positions of a DSA layer, or the window {p-W+1..p} of an SWA layer):
-//   s_i = sm_scale * Q[h] . K[row(b, i)][g],   g = h / (64 / G)
-//   O[h] = sum_i e^{s_i} V[row(b, i)][g] / (sum_i e^{s_i} + e^{sink_h})
-// ("Naive-N0.5-Flash: no full-attention layers, and a runtime built by AI":
-// property table -- 64 query heads, qk dim 192, v dim 128, GQA4 / GQA8;
-// "Inside a DSA layer" -- the main heads gather and attend to only the
-// selected keys; the sink column in the softmax).
-//
-// Kernel 1 (gather_attn_kernel), grid (splits, G, B*T), 4 warps: one CTA
-// takes 64 keys of one KV head, gathers their K and V rows into shared memory
-// with 16-byte cp.async, and computes for the 64/G query heads of that group
-//   S = Q K^T  and  O = softmax_partial(S) V
-// on the tensor cores (mma.sync m16n8k16 bf16 -> fp32; the query heads of a
-// group form the 16-row M dimension).  Each warp owns 16 keys; the four warps
-// merge their (max, sum, O) in shared memory and the CTA writes one partial.
-// Kernel 2 (combine_kernel): log-sum-exp merge of the partials of all splits
-// plus the sink term, normalisation, bf16 output and optional lse.
+// attention.cu -- standalone split-KV attention kernels (sparse_gqa_attn_decode,
+// swa_attn_decode) and their launcher.  The device code is in
+// attention_impl.cuh.
 #include <algorithm>
-#include <cmath>
 
-#include "common.cuh"
-#include "kernels.h"
+#include "attention_impl.cuh"
 
 namespace dsa {
 namespace attn {
-
-constexpr int kChunk = kAttnChunk;   // keys per CTA
-constexpr int kThreads = 128;
-constexpr int kQS = DSA_QK_DIM + 8;  // padded smem row stride of Q and K (elements)
-constexpr int kVS = DSA_V_DIM + 8;   // padded smem row stride of V
-constexpr float kLog2e = 1.4426950408889634f;
-
-struct Params {
-    const __nv_bfloat16 *Q;
-    const __nv_bfloat16 *K;
-    const __nv_bfloat16 *V;
-    int G;
-    const int32_t *block_table;
-    int32_t max_pages, page_size;
-    int64_t seq_stride, num_rows;
-    const int32_t *idx;
-    const int32_t *count;
-    int idx_stride;
-    const int32_t *q_pos;
-    int window;
-    int T;
-    int splits;
-    float scale_log2;   // sm_scale * log2(e)
-    float *part_o;
-    float *part_ml;
-    uint32_t *status;
-};
-
-struct Smem {
-    __nv_bfloat16 q[16 * kQS];
-    __nv_bfloat16 k[kChunk * kQS];
-    __nv_bfloat16 v[kChunk * kVS];
-    int64_t row[kChunk];
-    float m[4][16];
-    float l[4][16];
-};
-
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
-__device__ __forceinline__ bool key_row(const Params &p, int b, int64_t pos, int64_t *row) {
-    if (pos < 0) return false;
-    if (p.block_table == nullptr) {
-        if (pos >= p.seq_stride) return false;
-        *row = (int64_t)b * p.seq_stride + pos;
-    } else {
-        int64_t page = pos / p.page_size;
-        if (page >= p.max_pages) return false;
-        int32_t id = __ldg(p.block_table + (int64_t)b * p.max_pages + page);
-        if (id < 0) return false;
-        *row = (int64_t)id * p.page_size + pos % p.page_size;
-    }
-    return *row < p.num_rows;
-}
 
 __global__ void __launch_bounds__(kThreads)
 gather_attn_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    const int split = blockIdx.x, g = blockIdx.y, bt = blockIdx.z;
-    const int b = bt / p.T;
-    const int hpg = DSA_Q_HEADS / p.G;
-    const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
-
-    // ---- the key set of this split
-    int n_total, win_lo = 0;
-    if (p.idx) {
-        n_total = min(__ldg(p.count + bt), p.idx_stride);
-    } else {
-        const int32_t pq = __ldg(p.q_pos + bt);
-        win_lo = max(0, pq - p.window + 1);
-        n_total = pq >= 0 ? pq - win_lo + 1 : 0;
-    }
-    const int k0 = split * kChunk;
-    const int nk = min(kChunk, n_total - k0);
-    float *ml = p.part_ml + (((int64_t)bt * DSA_Q_HEADS + g * hpg) * p.splits + split) * 2;
-    if (nk <= 0) {   // empty split: contributes nothing to the combine
-        if (tid < hpg) {
-            ml[(int64_t)tid * p.splits * 2 + 0] = -INFINITY;
-            ml[(int64_t)tid * p.splits * 2 + 1] = 0.f;
-        }
-        return;
-    }
-
-    // ---- positions -> cache rows (invalid ones are flagged and masked)
-    if (tid < kChunk) {
-        int64_t row = -1;
-        if (tid < nk) {
-            int64_t pos = p.idx ? (int64_t)__ldg(p.idx + (int64_t)bt * p.idx_stride + k0 + tid)
-                                : (int64_t)(win_lo + k0 + tid);
-            if (!key_row(p, b, pos, &row)) {
-                flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX);
-                row = -1;
-            }
-        }
-        sm.row[tid] = row;
-    }
-    // ---- Q rows of this head group (rows >= hpg are zero)
-    const __nv_bfloat16 *qg = p.Q + ((int64_t)bt * DSA_Q_HEADS + g * hpg) * DSA_QK_DIM;
-    for (int c = tid; c < 16 * (DSA_QK_DIM / 8); c += kThreads) {
-        int r = c / (DSA_QK_DIM / 8), col = (c % (DSA_QK_DIM / 8)) * 8;
-        __nv_bfloat16 *dst = sm.q + r * kQS + col;
-        if (r < hpg) cp_async16(dst, qg + (int64_t)r * DSA_QK_DIM + col);
-        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    // ---- gather K and V rows
-    const int G = p.G;
-    for (int c = tid; c < kChunk * (DSA_QK_DIM / 8); c += kThreads) {
-        int r = c / (DSA_QK_DIM / 8), col = (c % (DSA_QK_DIM / 8)) * 8;
-        __nv_bfloat16 *dst = sm.k + r * kQS + col;
-        int64_t row = sm.row[r];
-        if (row >= 0) cp_async16(dst, p.K + (row * G + g) * DSA_QK_DIM + col);
-        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
-    for (int c = tid; c < kChunk * (DSA_V_DIM / 8); c += kThreads) {
-        int r = c / (DSA_V_DIM / 8), col = (c % (DSA_V_DIM / 8)) * 8;
-        __nv_bfloat16 *dst = sm.v + r * kVS + col;
-        int64_t row = sm.row[r];
-        if (row >= 0) cp_async16(dst, p.V + (row * G + g) * DSA_V_DIM + col);
-        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-
-    // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8)
-    const int key0 = warp * 16;
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    const uint32_t q_base = smem_u32(sm.q), k_base = smem_u32(sm.k), v_base = smem_u32(sm.v);
-#pragma unroll
-    for (int kk = 0; kk < DSA_QK_DIM / 16; ++kk) {
-        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-        ldsm_x4(q_base + ((lane & 15) * kQS + kk * 16 + (lane >> 4) * 8) * 2, a0, a1, a2, a3);
-        ldsm_x4(k_base + ((key0 + (lane >> 4) * 8 + (lane & 7)) * kQS + kk * 16 + ((lane >> 3) & 1) * 8) * 2,
-                b0, b1, b2, b3);
-        mma_bf16(s[0], a0, a1, a2, a3, b0, b1);
-        mma_bf16(s[1], a0, a1, a2, a3, b2, b3);
-    }
-
-    // ---- partial softmax (log2 domain); rows g0 = lane/4 and g0 + 8
-    const int g0 = lane >> 2, cq = lane & 3;
-    float mrow[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int key = key0 + nt * 8 + cq * 2 + (e & 1);
-            float v = (key < nk && sm.row[key] >= 0) ? s[nt][e] * p.scale_log2 : -INFINITY;
-            s[nt][e] = v;
-            mrow[e >> 1] = fmaxf(mrow[e >> 1], v);
-        }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        mrow[r] = fmaxf(mrow[r], __shfl_xor_sync(0xffffffffu, mrow[r], 1));
-        mrow[r] = fmaxf(mrow[r], __shfl_xor_sync(0xffffffffu, mrow[r], 2));
-    }
-    float lrow[2] = {0.f, 0.f};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float m = mrow[e >> 1];
-            const float pe = (m == -INFINITY) ? 0.f : exp2f(s[nt][e] - m);
-            s[nt][e] = pe;
-            lrow[e >> 1] += pe;
-        }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
-        lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
-    }
-
-    // ---- O_w = P V (P as the A operand straight from the S accumulators)
-    const uint32_t pa0 = pack_bf16(s[0][0], s[0][1]), pa1 = pack_bf16(s[0][2], s[0][3]);
-    const uint32_t pa2 = pack_bf16(s[1][0], s[1][1]), pa3 = pack_bf16(s[1][2], s[1][3]);
-    float o[DSA_V_DIM / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < DSA_V_DIM / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-#pragma unroll
-    for (int dp = 0; dp < DSA_V_DIM / 16; ++dp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(v_base + ((key0 + (lane & 7) + ((lane >> 3) & 1) * 8) * kVS + dp * 16 + (lane >> 4) * 8) * 2,
-                  b0, b1, b2, b3);
-        mma_bf16(o[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
-        mma_bf16(o[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
-    }
-
-    // ---- merge the four warps: (m, l) per row, then O through shared memory
-    if (cq == 0) {
-        sm.m[warp][g0] = mrow[0];
-        sm.m[warp][g0 + 8] = mrow[1];
-        sm.l[warp][g0] = lrow[0];
-        sm.l[warp][g0 + 8] = lrow[1];
-    }
-    __syncthreads();   // K/V tiles are no longer read: reuse them for the O exchange
-    float *so = reinterpret_cast<float *>(sm.k);   // [4 warps][16 rows][128]
-    float scale_row[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int row = g0 + 8 * r;
-        float M = fmaxf(fmaxf(sm.m[0][row], sm.m[1][row]), fmaxf(sm.m[2][row], sm.m[3][row]));
-        scale_row[r] = (mrow[r] == -INFINITY) ? 0.f : exp2f(mrow[r] - M);
-    }
-#pragma unroll
-    for (int nt = 0; nt < DSA_V_DIM / 8; ++nt) {
-        const int col = nt * 8 + cq * 2;
-        float *d0 = so + (warp * 16 + g0) * DSA_V_DIM + col;
-        float *d1 = so + (warp * 16 + g0 + 8) * DSA_V_DIM + col;
-        *reinterpret_cast<float2 *>(d0) = make_float2(o[nt][0] * scale_row[0], o[nt][1] * scale_row[0]);
-        *reinterpret_cast<float2 *>(d1) = make_float2(o[nt][2] * scale_row[1], o[nt][3] * scale_row[1]);
-    }
-    __syncthreads();
-    // each thread: one head row (tid / 8) and 16 columns
-    {
-        const int row = tid >> 3, c0 = (tid & 7) * 16;
-        if (row < hpg) {
-            float M = fmaxf(fmaxf(sm.m[0][row], sm.m[1][row]), fmaxf(sm.m[2][row], sm.m[3][row]));
-            float L = 0.f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-                L += (sm.m[w][row] == -INFINITY) ? 0.f : sm.l[w][row] * exp2f(sm.m[w][row] - M);
-            float *dst = p.part_o + (((int64_t)bt * DSA_Q_HEADS + g * hpg + row) * p.splits + split) * DSA_V_DIM + c0;
-#pragma unroll
-            for (int c = 0; c < 16; c += 4) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    float4 v = *reinterpret_cast<const float4 *>(so + (w * 16 + row) * DSA_V_DIM + c0 + c);
-                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-                }
-                *reinterpret_cast<float4 *>(dst + c) = acc;
-            }
-            if ((tid & 7) == 0) {
-                ml[(int64_t)row * p.splits * 2 + 0] = M;
-                ml[(int64_t)row * p.splits * 2 + 1] = L;
-            }
-        }
-    }
+    attn_unit(p, sm, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x, 0);
 }
 
-// One warp per (query, head): merge the splits and the sink, normalise.
-// Lane j holds split j's (max, sum); the O partials are read with all loads of
-// a group independent of one another.  splits <= 32.
+// One warp per (query, head).
 __global__ void __launch_bounds__(128)
-combine_kernel(const float *part_o, const float *part_ml, int rows, int splits, const float *sink, int T,
+combine_kernel(const float *part_o, const float *part_ml, int rows, int splits, const float *sink,
                __nv_bfloat16 *O, float *lse) {
-    const int gw = blockIdx.x * 4 + warp_id(), lane = lane_id();
+    const int gw = blockIdx.x * 4 + warp_id();
     if (gw >= rows) return;
-    const int h = gw % DSA_Q_HEADS;
-    const float *ml = part_ml + (int64_t)gw * splits * 2;
-    const float mj = lane < splits ? ml[2 * lane] : -INFINITY;
-    const float lj = lane < splits ? ml[2 * lane + 1] : 0.f;
-    const float sk = sink ? __ldg(sink + h) * kLog2e : -INFINITY;
-    float M = fmaxf(mj, sk);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float wj = (mj == -INFINITY) ? 0.f : exp2f(mj - M);
-    float L = lj * wj;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (sink && M != -INFINITY) L += exp2f(sk - M);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float *po = part_o + (int64_t)gw * splits * DSA_V_DIM + lane * 4;
-    for (int j0 = 0; j0 < splits; j0 += 8) {
-        float4 v[8];
-        float w[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = j0 + u;
-            w[u] = __shfl_sync(0xffffffffu, wj, j & 31);
-            v[u] = (j < splits && w[u] != 0.f) ? *reinterpret_cast<const float4 *>(po + (int64_t)j * DSA_V_DIM)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (j0 + u < splits && w[u] != 0.f) {
-                acc.x += v[u].x * w[u]; acc.y += v[u].y * w[u]; acc.z += v[u].z * w[u]; acc.w += v[u].w * w[u];
-            }
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t *>(&lo);
-    packed.y = *reinterpret_cast<uint32_t *>(&hi);
-    *reinterpret_cast<uint2 *>(O + (int64_t)gw * DSA_V_DIM + lane * 4) = packed;
-    if (lse && lane == 0) lse[gw] = (L > 0.f) ? (M + log2f(L)) / kLog2e : -INFINITY;
+    combine_row(part_o, part_ml, gw, splits, sink, O, lse);
 }
 
 }  // namespace attn
@@ -351,29 +34,7 @@ size_t attn_partial_bytes(int B, int T, int max_keys) {
 
 int launch_attention(const AttnArgs &a, cudaStream_t stream) {
     using namespace attn;
-    const dsa_kv_t *kv = a.kv;
-    Params p;
-    p.Q = a.Q;
-    p.K = reinterpret_cast<const __nv_bfloat16 *>(kv->k);
-    p.V = reinterpret_cast<const __nv_bfloat16 *>(kv->v);
-    p.G = kv->num_kv_heads;
-    p.block_table = kv->block_table;
-    p.max_pages = kv->max_pages;
-    p.page_size = kv->page_size;
-    p.seq_stride = kv->seq_stride;
-    p.num_rows = kv->num_rows;
-    p.idx = a.idx;
-    p.count = a.count;
-    p.idx_stride = a.idx_stride;
-    p.q_pos = a.q_pos;
-    p.window = a.window;
-    p.T = a.T;
-    p.splits = (a.max_keys + kChunk - 1) / kChunk;
-    p.scale_log2 = a.sm_scale * kLog2e;
-    p.part_o = a.part_o;
-    p.part_ml = a.part_ml;
-    p.status = a.status;
-
+    Params p = make_params(a);
     const size_t smem = sizeof(Smem);
     cudaError_t e = cudaFuncSetAttribute(gather_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
@@ -386,8 +47,7 @@ int launch_attention(const AttnArgs &a, cudaStream_t stream) {
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
     const int rows = a.B * a.T * DSA_Q_HEADS;
-    combine_kernel<<<(rows + 3) / 4, 128, 0, stream>>>(a.part_o, a.part_ml, rows, p.splits, a.sink, a.T, a.O,
-                                                       a.lse);
+    combine_kernel<<<(rows + 3) / 4, 128, 0, stream>>>(a.part_o, a.part_ml, rows, p.splits, a.sink, a.O, a.lse);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     return DSA_OK;

@@ -1,0 +1,218 @@
+// fused.cu -- the whole DSA decode layer-step in one persistent, cooperative
+// kernel: lightning indexer -> top-k selection -> split-KV sparse attention ->
+// split combine, with grid-wide barriers between the phases and no launch in
+// between.  ("Naive-N0.5-Flash: no full-attention layers, and a runtime built
+// by AI", section "The runtime is the actual claim", describes a DSA layer run
+// as one cooperative kernel on 148 CTAs; this is this library's own design of
+// that idea for B200, built from the same device code as the standalone
+// kernels.)
+//
+// Grid: two CTAs per SM (as the indexer), 320 threads each, all co-resident
+// (cooperative launch).
+//   phase 1  indexer body (indexer_impl.cuh); scores to the workspace and, when
+//            it fits, each CTA's first-digit histogram of its scores added into
+//            the rows' global histograms, which saves the selection one pass
+//            and one barrier;
+//   phase 2  selection (topk_impl.cuh): each query row is shared by
+//            C = grid / rows CTAs;
+//   phase 3  attention units (attention_impl.cuh): two teams of four warps per
+//            CTA, one (query, KV head, 64-key split) unit per team at a time;
+//   phase 4  combine: one warp per (query, head).
+#include <algorithm>
+
+#include "attention_impl.cuh"
+#include "indexer_impl.cuh"
+#include "kernels.h"
+#include "topk_impl.cuh"
+
+namespace dsa {
+namespace fused {
+
+constexpr int kThreads = indexer::kThreads;   // 320
+constexpr int kWarps = kThreads / 32;
+constexpr int kTeams = 2;                     // attention teams of 4 warps
+constexpr int kMaxRows = 16;                  // B * T handled by the fused path
+constexpr int kMaxHistRows = 4;               // rows whose first histogram the indexer builds
+
+static_assert(kTeams * 4 <= kWarps, "attention teams must fit in the CTA");
+
+struct Params {
+    indexer::Params ix;
+    topk::Params tk;
+    attn::Params at;
+    const float *sink;
+    __nv_bfloat16 *O;
+    float *lse;
+    uint32_t *grid_bar;   // [0] arrivals, [1] exits
+    int rows;             // B * T
+    int C;                // CTAs per row in the selection phase
+    int hist_ready;
+};
+
+constexpr size_t smem_align(size_t x) { return (x + 127) & ~size_t(127); }
+
+// Barrier of all CTAs of the grid (bounded spin).
+__device__ bool grid_sync(uint32_t *bar, uint32_t target, uint32_t *status, uint32_t *flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t ok = 1;
+        __threadfence();
+        atomicAdd(bar, 1u);
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(bar) < target) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                flag_error(status, DSA_ERR_DEVICE_TIMEOUT);
+                ok = 0;
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+        *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, indexer::kCtasPerSm)
+dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
+                       const __grid_constant__ CUtensorMap tmap_q, const Params fp) {
+    // the dynamic buffer is aligned by hand (its 1 KB slack is part of the budget), so the
+    // static shared memory of this kernel stays a few bytes
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint32_t sync_flag;
+    const uint32_t G = gridDim.x;
+    uint32_t *status = fp.ix.status;
+
+    // ---- phase 1: indexer
+    indexer::run_indexer(&tmap_k, &tmap_ks, &tmap_q, fp.ix, smem, blockIdx.x, G);
+    if (!grid_sync(fp.grid_bar, 1 * G, status, &sync_flag)) return;
+
+    // ---- phase 2: selection
+    if ((int)blockIdx.x < fp.rows * fp.C) {
+        auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(smem);
+        uint32_t *cache = reinterpret_cast<uint32_t *>(smem + smem_align(sizeof(topk::Shared<kThreads>)));
+        topk::select_row<kThreads>(fp.tk, sh, cache, blockIdx.x / fp.C, blockIdx.x % fp.C, fp.C, fp.hist_ready != 0);
+    }
+    if (!grid_sync(fp.grid_bar, 2 * G, status, &sync_flag)) return;
+
+    // ---- phase 3: attention units
+    {
+        const int team = warp_id() / 4;
+        if (team < kTeams) {
+            attn::Smem &sm = *reinterpret_cast<attn::Smem *>(smem + team * smem_align(sizeof(attn::Smem)));
+            const int G_kv = fp.at.G, splits = fp.at.splits;
+            const int units = fp.rows * G_kv * splits;
+            for (int u = team * (int)G + (int)blockIdx.x; u < units; u += kTeams * (int)G) {
+                const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
+                attn::attn_unit(fp.at, sm, split, g, bt, threadIdx.x & 127, 1 + team);
+            }
+        }
+    }
+    if (!grid_sync(fp.grid_bar, 3 * G, status, &sync_flag)) return;
+
+    // ---- phase 4: combine, one warp per (query, head)
+    for (int gw = blockIdx.x * kWarps + warp_id(); gw < fp.rows * DSA_Q_HEADS; gw += G * kWarps)
+        attn::combine_row(fp.at.part_o, fp.at.part_ml, gw, fp.at.splits, fp.sink, fp.O, fp.lse);
+
+    // ---- the last CTA out resets the grid barrier for the next call
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(fp.grid_bar + 1, 1u) == G - 1) {
+            atomicExch(fp.grid_bar, 0u);
+            atomicExch(fp.grid_bar + 1, 0u);
+        }
+    }
+}
+
+}  // namespace fused
+
+int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
+    using namespace fused;
+    const DeviceInfo &dev = device_info();
+    plan->ok = false;
+    const int rows = B * T;
+    if (dev.num_sms <= 0 || rows > kMaxRows) return DSA_OK;
+    const int64_t max_tiles = (int64_t)B * ((Lmax + indexer::kTile - 1) / indexer::kTile);
+    // every CTA takes part in every phase: at least one CTA per row for the selection
+    const int grid = (int)std::max<int64_t>(
+        rows, std::min<int64_t>((int64_t)dev.num_sms * indexer::kCtasPerSm, max_tiles));
+    plan->grid = grid;
+    plan->rows = rows;
+    plan->C = std::max(1, grid / rows);
+    plan->scratch_bytes = (size_t)rows * topk::scratch_words(plan->C) * 4 + 256;   // + grid barrier words
+    plan->ok = true;
+    return DSA_OK;
+}
+
+int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
+                 int32_t *count, uint32_t *scratch, cudaStream_t stream) {
+    using namespace fused;
+    const DeviceInfo &dev = device_info();
+    // leave room for the kernel's few bytes of static shared memory next to the dynamic part
+    const size_t budget = std::min<size_t>(dev.smem_optin, kHalfSmSmem) - 256;
+    uint32_t *row_scratch = scratch + 64;   // the first 256 bytes hold the grid barrier words
+    const int row_words = topk::scratch_words(plan.C);
+
+    // indexer phase, with the first histogram when the rows' histograms fit
+    IndexerLaunch L;
+    int hist_rows = plan.rows <= kMaxHistRows ? plan.rows : 0;
+    int rc = prepare_indexer(ia, hist_rows, row_words, row_scratch + topk::kHist1, budget, &L);
+    if (rc == DSA_OK && hist_rows && L.p.stages < 4) hist_rows = 0;   // keep the stream at least 4 stages deep
+    if (rc != DSA_OK || hist_rows == 0) {
+        hist_rows = 0;
+        if ((rc = prepare_indexer(ia, 0, 0, nullptr, budget, &L))) return rc;
+    }
+    // the indexer body spreads its tiles over however many CTAs run it
+
+    Params fp;
+    fp.ix = L.p;
+    fp.at = attn::make_params(aa);
+    fp.sink = aa.sink;
+    fp.O = aa.O;
+    fp.lse = aa.lse;
+    fp.grid_bar = scratch;
+    fp.rows = plan.rows;
+    fp.C = plan.C;
+    fp.hist_ready = hist_rows > 0;
+
+    // selection phase: same parameters as the standalone selection
+    const size_t attn_smem = kTeams * smem_align(sizeof(attn::Smem));
+    const size_t top_fixed = smem_align(sizeof(topk::Shared<kThreads>));
+    const size_t smem = std::max({L.smem, attn_smem + 1024, top_fixed + 1024 + 4096});
+    if (smem > budget) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "fused kernel shared memory does not fit");
+    topk::Params &tp = fp.tk;
+    tp.scores = ia.scores;
+    tp.stride = ia.scores_stride;
+    tp.q_pos = ia.q_pos;
+    tp.rows = plan.rows;
+    tp.K = top_k;
+    tp.C = plan.C;
+    tp.idx = idx;
+    tp.count = count;
+    tp.scratch = row_scratch;
+    tp.scratch_row_words = row_words;
+    tp.status = ia.status;
+    tp.cache_keys = (int)((smem - 1024 - top_fixed) / 4);
+    tp.Lmax = ia.Lmax;
+
+    cudaError_t e = cudaFuncSetAttribute(dsa_layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fused)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // the phases wait on every CTA
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, dsa_layer_fused_kernel, L.tmap_k, L.tmap_ks, L.tmap_q, fp);
+    if (e != cudaSuccess) return cuda_fail(e, "fused layer-step launch");
+    return DSA_OK;
+}
+
+}  // namespace dsa

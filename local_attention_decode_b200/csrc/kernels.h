@@ -40,6 +40,14 @@ struct IndexerArgs {
 };
 int launch_indexer(const IndexerArgs &a, cudaStream_t stream);
 
+namespace indexer { struct Params; }
+// Everything a launch of the indexer body needs: tensor maps, parameters,
+// dynamic shared memory and grid (two CTAs per SM).  hist_rows > 0 adds each
+// CTA's first-digit histogram of the visible scores into hist_global.
+struct IndexerLaunch;
+int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uint32_t *hist_global,
+                    size_t smem_budget, IndexerLaunch *out);
+
 // ----------------------------------------------------------------- top-k
 struct TopkPlan {
     int rows = 0;          // B * T
@@ -78,5 +86,21 @@ struct AttnArgs {
 };
 size_t attn_partial_bytes(int B, int T, int max_keys);
 int launch_attention(const AttnArgs &a, cudaStream_t stream);
+
+// --------------------------------------------------------- fused layer-step
+struct FusedPlan {
+    bool ok = false;            // false: use the separate kernels
+    int grid = 0;               // CTAs (two per SM)
+    int rows = 0;               // B * T
+    int C = 1;                  // CTAs per row in the selection phase
+    size_t scratch_bytes = 0;   // grid barrier words + per-row selection scratch
+};
+int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan);
+int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
+                 int32_t *count, uint32_t *scratch, cudaStream_t stream);
+
+// Largest dynamic shared memory (bytes, including 1 KB of alignment slack) a
+// CTA may use when two CTAs share an SM.
+constexpr size_t kHalfSmSmem = 228 * 1024 / 2 - 1024;
 
 }  // namespace dsa

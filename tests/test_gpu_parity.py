@@ -254,6 +254,24 @@ def test_layer_decode_is_deterministic():
                            y.view(torch.uint8) if y.dtype == torch.bfloat16 else y)
 
 
+@pytest.mark.parametrize("seq_lens,T,page_size", [([65536], 4, 0), ([3000, 9000], 2, 64), ([20000] * 5, 4, 0)])
+def test_layer_decode_equals_separate_calls(seq_lens, T, page_size):
+    """dsa_layer_decode (one fused launch for B*T <= 16 rows, separate kernels
+    above) gives exactly what the three separate entry points give."""
+    wl = make_decode_workload(seed=80, seq_lens=seq_lens, T=T, device=DEV, page_size=page_size, n_needles=8)
+    O, lse, idx, cnt = run_layer(wl)
+    Lmax = int(wl.q_pos.max()) + 1
+    scores = run_indexer(wl, Lmax)
+    idx2, cnt2 = run_topk(scores, wl.q_pos, 2048)
+    assert torch.equal(cnt, cnt2) and torch.equal(idx, idx2)
+    O2 = torch.empty_like(O)
+    lse2 = torch.empty_like(lse)
+    ws = dsa.alloc_workspace(dsa.OP_SPARSE_ATTN, wl.B, wl.T, 1, 2048)
+    dsa.sparse_gqa_attn_decode(wl.Q, kv_for(wl, with_index=False), idx2, cnt2, 2048, wl.sink, SM, O2, lse2, ws)
+    assert torch.equal(O.view(torch.int16), O2.view(torch.int16))
+    assert torch.equal(lse, lse2)
+
+
 def test_layer_decode_1m_context_sampled():
     """Native 1,048,576-token context: scores at sampled positions and every
     needle against the oracle; the selection bit-exact against the oracle's
