@@ -12,16 +12,16 @@ __global__ void __launch_bounds__(kThreads)
 gather_attn_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    attn_unit(p, sm, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x, 0);
+    attn_unit<0>(p, sm, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
 }
 
-// One warp per (query, head).
-__global__ void __launch_bounds__(128)
-combine_kernel(const float *part_o, const float *part_ml, int rows, int splits, const float *sink,
-               __nv_bfloat16 *O, float *lse) {
-    const int gw = blockIdx.x * 4 + warp_id();
-    if (gw >= rows) return;
-    combine_row(part_o, part_ml, gw, splits, sink, O, lse);
+// One CTA per (query, head), as in the fused layer-step (same arithmetic).
+constexpr int kCombineThreads = 256;
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(const float *part_o, const float *part_ml, int splits, const float *sink, __nv_bfloat16 *O,
+               float *lse) {
+    __shared__ float red[32 * DSA_V_DIM + 64];
+    combine_row_cta<kCombineThreads>(part_o, part_ml, blockIdx.x, splits, sink, O, lse, red);
 }
 
 }  // namespace attn
@@ -47,7 +47,7 @@ int launch_attention(const AttnArgs &a, cudaStream_t stream) {
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
     const int rows = a.B * a.T * DSA_Q_HEADS;
-    combine_kernel<<<(rows + 3) / 4, 128, 0, stream>>>(a.part_o, a.part_ml, rows, p.splits, a.sink, a.O, a.lse);
+    combine_kernel<<<rows, kCombineThreads, 0, stream>>>(a.part_o, a.part_ml, p.splits, a.sink, a.O, a.lse);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     return DSA_OK;

@@ -65,8 +65,11 @@ struct Smem {
     float l[4][16];
 };
 
-__device__ __forceinline__ void team_sync(int bar_id) {
-    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+// Barrier of one 128-thread team; the barrier id is a compile-time constant so
+// that the kernel reserves only the barriers it uses.
+template <int BAR>
+__device__ __forceinline__ void team_sync() {
+    asm volatile("bar.sync %0, 128;" ::"n"(BAR) : "memory");
 }
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
@@ -114,9 +117,10 @@ __device__ __forceinline__ bool key_row(const Params &p, int b, int64_t pos, int
 
 // One split-KV unit: keys [split * 64, split * 64 + 64) of query bt and KV
 // head g, by a team of 128 threads (tid 0..127) synchronised with the named
-// barrier `bar_id`; writes the unit's partial (O, max, sum) for the 64/G
+// barrier BAR; writes the unit's partial (O, max, sum) for the 64/G
 // query heads of the group.
-__device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid, int bar_id) {
+template <int BAR>
+__device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid) {
     const int b = bt / p.T;
     const int hpg = DSA_Q_HEADS / p.G;
     const int warp = tid >> 5, lane = tid & 31;
@@ -162,7 +166,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         if (r < hpg) cp_async16(dst, qg + (int64_t)r * DSA_QK_DIM + col);
         else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
-    team_sync(bar_id);
+    team_sync<BAR>();
     // ---- gather K and V rows
     const int G = p.G;
     for (int c = tid; c < kChunk * (DSA_QK_DIM / 8); c += kThreads) {
@@ -180,7 +184,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
     cp_async_wait_all();
-    team_sync(bar_id);
+    team_sync<BAR>();
 
     // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8)
     const int key0 = warp * 16;
@@ -251,7 +255,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         sm.l[warp][g0] = lrow[0];
         sm.l[warp][g0 + 8] = lrow[1];
     }
-    team_sync(bar_id);   // K/V tiles are no longer read: reuse them for the O exchange
+    team_sync<BAR>();   // K/V tiles are no longer read: reuse them for the O exchange
     float *so = reinterpret_cast<float *>(sm.k);   // [4 warps][16 rows][128]
     float scale_row[2];
 #pragma unroll
@@ -268,7 +272,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         *reinterpret_cast<float2 *>(d0) = make_float2(o[nt][0] * scale_row[0], o[nt][1] * scale_row[0]);
         *reinterpret_cast<float2 *>(d1) = make_float2(o[nt][2] * scale_row[1], o[nt][3] * scale_row[1]);
     }
-    team_sync(bar_id);
+    team_sync<BAR>();
     // each thread: one head row (tid / 8) and 16 columns
     {
         const int row = tid >> 3, c0 = (tid & 7) * 16;
@@ -343,6 +347,59 @@ __device__ __forceinline__ void combine_row(const float *part_o, const float *pa
     packed.y = *reinterpret_cast<uint32_t *>(&hi);
     *reinterpret_cast<uint2 *>(O + (int64_t)gw * DSA_V_DIM + lane * 4) = packed;
     if (lse && lane == 0) lse[gw] = (L > 0.f) ? (M + log2f(L)) / kLog2e : -INFINITY;
+}
+
+// Merge of the splits of one (query, head) row gw by a whole CTA of NT
+// threads (NT >= 8 * splits, splits <= 32): thread (split s, slice k) loads
+// its split's 16-value slice and statistics, all loads issued at once; the
+// weighted slices are summed over the splits through shared memory `red`
+// (32 * 128 + 64 floats).
+template <int NT>
+__device__ void combine_row_cta(const float *part_o, const float *part_ml, int gw, int splits, const float *sink,
+                                __nv_bfloat16 *O, float *lse, float *red) {
+    static_assert(NT >= 256, "eight threads per split");
+    const int t = threadIdx.x, s = t >> 3, k = t & 7;
+    float *msm = red + 32 * DSA_V_DIM, *lsm = msm + 32;
+    const float *ml = part_ml + (int64_t)gw * splits * 2;
+    const float *po = part_o + ((int64_t)gw * splits + s) * DSA_V_DIM + k * 16;
+    float m = -INFINITY, l = 0.f;
+    float4 v[4];
+    if (s < splits) {
+        m = __ldcg(ml + 2 * s);
+        l = __ldcg(ml + 2 * s + 1);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4 *>(po) + u);
+    }
+    if (k == 0 && s < 32) msm[s] = m;
+    __syncthreads();
+    const int h = gw % DSA_Q_HEADS;
+    const float sk = sink ? __ldg(sink + h) * kLog2e : -INFINITY;
+    float M = sk;
+    for (int j = 0; j < splits; ++j) M = fmaxf(M, msm[j]);
+    const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
+    if (s < 32) {
+        float *dst = red + s * DSA_V_DIM + k * 16;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float4 x = (s < splits && w != 0.f) ? v[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+            dst[4 * u + 0] = x.x * w;
+            dst[4 * u + 1] = x.y * w;
+            dst[4 * u + 2] = x.z * w;
+            dst[4 * u + 3] = x.w * w;
+        }
+        if (k == 0) lsm[s] = (s < splits && w != 0.f) ? l * w : 0.f;
+    }
+    __syncthreads();
+    if (t < DSA_V_DIM) {
+        float acc = 0.f, L = (sink && M != -INFINITY) ? exp2f(sk - M) : 0.f;
+        for (int j = 0; j < splits; ++j) {
+            acc += red[j * DSA_V_DIM + t];
+            L += lsm[j];
+        }
+        O[(int64_t)gw * DSA_V_DIM + t] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+        if (lse && t == 0) lse[gw] = (L > 0.f) ? (M + log2f(L)) / kLog2e : -INFINITY;
+    }
+    __syncthreads();
 }
 
 // Kernel parameters of the attention described by `a`.

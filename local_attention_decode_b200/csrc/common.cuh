@@ -103,6 +103,33 @@ __device__ __forceinline__ void tma_load_1d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// L2 policy for data read exactly once (the streamed key cache): its lines are
+// the first to go, so the stream does not push the kernel's code, scores and
+// scratch out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int32_t x,
+                                                 int32_t y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_1d_hint(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int32_t x,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3}], [%2], %4;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -186,6 +213,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 
 // ------------------------------------------------------------------ misc
+// Warp-level histogram increment: lanes with `active` add 1 to hist[bin].
+// When every active lane has the same bin (the common case for a narrow score
+// distribution) one atomic adds them all; otherwise each lane adds its own.
+// All 32 lanes must call it.
+__device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool active) {
+    const uint32_t amask = __ballot_sync(0xffffffffu, active);
+    if (amask == 0) return;
+    const uint32_t bmin = __reduce_min_sync(0xffffffffu, active ? bin : 0xFFFFFFFFu);
+    const uint32_t bmax = __reduce_max_sync(0xffffffffu, active ? bin : 0u);
+    if (bmin == bmax) {
+        if ((threadIdx.x & 31) == (uint32_t)(__ffs(amask) - 1)) atomicAdd(&hist[bmin], (uint32_t)__popc(amask));
+    } else if (active) {
+        atomicAdd(&hist[bin], 1u);
+    }
+}
+
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 

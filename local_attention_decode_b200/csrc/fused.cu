@@ -7,7 +7,7 @@
 // that idea for B200, built from the same device code as the standalone
 // kernels.)
 //
-// Grid: two CTAs per SM (as the indexer), 320 threads each, all co-resident
+// Grid: one CTA per SM (as the indexer), 640 threads each, all co-resident
 // (cooperative launch).
 //   phase 1  indexer body (indexer_impl.cuh); scores to the workspace and, when
 //            it fits, each CTA's first-digit histogram of its scores added into
@@ -15,9 +15,9 @@
 //            and one barrier;
 //   phase 2  selection (topk_impl.cuh): each query row is shared by
 //            C = grid / rows CTAs;
-//   phase 3  attention units (attention_impl.cuh): two teams of four warps per
-//            CTA, one (query, KV head, 64-key split) unit per team at a time;
-//   phase 4  combine: one warp per (query, head).
+//   phase 3  attention units (attention_impl.cuh): four teams of four warps
+//            per CTA, one (query, KV head, 64-key split) unit per team at a time;
+//   phase 4  combine: one CTA per (query, head).
 #include <algorithm>
 
 #include "attention_impl.cuh"
@@ -28,13 +28,13 @@
 namespace dsa {
 namespace fused {
 
-constexpr int kThreads = indexer::kThreads;   // 320
+constexpr int kThreads = indexer::kThreads;   // 640
 constexpr int kWarps = kThreads / 32;
-constexpr int kTeams = 2;                     // attention teams of 4 warps
+constexpr int kTeams = 4;                     // attention teams of 4 warps (named barriers 1..4)
 constexpr int kMaxRows = 16;                  // B * T handled by the fused path
-constexpr int kMaxHistRows = 4;               // rows whose first histogram the indexer builds
+constexpr int kMaxHistRows = 8;               // rows whose first histogram the indexer builds
 
-static_assert(kTeams * 4 <= kWarps, "attention teams must fit in the CTA");
+static_assert(kTeams * 4 <= kWarps, "the attention teams must fit in the CTA");
 
 struct Params {
     indexer::Params ix;
@@ -49,7 +49,7 @@ struct Params {
     int hist_ready;
 };
 
-constexpr size_t smem_align(size_t x) { return (x + 127) & ~size_t(127); }
+__host__ __device__ constexpr size_t smem_align(size_t x) { return (x + 127) & ~size_t(127); }
 
 // Barrier of all CTAs of the grid (bounded spin).
 __device__ bool grid_sync(uint32_t *bar, uint32_t target, uint32_t *status, uint32_t *flag) {
@@ -74,7 +74,7 @@ __device__ bool grid_sync(uint32_t *bar, uint32_t target, uint32_t *status, uint
     return *flag != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, indexer::kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
 dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
                        const __grid_constant__ CUtensorMap tmap_q, const Params fp) {
     // the dynamic buffer is aligned by hand (its 1 KB slack is part of the budget), so the
@@ -89,11 +89,13 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     indexer::run_indexer(&tmap_k, &tmap_ks, &tmap_q, fp.ix, smem, blockIdx.x, G);
     if (!grid_sync(fp.grid_bar, 1 * G, status, &sync_flag)) return;
 
-    // ---- phase 2: selection
+    // ---- phase 2: selection (candidate runs when the indexer built the first histogram;
+    //      the round-by-round path otherwise, or when the candidates would not fit)
     if ((int)blockIdx.x < fp.rows * fp.C) {
         auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(smem);
         uint32_t *cache = reinterpret_cast<uint32_t *>(smem + smem_align(sizeof(topk::Shared<kThreads>)));
-        topk::select_row<kThreads>(fp.tk, sh, cache, blockIdx.x / fp.C, blockIdx.x % fp.C, fp.C, fp.hist_ready != 0);
+        const int row = blockIdx.x / fp.C, c = blockIdx.x % fp.C;
+        topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, fp.hist_ready != 0);
     }
     if (!grid_sync(fp.grid_bar, 2 * G, status, &sync_flag)) return;
 
@@ -106,15 +108,21 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
             const int units = fp.rows * G_kv * splits;
             for (int u = team * (int)G + (int)blockIdx.x; u < units; u += kTeams * (int)G) {
                 const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
-                attn::attn_unit(fp.at, sm, split, g, bt, threadIdx.x & 127, 1 + team);
+                switch (team) {
+                    case 0: attn::attn_unit<1>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
+                    case 1: attn::attn_unit<2>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
+                    case 2: attn::attn_unit<3>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
+                    default: attn::attn_unit<4>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
+                }
             }
         }
     }
     if (!grid_sync(fp.grid_bar, 3 * G, status, &sync_flag)) return;
 
-    // ---- phase 4: combine, one warp per (query, head)
-    for (int gw = blockIdx.x * kWarps + warp_id(); gw < fp.rows * DSA_Q_HEADS; gw += G * kWarps)
-        attn::combine_row(fp.at.part_o, fp.at.part_ml, gw, fp.at.splits, fp.sink, fp.O, fp.lse);
+    // ---- phase 4: combine, one CTA per (query, head)
+    for (int gw = blockIdx.x; gw < fp.rows * DSA_Q_HEADS; gw += G)
+        attn::combine_row_cta<kThreads>(fp.at.part_o, fp.at.part_ml, gw, fp.at.splits, fp.sink, fp.O, fp.lse,
+                                        reinterpret_cast<float *>(smem));
 
     // ---- the last CTA out resets the grid barrier for the next call
     __syncthreads();
@@ -129,6 +137,13 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
 
 }  // namespace fused
 
+// Largest dynamic shared memory of the fused kernel: half an SM, minus room
+// for its few bytes of static shared memory.
+static size_t fused_smem_budget() {
+    // one CTA per SM; leave room for the kernel's few bytes of static shared memory
+    return device_info().smem_optin - 256;
+}
+
 int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
     using namespace fused;
     const DeviceInfo &dev = device_info();
@@ -136,13 +151,23 @@ int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
     const int rows = B * T;
     if (dev.num_sms <= 0 || rows > kMaxRows) return DSA_OK;
     const int64_t max_tiles = (int64_t)B * ((Lmax + indexer::kTile - 1) / indexer::kTile);
+    // all CTAs must be resident at once (the phases wait on each other): as many as fit
+    int per_sm = 0;
+    cudaError_t e = cudaFuncSetAttribute(dsa_layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)fused_smem_budget());
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dsa_layer_fused_kernel, kThreads,
+                                                          fused_smem_budget());
+    if (e != cudaSuccess) return cuda_fail(e, "occupancy of the fused kernel");
+    per_sm = std::min(per_sm, 1);
+    if (per_sm < 1 || rows > per_sm * dev.num_sms) return DSA_OK;
     // every CTA takes part in every phase: at least one CTA per row for the selection
     const int grid = (int)std::max<int64_t>(
-        rows, std::min<int64_t>((int64_t)dev.num_sms * indexer::kCtasPerSm, max_tiles));
+        rows, std::min<int64_t>((int64_t)dev.num_sms * per_sm, max_tiles));
     plan->grid = grid;
     plan->rows = rows;
     plan->C = std::max(1, grid / rows);
-    plan->scratch_bytes = (size_t)rows * topk::scratch_words(plan->C) * 4 + 256;   // + grid barrier words
+    plan->scratch_bytes = (size_t)rows * topk::scratch_words(plan->C, topk::kListCap) * 4 + 256;   // + grid barrier words
     plan->ok = true;
     return DSA_OK;
 }
@@ -150,17 +175,15 @@ int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
 int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
                  int32_t *count, uint32_t *scratch, cudaStream_t stream) {
     using namespace fused;
-    const DeviceInfo &dev = device_info();
-    // leave room for the kernel's few bytes of static shared memory next to the dynamic part
-    const size_t budget = std::min<size_t>(dev.smem_optin, kHalfSmSmem) - 256;
+    const size_t budget = fused_smem_budget();
     uint32_t *row_scratch = scratch + 64;   // the first 256 bytes hold the grid barrier words
-    const int row_words = topk::scratch_words(plan.C);
+    const int row_words = topk::scratch_words(plan.C, topk::kListCap);
 
     // indexer phase, with the first histogram when the rows' histograms fit
     IndexerLaunch L;
     int hist_rows = plan.rows <= kMaxHistRows ? plan.rows : 0;
     int rc = prepare_indexer(ia, hist_rows, row_words, row_scratch + topk::kHist1, budget, &L);
-    if (rc == DSA_OK && hist_rows && L.p.stages < 4) hist_rows = 0;   // keep the stream at least 4 stages deep
+    if (rc == DSA_OK && hist_rows && L.p.stages < 3) hist_rows = 0;   // keep the stream at least 3 stages deep
     if (rc != DSA_OK || hist_rows == 0) {
         hist_rows = 0;
         if ((rc = prepare_indexer(ia, 0, 0, nullptr, budget, &L))) return rc;
@@ -195,7 +218,16 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     tp.scratch = row_scratch;
     tp.scratch_row_words = row_words;
     tp.status = ia.status;
-    tp.cache_keys = (int)((smem - 1024 - top_fixed) / 4);
+    {   // shared memory after the fixed part: the CTA's slice of keys, then the candidate list
+        const int64_t avail = (int64_t)(smem - 1024 - top_fixed) / 4;
+        const int64_t chunk = ((ia.Lmax + plan.C - 1) / plan.C + 3) & ~int64_t(3);
+        int64_t list = topk::kListCap;
+        if (chunk + 2 * list > avail) list = std::max<int64_t>(0, (avail - chunk) / 2);
+        if (list < 1024) list = std::min<int64_t>(topk::kListCap, avail / 4);   // slices too long to cache
+        tp.smem_list = (int)list;
+        tp.cache_keys = (int)(avail - 2 * list);
+    }
+    tp.list_cap = topk::kListCap;
     tp.Lmax = ia.Lmax;
 
     cudaError_t e = cudaFuncSetAttribute(dsa_layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

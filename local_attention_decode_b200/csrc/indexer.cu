@@ -11,7 +11,7 @@
 namespace dsa {
 namespace indexer {
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
                const __grid_constant__ CUtensorMap tmap_q, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -84,12 +84,13 @@ int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uin
         if (rc) return rc;
     }
 
-    // stages: as many as fit next to the tables (2..8) in smem_budget bytes
-    // (1 KB of which is alignment slack)
-    const size_t budget = std::min<size_t>(smem_budget, kHalfSmSmem) - 1024;
-    int S = 8;
-    while (S > 2 && Layout(S, T, a.B, hist_rows).total > budget) --S;
-    Layout lay(S, T, a.B, hist_rows);
+    // stages per pipeline: as many as fit next to the tables (2..8) in
+    // smem_budget bytes (1 KB of which is alignment slack)
+    const size_t budget = std::min<size_t>(smem_budget, dev.smem_optin) - 1024;
+    const bool q_resident = a.B == 1;
+    int S = kMaxStages;
+    while (S > 2 && Layout(S, T, a.B, hist_rows, q_resident).total > budget) --S;
+    Layout lay(S, T, a.B, hist_rows, q_resident);
     if (lay.total > budget)
         return fail(DSA_ERR_UNSUPPORTED_SHAPE, "indexer shared memory does not fit (T=%d, B=%d)", T, a.B);
     out->smem = lay.total + 1024;
@@ -111,13 +112,14 @@ int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uin
     p.status = a.status;
     p.stages = S;
     p.rows_per_load = R;
-    p.groups = std::max(1, std::min(kMaxGroups, kMaxTmemCols / N));
+    p.groups = std::max(1, std::min(kMaxGroups, 512 / (kPipes * N)));
     p.hist_rows = hist_rows;
     p.hist_row_words = hist_row_words;
     p.hist_global = hist_global;
+    p.q_resident = q_resident ? 1 : 0;
 
     const int64_t max_tiles = (int64_t)a.B * ((a.Lmax + kTile - 1) / kTile);
-    out->grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)dev.num_sms * kCtasPerSm, max_tiles));
+    out->grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)dev.num_sms, max_tiles));
     return DSA_OK;
 }
 

@@ -42,7 +42,7 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream);
 
 namespace indexer { struct Params; }
 // Everything a launch of the indexer body needs: tensor maps, parameters,
-// dynamic shared memory and grid (two CTAs per SM).  hist_rows > 0 adds each
+// dynamic shared memory and grid (one CTA per SM, two pipelines per CTA).  hist_rows > 0 adds each
 // CTA's first-digit histogram of the visible scores into hist_global.
 struct IndexerLaunch;
 int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uint32_t *hist_global,
@@ -54,11 +54,15 @@ struct TopkPlan {
     int ctas_per_row = 1;  // C
     int threads = 512;
     int cache_keys = 0;    // keys cached in shared memory per CTA
+    int list_cap = 0;      // candidate-list entries per row in the scratch
+    int smem_list = 0;     // candidate-list entries that fit in shared memory
     int64_t Lmax = 0;      // positions held by each scores row
     size_t smem = 0;
     size_t scratch_bytes = 0;  // cross-CTA scratch (only when C > 1)
 };
-int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan);
+// max_scratch_bytes bounds scratch_bytes by shortening the candidate list
+// (down to none: the selection then exchanges every digit).
+int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_scratch_bytes = SIZE_MAX);
 int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const int32_t *q_pos,
                 int top_k, int32_t *idx, int32_t *count, uint32_t *scratch, uint32_t *status,
                 cudaStream_t stream);
@@ -99,8 +103,5 @@ int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan);
 int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
                  int32_t *count, uint32_t *scratch, cudaStream_t stream);
 
-// Largest dynamic shared memory (bytes, including 1 KB of alignment slack) a
-// CTA may use when two CTAs share an SM.
-constexpr size_t kHalfSmSmem = 228 * 1024 / 2 - 1024;
 
 }  // namespace dsa

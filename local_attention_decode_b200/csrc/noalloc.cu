@@ -56,7 +56,7 @@ extern "C" int dsa_topk_select_noalloc(const float *scores, int64_t scores_strid
     if (top_k < 1 || top_k > DSA_MAX_TOPK)
         return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
     TopkPlan plan;
-    int rc = plan_topk(B, T, Lmax, top_k, &plan);
+    int rc = plan_topk(B, T, Lmax, top_k, &plan, kStaticScratchBytes - kStatusBytes);
     if (rc) return rc;
     const size_t need = kStatusBytes + plan.scratch_bytes;
     if (need > kStaticScratchBytes)

@@ -10,7 +10,7 @@ namespace topk {
 
 constexpr int kThreads = 512;
 constexpr int kMinChunk = 4096;             // keys per CTA below which a row is not split further
-constexpr int kMaxCacheKeys = 40 * 1024;    // 160 KB of cached keys per CTA
+constexpr int kMaxCacheKeys = 32 * 1024;    // 128 KB of cached keys per CTA
 
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const Params p) {
@@ -22,7 +22,7 @@ topk_kernel(const Params p) {
 
 }  // namespace topk
 
-int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan) {
+int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_scratch_bytes) {
     using namespace topk;
     const DeviceInfo &dev = device_info();
     plan->rows = B * T;
@@ -37,8 +37,21 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan) {
     int64_t chunk = ((Lmax + C - 1) / C + 3) & ~int64_t(3);
     plan->ctas_per_row = C;
     plan->cache_keys = (int)std::min<int64_t>(chunk, kMaxCacheKeys);
-    plan->smem = sizeof(Shared<kThreads>) + (size_t)plan->cache_keys * 4;
-    plan->scratch_bytes = C > 1 ? (size_t)plan->rows * scratch_words(C) * 4 : 0;
+    plan->list_cap = 0;
+    plan->smem_list = 0;
+    plan->scratch_bytes = 0;
+    if (C > 1) {
+        int cap = kListCap;
+        const size_t fixed = (size_t)plan->rows * scratch_words(C, 0) * 4;
+        if (fixed > max_scratch_bytes) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top-k scratch exceeds %zu bytes", max_scratch_bytes);
+        cap = (int)std::min<size_t>(cap, (max_scratch_bytes - fixed) / ((size_t)plan->rows * 8));
+        plan->list_cap = cap & ~3;
+        const size_t used = sizeof(Shared<kThreads>) + (size_t)plan->cache_keys * 4;
+        const size_t room = dev.smem_optin > used ? (dev.smem_optin - used) / 8 : 0;
+        plan->smem_list = (int)std::min<size_t>(plan->list_cap, room);
+        plan->scratch_bytes = (size_t)plan->rows * scratch_words(C, plan->list_cap) * 4;
+    }
+    plan->smem = sizeof(Shared<kThreads>) + ((size_t)plan->cache_keys + 2 * (size_t)plan->smem_list) * 4;
     return DSA_OK;
 }
 
@@ -55,9 +68,11 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
     p.idx = idx;
     p.count = count;
     p.scratch = scratch;
-    p.scratch_row_words = scratch_words(plan.ctas_per_row);
+    p.scratch_row_words = scratch_words(plan.ctas_per_row, plan.list_cap);
     p.status = status;
     p.cache_keys = plan.cache_keys;
+    p.list_cap = plan.list_cap;
+    p.smem_list = plan.smem_list;
     p.Lmax = plan.Lmax;
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(topk)");

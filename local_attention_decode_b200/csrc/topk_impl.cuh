@@ -8,16 +8,31 @@
 // full-attention layers' means" -- argsort(...)[..., :index_top_k] -- and "How
 // much of this did AI actually build?" -- the stable-tie argsort).
 //
-// Exact radix select on the order-preserving 32-bit image of each score:
-// three digit rounds (11 + 11 + 10 bits) narrow the threshold key T* and the
-// number of ties at T* that still fit; one ordered compaction pass then emits,
-// in increasing position order, every position with key > T* and the first
-// ties positions with key == T*.  C CTAs share a row: each owns a contiguous
-// slice, keeps it in shared memory when it fits, adds its non-zero histogram
-// bins into the row's global histogram, and waits on a per-row counter barrier
-// (bounded spin) between rounds.  Per-CTA (greater, equal) counts give each CTA
-// its output offset, so the output order is a pure function of the scores.
-// The row's scratch words are zeroed again before the CTAs leave.
+// Exact radix select on the order-preserving 32-bit image of each score, in
+// three digits (11 + 11 + 10 bits), giving the threshold key T* and the number
+// `ties` of keys equal to T* that are taken; the output is, in increasing
+// position order, every position with key > T* and the first `ties` positions
+// with key == T*.  C CTAs share a row, each owning a contiguous slice that it
+// keeps in shared memory when it fits.
+//
+//   digit 1     the row's 2048-bin histogram of the top 11 bits -- built by the
+//               producer of the scores, or by the CTAs adding their slices'
+//               histograms into the row's global histogram and meeting at a
+//               barrier -- gives the threshold bin b1;
+//   list        every CTA appends its keys of bin b1, with their positions, to
+//               the row's candidate list and publishes how many of its keys lie
+//               above bin b1; one barrier;
+//   digits 2, 3 each CTA loads the whole list and finishes the select on it
+//               alone; its output offset is the earlier CTAs' counts above b1
+//               plus the list entries that lie before its slice.  When the list
+//               does not fit in shared memory (many keys share the threshold
+//               bin, e.g. heavy ties), digits 2 and 3 are exchanged like digit
+//               1, and so are the per-CTA (greater, equal) counts after them;
+//   emission    each warp compacts its part of the slice with ballots, from its
+//               own offset in the row's output.
+//
+// The output is a pure function of the scores.  The last CTA of a row to leave
+// clears the row's scratch words for the next call.
 #pragma once
 
 #include "common.cuh"
@@ -27,11 +42,19 @@ namespace topk {
 
 constexpr int kBins = 2048;                 // largest digit: 11 bits
 constexpr int kUnroll = 8;                  // independent loads in flight per thread
+constexpr int kListCap = 12288;             // candidate-list entries per row (global scratch)
 
-// Per-row scratch (u32 words), used when C > 1 (or when the first histogram
-// is produced by the indexer).
+// Per-row scratch (u32 words), used when C > 1 or when the first histogram is
+// produced by the indexer:
+//   [kHist1, +2048) [kHist2, +2048) [kHist3, +1024)  digit histograms
+//   [kCnt, +2C)      per-CTA (greater, equal) counts at T* (exchange path)
+//   [kCnt+2C, +C)    per-CTA counts of keys above bin b1
+//   ctl_base(C):     [0] barrier arrivals, [1] CTAs done, [2] list length
+//   list_base(C):    list_cap keys, then list_cap positions
 constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kCnt = 5120;
-__host__ __device__ constexpr int scratch_words(int C) { return kCnt + 2 * C + 2; }   // + barrier, exit
+__host__ __device__ constexpr int ctl_base(int C) { return kCnt + 3 * C; }
+__host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + 3 + 3) & ~3; }
+__host__ __device__ constexpr int scratch_words(int C, int list_cap) { return list_base(C) + 2 * list_cap; }
 
 struct Params {
     const float *scores;
@@ -43,7 +66,9 @@ struct Params {
     uint32_t *scratch;
     int scratch_row_words;
     uint32_t *status;
-    int cache_keys;
+    int cache_keys;        // keys of the slice kept in shared memory
+    int list_cap;          // list entries in the row's global scratch
+    int smem_list;         // list entries that fit in shared memory after the cache (<= list_cap)
     int64_t Lmax;
 };
 
@@ -51,16 +76,19 @@ template <int NT>
 struct alignas(16) Shared {
     uint32_t hist[kBins];
     uint32_t warp_tmp[NT / 32];
-    uint32_t warp_tmp2[NT / 32];
+    uint32_t warp_a[NT / 32];
+    uint32_t warp_b[NT / 32];
     int bin;
     uint32_t above;
+    uint32_t total;
     uint32_t ok;
+    uint32_t base;
 };
 
 // Inclusive block scan of one value per thread (all NT threads); returns the
 // inclusive prefix and writes the block total to *total.
 template <int NT>
-__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, uint32_t *total) {
+__device__ __noinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, uint32_t *total) {
     constexpr int NW = NT / 32;
     const int lane = lane_id(), warp = warp_id();
 #pragma unroll
@@ -87,9 +115,10 @@ __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, u
 }
 
 // Threshold bin of sh->hist[0..nbins): the bin b with above(b) < K <= above(b) + h[b],
-// above(b) = number of keys in bins > b.  Result in sh->bin / sh->above.
+// above(b) = number of keys in bins > b.  Result in sh->bin / sh->above, the
+// histogram's total in sh->total.
 template <int NT>
-__device__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
+__device__ __noinline__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
     const int per = (nbins + NT - 1) / NT;
     const int lo = threadIdx.x * per;
     uint32_t mine = 0;
@@ -97,6 +126,7 @@ __device__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
         if (lo + j < nbins) mine += sh->hist[lo + j];
     uint32_t total;
     uint32_t incl = block_scan<NT>(mine, sh->warp_tmp, &total);
+    if (threadIdx.x == 0) sh->total = total;
     uint32_t above = total - incl;      // keys in bins after this thread's range
     for (int j = per - 1; j >= 0; --j) {
         if (lo + j >= nbins) continue;
@@ -108,6 +138,33 @@ __device__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
         above += h;
     }
     __syncthreads();
+}
+
+// Loads nb (<= kBins) histogram words from global memory into sh->hist, all
+// loads of a thread in flight together.
+template <int NT>
+__device__ __forceinline__ void load_hist(Shared<NT> *sh, const uint32_t *g, int nb) {
+    constexpr int kPer = (kBins + NT - 1) / NT;
+    uint32_t v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int j = u * NT + threadIdx.x;
+        v[u] = j < nb ? __ldcg(g + j) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int j = u * NT + threadIdx.x;
+        if (j < nb) sh->hist[j] = v[u];
+    }
+    __syncthreads();
+}
+
+// Sum of a[0 .. upto) (upto <= 32), returned in every lane of the warp.
+__device__ __forceinline__ uint32_t warp_sum_prefix(const uint32_t *a, int upto) {
+    uint32_t v = lane_id() < upto ? a[lane_id()] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
 // Barrier among the C CTAs of a row: arrive, then wait (bounded) until
@@ -135,11 +192,95 @@ __device__ bool row_barrier(Shared<NT> *sh, uint32_t *bar, uint32_t target, uint
     return sh->ok != 0;
 }
 
+// The slice [0, len) split into one part per warp, each a whole number of
+// 32-key groups: [wlo, whi).
+template <int NT>
+__device__ __forceinline__ void warp_part(int64_t len, int64_t *wlo, int64_t *whi) {
+    constexpr int NW = NT / 32;
+    const int64_t sub = ((len + NW - 1) / NW + 31) & ~int64_t(31);
+    const int64_t a = (int64_t)warp_id() * sub;
+    *wlo = a < len ? a : len;
+    *whi = a + sub < len ? a + sub : len;
+}
+
+// Per-warp counts over the slice: keys > hi_k into sh->warp_a[warp], keys in
+// [lo_k, hi_k] into sh->warp_b[warp].  Ends with a __syncthreads().
+template <int NT, class KeyAt>
+__device__ __forceinline__ void warp_counts(Shared<NT> *sh, int64_t len, KeyAt key_at, uint32_t lo_k, uint32_t hi_k) {
+    int64_t wlo, whi;
+    warp_part<NT>(len, &wlo, &whi);
+    uint32_t g = 0, e = 0;
+    for (int64_t base = wlo; base < whi; base += 32 * kUnroll) {
+        uint32_t kk[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t j = base + u * 32 + lane_id();
+            kk[u] = j < whi ? key_at(j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const bool valid = base + u * 32 + lane_id() < whi;
+            g += valid && kk[u] > hi_k;
+            e += valid && kk[u] >= lo_k && kk[u] <= hi_k;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
+    if (lane_id() == 0) {
+        sh->warp_a[warp_id()] = g;
+        sh->warp_b[warp_id()] = e;
+    }
+    __syncthreads();
+}
+
+// This CTA's part of the output, after warp_counts(T, T): in position order,
+// its keys > T and its keys == T whose row-wide rank among the keys == T
+// (eq_before + rank within the CTA) is below `ties`, written from
+// out[out_pos] on (never at or past K).
+template <int NT, class KeyAt>
+__device__ __forceinline__ void emit_slice(Shared<NT> *sh, int64_t len, int64_t lo, KeyAt key_at, uint32_t T,
+                                           uint32_t ties, uint32_t eq_before, uint32_t out_pos, int32_t *out, int K) {
+    const int warp = warp_id(), lane = lane_id();
+    uint32_t eq_seen = eq_before + warp_sum_prefix(sh->warp_b, warp);
+    if (sh->warp_a[warp] == 0 && (sh->warp_b[warp] == 0 || eq_seen >= ties)) return;   // nothing selected here
+    int64_t wlo, whi;
+    warp_part<NT>(len, &wlo, &whi);
+    const uint32_t cta_eq = eq_before < ties ? eq_before : ties;
+    uint32_t o = out_pos + warp_sum_prefix(sh->warp_a, warp) + ((eq_seen < ties ? eq_seen : ties) - cta_eq);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t base = wlo; base < whi; base += 32 * kUnroll) {
+        uint32_t kk[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t j = base + u * 32 + lane;
+            kk[u] = j < whi ? key_at(j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t j = base + u * 32 + lane;
+            const bool valid = j < whi;
+            const bool is_eq = valid && kk[u] == T;
+            const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
+            const bool sel = (valid && kk[u] > T) || (is_eq && eq_seen + __popc(em & lt) < ties);
+            const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+                const uint32_t at = o + __popc(sm & lt);
+                if (at < (uint32_t)K) out[at] = (int32_t)(lo + j);
+            }
+            o += __popc(sm);
+            eq_seen += __popc(em);
+        }
+    }
+}
+
 // Selection of row `row` by CTA c of the C CTAs that share it.  All NT
-// threads of the CTA call this.  `cache` holds p.cache_keys keys.
-// hist1_ready: the row's first-digit histogram is already complete in the
-// row's global scratch (built by the producer of the scores), so the first
-// round reads it instead of counting.
+// threads of the CTA call this.  `cache` holds p.cache_keys keys followed by
+// 2 * p.smem_list list words.  hist1_ready: the row's first-digit histogram is
+// already complete in the row's global scratch (built by the producer of the
+// scores).
 template <int NT>
 __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int row, int c, int C,
                            bool hist1_ready) {
@@ -152,6 +293,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     int32_t *out = p.idx + (int64_t)row * K;
     const float *src = p.scores + (int64_t)row * p.stride;
     uint32_t *rs = (C > 1 || hist1_ready) ? p.scratch + (int64_t)row * p.scratch_row_words : nullptr;
+    uint32_t *ctl = rs ? rs + ctl_base(C) : nullptr;
 
     if (n <= K) {   // every visible position is selected (same decision in all CTAs of the row)
         if (c == 0) {
@@ -170,23 +312,10 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     const int64_t hi = n < lo + chunk ? n : lo + chunk;
     const int64_t len = hi - lo;
     const bool cached = len <= p.cache_keys;
+    uint32_t *lkey = cache + p.cache_keys, *lpos = lkey + p.smem_list;
 
     // scores may have been written earlier in the same kernel: read them through L2 (no .nc loads)
     auto key_at = [&](int64_t j) -> uint32_t { return cached ? cache[j] : float_order_key(__ldcg(src + lo + j)); };
-    // Visits keys j = base + u * NT + tid in batches of kUnroll per thread,
-    // all loads of a batch issued before any is used.
-    auto for_each_key = [&](auto &&fn) {
-        for (int64_t base = 0; base < len; base += (int64_t)kUnroll * NT) {
-            uint32_t kk[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t j = base + u * NT + threadIdx.x;
-                kk[u] = j < len ? key_at(j) : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) fn(base + u * NT + threadIdx.x, kk[u]);
-        }
-    };
     if (cached) {
         for (int64_t base = 0; base < len; base += (int64_t)kUnroll * NT) {
             float v[kUnroll];
@@ -203,129 +332,212 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
         }
         __syncthreads();
     }
-
-    // ---- three digit rounds
-    uint32_t prefix = 0, mask = 0, Krem = (uint32_t)K;
+    // Histogram (into sh->hist) of the slice keys that share `prefix` under
+    // `mask`, by the nb-bin digit at `shift`.
+    auto slice_hist = [&](uint32_t prefix, uint32_t mask, int shift, int nb) {
+        for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+        __syncthreads();
+        for (int64_t base = 0; base < len; base += (int64_t)kUnroll * NT) {
+            uint32_t kk[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t j = base + u * NT + threadIdx.x;
+                kk[u] = j < len ? key_at(j) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const bool active = base + u * NT + threadIdx.x < len && (kk[u] & mask) == prefix;
+                warp_hist_add(sh->hist, (kk[u] >> shift) & (nb - 1), active);
+            }
+        }
+        __syncthreads();
+    };
     uint32_t barrier_no = 0;
-    const int shifts[3] = {21, 10, 0};
-    const int nbits[3] = {11, 11, 10};
-    const int hoff[3] = {kHist1, kHist2, kHist3};
-    for (int r = 0; r < 3; ++r) {
-        const int nb = 1 << nbits[r], sh_ = shifts[r];
-        if (r == 0 && hist1_ready) {
-            for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = __ldcg(rs + kHist1 + j);
-            __syncthreads();
-        } else {
-            for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
-            __syncthreads();
-            // warp-aggregated increments: lanes that hit the same bin add once
-            for_each_key([&](int64_t j, uint32_t k) {
-                bool active = j < len && (k & mask) == prefix;
-                uint32_t bin = active ? (k >> sh_) & (nb - 1) : 0xFFFFFFFFu;
-                uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                if (active && lane_id() == __ffs(peers) - 1) atomicAdd(&sh->hist[bin], (uint32_t)__popc(peers));
-            });
-            __syncthreads();
-            if (C > 1) {
-                uint32_t *g = rs + hoff[r];
-                for (int j = threadIdx.x; j < nb; j += NT)
-                    if (sh->hist[j]) atomicAdd(g + j, sh->hist[j]);
-                if (!row_barrier<NT>(sh, rs + kCnt + 2 * C, ++barrier_no * C, p.status)) return;
-                for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = __ldcg(g + j);
-                __syncthreads();
-            }
-        }
-        find_threshold<NT>(sh, nb, Krem);
-        prefix |= (uint32_t)sh->bin << sh_;
-        mask |= (uint32_t)(nb - 1) << sh_;
-        Krem -= sh->above;
-        __syncthreads();
-    }
-    const uint32_t Tstar = prefix;
-    const uint32_t ties = Krem;   // how many keys equal to T* are taken (>= 1)
+    // Adds this CTA's histogram into the row's global one at g, waits for the
+    // other CTAs of the row, and loads the row's histogram back.
+    auto exchange_hist = [&](uint32_t *g, int nb) -> bool {
+        for (int j = threadIdx.x; j < nb; j += NT)
+            if (sh->hist[j]) atomicAdd(g + j, sh->hist[j]);
+        if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return false;
+        load_hist<NT>(sh, g, nb);
+        return true;
+    };
 
-    // ---- per-CTA counts of keys > T* and == T*
-    uint32_t gt = 0, eq = 0;
-    for_each_key([&](int64_t j, uint32_t k) {
-        gt += j < len && k > Tstar;
-        eq += j < len && k == Tstar;
-    });
-    uint32_t tot_gt, tot_eq;
-    block_scan<NT>(gt, sh->warp_tmp, &tot_gt);
-    block_scan<NT>(eq, sh->warp_tmp, &tot_eq);
-    uint32_t gt_before = 0, eq_before = 0;
+    // ---- digit 1
+    if (hist1_ready) {
+        load_hist<NT>(sh, rs + kHist1, kBins);
+    } else {
+        slice_hist(0u, 0u, 21, kBins);
+        if (C > 1 && !exchange_hist(rs + kHist1, kBins)) return;
+    }
+    find_threshold<NT>(sh, kBins, (uint32_t)K);
+    // a histogram that does not count this row's n scores (a position the
+    // producer rejected): select nothing
+    const bool empty = hist1_ready && sh->total != (uint32_t)n;
+    uint32_t prefix = (uint32_t)sh->bin << 21, mask = 0xFFE00000u, Krem = (uint32_t)K - sh->above;
+    __syncthreads();
+
+    // ---- the candidate list: every key of bin b1 in the row, with its position
+    bool use_list = false;
+    uint32_t m = 0;
     if (C > 1) {
-        uint32_t *cnt = rs + kCnt;
-        if (threadIdx.x == 0) {
-            cnt[2 * c] = tot_gt;
-            cnt[2 * c + 1] = tot_eq;
-        }
-        if (!row_barrier<NT>(sh, rs + kCnt + 2 * C, ++barrier_no * C, p.status)) return;
-        // every CTA has read the histograms: clear this CTA's share for the next call
-        for (int j = c * NT + threadIdx.x; j < kCnt; j += C * NT) rs[j] = 0;
-        uint32_t a = 0, e = 0;
-        for (int j = threadIdx.x; j < c; j += NT) {
-            a += __ldcg(cnt + 2 * j);
-            e += __ldcg(cnt + 2 * j + 1);
-        }
-        uint32_t t1, t2;
-        block_scan<NT>(a, sh->warp_tmp, &t1);
-        block_scan<NT>(e, sh->warp_tmp, &t2);
-        gt_before = t1;
-        eq_before = t2;
-    } else if (hist1_ready) {
-        __syncthreads();
-        for (int j = threadIdx.x; j < kHist2; j += NT) rs[j] = 0;
-    }
-    const uint32_t quota = eq_before >= ties ? 0u : min(ties - eq_before, tot_eq);
-    uint32_t out_pos = gt_before + min(eq_before, ties);
-
-    // ---- ordered compaction: 4 consecutive keys per thread per step
-    uint32_t eq_seen = 0;
-    for (int64_t base = 0; base < len; base += 4 * NT) {
-        uint32_t kk[4];
-        uint32_t e_cnt = 0;
-        const int64_t j0 = base + 4 * threadIdx.x;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            kk[u] = (j0 + u < len) ? key_at(j0 + u) : 0u;
-            e_cnt += (j0 + u < len) && kk[u] == Tstar;
-        }
-        uint32_t e_tot;
-        uint32_t e_incl = block_scan<NT>(e_cnt, sh->warp_tmp, &e_tot);
-        uint32_t e_rank = eq_seen + e_incl - e_cnt;
-        uint32_t sel[4], s_cnt = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            bool valid = j0 + u < len;
-            bool is_eq = valid && kk[u] == Tstar;
-            sel[u] = valid && (kk[u] > Tstar || (is_eq && e_rank < quota));
-            e_rank += is_eq;
-            s_cnt += sel[u];
-        }
-        uint32_t s_tot;
-        uint32_t s_incl = block_scan<NT>(s_cnt, sh->warp_tmp2, &s_tot);
-        uint32_t o = out_pos + s_incl - s_cnt;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (sel[u]) out[o++] = (int32_t)(lo + j0 + u);
-        out_pos += s_tot;
-        eq_seen += e_tot;
-    }
-    if (c == 0 && threadIdx.x == 0) p.count[row] = K;
-
-    if (C > 1) {   // the last CTA of the row out clears the counts and the barrier words
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t *bar = rs + kCnt + 2 * C;
-            __threadfence();
-            uint32_t done = atomicAdd(bar + 1, 1u);
-            if (done == (uint32_t)C - 1) {
-                for (int j = 0; j < 2 * C; ++j) rs[kCnt + j] = 0;
-                atomicExch(bar, 0u);
-                atomicExch(bar + 1, 0u);
+        if (!empty) {
+            warp_counts<NT>(sh, len, key_at, prefix, prefix | ~mask);
+            if (threadIdx.x == 0) {
+                uint32_t above = 0, mine = 0;
+                for (int w = 0; w < NT / 32; ++w) {
+                    above += sh->warp_a[w];
+                    mine += sh->warp_b[w];
+                }
+                rs[kCnt + 2 * C + c] = above;
+                sh->base = mine ? atomicAdd(ctl + 2, mine) : 0u;
+            }
+            __syncthreads();
+            const int warp = warp_id(), lane = lane_id();
+            if (sh->warp_b[warp]) {
+                int64_t wlo, whi;
+                warp_part<NT>(len, &wlo, &whi);
+                uint32_t at = sh->base + warp_sum_prefix(sh->warp_b, warp);
+                uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+                for (int64_t base = wlo; base < whi; base += 32) {
+                    const int64_t j = base + lane;
+                    const uint32_t k = j < whi ? key_at(j) : 0u;
+                    const bool in = j < whi && (k & mask) == prefix;
+                    const uint32_t bm = __ballot_sync(0xffffffffu, in);
+                    if (in) {
+                        const uint32_t slot = at + __popc(bm & ((1u << lane) - 1u));
+                        if (slot < (uint32_t)p.list_cap) {
+                            gkey[slot] = k;
+                            gpos[slot] = (uint32_t)(lo + j);
+                        }
+                    }
+                    at += __popc(bm);
+                }
             }
         }
+        if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
+        m = __ldcg(ctl + 2);
+        use_list = m <= (uint32_t)p.smem_list;
+        if (use_list && !empty) {
+            const uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+            for (uint32_t base = 0; base < m; base += 4 * NT) {
+                uint32_t kv[4], pv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t j = base + u * NT + threadIdx.x;
+                    kv[u] = j < m ? __ldcg(gkey + j) : 0u;
+                    pv[u] = j < m ? __ldcg(gpos + j) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t j = base + u * NT + threadIdx.x;
+                    if (j < m) {
+                        lkey[j] = kv[u];
+                        lpos[j] = pv[u];
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    if (!empty) {
+        // ---- digits 2 and 3
+        const int shifts[2] = {10, 0};
+        const int nbits[2] = {11, 10};
+        const int hoff[2] = {kHist2, kHist3};
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int nb = 1 << nbits[r], sh_ = shifts[r];
+            if (use_list) {
+                for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+                __syncthreads();
+                for (uint32_t j = threadIdx.x; j < ((m + 31u) & ~31u); j += NT) {   // whole warps
+                    const uint32_t k = j < m ? lkey[j] : 0u;
+                    warp_hist_add(sh->hist, (k >> sh_) & (nb - 1), j < m && (k & mask) == prefix);
+                }
+                __syncthreads();
+            } else {
+                slice_hist(prefix, mask, sh_, nb);
+                if (C > 1 && !exchange_hist(rs + hoff[r], nb)) return;
+            }
+            find_threshold<NT>(sh, nb, Krem);
+            prefix |= (uint32_t)sh->bin << sh_;
+            mask |= (uint32_t)(nb - 1) << sh_;
+            Krem -= sh->above;
+            __syncthreads();
+        }
+        const uint32_t Tstar = prefix;
+        const uint32_t ties = Krem;   // keys equal to T* that are taken (>= 1)
+
+        // ---- this CTA's offset in the row's output
+        warp_counts<NT>(sh, len, key_at, Tstar, Tstar);
+        uint32_t gt_before = 0, eq_before = 0;
+        if (use_list) {
+            // earlier CTAs: all their keys above bin b1, and their list entries > T* / == T*
+            uint32_t a = 0, e = 0;
+            for (int j = threadIdx.x; j < c; j += NT) a += __ldcg(rs + kCnt + 2 * C + j);
+            for (uint32_t j = threadIdx.x; j < m; j += NT)
+                if ((int64_t)lpos[j] < lo) {
+                    a += lkey[j] > Tstar;
+                    e += lkey[j] == Tstar;
+                }
+            block_scan<NT>(a, sh->warp_tmp, &gt_before);
+            block_scan<NT>(e, sh->warp_tmp, &eq_before);
+        } else if (C > 1) {
+            uint32_t *cnt = rs + kCnt;
+            if (threadIdx.x == 0) {
+                uint32_t g = 0, e = 0;
+                for (int w = 0; w < NT / 32; ++w) {
+                    g += sh->warp_a[w];
+                    e += sh->warp_b[w];
+                }
+                cnt[2 * c] = g;
+                cnt[2 * c + 1] = e;
+            }
+            if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
+            uint32_t a = 0, e = 0;
+            for (int j = threadIdx.x; j < c; j += NT) {
+                a += __ldcg(cnt + 2 * j);
+                e += __ldcg(cnt + 2 * j + 1);
+            }
+            block_scan<NT>(a, sh->warp_tmp, &gt_before);
+            block_scan<NT>(e, sh->warp_tmp, &eq_before);
+        }
+
+        // ---- emission
+        emit_slice<NT>(sh, len, lo, key_at, Tstar, ties, eq_before, gt_before + min(eq_before, ties), out, K);
+        if (c == 0 && threadIdx.x == 0) p.count[row] = K;
+    } else if (c == 0) {
+        for (int j = threadIdx.x; j < K; j += NT) out[j] = -1;
+        if (threadIdx.x == 0) p.count[row] = 0;
+    }
+
+    // ---- the last CTA of the row to leave clears the row's words for the next call
+    __syncthreads();
+    if (C > 1) {
+        if (threadIdx.x == 0) {
+            __threadfence();
+            sh->ok = atomicAdd(ctl + 1, 1u) == (uint32_t)C - 1;
+        }
+        __syncthreads();
+        if (sh->ok) {
+            __threadfence();
+            for (int j = threadIdx.x; j < ctl_base(C); j += NT) rs[j] = 0;
+            const uint32_t used = m < (uint32_t)p.list_cap ? m : (uint32_t)p.list_cap;
+            uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+            for (uint32_t j = threadIdx.x; j < used; j += NT) {
+                gkey[j] = 0;
+                gpos[j] = 0;
+            }
+            if (threadIdx.x == 0) {
+                ctl[0] = 0;
+                ctl[1] = 0;
+                ctl[2] = 0;
+            }
+        }
+    } else if (hist1_ready) {
+        for (int j = threadIdx.x; j < kHist2; j += NT) rs[j] = 0;
     }
 }
 
