@@ -34,7 +34,7 @@ constexpr int kTeams = 4;                     // attention teams of 4 warps (nam
 constexpr int kMaxRows = 16;                  // B * T handled by the fused path
 constexpr int kMaxHistRows = 8;               // rows whose first histogram the indexer builds
 
-static_assert(kTeams * 4 <= kWarps, "the attention teams must fit in the CTA");
+static_assert(kTeams * 4 < kWarps, "the attention teams must leave warps free in the CTA");
 
 struct Params {
     indexer::Params ix;
@@ -95,7 +95,7 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(smem);
         uint32_t *cache = reinterpret_cast<uint32_t *>(smem + smem_align(sizeof(topk::Shared<kThreads>)));
         const int row = blockIdx.x / fp.C, c = blockIdx.x % fp.C;
-        topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, fp.hist_ready != 0);
+        topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, fp.hist_ready != 0, true);
     }
     if (!grid_sync(fp.grid_bar, 2 * G, status, &sync_flag)) return;
 
@@ -115,9 +115,14 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
                     default: attn::attn_unit<4>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
                 }
             }
+        } else if ((int)blockIdx.x < fp.rows * fp.C && (fp.C > 1 || fp.hist_ready)) {
+            // the warps outside the teams clear the selection scratch for the next call
+            constexpr int kFree = kThreads - kTeams * 128;
+            topk::clear_row_share(fp.tk, blockIdx.x / fp.C, blockIdx.x % fp.C, fp.C, threadIdx.x - kTeams * 128, kFree);
         }
     }
     if (!grid_sync(fp.grid_bar, 3 * G, status, &sync_flag)) return;
+    if ((int)blockIdx.x < fp.rows * fp.C && blockIdx.x % fp.C == 0) topk::reset_row_ctl(fp.tk, blockIdx.x / fp.C, fp.C);
 
     // ---- phase 4: combine, one CTA per (query, head)
     for (int gw = blockIdx.x; gw < fp.rows * DSA_Q_HEADS; gw += G)
@@ -221,11 +226,13 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     {   // shared memory after the fixed part: the CTA's slice of keys, then the candidate list
         const int64_t avail = (int64_t)(smem - 1024 - top_fixed) / 4;
         const int64_t chunk = ((ia.Lmax + plan.C - 1) / plan.C + 3) & ~int64_t(3);
-        int64_t list = topk::kListCap;
-        if (chunk + 2 * list > avail) list = std::max<int64_t>(0, (avail - chunk) / 2);
-        if (list < 1024) list = std::min<int64_t>(topk::kListCap, avail / 4);   // slices too long to cache
+        const int64_t list = std::min<int64_t>(topk::kSmemList, avail / 8);
+        int64_t cand = std::min<int64_t>(topk::kCandCap, std::max<int64_t>(0, (avail - chunk) / 2 - list));
+        if (cand < 1024) cand = std::min<int64_t>(topk::kCandCap, (avail - 2 * list) / 4);   // slices too long to cache
+        cand = std::max<int64_t>(0, cand) / kWarps * kWarps;
         tp.smem_list = (int)list;
-        tp.cache_keys = (int)(avail - 2 * list);
+        tp.cand_cap = (int)cand;
+        tp.cache_keys = (int)(avail - 2 * list - 2 * cand);
     }
     tp.list_cap = topk::kListCap;
     tp.Lmax = ia.Lmax;

@@ -56,6 +56,7 @@ struct TopkPlan {
     int cache_keys = 0;    // keys cached in shared memory per CTA
     int list_cap = 0;      // candidate-list entries per row in the scratch
     int smem_list = 0;     // candidate-list entries that fit in shared memory
+    int cand_cap = 0;      // per-warp candidate entries in shared memory, all warps together
     int64_t Lmax = 0;      // positions held by each scores row
     size_t smem = 0;
     size_t scratch_bytes = 0;  // cross-CTA scratch (only when C > 1)

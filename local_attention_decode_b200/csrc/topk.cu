@@ -39,6 +39,7 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
     plan->cache_keys = (int)std::min<int64_t>(chunk, kMaxCacheKeys);
     plan->list_cap = 0;
     plan->smem_list = 0;
+    plan->cand_cap = 0;
     plan->scratch_bytes = 0;
     if (C > 1) {
         int cap = kListCap;
@@ -47,11 +48,14 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
         cap = (int)std::min<size_t>(cap, (max_scratch_bytes - fixed) / ((size_t)plan->rows * 8));
         plan->list_cap = cap & ~3;
         const size_t used = sizeof(Shared<kThreads>) + (size_t)plan->cache_keys * 4;
-        const size_t room = dev.smem_optin > used ? (dev.smem_optin - used) / 8 : 0;
-        plan->smem_list = (int)std::min<size_t>(plan->list_cap, room);
+        size_t room = dev.smem_optin > used ? (dev.smem_optin - used) / 8 : 0;   // (key, position) pairs
+        plan->smem_list = (int)std::min<size_t>({(size_t)plan->list_cap, (size_t)kSmemList, room});
+        room -= plan->smem_list;
+        plan->cand_cap = (int)(std::min<size_t>(kCandCap, room) / (kThreads / 32) * (kThreads / 32));
         plan->scratch_bytes = (size_t)plan->rows * scratch_words(C, plan->list_cap) * 4;
     }
-    plan->smem = sizeof(Shared<kThreads>) + ((size_t)plan->cache_keys + 2 * (size_t)plan->smem_list) * 4;
+    plan->smem = sizeof(Shared<kThreads>) +
+                 ((size_t)plan->cache_keys + 2 * (size_t)plan->smem_list + 2 * (size_t)plan->cand_cap) * 4;
     return DSA_OK;
 }
 
@@ -73,6 +77,7 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
     p.cache_keys = plan.cache_keys;
     p.list_cap = plan.list_cap;
     p.smem_list = plan.smem_list;
+    p.cand_cap = plan.cand_cap;
     p.Lmax = plan.Lmax;
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(topk)");

@@ -18,16 +18,17 @@
 //   digit 1     the row's 2048-bin histogram of the top 11 bits -- built by the
 //               producer of the scores, or by the CTAs adding their slices'
 //               histograms into the row's global histogram and meeting at a
-//               barrier -- gives the threshold bin b1;
-//   list        every CTA appends its keys of bin b1, with their positions, to
-//               the row's candidate list and publishes how many of its keys lie
-//               above bin b1; one barrier;
-//   digits 2, 3 each CTA loads the whole list and finishes the select on it
-//               alone; its output offset is the earlier CTAs' counts above b1
-//               plus the list entries that lie before its slice.  When the list
-//               does not fit in shared memory (many keys share the threshold
-//               bin, e.g. heavy ties), digits 2 and 3 are exchanged like digit
-//               1, and so are the per-CTA (greater, equal) counts after them;
+//               barrier -- gives the threshold bin;
+//   digit 2     the same exchange for the next 11 bits of the keys in that bin;
+//   list        every CTA appends its keys that share the threshold's top 22
+//               bits, with their positions, to the row's candidate list and
+//               publishes how many of its keys lie above them; one barrier;
+//   digit 3     each CTA loads the (short) list and finishes the select on it
+//               alone; its output offset is the earlier CTAs' counts above the
+//               22-bit bin plus the list entries that lie before its slice.
+//               When the list does not fit in shared memory (many keys share
+//               the 22-bit bin, e.g. heavy ties), digit 3 is exchanged like the
+//               others, and so are the per-CTA (greater, equal) counts at T*;
 //   emission    each warp compacts its part of the slice with ballots, from its
 //               own offset in the row's output.
 //
@@ -43,17 +44,20 @@ namespace topk {
 constexpr int kBins = 2048;                 // largest digit: 11 bits
 constexpr int kUnroll = 8;                  // independent loads in flight per thread
 constexpr int kListCap = 12288;             // candidate-list entries per row (global scratch)
+constexpr int kSmemList = 4096;             // candidate-list entries a CTA takes into shared memory
+constexpr int kCandCap = 8192;              // per-warp candidates a CTA keeps in shared memory, in all
 
 // Per-row scratch (u32 words), used when C > 1 or when the first histogram is
 // produced by the indexer:
 //   [kHist1, +2048) [kHist2, +2048) [kHist3, +1024)  digit histograms
 //   [kCnt, +2C)      per-CTA (greater, equal) counts at T* (exchange path)
-//   [kCnt+2C, +C)    per-CTA counts of keys above bin b1
-//   ctl_base(C):     [0] barrier arrivals, [1] CTAs done, [2] list length
+//   [kCnt+2C, +C)    per-CTA counts of keys above the 22-bit threshold bin
+//   ctl_base(C):     [0] barrier arrivals, [1] CTAs done, [2] list length,
+//                    [3] a CTA's candidates overflowed its shared memory
 //   list_base(C):    list_cap keys, then list_cap positions
 constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kCnt = 5120;
 __host__ __device__ constexpr int ctl_base(int C) { return kCnt + 3 * C; }
-__host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + 3 + 3) & ~3; }
+__host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + 4 + 3) & ~3; }
 __host__ __device__ constexpr int scratch_words(int C, int list_cap) { return list_base(C) + 2 * list_cap; }
 
 struct Params {
@@ -69,6 +73,7 @@ struct Params {
     int cache_keys;        // keys of the slice kept in shared memory
     int list_cap;          // list entries in the row's global scratch
     int smem_list;         // list entries that fit in shared memory after the cache (<= list_cap)
+    int cand_cap;          // candidate entries in shared memory after the list (a multiple of NT / 32)
     int64_t Lmax;
 };
 
@@ -78,6 +83,7 @@ struct alignas(16) Shared {
     uint32_t warp_tmp[NT / 32];
     uint32_t warp_a[NT / 32];
     uint32_t warp_b[NT / 32];
+    uint32_t warp_c[NT / 32];
     int bin;
     uint32_t above;
     uint32_t total;
@@ -116,26 +122,60 @@ __device__ __noinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, uint
 
 // Threshold bin of sh->hist[0..nbins): the bin b with above(b) < K <= above(b) + h[b],
 // above(b) = number of keys in bins > b.  Result in sh->bin / sh->above, the
-// histogram's total in sh->total.
+// histogram's total in sh->total (bin 0, above 0 when K exceeds the total).
+// nbins is 1024 or 2048.  One warp searches: each lane sums a run of nbins / 32
+// bins, a suffix scan over the lanes finds the run, the warp then splits that run.
 template <int NT>
 __device__ __noinline__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
-    const int per = (nbins + NT - 1) / NT;
-    const int lo = threadIdx.x * per;
-    uint32_t mine = 0;
-    for (int j = 0; j < per; ++j)
-        if (lo + j < nbins) mine += sh->hist[lo + j];
-    uint32_t total;
-    uint32_t incl = block_scan<NT>(mine, sh->warp_tmp, &total);
-    if (threadIdx.x == 0) sh->total = total;
-    uint32_t above = total - incl;      // keys in bins after this thread's range
-    for (int j = per - 1; j >= 0; --j) {
-        if (lo + j >= nbins) continue;
-        uint32_t h = sh->hist[lo + j];
-        if (above < K && K <= above + h) {
-            sh->bin = lo + j;
-            sh->above = above;
+    if (warp_id() == 0) {
+        const int lane = lane_id();
+        const int per = nbins >> 5;
+        const uint32_t *h = sh->hist + lane * per;
+        uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+        for (int j = 0; j < per; j += 4) {   // rotated: no bank conflicts
+            s0 += h[(j + lane) & (per - 1)];
+            s1 += h[(j + 1 + lane) & (per - 1)];
+            s2 += h[(j + 2 + lane) & (per - 1)];
+            s3 += h[(j + 3 + lane) & (per - 1)];
         }
-        above += h;
+        const uint32_t s = (s0 + s1) + (s2 + s3);
+        uint32_t incl = s;   // keys in this lane's run and all higher runs
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += u;
+        }
+        const uint32_t above_run = incl - s;
+        const uint32_t total = __shfl_sync(0xffffffffu, incl, 0);
+        const uint32_t hit = __ballot_sync(0xffffffffu, above_run < K && K <= incl);
+        if (lane == 0) {
+            sh->total = total;
+            sh->bin = 0;
+            sh->above = 0;
+        }
+        if (hit) {
+            const int L = __ffs(hit) - 1;
+            const uint32_t base = __shfl_sync(0xffffffffu, above_run, L);
+            const int q = per >> 5;   // bins of run L per lane: 2 or 1
+            const int b0 = L * per + lane * q;
+            uint32_t t = 0;
+            for (int j = 0; j < q; ++j) t += sh->hist[b0 + j];
+            uint32_t inc2 = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t u = __shfl_down_sync(0xffffffffu, inc2, o);
+                if (lane + o < 32) inc2 += u;
+            }
+            uint32_t run = base + inc2 - t;   // keys above this lane's bins
+            for (int j = q - 1; j >= 0; --j) {
+                const uint32_t hb = sh->hist[b0 + j];
+                if (run < K && K <= run + hb) {
+                    sh->bin = b0 + j;
+                    sh->above = run;
+                }
+                run += hb;
+            }
+        }
     }
     __syncthreads();
 }
@@ -203,27 +243,47 @@ __device__ __forceinline__ void warp_part(int64_t len, int64_t *wlo, int64_t *wh
     *whi = a + sub < len ? a + sub : len;
 }
 
+// Calls fn(j, valid, k) for the keys j of this warp's part [wlo, whi), 32
+// consecutive keys per call, in position order (all lanes call fn together).
+// Keys cached in shared memory are read one group at a time (compact code);
+// keys read from global memory are fetched kUnroll groups at a time.
+template <class KeyAt, class Fn>
+__device__ __forceinline__ void warp_walk(int64_t wlo, int64_t whi, bool cached, const uint32_t *cache,
+                                          KeyAt key_at, Fn fn) {
+    const int lane = lane_id();
+    if (cached) {
+#pragma unroll 1
+        for (int64_t j0 = wlo; j0 < whi; j0 += 32) {
+            const int64_t j = j0 + lane;
+            const bool valid = j < whi;
+            fn(j, valid, valid ? cache[j] : 0u);
+        }
+    } else {
+        for (int64_t base = wlo; base < whi; base += 32 * kUnroll) {
+            uint32_t kk[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t j = base + u * 32 + lane;
+                kk[u] = j < whi ? key_at(j) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) fn(base + u * 32 + lane, base + u * 32 + lane < whi, kk[u]);
+        }
+    }
+}
+
 // Per-warp counts over the slice: keys > hi_k into sh->warp_a[warp], keys in
 // [lo_k, hi_k] into sh->warp_b[warp].  Ends with a __syncthreads().
 template <int NT, class KeyAt>
-__device__ __forceinline__ void warp_counts(Shared<NT> *sh, int64_t len, KeyAt key_at, uint32_t lo_k, uint32_t hi_k) {
+__device__ __forceinline__ void warp_counts(Shared<NT> *sh, int64_t len, bool cached, const uint32_t *cache,
+                                            KeyAt key_at, uint32_t lo_k, uint32_t hi_k) {
     int64_t wlo, whi;
     warp_part<NT>(len, &wlo, &whi);
     uint32_t g = 0, e = 0;
-    for (int64_t base = wlo; base < whi; base += 32 * kUnroll) {
-        uint32_t kk[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t j = base + u * 32 + lane_id();
-            kk[u] = j < whi ? key_at(j) : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const bool valid = base + u * 32 + lane_id() < whi;
-            g += valid && kk[u] > hi_k;
-            e += valid && kk[u] >= lo_k && kk[u] <= hi_k;
-        }
-    }
+    warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t, bool valid, uint32_t k) {
+        g += valid && k > hi_k;
+        e += valid && k >= lo_k && k <= hi_k;
+    });
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         g += __shfl_xor_sync(0xffffffffu, g, o);
@@ -241,8 +301,9 @@ __device__ __forceinline__ void warp_counts(Shared<NT> *sh, int64_t len, KeyAt k
 // (eq_before + rank within the CTA) is below `ties`, written from
 // out[out_pos] on (never at or past K).
 template <int NT, class KeyAt>
-__device__ __forceinline__ void emit_slice(Shared<NT> *sh, int64_t len, int64_t lo, KeyAt key_at, uint32_t T,
-                                           uint32_t ties, uint32_t eq_before, uint32_t out_pos, int32_t *out, int K) {
+__device__ __forceinline__ void emit_slice(Shared<NT> *sh, int64_t len, int64_t lo, bool cached, const uint32_t *cache,
+                                           KeyAt key_at, uint32_t T, uint32_t ties, uint32_t eq_before,
+                                           uint32_t out_pos, int32_t *out, int K) {
     const int warp = warp_id(), lane = lane_id();
     uint32_t eq_seen = eq_before + warp_sum_prefix(sh->warp_b, warp);
     if (sh->warp_a[warp] == 0 && (sh->warp_b[warp] == 0 || eq_seen >= ties)) return;   // nothing selected here
@@ -251,39 +312,29 @@ __device__ __forceinline__ void emit_slice(Shared<NT> *sh, int64_t len, int64_t 
     const uint32_t cta_eq = eq_before < ties ? eq_before : ties;
     uint32_t o = out_pos + warp_sum_prefix(sh->warp_a, warp) + ((eq_seen < ties ? eq_seen : ties) - cta_eq);
     const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t base = wlo; base < whi; base += 32 * kUnroll) {
-        uint32_t kk[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t j = base + u * 32 + lane;
-            kk[u] = j < whi ? key_at(j) : 0u;
+    warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
+        const bool is_eq = valid && k == T;
+        const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
+        const bool sel = (valid && k > T) || (is_eq && eq_seen + __popc(em & lt) < ties);
+        const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+            const uint32_t at = o + __popc(sm & lt);
+            if (at < (uint32_t)K) out[at] = (int32_t)(lo + j);
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t j = base + u * 32 + lane;
-            const bool valid = j < whi;
-            const bool is_eq = valid && kk[u] == T;
-            const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
-            const bool sel = (valid && kk[u] > T) || (is_eq && eq_seen + __popc(em & lt) < ties);
-            const uint32_t sm = __ballot_sync(0xffffffffu, sel);
-            if (sel) {
-                const uint32_t at = o + __popc(sm & lt);
-                if (at < (uint32_t)K) out[at] = (int32_t)(lo + j);
-            }
-            o += __popc(sm);
-            eq_seen += __popc(em);
-        }
-    }
+        o += __popc(sm);
+        eq_seen += __popc(em);
+    });
 }
 
 // Selection of row `row` by CTA c of the C CTAs that share it.  All NT
-// threads of the CTA call this.  `cache` holds p.cache_keys keys followed by
-// 2 * p.smem_list list words.  hist1_ready: the row's first-digit histogram is
+// threads of the CTA call this.  `cache` holds p.cache_keys keys, then
+// 2 * p.smem_list list words, then 2 * p.cand_cap candidate words.  hist1_ready: the row's first-digit histogram is
 // already complete in the row's global scratch (built by the producer of the
-// scores).
+// scores).  defer_clear: leave the row's scratch words for clear_row_share
+// and reset_row_ctl (called once every CTA of the row is past the selection).
 template <int NT>
 __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int row, int c, int C,
-                           bool hist1_ready) {
+                           bool hist1_ready, bool defer_clear = false) {
     const int K = p.K;
     int64_t n = (int64_t)__ldg(p.q_pos + row) + 1;
     if (n > p.Lmax) {   // a position beyond the scores buffer: flag it, select within the buffer
@@ -300,7 +351,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
             for (int j = threadIdx.x; j < K; j += NT) out[j] = j < n ? j : -1;
             if (threadIdx.x == 0) p.count[row] = (int32_t)(n > 0 ? n : 0);
         }
-        if (hist1_ready) {   // the producer's histogram is not needed: clear this CTA's share
+        if (hist1_ready && !defer_clear) {   // the producer's histogram is not needed: clear this CTA's share
             __syncthreads();
             for (int j = c * NT + threadIdx.x; j < kHist2; j += C * NT) rs[j] = 0;
         }
@@ -313,9 +364,24 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     const int64_t len = hi - lo;
     const bool cached = len <= p.cache_keys;
     uint32_t *lkey = cache + p.cache_keys, *lpos = lkey + p.smem_list;
+    constexpr int NW = NT / 32;
+    const int warp = warp_id(), lane = lane_id();
+    const uint32_t lt = (1u << lane) - 1u;
+    const int seg = p.cand_cap / NW;   // candidate entries per warp
+    uint32_t *wkey = lpos + p.smem_list + warp * seg, *wpos = wkey + p.cand_cap;
 
     // scores may have been written earlier in the same kernel: read them through L2 (no .nc loads)
     auto key_at = [&](int64_t j) -> uint32_t { return cached ? cache[j] : float_order_key(__ldcg(src + lo + j)); };
+    // the producer's histogram is fetched while the slice streams in
+    constexpr int kHistPer = (kBins + NT - 1) / NT;
+    uint32_t hv[kHistPer];
+    if (hist1_ready) {
+#pragma unroll
+        for (int u = 0; u < kHistPer; ++u) {
+            const int j = u * NT + threadIdx.x;
+            hv[u] = j < kBins ? __ldcg(rs + kHist1 + j) : 0u;
+        }
+    }
     if (cached) {
         for (int64_t base = 0; base < len; base += (int64_t)kUnroll * NT) {
             float v[kUnroll];
@@ -330,8 +396,15 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 if (j < len) cache[j] = float_order_key(v[u]);
             }
         }
-        __syncthreads();
     }
+    if (hist1_ready) {
+#pragma unroll
+        for (int u = 0; u < kHistPer; ++u) {
+            const int j = u * NT + threadIdx.x;
+            if (j < kBins) sh->hist[j] = hv[u];
+        }
+    }
+    __syncthreads();
     // Histogram (into sh->hist) of the slice keys that share `prefix` under
     // `mask`, by the nb-bin digit at `shift`.
     auto slice_hist = [&](uint32_t prefix, uint32_t mask, int shift, int nb) {
@@ -364,9 +437,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     };
 
     // ---- digit 1
-    if (hist1_ready) {
-        load_hist<NT>(sh, rs + kHist1, kBins);
-    } else {
+    if (!hist1_ready) {
         slice_hist(0u, 0u, 21, kBins);
         if (C > 1 && !exchange_hist(rs + kHist1, kBins)) return;
     }
@@ -376,42 +447,115 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     const bool empty = hist1_ready && sh->total != (uint32_t)n;
     uint32_t prefix = (uint32_t)sh->bin << 21, mask = 0xFFE00000u, Krem = (uint32_t)K - sh->above;
     __syncthreads();
+    // Narrows (prefix, mask, Krem) by the nb-bin digit at `shift`, from sh->hist.
+    auto take_digit = [&](int nb, int shift) {
+        find_threshold<NT>(sh, nb, Krem);
+        prefix |= (uint32_t)sh->bin << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
+        Krem -= sh->above;
+        __syncthreads();
+    };
 
-    // ---- the candidate list: every key of bin b1 in the row, with its position
+    // ---- digit 2, over the whole row; in the same pass each warp keeps, in
+    //      position order, its candidates: the keys at or above the threshold bin
+    if (!empty) {
+        for (int j = threadIdx.x; j < kBins; j += NT) sh->hist[j] = 0;
+        __syncthreads();
+        int64_t wlo, whi;
+        warp_part<NT>(len, &wlo, &whi);
+        uint32_t wc = 0;
+        warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
+            if (valid && (k & mask) == prefix) atomicAdd(&sh->hist[(k >> 10) & (kBins - 1)], 1u);
+            const bool cand = valid && k >= prefix;
+            const uint32_t cm = __ballot_sync(0xffffffffu, cand);
+            if (cand) {
+                const uint32_t slot = wc + __popc(cm & lt);
+                if (slot < (uint32_t)seg) {
+                    wkey[slot] = k;
+                    wpos[slot] = (uint32_t)(lo + j);
+                }
+            }
+            wc += __popc(cm);
+        });
+        if (lane == 0) sh->warp_a[warp] = wc;
+        __syncthreads();
+        if (C > 1 && threadIdx.x == 0) {
+            bool over = false;
+            for (int w = 0; w < NW; ++w) over |= sh->warp_a[w] > (uint32_t)seg;
+            if (over) atomicOr(ctl + 3, 1u);
+        }
+        if (C > 1 && !exchange_hist(rs + kHist2, kBins)) return;
+        take_digit(kBins, 10);
+    }
+    // every CTA's candidates fit: (read after the exchange, the same in every CTA)
+    const bool cand_ok = C > 1 && !empty && seg > 0 && __ldcg(ctl + 3) == 0u;
+
+    // ---- the candidate list: every key of the row whose top 22 bits are the
+    //      threshold's, with its position; each CTA publishes its count of keys
+    //      above them
     bool use_list = false;
     uint32_t m = 0;
     if (C > 1) {
         if (!empty) {
-            warp_counts<NT>(sh, len, key_at, prefix, prefix | ~mask);
+            const uint32_t hi22 = prefix | ~mask;
+            uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+            if (cand_ok) {
+                const uint32_t wc = sh->warp_a[warp];
+                uint32_t a = 0, e = 0;
+                for (uint32_t i = lane; i < wc; i += 32) {
+                    a += wkey[i] > hi22;
+                    e += (wkey[i] & mask) == prefix;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    a += __shfl_xor_sync(0xffffffffu, a, o);
+                    e += __shfl_xor_sync(0xffffffffu, e, o);
+                }
+                if (lane == 0) {
+                    sh->warp_c[warp] = a;
+                    sh->warp_b[warp] = e;
+                }
+            } else {
+                warp_counts<NT>(sh, len, cached, cache, key_at, prefix, hi22);   // above into warp_a, in-bin into warp_b
+                if (lane == 0) sh->warp_c[warp] = sh->warp_a[warp];
+            }
+            __syncthreads();
             if (threadIdx.x == 0) {
                 uint32_t above = 0, mine = 0;
-                for (int w = 0; w < NT / 32; ++w) {
-                    above += sh->warp_a[w];
+                for (int w = 0; w < NW; ++w) {
+                    above += sh->warp_c[w];
                     mine += sh->warp_b[w];
                 }
                 rs[kCnt + 2 * C + c] = above;
                 sh->base = mine ? atomicAdd(ctl + 2, mine) : 0u;
             }
             __syncthreads();
-            const int warp = warp_id(), lane = lane_id();
-            if (sh->warp_b[warp]) {
-                int64_t wlo, whi;
-                warp_part<NT>(len, &wlo, &whi);
+            if (sh->warp_b[warp]) {   // append this warp's keys of the 22-bit bin
                 uint32_t at = sh->base + warp_sum_prefix(sh->warp_b, warp);
-                uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
-                for (int64_t base = wlo; base < whi; base += 32) {
-                    const int64_t j = base + lane;
-                    const uint32_t k = j < whi ? key_at(j) : 0u;
-                    const bool in = j < whi && (k & mask) == prefix;
+                auto put = [&](bool in, uint32_t k, uint32_t pos) {
                     const uint32_t bm = __ballot_sync(0xffffffffu, in);
                     if (in) {
-                        const uint32_t slot = at + __popc(bm & ((1u << lane) - 1u));
+                        const uint32_t slot = at + __popc(bm & lt);
                         if (slot < (uint32_t)p.list_cap) {
                             gkey[slot] = k;
-                            gpos[slot] = (uint32_t)(lo + j);
+                            gpos[slot] = pos;
                         }
                     }
                     at += __popc(bm);
+                };
+                if (cand_ok) {
+                    const uint32_t wc = sh->warp_a[warp];
+                    for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
+                        const uint32_t i = i0 + lane;
+                        const uint32_t k = i < wc ? wkey[i] : 0u;
+                        put(i < wc && (k & mask) == prefix, k, i < wc ? wpos[i] : 0u);
+                    }
+                } else {
+                    int64_t wlo, whi;
+                    warp_part<NT>(len, &wlo, &whi);
+                    warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
+                        put(valid && (k & mask) == prefix, k, (uint32_t)(lo + j));
+                    });
                 }
             }
         }
@@ -442,39 +586,27 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     }
 
     if (!empty) {
-        // ---- digits 2 and 3
-        const int shifts[2] = {10, 0};
-        const int nbits[2] = {11, 10};
-        const int hoff[2] = {kHist2, kHist3};
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int nb = 1 << nbits[r], sh_ = shifts[r];
-            if (use_list) {
-                for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
-                __syncthreads();
-                for (uint32_t j = threadIdx.x; j < ((m + 31u) & ~31u); j += NT) {   // whole warps
-                    const uint32_t k = j < m ? lkey[j] : 0u;
-                    warp_hist_add(sh->hist, (k >> sh_) & (nb - 1), j < m && (k & mask) == prefix);
-                }
-                __syncthreads();
-            } else {
-                slice_hist(prefix, mask, sh_, nb);
-                if (C > 1 && !exchange_hist(rs + hoff[r], nb)) return;
-            }
-            find_threshold<NT>(sh, nb, Krem);
-            prefix |= (uint32_t)sh->bin << sh_;
-            mask |= (uint32_t)(nb - 1) << sh_;
-            Krem -= sh->above;
+        // ---- digit 3: on the list, or over the row
+        if (use_list) {
+            for (int j = threadIdx.x; j < 1024; j += NT) sh->hist[j] = 0;
             __syncthreads();
+            for (uint32_t j = threadIdx.x; j < m; j += NT) {
+                const uint32_t k = lkey[j];
+                if ((k & mask) == prefix) atomicAdd(&sh->hist[k & 1023u], 1u);
+            }
+            __syncthreads();
+        } else {
+            slice_hist(prefix, mask, 0, 1024);
+            if (C > 1 && !exchange_hist(rs + kHist3, 1024)) return;
         }
+        take_digit(1024, 0);
         const uint32_t Tstar = prefix;
         const uint32_t ties = Krem;   // keys equal to T* that are taken (>= 1)
 
         // ---- this CTA's offset in the row's output
-        warp_counts<NT>(sh, len, key_at, Tstar, Tstar);
         uint32_t gt_before = 0, eq_before = 0;
         if (use_list) {
-            // earlier CTAs: all their keys above bin b1, and their list entries > T* / == T*
+            // earlier CTAs: all their keys above the 22-bit bin, and their list entries > T* / == T*
             uint32_t a = 0, e = 0;
             for (int j = threadIdx.x; j < c; j += NT) a += __ldcg(rs + kCnt + 2 * C + j);
             for (uint32_t j = threadIdx.x; j < m; j += NT)
@@ -484,29 +616,71 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 }
             block_scan<NT>(a, sh->warp_tmp, &gt_before);
             block_scan<NT>(e, sh->warp_tmp, &eq_before);
-        } else if (C > 1) {
-            uint32_t *cnt = rs + kCnt;
-            if (threadIdx.x == 0) {
-                uint32_t g = 0, e = 0;
-                for (int w = 0; w < NT / 32; ++w) {
-                    g += sh->warp_a[w];
-                    e += sh->warp_b[w];
-                }
-                cnt[2 * c] = g;
-                cnt[2 * c + 1] = e;
-            }
-            if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
-            uint32_t a = 0, e = 0;
-            for (int j = threadIdx.x; j < c; j += NT) {
-                a += __ldcg(cnt + 2 * j);
-                e += __ldcg(cnt + 2 * j + 1);
-            }
-            block_scan<NT>(a, sh->warp_tmp, &gt_before);
-            block_scan<NT>(e, sh->warp_tmp, &eq_before);
         }
+        const uint32_t out_pos = gt_before + min(eq_before, ties);
 
         // ---- emission
-        emit_slice<NT>(sh, len, lo, key_at, Tstar, ties, eq_before, gt_before + min(eq_before, ties), out, K);
+        if (cand_ok && use_list) {
+            // from the candidates: per-warp counts at T*, then ordered compaction
+            const uint32_t wc = sh->warp_a[warp];
+            uint32_t g = 0, e = 0;
+            for (uint32_t i = lane; i < wc; i += 32) {
+                g += wkey[i] > Tstar;
+                e += wkey[i] == Tstar;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                g += __shfl_xor_sync(0xffffffffu, g, o);
+                e += __shfl_xor_sync(0xffffffffu, e, o);
+            }
+            if (lane == 0) {
+                sh->warp_b[warp] = g;
+                sh->warp_c[warp] = e;
+            }
+            __syncthreads();
+            uint32_t eq_seen = eq_before + warp_sum_prefix(sh->warp_c, warp);
+            const uint32_t cta_eq = eq_before < ties ? eq_before : ties;
+            uint32_t o = out_pos + warp_sum_prefix(sh->warp_b, warp) + ((eq_seen < ties ? eq_seen : ties) - cta_eq);
+            if (g || (e && eq_seen < ties)) {
+                for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
+                    const uint32_t i = i0 + lane;
+                    const uint32_t k = i < wc ? wkey[i] : 0u;
+                    const bool is_eq = i < wc && k == Tstar;
+                    const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
+                    const bool sel = (i < wc && k > Tstar) || (is_eq && eq_seen + __popc(em & lt) < ties);
+                    const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+                    if (sel) {
+                        const uint32_t at = o + __popc(sm & lt);
+                        if (at < (uint32_t)K) out[at] = (int32_t)wpos[i];
+                    }
+                    o += __popc(sm);
+                    eq_seen += __popc(em);
+                }
+            }
+        } else {
+            warp_counts<NT>(sh, len, cached, cache, key_at, Tstar, Tstar);
+            if (!use_list && C > 1) {   // exchange the per-CTA (greater, equal) counts at T*
+                uint32_t *cnt = rs + kCnt;
+                if (threadIdx.x == 0) {
+                    uint32_t g = 0, e = 0;
+                    for (int w = 0; w < NW; ++w) {
+                        g += sh->warp_a[w];
+                        e += sh->warp_b[w];
+                    }
+                    cnt[2 * c] = g;
+                    cnt[2 * c + 1] = e;
+                }
+                if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
+                uint32_t a = 0, e = 0;
+                for (int j = threadIdx.x; j < c; j += NT) {
+                    a += __ldcg(cnt + 2 * j);
+                    e += __ldcg(cnt + 2 * j + 1);
+                }
+                block_scan<NT>(a, sh->warp_tmp, &gt_before);
+                block_scan<NT>(e, sh->warp_tmp, &eq_before);
+            }
+            emit_slice<NT>(sh, len, lo, cached, cache, key_at, Tstar, ties, eq_before, gt_before + min(eq_before, ties), out, K);
+        }
         if (c == 0 && threadIdx.x == 0) p.count[row] = K;
     } else if (c == 0) {
         for (int j = threadIdx.x; j < K; j += NT) out[j] = -1;
@@ -514,6 +688,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     }
 
     // ---- the last CTA of the row to leave clears the row's words for the next call
+    if (defer_clear) return;
     __syncthreads();
     if (C > 1) {
         if (threadIdx.x == 0) {
@@ -534,11 +709,36 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 ctl[0] = 0;
                 ctl[1] = 0;
                 ctl[2] = 0;
+                ctl[3] = 0;
             }
         }
     } else if (hist1_ready) {
         for (int j = threadIdx.x; j < kHist2; j += NT) rs[j] = 0;
     }
+}
+
+// CTA c's share of clearing row `row`'s scratch for the next call, once no
+// CTA of the row reads it any more: the digit histograms, the counts and the
+// list entries used.  The control words stay for reset_row_ctl.
+// Threads tid < nt of the CTA take part.
+__device__ __forceinline__ void clear_row_share(const Params &p, int row, int c, int C, int tid, int nt) {
+    uint32_t *rs = p.scratch + (int64_t)row * p.scratch_row_words;
+    const int words = C > 1 ? ctl_base(C) : kHist2;
+    for (int j = c * nt + tid; j < words; j += C * nt) rs[j] = 0;
+    if (C > 1) {
+        const uint32_t m = __ldcg(rs + ctl_base(C) + 2);
+        const uint32_t used = m < (uint32_t)p.list_cap ? m : (uint32_t)p.list_cap;
+        uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+        for (uint32_t j = c * nt + tid; j < used; j += C * nt) {
+            gkey[j] = 0;
+            gpos[j] = 0;
+        }
+    }
+}
+
+// Resets row `row`'s control words, once every CTA of the row has read them.
+__device__ __forceinline__ void reset_row_ctl(const Params &p, int row, int C) {
+    if (C > 1 && threadIdx.x < 4) p.scratch[(int64_t)row * p.scratch_row_words + ctl_base(C) + threadIdx.x] = 0;
 }
 
 }  // namespace topk
