@@ -39,7 +39,7 @@ TOP_K = 2048
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "local_attention_decode_b200", "csrc")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_ctx_1m.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_ctx_1m.txt")
 FUSED_MAX_ROWS = 16   # dsa_layer_decode runs as one fused kernel for B * T <= 16
 
 
