@@ -80,7 +80,8 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     // the dynamic buffer is aligned by hand (its 1 KB slack is part of the budget), so the
     // static shared memory of this kernel stays a few bytes
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by an offset from the array itself, so the compiler keeps the shared address space
+    uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     __shared__ uint32_t sync_flag;
     const uint32_t G = gridDim.x;
     uint32_t *status = fp.ix.status;
@@ -95,7 +96,9 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(smem);
         uint32_t *cache = reinterpret_cast<uint32_t *>(smem + smem_align(sizeof(topk::Shared<kThreads>)));
         const int row = blockIdx.x / fp.C, c = blockIdx.x % fp.C;
-        topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, fp.hist_ready != 0, true);
+        bool done = false;
+        if (fp.hist_ready && fp.C > 1) done = topk::select_row_hist<kThreads>(fp.tk, sh, cache, row, c, fp.C);
+        if (!done) topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, fp.hist_ready != 0, true);
     }
     if (!grid_sync(fp.grid_bar, 2 * G, status, &sync_flag)) return;
 
@@ -226,13 +229,13 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     {   // shared memory after the fixed part: the CTA's slice of keys, then the candidate list
         const int64_t avail = (int64_t)(smem - 1024 - top_fixed) / 4;
         const int64_t chunk = ((ia.Lmax + plan.C - 1) / plan.C + 3) & ~int64_t(3);
-        const int64_t list = std::min<int64_t>(topk::kSmemList, avail / 8);
-        int64_t cand = std::min<int64_t>(topk::kCandCap, std::max<int64_t>(0, (avail - chunk) / 2 - list));
-        if (cand < 1024) cand = std::min<int64_t>(topk::kCandCap, (avail - 2 * list) / 4);   // slices too long to cache
-        cand = std::max<int64_t>(0, cand) / kWarps * kWarps;
+        const int64_t cand = std::min<int64_t>(topk::kCandCap, avail / 4) / kWarps * kWarps;
+        const int64_t rest = avail - 2 * cand;
+        int64_t list = std::min<int64_t>(topk::kListCap, std::max<int64_t>(0, (rest - chunk) / 2));
+        if (list < 1024) list = std::min<int64_t>(topk::kListCap, rest / 4);   // slices too long to cache
         tp.smem_list = (int)list;
         tp.cand_cap = (int)cand;
-        tp.cache_keys = (int)(avail - 2 * list - 2 * cand);
+        tp.cache_keys = (int)(rest - 2 * list);
     }
     tp.list_cap = topk::kListCap;
     tp.Lmax = ia.Lmax;

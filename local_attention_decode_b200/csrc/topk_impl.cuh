@@ -53,11 +53,13 @@ constexpr int kCandCap = 8192;              // per-warp candidates a CTA keeps i
 //   [kCnt, +2C)      per-CTA (greater, equal) counts at T* (exchange path)
 //   [kCnt+2C, +C)    per-CTA counts of keys above the 22-bit threshold bin
 //   ctl_base(C):     [0] barrier arrivals, [1] CTAs done, [2] list length,
-//                    [3] a CTA's candidates overflowed its shared memory
+//                    [3] a CTA's candidates overflowed its shared memory,
+//                    [4] list length of the one-barrier path (select_row_hist)
 //   list_base(C):    list_cap keys, then list_cap positions
 constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kCnt = 5120;
 __host__ __device__ constexpr int ctl_base(int C) { return kCnt + 3 * C; }
-__host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + 4 + 3) & ~3; }
+constexpr int kCtlWords = 5;
+__host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + kCtlWords + 3) & ~3; }
 __host__ __device__ constexpr int scratch_words(int C, int list_cap) { return list_base(C) + 2 * list_cap; }
 
 struct Params {
@@ -94,7 +96,7 @@ struct alignas(16) Shared {
 // Inclusive block scan of one value per thread (all NT threads); returns the
 // inclusive prefix and writes the block total to *total.
 template <int NT>
-__device__ __noinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, uint32_t *total) {
+__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, uint32_t *total) {
     constexpr int NW = NT / 32;
     const int lane = lane_id(), warp = warp_id();
 #pragma unroll
@@ -126,7 +128,7 @@ __device__ __noinline__ uint32_t block_scan(uint32_t v, uint32_t *warp_tmp, uint
 // nbins is 1024 or 2048.  One warp searches: each lane sums a run of nbins / 32
 // bins, a suffix scan over the lanes finds the run, the warp then splits that run.
 template <int NT>
-__device__ __noinline__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
+__device__ __forceinline__ void find_threshold(Shared<NT> *sh, int nbins, uint32_t K) {
     if (warp_id() == 0) {
         const int lane = lane_id();
         const int per = nbins >> 5;
@@ -706,15 +708,214 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 gpos[j] = 0;
             }
             if (threadIdx.x == 0) {
-                ctl[0] = 0;
-                ctl[1] = 0;
-                ctl[2] = 0;
-                ctl[3] = 0;
+                for (int j = 0; j < kCtlWords; ++j) ctl[j] = 0;
             }
         }
     } else if (hist1_ready) {
         for (int j = threadIdx.x; j < kHist2; j += NT) rs[j] = 0;
     }
+}
+
+// One-barrier selection of row `row` by CTA c of C (C > 1), for a row whose
+// first-digit histogram is already complete in the row's global scratch.
+// Each thread holds up to kHistRegs keys of its warp's part of the slice in
+// registers.  With the threshold bin b1 of the top 11 bits known from the
+// histogram, every key at or above bin b1 (above(b1) + h[b1] keys in the row,
+// about 11.5K at 1M context) is appended with its position to the row's list;
+// after one barrier each CTA loads the whole list into shared memory and
+// resolves digits 2 and 3 on it, takes its output offset from the list
+// entries that lie before its slice, and emits its own candidates (kept per
+// warp, in position order, in shared memory).
+// Returns false, before touching anything shared, when the row does not
+// qualify (the same decision in every CTA of the row): the caller then runs
+// select_row.  `cache` is laid out as for select_row; p.cand_cap / (NT / 32)
+// must be at least kHistRegs * 32.
+constexpr int kHistRegs = 12;
+template <int NT>
+__device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache, int row, int c, int C) {
+    constexpr int NW = NT / 32;
+    const int K = p.K;
+    const int64_t n = (int64_t)__ldg(p.q_pos + row) + 1;
+    if (n > p.Lmax || n <= K) return false;
+    const int64_t chunk = ((n + C - 1) / C + 3) & ~int64_t(3);
+    if (chunk > (int64_t)kHistRegs * 32 * NW || p.cand_cap / NW < kHistRegs * 32) return false;
+    const int64_t lo = n < (int64_t)c * chunk ? n : (int64_t)c * chunk;
+    const int64_t hi = n < lo + chunk ? n : lo + chunk;
+    const int64_t len = hi - lo;
+    const int warp = warp_id(), lane = lane_id();
+    const uint32_t lt = (1u << lane) - 1u;
+    int32_t *out = p.idx + (int64_t)row * K;
+    const float *src = p.scores + (int64_t)row * p.stride;
+    uint32_t *rs = p.scratch + (int64_t)row * p.scratch_row_words;
+    uint32_t *ctl = rs + ctl_base(C);
+    uint32_t *lkey = cache + p.cache_keys, *lpos = lkey + p.smem_list;
+    const int seg = p.cand_cap / NW;
+    uint32_t *wkey = lpos + p.smem_list + warp * seg, *wpos = wkey + p.cand_cap;
+
+    // ---- the row's histogram and this thread's keys, all loads in flight together
+    int64_t wlo, whi;
+    warp_part<NT>(len, &wlo, &whi);
+    constexpr int kHistPer = (kBins + NT - 1) / NT;
+    uint32_t hv[kHistPer];
+#pragma unroll
+    for (int u = 0; u < kHistPer; ++u) {
+        const int j = u * NT + threadIdx.x;
+        hv[u] = j < kBins ? __ldcg(rs + kHist1 + j) : 0u;
+    }
+    float v[kHistRegs];
+#pragma unroll
+    for (int i = 0; i < kHistRegs; ++i) {
+        const int64_t j = wlo + i * 32 + lane;
+        v[i] = j < whi ? __ldcg(src + lo + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kHistPer; ++u) {
+        const int j = u * NT + threadIdx.x;
+        if (j < kBins) sh->hist[j] = hv[u];
+    }
+    __syncthreads();
+    find_threshold<NT>(sh, kBins, (uint32_t)K);
+    const uint32_t b1 = (uint32_t)sh->bin;
+    const uint32_t m = sh->above + sh->hist[b1];   // keys at or above bin b1 in the row
+    if (sh->total != (uint32_t)n || m > (uint32_t)p.smem_list || m > (uint32_t)p.list_cap) return false;
+    uint32_t prefix = b1 << 21, mask = 0xFFE00000u, Krem = (uint32_t)K - sh->above;
+    __syncthreads();
+
+    // ---- this warp's candidates, in position order, into its segment
+    uint32_t wc = 0;
+#pragma unroll
+    for (int i = 0; i < kHistRegs; ++i) {
+        const int64_t j = wlo + i * 32 + lane;
+        const uint32_t k = float_order_key(v[i]);
+        const bool cand = j < whi && k >= prefix;
+        const uint32_t cm = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+            const uint32_t slot = wc + __popc(cm & lt);
+            wkey[slot] = k;
+            wpos[slot] = (uint32_t)(lo + j);
+        }
+        wc += __popc(cm);
+    }
+    if (lane == 0) sh->warp_a[warp] = wc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t tot = 0;
+        for (int w = 0; w < NW; ++w) tot += sh->warp_a[w];
+        sh->base = tot ? atomicAdd(ctl + 4, tot) : 0u;
+    }
+    __syncthreads();
+    {   // append them to the row's list
+        const uint32_t at = sh->base + warp_sum_prefix(sh->warp_a, warp);
+        uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+        for (uint32_t i = lane; i < wc; i += 32) {
+            if (at + i < (uint32_t)p.list_cap) {
+                gkey[at + i] = wkey[i];
+                gpos[at + i] = wpos[i];
+            }
+        }
+    }
+    if (!row_barrier<NT>(sh, ctl, (uint32_t)C, p.status)) return true;
+
+    // ---- the whole list into shared memory
+    {
+        const uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+        for (uint32_t base = 0; base < m; base += 4 * NT) {
+            uint32_t kv[4], pv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t j = base + u * NT + threadIdx.x;
+                kv[u] = j < m ? __ldcg(gkey + j) : 0u;
+                pv[u] = j < m ? __ldcg(gpos + j) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t j = base + u * NT + threadIdx.x;
+                if (j < m) {
+                    lkey[j] = kv[u];
+                    lpos[j] = pv[u];
+                }
+            }
+        }
+    }
+    // ---- digits 2 and 3 on the list
+#pragma unroll 1
+    for (int r = 0; r < 2; ++r) {
+        const int shift = r == 0 ? 10 : 0, nb = r == 0 ? kBins : 1024;
+        for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+        __syncthreads();
+        for (uint32_t base = threadIdx.x; base < m; base += 4 * NT) {   // four loads in flight
+            uint32_t k4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) k4[u] = base + u * NT < m ? lkey[base + u * NT] : ~prefix;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if ((k4[u] & mask) == prefix) atomicAdd(&sh->hist[(k4[u] >> shift) & (uint32_t)(nb - 1)], 1u);
+        }
+        __syncthreads();
+        find_threshold<NT>(sh, nb, Krem);
+        prefix |= (uint32_t)sh->bin << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
+        Krem -= sh->above;
+        __syncthreads();
+    }
+    const uint32_t Tstar = prefix, ties = Krem;
+
+    // ---- offset: list entries before this slice (greater in the high half, equal in the low)
+    uint32_t ge = 0;
+    for (uint32_t base = threadIdx.x; base < m; base += 4 * NT) {   // four entries in flight
+        uint32_t k4[4], p4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool in = base + u * NT < m;
+            k4[u] = in ? lkey[base + u * NT] : 0u;
+            p4[u] = in ? lpos[base + u * NT] : 0xFFFFFFFFu;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if ((int64_t)p4[u] < lo) ge += k4[u] > Tstar ? 0x10000u : (k4[u] == Tstar ? 1u : 0u);
+    }
+    uint32_t before;
+    block_scan<NT>(ge, sh->warp_tmp, &before);
+    const uint32_t gt_before = before >> 16, eq_before = before & 0xFFFFu;
+    const uint32_t out_pos = gt_before + (eq_before < ties ? eq_before : ties);
+
+    // ---- emission of this CTA's candidates
+    uint32_t g = 0, e = 0;
+    for (uint32_t i = lane; i < wc; i += 32) {
+        g += wkey[i] > Tstar;
+        e += wkey[i] == Tstar;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
+    if (lane == 0) {
+        sh->warp_b[warp] = g;
+        sh->warp_c[warp] = e;
+    }
+    __syncthreads();
+    uint32_t eq_seen = eq_before + warp_sum_prefix(sh->warp_c, warp);
+    const uint32_t cta_eq = eq_before < ties ? eq_before : ties;
+    uint32_t o = out_pos + warp_sum_prefix(sh->warp_b, warp) + ((eq_seen < ties ? eq_seen : ties) - cta_eq);
+    if (g || (e && eq_seen < ties)) {
+        for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
+            const uint32_t i = i0 + lane;
+            const uint32_t k = i < wc ? wkey[i] : 0u;
+            const bool is_eq = i < wc && k == Tstar;
+            const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
+            const bool sel = (i < wc && k > Tstar) || (is_eq && eq_seen + __popc(em & lt) < ties);
+            const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+                const uint32_t at = o + __popc(sm & lt);
+                if (at < (uint32_t)K) out[at] = (int32_t)wpos[i];
+            }
+            o += __popc(sm);
+            eq_seen += __popc(em);
+        }
+    }
+    if (c == 0 && threadIdx.x == 0) p.count[row] = K;
+    return true;
 }
 
 // CTA c's share of clearing row `row`'s scratch for the next call, once no
@@ -726,7 +927,8 @@ __device__ __forceinline__ void clear_row_share(const Params &p, int row, int c,
     const int words = C > 1 ? ctl_base(C) : kHist2;
     for (int j = c * nt + tid; j < words; j += C * nt) rs[j] = 0;
     if (C > 1) {
-        const uint32_t m = __ldcg(rs + ctl_base(C) + 2);
+        const uint32_t m2 = __ldcg(rs + ctl_base(C) + 2), m4 = __ldcg(rs + ctl_base(C) + 4);
+        const uint32_t m = m2 > m4 ? m2 : m4;
         const uint32_t used = m < (uint32_t)p.list_cap ? m : (uint32_t)p.list_cap;
         uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
         for (uint32_t j = c * nt + tid; j < used; j += C * nt) {
@@ -738,7 +940,7 @@ __device__ __forceinline__ void clear_row_share(const Params &p, int row, int c,
 
 // Resets row `row`'s control words, once every CTA of the row has read them.
 __device__ __forceinline__ void reset_row_ctl(const Params &p, int row, int C) {
-    if (C > 1 && threadIdx.x < 4) p.scratch[(int64_t)row * p.scratch_row_words + ctl_base(C) + threadIdx.x] = 0;
+    if (C > 1 && threadIdx.x < kCtlWords) p.scratch[(int64_t)row * p.scratch_row_words + ctl_base(C) + threadIdx.x] = 0;
 }
 
 }  // namespace topk
