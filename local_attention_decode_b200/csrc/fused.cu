@@ -98,7 +98,7 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         const int row = blockIdx.x / fp.C, c = blockIdx.x % fp.C;
         bool done = false;
         if (fp.hist_ready && fp.C > 1) done = topk::select_row_hist<kThreads>(fp.tk, sh, cache, row, c, fp.C);
-        if (!done) topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, fp.hist_ready != 0, true);
+        if (!done) topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, true);
     }
     if (!grid_sync(fp.grid_bar, 2 * G, status, &sync_flag)) return;
 
@@ -190,7 +190,7 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     // indexer phase, with the first histogram when the rows' histograms fit
     IndexerLaunch L;
     int hist_rows = plan.rows <= kMaxHistRows ? plan.rows : 0;
-    int rc = prepare_indexer(ia, hist_rows, row_words, row_scratch + topk::kHist1, budget, &L);
+    int rc = prepare_indexer(ia, hist_rows, row_words, row_scratch + topk::kHistI, budget, &L);
     if (rc == DSA_OK && hist_rows && L.p.stages < 3) hist_rows = 0;   // keep the stream at least 3 stages deep
     if (rc != DSA_OK || hist_rows == 0) {
         hist_rows = 0;

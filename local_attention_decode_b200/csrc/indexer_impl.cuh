@@ -25,7 +25,7 @@
 //                 accumulator and every GE-th tile of the pipeline:
 //                 tcgen05.ld of one key row per thread, ReLU, per-head
 //                 weighting, key scale, causal mask, coalesced fp32 store,
-//                 optionally the first-digit histogram of the selection.
+//                 optionally a histogram of the scores for the selection.
 #pragma once
 
 #include "common.cuh"
@@ -42,7 +42,11 @@ constexpr int kEpiWarp0 = 2 * kPipes;     // first epilogue warp
 constexpr int kThreads = 32 * (kEpiWarp0 + kPipes * kMaxGroups * kEpiWarps);   // 640
 constexpr int kMaxStages = 8;             // per pipeline
 constexpr int kKsStageBytes = 1024;       // key-scale slots of one stage
-constexpr int kHistBins = 2048;           // first radix digit of the selection (11 bits)
+// Score histogram for the selection: bits 30..20 of the order key of each
+// non-negative score (2048 bins, eight per octave), and one bin (2048) that
+// counts the negative scores; kHistWords words per row.
+constexpr int kHistBins = 2048;
+constexpr int kHistWords = 2052;
 
 // Byte offset, inside a stage's key-scale area, of the scale of tile row r.
 __host__ __device__ __forceinline__ int ks_slot_offset(int r, int R) {
@@ -67,9 +71,9 @@ struct Params {
     int stages;          // per pipeline
     int rows_per_load;   // R: rows per TMA box (128, or the page size when pages are smaller)
     int groups;          // epilogue groups per pipeline (1..kMaxGroups)
-    // optional first-digit histogram of the visible scores (top 11 bits of
-    // the order key), added into hist_global[row * hist_row_words + bin] for
-    // rows b * T + t < hist_rows; hist_rows == 0 turns it off
+    // optional histogram of the visible scores (see kHistWords), added into
+    // hist_global[row * hist_row_words + bin] for rows b * T + t < hist_rows;
+    // hist_rows == 0 turns it off
     int hist_rows;
     int hist_row_words;
     uint32_t *hist_global;
@@ -110,7 +114,7 @@ struct Layout {
         epi_off = (epi_off + 15) & ~15u;
         // per epilogue warp: 16*T coefficients + T positions
         hist_off = epi_off + kPipes * kMaxGroups * kEpiWarps * (16 * T + T) * 4;
-        total = hist_off + hist_rows * kHistBins * 4;
+        total = hist_off + hist_rows * kHistWords * 4;
     }
 };
 
@@ -177,7 +181,7 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
         if (lane == 0) tile_pre[0] = 0;
     }
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [hist_rows][2048] or empty
-    for (int j = threadIdx.x; j < p.hist_rows * kHistBins; j += blockDim.x) hist[j] = 0;
+    for (int j = threadIdx.x; j < p.hist_rows * kHistWords; j += blockDim.x) hist[j] = 0;
     __syncthreads();
 
     const int total = tile_pre[B];
@@ -347,8 +351,11 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
                 for (int h = 0; h < 16; ++h) sum = fmaf(coef[16 * t + h], fmaxf(acc[h], 0.f), sum);
                 const bool visible = pos < len && pos <= qp[t];
                 if (pos < len) out[(int64_t)t * p.scores_stride] = visible ? ks * sum : -INFINITY;
-                if (p.hist_rows)   // first-digit histogram of the visible scores
-                    warp_hist_add(hist, (b * T + t) * kHistBins + (float_order_key(ks * sum) >> 21), visible);
+                if (p.hist_rows) {   // histogram of the visible scores
+                    const uint32_t key = float_order_key(ks * sum);
+                    const uint32_t bin = (key >> 31) ? ((key >> 20) & (kHistBins - 1)) : (uint32_t)kHistBins;
+                    warp_hist_add(hist, (b * T + t) * kHistWords + bin, visible);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -381,8 +388,8 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
         mbar_inval(&bars->q_full);
     }
     // add this CTA's histogram into the rows' global histograms
-    for (int j = threadIdx.x; j < p.hist_rows * kHistBins; j += blockDim.x)
-        if (hist[j]) atomicAdd(p.hist_global + (int64_t)(j / kHistBins) * p.hist_row_words + (j % kHistBins), hist[j]);
+    for (int j = threadIdx.x; j < p.hist_rows * kHistWords; j += blockDim.x)
+        if (hist[j]) atomicAdd(p.hist_global + (int64_t)(j / kHistWords) * p.hist_row_words + (j % kHistWords), hist[j]);
     __syncthreads();
 }
 

@@ -17,7 +17,7 @@ topk_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Shared<kThreads> *sh = reinterpret_cast<Shared<kThreads> *>(smem_raw);
     uint32_t *cache = reinterpret_cast<uint32_t *>(smem_raw + sizeof(Shared<kThreads>));
-    select_row<kThreads>(p, sh, cache, blockIdx.x / p.C, blockIdx.x % p.C, p.C, false);
+    select_row<kThreads>(p, sh, cache, blockIdx.x / p.C, blockIdx.x % p.C, p.C);
 }
 
 }  // namespace topk

@@ -50,13 +50,15 @@ constexpr int kCandCap = 8192;              // per-warp candidates a CTA keeps i
 // Per-row scratch (u32 words), used when C > 1 or when the first histogram is
 // produced by the indexer:
 //   [kHist1, +2048) [kHist2, +2048) [kHist3, +1024)  digit histograms
+//   [kHistI, +2052)  the histogram built by the indexer: bits 30..20 of the
+//                    non-negative keys (2048 bins) and the count of negative keys
 //   [kCnt, +2C)      per-CTA (greater, equal) counts at T* (exchange path)
 //   [kCnt+2C, +C)    per-CTA counts of keys above the 22-bit threshold bin
 //   ctl_base(C):     [0] barrier arrivals, [1] CTAs done, [2] list length,
 //                    [3] a CTA's candidates overflowed its shared memory,
 //                    [4] list length of the one-barrier path (select_row_hist)
 //   list_base(C):    list_cap keys, then list_cap positions
-constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kCnt = 5120;
+constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kHistI = 5120, kCnt = 5120 + 2052;
 __host__ __device__ constexpr int ctl_base(int C) { return kCnt + 3 * C; }
 constexpr int kCtlWords = 5;
 __host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + kCtlWords + 3) & ~3; }
@@ -330,13 +332,12 @@ __device__ __forceinline__ void emit_slice(Shared<NT> *sh, int64_t len, int64_t 
 
 // Selection of row `row` by CTA c of the C CTAs that share it.  All NT
 // threads of the CTA call this.  `cache` holds p.cache_keys keys, then
-// 2 * p.smem_list list words, then 2 * p.cand_cap candidate words.  hist1_ready: the row's first-digit histogram is
-// already complete in the row's global scratch (built by the producer of the
-// scores).  defer_clear: leave the row's scratch words for clear_row_share
-// and reset_row_ctl (called once every CTA of the row is past the selection).
+// 2 * p.smem_list list words, then 2 * p.cand_cap candidate words.
+// defer_clear: leave the row's scratch words for clear_row_share and
+// reset_row_ctl (called once every CTA of the row is past the selection).
 template <int NT>
 __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int row, int c, int C,
-                           bool hist1_ready, bool defer_clear = false) {
+                           bool defer_clear = false) {
     const int K = p.K;
     int64_t n = (int64_t)__ldg(p.q_pos + row) + 1;
     if (n > p.Lmax) {   // a position beyond the scores buffer: flag it, select within the buffer
@@ -345,17 +346,13 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     }
     int32_t *out = p.idx + (int64_t)row * K;
     const float *src = p.scores + (int64_t)row * p.stride;
-    uint32_t *rs = (C > 1 || hist1_ready) ? p.scratch + (int64_t)row * p.scratch_row_words : nullptr;
+    uint32_t *rs = C > 1 ? p.scratch + (int64_t)row * p.scratch_row_words : nullptr;
     uint32_t *ctl = rs ? rs + ctl_base(C) : nullptr;
 
     if (n <= K) {   // every visible position is selected (same decision in all CTAs of the row)
         if (c == 0) {
             for (int j = threadIdx.x; j < K; j += NT) out[j] = j < n ? j : -1;
             if (threadIdx.x == 0) p.count[row] = (int32_t)(n > 0 ? n : 0);
-        }
-        if (hist1_ready && !defer_clear) {   // the producer's histogram is not needed: clear this CTA's share
-            __syncthreads();
-            for (int j = c * NT + threadIdx.x; j < kHist2; j += C * NT) rs[j] = 0;
         }
         return;
     }
@@ -374,16 +371,6 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
 
     // scores may have been written earlier in the same kernel: read them through L2 (no .nc loads)
     auto key_at = [&](int64_t j) -> uint32_t { return cached ? cache[j] : float_order_key(__ldcg(src + lo + j)); };
-    // the producer's histogram is fetched while the slice streams in
-    constexpr int kHistPer = (kBins + NT - 1) / NT;
-    uint32_t hv[kHistPer];
-    if (hist1_ready) {
-#pragma unroll
-        for (int u = 0; u < kHistPer; ++u) {
-            const int j = u * NT + threadIdx.x;
-            hv[u] = j < kBins ? __ldcg(rs + kHist1 + j) : 0u;
-        }
-    }
     if (cached) {
         for (int64_t base = 0; base < len; base += (int64_t)kUnroll * NT) {
             float v[kUnroll];
@@ -397,13 +384,6 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 const int64_t j = base + u * NT + threadIdx.x;
                 if (j < len) cache[j] = float_order_key(v[u]);
             }
-        }
-    }
-    if (hist1_ready) {
-#pragma unroll
-        for (int u = 0; u < kHistPer; ++u) {
-            const int j = u * NT + threadIdx.x;
-            if (j < kBins) sh->hist[j] = hv[u];
         }
     }
     __syncthreads();
@@ -439,14 +419,9 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     };
 
     // ---- digit 1
-    if (!hist1_ready) {
-        slice_hist(0u, 0u, 21, kBins);
-        if (C > 1 && !exchange_hist(rs + kHist1, kBins)) return;
-    }
+    slice_hist(0u, 0u, 21, kBins);
+    if (C > 1 && !exchange_hist(rs + kHist1, kBins)) return;
     find_threshold<NT>(sh, kBins, (uint32_t)K);
-    // a histogram that does not count this row's n scores (a position the
-    // producer rejected): select nothing
-    const bool empty = hist1_ready && sh->total != (uint32_t)n;
     uint32_t prefix = (uint32_t)sh->bin << 21, mask = 0xFFE00000u, Krem = (uint32_t)K - sh->above;
     __syncthreads();
     // Narrows (prefix, mask, Krem) by the nb-bin digit at `shift`, from sh->hist.
@@ -460,37 +435,35 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
 
     // ---- digit 2, over the whole row; in the same pass each warp keeps, in
     //      position order, its candidates: the keys at or above the threshold bin
-    if (!empty) {
-        for (int j = threadIdx.x; j < kBins; j += NT) sh->hist[j] = 0;
-        __syncthreads();
-        int64_t wlo, whi;
-        warp_part<NT>(len, &wlo, &whi);
-        uint32_t wc = 0;
-        warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
-            if (valid && (k & mask) == prefix) atomicAdd(&sh->hist[(k >> 10) & (kBins - 1)], 1u);
-            const bool cand = valid && k >= prefix;
-            const uint32_t cm = __ballot_sync(0xffffffffu, cand);
-            if (cand) {
-                const uint32_t slot = wc + __popc(cm & lt);
-                if (slot < (uint32_t)seg) {
-                    wkey[slot] = k;
-                    wpos[slot] = (uint32_t)(lo + j);
-                }
+    for (int j = threadIdx.x; j < kBins; j += NT) sh->hist[j] = 0;
+    __syncthreads();
+    int64_t wlo, whi;
+    warp_part<NT>(len, &wlo, &whi);
+    uint32_t wc = 0;
+    warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
+        if (valid && (k & mask) == prefix) atomicAdd(&sh->hist[(k >> 10) & (kBins - 1)], 1u);
+        const bool cand = valid && k >= prefix;
+        const uint32_t cm = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+            const uint32_t slot = wc + __popc(cm & lt);
+            if (slot < (uint32_t)seg) {
+                wkey[slot] = k;
+                wpos[slot] = (uint32_t)(lo + j);
             }
-            wc += __popc(cm);
-        });
-        if (lane == 0) sh->warp_a[warp] = wc;
-        __syncthreads();
-        if (C > 1 && threadIdx.x == 0) {
-            bool over = false;
-            for (int w = 0; w < NW; ++w) over |= sh->warp_a[w] > (uint32_t)seg;
-            if (over) atomicOr(ctl + 3, 1u);
         }
-        if (C > 1 && !exchange_hist(rs + kHist2, kBins)) return;
-        take_digit(kBins, 10);
+        wc += __popc(cm);
+    });
+    if (lane == 0) sh->warp_a[warp] = wc;
+    __syncthreads();
+    if (C > 1 && threadIdx.x == 0) {
+        bool over = false;
+        for (int w = 0; w < NW; ++w) over |= sh->warp_a[w] > (uint32_t)seg;
+        if (over) atomicOr(ctl + 3, 1u);
     }
+    if (C > 1 && !exchange_hist(rs + kHist2, kBins)) return;
+    take_digit(kBins, 10);
     // every CTA's candidates fit: (read after the exchange, the same in every CTA)
-    const bool cand_ok = C > 1 && !empty && seg > 0 && __ldcg(ctl + 3) == 0u;
+    const bool cand_ok = C > 1 && seg > 0 && __ldcg(ctl + 3) == 0u;
 
     // ---- the candidate list: every key of the row whose top 22 bits are the
     //      threshold's, with its position; each CTA publishes its count of keys
@@ -498,73 +471,71 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     bool use_list = false;
     uint32_t m = 0;
     if (C > 1) {
-        if (!empty) {
-            const uint32_t hi22 = prefix | ~mask;
-            uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+        const uint32_t hi22 = prefix | ~mask;
+        uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
+        if (cand_ok) {
+            const uint32_t wc = sh->warp_a[warp];
+            uint32_t a = 0, e = 0;
+            for (uint32_t i = lane; i < wc; i += 32) {
+                a += wkey[i] > hi22;
+                e += (wkey[i] & mask) == prefix;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, o);
+                e += __shfl_xor_sync(0xffffffffu, e, o);
+            }
+            if (lane == 0) {
+                sh->warp_c[warp] = a;
+                sh->warp_b[warp] = e;
+            }
+        } else {
+            warp_counts<NT>(sh, len, cached, cache, key_at, prefix, hi22);   // above into warp_a, in-bin into warp_b
+            if (lane == 0) sh->warp_c[warp] = sh->warp_a[warp];
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t above = 0, mine = 0;
+            for (int w = 0; w < NW; ++w) {
+                above += sh->warp_c[w];
+                mine += sh->warp_b[w];
+            }
+            rs[kCnt + 2 * C + c] = above;
+            sh->base = mine ? atomicAdd(ctl + 2, mine) : 0u;
+        }
+        __syncthreads();
+        if (sh->warp_b[warp]) {   // append this warp's keys of the 22-bit bin
+            uint32_t at = sh->base + warp_sum_prefix(sh->warp_b, warp);
+            auto put = [&](bool in, uint32_t k, uint32_t pos) {
+                const uint32_t bm = __ballot_sync(0xffffffffu, in);
+                if (in) {
+                    const uint32_t slot = at + __popc(bm & lt);
+                    if (slot < (uint32_t)p.list_cap) {
+                        gkey[slot] = k;
+                        gpos[slot] = pos;
+                    }
+                }
+                at += __popc(bm);
+            };
             if (cand_ok) {
                 const uint32_t wc = sh->warp_a[warp];
-                uint32_t a = 0, e = 0;
-                for (uint32_t i = lane; i < wc; i += 32) {
-                    a += wkey[i] > hi22;
-                    e += (wkey[i] & mask) == prefix;
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    a += __shfl_xor_sync(0xffffffffu, a, o);
-                    e += __shfl_xor_sync(0xffffffffu, e, o);
-                }
-                if (lane == 0) {
-                    sh->warp_c[warp] = a;
-                    sh->warp_b[warp] = e;
+                for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
+                    const uint32_t i = i0 + lane;
+                    const uint32_t k = i < wc ? wkey[i] : 0u;
+                    put(i < wc && (k & mask) == prefix, k, i < wc ? wpos[i] : 0u);
                 }
             } else {
-                warp_counts<NT>(sh, len, cached, cache, key_at, prefix, hi22);   // above into warp_a, in-bin into warp_b
-                if (lane == 0) sh->warp_c[warp] = sh->warp_a[warp];
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                uint32_t above = 0, mine = 0;
-                for (int w = 0; w < NW; ++w) {
-                    above += sh->warp_c[w];
-                    mine += sh->warp_b[w];
-                }
-                rs[kCnt + 2 * C + c] = above;
-                sh->base = mine ? atomicAdd(ctl + 2, mine) : 0u;
-            }
-            __syncthreads();
-            if (sh->warp_b[warp]) {   // append this warp's keys of the 22-bit bin
-                uint32_t at = sh->base + warp_sum_prefix(sh->warp_b, warp);
-                auto put = [&](bool in, uint32_t k, uint32_t pos) {
-                    const uint32_t bm = __ballot_sync(0xffffffffu, in);
-                    if (in) {
-                        const uint32_t slot = at + __popc(bm & lt);
-                        if (slot < (uint32_t)p.list_cap) {
-                            gkey[slot] = k;
-                            gpos[slot] = pos;
-                        }
-                    }
-                    at += __popc(bm);
-                };
-                if (cand_ok) {
-                    const uint32_t wc = sh->warp_a[warp];
-                    for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
-                        const uint32_t i = i0 + lane;
-                        const uint32_t k = i < wc ? wkey[i] : 0u;
-                        put(i < wc && (k & mask) == prefix, k, i < wc ? wpos[i] : 0u);
-                    }
-                } else {
-                    int64_t wlo, whi;
-                    warp_part<NT>(len, &wlo, &whi);
-                    warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
-                        put(valid && (k & mask) == prefix, k, (uint32_t)(lo + j));
-                    });
-                }
+                int64_t wlo, whi;
+                warp_part<NT>(len, &wlo, &whi);
+                warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
+                    put(valid && (k & mask) == prefix, k, (uint32_t)(lo + j));
+                });
             }
         }
         if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
         m = __ldcg(ctl + 2);
         use_list = m <= (uint32_t)p.smem_list;
-        if (use_list && !empty) {
+        if (use_list) {
             const uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
             for (uint32_t base = 0; base < m; base += 4 * NT) {
                 uint32_t kv[4], pv[4];
@@ -587,107 +558,102 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
         }
     }
 
-    if (!empty) {
-        // ---- digit 3: on the list, or over the row
-        if (use_list) {
-            for (int j = threadIdx.x; j < 1024; j += NT) sh->hist[j] = 0;
-            __syncthreads();
-            for (uint32_t j = threadIdx.x; j < m; j += NT) {
-                const uint32_t k = lkey[j];
-                if ((k & mask) == prefix) atomicAdd(&sh->hist[k & 1023u], 1u);
-            }
-            __syncthreads();
-        } else {
-            slice_hist(prefix, mask, 0, 1024);
-            if (C > 1 && !exchange_hist(rs + kHist3, 1024)) return;
+    // ---- digit 3: on the list, or over the row
+    if (use_list) {
+        for (int j = threadIdx.x; j < 1024; j += NT) sh->hist[j] = 0;
+        __syncthreads();
+        for (uint32_t j = threadIdx.x; j < m; j += NT) {
+            const uint32_t k = lkey[j];
+            if ((k & mask) == prefix) atomicAdd(&sh->hist[k & 1023u], 1u);
         }
-        take_digit(1024, 0);
-        const uint32_t Tstar = prefix;
-        const uint32_t ties = Krem;   // keys equal to T* that are taken (>= 1)
+        __syncthreads();
+    } else {
+        slice_hist(prefix, mask, 0, 1024);
+        if (C > 1 && !exchange_hist(rs + kHist3, 1024)) return;
+    }
+    take_digit(1024, 0);
+    const uint32_t Tstar = prefix;
+    const uint32_t ties = Krem;   // keys equal to T* that are taken (>= 1)
 
-        // ---- this CTA's offset in the row's output
-        uint32_t gt_before = 0, eq_before = 0;
-        if (use_list) {
-            // earlier CTAs: all their keys above the 22-bit bin, and their list entries > T* / == T*
-            uint32_t a = 0, e = 0;
-            for (int j = threadIdx.x; j < c; j += NT) a += __ldcg(rs + kCnt + 2 * C + j);
-            for (uint32_t j = threadIdx.x; j < m; j += NT)
-                if ((int64_t)lpos[j] < lo) {
-                    a += lkey[j] > Tstar;
-                    e += lkey[j] == Tstar;
+    // ---- this CTA's offset in the row's output
+    uint32_t gt_before = 0, eq_before = 0;
+    if (use_list) {
+        // earlier CTAs: all their keys above the 22-bit bin, and their list entries > T* / == T*
+        uint32_t a = 0, e = 0;
+        for (int j = threadIdx.x; j < c; j += NT) a += __ldcg(rs + kCnt + 2 * C + j);
+        for (uint32_t j = threadIdx.x; j < m; j += NT)
+            if ((int64_t)lpos[j] < lo) {
+                a += lkey[j] > Tstar;
+                e += lkey[j] == Tstar;
+            }
+        block_scan<NT>(a, sh->warp_tmp, &gt_before);
+        block_scan<NT>(e, sh->warp_tmp, &eq_before);
+    }
+    const uint32_t out_pos = gt_before + min(eq_before, ties);
+
+    // ---- emission
+    if (cand_ok && use_list) {
+        // from the candidates: per-warp counts at T*, then ordered compaction
+        const uint32_t wc = sh->warp_a[warp];
+        uint32_t g = 0, e = 0;
+        for (uint32_t i = lane; i < wc; i += 32) {
+            g += wkey[i] > Tstar;
+            e += wkey[i] == Tstar;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+        }
+        if (lane == 0) {
+            sh->warp_b[warp] = g;
+            sh->warp_c[warp] = e;
+        }
+        __syncthreads();
+        uint32_t eq_seen = eq_before + warp_sum_prefix(sh->warp_c, warp);
+        const uint32_t cta_eq = eq_before < ties ? eq_before : ties;
+        uint32_t o = out_pos + warp_sum_prefix(sh->warp_b, warp) + ((eq_seen < ties ? eq_seen : ties) - cta_eq);
+        if (g || (e && eq_seen < ties)) {
+            for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
+                const uint32_t i = i0 + lane;
+                const uint32_t k = i < wc ? wkey[i] : 0u;
+                const bool is_eq = i < wc && k == Tstar;
+                const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
+                const bool sel = (i < wc && k > Tstar) || (is_eq && eq_seen + __popc(em & lt) < ties);
+                const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+                if (sel) {
+                    const uint32_t at = o + __popc(sm & lt);
+                    if (at < (uint32_t)K) out[at] = (int32_t)wpos[i];
                 }
+                o += __popc(sm);
+                eq_seen += __popc(em);
+            }
+        }
+    } else {
+        warp_counts<NT>(sh, len, cached, cache, key_at, Tstar, Tstar);
+        if (!use_list && C > 1) {   // exchange the per-CTA (greater, equal) counts at T*
+            uint32_t *cnt = rs + kCnt;
+            if (threadIdx.x == 0) {
+                uint32_t g = 0, e = 0;
+                for (int w = 0; w < NW; ++w) {
+                    g += sh->warp_a[w];
+                    e += sh->warp_b[w];
+                }
+                cnt[2 * c] = g;
+                cnt[2 * c + 1] = e;
+            }
+            if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
+            uint32_t a = 0, e = 0;
+            for (int j = threadIdx.x; j < c; j += NT) {
+                a += __ldcg(cnt + 2 * j);
+                e += __ldcg(cnt + 2 * j + 1);
+            }
             block_scan<NT>(a, sh->warp_tmp, &gt_before);
             block_scan<NT>(e, sh->warp_tmp, &eq_before);
         }
-        const uint32_t out_pos = gt_before + min(eq_before, ties);
-
-        // ---- emission
-        if (cand_ok && use_list) {
-            // from the candidates: per-warp counts at T*, then ordered compaction
-            const uint32_t wc = sh->warp_a[warp];
-            uint32_t g = 0, e = 0;
-            for (uint32_t i = lane; i < wc; i += 32) {
-                g += wkey[i] > Tstar;
-                e += wkey[i] == Tstar;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                g += __shfl_xor_sync(0xffffffffu, g, o);
-                e += __shfl_xor_sync(0xffffffffu, e, o);
-            }
-            if (lane == 0) {
-                sh->warp_b[warp] = g;
-                sh->warp_c[warp] = e;
-            }
-            __syncthreads();
-            uint32_t eq_seen = eq_before + warp_sum_prefix(sh->warp_c, warp);
-            const uint32_t cta_eq = eq_before < ties ? eq_before : ties;
-            uint32_t o = out_pos + warp_sum_prefix(sh->warp_b, warp) + ((eq_seen < ties ? eq_seen : ties) - cta_eq);
-            if (g || (e && eq_seen < ties)) {
-                for (uint32_t i0 = 0; i0 < wc; i0 += 32) {
-                    const uint32_t i = i0 + lane;
-                    const uint32_t k = i < wc ? wkey[i] : 0u;
-                    const bool is_eq = i < wc && k == Tstar;
-                    const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
-                    const bool sel = (i < wc && k > Tstar) || (is_eq && eq_seen + __popc(em & lt) < ties);
-                    const uint32_t sm = __ballot_sync(0xffffffffu, sel);
-                    if (sel) {
-                        const uint32_t at = o + __popc(sm & lt);
-                        if (at < (uint32_t)K) out[at] = (int32_t)wpos[i];
-                    }
-                    o += __popc(sm);
-                    eq_seen += __popc(em);
-                }
-            }
-        } else {
-            warp_counts<NT>(sh, len, cached, cache, key_at, Tstar, Tstar);
-            if (!use_list && C > 1) {   // exchange the per-CTA (greater, equal) counts at T*
-                uint32_t *cnt = rs + kCnt;
-                if (threadIdx.x == 0) {
-                    uint32_t g = 0, e = 0;
-                    for (int w = 0; w < NW; ++w) {
-                        g += sh->warp_a[w];
-                        e += sh->warp_b[w];
-                    }
-                    cnt[2 * c] = g;
-                    cnt[2 * c + 1] = e;
-                }
-                if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
-                uint32_t a = 0, e = 0;
-                for (int j = threadIdx.x; j < c; j += NT) {
-                    a += __ldcg(cnt + 2 * j);
-                    e += __ldcg(cnt + 2 * j + 1);
-                }
-                block_scan<NT>(a, sh->warp_tmp, &gt_before);
-                block_scan<NT>(e, sh->warp_tmp, &eq_before);
-            }
-            emit_slice<NT>(sh, len, lo, cached, cache, key_at, Tstar, ties, eq_before, gt_before + min(eq_before, ties), out, K);
-        }
-        if (c == 0 && threadIdx.x == 0) p.count[row] = K;
-    } else if (c == 0) {
-        for (int j = threadIdx.x; j < K; j += NT) out[j] = -1;
-        if (threadIdx.x == 0) p.count[row] = 0;
+        emit_slice<NT>(sh, len, lo, cached, cache, key_at, Tstar, ties, eq_before, gt_before + min(eq_before, ties), out, K);
     }
+    if (c == 0 && threadIdx.x == 0) p.count[row] = K;
 
     // ---- the last CTA of the row to leave clears the row's words for the next call
     if (defer_clear) return;
@@ -711,25 +677,26 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 for (int j = 0; j < kCtlWords; ++j) ctl[j] = 0;
             }
         }
-    } else if (hist1_ready) {
-        for (int j = threadIdx.x; j < kHist2; j += NT) rs[j] = 0;
     }
 }
 
 // One-barrier selection of row `row` by CTA c of C (C > 1), for a row whose
-// first-digit histogram is already complete in the row's global scratch.
-// Each thread holds up to kHistRegs keys of its warp's part of the slice in
-// registers.  With the threshold bin b1 of the top 11 bits known from the
-// histogram, every key at or above bin b1 (above(b1) + h[b1] keys in the row,
-// about 11.5K at 1M context) is appended with its position to the row's list;
-// after one barrier each CTA loads the whole list into shared memory and
-// resolves digits 2 and 3 on it, takes its output offset from the list
-// entries that lie before its slice, and emits its own candidates (kept per
-// warp, in position order, in shared memory).
+// score histogram the indexer has already built in the row's scratch
+// (kHistI: bits 30..20 of the non-negative keys, eight bins per octave, and
+// the count of negative keys).  Each thread holds up to kHistRegs keys of its
+// warp's part of the slice in registers.  With the threshold bin b1 known from
+// the histogram, every key at or above it (above(b1) + h[b1] keys in the row)
+// is appended with its position to the row's list; after one barrier each CTA
+// loads the whole list into shared memory, resolves the remaining 20 bits
+// (two 10-bit digits) on it, takes its output offset from the list entries
+// that lie before its slice, and emits its own candidates (kept per warp, in
+// position order, in shared memory).
 // Returns false, before touching anything shared, when the row does not
-// qualify (the same decision in every CTA of the row): the caller then runs
-// select_row.  `cache` is laid out as for select_row; p.cand_cap / (NT / 32)
-// must be at least kHistRegs * 32.
+// qualify (the same decision in every CTA of the row): the threshold lies
+// among negative scores, the list would not fit, the slices are too long for
+// the registers, or the histogram does not count this row's scores.  The
+// caller then runs select_row.  `cache` is laid out as for select_row;
+// p.cand_cap / (NT / 32) must be at least kHistRegs * 32.
 constexpr int kHistRegs = 12;
 template <int NT>
 __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache, int row, int c, int C) {
@@ -760,8 +727,9 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
 #pragma unroll
     for (int u = 0; u < kHistPer; ++u) {
         const int j = u * NT + threadIdx.x;
-        hv[u] = j < kBins ? __ldcg(rs + kHist1 + j) : 0u;
+        hv[u] = j < kBins ? __ldcg(rs + kHistI + j) : 0u;
     }
+    const uint32_t negatives = __ldcg(rs + kHistI + kBins);
     float v[kHistRegs];
 #pragma unroll
     for (int i = 0; i < kHistRegs; ++i) {
@@ -777,8 +745,12 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
     find_threshold<NT>(sh, kBins, (uint32_t)K);
     const uint32_t b1 = (uint32_t)sh->bin;
     const uint32_t m = sh->above + sh->hist[b1];   // keys at or above bin b1 in the row
-    if (sh->total != (uint32_t)n || m > (uint32_t)p.smem_list || m > (uint32_t)p.list_cap) return false;
-    uint32_t prefix = b1 << 21, mask = 0xFFE00000u, Krem = (uint32_t)K - sh->above;
+    // the histogram must count exactly this row's n scores, and the threshold
+    // must lie among the non-negative ones
+    if (sh->total + negatives != (uint32_t)n || sh->total < (uint32_t)K || m > (uint32_t)p.smem_list ||
+        m > (uint32_t)p.list_cap)
+        return false;
+    uint32_t prefix = 0x80000000u | (b1 << 20), mask = 0xFFF00000u, Krem = (uint32_t)K - sh->above;
     __syncthreads();
 
     // ---- this warp's candidates, in position order, into its segment
@@ -840,7 +812,7 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
     // ---- digits 2 and 3 on the list
 #pragma unroll 1
     for (int r = 0; r < 2; ++r) {
-        const int shift = r == 0 ? 10 : 0, nb = r == 0 ? kBins : 1024;
+        const int shift = r == 0 ? 10 : 0, nb = 1024;
         for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
         __syncthreads();
         for (uint32_t base = threadIdx.x; base < m; base += 4 * NT) {   // four loads in flight
@@ -924,7 +896,7 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
 // Threads tid < nt of the CTA take part.
 __device__ __forceinline__ void clear_row_share(const Params &p, int row, int c, int C, int tid, int nt) {
     uint32_t *rs = p.scratch + (int64_t)row * p.scratch_row_words;
-    const int words = C > 1 ? ctl_base(C) : kHist2;
+    const int words = C > 1 ? ctl_base(C) : kCnt;
     for (int j = c * nt + tid; j < words; j += C * nt) rs[j] = 0;
     if (C > 1) {
         const uint32_t m2 = __ldcg(rs + ctl_base(C) + 2), m4 = __ldcg(rs + ctl_base(C) + 4);

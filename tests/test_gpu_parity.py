@@ -272,6 +272,31 @@ def test_layer_decode_equals_separate_calls(seq_lens, T, page_size):
     assert torch.equal(lse, lse2)
 
 
+@pytest.mark.parametrize("weights", ["negative", "mixed", "zero_query"])
+def test_layer_decode_selection_fallbacks(weights):
+    """Rows the fused kernel's one-barrier selection does not take (threshold
+    among negative scores; one histogram bin holding every score) go through
+    the general selection and still equal the separate calls and the oracle."""
+    wl = make_decode_workload(seed=81, seq_lens=[30000], T=2, device=DEV, n_needles=4)
+    g = torch.Generator(device=DEV).manual_seed(5)
+    if weights == "negative":
+        wl.w = -torch.rand(wl.w.shape, generator=g, device=DEV) / 16
+    elif weights == "mixed":
+        wl.w = (torch.rand(wl.w.shape, generator=g, device=DEV) - 0.5) / 8
+    else:   # every score 0: all tied, the lowest positions win
+        wl.q8 = torch.zeros_like(wl.q8)
+    O, lse, idx, cnt = run_layer(wl)
+    scores = run_indexer(wl)
+    idx2, cnt2 = run_topk(scores, wl.q_pos, 2048)
+    assert torch.equal(cnt, cnt2) and torch.equal(idx, idx2)
+    for t in range(wl.T):
+        ref_idx, _ = oracle.topk(scores[0, t, :int(wl.q_pos[0, t]) + 1].cpu().numpy(), 2048)
+        assert np.array_equal(idx[0, t].cpu().numpy(), np.sort(ref_idx))
+    if weights == "zero_query":
+        assert np.array_equal(idx[0, 0].cpu().numpy(), np.arange(2048))
+    _check_layer(wl, O, lse, idx, cnt)
+
+
 def test_layer_decode_1m_context_sampled():
     """Native 1,048,576-token context: scores at sampled positions and every
     needle against the oracle; the selection bit-exact against the oracle's
