@@ -50,6 +50,9 @@ WORKLOAD_DESC = {
                      "positions 65,532..65,535, context 65,536, top-2048, GQA4, sink, 64 needles",
     "tiny_8k": "tiny_8k: DSA decode layer-step, batch 1, 1 query token, context 8,192, top-2048, GQA4, sink, "
                "16 needles",
+    "ragged_b64_mix": "ragged_b64_mix: 64 sequences, 1 query token each, contexts log-uniform in [4,096, 262,144] "
+                      "(seed 3), paged caches (64-position pages); one mix = 5 SWA layer-steps (window 128, GQA8, "
+                      "window-only caches) + 1 DSA layer-step (top-2048, GQA4, sink)",
 }
 
 
@@ -200,6 +203,94 @@ def barrier(device=None):
 def throughput(tokens_per_rank_step: int, steps: int, world: int, slowest_s: float) -> float:
     """Whole-job tokens per second: all ranks' tokens over the slowest rank's time."""
     return tokens_per_rank_step * steps * world / slowest_s
+
+
+# ------------------------------------------------------ the ragged batch mix
+MIX_METRIC = "ragged 64-sequence decode layer-mix (5 SWA + 1 DSA layer-steps) tok/s"
+
+
+def run_mix(args, rank, world, local_rank):
+    """One step = the layer pattern's repeating mix over the ragged serving
+    batch: five SWA layer-steps (each on its own window-only paged cache) and
+    one DSA layer-step (dsa_layer_decode, 64 rows: separate kernels), all 64
+    sequences one token each.  L2 flushed before each mix."""
+    import torch
+    import local_attention_decode_b200 as dsa
+    from workloads import CONFIGS, make_decode_workload, make_swa_window_workload
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS["ragged_b64"]
+    wl = make_decode_workload(device=dev, **cfg)
+    lens = wl.layout.seq_lens
+    B = wl.B
+    Lmax = max(lens)
+    sm_scale = 1.0 / math.sqrt(192)
+    kv = dsa.KV(k=wl.K, v=wl.V, index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G,
+                block_table=wl.layout.block_table, page_size=wl.layout.page_size, num_rows=wl.layout.num_rows)
+    swa = [make_swa_window_workload(100 + i, lens, device=dev) for i in range(5)]
+    swa_kv = [dsa.KV(k=s.K, v=s.V, num_kv_heads=s.G, block_table=s.layout.block_table,
+                     page_size=s.layout.page_size, num_rows=s.layout.num_rows) for s in swa]
+    O = torch.empty((B, 1, 64, 128), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((B, 1, TOP_K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, 1), dtype=torch.int32, device=dev)
+    ws = dsa.alloc_workspace(dsa.OP_LAYER, B, 1, Lmax, TOP_K, device=dev)
+    ws_swa = dsa.alloc_workspace(dsa.OP_SWA_ATTN, B, 1, 1, 128, device=dev)
+    flush = L2Flush(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for s, k in zip(swa, swa_kv):
+            dsa.swa_attn_decode(s.Q, k, s.q_pos, 128, s.sink, sm_scale, O, None, ws_swa)
+        dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, Lmax, TOP_K, wl.sink, sm_scale, O,
+                             None, idx, cnt, ws)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for i in range(K):
+        flush()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clocks = sampler.stop()
+    for w_ in (ws, ws_swa):
+        st, _ = dsa.dsa_check_device_status(w_)
+        if st != dsa.DSA_OK:
+            raise RuntimeError(f"device status {st} after the timed steps")
+    ms = [a.elapsed_time(b) for a, b in ev]
+    total_s = max_over_ranks(sum(ms) / 1e3, dev)
+    peak, peak_kind = measured_peaks()
+    dsa_bytes = sum(indexer_bytes(L, 1) for L in lens) + sum(gathered_bytes(1, min(TOP_K, L)) for L in lens)
+    swa_bytes = 5 * sum(min(128, L) * 8 * (192 + 128) * 2 for L in lens)
+    mix_bytes = dsa_bytes + swa_bytes
+    return {
+        "metric": MIX_METRIC, "value": throughput(B, K, world, total_s), "unit": "tok/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": total_s * 1e3 / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC["ragged_b64_mix"], "batch": B, "query_tokens": 1,
+                   "contexts": {"min": min(lens), "max": max(lens), "total": sum(lens)}, "top_k": TOP_K,
+                   "seed": cfg["seed"], "parallelism": f"replicas x{world}",
+                   "l2": "flushed before each mix outside the timed events"},
+        "us_per_mix": total_s * 1e6 / K,
+        "roofline": {"kernel": "whole mix (5 swa_attn_decode + dsa_layer_decode launches)", "bound": "hbm",
+                     "achieved": mix_bytes / (total_s / K) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": mix_bytes / (total_s / K) / 1e9 / peak, "peak_kind": peak_kind, "traffic": None,
+                     "algorithmic_bytes_per_launch": mix_bytes},
+        "e2e": None,
+        "gpu_launches": (5 * 2 + 4) * K,
+        "clocks": clocks,
+    }
 
 
 # ------------------------------------------------------------------ ours
@@ -485,7 +576,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m"], default=WORKLOAD,
+    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m", "ragged_b64_mix"], default=WORKLOAD,
                     help="decode workload recipe (workloads.CONFIGS); the headline metric is on ctx_1m")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -506,7 +597,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_mix if args.workload == "ragged_b64_mix" else run_ours)(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and args.workload == WORKLOAD:
                 line["cpu_baseline"] = cpu_baseline_line()

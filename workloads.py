@@ -208,6 +208,51 @@ def ragged_batch_lengths(seed: int = 3, B: int = 64):
     return log_uniform_lengths(seed, B, 4096, 262144)
 
 
+# The ragged serving batch: 64 sequences, contexts log-uniform in
+# [4,096, 262,144], paged caches with 64-position pages.  One "mix" is the
+# five SWA layer-steps and one DSA layer-step the layer pattern repeats.
+CONFIGS["ragged_b64"] = dict(seed=3, seq_lens=ragged_batch_lengths(3, 64), T=1, page_size=64, n_needles=4,
+                             needle_mode="uniform")
+
+
+def make_swa_window_workload(seed: int, seq_lens, window: int = 128, page_size: int = 64, G: int = 8,
+                             device="cpu") -> DecodeWorkload:
+    """An SWA layer's decode inputs for sequences of the given lengths, T = 1.
+
+    Only the pages that hold the last `window` positions of each sequence are
+    allocated (the rest of the block table is -1): an SWA layer never reads
+    further back.  Q ~ N(0,1)/sqrt(192) and K, V ~ N(0,1)/sqrt(192) bf16, sink
+    ~ N(0,1), as for the DSA layers; no index keys."""
+    device = torch.device(device)
+    seq_lens = [int(x) for x in seq_lens]
+    B = len(seq_lens)
+    g = torch.Generator(device=device).manual_seed(seed)
+    gc = torch.Generator(device="cpu").manual_seed(seed + 7919)
+    max_pages = max(math.ceil(L / page_size) for L in seq_lens)
+    bt = torch.full((B, max_pages), -1, dtype=torch.int32)
+    first = [max(0, L - window) // page_size for L in seq_lens]
+    last = [(L - 1) // page_size for L in seq_lens]
+    total = sum(l - f + 1 for f, l in zip(first, last))
+    perm = torch.randperm(total, generator=gc).to(torch.int32)
+    off = 0
+    for b in range(B):
+        n = last[b] - first[b] + 1
+        bt[b, first[b]:last[b] + 1] = perm[off:off + n]
+        off += n
+    layout = KVLayout(seq_lens=seq_lens, page_size=page_size, block_table=bt.to(device), num_rows=total * page_size)
+    rows = layout.num_rows
+    std = 1.0 / math.sqrt(QK_DIM)
+    Q = (torch.randn((B, 1, Q_HEADS, QK_DIM), generator=g, device=device) * std).to(torch.bfloat16)
+    K = (torch.randn((rows, G, QK_DIM), generator=g, device=device) * std).to(torch.bfloat16)
+    V = (torch.randn((rows, G, V_DIM), generator=g, device=device) * std).to(torch.bfloat16)
+    sink = torch.randn((Q_HEADS,), generator=g, device=device).float()
+    q_pos = torch.tensor([[L - 1] for L in seq_lens], dtype=torch.int32, device=device)
+    empty8 = torch.empty((0,), dtype=torch.uint8, device=device)
+    emptyf = torch.empty((0,), dtype=torch.float32, device=device)
+    return DecodeWorkload(layout=layout, q_pos=q_pos, q8=empty8, q_scale=emptyf, w=emptyf, k8=empty8,
+                          k_scale=emptyf, Q=Q, K=K, V=V, sink=sink, needles=[], G=G)
+
+
 # ---------------------------------------------------------------- views
 def bits16(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 bit patterns (host copy)."""
