@@ -50,6 +50,8 @@ WORKLOAD_DESC = {
                      "positions 65,532..65,535, context 65,536, top-2048, GQA4, sink, 64 needles",
     "tiny_8k": "tiny_8k: DSA decode layer-step, batch 1, 1 query token, context 8,192, top-2048, GQA4, sink, "
                "16 needles",
+    "prefill_8k_1m": "prefill_8k_1m: DSA layer over 8,192 query tokens at positions 1,040,384..1,048,575 of a "
+                     "1,048,576-token context, causal, top-2048 each, GQA4, sink, 256 Zipf needles",
     "ragged_b64_mix": "ragged_b64_mix: 64 sequences, 1 query token each, contexts log-uniform in [4,096, 262,144] "
                       "(seed 3), paged caches (64-position pages); one mix = 5 SWA layer-steps (window 128, GQA8, "
                       "window-only caches) + 1 DSA layer-step (top-2048, GQA4, sink)",
@@ -289,6 +291,90 @@ def run_mix(args, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": mix_bytes},
         "e2e": None,
         "gpu_launches": (5 * 2 + 4) * K,
+        "clocks": clocks,
+    }
+
+
+# ------------------------------------------------------------- the prefill
+PREFILL_METRIC = "chunked-prefill DSA layer (8,192 query tokens at 1M context) tok/s"
+
+
+def run_prefill(args, rank, world, local_rank):
+    """One step = dsa_prefill over 8,192 query tokens at positions
+    1,040,384..1,048,575 of a 1,048,576-token cache (each causal), i.e. 512
+    fused layer-step launches of 16 tokens.  L2 flushed before each step."""
+    import torch
+    import local_attention_decode_b200 as dsa
+    from workloads import CONFIGS, make_decode_workload
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS["prefill_8k_1m"]
+    wl = make_decode_workload(device=dev, **cfg)
+    NQ = wl.T
+    L = wl.layout.seq_lens[0]
+    sm_scale = 1.0 / math.sqrt(192)
+    kv = dsa.KV(k=wl.K, v=wl.V, index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G,
+                seq_stride=wl.layout.seq_stride, num_rows=wl.layout.num_rows)
+    O = torch.empty((NQ, 64, 128), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((NQ, TOP_K), dtype=torch.int32, device=dev)
+    ws = dsa.alloc_workspace(dsa.OP_PREFILL, 1, NQ, L, TOP_K, device=dev)
+    q8, qs, w, Q, qp = wl.q8[0], wl.q_scale[0], wl.w[0], wl.Q[0], wl.q_pos[0]
+    flush = L2Flush(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dsa.dsa_prefill(q8, qs, w, Q, kv, qp, L, TOP_K, wl.sink, sm_scale, O, None, idx, None, ws)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for i in range(K):
+        flush()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clocks = sampler.stop()
+    st, _ = dsa.dsa_check_device_status(ws)
+    if st != dsa.DSA_OK:
+        raise RuntimeError(f"device status {st} after the timed steps")
+    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / 1e3, dev)
+    step_s = total_s / K
+    pos = wl.q_pos[0].cpu().double()
+    flops = float(((pos + 1) * 16 * 128 * 2).sum())          # the indexer contraction, causal
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        fp8_peak, fp8_kind = 2.0 * bf16, "measured bf16 x 2 (nominal fp8 : bf16 ratio)"
+    except Exception:
+        fp8_peak, fp8_kind = 2.0 * 1590.0, "fallback bf16 x 2"
+    key_bytes = -(-NQ // 16) * indexer_bytes(L, 16)          # keys streamed once per 16-token block
+    peak, peak_kind = measured_peaks()
+    return {
+        "metric": PREFILL_METRIC, "value": throughput(NQ, K, world, total_s), "unit": "tok/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC["prefill_8k_1m"], "query_tokens": NQ, "context": L, "top_k": TOP_K,
+                   "seed": cfg["seed"], "parallelism": f"replicas x{world}",
+                   "l2": "flushed before each step outside the timed events"},
+        "roofline": {"kernel": "dsa_layer_fused_kernel x 512 (16-token blocks)", "bound": "tensor",
+                     "achieved": flops / step_s / 1e12, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": flops / step_s / 1e12 / fp8_peak, "peak_kind": fp8_kind, "traffic": None,
+                     "algorithmic_flops_per_step": flops},
+        "hbm_view": {"key_bytes_per_step": key_bytes, "achieved_GBps": key_bytes / step_s / 1e9, "peak": peak,
+                     "frac": key_bytes / step_s / 1e9 / peak, "peak_kind": peak_kind},
+        "e2e": None,
+        "gpu_launches": -(-NQ // 16) * K,
         "clocks": clocks,
     }
 
@@ -576,7 +662,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m", "ragged_b64_mix"], default=WORKLOAD,
+    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m", "ragged_b64_mix", "prefill_8k_1m"],
+                    default=WORKLOAD,
                     help="decode workload recipe (workloads.CONFIGS); the headline metric is on ctx_1m")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -597,7 +684,8 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = (run_mix if args.workload == "ragged_b64_mix" else run_ours)(args, rank, world, local_rank)
+        run = {"ragged_b64_mix": run_mix, "prefill_8k_1m": run_prefill}.get(args.workload, run_ours)
+        line = run(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and args.workload == WORKLOAD:
                 line["cpu_baseline"] = cpu_baseline_line()

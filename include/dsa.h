@@ -84,6 +84,7 @@ extern "C" {
 #define DSA_OP_SPARSE_ATTN 2
 #define DSA_OP_SWA_ATTN    3
 #define DSA_OP_LAYER       4
+#define DSA_OP_PREFILL     5   /* B = 1, T = NQ query tokens of dsa_prefill */
 
 /*
  * KV-cache description.  One "row" holds one position of one sequence:
@@ -210,6 +211,29 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
                      void *stream, void *const *stage_events);
 
 /*
+ * dsa_prefill -- the DSA layer for NQ query tokens of ONE sequence (a
+ * prefill chunk, or any block of queries over a shared cache): for each query
+ * token t at position q_pos[t], exactly the decode layer-step -- indexer
+ * scores over its visible keys 0..q_pos[t] (causal), the top_k selection, the
+ * sparse GQA attention with the sink -- as dsa_layer_decode computes it.  The
+ * queries run DSA_MAX_T at a time (one dsa_layer_decode per block, enqueued on
+ * `stream`, reusing the workspace), so at most DSA_MAX_T x Lmax scores exist
+ * at once, never the NQ x Lmax matrix.
+ *   q8       e4m3 [NQ][16][128]      q_scale, w  f32 [NQ][16]
+ *   Q        bf16 [NQ][64][192]      q_pos       int32 [NQ], each < Lmax
+ *   kv       the sequence's caches (B = 1), as for dsa_layer_decode
+ *   O        bf16 [NQ][64][128]      lse         f32 [NQ][64] or NULL
+ *   idx_out  int32 [NQ][top_k] or NULL; count_out int32 [NQ] or NULL
+ * Workspace: dsa_workspace_size(DSA_OP_PREFILL, 1, NQ, Lmax, top_k).
+ * Errors as for dsa_layer_decode; a failing block stops the call (earlier
+ * blocks stay enqueued).
+ */
+int dsa_prefill(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+                const int32_t *q_pos, int NQ, int64_t Lmax, int top_k, const float *sink, float sm_scale,
+                void *O, float *lse, int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
+                void *stream);
+
+/*
  * dsa_topk_select_noalloc -- the selection of dsa_topk_select for callers
  * that cannot allocate device memory and so cannot provide a workspace: a
  * framework that owns every device allocation and refuses new ones after it
@@ -222,8 +246,10 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
  * every GPU that loads the library holds it until the process exits.  A call
  * whose scratch need exceeds it returns DSA_ERR_UNSUPPORTED_SHAPE with a
  * message (use dsa_topk_select with a workspace then); on a 148-SM B200 the
- * largest need is about 1.6 MB (74 query rows split two CTAs each), so every
- * shape dsa_topk_select accepts fits.
+ * largest fixed need is about 1.5 MB (74 query rows split two CTAs each) and
+ * the selection's candidate list is shortened to the room left (down to none,
+ * which exchanges every digit instead), so every shape dsa_topk_select
+ * accepts fits.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make

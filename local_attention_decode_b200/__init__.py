@@ -35,11 +35,12 @@ DSA_ERR_WORKSPACE_TOO_SMALL = 3
 DSA_ERR_CUDA = 4
 DSA_ERR_DEVICE_TIMEOUT = 5
 DSA_ERR_DEVICE_BAD_INDEX = 6
-OP_INDEXER, OP_TOPK, OP_SPARSE_ATTN, OP_SWA_ATTN, OP_LAYER = range(5)
+OP_INDEXER, OP_TOPK, OP_SPARSE_ATTN, OP_SWA_ATTN, OP_LAYER, OP_PREFILL = range(6)
 
 EXPORTED = ("dsa_last_error", "dsa_get_dims", "dsa_workspace_size", "dsa_workspace_init",
             "dsa_check_device_status", "dsa_indexer_scores", "dsa_topk_select",
-            "sparse_gqa_attn_decode", "swa_attn_decode", "dsa_layer_decode", "dsa_topk_select_noalloc")
+            "sparse_gqa_attn_decode", "swa_attn_decode", "dsa_layer_decode", "dsa_topk_select_noalloc",
+            "dsa_prefill")
 
 
 class DSAError(RuntimeError):
@@ -79,6 +80,7 @@ _lib.swa_attn_decode.argtypes = [P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I32, 
 _lib.dsa_topk_select_noalloc.argtypes = [P, I64, P, I32, I32, I64, I32, P, P, P]
 _lib.dsa_layer_decode.argtypes = [P, P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I64, I32, P, F32, P, P, P, P,
                                   P, SZ, P, P]
+_lib.dsa_prefill.argtypes = [P, P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I64, I32, P, F32, P, P, P, P, P, SZ, P]
 for _name in EXPORTED[1:]:
     getattr(_lib, _name).restype = ctypes.c_int
 
@@ -243,3 +245,18 @@ def dsa_layer_decode(q8, q_scale, w, Q, kv: KV, q_pos, Lmax: int, top_k: int, si
                                  _ptr(lse, torch.float32, "lse"), _ptr(idx_out, torch.int32, "idx_out"),
                                  _ptr(count_out, torch.int32, "count_out"), _ptr(ws, torch.uint8, "ws"),
                                  ws.numel(), _stream(stream), ev))
+
+
+def dsa_prefill(q8, q_scale, w, Q, kv: KV, q_pos, Lmax: int, top_k: int, sink, sm_scale: float, O, lse=None,
+                idx_out=None, count_out=None, ws=None, stream=None):
+    """NQ query tokens of one sequence: q8 [NQ, 16, 128], Q [NQ, 64, 192], q_pos [NQ], O [NQ, 64, 128]."""
+    if q8.dim() != 3 or tuple(q8.shape[1:]) != (16, 128):
+        raise ValueError("q8 must be [NQ, 16, 128]")
+    NQ = int(q8.shape[0])
+    _check(_lib.dsa_prefill(_ptr(q8, torch.uint8, "q8"), _ptr(q_scale, torch.float32, "q_scale"),
+                            _ptr(w, torch.float32, "w"), _ptr(Q, torch.bfloat16, "Q"), kv.ref,
+                            _ptr(q_pos, torch.int32, "q_pos"), NQ, int(Lmax), int(top_k),
+                            _ptr(sink, torch.float32, "sink"), float(sm_scale), _ptr(O, torch.bfloat16, "O"),
+                            _ptr(lse, torch.float32, "lse"), _ptr(idx_out, torch.int32, "idx_out"),
+                            _ptr(count_out, torch.int32, "count_out"), _ptr(ws, torch.uint8, "ws"),
+                            ws.numel(), _stream(stream)))

@@ -140,10 +140,11 @@ static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan 
             int rc = plan_topk(B, T, Lmax, top_k, &w->tp);
             if (rc) return rc;
             if ((rc = plan_fused(B, T, Lmax, top_k, &w->fp))) return rc;
+            // the self-cleaning selection scratch first: its offset does not depend on the shape
+            w->topk = take(std::max(w->tp.scratch_bytes, w->fp.ok ? w->fp.scratch_bytes : 0));
             w->scores = take((size_t)B * T * Lmax * 4);
             w->idx = take((size_t)B * T * top_k * 4);
             w->count = take((size_t)B * T * 4);
-            w->topk = take(std::max(w->tp.scratch_bytes, w->fp.ok ? w->fp.scratch_bytes : 0));
             const int splits = (top_k + kAttnChunk - 1) / kAttnChunk;
             const size_t rows = (size_t)B * T * DSA_Q_HEADS * splits;
             w->part_o = take(rows * DSA_V_DIM * 4);
@@ -191,8 +192,54 @@ int dsa_get_dims(int32_t *dims, int n) {
     return DSA_OK;
 }
 
+// Workspace of dsa_prefill: one layout for all of its query blocks
+// (DSA_MAX_T tokens each, the last one possibly shorter), every region sized
+// for the largest block, so that each block finds the self-cleaning selection
+// scratch where the previous one left it clean.  full / tail: the plans the
+// blocks run with (the tail's selection and launch plans, the shared offsets).
+static int plan_prefill(int NQ, int64_t Lmax, int top_k, WsPlan *full, WsPlan *tail) {
+    const int T0 = std::min(NQ, DSA_MAX_T), T1 = NQ % DSA_MAX_T ? NQ % DSA_MAX_T : T0;
+    WsPlan a, b;
+    int rc = plan_workspace(DSA_OP_LAYER, 1, T0, Lmax, top_k, &a);
+    if (rc) return rc;
+    if ((rc = plan_workspace(DSA_OP_LAYER, 1, T1, Lmax, top_k, &b))) return rc;
+    // the layer layout puts the selection scratch right after the status word
+    // in both plans; the later regions start after the larger of the two
+    const size_t topk_end = std::max(a.scores, b.scores);
+    const size_t shift = topk_end - a.scores;   // a is the larger block: move its later regions past both
+    for (WsPlan *w : {&a}) {
+        w->scores += shift;
+        w->idx += shift;
+        w->count += shift;
+        w->part_o += shift;
+        w->part_ml += shift;
+        w->total += shift;
+    }
+    b.scores = a.scores;
+    b.idx = a.idx;
+    b.count = a.count;
+    b.part_o = a.part_o;
+    b.part_ml = a.part_ml;
+    b.total = a.total;
+    *full = a;
+    *tail = b;
+    return DSA_OK;
+}
+
 int dsa_workspace_size(int op, int B, int T, int64_t Lmax, int top_k, size_t *bytes) {
     if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
+    if (op == DSA_OP_PREFILL) {
+        if (B != 1) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "DSA_OP_PREFILL takes one sequence (B = 1), got B=%d", B);
+        if (T < 1) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "NQ=%d < 1", T);
+        if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
+        if (top_k < 1 || top_k > DSA_MAX_TOPK)
+            return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
+        WsPlan full, tail;
+        int rc = plan_prefill(T, Lmax, top_k, &full, &tail);
+        if (rc) return rc;
+        *bytes = full.total;
+        return DSA_OK;
+    }
     int rc = check_common(B, T);
     if (rc) return rc;
     if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
@@ -310,10 +357,14 @@ int swa_attn_decode(const void *Q, const dsa_kv_t *kv, const int32_t *q_pos, int
                             stream, DSA_OP_SWA_ATTN);
 }
 
-int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+static int layer_run(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
                      const int32_t *q_pos, int B, int T, int64_t Lmax, int top_k, const float *sink, float sm_scale,
-                     void *O, float *lse, int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
-                     void *stream, void *const *stage_events) {
+                     void *O, float *lse, int32_t *idx_out, int32_t *count_out, void *ws, const WsPlan &wp,
+                     cudaStream_t s, void *const *stage_events);
+
+// Argument checks shared by dsa_layer_decode and dsa_prefill.
+static int check_layer_args(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+                            const int32_t *q_pos, int B, int T, int64_t Lmax, int top_k, float sm_scale, const void *O) {
     if (!q8 || !q_scale || !w || !Q || !q_pos || !O) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
     if (!aligned16(q8) || !aligned16(Q) || !aligned16(O)) return fail(DSA_ERR_INVALID_ARG, "q8 / Q / O not 16-byte aligned");
     int rc = check_common(B, T);
@@ -324,10 +375,28 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
     if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
     if (top_k < 1 || top_k > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
     if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+    return DSA_OK;
+}
+
+int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+                     const int32_t *q_pos, int B, int T, int64_t Lmax, int top_k, const float *sink, float sm_scale,
+                     void *O, float *lse, int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
+                     void *stream, void *const *stage_events) {
+    int rc = check_layer_args(q8, q_scale, w, Q, kv, q_pos, B, T, Lmax, top_k, sm_scale, O);
+    if (rc) return rc;
     WsPlan wp;
     if (rc = plan_workspace(DSA_OP_LAYER, B, T, Lmax, top_k, &wp); rc) return rc;
     if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return layer_run(q8, q_scale, w, Q, kv, q_pos, B, T, Lmax, top_k, sink, sm_scale, O, lse, idx_out, count_out, ws,
+                     wp, static_cast<cudaStream_t>(stream), stage_events);
+}
+
+// The layer-step on a checked workspace with plan wp.
+static int layer_run(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+                     const int32_t *q_pos, int B, int T, int64_t Lmax, int top_k, const float *sink, float sm_scale,
+                     void *O, float *lse, int32_t *idx_out, int32_t *count_out, void *ws, const WsPlan &wp,
+                     cudaStream_t s, void *const *stage_events) {
+    int rc = DSA_OK;
     uint32_t *status = at<uint32_t>(ws, wp.status);
     float *scores = at<float>(ws, wp.scores);
     int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, wp.idx);
@@ -394,3 +463,28 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
 }
 
 }  // extern "C"
+
+int dsa_prefill(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
+                const int32_t *q_pos, int NQ, int64_t Lmax, int top_k, const float *sink, float sm_scale, void *O,
+                float *lse, int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes, void *stream) {
+    if (NQ < 1) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "NQ=%d < 1", NQ);
+    int rc = check_layer_args(q8, q_scale, w, Q, kv, q_pos, 1, std::min(NQ, DSA_MAX_T), Lmax, top_k, sm_scale, O);
+    if (rc) return rc;
+    WsPlan full, tail;
+    if ((rc = plan_prefill(NQ, Lmax, top_k, &full, &tail))) return rc;
+    if ((rc = check_ws(ws, ws_bytes, full))) return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // one layer-step per block of DSA_MAX_T query tokens, on the one layout
+    for (int t0 = 0; t0 < NQ; t0 += DSA_MAX_T) {
+        const int T = std::min(DSA_MAX_T, NQ - t0);
+        rc = layer_run(static_cast<const uint8_t *>(q8) + (size_t)t0 * DSA_INDEX_HEADS * DSA_INDEX_DIM,
+                       q_scale + (size_t)t0 * DSA_INDEX_HEADS, w + (size_t)t0 * DSA_INDEX_HEADS,
+                       static_cast<const __nv_bfloat16 *>(Q) + (size_t)t0 * DSA_Q_HEADS * DSA_QK_DIM, kv, q_pos + t0,
+                       1, T, Lmax, top_k, sink, sm_scale,
+                       static_cast<__nv_bfloat16 *>(O) + (size_t)t0 * DSA_Q_HEADS * DSA_V_DIM,
+                       lse ? lse + (size_t)t0 * DSA_Q_HEADS : nullptr, idx_out ? idx_out + (size_t)t0 * top_k : nullptr,
+                       count_out ? count_out + t0 : nullptr, ws, T == DSA_MAX_T || T == NQ ? full : tail, s, nullptr);
+        if (rc) return rc;
+    }
+    return DSA_OK;
+}

@@ -121,7 +121,8 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         } else if ((int)blockIdx.x < fp.rows * fp.C && (fp.C > 1 || fp.hist_ready)) {
             // the warps outside the teams clear the selection scratch for the next call
             constexpr int kFree = kThreads - kTeams * 128;
-            topk::clear_row_share(fp.tk, blockIdx.x / fp.C, blockIdx.x % fp.C, fp.C, threadIdx.x - kTeams * 128, kFree);
+            topk::clear_row_share(fp.tk, blockIdx.x / fp.C, blockIdx.x % fp.C, fp.C, fp.hist_ready != 0,
+                                  threadIdx.x - kTeams * 128, kFree);
         }
     }
     if (!grid_sync(fp.grid_bar, 3 * G, status, &sync_flag)) return;
@@ -175,7 +176,7 @@ int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
     plan->grid = grid;
     plan->rows = rows;
     plan->C = std::max(1, grid / rows);
-    plan->scratch_bytes = (size_t)rows * topk::scratch_words(plan->C, topk::kListCap) * 4 + 256;   // + grid barrier words
+    plan->scratch_bytes = (size_t)rows * topk::scratch_words(plan->C, topk::kListCap, true) * 4 + 256;   // + grid barrier words
     plan->ok = true;
     return DSA_OK;
 }
@@ -185,12 +186,12 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     using namespace fused;
     const size_t budget = fused_smem_budget();
     uint32_t *row_scratch = scratch + 64;   // the first 256 bytes hold the grid barrier words
-    const int row_words = topk::scratch_words(plan.C, topk::kListCap);
+    const int row_words = topk::scratch_words(plan.C, topk::kListCap, true);
 
     // indexer phase, with the first histogram when the rows' histograms fit
     IndexerLaunch L;
     int hist_rows = plan.rows <= kMaxHistRows ? plan.rows : 0;
-    int rc = prepare_indexer(ia, hist_rows, row_words, row_scratch + topk::kHistI, budget, &L);
+    int rc = prepare_indexer(ia, hist_rows, row_words, row_scratch + topk::histi_base(plan.C, topk::kListCap), budget, &L);
     if (rc == DSA_OK && hist_rows && L.p.stages < 3) hist_rows = 0;   // keep the stream at least 3 stages deep
     if (rc != DSA_OK || hist_rows == 0) {
         hist_rows = 0;

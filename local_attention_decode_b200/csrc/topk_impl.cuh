@@ -50,19 +50,24 @@ constexpr int kCandCap = 8192;              // per-warp candidates a CTA keeps i
 // Per-row scratch (u32 words), used when C > 1 or when the first histogram is
 // produced by the indexer:
 //   [kHist1, +2048) [kHist2, +2048) [kHist3, +1024)  digit histograms
-//   [kHistI, +2052)  the histogram built by the indexer: bits 30..20 of the
-//                    non-negative keys (2048 bins) and the count of negative keys
 //   [kCnt, +2C)      per-CTA (greater, equal) counts at T* (exchange path)
 //   [kCnt+2C, +C)    per-CTA counts of keys above the 22-bit threshold bin
 //   ctl_base(C):     [0] barrier arrivals, [1] CTAs done, [2] list length,
 //                    [3] a CTA's candidates overflowed its shared memory,
 //                    [4] list length of the one-barrier path (select_row_hist)
 //   list_base(C):    list_cap keys, then list_cap positions
-constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kHistI = 5120, kCnt = 5120 + 2052;
+//   histi_base(C, list_cap), only when the indexer builds it: kHistIWords
+//                    words, bits 30..20 of the non-negative keys (2048 bins)
+//                    and the count of negative keys
+constexpr int kHist1 = 0, kHist2 = 2048, kHist3 = 4096, kCnt = 5120;
+constexpr int kHistIWords = 2052;
 __host__ __device__ constexpr int ctl_base(int C) { return kCnt + 3 * C; }
 constexpr int kCtlWords = 5;
 __host__ __device__ constexpr int list_base(int C) { return (ctl_base(C) + kCtlWords + 3) & ~3; }
-__host__ __device__ constexpr int scratch_words(int C, int list_cap) { return list_base(C) + 2 * list_cap; }
+__host__ __device__ constexpr int histi_base(int C, int list_cap) { return list_base(C) + 2 * list_cap; }
+__host__ __device__ constexpr int scratch_words(int C, int list_cap, bool histi = false) {
+    return histi_base(C, list_cap) + (histi ? kHistIWords : 0);
+}
 
 struct Params {
     const float *scores;
@@ -682,7 +687,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
 
 // One-barrier selection of row `row` by CTA c of C (C > 1), for a row whose
 // score histogram the indexer has already built in the row's scratch
-// (kHistI: bits 30..20 of the non-negative keys, eight bins per octave, and
+// (at histi_base: bits 30..20 of the non-negative keys, eight bins per octave, and
 // the count of negative keys).  Each thread holds up to kHistRegs keys of its
 // warp's part of the slice in registers.  With the threshold bin b1 known from
 // the histogram, every key at or above it (above(b1) + h[b1] keys in the row)
@@ -727,9 +732,9 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
 #pragma unroll
     for (int u = 0; u < kHistPer; ++u) {
         const int j = u * NT + threadIdx.x;
-        hv[u] = j < kBins ? __ldcg(rs + kHistI + j) : 0u;
+        hv[u] = j < kBins ? __ldcg(rs + histi_base(C, p.list_cap) + j) : 0u;
     }
-    const uint32_t negatives = __ldcg(rs + kHistI + kBins);
+    const uint32_t negatives = __ldcg(rs + histi_base(C, p.list_cap) + kBins);
     float v[kHistRegs];
 #pragma unroll
     for (int i = 0; i < kHistRegs; ++i) {
@@ -892,13 +897,17 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
 
 // CTA c's share of clearing row `row`'s scratch for the next call, once no
 // CTA of the row reads it any more: the digit histograms, the counts and the
-// list entries used.  The control words stay for reset_row_ctl.
+// list entries used, and the indexer's histogram when it was built (histi).
+// The control words stay for reset_row_ctl.
 // Threads tid < nt of the CTA take part.
-__device__ __forceinline__ void clear_row_share(const Params &p, int row, int c, int C, int tid, int nt) {
+__device__ __forceinline__ void clear_row_share(const Params &p, int row, int c, int C, bool histi, int tid, int nt) {
     uint32_t *rs = p.scratch + (int64_t)row * p.scratch_row_words;
-    const int words = C > 1 ? ctl_base(C) : kCnt;
-    for (int j = c * nt + tid; j < words; j += C * nt) rs[j] = 0;
+    if (histi) {
+        uint32_t *hi = rs + histi_base(C, p.list_cap);
+        for (int j = c * nt + tid; j < kHistIWords; j += C * nt) hi[j] = 0;
+    }
     if (C > 1) {
+        for (int j = c * nt + tid; j < ctl_base(C); j += C * nt) rs[j] = 0;
         const uint32_t m2 = __ldcg(rs + ctl_base(C) + 2), m4 = __ldcg(rs + ctl_base(C) + 4);
         const uint32_t m = m2 > m4 ? m2 : m4;
         const uint32_t used = m < (uint32_t)p.list_cap ? m : (uint32_t)p.list_cap;

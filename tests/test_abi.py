@@ -26,7 +26,8 @@ def dsa():
 def test_header_declares_the_expected_entry_points():
     names = _declared_functions()
     for n in ("dsa_indexer_scores", "dsa_topk_select", "sparse_gqa_attn_decode", "swa_attn_decode",
-              "dsa_layer_decode", "dsa_workspace_size", "dsa_check_device_status", "dsa_last_error"):
+              "dsa_layer_decode", "dsa_prefill", "dsa_workspace_size", "dsa_check_device_status",
+              "dsa_last_error"):
         assert n in names
 
 
@@ -90,3 +91,18 @@ def test_workspace_sizes_grow_with_the_problem(dsa):
     a = dsa.workspace_size(dsa.OP_LAYER, 1, 1, 8192, 2048)
     b = dsa.workspace_size(dsa.OP_LAYER, 1, 4, 65536, 2048)
     assert b > a > 8192 * 4
+
+
+def test_prefill_workspace_covers_every_block(dsa):
+    """dsa_prefill runs 16-token blocks and a shorter last one on one
+    workspace layout: at least what each block needs, at most what both would
+    need side by side."""
+    for nq, last in ((40, 8), (16, 16), (5, 5)):
+        need = dsa.workspace_size(dsa.OP_PREFILL, 1, nq, 8192, 2048)
+        sizes = [dsa.workspace_size(dsa.OP_LAYER, 1, t, 8192, 2048) for t in {min(16, nq), last}]
+        assert max(sizes) <= need <= sum(sizes)
+    size = ctypes.c_size_t(0)
+    assert dsa._lib.dsa_workspace_size(dsa.OP_PREFILL, 2, 40, 8192, 2048, ctypes.byref(size)) == \
+        dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert dsa._lib.dsa_workspace_size(dsa.OP_PREFILL, 1, 0, 8192, 2048, ctypes.byref(size)) == \
+        dsa.DSA_ERR_UNSUPPORTED_SHAPE

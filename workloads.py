@@ -215,6 +215,11 @@ CONFIGS["ragged_b64"] = dict(seed=3, seq_lens=ragged_batch_lengths(3, 64), T=1, 
                              needle_mode="uniform")
 
 
+# The chunked prefill: the last 8,192 positions (1,040,384..1,048,575) of a
+# 1,048,576-token context, each query token attending causally.
+CONFIGS["prefill_8k_1m"] = dict(seed=4, seq_lens=[1048576], T=8192, n_needles=256, needle_mode="zipf")
+
+
 def make_swa_window_workload(seed: int, seq_lens, window: int = 128, page_size: int = 64, G: int = 8,
                              device="cpu") -> DecodeWorkload:
     """An SWA layer's decode inputs for sequences of the given lengths, T = 1.
