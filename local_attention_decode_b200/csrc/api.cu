@@ -424,6 +424,7 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
         a.part_o = at<float>(ws, wp.part_o);
         a.part_ml = at<float>(ws, wp.part_ml);
         a.status = status;
+        a.padded = 1;   // the fused selection pads every idx row with -1
         rc = launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s);
         if (rc == DSA_OK) {
             for (int i = 1; i <= 4; ++i)

@@ -12,7 +12,7 @@ __global__ void __launch_bounds__(kThreads)
 gather_attn_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    attn_unit<0>(p, sm, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
+    attn_unit(p, sm, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x, 0);
 }
 
 // One CTA per (query, head), as in the fused layer-step (same arithmetic).

@@ -54,6 +54,7 @@ struct Params {
     float *part_o;
     float *part_ml;
     uint32_t *status;
+    int padded;         // idx rows are full length, -1 past the selection: count is not read
 };
 
 struct Smem {
@@ -65,17 +66,20 @@ struct Smem {
     float l[4][16];
 };
 
-// Barrier of one 128-thread team; the barrier id is a compile-time constant so
-// that the kernel reserves only the barriers it uses.
-template <int BAR>
-__device__ __forceinline__ void team_sync() {
-    asm volatile("bar.sync %0, 128;" ::"n"(BAR) : "memory");
+// Barrier of one 128-thread team.  The id is a run-time value, so that all
+// teams of a CTA run one copy of the unit's code (one set of instruction-cache
+// lines to fetch instead of one per team).
+__device__ __forceinline__ void team_sync(int bar) {
+    asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -117,10 +121,9 @@ __device__ __forceinline__ bool key_row(const Params &p, int b, int64_t pos, int
 
 // One split-KV unit: keys [split * 64, split * 64 + 64) of query bt and KV
 // head g, by a team of 128 threads (tid 0..127) synchronised with the named
-// barrier BAR; writes the unit's partial (O, max, sum) for the 64/G
+// barrier `bar`; writes the unit's partial (O, max, sum) for the 64/G
 // query heads of the group.
-template <int BAR>
-__device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid) {
+__device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid, int bar) {
     const int b = bt / p.T;
     const int hpg = DSA_Q_HEADS / p.G;
     const int warp = tid >> 5, lane = tid & 31;
@@ -128,7 +131,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
     // ---- the key set of this split
     int n_total, win_lo = 0;
     if (p.idx) {
-        n_total = min(__ldcg(p.count + bt), p.idx_stride);
+        n_total = p.padded ? p.idx_stride : min(__ldcg(p.count + bt), p.idx_stride);
     } else {
         const int32_t pq = __ldg(p.q_pos + bt);
         win_lo = max(0, pq - p.window + 1);
@@ -151,7 +154,9 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         if (tid < nk) {
             int64_t pos = p.idx ? (int64_t)__ldcg(p.idx + (int64_t)bt * p.idx_stride + k0 + tid)
                                 : (int64_t)(win_lo + k0 + tid);
-            if (!key_row(p, b, pos, &row)) {
+            if (p.padded && pos < 0) {
+                row = -1;   // past the selection
+            } else if (!key_row(p, b, pos, &row)) {
                 flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX);
                 row = -1;
             }
@@ -166,7 +171,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         if (r < hpg) cp_async16(dst, qg + (int64_t)r * DSA_QK_DIM + col);
         else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
-    team_sync<BAR>();
+    team_sync(bar);
     // ---- gather K and V rows
     const int G = p.G;
     for (int c = tid; c < kChunk * (DSA_QK_DIM / 8); c += kThreads) {
@@ -176,6 +181,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         if (row >= 0) cp_async16(dst, p.K + (row * G + g) * DSA_QK_DIM + col);
         else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
+    cp_async_commit();   // Q and K: the first group
     for (int c = tid; c < kChunk * (DSA_V_DIM / 8); c += kThreads) {
         int r = c / (DSA_V_DIM / 8), col = (c % (DSA_V_DIM / 8)) * 8;
         __nv_bfloat16 *dst = sm.v + r * kVS + col;
@@ -183,8 +189,9 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         if (row >= 0) cp_async16(dst, p.V + (row * G + g) * DSA_V_DIM + col);
         else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
-    cp_async_wait_all();
-    team_sync<BAR>();
+    cp_async_commit();   // V: the second group
+    cp_async_wait_group<1>();   // Q and K have landed; V may still be in flight
+    team_sync(bar);
 
     // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8)
     const int key0 = warp * 16;
@@ -239,6 +246,8 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
     float o[DSA_V_DIM / 8][4];
 #pragma unroll
     for (int nt = 0; nt < DSA_V_DIM / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    cp_async_wait_group<0>();
+    team_sync(bar);
 #pragma unroll
     for (int dp = 0; dp < DSA_V_DIM / 16; ++dp) {
         uint32_t b0, b1, b2, b3;
@@ -255,7 +264,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         sm.l[warp][g0] = lrow[0];
         sm.l[warp][g0 + 8] = lrow[1];
     }
-    team_sync<BAR>();   // K/V tiles are no longer read: reuse them for the O exchange
+    team_sync(bar);   // K/V tiles are no longer read: reuse them for the O exchange
     float *so = reinterpret_cast<float *>(sm.k);   // [4 warps][16 rows][128]
     float scale_row[2];
 #pragma unroll
@@ -272,7 +281,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         *reinterpret_cast<float2 *>(d0) = make_float2(o[nt][0] * scale_row[0], o[nt][1] * scale_row[0]);
         *reinterpret_cast<float2 *>(d1) = make_float2(o[nt][2] * scale_row[1], o[nt][3] * scale_row[1]);
     }
-    team_sync<BAR>();
+    team_sync(bar);
     // each thread: one head row (tid / 8) and 16 columns
     {
         const int row = tid >> 3, c0 = (tid & 7) * 16;
@@ -426,6 +435,7 @@ inline Params make_params(const AttnArgs &a) {
     p.part_o = a.part_o;
     p.part_ml = a.part_ml;
     p.status = a.status;
+    p.padded = a.padded;
     return p;
 }
 

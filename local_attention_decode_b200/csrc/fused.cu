@@ -74,6 +74,7 @@ __device__ bool grid_sync(uint32_t *bar, uint32_t target, uint32_t *status, uint
     return *flag != 0;
 }
 
+
 __global__ void __launch_bounds__(kThreads, 1)
 dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
                        const __grid_constant__ CUtensorMap tmap_q, const Params fp) {
@@ -111,12 +112,7 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
             const int units = fp.rows * G_kv * splits;
             for (int u = team * (int)G + (int)blockIdx.x; u < units; u += kTeams * (int)G) {
                 const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
-                switch (team) {
-                    case 0: attn::attn_unit<1>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
-                    case 1: attn::attn_unit<2>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
-                    case 2: attn::attn_unit<3>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
-                    default: attn::attn_unit<4>(fp.at, sm, split, g, bt, threadIdx.x & 127); break;
-                }
+                attn::attn_unit(fp.at, sm, split, g, bt, threadIdx.x & 127, 1 + team);
             }
         } else if ((int)blockIdx.x < fp.rows * fp.C && (fp.C > 1 || fp.hist_ready)) {
             // the warps outside the teams clear the selection scratch for the next call

@@ -88,6 +88,7 @@ struct AttnArgs {
     float *part_ml;         // [B*T][64][splits][2]
     uint32_t *status;
     void *mid_event = nullptr;  // optional cudaEvent_t recorded between the gather and the combine
+    int padded = 0;             // idx rows full length, -1 past the selection (count not read)
 };
 size_t attn_partial_bytes(int B, int T, int max_keys);
 int launch_attention(const AttnArgs &a, cudaStream_t stream);
