@@ -241,11 +241,11 @@ def run_mix(args, rank, world, local_rank):
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(stage=None):
         for s, k in zip(swa, swa_kv):
             dsa.swa_attn_decode(s.Q, k, s.q_pos, 128, s.sink, sm_scale, O, None, ws_swa)
         dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, Lmax, TOP_K, wl.sink, sm_scale, O,
-                             None, idx, cnt, ws)
+                             None, idx, cnt, ws, stage_events=stage)
 
     for _ in range(args.warmup):
         flush()
@@ -253,6 +253,10 @@ def run_mix(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    stages = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for st_ in stages:
+        for e_ in st_:
+            e_.record(stream)   # materialise the handles the C API records into
     sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
     barrier(dev)
     torch.cuda.synchronize(dev)
@@ -260,11 +264,17 @@ def run_mix(args, rank, world, local_rank):
     for i in range(K):
         flush()
         ev[i][0].record(stream)
-        step()
+        step(stages[i])
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier(dev)
     clocks = sampler.stop()
+    med = lambda xs: statistics.median(xs) * 1e3
+    stage_us = {"swa_x5": med([ev[i][0].elapsed_time(stages[i][0]) for i in range(K)]),
+                "dsa_indexer": med([stages[i][0].elapsed_time(stages[i][1]) for i in range(K)]),
+                "dsa_topk": med([stages[i][1].elapsed_time(stages[i][2]) for i in range(K)]),
+                "dsa_attention": med([stages[i][2].elapsed_time(stages[i][3]) for i in range(K)]),
+                "dsa_combine": med([stages[i][3].elapsed_time(stages[i][4]) for i in range(K)])}
     for w_ in (ws, ws_swa):
         st, _ = dsa.dsa_check_device_status(w_)
         if st != dsa.DSA_OK:
@@ -285,6 +295,7 @@ def run_mix(args, rank, world, local_rank):
                    "seed": cfg["seed"], "parallelism": f"replicas x{world}",
                    "l2": "flushed before each mix outside the timed events"},
         "us_per_mix": total_s * 1e6 / K,
+        "stage_us_median": stage_us,
         "roofline": {"kernel": "whole mix (5 swa_attn_decode + dsa_layer_decode launches)", "bound": "hbm",
                      "achieved": mix_bytes / (total_s / K) / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": mix_bytes / (total_s / K) / 1e9 / peak, "peak_kind": peak_kind, "traffic": None,
@@ -420,7 +431,11 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {st} after warm-up")
 
     K = args.steps
+    fused = B * T <= FUSED_MAX_ROWS
+    # one fused kernel: only the events around it (no event records between its end and the last event)
     stage = [new_events(5) for _ in range(K)]
+    if fused:
+        stage = [[ev[0], None, None, None, ev[4]] for ev in stage]
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
     barrier(dev)
@@ -434,15 +449,15 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
 
     step_ms = [stage[i][0].elapsed_time(stage[i][4]) for i in range(K)]
-    idx_ms = [stage[i][0].elapsed_time(stage[i][1]) for i in range(K)]
-    topk_ms = [stage[i][1].elapsed_time(stage[i][2]) for i in range(K)]
-    attn_ms = [stage[i][2].elapsed_time(stage[i][3]) for i in range(K)]
-    comb_ms = [stage[i][3].elapsed_time(stage[i][4]) for i in range(K)]
+    if not fused:
+        idx_ms = [stage[i][0].elapsed_time(stage[i][1]) for i in range(K)]
+        topk_ms = [stage[i][1].elapsed_time(stage[i][2]) for i in range(K)]
+        attn_ms = [stage[i][2].elapsed_time(stage[i][3]) for i in range(K)]
+        comb_ms = [stage[i][3].elapsed_time(stage[i][4]) for i in range(K)]
     total_s = max_over_ranks(sum(step_ms) / 1e3, dev)
     st, _ = dsa.dsa_check_device_status(ws)
     if st != dsa.DSA_OK:
         raise RuntimeError(f"device status {st} after the timed steps")
-    fused = B * T <= FUSED_MAX_ROWS
 
     # the indexer on its own (dsa_indexer_scores), same inputs, for its HBM rate
     idx_ws = dsa.alloc_workspace(dsa.OP_INDEXER, B, T, L, 1, device=dev)

@@ -202,7 +202,10 @@ int swa_attn_decode(const void *Q, const dsa_kv_t *kv, const int32_t *q_pos, int
  * copies of the selection (NULL = not wanted).
  * stage_events: NULL, or an array of 5 cudaEvent_t recorded on `stream`
  * before the indexer, before the selection, before the attention, before the
- * combine and at the end (for per-stage timing).
+ * combine and at the end (for per-stage timing); NULL entries are skipped.
+ * Event 0 is recorded after the host-side preparation, right before the first
+ * kernel.  When the step runs as one fused kernel (B*T <= 16), events 1-4 are
+ * all recorded after it.
  */
 int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const void *Q,
                      const dsa_kv_t *kv, const int32_t *q_pos, int B, int T, int64_t Lmax,

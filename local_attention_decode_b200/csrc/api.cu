@@ -402,7 +402,6 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
     int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, wp.idx);
     int32_t *count = count_out ? count_out : at<int32_t>(ws, wp.count);
 
-    if (rc = record(stage_events, 0, s); rc) return rc;
     IndexerArgs ia{static_cast<const uint8_t *>(q8), q_scale, w, kv, q_pos, B, T, Lmax, scores, Lmax, status};
     if (wp.fp.ok) {
         // one cooperative launch for the whole layer-step
@@ -425,7 +424,8 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
         a.part_ml = at<float>(ws, wp.part_ml);
         a.status = status;
         a.padded = 1;   // the fused selection pads every idx row with -1
-        rc = launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s);
+        rc = launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s,
+                          stage_events ? stage_events[0] : nullptr);
         if (rc == DSA_OK) {
             for (int i = 1; i <= 4; ++i)
                 if (rc = record(stage_events, i, s); rc) return rc;
@@ -434,6 +434,7 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
         if (rc != DSA_ERR_UNSUPPORTED_SHAPE) return rc;
         // the fused kernel does not fit this shape: run the separate kernels
     }
+    if (rc = record(stage_events, 0, s); rc) return rc;
     if (rc = launch_indexer(ia, s); rc) return rc;
     if (rc = record(stage_events, 1, s); rc) return rc;
     if (rc = launch_topk(wp.tp, scores, Lmax, q_pos, top_k, idx, count, at<uint32_t>(ws, wp.topk), status, s); rc)

@@ -178,7 +178,8 @@ int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
 }
 
 int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
-                 int32_t *count, uint32_t *scratch, cudaStream_t stream) {
+                 int32_t *count, uint32_t *scratch, cudaStream_t stream,
+                 void *start_event) {
     using namespace fused;
     const size_t budget = fused_smem_budget();
     uint32_t *row_scratch = scratch + 64;   // the first 256 bytes hold the grid barrier words
@@ -249,6 +250,10 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (start_event) {   // recorded after the host-side preparation, right before the launch
+        e = cudaEventRecord(static_cast<cudaEvent_t>(start_event), stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
     e = cudaLaunchKernelEx(&cfg, dsa_layer_fused_kernel, L.tmap_k, L.tmap_ks, L.tmap_q, fp);
     if (e != cudaSuccess) return cuda_fail(e, "fused layer-step launch");
     return DSA_OK;

@@ -103,7 +103,8 @@ struct FusedPlan {
 };
 int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan);
 int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
-                 int32_t *count, uint32_t *scratch, cudaStream_t stream);
+                 int32_t *count, uint32_t *scratch, cudaStream_t stream,
+                 void *start_event = nullptr);
 
 
 }  // namespace dsa
