@@ -12,7 +12,7 @@ constexpr int kThreads = 512;
 constexpr int kMinChunk = 4096;             // keys per CTA below which a row is not split further
 constexpr int kMaxCacheKeys = 32 * 1024;    // 128 KB of cached keys per CTA
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 topk_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Shared<kThreads> *sh = reinterpret_cast<Shared<kThreads> *>(smem_raw);

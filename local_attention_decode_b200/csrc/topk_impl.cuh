@@ -43,6 +43,7 @@ namespace topk {
 
 constexpr int kBins = 2048;                 // largest digit: 11 bits
 constexpr int kUnroll = 8;                  // independent loads in flight per thread
+constexpr int kUnrollGlobal = 16;           // the same, for slices read from global memory
 constexpr int kListCap = 12288;             // candidate-list entries per row (global scratch)
 constexpr int kSmemList = 4096;             // candidate-list entries a CTA takes into shared memory
 constexpr int kCandCap = 8192;              // per-warp candidates a CTA keeps in shared memory, in all
@@ -255,7 +256,7 @@ __device__ __forceinline__ void warp_part(int64_t len, int64_t *wlo, int64_t *wh
 // Calls fn(j, valid, k) for the keys j of this warp's part [wlo, whi), 32
 // consecutive keys per call, in position order (all lanes call fn together).
 // Keys cached in shared memory are read one group at a time (compact code);
-// keys read from global memory are fetched kUnroll groups at a time.
+// keys read from global memory are fetched kUnrollGlobal groups at a time.
 template <class KeyAt, class Fn>
 __device__ __forceinline__ void warp_walk(int64_t wlo, int64_t whi, bool cached, const uint32_t *cache,
                                           KeyAt key_at, Fn fn) {
@@ -268,15 +269,15 @@ __device__ __forceinline__ void warp_walk(int64_t wlo, int64_t whi, bool cached,
             fn(j, valid, valid ? cache[j] : 0u);
         }
     } else {
-        for (int64_t base = wlo; base < whi; base += 32 * kUnroll) {
-            uint32_t kk[kUnroll];
+        for (int64_t base = wlo; base < whi; base += 32 * kUnrollGlobal) {
+            uint32_t kk[kUnrollGlobal];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
+            for (int u = 0; u < kUnrollGlobal; ++u) {
                 const int64_t j = base + u * 32 + lane;
                 kk[u] = j < whi ? key_at(j) : 0u;
             }
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) fn(base + u * 32 + lane, base + u * 32 + lane < whi, kk[u]);
+            for (int u = 0; u < kUnrollGlobal; ++u) fn(base + u * 32 + lane, base + u * 32 + lane < whi, kk[u]);
         }
     }
 }
@@ -397,19 +398,11 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     auto slice_hist = [&](uint32_t prefix, uint32_t mask, int shift, int nb) {
         for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
         __syncthreads();
-        for (int64_t base = 0; base < len; base += (int64_t)kUnroll * NT) {
-            uint32_t kk[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t j = base + u * NT + threadIdx.x;
-                kk[u] = j < len ? key_at(j) : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const bool active = base + u * NT + threadIdx.x < len && (kk[u] & mask) == prefix;
-                warp_hist_add(sh->hist, (kk[u] >> shift) & (nb - 1), active);
-            }
-        }
+        int64_t wlo, whi;
+        warp_part<NT>(len, &wlo, &whi);
+        warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t, bool valid, uint32_t k) {
+            warp_hist_add(sh->hist, (k >> shift) & (nb - 1), valid && (k & mask) == prefix);
+        });
         __syncthreads();
     };
     uint32_t barrier_no = 0;
