@@ -767,15 +767,11 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
         wc += __popc(cm);
     }
     if (lane == 0) sh->warp_a[warp] = wc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t tot = 0;
-        for (int w = 0; w < NW; ++w) tot += sh->warp_a[w];
-        sh->base = tot ? atomicAdd(ctl + 4, tot) : 0u;
-    }
-    __syncthreads();
-    {   // append them to the row's list
-        const uint32_t at = sh->base + warp_sum_prefix(sh->warp_a, warp);
+    __syncwarp();
+    {   // append them to the row's list, one atomic per warp
+        uint32_t at = 0;
+        if (lane == 0 && wc) at = atomicAdd(ctl + 4, wc);
+        at = __shfl_sync(0xffffffffu, at, 0);
         uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
         for (uint32_t i = lane; i < wc; i += 32) {
             if (at + i < (uint32_t)p.list_cap) {
@@ -784,9 +780,11 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
             }
         }
     }
+    for (int j = threadIdx.x; j < 1024; j += NT) sh->hist[j] = 0;   // for digit 2, filled while the list loads
     if (!row_barrier<NT>(sh, ctl, (uint32_t)C, p.status)) return true;
 
-    // ---- the whole list into shared memory
+    // ---- the whole list into shared memory, with the digit-2 histogram of
+    //      the keys in the threshold bin on the way
     {
         const uint32_t *gkey = rs + list_base(C), *gpos = gkey + p.list_cap;
         for (uint32_t base = 0; base < m; base += 4 * NT) {
@@ -803,25 +801,29 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
                 if (j < m) {
                     lkey[j] = kv[u];
                     lpos[j] = pv[u];
+                    if ((kv[u] & mask) == prefix) atomicAdd(&sh->hist[(kv[u] >> 10) & 1023u], 1u);
                 }
             }
         }
+        __syncthreads();
     }
-    // ---- digits 2 and 3 on the list
+    // ---- digits 2 (histogram ready) and 3 on the list
 #pragma unroll 1
     for (int r = 0; r < 2; ++r) {
         const int shift = r == 0 ? 10 : 0, nb = 1024;
-        for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
-        __syncthreads();
-        for (uint32_t base = threadIdx.x; base < m; base += 4 * NT) {   // four loads in flight
-            uint32_t k4[4];
+        if (r == 1) {
+            for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+            __syncthreads();
+            for (uint32_t base = threadIdx.x; base < m; base += 4 * NT) {   // four loads in flight
+                uint32_t k4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) k4[u] = base + u * NT < m ? lkey[base + u * NT] : ~prefix;
+                for (int u = 0; u < 4; ++u) k4[u] = base + u * NT < m ? lkey[base + u * NT] : ~prefix;
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if ((k4[u] & mask) == prefix) atomicAdd(&sh->hist[(k4[u] >> shift) & (uint32_t)(nb - 1)], 1u);
+                for (int u = 0; u < 4; ++u)
+                    if ((k4[u] & mask) == prefix) atomicAdd(&sh->hist[(k4[u] >> shift) & (uint32_t)(nb - 1)], 1u);
+            }
+            __syncthreads();
         }
-        __syncthreads();
         find_threshold<NT>(sh, nb, Krem);
         prefix |= (uint32_t)sh->bin << shift;
         mask |= (uint32_t)(nb - 1) << shift;
