@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -80,13 +81,22 @@ def gathered_bytes(T: int, top_k: int, G: int = 4) -> int:
     return T * top_k * G * (192 + 128) * 2
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without its comments and trailing blanks (string literals
+    in these sources contain no comment markers)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_sources_sha() -> str:
-    """Hash of the CUDA sources the timed kernels are built from."""
+    """Hash of the code (comments excluded) of the CUDA sources the timed
+    kernels are built from."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
-            h.update(open(os.path.join(CSRC, name), "rb").read())
+            h.update(_strip_comments(open(os.path.join(CSRC, name)).read()).encode())
     return h.hexdigest()
 
 

@@ -9,14 +9,17 @@
 //
 // Grid: one CTA per SM (as the indexer), 640 threads each, all co-resident
 // (cooperative launch).
-//   phase 1  indexer body (indexer_impl.cuh); scores to the workspace and, when
-//            it fits, each CTA's first-digit histogram of its scores added into
-//            the rows' global histograms, which saves the selection one pass
-//            and one barrier;
-//   phase 2  selection (topk_impl.cuh): each query row is shared by
-//            C = grid / rows CTAs;
+//   phase 1  indexer body (indexer_impl.cuh); scores to the workspace and,
+//            for up to kMaxHistRows rows, each CTA's histogram of its scores
+//            (bits 30..20 of the non-negative keys, plus a count of the
+//            negative ones) added into the rows' global histograms;
+//   phase 2  selection (topk_impl.cuh), each query row shared by
+//            C = grid / rows CTAs: the one-barrier path from that histogram
+//            where the row qualifies, the general path otherwise;
 //   phase 3  attention units (attention_impl.cuh): four teams of four warps
-//            per CTA, one (query, KV head, 64-key split) unit per team at a time;
+//            per CTA, one (query, KV head, 64-key split) unit per team at a
+//            time, reading the -1-padded selection; the four other warps
+//            clear the selection scratch for the next call;
 //   phase 4  combine: one CTA per (query, head).
 #include <algorithm>
 
