@@ -17,8 +17,9 @@
 // the tensor cores (mma.sync m16n8k16 bf16 -> fp32; the query heads of a group
 // form the 16-row M dimension).  Each warp owns 16 keys; the four warps merge
 // their (max, sum, O) in shared memory and the team writes one partial.
-// combine_row: log-sum-exp merge of the partials of all splits plus the sink
-// term, normalisation, bf16 output and optional lse.
+// combine_row_cta: log-sum-exp merge of the partials of all splits plus the
+// sink term, normalisation, bf16 output and optional lse, one CTA per
+// (query, head).
 #pragma once
 
 #include <cmath>
@@ -308,54 +309,6 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
             }
         }
     }
-}
-
-// Merge of the splits of one (query, head) row gw by one warp, plus the sink,
-// normalised to bf16.  Lane j holds split j's (max, sum); the O partials are
-// read with all loads of a group independent of one another.  splits <= 32.
-__device__ __forceinline__ void combine_row(const float *part_o, const float *part_ml, int gw, int splits,
-                                            const float *sink, __nv_bfloat16 *O, float *lse) {
-    const int lane = lane_id();
-    const int h = gw % DSA_Q_HEADS;
-    const float *ml = part_ml + (int64_t)gw * splits * 2;
-    const float mj = lane < splits ? __ldcg(ml + 2 * lane) : -INFINITY;
-    const float lj = lane < splits ? __ldcg(ml + 2 * lane + 1) : 0.f;
-    const float sk = sink ? __ldg(sink + h) * kLog2e : -INFINITY;
-    float M = fmaxf(mj, sk);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float wj = (mj == -INFINITY) ? 0.f : exp2f(mj - M);
-    float L = lj * wj;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (sink && M != -INFINITY) L += exp2f(sk - M);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float *po = part_o + (int64_t)gw * splits * DSA_V_DIM + lane * 4;
-    for (int j0 = 0; j0 < splits; j0 += 8) {
-        float4 v[8];
-        float w[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = j0 + u;
-            w[u] = __shfl_sync(0xffffffffu, wj, j & 31);
-            v[u] = (j < splits && w[u] != 0.f) ? __ldcg(reinterpret_cast<const float4 *>(po + (int64_t)j * DSA_V_DIM))
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (j0 + u < splits && w[u] != 0.f) {
-                acc.x += v[u].x * w[u]; acc.y += v[u].y * w[u]; acc.z += v[u].z * w[u]; acc.w += v[u].w * w[u];
-            }
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t *>(&lo);
-    packed.y = *reinterpret_cast<uint32_t *>(&hi);
-    *reinterpret_cast<uint2 *>(O + (int64_t)gw * DSA_V_DIM + lane * 4) = packed;
-    if (lse && lane == 0) lse[gw] = (L > 0.f) ? (M + log2f(L)) / kLog2e : -INFINITY;
 }
 
 // Merge of the splits of one (query, head) row gw by a whole CTA of NT

@@ -43,7 +43,7 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream);
 namespace indexer { struct Params; }
 // Everything a launch of the indexer body needs: tensor maps, parameters,
 // dynamic shared memory and grid (one CTA per SM, two pipelines per CTA).  hist_rows > 0 adds each
-// CTA's first-digit histogram of the visible scores into hist_global.
+// CTA's histogram of the visible scores (see indexer::kHistWords) into hist_global.
 struct IndexerLaunch;
 int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uint32_t *hist_global,
                     size_t smem_budget, IndexerLaunch *out);
@@ -96,7 +96,7 @@ int launch_attention(const AttnArgs &a, cudaStream_t stream);
 // --------------------------------------------------------- fused layer-step
 struct FusedPlan {
     bool ok = false;            // false: use the separate kernels
-    int grid = 0;               // CTAs (two per SM)
+    int grid = 0;               // CTAs (one per SM)
     int rows = 0;               // B * T
     int C = 1;                  // CTAs per row in the selection phase
     size_t scratch_bytes = 0;   // grid barrier words + per-row selection scratch

@@ -8,18 +8,19 @@
 // full-attention layers' means" -- argsort(...)[..., :index_top_k] -- and "How
 // much of this did AI actually build?" -- the stable-tie argsort).
 //
-// Exact radix select on the order-preserving 32-bit image of each score, in
-// three digits (11 + 11 + 10 bits), giving the threshold key T* and the number
-// `ties` of keys equal to T* that are taken; the output is, in increasing
-// position order, every position with key > T* and the first `ties` positions
-// with key == T*.  C CTAs share a row, each owning a contiguous slice that it
-// keeps in shared memory when it fits.
+// Exact radix select on the order-preserving 32-bit image of each score,
+// giving the threshold key T* and the number `ties` of keys equal to T* that
+// are taken; the output is, in increasing position order, every position with
+// key > T* and the first `ties` positions with key == T*.  C CTAs share a row,
+// each owning a contiguous slice.  Two paths:
 //
-//   digit 1     the row's 2048-bin histogram of the top 11 bits -- built by the
-//               producer of the scores, or by the CTAs adding their slices'
-//               histograms into the row's global histogram and meeting at a
-//               barrier -- gives the threshold bin;
-//   digit 2     the same exchange for the next 11 bits of the keys in that bin;
+// General path (select_row; 11 + 11 + 10-bit digits), slices kept in shared
+// memory when they fit:
+//   digit 1     the CTAs add their slices' 2048-bin histograms of the top 11
+//               bits into the row's global histogram and meet at a barrier;
+//   digit 2     the same exchange for the next 11 bits of the keys in the
+//               threshold bin; in the same pass each warp keeps its candidates
+//               (keys at or above the threshold bin) in shared memory;
 //   list        every CTA appends its keys that share the threshold's top 22
 //               bits, with their positions, to the row's candidate list and
 //               publishes how many of its keys lie above them; one barrier;
@@ -29,11 +30,19 @@
 //               When the list does not fit in shared memory (many keys share
 //               the 22-bit bin, e.g. heavy ties), digit 3 is exchanged like the
 //               others, and so are the per-CTA (greater, equal) counts at T*;
-//   emission    each warp compacts its part of the slice with ballots, from its
-//               own offset in the row's output.
+//   emission    each warp compacts its candidates (or its part of the slice)
+//               with ballots, from its own offset in the row's output.
 //
-// The output is a pure function of the scores.  The last CTA of a row to leave
-// clears the row's scratch words for the next call.
+// One-barrier path (select_row_hist; fused kernel): the indexer has already
+// built the row's histogram of bits 30..20 (eight bins per octave) of the
+// non-negative keys.  The threshold bin comes from it; every key at or above
+// that bin goes, with its position, to a row-wide list; after one barrier each
+// CTA resolves the remaining 20 bits on the list in shared memory, takes its
+// offset from the list entries before its slice, and emits its candidates.
+//
+// The output is a pure function of the scores.  The row's scratch words are
+// zeroed again for the next call (by the last CTA to leave, or, in the fused
+// kernel, by clear_row_share / reset_row_ctl after a grid barrier).
 #pragma once
 
 #include "common.cuh"
