@@ -22,8 +22,12 @@
  *     memory of the current CUDA device.  The caller owns every buffer; the
  *     library allocates nothing.  Scratch memory is the caller's workspace
  *     (`ws`, `ws_bytes`); `dsa_workspace_size` gives the size each call needs.
- *     A workspace must be zero when first used (`dsa_workspace_init`); the
- *     calls leave it zeroed again when they finish.
+ *     A workspace must be zero when first used (`dsa_workspace_init`).  The
+ *     parts that must start at zero (the selection's cross-CTA scratch and
+ *     barrier words) are zeroed again by each call before it finishes; the
+ *     status word keeps device errors until `dsa_check_device_status` reads
+ *     it; scores, selections and attention partials are simply overwritten.
+ *     After a device error (a wait that ran out) re-initialise the workspace.
  *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *     default stream).  Host-side argument checks return before anything is
  *     enqueued.  Device-side checks (positions out of range, a bounded wait
