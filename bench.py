@@ -235,6 +235,18 @@ def read_stream_gbps(torch, dev, stream) -> float:
     return (1 << 30) / (best / 1e3) / 1e9
 
 
+def decode_config(workload: str, world: int) -> dict:
+    """The `config` object of a decode workload's line (both arms)."""
+    from workloads import CONFIGS
+    cfg = CONFIGS[workload]
+    return {
+        "workload": WORKLOAD_DESC[workload],
+        "batch": len(cfg["seq_lens"]), "query_tokens": cfg["T"], "context": max(cfg["seq_lens"]), "top_k": TOP_K,
+        "seed": cfg["seed"], "needles": cfg["n_needles"], "parallelism": f"replicas x{world}",
+        "l2": "flushed between steps outside the timed events (256 MB write, then 256 MB read so no dirty lines remain)",
+    }
+
+
 # ------------------------------------------------------ the ragged batch mix
 MIX_METRIC = "ragged 64-sequence decode layer-mix (5 SWA + 1 DSA layer-steps) tok/s"
 
@@ -536,12 +548,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
         "data": "synthetic",
-        "config": {
-            "workload": WORKLOAD_DESC[args.workload],
-            "batch": B, "query_tokens": T, "context": L, "top_k": TOP_K, "seed": cfg["seed"],
-            "needles": cfg["n_needles"], "parallelism": f"replicas x{world}",
-            "l2": "flushed between steps outside the timed events (256 MB write, then 256 MB read so no dirty lines remain)",
-        },
+        "config": decode_config(args.workload, world),
         "us_per_layer_step": total_s * 1e6 / K,
         "path": "one fused cooperative kernel" if fused else "four kernels",
         "stage_us_median": ({"fused_layer_step": statistics.median(step_ms) * 1e3} if fused else {
@@ -698,8 +705,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "ctx_1m: DSA decode layer-step, batch 1, 1 query token, context 1,048,576, "
-                               "top-2048, GQA4, sink", "context": L_CTX, "top_k": TOP_K},
+        "config": decode_config(WORKLOAD, world),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: the CPU oracle on the first {n} keys of the ctx_1m recipe, "
                                    f"indexer and selection scaled by {L_CTX}/{n}"},
