@@ -10,6 +10,7 @@ indexer scores -> top-k positions -> attention over the selected keys.
 """
 from .oracle import (  # noqa: F401
     build_oracle,
+    set_threads,
     e4m3_to_float64,
     bf16_to_float64,
     fp8_dot,
@@ -20,4 +21,10 @@ from .oracle import (  # noqa: F401
     swa_indices,
     dsa_layer_decode,
     swa_layer_decode,
+    layernorm,
+    rope_partial,
+    e4m3_encode,
+    index_k_produce,
+    index_q_produce,
+    indexer_kl,
 )

@@ -36,6 +36,29 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads: the loops over key positions (indexer) and over heads (attention)
+ * may run on several host threads.  Every output element is computed by one
+ * thread with the same loop order as on one thread, so the results do not
+ * depend on the thread count. */
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : 1);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* ---------------------------------------------------------------- formats */
 
@@ -89,6 +112,7 @@ void oracle_indexer_scores(const uint8_t *q8, const float *q_scale,
                            const float *k_scale, const int32_t *q_pos,
                            int T, int H, int D, int64_t L, float *scores) {
     for (int t = 0; t < T; ++t) {
+#pragma omp parallel for schedule(static)
         for (int64_t s = 0; s < L; ++s) {
             if (s > q_pos[t]) {
                 scores[(int64_t)t * L + s] = -INFINITY;
@@ -199,8 +223,9 @@ void oracle_gqa_attention(const uint16_t *Q, const uint16_t *K,
                           double sm_scale, double *out, double *lse) {
     (void)L;
     int hpg = H / G;
-    double *s = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+#pragma omp parallel for schedule(static)
     for (int h = 0; h < H; ++h) {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
         int g = h / hpg;
         double m = -INFINITY;
         for (int i = 0; i < n; ++i) {
@@ -218,6 +243,7 @@ void oracle_gqa_attention(const uint16_t *Q, const uint16_t *K,
         for (int d = 0; d < Dv; ++d) out[(int64_t)h * Dv + d] = 0.0;
         if (m == -INFINITY) {               /* nothing to attend to */
             if (lse) lse[h] = -INFINITY;
+            free(s);
             continue;
         }
         for (int i = 0; i < n; ++i) {
@@ -230,8 +256,8 @@ void oracle_gqa_attention(const uint16_t *Q, const uint16_t *K,
         if (sink) den += exp(sk - m);
         for (int d = 0; d < Dv; ++d) out[(int64_t)h * Dv + d] /= den;
         if (lse) lse[h] = m + log(den);
+        free(s);
     }
-    free(s);
 }
 
 /* Sliding-window index set of the query at 0-based position p: the keys with
@@ -244,4 +270,160 @@ int oracle_swa_indices(int64_t p, int window, int32_t *idx) {
     int n = 0;
     for (int64_t j = lo; j <= p; ++j) idx[n++] = (int32_t)j;
     return n;
+}
+
+/* ------------------------------------------- index-K / index-Q producer (f1) */
+
+/* The indexer's key path before the cache: "normalises the key, applies RoPE,
+ * rounds both to fp8_e4m3" [EXPL, "Inside a DSA layer: the lightning
+ * indexer"; its figure: LayerNorm, partial RoPE, FP8 quantization], with the
+ * partial rotary layout of the inherited attention block ("partial RoPE on a
+ * third of each head", a rope base of 10,000,000 on the sparse layers [EXPL,
+ * same section]).  The readings this follows where the page is silent:
+ *   - LayerNorm over the 128 dims with a learned weight and bias;
+ *   - RoPE on the first `rot` dims in the rotate-half arrangement: dim i and
+ *     dim i + rot/2 (i < rot/2) form a pair turned by the angle
+ *     pos * base^(-2i / rot); the other dims pass unchanged;
+ *   - e4m3 per token: scale = amax / 448 (1 for an all-zero token), value /
+ *     scale rounded to the nearest e4m3 value, ties to the even code,
+ *     saturating at +-448.
+ * Real arithmetic in double.  The quantisation decision is taken in fp32, as
+ * the kernel takes it: the rotated value is rounded to float, the scale is
+ * float(amax) / 448 in float, and the code is chosen for float(v / scale). */
+
+/* LayerNorm of x[0..D): (x - mean) / sqrt(var + eps) * w + b, var the
+ * population variance. */
+void oracle_layernorm(const double *x, int D, const float *w, const float *b, double eps, double *y) {
+    double mean = 0.0;
+    for (int i = 0; i < D; ++i) mean += x[i];
+    mean /= D;
+    double var = 0.0;
+    for (int i = 0; i < D; ++i) var += (x[i] - mean) * (x[i] - mean);
+    var /= D;
+    double inv = 1.0 / sqrt(var + eps);
+    for (int i = 0; i < D; ++i) y[i] = (x[i] - mean) * inv * (double)w[i] + (double)b[i];
+}
+
+/* Partial rotary embedding of x[0..D) at position pos, in place. */
+void oracle_rope_partial(double *x, int D, int rot, int64_t pos, double base) {
+    (void)D;
+    int h = rot / 2;
+    for (int i = 0; i < h; ++i) {
+        double inv_freq = pow(base, -2.0 * (double)i / (double)rot);
+        double ang = (double)pos * inv_freq;
+        double c = cos(ang), s = sin(ang);
+        double a = x[i], b = x[i + h];
+        x[i] = a * c - b * s;
+        x[i + h] = b * c + a * s;
+    }
+}
+
+/* The e4m3 code nearest to v (ties to the even code), saturating at +-448;
+ * the sign of v (also of a zero) is kept.  From the format definition: the
+ * candidates are the 127 non-negative finite codes 0x00..0x7E. */
+uint8_t oracle_e4m3_encode(float v) {
+    int neg = signbit(v) ? 1 : 0;
+    double a = fabs((double)v);
+    if (a >= 448.0) return (uint8_t)(0x7E | (neg << 7));
+    int best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(oracle_e4m3_to_double((uint8_t)c) - a);
+        if (d < bestd || (d == bestd && (c & 1) == 0)) {
+            bestd = d;
+            best = c;
+        }
+    }
+    return (uint8_t)(best | (neg << 7));
+}
+
+/* Per-token quantisation of n real values (rounded to float first). */
+static float oracle_quantize_token(const double *y, int n, uint8_t *codes) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float f = fabsf((float)y[i]);
+        if (f > amax) amax = f;
+    }
+    float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode((float)y[i] / scale);
+    return scale;
+}
+
+/* One token's index key: bf16 k[D] -> LayerNorm -> partial RoPE at pos ->
+ * e4m3 codes[D] and the token's scale.  y_out (optional) gets the real
+ * values before quantisation. */
+float oracle_index_k_produce(const uint16_t *k, const float *ln_w, const float *ln_b, double eps, int D, int rot,
+                             double base, int64_t pos, uint8_t *codes, double *y_out) {
+    double x[512], y[512];
+    for (int i = 0; i < D; ++i) x[i] = oracle_bf16_to_double(k[i]);
+    oracle_layernorm(x, D, ln_w, ln_b, eps, y);
+    oracle_rope_partial(y, D, rot, pos, base);
+    if (y_out)
+        for (int i = 0; i < D; ++i) y_out[i] = y[i];
+    return oracle_quantize_token(y, D, codes);
+}
+
+/* One token's index query: bf16 q[H][D] -> partial RoPE at pos on every head
+ * -> e4m3 codes[H][D] with one scale for the whole token (returned). */
+float oracle_index_q_produce(const uint16_t *q, int H, int D, int rot, double base, int64_t pos, uint8_t *codes,
+                             double *y_out) {
+    double *y = (double *)malloc(sizeof(double) * (size_t)H * D);
+    for (int h = 0; h < H; ++h) {
+        for (int i = 0; i < D; ++i) y[h * D + i] = oracle_bf16_to_double(q[h * D + i]);
+        oracle_rope_partial(y + h * D, D, rot, pos, base);
+    }
+    if (y_out)
+        for (int i = 0; i < H * D; ++i) y_out[i] = y[i];
+    float s = oracle_quantize_token(y, H * D, codes);
+    free(y);
+    return s;
+}
+
+/* --------------------------------------- indexer warm-up KL target (f4) */
+
+/* The indexer warm-up trains only the indexer, "aligned to a full-attention
+ * reference by a KL objective" [EXPL, "Inside a DSA layer: the lightning
+ * indexer"; BLOG, "What's genuinely new": the layers being converted keep
+ * full attention and supervise the indexer through a KL-divergence loss].
+ * Reading (the pages give no formula): for a query token at position p,
+ * over its visible keys s = 0..p,
+ *   target  P[s] = (1/H) sum_h softmax_s(sm_scale * Q[h] . K[s][h / (H/G)])
+ *           (each head's dense attention distribution over the keys, no
+ *           sink, averaged over the H heads),
+ *   indexer R[s] = softmax_s(I[s]) of the indexer scores,
+ *   loss    KL(P || R) = sum_s P[s] (log P[s] - log R[s]).
+ * Q [H][Dk] bf16; K [L][G][Dk] bf16 (rows 0..p are the visible keys);
+ * I [p + 1] indexer scores.  Writes P[0..p] and returns the KL. */
+double oracle_indexer_kl(const uint16_t *Q, const uint16_t *K, int H, int G, int Dk, const float *I, int64_t p,
+                         double sm_scale, double *P) {
+    int64_t n = p + 1;
+    int hpg = H / G;
+    double *s = (double *)malloc(sizeof(double) * (size_t)n);
+    for (int64_t j = 0; j < n; ++j) P[j] = 0.0;
+    for (int h = 0; h < H; ++h) {
+        int g = h / hpg;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            const uint16_t *kr = K + (j * G + g) * Dk;
+            double dot = 0.0;
+            for (int d = 0; d < Dk; ++d)
+                dot += oracle_bf16_to_double(Q[(int64_t)h * Dk + d]) * oracle_bf16_to_double(kr[d]);
+            s[j] = sm_scale * dot;
+            if (s[j] > m) m = s[j];
+        }
+        double den = 0.0;
+        for (int64_t j = 0; j < n; ++j) den += exp(s[j] - m);
+        for (int64_t j = 0; j < n; ++j) P[j] += exp(s[j] - m) / den / H;
+    }
+    free(s);
+    double mi = -INFINITY;
+    for (int64_t j = 0; j < n; ++j)
+        if ((double)I[j] > mi) mi = (double)I[j];
+    double li = 0.0;
+    for (int64_t j = 0; j < n; ++j) li += exp((double)I[j] - mi);
+    double lse_i = mi + log(li);
+    double kl = 0.0;
+    for (int64_t j = 0; j < n; ++j)
+        if (P[j] > 0.0) kl += P[j] * (log(P[j]) - ((double)I[j] - lse_i));
+    return kl;
 }

@@ -14,11 +14,12 @@ _lib = None
 
 
 def build_oracle(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so with gcc (plain -O2, one thread)."""
+    """Compile oracle.c into liboracle.so with gcc (plain -O2; OpenMP for the
+    loops over positions and heads, one thread unless set_threads says more)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp.%d" % os.getpid()
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -47,6 +48,26 @@ def _load():
                                              ctypes.c_double, P, P]
         lib.oracle_swa_indices.restype = ctypes.c_int
         lib.oracle_swa_indices.argtypes = [ctypes.c_int64, ctypes.c_int, P]
+        lib.oracle_layernorm.restype = None
+        lib.oracle_layernorm.argtypes = [P, ctypes.c_int, P, P, ctypes.c_double, P]
+        lib.oracle_rope_partial.restype = None
+        lib.oracle_rope_partial.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_double]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_index_k_produce.restype = ctypes.c_float
+        lib.oracle_index_k_produce.argtypes = [P, P, P, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                               ctypes.c_int64, P, P]
+        lib.oracle_index_q_produce.restype = ctypes.c_float
+        lib.oracle_index_q_produce.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                               ctypes.c_int64, P, P]
+        lib.oracle_indexer_kl.restype = ctypes.c_double
+        lib.oracle_indexer_kl.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, ctypes.c_int64,
+                                          ctypes.c_double, P]
+        lib.oracle_set_threads.restype = None
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_set_threads(1)   # one thread unless asked (results do not depend on it)
         _lib = lib
     return _lib
 
@@ -54,6 +75,13 @@ def _load():
 def _c(a, dtype):
     a = np.ascontiguousarray(a, dtype=dtype)
     return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> int:
+    """Host threads for the position / head loops; returns the count in use."""
+    lib = _load()
+    lib.oracle_set_threads(int(n))
+    return lib.oracle_max_threads()
 
 
 def e4m3_to_float64(codes) -> np.ndarray:
@@ -186,3 +214,69 @@ def swa_layer_decode(Q, K, V, q_pos, window, sink, sm_scale):
         idx = swa_indices(int(q_pos[t]), window)
         out[t], lse[t] = gqa_attention(Q[t], K, V, idx, sink, sm_scale)
     return dict(out=out, lse=lse)
+
+
+# ------------------------------------------------ index-K / index-Q producer
+def layernorm(x, w, b, eps: float) -> np.ndarray:
+    lib = _load()
+    x, px = _c(x, np.float64)
+    w, pw = _c(w, np.float32)
+    b, pb = _c(b, np.float32)
+    y = np.empty_like(x)
+    lib.oracle_layernorm(px, x.shape[0], pw, pb, float(eps), y.ctypes.data_as(ctypes.c_void_p))
+    return y
+
+
+def rope_partial(x, rot: int, pos: int, base: float) -> np.ndarray:
+    lib = _load()
+    y = np.ascontiguousarray(x, dtype=np.float64).copy()
+    lib.oracle_rope_partial(y.ctypes.data_as(ctypes.c_void_p), y.shape[0], int(rot), int(pos), float(base))
+    return y
+
+
+def e4m3_encode(v) -> np.ndarray:
+    lib = _load()
+    v = np.asarray(v, dtype=np.float32)
+    return np.array([lib.oracle_e4m3_encode(float(x)) for x in v.reshape(-1)], dtype=np.uint8).reshape(v.shape)
+
+
+def index_k_produce(k_bits, ln_w, ln_b, eps: float, rot: int, base: float, pos: int):
+    """One token's index key: bf16 bits k [D] -> (codes [D] uint8, scale, y [D] before quantisation)."""
+    lib = _load()
+    k, pk = _c(k_bits, np.uint16)
+    w, pw = _c(ln_w, np.float32)
+    b, pb = _c(ln_b, np.float32)
+    D = k.shape[0]
+    codes = np.empty(D, np.uint8)
+    y = np.empty(D, np.float64)
+    s = lib.oracle_index_k_produce(pk, pw, pb, float(eps), D, int(rot), float(base), int(pos),
+                                   codes.ctypes.data_as(ctypes.c_void_p), y.ctypes.data_as(ctypes.c_void_p))
+    return codes, float(np.float32(s)), y
+
+
+def index_q_produce(q_bits, rot: int, base: float, pos: int):
+    """One token's index query: bf16 bits q [H, D] -> (codes [H, D], scale, y [H, D])."""
+    lib = _load()
+    q, pq = _c(q_bits, np.uint16)
+    H, D = q.shape
+    codes = np.empty((H, D), np.uint8)
+    y = np.empty((H, D), np.float64)
+    s = lib.oracle_index_q_produce(pq, H, D, int(rot), float(base), int(pos),
+                                   codes.ctypes.data_as(ctypes.c_void_p), y.ctypes.data_as(ctypes.c_void_p))
+    return codes, float(np.float32(s)), y
+
+
+# ------------------------------------------------ indexer warm-up KL target
+def indexer_kl(Q_bits, K_bits, I, p: int, sm_scale: float):
+    """One query token at position p: Q [H, Dk] bf16 bits, K [L, G, Dk] bf16
+    bits (rows 0..p visible), I [>= p + 1] indexer scores.  Returns (KL, P [p + 1])."""
+    lib = _load()
+    Q, pQ = _c(Q_bits, np.uint16)
+    K = np.ascontiguousarray(K_bits, dtype=np.uint16)
+    H, Dk = Q.shape
+    G = K.shape[1]
+    I, pI = _c(np.asarray(I)[: p + 1], np.float32)
+    P = np.empty(p + 1, np.float64)
+    kl = lib.oracle_indexer_kl(pQ, K.ctypes.data_as(ctypes.c_void_p), H, G, Dk, pI, int(p), float(sm_scale),
+                               P.ctypes.data_as(ctypes.c_void_p))
+    return float(kl), P

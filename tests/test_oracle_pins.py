@@ -373,3 +373,174 @@ def test_stack_constants_from_the_pages():
     W, K, Lmax = int(g["sliding_window"][0]), int(g["index_top_k"][0]), int(g["max_position_embeddings"][0])
     assert 39 * W + 9 * K == int(g["backbone_keys_per_token_sparse"][0])
     assert 39 * W + 9 * Lmax == int(g["backbone_keys_per_token_if_dense"][0])
+
+
+def test_oracle_results_do_not_depend_on_the_thread_count():
+    """The all-core timing of the oracle computes the same numbers as one
+    thread: each score and each head's output keeps its own summation order."""
+    from workloads import bits16, make_decode_workload
+    wl = make_decode_workload(seed=5, seq_lens=[5000], T=2, n_needles=4)
+    args = (wl.q8[0].numpy(), wl.q_scale[0].numpy(), wl.w[0].numpy(), wl.k8.numpy(), wl.k_scale.numpy(),
+            wl.q_pos[0].numpy())
+    sel = np.arange(0, 5000, 3, dtype=np.int32)
+    try:
+        oracle.set_threads(1)
+        s1 = oracle.indexer_scores(*args)
+        o1, l1 = oracle.gqa_attention(bits16(wl.Q[0, 0]), bits16(wl.K), bits16(wl.V), sel, wl.sink.numpy(), 0.07)
+        oracle.set_threads(4)
+        s4 = oracle.indexer_scores(*args)
+        o4, l4 = oracle.gqa_attention(bits16(wl.Q[0, 0]), bits16(wl.K), bits16(wl.V), sel, wl.sink.numpy(), 0.07)
+    finally:
+        oracle.set_threads(1)
+    assert np.array_equal(s1.view(np.uint32), s4.view(np.uint32))
+    assert np.array_equal(o1, o4) and np.array_equal(l1, l4)
+
+
+# ------------------------------------------------- index-K / index-Q producer
+def _bf16_bits(values):
+    return bits16(torch.tensor([float(v) for v in values], dtype=torch.float32).to(torch.bfloat16))
+
+
+def test_index_key_producer_hand_worked_example():
+    g = load_golden("index_producer_worked_example.txt")
+    k = _bf16_bits(g["k_bf16_values"])
+    ones, zeros = np.ones(4, np.float32), np.zeros(4, np.float32)
+    codes, scale, y = oracle.index_k_produce(k, ones, zeros, 0.0, int(g["k_rot"][0]), float(g["k_base"][0]),
+                                             int(g["k_pos"][0]))
+    assert np.allclose(y, _floats(g["k_y"]).astype(np.float64), rtol=0, atol=1e-9 + 1e-6)
+    assert scale == np.float32(float(g["k_scale"][0]))
+    assert np.array_equal(codes, _codes(g["k_codes"]))
+
+
+def test_index_query_producer_hand_worked_example():
+    g = load_golden("index_producer_worked_example.txt")
+    q = _bf16_bits(g["q_bf16_values"]).reshape(2, 4)
+    codes, scale, y = oracle.index_q_produce(q, int(g["q_rot"][0]), float(g["q_base"][0]), int(g["q_pos"][0]))
+    assert np.allclose(y.reshape(-1), _floats(g["q_y"]).astype(np.float64), atol=1e-6)
+    assert scale == np.float32(float(g["q_scale"][0]))
+    assert np.array_equal(codes.reshape(-1), _codes(g["q_codes"]))   # includes a tie broken to the even code
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    """Round-to-nearest-even onto the e4m3 grid, checked against torch's
+    float8_e4m3fn conversion on random values, every grid point and every
+    midpoint between neighbours (within +-448, where torch does not saturate)."""
+    grid = torch.arange(0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mids = (grid[1:] + grid[:-1]) / 2
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([grid, mids, rng.uniform(-448, 448, 3000), rng.normal(0, 1, 3000),
+                           rng.normal(0, 1e-3, 1000)]).astype(np.float32)
+    vals = np.concatenate([vals, -vals])
+    mine = oracle.e4m3_encode(vals)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(mine, ref)
+    assert list(oracle.e4m3_encode(np.array([448.0, 449.0, 1e6, -1e6], np.float32))) == [0x7E, 0x7E, 0x7E, 0xFE]
+
+
+def test_layernorm_closed_forms():
+    rng = np.random.default_rng(4)
+    x = rng.normal(3.0, 2.0, 128)
+    ones, zeros = np.ones(128, np.float32), np.zeros(128, np.float32)
+    y = oracle.layernorm(x, ones, zeros, 0.0)
+    assert abs(y.mean()) < 1e-12 and abs((y * y).mean() - 1.0) < 1e-12
+    # invariant under x -> a x + c (a > 0) without eps
+    assert np.allclose(oracle.layernorm(2.5 * x - 7.0, ones, zeros, 0.0), y, atol=1e-12)
+    # weight and bias act per dimension after the normalisation
+    w = rng.uniform(0.5, 2, 128).astype(np.float32)
+    b = rng.normal(0, 1, 128).astype(np.float32)
+    assert np.allclose(oracle.layernorm(x, w, b, 0.0), y * w + b, atol=1e-12)
+    # eps enters as sqrt(var + eps)
+    var = x.var()
+    assert np.allclose(oracle.layernorm(x, ones, zeros, 0.5), (x - x.mean()) / np.sqrt(var + 0.5), atol=1e-12)
+
+
+def test_partial_rope_is_a_complex_rotation_of_the_half_pairs():
+    """Pairs (i, i + rot/2) as complex numbers x_i + i x_{i+h} multiplied by
+    exp(i pos base^(-2i/rot)); the dims past rot unchanged."""
+    rng = np.random.default_rng(6)
+    D, rot, base = 128, 42, 1e7
+    x = rng.normal(0, 1, D)
+    for pos in (0, 1, 17, 65535, 1048575):
+        y = oracle.rope_partial(x, rot, pos, base)
+        h = rot // 2
+        z = (x[:h] + 1j * x[h:rot]) * np.exp(1j * pos * base ** (-2.0 * np.arange(h) / rot))
+        assert np.allclose(y[:h], z.real, atol=1e-9) and np.allclose(y[h:rot], z.imag, atol=1e-9)
+        assert np.array_equal(y[rot:], x[rot:])
+    assert np.array_equal(oracle.rope_partial(x, 0, 12345, base), x)
+
+
+def test_partial_rope_depends_on_relative_position_only():
+    rng = np.random.default_rng(7)
+    q, k = rng.normal(0, 1, 128), rng.normal(0, 1, 128)
+    rot, base = 42, 1e7
+    d1 = oracle.rope_partial(q, rot, 1000, base) @ oracle.rope_partial(k, rot, 700, base)
+    d2 = oracle.rope_partial(q, rot, 51300, base) @ oracle.rope_partial(k, rot, 51000, base)
+    assert abs(d1 - d2) < 1e-9
+    back = oracle.rope_partial(oracle.rope_partial(q, rot, 777, base), rot, -777, base)
+    assert np.allclose(back, q, atol=1e-12)
+
+
+def test_producer_scale_maps_the_largest_magnitude_to_448():
+    rng = np.random.default_rng(8)
+    k = bits16(torch.from_numpy(rng.normal(0, 1, 128).astype(np.float32)).to(torch.bfloat16))
+    w = rng.uniform(0.5, 1.5, 128).astype(np.float32)
+    b = rng.normal(0, 0.1, 128).astype(np.float32)
+    codes, scale, y = oracle.index_k_produce(k, w, b, 1e-5, 42, 1e7, 123456)
+    y32 = y.astype(np.float32)
+    assert scale == np.float32(np.abs(y32).max()) / np.float32(448.0)
+    assert codes[np.argmax(np.abs(y32))] & 0x7F == 0x7E
+    # dequantised codes reproduce the values within half an e4m3 step (relative 1/16) or the subnormal step
+    deq = oracle.e4m3_to_float64(codes) * scale
+    assert np.all(np.abs(deq - y) <= np.maximum(np.abs(y) / 16, scale * 2.0 ** -10) + 1e-7)
+
+
+# --------------------------------------------- indexer warm-up KL target
+def _kl_inputs(seed, n, H=8, G=2, Dk=16, std=1.0):
+    rng = np.random.default_rng(seed)
+    Q = bits16(torch.from_numpy(rng.normal(0, std, (H, Dk)).astype(np.float32)).to(torch.bfloat16))
+    K = bits16(torch.from_numpy(rng.normal(0, std, (n, G, Dk)).astype(np.float32)).to(torch.bfloat16))
+    I = rng.normal(0, 2, n).astype(np.float32)
+    return Q, K, I
+
+
+def test_kl_target_is_the_head_mean_of_softmax_attention():
+    """The target equals torch's float64 softmax of the scaled logits, averaged
+    over heads; each head reads its contiguous KV group."""
+    Q, K, I = _kl_inputs(1, 300)
+    sm = 0.25
+    kl, P = oracle.indexer_kl(Q, K, I, 299, sm)
+    q = torch.from_numpy(oracle.bf16_to_float64(Q))
+    k = torch.from_numpy(oracle.bf16_to_float64(K))
+    H, G = q.shape[0], k.shape[1]
+    logits = torch.stack([sm * k[:, h // (H // G)] @ q[h] for h in range(H)])
+    ref = torch.softmax(logits, dim=-1).mean(0).numpy()
+    assert np.allclose(P, ref, rtol=1e-12, atol=1e-15)
+    assert abs(P.sum() - 1.0) < 1e-12
+    r = torch.log_softmax(torch.from_numpy(I.astype(np.float64)), 0).numpy()
+    assert abs(kl - float((ref * (np.log(ref) - r)).sum())) < 1e-12
+    # a strided head -> KV mapping gives a different target
+    logits_s = torch.stack([sm * k[:, h % G] @ q[h] for h in range(H)])
+    assert not np.allclose(P, torch.softmax(logits_s, dim=-1).mean(0).numpy(), atol=1e-6)
+
+
+def test_kl_is_zero_when_the_indexer_matches_the_target():
+    Q, K, I = _kl_inputs(2, 200)
+    _, P = oracle.indexer_kl(Q, K, I, 199, 0.3)
+    kl, _ = oracle.indexer_kl(Q, K, (np.log(P) + 5.0).astype(np.float32), 199, 0.3)
+    assert abs(kl) < 1e-6                      # float32 rounding of the matched scores only
+    kl1, _ = oracle.indexer_kl(Q, K, I, 0, 0.3)   # a single visible key: both distributions are [1]
+    assert kl1 == 0.0
+
+
+def test_kl_closed_form_for_uniform_attention_and_shift_invariance():
+    Q, K, I = _kl_inputs(3, 500)
+    Qz = np.zeros_like(Q)                      # every logit 0: each head uniform over the keys
+    n = 400
+    kl, P = oracle.indexer_kl(Qz, K, I, n - 1, 0.1)
+    i = I[:n].astype(np.float64)
+    lse = i.max() + np.log(np.exp(i - i.max()).sum())
+    assert np.allclose(P, 1.0 / n)
+    assert abs(kl - (-np.log(n) - i.mean() + lse)) < 1e-10
+    kl2, _ = oracle.indexer_kl(Qz, K, I + np.float32(3.0), n - 1, 0.1)
+    assert abs(kl2 - kl) < 1e-6
+    assert kl > 0
