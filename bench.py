@@ -324,6 +324,19 @@ def run_mix(args, rank, world, local_rank):
         eager[i][1].record(stream)
     torch.cuda.synchronize(dev)
     eager_us = statistics.median([a.elapsed_time(b) for a, b in eager]) * 1e3
+    # the same mix as one dsa_layer_chain (programmatic dependent launches)
+    chain_steps = [dsa.swa_step(s.Q, k, s.q_pos, 128, s.sink, sm_scale, O, None, ws_swa) for s, k in zip(swa, swa_kv)]
+    chain_steps.append(dsa.dsa_step(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, Lmax, TOP_K, wl.sink, sm_scale, O,
+                                    None, idx, cnt, ws))
+    chained = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush()
+        torch.cuda._sleep(sleep_cycles)
+        chained[i][0].record(stream)
+        dsa.dsa_layer_chain(chain_steps)
+        chained[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    chained_us = statistics.median([a.elapsed_time(b) for a, b in chained]) * 1e3
     med = lambda xs: statistics.median(xs) * 1e3
     stage_us = {"swa_x5": med([ev[i][0].elapsed_time(stages[i][0]) for i in range(K)]),
                 "dsa_indexer": med([stages[i][0].elapsed_time(stages[i][1]) for i in range(K)]),
@@ -352,13 +365,121 @@ def run_mix(args, rank, world, local_rank):
         "us_per_mix": total_s * 1e6 / K,
         "timing": "device time: the mix is fully enqueued before its first event (host ahead)",
         "us_per_mix_eager_median": eager_us,
+        "us_per_mix_chained": chained_us,
         "stage_us_median": stage_us,
         "roofline": {"kernel": "whole mix (5 swa_attn_decode + dsa_layer_decode launches)", "bound": "hbm",
                      "achieved": mix_bytes / (total_s / K) / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": mix_bytes / (total_s / K) / 1e9 / peak, "peak_kind": peak_kind, "traffic": None,
                      "algorithmic_bytes_per_launch": mix_bytes},
         "e2e": None,
-        "gpu_launches": (5 * 2 + 4) * K,
+        "gpu_launches": (5 + 4) * K,   # one kernel per SWA step, four for the 64-row DSA step
+        "clocks": clocks,
+    }
+
+
+# ---------------------------------------------------- the layer stack step
+STACK_METRIC = "attention-only decode stack step (39 SWA + 9 DSA layer-steps) at 1M context, tok/s"
+DSA_LAYERS = (0, 5, 11, 17, 23, 29, 35, 41, 47)   # the layer pattern: 48 layers, DSA at these
+
+
+def run_stack(args, rank, world, local_rank):
+    """One step = the attention of every layer of the stack for one new token
+    at 1,048,576 context: 48 layer-steps in the layer pattern's order, each DSA
+    layer with its own 1M-context cache (index keys, K, V), each SWA layer its
+    own window-only cache; enqueued as one dsa_layer_chain (the timed value)
+    and as 48 separate calls (reported beside it).  L2 flushed before each
+    stack step, not between layers."""
+    import torch
+    import local_attention_decode_b200 as dsa
+    from workloads import CONFIGS, make_decode_workload, make_swa_window_workload
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = dict(CONFIGS["ctx_1m"])
+    L = cfg["seq_lens"][0]
+    sm_scale = 1.0 / math.sqrt(192)
+    steps, keep = [], []
+    O = torch.empty((1, 1, 64, 128), dtype=torch.bfloat16, device=dev)
+    ws_swa = dsa.alloc_workspace(dsa.OP_SWA_ATTN, 1, 1, 1, 128, device=dev)
+    ws_dsa = dsa.alloc_workspace(dsa.OP_LAYER, 1, 1, L, TOP_K, device=dev)
+    calls = []
+    for layer in range(48):
+        if layer in DSA_LAYERS:
+            wl = make_decode_workload(device=dev, **dict(cfg, seed=1000 + layer))
+            kv = dsa.KV(k=wl.K, v=wl.V, index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G,
+                        seq_stride=wl.layout.seq_stride, num_rows=wl.layout.num_rows)
+            steps.append(dsa.dsa_step(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, L, TOP_K, wl.sink, sm_scale, O,
+                                      None, None, None, ws_dsa))
+            calls.append(lambda wl=wl, kv=kv: dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, L,
+                                                                   TOP_K, wl.sink, sm_scale, O, ws=ws_dsa))
+        else:
+            wl = make_swa_window_workload(2000 + layer, [L], device=dev)
+            kv = dsa.KV(k=wl.K, v=wl.V, num_kv_heads=wl.G, block_table=wl.layout.block_table,
+                        page_size=wl.layout.page_size, num_rows=wl.layout.num_rows)
+            steps.append(dsa.swa_step(wl.Q, kv, wl.q_pos, 128, wl.sink, sm_scale, O, None, ws_swa))
+            calls.append(lambda wl=wl, kv=kv: dsa.swa_attn_decode(wl.Q, kv, wl.q_pos, 128, wl.sink, sm_scale, O,
+                                                                  None, ws_swa))
+        keep.append((wl, kv))
+    flush = L2Flush(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def chained():
+        dsa.dsa_layer_chain(steps)
+
+    def eager():
+        for c in calls:
+            c()
+
+    def timed(fn, K):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            flush()
+            torch.cuda._sleep(4_000_000)   # the host enqueues the whole stack ahead of the GPU
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return [a.elapsed_time(b) for a, b in ev]
+
+    for _ in range(args.warmup):
+        flush()
+        chained()
+        eager()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    barrier(dev)
+    sampler.start()
+    ms = timed(chained, K)
+    barrier(dev)
+    clocks = sampler.stop()
+    ms_eager = timed(eager, K)
+    for w_ in (ws_swa, ws_dsa):
+        st, _ = dsa.dsa_check_device_status(w_)
+        if st != dsa.DSA_OK:
+            raise RuntimeError(f"device status {st} after the stack steps")
+    total_s = max_over_ranks(sum(ms) / 1e3, dev)
+    peak, peak_kind = measured_peaks()
+    dsa_bytes = len(DSA_LAYERS) * (indexer_bytes(L, 1) + gathered_bytes(1, TOP_K))
+    swa_bytes = (48 - len(DSA_LAYERS)) * 128 * 8 * (192 + 128) * 2
+    step_s = total_s / K
+    return {
+        "metric": STACK_METRIC, "value": throughput(1, K, world, total_s), "unit": "tok/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
+        "data": "synthetic",
+        "config": {"workload": "48 layer-steps of one decode token at 1,048,576 context: DSA (top-2048, GQA4, sink) "
+                               "at layers 0, 5, 11, 17, 23, 29, 35, 41, 47, SWA (window 128, GQA8, sink) at the "
+                               "other 39; each layer its own cache", "parallelism": f"replicas x{world}",
+                   "l2": "flushed before each stack step outside the timed events"},
+        "us_per_stack_chained": step_s * 1e6,
+        "us_per_stack_eager_median": statistics.median(ms_eager) * 1e3,
+        "roofline": {"kernel": "whole stack (9 DSA + 39 SWA layer-steps)", "bound": "hbm",
+                     "achieved": (dsa_bytes + swa_bytes) / step_s / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": (dsa_bytes + swa_bytes) / step_s / 1e9 / peak, "peak_kind": peak_kind, "traffic": None,
+                     "algorithmic_bytes_per_launch": dsa_bytes + swa_bytes},
+        "e2e": None,
+        "gpu_launches": None,
         "clocks": clocks,
     }
 
@@ -525,6 +646,9 @@ def run_ours(args, rank, world, local_rank):
     iev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
     for i in range(3 + K2):
         flush()
+        # a bounded GPU sleep (outside the events) holds the stream while the
+        # host prepares the call, so the events see only the kernel
+        torch.cuda._sleep(200_000)
         if i >= 3:
             iev[i - 3][0].record(stream)
         dsa.dsa_indexer_scores(wl.q8, wl.q_scale, wl.w, ikv, wl.q_pos, L, scores, idx_ws)
@@ -596,51 +720,72 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": (1 if fused else 4) * K,
         "clocks": clocks,
+        "_workload": wl,
     }
     return line
 
 
 def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
-    """Same metric through the public API with host buffers: per step the new
-    token's inputs (index query + scales + weights, backbone query, position,
-    and its index-key / K / V cache row) go host -> device from pinned memory,
-    the layer-step runs, and the output and selection come back to the host."""
+    """Same metric through the public API with host buffers.  Per step, the new
+    token's raw inputs -- its index query (16 heads) and index key before
+    normalisation, RoPE and fp8 (bf16), the head weights, the backbone query,
+    its position, and its backbone K / V rows -- go host -> device in one copy
+    from pinned memory; dsa_index_produce normalises, rotates and quantises the
+    index key into the cache row and the index queries into their e4m3 codes;
+    the K / V rows are written into the cache; the layer-step runs; the output
+    and the selection come back to the host in one copy."""
     B, T = wl.B, wl.T
     L = wl.layout.seq_lens[0]
+    G = wl.G
     row = L - 1
-    h_q8 = wl.q8.cpu().pin_memory()
-    h_qs = wl.q_scale.cpu().pin_memory()
-    h_w = wl.w.cpu().pin_memory()
-    h_Q = wl.Q.cpu().pin_memory()
-    h_pos = wl.q_pos.cpu().pin_memory()
-    h_k8 = wl.k8[row].cpu().pin_memory()
-    h_ks = wl.k_scale[row:row + 1].cpu().pin_memory()
-    h_K = wl.K[row].cpu().pin_memory()
-    h_V = wl.V[row].cpu().pin_memory()
-    d_q8, d_qs, d_w = torch.empty_like(wl.q8), torch.empty_like(wl.q_scale), torch.empty_like(wl.w)
-    d_Q, d_pos = torch.empty_like(wl.Q), torch.empty_like(wl.q_pos)
-    O = torch.empty((B, T, 64, 128), dtype=torch.bfloat16, device=dev)
-    idx = torch.empty((B, T, TOP_K), dtype=torch.int32, device=dev)
+    g = torch.Generator(device="cpu").manual_seed(77)
+    # packed per-step input: each part 256-byte aligned inside one buffer
+    parts = [("q_in", torch.bfloat16, (B, T, 16, 128)), ("k_in", torch.bfloat16, (B, T, 128)),
+             ("w", torch.float32, (B, T, 16)), ("Q", torch.bfloat16, (B, T, 64, 192)),
+             ("pos", torch.int32, (B, T)), ("K", torch.bfloat16, (G, 192)), ("V", torch.bfloat16, (G, 128))]
+    offs, off = {}, 0
+    for name, dt, shape in parts:
+        nbytes = math.prod(shape) * torch.tensor([], dtype=dt).element_size()
+        offs[name] = (off, dt, shape, nbytes)
+        off = (off + nbytes + 255) // 256 * 256
+    h_in = torch.empty(off, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(off, dtype=torch.uint8, device=dev)
+
+    def view(buf, name):
+        o, dt, shape, nbytes = offs[name]
+        return buf[o:o + nbytes].view(dt).view(shape)
+
+    view(h_in, "q_in").copy_(torch.randn((B, T, 16, 128), generator=g).to(torch.bfloat16))
+    view(h_in, "k_in").copy_(torch.randn((B, T, 128), generator=g).to(torch.bfloat16))
+    view(h_in, "w").copy_(wl.w.cpu())
+    view(h_in, "Q").copy_(wl.Q.cpu())
+    view(h_in, "pos").copy_(wl.q_pos.cpu())
+    view(h_in, "K").copy_(wl.K[row].cpu())
+    view(h_in, "V").copy_(wl.V[row].cpu())
+    d_qin, d_kin, d_w, d_Q, d_pos, d_K, d_V = (view(d_in, n) for n, _, _ in parts)
+    ln_w = torch.ones(128, device=dev)
+    ln_b = torch.zeros(128, device=dev)
+    q8 = torch.empty((B, T, 16, 128), dtype=torch.uint8, device=dev)
+    qs = torch.empty((B, T, 16), dtype=torch.float32, device=dev)
+    ws_p = dsa.alloc_workspace(dsa.OP_PRODUCE, B, T, 1, 1, device=dev)
+    # outputs: O and the selection in one device buffer, read back in one copy
+    o_bytes = B * T * 64 * 128 * 2
+    i_bytes = B * T * TOP_K * 4
+    d_out = torch.empty(o_bytes + i_bytes, dtype=torch.uint8, device=dev)
+    h_out = torch.empty(o_bytes + i_bytes, dtype=torch.uint8).pin_memory()
+    O = d_out[:o_bytes].view(torch.bfloat16).view(B, T, 64, 128)
+    idx = d_out[o_bytes:].view(torch.int32).view(B, T, TOP_K)
     cnt = torch.empty((B, T), dtype=torch.int32, device=dev)
-    h_O = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-    h_idx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    h_in = [h_q8, h_qs, h_w, h_Q, h_pos, h_k8, h_ks, h_K, h_V]
-    h2d = sum(t.numel() * t.element_size() for t in h_in)
-    d2h = h_O.numel() * h_O.element_size() + h_idx.numel() * h_idx.element_size()
+    h2d = off
+    d2h = o_bytes + i_bytes
 
     def step():
-        d_q8.copy_(h_q8, non_blocking=True)
-        d_qs.copy_(h_qs, non_blocking=True)
-        d_w.copy_(h_w, non_blocking=True)
-        d_Q.copy_(h_Q, non_blocking=True)
-        d_pos.copy_(h_pos, non_blocking=True)
-        wl.k8[row].copy_(h_k8, non_blocking=True)
-        wl.k_scale[row:row + 1].copy_(h_ks, non_blocking=True)
-        wl.K[row].copy_(h_K, non_blocking=True)
-        wl.V[row].copy_(h_V, non_blocking=True)
-        dsa.dsa_layer_decode(d_q8, d_qs, d_w, d_Q, kv, d_pos, L, TOP_K, wl.sink, sm_scale, O, None, idx, cnt, ws)
-        h_O.copy_(O, non_blocking=True)
-        h_idx.copy_(idx, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
+        dsa.dsa_index_produce(d_kin, d_qin, ln_w, ln_b, 1e-5, 42, 1e7, kv, d_pos, q8, qs, ws_p)
+        wl.K[row].copy_(d_K, non_blocking=True)
+        wl.V[row].copy_(d_V, non_blocking=True)
+        dsa.dsa_layer_decode(q8, qs, d_w, d_Q, kv, d_pos, L, TOP_K, wl.sink, sm_scale, O, None, idx, cnt, ws)
+        h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
         flush()
@@ -657,75 +802,136 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
         evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier(dev)
+    for w_ in (ws, ws_p):
+        st, _ = dsa.dsa_check_device_status(w_)
+        if st != dsa.DSA_OK:
+            raise RuntimeError(f"device status {st} in the end-to-end steps")
     total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
     import torch.distributed as dist
     world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
     return {"value": throughput(B * T, K, world, total_s), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K}
+            "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K,
+            "per_step": "1 pinned H2D copy of the token's raw inputs; dsa_index_produce (index key into the cache, "
+                        "index query codes); 2 device copies of the K/V rows into the cache; dsa_layer_decode; "
+                        "1 D2H copy of O and the selection"}
 
 
 # ------------------------------------------------------- CPU oracle timing
-def oracle_sample(n_keys: int, seed: int = 2):
-    """Time the CPU oracle on a contiguous sample of n_keys keys of the 1M
-    workload's recipe (indexer + top-k over the sample, attention over 2,048
-    keys) and scale the indexer and selection linearly to 1,048,576 keys.
-    Returns (seconds per full layer-step, seconds measured)."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_step(host, n_keys: int):
+    """One layer-step of the CPU oracle on the first n_keys keys of a host copy
+    of the workload (`host`: q8, q_scale, w, k8, k_scale, Q, sink, K/V row
+    getter): indexer over the n_keys keys, top-2048, attention over the
+    selected rows.  Returns (seconds of indexer + selection, seconds of
+    attention)."""
     import numpy as np
     import oracle
-    from workloads import bits16, make_decode_workload
-    wl = make_decode_workload(seed=seed, seq_lens=[max(n_keys, TOP_K)], T=1, n_needles=4, needle_mode="zipf")
-    n = wl.layout.seq_lens[0]
     t0 = time.perf_counter()
-    s = oracle.indexer_scores(wl.q8[0].numpy(), wl.q_scale[0].numpy(), wl.w[0].numpy(), wl.k8.numpy(),
-                              wl.k_scale.numpy(), wl.q_pos[0].numpy())
+    s = oracle.indexer_scores(host["q8"], host["q_scale"], host["w"], host["k8"][:n_keys], host["k_scale"][:n_keys],
+                              np.array([n_keys - 1], np.int32))
     sel, c = oracle.topk(s[0], TOP_K)
     t1 = time.perf_counter()
-    sel = sel[:c] if c else np.arange(min(n, TOP_K), dtype=np.int32)
-    oracle.gqa_attention(bits16(wl.Q[0, 0]), bits16(wl.K), bits16(wl.V), sel, wl.sink.numpy(),
+    sel = sel[:c]
+    Kr, Vr = host["kv_rows"](sel)
+    oracle.gqa_attention(host["Q"], Kr, Vr, np.arange(len(sel), dtype=np.int32), host["sink"],
                          1.0 / math.sqrt(192))
     t2 = time.perf_counter()
-    full = (t1 - t0) * (L_CTX / n) + (t2 - t1)
-    return full, t2 - t0
+    return t1 - t0, t2 - t1
 
 
-def cpu_baseline_line(target_s: float = 15.0):
-    n = 16384
-    full, spent = oracle_sample(n)
-    # grow the sample toward the target CPU time
-    per_key = max(1e-7, (spent - 0.3) / n)
-    n2 = int(min(L_CTX, max(n, (target_s - spent) / per_key)))
-    if n2 > n:
-        full, spent2 = oracle_sample(n2)
-        n, spent = n2, spent + spent2
-    return {"value": 1.0 / full, "unit": "tok/s", "cores": 1, "kind": "oracle",
-            "sample": f"one layer-step of the ctx_1m recipe on the first {n} keys (indexer + top-2048 over them, "
-                      f"attention over 2,048 keys), indexer and selection time scaled by {L_CTX}/{n}; "
-                      f"single-threaded C oracle in double; {spent:.1f} s of CPU"}
+def host_copy(wl):
+    """Host arrays of a one-sequence, one-token decode workload for the oracle
+    (the K/V rows are copied only where the selection points)."""
+    from workloads import bits16
+    K, V = wl.K, wl.V
+    return {"q8": wl.q8[0].cpu().numpy(), "q_scale": wl.q_scale[0].cpu().numpy(), "w": wl.w[0].cpu().numpy(),
+            "k8": wl.k8.cpu().numpy(), "k_scale": wl.k_scale.cpu().numpy(), "Q": bits16(wl.Q[0, 0]),
+            "sink": wl.sink.cpu().numpy(),
+            "kv_rows": lambda sel: (bits16(K[sel]), bits16(V[sel]))}
+
+
+def cpu_baseline_line(wl, full_budget_s: float = 40.0):
+    """The oracle on the host cores, on this run's own ctx_1m inputs: the whole
+    1,048,576-key step on all cores (timed, not extrapolated) when a first
+    sample says it fits the budget, and a single-core sample of 65,536 keys
+    scaled to the full context beside it."""
+    import oracle
+    host = host_copy(wl)
+    L = host["k8"].shape[0]
+    cores = oracle.set_threads(host_cores())
+    n0 = min(L, 65536)
+    a, b = oracle_step(host, n0)
+    est = a * L / n0 + b
+    if est <= full_budget_s:
+        a, b = oracle_step(host, L)
+        all_s, all_kind = a + b, f"the whole {L}-key step, timed"
+    else:
+        all_s, all_kind = est, f"the first {n0} keys, indexer and selection time scaled by {L}/{n0}"
+    oracle.set_threads(1)
+    a1, b1 = oracle_step(host, n0)
+    one_s = a1 * L / n0 + b1
+    return {"value": 1.0 / all_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cores": host_cores(),
+            "sample": f"one ctx_1m layer-step (indexer over the keys, top-2048, attention over the selection) of "
+                      f"this run's inputs on {cores} host threads: {all_kind}; C oracle in double",
+            "single_core": {"value": 1.0 / one_s, "unit": "tok/s", "cores": 1,
+                            "sample": f"first {n0} keys on one thread, indexer and selection scaled by {L}/{n0}"}}
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step one ctx_1m layer-step on all
+    host cores -- the whole 1,048,576 keys when (steps + warm-up) of those fit
+    about 150 s, otherwise the first n keys with the indexer and selection
+    time scaled by 1,048,576 / n (and labelled as extrapolated)."""
     if rank != 0:
         return None
-    budget_s = 150.0
+    import oracle
+    from workloads import CONFIGS, make_decode_workload
+    wl = make_decode_workload(**CONFIGS[WORKLOAD])
+    host = host_copy(wl)
+    L = host["k8"].shape[0]
+    cores = oracle.set_threads(host_cores())
     steps = args.steps + args.warmup
-    per_step = budget_s / max(1, steps)
-    n = int(max(TOP_K, min(65536, per_step / 1.1e-4)))
+    budget_s = 150.0
+    n0 = min(L, 65536)
+    a, b = oracle_step(host, n0)
+    per_key = a / n0
+    n = int(min(L, max(TOP_K, (budget_s / steps - b) / max(per_key, 1e-12))))
+    n = max(TOP_K, n - n % 128)
     times = []
     for i in range(steps):
-        full, _ = oracle_sample(n)
+        a, b = oracle_step(host, n)
         if i >= args.warmup:
-            times.append(full)
+            times.append(a * L / n + b)
     total = sum(times)
     value = len(times) / total
-    cores = 1
+    how = (f"each step the whole {L}-key ctx_1m layer-step on {cores} host threads, timed" if n == L else
+           f"each step the first {n} keys of the ctx_1m inputs on {cores} host threads, indexer and selection "
+           f"time extrapolated by {L}/{n} (the full step does not fit the run's time budget)")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": decode_config(WORKLOAD, world),
-        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: the CPU oracle on the first {n} keys of the ctx_1m recipe, "
-                                   f"indexer and selection scaled by {L_CTX}/{n}"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": how,
+                         "cpu_model": cpu_model(), "extrapolated": n != L},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -736,7 +942,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m", "ragged_b64_mix", "prefill_8k_1m"],
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the ragged-mix and prefill lines that the default run adds as extra keys")
+    ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m", "ragged_b64_mix", "prefill_8k_1m",
+                                           "stack_1m"],
                     default=WORKLOAD,
                     help="decode workload recipe (workloads.CONFIGS); the headline metric is on ctx_1m")
     args = ap.parse_args()
@@ -758,15 +967,43 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run = {"ragged_b64_mix": run_mix, "prefill_8k_1m": run_prefill}.get(args.workload, run_ours)
+        run = {"ragged_b64_mix": run_mix, "prefill_8k_1m": run_prefill, "stack_1m": run_stack}.get(args.workload,
+                                                                                                    run_ours)
         line = run(args, rank, world, local_rank)
+        wl = line.pop("_workload", None)
+        if args.workload == WORKLOAD and not args.no_secondary:
+            # the other benchmarked workloads, a few steps each, as extra keys
+            line["secondary"] = secondary_lines(args, rank, world, local_rank)
         if rank == 0:
-            if world == 1 and args.workload == WORKLOAD:
-                line["cpu_baseline"] = cpu_baseline_line()
+            if world == 1 and args.workload == WORKLOAD and wl is not None:
+                line["cpu_baseline"] = cpu_baseline_line(wl)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             dist.destroy_process_group()
+
+
+def secondary_lines(args, rank, world, local_rank):
+    """The ragged 64-sequence layer mix and the chunked prefill, a few timed
+    steps each (every rank runs them; the same collective steps on all ranks)."""
+    import torch
+    out = {}
+    for name, fn, steps in (("ragged_b64_mix", run_mix, 20), ("stack_1m", run_stack, 10),
+                            ("prefill_8k_1m", run_prefill, 3)):
+        sub = argparse.Namespace(**vars(args))
+        sub.steps, sub.warmup, sub.workload = steps, 3, name
+        try:
+            line = fn(sub, rank, world, local_rank)
+            out[name] = {k: line[k] for k in ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "roofline",
+                                             "clocks", "gpu_launches", "config") if k in line}
+            for k in ("us_per_mix", "stage_us_median", "hbm_view", "us_per_stack_chained", "us_per_stack_eager_median",
+                      "us_per_mix_eager_median", "us_per_mix_chained"):
+                if k in line:
+                    out[name][k] = line[k]
+        except Exception as e:   # reported, not fatal for the headline line
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.empty_cache()
+    return out
 
 
 if __name__ == "__main__":

@@ -89,6 +89,8 @@ extern "C" {
 #define DSA_OP_SWA_ATTN    3
 #define DSA_OP_LAYER       4
 #define DSA_OP_PREFILL     5   /* B = 1, T = NQ query tokens of dsa_prefill */
+#define DSA_OP_PRODUCE     6   /* dsa_index_produce (the status word only) */
+#define DSA_OP_KL          7   /* dsa_indexer_kl */
 
 /*
  * KV-cache description.  One "row" holds one position of one sequence:
@@ -135,12 +137,35 @@ int dsa_workspace_size(int op, int B, int T, int64_t Lmax, int top_k, size_t *by
 /* Zeroes a workspace (cudaMemsetAsync on `stream`). */
 int dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
-/* Synchronises `stream`, then reads and clears the device status word held in
- * the workspace.  *status receives DSA_OK, DSA_ERR_DEVICE_TIMEOUT or
- * DSA_ERR_DEVICE_BAD_INDEX (a bitwise OR of 1 << code for each kind seen is
- * returned in *flags if flags is not NULL).  After a device error the
- * workspace must be re-initialised with dsa_workspace_init. */
+/* Synchronises `stream`, then reads the device status word held in the
+ * workspace and clears its error bits.  *status receives DSA_OK,
+ * DSA_ERR_DEVICE_TIMEOUT or DSA_ERR_DEVICE_BAD_INDEX; *flags (if not NULL)
+ * receives the whole word: bit (1 << code) for each kind of error seen, and
+ * DSA_STATUS_NEEDS_INIT when a cross-CTA wait ran out.
+ * After a timeout the workspace must be re-initialised with
+ * dsa_workspace_init: DSA_STATUS_NEEDS_INIT stays set until then (reading the
+ * status does not clear it), and until then the calls that use the
+ * workspace's cross-CTA scratch (dsa_topk_select with more than one CTA per
+ * row, dsa_layer_decode, dsa_prefill) compute nothing and report
+ * DSA_ERR_DEVICE_TIMEOUT again, instead of running on a half-updated
+ * scratch. */
+#define DSA_STATUS_NEEDS_INIT 0x80000000u
 int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags);
+
+/* Failure injection, for tests of the device-side failure path (no page
+ * counterpart; an interface of this library).  While DSA_INJECT_BARRIER_TIMEOUT
+ * is set (process-wide, for launches made from any host thread), every launch
+ * of a kernel whose CTAs wait on one another (dsa_topk_select with more than
+ * one CTA per row, the fused dsa_layer_decode) makes its first cross-CTA
+ * barrier wait for one arrival more than will ever come, and bounds that wait
+ * by wait_limit_ns (1e3 .. 1e9) instead of the normal 2 s: the wait runs out,
+ * the kernel records DSA_ERR_DEVICE_TIMEOUT (and DSA_STATUS_NEEDS_INIT) in the
+ * workspace and returns, and the GPU stays usable.  Nothing faults or hangs.
+ * DSA_INJECT_NONE (wait_limit_ns ignored) restores normal operation.
+ * Returns DSA_ERR_INVALID_ARG for an unknown kind or limit. */
+#define DSA_INJECT_NONE            0
+#define DSA_INJECT_BARRIER_TIMEOUT 1
+int dsa_debug_inject(int kind, int64_t wait_limit_ns);
 
 /*
  * dsa_indexer_scores -- lightning-indexer scores of every visible key
@@ -156,6 +181,57 @@ int dsa_indexer_scores(const void *q8, const float *q_scale, const float *w,
                        const dsa_kv_t *kv, const int32_t *q_pos, int B, int T,
                        int64_t Lmax, float *scores, int64_t scores_stride,
                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_index_produce -- the indexer's inputs for B x T new tokens ("Inside a
+ * DSA layer: the lightning indexer": the indexer normalises its key, applies
+ * RoPE, and rounds both query and key to fp8_e4m3; the section's figure names
+ * LayerNorm, partial RoPE and FP8 quantisation; the same section gives the
+ * attention block's partial RoPE on a third of each head and a rope base of
+ * 10,000,000 on the sparse layers):
+ *   key   y = LayerNorm(k_in[b][t]) (population variance, ln_eps, weight
+ *         ln_w[128], bias ln_b[128]), then partial RoPE at p = q_pos[b][t];
+ *         index_k[row(b, p)] = e4m3(y / s), index_k_scale[row(b, p)] = s,
+ *         s = max|y| / 448 (1 for an all-zero y);
+ *   query (when q_in is not NULL) every head of q_in[b][t] turned by the same
+ *         partial RoPE at p; q8_out[b][t] = e4m3(y / s) with ONE scale s for
+ *         the token's 16 heads, written to all 16 entries of q_scale_out[b][t].
+ * Partial RoPE: dims i and i + rope_dim/2 (i < rope_dim/2) are rotated
+ * together by the angle p * rope_base^(-2i / rope_dim) (x_i cos - x_{i+h}
+ * sin, x_{i+h} cos + x_i sin); dims >= rope_dim pass unchanged.  rope_dim is
+ * even, 0..128 (0.334 x 128 rounds down to 42).  e4m3 conversion: nearest
+ * value, ties to the even code, saturating at +-448, taken in fp32.
+ *   k_in   bf16 [B][T][128]          q_in     bf16 [B][T][16][128] or NULL
+ *   q8_out uint8 [B][T][16][128]     q_scale_out float [B][T][16]
+ *   kv     the index-key cache (index_k, index_k_scale and the layout) written
+ *          at each token's position; a position outside it is flagged
+ *          DSA_ERR_DEVICE_BAD_INDEX in the workspace and not written.
+ * Workspace: dsa_workspace_size(DSA_OP_PRODUCE, ...) bytes (the status word).
+ */
+int dsa_index_produce(const void *k_in, const void *q_in, const float *ln_w, const float *ln_b, float ln_eps,
+                      int rope_dim, double rope_base, const dsa_kv_t *kv, const int32_t *q_pos, int B, int T,
+                      void *q8_out, float *q_scale_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_indexer_kl -- the indexer warm-up target and loss for B x T query
+ * tokens ("Inside a DSA layer: the lightning indexer": the indexer is trained
+ * first, alone, aligned to a full-attention reference by a KL objective; "2,122
+ * tok/s, Zero Full-Attention Layers", "What's genuinely new": the converted
+ * layers keep full attention and supervise the indexer through a KL loss).
+ * For query (b, t) at p = q_pos[b][t], over its visible keys s = 0..p:
+ *   P[s]  = (1/64) sum_h softmax_s(sm_scale * Q[b][t][h] . K[row(b,s)][h / (64/G)])
+ *           (dense attention of each head, no sink, averaged over the heads)
+ *   kl_out[b][t] = sum_s P[s] (ln P[s] - ln softmax_s(scores[b][t][s]))
+ * target_out (float [B][T][target_stride], or NULL) receives P[0..p].
+ * Q bf16 [B][T][64][192]; kv: the backbone keys (k, num_kv_heads, layout);
+ * scores: the indexer's output for the same tokens (dsa_indexer_scores).
+ * Logits on the tensor cores (bf16 operands, fp32 accumulation), softmax and
+ * KL in fp32; every reduction in a fixed order (run-to-run identical).
+ * Workspace: dsa_workspace_size(DSA_OP_KL, B, T, Lmax, 1, ...).
+ */
+int dsa_indexer_kl(const void *Q, const dsa_kv_t *kv, const float *scores, int64_t scores_stride,
+                   const int32_t *q_pos, int B, int T, int64_t Lmax, float sm_scale, float *kl_out, float *target_out,
+                   int64_t target_stride, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * dsa_topk_select -- for each query (b, t): the min(top_k, n) positions among
@@ -216,6 +292,88 @@ int dsa_layer_decode(const void *q8, const float *q_scale, const float *w, const
                      int top_k, const float *sink, float sm_scale, void *O, float *lse,
                      int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
                      void *stream, void *const *stage_events);
+
+/*
+ * dsa_layer_chain -- a sequence of decode layer-steps enqueued as one chain,
+ * the way a layer stack runs them ("The runtime is the actual claim": the
+ * kernels of dependent steps chained with programmatic dependent launch).
+ * Step i is exactly the call its kind names -- swa_attn_decode (window =
+ * top_k) or dsa_layer_decode -- with the step's arguments, in order on
+ * `stream`, and the outputs are bit-identical to making those calls one by
+ * one.  The difference is the launch: every kernel that is not a
+ * cooperative launch is enqueued as a programmatic dependent of the kernel
+ * before it, so it is scheduled while that kernel finishes and waits for its
+ * completion (and memory) before it touches anything; the cooperative
+ * kernels (the fused layer-step, a multi-CTA selection) keep plain stream
+ * order.  Every step is checked before anything is enqueued: an error in any
+ * step returns before the first launch.  Steps may share a workspace (they
+ * run one after another) or have their own.
+ */
+#define DSA_STEP_SWA 1
+#define DSA_STEP_DSA 2
+typedef struct dsa_layer_step {
+    int32_t          kind;        /* DSA_STEP_SWA or DSA_STEP_DSA */
+    int32_t          B, T;
+    int32_t          top_k;       /* DSA: top_k; SWA: the window */
+    int64_t          Lmax;        /* DSA: as for dsa_layer_decode */
+    const void      *q8;          /* DSA only: index queries, scales, head weights */
+    const float     *q_scale;
+    const float     *w;
+    const void      *Q;
+    const dsa_kv_t  *kv;
+    const int32_t   *q_pos;
+    const float     *sink;        /* or NULL */
+    float            sm_scale;
+    int32_t          reserved;
+    void            *O;
+    float           *lse;         /* or NULL */
+    int32_t         *idx_out;     /* DSA, or NULL */
+    int32_t         *count_out;   /* DSA, or NULL */
+    void            *ws;
+    size_t           ws_bytes;
+} dsa_layer_step_t;
+int dsa_layer_chain(const dsa_layer_step_t *steps, int n_steps, void *stream);
+
+/*
+ * Context-sharded decode: the DSA layer-step with each sequence's context
+ * split over n_ranks ranks, rank r holding the contiguous slice of positions
+ * [shard_offset, shard_offset + shard_len) in its own caches (a design of this
+ * library for multi-GPU decode; the pages describe the training system's
+ * sequence parallelism -- Ulysses for the DSA layers, "2,122 tok/s, Zero
+ * Full-Attention Layers", "What's genuinely new" -- not a decode split).
+ * Per rank, with the exchanges done by the caller's collectives:
+ *   1. dsa_shard_positions: q_pos_local = min(q_pos - shard_offset, shard_len - 1)
+ *      (every query must sit at or after the slice's start; one before it is
+ *      flagged DSA_ERR_DEVICE_BAD_INDEX in the workspace status word);
+ *   2. dsa_indexer_scores + dsa_topk_select on the slice with q_pos_local;
+ *   3. dsa_shard_candidates: the local selection as (score, global position)
+ *      pairs, cand_score float [B][T][top_k] / cand_pos int32 [B][T][top_k],
+ *      (-inf, -1) past the local count;
+ *   4. all-gather of the pairs in rank order -> [n_ranks][B][T][top_k];
+ *   5. dsa_shard_merge: the global top_k of every row (score descending, ties
+ *      to the lower position -- the one-GPU rule) in position order into
+ *      idx_out / count_out, and this rank's share as local positions,
+ *      compacted and -1 padded, into local_idx / local_count (optional);
+ *   6. sparse_gqa_attn_decode over (local_idx, local_count) with sink = NULL,
+ *      giving O_r and lse_r (lse_r = -inf for a rank with no share);
+ *   7. all-gather of (O_r, lse_r) in rank order;
+ *   8. dsa_shard_combine: O = sum_r e^{lse_r - LSE} O_r with
+ *      LSE = ln(sum_r e^{lse_r} + e^{sink}), the sink added once (sink may be
+ *      NULL); lse receives LSE.
+ * The merged selection equals the one-GPU selection over the whole context
+ * bit for bit; the output equals the one-GPU output within the attention
+ * tolerance (the sum is split by owner).  n_ranks 1..8.  These calls need no
+ * workspace except dsa_shard_positions (DSA_OP_PRODUCE, the status word).
+ */
+int dsa_shard_positions(const int32_t *q_pos, int B, int T, int64_t shard_offset, int64_t shard_len,
+                        int32_t *q_pos_local, void *ws, size_t ws_bytes, void *stream);
+int dsa_shard_candidates(const float *scores, int64_t scores_stride, const int32_t *idx, int B, int T, int top_k,
+                         int64_t shard_offset, float *cand_score, int32_t *cand_pos, void *stream);
+int dsa_shard_merge(const float *cand_score, const int32_t *cand_pos, int n_ranks, int B, int T, int top_k,
+                    int64_t shard_offset, int64_t shard_len, int32_t *idx_out, int32_t *count_out,
+                    int32_t *local_idx, int32_t *local_count, void *stream);
+int dsa_shard_combine(const void *O_all, const float *lse_all, int n_ranks, int B, int T, const float *sink, void *O,
+                      float *lse, void *stream);
 
 /*
  * dsa_prefill -- the DSA layer for NQ query tokens of ONE sequence (a

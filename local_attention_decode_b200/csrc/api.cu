@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -45,6 +46,43 @@ const DeviceInfo &device_info() {
         }
     }
     return d;
+}
+
+int ensure_smem_limit(const void *kernel, size_t bytes, const char *what) {
+    struct Entry { const void *kernel; int device; size_t bytes; };
+    static std::mutex mu;
+    static Entry cache[64];
+    static int used = 0;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lock(mu);
+    Entry *hit = nullptr;
+    for (int i = 0; i < used; ++i)
+        if (cache[i].kernel == kernel && cache[i].device == dev) hit = &cache[i];
+    if (hit && hit->bytes >= bytes) return DSA_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    if (!hit && used < 64) hit = &cache[used++];
+    if (hit) *hit = Entry{kernel, dev, bytes};
+    return DSA_OK;
+}
+
+static thread_local bool g_pdl = false;
+bool pdl_launches() { return g_pdl; }
+void set_pdl_launches(bool on) { g_pdl = on; }
+
+// Failure injection (dsa_debug_inject): process-wide, read at each launch.
+static std::atomic<int> g_inject_kind{DSA_INJECT_NONE};
+static std::atomic<int64_t> g_inject_limit_ns{0};
+
+BarrierCfg barrier_cfg() {
+    BarrierCfg c;
+    if (g_inject_kind.load() == DSA_INJECT_BARRIER_TIMEOUT) {
+        c.limit_ns = (uint64_t)g_inject_limit_ns.load();
+        c.extra = 1;
+    }
+    return c;
 }
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -109,6 +147,8 @@ struct WsPlan {
     size_t status = 0, scores = 0, idx = 0, count = 0, topk = 0, part_o = 0, part_ml = 0, total = 0;
     TopkPlan tp;
     FusedPlan fp;
+    CapturePlan cp;
+    size_t kl = 0;
 };
 
 static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan *w) {
@@ -121,6 +161,10 @@ static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan 
     };
     switch (op) {
         case DSA_OP_INDEXER:
+        case DSA_OP_PRODUCE:
+            break;
+        case DSA_OP_KL:
+            w->kl = take(kl_workspace_bytes(B, T, Lmax));
             break;
         case DSA_OP_TOPK: {
             int rc = plan_topk(B, T, Lmax, top_k, &w->tp);
@@ -130,7 +174,7 @@ static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan 
         }
         case DSA_OP_SPARSE_ATTN:
         case DSA_OP_SWA_ATTN: {
-            const int splits = (top_k + kAttnChunk - 1) / kAttnChunk;
+            const int splits = attn_splits(top_k);
             const size_t rows = (size_t)B * T * DSA_Q_HEADS * splits;
             w->part_o = take(rows * DSA_V_DIM * 4);
             w->part_ml = take(rows * 2 * 4);
@@ -140,12 +184,14 @@ static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan 
             int rc = plan_topk(B, T, Lmax, top_k, &w->tp);
             if (rc) return rc;
             if ((rc = plan_fused(B, T, Lmax, top_k, &w->fp))) return rc;
+            if ((rc = plan_capture(B, T, Lmax, top_k, &w->cp))) return rc;
             // the self-cleaning selection scratch first: its offset does not depend on the shape
-            w->topk = take(std::max(w->tp.scratch_bytes, w->fp.ok ? w->fp.scratch_bytes : 0));
+            w->topk = take(std::max({w->tp.scratch_bytes, w->fp.ok ? w->fp.scratch_bytes : 0,
+                                     w->cp.ok ? w->cp.scratch_bytes : 0}));
             w->scores = take((size_t)B * T * Lmax * 4);
             w->idx = take((size_t)B * T * top_k * 4);
             w->count = take((size_t)B * T * 4);
-            const int splits = (top_k + kAttnChunk - 1) / kAttnChunk;
+            const int splits = attn_splits(top_k);
             const size_t rows = (size_t)B * T * DSA_Q_HEADS * splits;
             w->part_o = take(rows * DSA_V_DIM * 4);
             w->part_ml = take(rows * 2 * 4);
@@ -264,12 +310,29 @@ int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags
     uint32_t word = 0;
     cudaError_t e = cudaStreamSynchronize(s);
     if (e == cudaSuccess) e = cudaMemcpy(&word, ws, 4, cudaMemcpyDeviceToHost);
-    if (e == cudaSuccess && word) e = cudaMemset(ws, 0, 4);
+    // the error bits are cleared by reading them; the re-initialisation bit
+    // stays until dsa_workspace_init
+    const uint32_t keep = word & kNeedsInitBit;
+    if (e == cudaSuccess && word != keep) e = cudaMemcpy(ws, &keep, 4, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     if (flags) *flags = word;
     *status = (word & (1u << DSA_ERR_DEVICE_TIMEOUT))     ? DSA_ERR_DEVICE_TIMEOUT
               : (word & (1u << DSA_ERR_DEVICE_BAD_INDEX)) ? DSA_ERR_DEVICE_BAD_INDEX
                                                           : DSA_OK;
+    return DSA_OK;
+}
+
+int dsa_debug_inject(int kind, int64_t wait_limit_ns) {
+    if (kind == DSA_INJECT_NONE) {
+        g_inject_kind.store(DSA_INJECT_NONE);
+        g_inject_limit_ns.store(0);
+        return DSA_OK;
+    }
+    if (kind != DSA_INJECT_BARRIER_TIMEOUT) return fail(DSA_ERR_INVALID_ARG, "unknown injection kind %d", kind);
+    if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000)
+        return fail(DSA_ERR_INVALID_ARG, "wait_limit_ns=%lld outside [1e3, 1e9]", (long long)wait_limit_ns);
+    g_inject_limit_ns.store(wait_limit_ns);
+    g_inject_kind.store(kind);
     return DSA_OK;
 }
 
@@ -290,6 +353,53 @@ int dsa_indexer_scores(const void *q8, const float *q_scale, const float *w, con
     IndexerArgs a{static_cast<const uint8_t *>(q8), q_scale, w, kv, q_pos, B, T, Lmax, scores, scores_stride,
                   at<uint32_t>(ws, wp.status)};
     return launch_indexer(a, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_index_produce(const void *k_in, const void *q_in, const float *ln_w, const float *ln_b, float ln_eps,
+                      int rope_dim, double rope_base, const dsa_kv_t *kv, const int32_t *q_pos, int B, int T,
+                      void *q8_out, float *q_scale_out, void *ws, size_t ws_bytes, void *stream) {
+    if (!k_in || !ln_w || !ln_b || !q_pos) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (q_in && (!q8_out || !q_scale_out)) return fail(DSA_ERR_INVALID_ARG, "q_in given without q8_out / q_scale_out");
+    if (!aligned16(k_in) || (q_in && (!aligned16(q_in) || !aligned16(q8_out))))
+        return fail(DSA_ERR_INVALID_ARG, "k_in / q_in / q8_out not 16-byte aligned");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (rc = check_kv_index(kv); rc) return rc;
+    if (rope_dim < 0 || rope_dim > DSA_INDEX_DIM || rope_dim % 2)
+        return fail(DSA_ERR_INVALID_ARG, "rope_dim=%d: need an even number in [0, %d]", rope_dim, DSA_INDEX_DIM);
+    if (!(rope_base > 1.0) || !std::isfinite(rope_base)) return fail(DSA_ERR_INVALID_ARG, "rope_base must be > 1");
+    if (!(ln_eps >= 0.f) || !std::isfinite(ln_eps)) return fail(DSA_ERR_INVALID_ARG, "ln_eps must be >= 0");
+    WsPlan wp;
+    if (rc = plan_workspace(DSA_OP_PRODUCE, B, T, 1, 1, &wp); rc) return rc;
+    if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
+    ProduceArgs a{static_cast<const __nv_bfloat16 *>(k_in), static_cast<const __nv_bfloat16 *>(q_in), ln_w, ln_b,
+                  ln_eps, rope_dim, rope_base, kv, q_pos, B, T, static_cast<uint8_t *>(q8_out), q_scale_out,
+                  at<uint32_t>(ws, wp.status)};
+    return launch_index_produce(a, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_indexer_kl(const void *Q, const dsa_kv_t *kv, const float *scores, int64_t scores_stride,
+                   const int32_t *q_pos, int B, int T, int64_t Lmax, float sm_scale, float *kl_out, float *target_out,
+                   int64_t target_stride, void *ws, size_t ws_bytes, void *stream) {
+    if (!Q || !scores || !q_pos || !kl_out) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(Q)) return fail(DSA_ERR_INVALID_ARG, "Q not 16-byte aligned");
+    int rc = check_common(B, T);
+    if (rc) return rc;
+    if (rc = check_kv_layout(kv); rc) return rc;
+    if (!kv->k || !aligned16(kv->k)) return fail(DSA_ERR_INVALID_ARG, "kv.k is NULL or not 16-byte aligned");
+    const int G = kv->num_kv_heads;
+    if (G < 1 || DSA_Q_HEADS % G || DSA_Q_HEADS / G > 16)
+        return fail(DSA_ERR_UNSUPPORTED_SHAPE, "num_kv_heads=%d: need a divisor of 64 with at most 16 heads per group", G);
+    if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
+    if (scores_stride < Lmax) return fail(DSA_ERR_INVALID_ARG, "scores_stride < Lmax");
+    if (target_out && target_stride < Lmax) return fail(DSA_ERR_INVALID_ARG, "target_stride < Lmax");
+    if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+    WsPlan wp;
+    if (rc = plan_workspace(DSA_OP_KL, B, T, Lmax, 1, &wp); rc) return rc;
+    if (rc = check_ws(ws, ws_bytes, wp); rc) return rc;
+    KlArgs a{static_cast<const __nv_bfloat16 *>(Q), kv, scores, scores_stride, q_pos, B, T, Lmax, sm_scale, kl_out,
+             target_out, target_stride, at<void>(ws, wp.kl), at<uint32_t>(ws, wp.status)};
+    return launch_indexer_kl(a, static_cast<cudaStream_t>(stream));
 }
 
 int dsa_topk_select(const float *scores, int64_t scores_stride, const int32_t *q_pos, int B, int T, int64_t Lmax,
@@ -403,7 +513,7 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
     int32_t *count = count_out ? count_out : at<int32_t>(ws, wp.count);
 
     IndexerArgs ia{static_cast<const uint8_t *>(q8), q_scale, w, kv, q_pos, B, T, Lmax, scores, Lmax, status};
-    if (wp.fp.ok) {
+    if (wp.cp.ok || wp.fp.ok) {
         // one cooperative launch for the whole layer-step
         AttnArgs a;
         a.Q = static_cast<const __nv_bfloat16 *>(Q);
@@ -424,8 +534,13 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
         a.part_ml = at<float>(ws, wp.part_ml);
         a.status = status;
         a.padded = 1;   // the fused selection pads every idx row with -1
-        rc = launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s,
-                          stage_events ? stage_events[0] : nullptr);
+        if (wp.cp.ok)
+            rc = launch_capture(wp.cp, ia, a, top_k, idx, count, at<uint8_t>(ws, wp.topk), s,
+                                stage_events ? stage_events[0] : nullptr);
+        if (!wp.cp.ok || rc == DSA_ERR_UNSUPPORTED_SHAPE)
+            rc = wp.fp.ok ? launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s,
+                                         stage_events ? stage_events[0] : nullptr)
+                          : DSA_ERR_UNSUPPORTED_SHAPE;
         if (rc == DSA_OK) {
             for (int i = 1; i <= 4; ++i)
                 if (rc = record(stage_events, i, s); rc) return rc;
@@ -489,4 +604,113 @@ int dsa_prefill(const void *q8, const float *q_scale, const float *w, const void
         if (rc) return rc;
     }
     return DSA_OK;
+}
+
+// ------------------------------------------------------------- the chain
+// Checks of one chain step, exactly those its own entry point makes before
+// enqueueing anything.
+static int check_step(const dsa_layer_step_t &st) {
+    WsPlan wp;
+    int rc;
+    if (st.kind == DSA_STEP_DSA) {
+        if ((rc = check_layer_args(st.q8, st.q_scale, st.w, st.Q, st.kv, st.q_pos, st.B, st.T, st.Lmax, st.top_k,
+                                   st.sm_scale, st.O)))
+            return rc;
+        if ((rc = plan_workspace(DSA_OP_LAYER, st.B, st.T, st.Lmax, st.top_k, &wp))) return rc;
+        return check_ws(st.ws, st.ws_bytes, wp);
+    }
+    if (st.kind == DSA_STEP_SWA) {
+        if (!st.q_pos) return fail(DSA_ERR_INVALID_ARG, "q_pos is NULL");
+        if (!st.Q || !st.O) return fail(DSA_ERR_INVALID_ARG, "Q / O is NULL");
+        if (!aligned16(st.Q) || !aligned16(st.O)) return fail(DSA_ERR_INVALID_ARG, "Q / O not 16-byte aligned");
+        if ((rc = check_common(st.B, st.T))) return rc;
+        if ((rc = check_kv_backbone(st.kv))) return rc;
+        if (st.top_k < 1 || st.top_k > DSA_MAX_TOPK)
+            return fail(DSA_ERR_UNSUPPORTED_SHAPE, "window=%d outside [1, %d]", st.top_k, DSA_MAX_TOPK);
+        if (!(st.sm_scale > 0.f) || !std::isfinite(st.sm_scale))
+            return fail(DSA_ERR_INVALID_ARG, "sm_scale must be finite and > 0");
+        if ((rc = plan_workspace(DSA_OP_SWA_ATTN, st.B, st.T, 1, st.top_k, &wp))) return rc;
+        return check_ws(st.ws, st.ws_bytes, wp);
+    }
+    return fail(DSA_ERR_INVALID_ARG, "unknown step kind %d", st.kind);
+}
+
+extern "C" int dsa_layer_chain(const dsa_layer_step_t *steps, int n_steps, void *stream) {
+    if (!steps || n_steps < 1) return fail(DSA_ERR_INVALID_ARG, "steps is NULL or n_steps < 1");
+    for (int i = 0; i < n_steps; ++i) {
+        if (int rc = check_step(steps[i])) {
+            char msg[512];
+            snprintf(msg, sizeof msg, "%s", dsa_last_error());
+            return fail(rc, "step %d: %s", i, msg);
+        }
+    }
+    struct Pdl {   // the chained launch mode for this thread, restored on every exit
+        Pdl() { set_pdl_launches(true); }
+        ~Pdl() { set_pdl_launches(false); }
+    } pdl;
+    for (int i = 0; i < n_steps; ++i) {
+        const dsa_layer_step_t &st = steps[i];
+        int rc;
+        if (st.kind == DSA_STEP_DSA)
+            rc = dsa_layer_decode(st.q8, st.q_scale, st.w, st.Q, st.kv, st.q_pos, st.B, st.T, st.Lmax, st.top_k,
+                                  st.sink, st.sm_scale, st.O, st.lse, st.idx_out, st.count_out, st.ws, st.ws_bytes,
+                                  stream, nullptr);
+        else
+            rc = swa_attn_decode(st.Q, st.kv, st.q_pos, st.B, st.T, st.top_k, st.sink, st.sm_scale, st.O, st.lse,
+                                 st.ws, st.ws_bytes, stream);
+        if (rc) {
+            char msg[512];
+            snprintf(msg, sizeof msg, "%s", dsa_last_error());
+            return fail(rc, "step %d: %s", i, msg);
+        }
+    }
+    return DSA_OK;
+}
+
+// ------------------------------------------------- context-sharded decode
+extern "C" int dsa_shard_positions(const int32_t *q_pos, int B, int T, int64_t shard_offset, int64_t shard_len,
+                                   int32_t *q_pos_local, void *ws, size_t ws_bytes, void *stream) {
+    if (!q_pos || !q_pos_local) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (int rc = check_common(B, T)) return rc;
+    if (shard_offset < 0 || shard_len < 1) return fail(DSA_ERR_INVALID_ARG, "shard offset / length");
+    WsPlan wp;
+    if (int rc = plan_workspace(DSA_OP_PRODUCE, B, T, 1, 1, &wp)) return rc;
+    if (int rc = check_ws(ws, ws_bytes, wp)) return rc;
+    uint32_t *status = at<uint32_t>(ws, wp.status);
+    // a query before the slice is flagged as a bad index in the status word
+    return launch_shard_positions(q_pos, B * T, shard_offset, shard_len, q_pos_local, status,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dsa_shard_candidates(const float *scores, int64_t scores_stride, const int32_t *idx, int B, int T,
+                                    int top_k, int64_t shard_offset, float *cand_score, int32_t *cand_pos,
+                                    void *stream) {
+    if (!scores || !idx || !cand_score || !cand_pos) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (int rc = check_common(B, T)) return rc;
+    if (top_k < 1 || top_k > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
+    if (shard_offset < 0) return fail(DSA_ERR_INVALID_ARG, "shard_offset < 0");
+    return launch_shard_candidates(scores, scores_stride, idx, top_k, B * T, shard_offset, cand_score, cand_pos,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dsa_shard_merge(const float *cand_score, const int32_t *cand_pos, int n_ranks, int B, int T, int top_k,
+                               int64_t shard_offset, int64_t shard_len, int32_t *idx_out, int32_t *count_out,
+                               int32_t *local_idx, int32_t *local_count, void *stream) {
+    if (!cand_score || !cand_pos || !idx_out || !count_out) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if ((local_idx == nullptr) != (local_count == nullptr))
+        return fail(DSA_ERR_INVALID_ARG, "local_idx and local_count go together");
+    if (int rc = check_common(B, T)) return rc;
+    if (n_ranks < 1 || n_ranks > 8) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "n_ranks=%d outside [1, 8]", n_ranks);
+    if (top_k < 1 || top_k > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
+    return launch_shard_merge(cand_score, cand_pos, n_ranks, top_k, B * T, shard_offset, shard_len, idx_out, count_out,
+                              local_idx, local_count, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dsa_shard_combine(const void *O_all, const float *lse_all, int n_ranks, int B, int T, const float *sink,
+                                 void *O, float *lse, void *stream) {
+    if (!O_all || !lse_all || !O) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (int rc = check_common(B, T)) return rc;
+    if (n_ranks < 1 || n_ranks > 8) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "n_ranks=%d outside [1, 8]", n_ranks);
+    return launch_shard_combine(static_cast<const __nv_bfloat16 *>(O_all), lse_all, n_ranks, B * T, sink,
+                                static_cast<__nv_bfloat16 *>(O), lse, static_cast<cudaStream_t>(stream));
 }

@@ -50,7 +50,8 @@ struct Params {
     const int32_t *q_pos;
     int window;
     int T;
-    int splits;
+    int n_teams;        // 64-key team chunks per CTA unit (1..4)
+    int splits;         // CTA units per (query, KV head): ceil(max_keys / (64 * n_teams))
     float scale_log2;   // sm_scale * log2(e)
     float *part_o;
     float *part_ml;
@@ -65,6 +66,15 @@ struct Smem {
     int64_t row[kChunk];
     float m[4][16];
     float l[4][16];
+    float tm[16];   // the team's result: per head row, the max logit (log2 domain) ...
+    float tl[16];   // ... and the sum of exp2(logit - max); its O is in the first 8 KB of k
+};
+
+// The teams' shared memory of a CTA: team t at base + t * stride.
+struct TeamSmem {
+    uint8_t *base;
+    uint32_t stride;
+    __device__ __forceinline__ Smem &operator[](int t) const { return *reinterpret_cast<Smem *>(base + t * stride); }
 };
 
 // Barrier of one 128-thread team.  The id is a run-time value, so that all
@@ -120,11 +130,15 @@ __device__ __forceinline__ bool key_row(const Params &p, int b, int64_t pos, int
     return *row < p.num_rows;
 }
 
-// One split-KV unit: keys [split * 64, split * 64 + 64) of query bt and KV
+// One team chunk: keys [chunk * 64, chunk * 64 + 64) of query bt and KV
 // head g, by a team of 128 threads (tid 0..127) synchronised with the named
-// barrier `bar`; writes the unit's partial (O, max, sum) for the 64/G
-// query heads of the group.
-__device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid, int bar) {
+// barrier `bar`; leaves the chunk's result (per head row of the group: max
+// logit, sum of exponentials, and the unnormalised O) in the team's shared
+// memory (sm.tm, sm.tl, the first 16 x 128 floats of sm.k) for cta_merge.
+// sel_smem: the query's selection (-1 padded, the p.padded layout) already
+// in shared memory, read instead of p.idx.
+__device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, int g, int bt, int tid, int bar,
+                                          const int32_t *sel_smem = nullptr) {
     const int b = bt / p.T;
     const int hpg = DSA_Q_HEADS / p.G;
     const int warp = tid >> 5, lane = tid & 31;
@@ -138,13 +152,12 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         win_lo = max(0, pq - p.window + 1);
         n_total = pq >= 0 ? pq - win_lo + 1 : 0;
     }
-    const int k0 = split * kChunk;
+    const int k0 = chunk * kChunk;
     const int nk = min(kChunk, n_total - k0);
-    float *ml = p.part_ml + (((int64_t)bt * DSA_Q_HEADS + g * hpg) * p.splits + split) * 2;
-    if (nk <= 0) {   // empty split: contributes nothing to the combine
-        if (tid < hpg) {
-            ml[(int64_t)tid * p.splits * 2 + 0] = -INFINITY;
-            ml[(int64_t)tid * p.splits * 2 + 1] = 0.f;
+    if (nk <= 0) {   // empty chunk: contributes nothing to the merge
+        if (tid < 16) {
+            sm.tm[tid] = -INFINITY;
+            sm.tl[tid] = 0.f;
         }
         return;
     }
@@ -153,8 +166,9 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
     if (tid < kChunk) {
         int64_t row = -1;
         if (tid < nk) {
-            int64_t pos = p.idx ? (int64_t)__ldcg(p.idx + (int64_t)bt * p.idx_stride + k0 + tid)
-                                : (int64_t)(win_lo + k0 + tid);
+            int64_t pos = sel_smem ? (int64_t)sel_smem[k0 + tid]
+                          : p.idx  ? (int64_t)__ldcg(p.idx + (int64_t)bt * p.idx_stride + k0 + tid)
+                                   : (int64_t)(win_lo + k0 + tid);
             if (p.padded && pos < 0) {
                 row = -1;   // past the selection
             } else if (!key_row(p, b, pos, &row)) {
@@ -283,32 +297,106 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int split, 
         *reinterpret_cast<float2 *>(d1) = make_float2(o[nt][2] * scale_row[1], o[nt][3] * scale_row[1]);
     }
     team_sync(bar);
-    // each thread: one head row (tid / 8) and 16 columns
-    {
-        const int row = tid >> 3, c0 = (tid & 7) * 16;
-        if (row < hpg) {
-            float M = fmaxf(fmaxf(sm.m[0][row], sm.m[1][row]), fmaxf(sm.m[2][row], sm.m[3][row]));
-            float L = 0.f;
+    // each thread: one head row (tid / 8) and 16 columns; the four warps'
+    // scaled O summed in registers, then written over warp 0's slot
+    const int row = tid >> 3, c0 = (tid & 7) * 16;
+    float4 acc[4];
+    float M = -INFINITY, L = 0.f;
+    if (row < hpg) {
+        M = fmaxf(fmaxf(sm.m[0][row], sm.m[1][row]), fmaxf(sm.m[2][row], sm.m[3][row]));
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-                L += (sm.m[w][row] == -INFINITY) ? 0.f : sm.l[w][row] * exp2f(sm.m[w][row] - M);
-            float *dst = p.part_o + (((int64_t)bt * DSA_Q_HEADS + g * hpg + row) * p.splits + split) * DSA_V_DIM + c0;
+        for (int w = 0; w < 4; ++w)
+            L += (sm.m[w][row] == -INFINITY) ? 0.f : sm.l[w][row] * exp2f(sm.m[w][row] - M);
 #pragma unroll
-            for (int c = 0; c < 16; c += 4) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < 4; ++c) {
+            acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    float4 v = *reinterpret_cast<const float4 *>(so + (w * 16 + row) * DSA_V_DIM + c0 + c);
-                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-                }
-                *reinterpret_cast<float4 *>(dst + c) = acc;
-            }
-            if ((tid & 7) == 0) {
-                ml[(int64_t)row * p.splits * 2 + 0] = M;
-                ml[(int64_t)row * p.splits * 2 + 1] = L;
+            for (int w = 0; w < 4; ++w) {
+                const float4 v = *reinterpret_cast<const float4 *>(so + (w * 16 + row) * DSA_V_DIM + c0 + 4 * c);
+                acc[c].x += v.x; acc[c].y += v.y; acc[c].z += v.z; acc[c].w += v.w;
             }
         }
     }
+    team_sync(bar);
+    if (row < hpg) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<float4 *>(so + row * DSA_V_DIM + c0 + 4 * c) = acc[c];
+        if ((tid & 7) == 0) {
+            sm.tm[row] = M;
+            sm.tl[row] = L;
+        }
+    }
+}
+
+// The merge of the n_teams team chunks of one CTA unit (query bt, KV head g,
+// unit `split`), by the threads t < n_teams * 128 of the CTA (after a barrier
+// that follows the teams' attn_unit): thread t takes four columns of head
+// rows t / 32, t / 32 + 4 n_teams, ... and merges the teams in order 0, 1, ...
+// (teams with no key skipped).  With one unit per
+// (query, KV head) (p.splits == 1) it finishes the output: the sink enters
+// the denominator, O is normalised and written in bf16, with the lse.
+// Otherwise it writes the unit's partial (O, max, sum) for the combine.
+__device__ __forceinline__ void cta_merge(const Params &p, const TeamSmem &teams, int split, int g, int bt, int t,
+                                          const float *sink, __nv_bfloat16 *O, float *lse) {
+    const int hpg = DSA_Q_HEADS / p.G, c = (t & 31) * 4, row_step = p.n_teams * 4;
+    for (int row = t >> 5; row < hpg; row += row_step) {
+        float M = -INFINITY;
+        for (int tm = 0; tm < p.n_teams; ++tm) M = fmaxf(M, teams[tm].tm[row]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float L = 0.f;
+        for (int tm = 0; tm < p.n_teams; ++tm) {
+            const float mt = teams[tm].tm[row];
+            if (mt == -INFINITY) continue;
+            const float w = exp2f(mt - M);
+            const float4 v = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(teams[tm].k) +
+                                                               row * DSA_V_DIM + c);
+            acc.x += v.x * w; acc.y += v.y * w; acc.z += v.z * w; acc.w += v.w * w;
+            L += teams[tm].tl[row] * w;
+        }
+        const int64_t gw = (int64_t)bt * DSA_Q_HEADS + g * hpg + row;
+        if (p.splits == 1) {
+            const float sk = sink ? __ldg(sink + g * hpg + row) * kLog2e : -INFINITY;
+            const float M2 = fmaxf(M, sk);
+            float den = 0.f, w = 0.f;
+            if (M2 != -INFINITY) {
+                w = (M == -INFINITY) ? 0.f : exp2f(M - M2);
+                den = L * w + (sink ? exp2f(sk - M2) : 0.f);
+            }
+            const float f = den > 0.f ? w / den : 0.f;
+            __nv_bfloat16 *o = O + gw * DSA_V_DIM + c;
+            o[0] = __float2bfloat16_rn(acc.x * f);
+            o[1] = __float2bfloat16_rn(acc.y * f);
+            o[2] = __float2bfloat16_rn(acc.z * f);
+            o[3] = __float2bfloat16_rn(acc.w * f);
+            if (lse && c == 0) lse[gw] = den > 0.f ? (M2 + log2f(den)) / kLog2e : -INFINITY;
+        } else {
+            *reinterpret_cast<float4 *>(p.part_o + (gw * p.splits + split) * DSA_V_DIM + c) = acc;
+            if (c == 0) {
+                p.part_ml[(gw * p.splits + split) * 2 + 0] = M;
+                p.part_ml[(gw * p.splits + split) * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+// One CTA unit: team tm < p.n_teams takes chunk split * n_teams + tm (team
+// barriers bar0 + tm), then the n_teams * 128 threads merge after the
+// barrier `cta_bar` (0 = __syncthreads, else a named barrier of those
+// threads).  Exactly the threads t < n_teams * 128 call it.  The teams'
+// shared memory may be reused after the call.
+__device__ __forceinline__ void cta_unit(const Params &p, const TeamSmem &teams, int split, int g, int bt, int bar0,
+                                         int cta_bar, const float *sink, __nv_bfloat16 *O, float *lse,
+                                         const int32_t *sel_smem = nullptr) {
+    const int t = threadIdx.x, tm = t >> 7;
+    auto cta_sync = [&]() {
+        if (cta_bar == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;" ::"r"(cta_bar), "r"(p.n_teams * 128) : "memory");
+    };
+    if (tm < p.n_teams) attn_unit(p, teams[tm], split * p.n_teams + tm, g, bt, t & 127, bar0 + tm, sel_smem);
+    cta_sync();
+    cta_merge(p, teams, split, g, bt, t, sink, O, lse);
+    if (p.splits > 1) __threadfence();   // the partial is visible before any later signal of this CTA
+    cta_sync();
 }
 
 // Merge of the splits of one (query, head) row gw by a whole CTA of NT
@@ -383,7 +471,8 @@ inline Params make_params(const AttnArgs &a) {
     p.q_pos = a.q_pos;
     p.window = a.window;
     p.T = a.T;
-    p.splits = (a.max_keys + kChunk - 1) / kChunk;
+    p.n_teams = attn_teams(a.max_keys);
+    p.splits = attn_splits(a.max_keys);
     p.scale_log2 = a.sm_scale * kLog2e;
     p.part_o = a.part_o;
     p.part_ml = a.part_ml;

@@ -1,0 +1,980 @@
+// capture.cu -- the DSA decode layer-step for up to four long query rows as
+// one cooperative kernel with a single grid barrier after the key stream.
+//
+// What it computes is exactly the layer-step of dsa_layer_decode: indexer
+// scores of every visible key, the top-k positions with ties to the lower
+// position, sparse GQA attention over them with the sink ("Naive-N0.5-Flash:
+// no full-attention layers, and a runtime built by AI", sections "Inside a DSA
+// layer: the lightning indexer" and "What 'no full-attention layers' means").
+// How it is organised is this library's own design for B200: the selection
+// work that depends on every score is cut down to a short list that the key
+// stream itself produces.
+//
+// Phase 1, the key stream (one CTA per SM, two TMA -> tcgen05 pipelines, four
+// epilogue groups of four warps; indexer_impl.cuh has the machinery).  Each
+// epilogue group owns a contiguous range of key tiles, so that its output is
+// in position order:
+//   * its first tile is a sample: the scores' 8-bins-per-octave histogram
+//     goes into the CTA's shared histogram; when all four groups of a CTA have
+//     added theirs, one of them adds the CTA's histogram into the row's global
+//     one; the last CTA to do so turns each row's sample histogram into a
+//     score threshold -- a bin edge below which the sample predicts about
+//     `oversample` x top_k keys -- and publishes it;
+//   * every tile: keys with score >= threshold are appended, with their
+//     positions, to the group's segment of the row's candidate list, in
+//     position order (a ballot per warp, an exchange of counts among the
+//     group's four warps per tile).  Every score is also stored, as the
+//     standalone indexer stores it (the fallback below reads them).
+// One grid barrier.  The segments' lengths tell whether the sample was good:
+// if every row holds at least top_k candidates (then the list holds every key
+// at or above the k-th largest score, since the threshold is below it) and no
+// segment overflowed, the fast path runs; otherwise the general path of the
+// fused layer-step does (the result is the same either way).
+// Phase 2 (fast), per CTA of a row: the row's candidates (a few thousand)
+// into shared memory in position order, an exact 11/11/10-bit radix select on
+// them, the selection compacted in position order into shared memory.  Its
+// attention units read the selection from there; the last unit of each KV
+// group of a row (a counter per group) combines that group's heads with the
+// sink, with the same arithmetic as the combine kernel.
+#include <algorithm>
+#include <mutex>
+
+#include "attention_impl.cuh"
+#include "indexer_impl.cuh"
+#include "kernels.h"
+#include "topk_impl.cuh"
+
+namespace dsa {
+namespace capture {
+
+using indexer::kEpiWarp0;
+using indexer::kEpiWarps;
+using indexer::kKeyBytes;
+using indexer::kMaxGroups;
+using indexer::kPipes;
+using indexer::kTile;
+
+constexpr int kThreads = indexer::kThreads;   // 640
+constexpr int kWarps = kThreads / 32;
+constexpr int kTeams = 4;                     // attention teams of 4 warps (named barriers 1..4)
+constexpr int kMaxRows = 4;                   // B * T on this path
+constexpr int kGroups = kPipes * kMaxGroups;  // epilogue groups per CTA
+constexpr int kBins = 2048;                   // sample histogram: bits 30..20 of the non-negative keys
+constexpr int kHistWords = kBins + 1;         // + the count of negative scores
+constexpr int kSegCap = 1024;                 // candidates one epilogue group may hold per row
+constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
+constexpr int kGroupBar0 = 5;                 // named barriers 5..8: the epilogue groups
+constexpr int kUnitBar = 9;                   // named barrier of the attention teams of a CTA unit
+constexpr int kSelBytes = DSA_MAX_TOPK * 4;   // the selection, at the start of shared memory in phase 2
+constexpr int64_t kMinContext = 8192;         // shorter contexts take the fused layer-step
+
+// control words at the start of the capture scratch
+enum {
+    kGridArrive = 0,
+    kGridExit = 1,
+    kSampleArrive = 2,
+    kReady = 3,
+    kOverflow = 4,
+    kThr = 8,                 // [kMaxRows] thresholds (order keys)
+    kTotal = 12,              // [kMaxRows] candidates per row
+    kCombine = 16,            // [kMaxRows][64] attention units done per (row, KV group)
+    kCtlWords = 512
+};
+
+static_assert(kCombine + kMaxRows * DSA_Q_HEADS <= kCtlWords, "control words");
+static_assert(kTeams * 4 < kWarps, "the attention teams must leave warps free in the CTA");
+
+struct Params {
+    indexer::Params ix;
+    topk::Params tk;          // the general selection (fallback)
+    attn::Params at;
+    const float *sink;
+    __nv_bfloat16 *O;
+    float *lse;
+    uint32_t *ctl;
+    uint32_t *sample_hist;    // [rows][kHistWords]
+    uint32_t *counts;         // [rows][NG]
+    uint2 *lists;             // [rows][NG][kSegCap] (order key, position)
+    BarrierCfg bar;
+    int rows, K, C, NG;
+    float oversample;
+};
+
+__host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
+
+// Shared memory of phase 1 (base aligned to 1024 bytes).
+struct Layout {
+    uint32_t k_off, q_off, ks_off, bar_off, tmem_off, len_off, tile_off, epi_off, hist_off, xch_off, misc_off, total;
+    __host__ __device__ Layout(int S, int T, int B) {
+        const int stages = kPipes * S, rows = B * T;
+        k_off = 0;
+        q_off = stages * kTile * kKeyBytes;
+        ks_off = q_off + rows * 16 * kKeyBytes;   // every row's query block, resident
+        bar_off = ks_off + stages * indexer::kKsStageBytes;
+        tmem_off = bar_off + (uint32_t)sizeof(indexer::Bars);
+        len_off = (tmem_off + 16 + 15) & ~15u;
+        tile_off = (len_off + 4 * (B + 1) + 15) & ~15u;
+        epi_off = (tile_off + 4 * (B + 1) + 15) & ~15u;
+        hist_off = epi_off + kGroups * kEpiWarps * (16 * T + T) * 4;
+        xch_off = hist_off + rows * kHistWords * 4;
+        misc_off = xch_off + kGroups * 2 * kEpiWarps * kMaxRows * 4;
+        total = misc_off + 32;   // [0] groups sampled, [1 + g] group g's role in the sample exchange
+    }
+};
+
+// Bin of a non-negative order key in the sample histogram; kBins for a
+// negative score.
+__device__ __forceinline__ uint32_t sample_bin(uint32_t key) {
+    return (key >> 31) ? ((key >> 20) & (kBins - 1)) : (uint32_t)kBins;
+}
+
+// The threshold of one row from its global sample histogram, by one warp:
+// the lower edge of the highest bin b whose count, with the bins above it,
+// reaches `target`; zero (take every key) when the sample's non-negative
+// scores do not reach it.  Zeroes the histogram for the next call.
+__device__ uint32_t row_threshold(uint32_t *hist, uint32_t target) {
+    const int lane = lane_id();
+    constexpr int kPer = kBins / 32;   // 64 bins per lane
+    uint32_t s = 0;
+    const uint4 *h4 = reinterpret_cast<const uint4 *>(hist + lane * kPer);
+#pragma unroll
+    for (int u = 0; u < kPer / 4; ++u) {
+        const uint4 v = __ldcg(h4 + u);
+        s += v.x + v.y + v.z + v.w;
+    }
+    uint32_t incl = s;   // keys in this lane's bins and all higher ones
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += u;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, incl >= target);
+    uint32_t thr = 0;
+    if (target > 0 && hit) {
+        const int L = 31 - __clz(hit);   // highest lane whose suffix reaches the target
+        const uint32_t above = __shfl_sync(0xffffffffu, incl - s, L);
+        // that lane's 64 bins, two per lane, then the same search over them
+        const uint32_t b0 = (uint32_t)(L * kPer + 2 * lane);
+        const uint32_t v0 = __ldcg(hist + b0), v1 = __ldcg(hist + b0 + 1);
+        const uint32_t t = v0 + v1;
+        uint32_t inc2 = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t u = __shfl_down_sync(0xffffffffu, inc2, o);
+            if (lane + o < 32) inc2 += u;
+        }
+        // bins b0 + 1 and b0 in descending order
+        const uint32_t run1 = above + inc2 - t + v1;   // keys in bins >= b0 + 1
+        const uint32_t run0 = run1 + v0;               // keys in bins >= b0
+        uint32_t mine = 0xFFFFFFFFu;
+        if (run1 >= target) mine = b0 + 1;
+        else if (run0 >= target) mine = b0;
+        uint32_t best = __reduce_max_sync(0xffffffffu, mine == 0xFFFFFFFFu ? 0u : mine + 1);
+        thr = best ? (0x80000000u | ((best - 1) << 20)) : 0u;
+    }
+    __syncwarp();
+    uint4 *w4 = reinterpret_cast<uint4 *>(hist + lane * kPer);
+#pragma unroll
+    for (int u = 0; u < kPer / 4; ++u) w4[u] = make_uint4(0, 0, 0, 0);
+    if (lane == 0) hist[kBins] = 0;
+    return thr;
+}
+
+// Phase 1: the indexer over this CTA's tiles with sampling and candidate
+// capture (see the file comment).  All kThreads threads call it.  On return
+// nothing is in flight, TMEM is released and the mbarriers are invalidated.
+__device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorMap *tmap_ks_p,
+                                    const CUtensorMap *tmap_q_p, const Params &cp, uint8_t *smem, int cta, int ncta) {
+    using namespace indexer;
+    const indexer::Params &p = cp.ix;
+    const CUtensorMap &tmap_k = *tmap_k_p, &tmap_ks = *tmap_ks_p, &tmap_q = *tmap_q_p;
+    const int S = p.stages, T = p.T, B = p.B, N = 16 * T, GE = p.groups, rows = B * T;
+    Layout lay(S, T, B);
+    Bars *bars = reinterpret_cast<Bars *>(smem + lay.bar_off);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.tmem_off);
+    int32_t *seq_len = reinterpret_cast<int32_t *>(smem + lay.len_off);
+    int32_t *tile_pre = reinterpret_cast<int32_t *>(smem + lay.tile_off);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [rows][kHistWords]
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags
+    uint32_t *ctl = cp.ctl;
+    const int warp = warp_id(), lane = lane_id();
+
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        int32_t mx = -1;
+        bool ok = true;
+        for (int t = 0; t < T; ++t) {
+            int32_t q = __ldg(p.q_pos + b * T + t);
+            if (q < 0) ok = false;
+            mx = max(mx, q);
+        }
+        const int64_t cap = p.block_table ? (int64_t)p.max_pages * p.page_size : p.seq_stride;
+        if (!ok || (int64_t)mx >= cap || (int64_t)mx >= p.Lmax) {
+            if (cta == 0) flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX);
+            mx = -1;
+        }
+        seq_len[b] = mx + 1;
+    }
+    for (int j = threadIdx.x; j < rows * kHistWords; j += blockDim.x) hist[j] = 0;
+    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < B; base += 32) {
+            const int b = base + lane;
+            int v = b < B ? (seq_len[b] + kTile - 1) / kTile : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (b < B) tile_pre[b + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) tile_pre[0] = 0;
+    }
+    __syncthreads();
+
+    const int total = tile_pre[B];
+    const int per = total / ncta, rem = total % ncta;
+    const int t_begin = cta * per + min(cta, rem);
+    const int n_tiles = per + (cta < rem ? 1 : 0);
+    const int half = (n_tiles + kPipes - 1) / kPipes;
+    auto pipe_begin = [&](int pp) { return t_begin + min(n_tiles, pp * half); };
+    auto pipe_count = [&](int pp) { return min(n_tiles, (pp + 1) * half) - min(n_tiles, pp * half); };
+    // group a of pipe pp owns a contiguous part of the pipe's tiles; the
+    // pipe's i-th tile is tile i / GE of group i % GE
+    auto group_count = [&](int pp, int a) { const int c = pipe_count(pp); return c / GE + (a < c % GE ? 1 : 0); };
+    auto tile_of = [&](int pp, int i) {
+        const int c = pipe_count(pp), a = i % GE;
+        return pipe_begin(pp) + a * (c / GE) + min(a, c % GE) + i / GE;
+    };
+
+    uint32_t tmem_cols = 32;
+    while (tmem_cols < (uint32_t)(kPipes * GE * N)) tmem_cols <<= 1;
+    if (threadIdx.x == 0) {
+        for (int pp = 0; pp < kPipes; ++pp) {
+            for (int s = 0; s < S; ++s) {
+                mbar_init(&bars->full[pp][s], 1);
+                mbar_init(&bars->empty[pp][s], 1 + kEpiWarps);
+            }
+            for (int a = 0; a < GE; ++a) {
+                mbar_init(&bars->tfull[pp][a], 1);
+                mbar_init(&bars->tempty[pp][a], kEpiWarps);
+            }
+            mbar_init(&bars->mma_done[pp], 1);
+        }
+        mbar_init(&bars->q_full, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_ks);
+        prefetch_tmap(&tmap_q);
+    }
+    if (warp == kPipes) {
+        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto locate = [&](int g, int &b, int &ti) {
+        int lo = 0, hi = B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tile_pre[mid] <= g) lo = mid; else hi = mid - 1;
+        }
+        b = lo;
+        while (b < B - 1 && tile_pre[b + 1] <= g) ++b;
+        ti = g - tile_pre[b];
+    };
+    const uint32_t stage_tx = kTile * kKeyBytes + kTile * 4;
+    const bool any_tiles = pipe_count(0) + pipe_count(1) > 0;
+
+    if (warp < kPipes) {
+        // ------------------------------------------------------------ producer
+        const int pp = warp;
+        const int n_p = pipe_count(pp);
+        if (lane == 0 && n_p > 0) {
+            const uint64_t stream_policy = l2_evict_first_policy();
+            int issued = 0;
+            for (int i = 0; i < n_p; ++i) {
+                const int s = i % S, st = pp * S + s;
+                if (i >= S && !mbar_wait(&bars->empty[pp][s], ((i / S) & 1) ^ 1, p.status)) break;
+                if (pp == 0 && i == 0) {   // every row's query block, once
+                    mbar_arrive_expect_tx(&bars->q_full, rows * 16 * kKeyBytes);
+                    for (int b = 0; b < B; ++b)
+                        tma_load_2d(smem + lay.q_off + b * N * kKeyBytes, &tmap_q, &bars->q_full, 0, b * N);
+                }
+                mbar_arrive_expect_tx(&bars->full[pp][s], stage_tx);
+                int b, ti;
+                locate(tile_of(pp, i), b, ti);
+                uint8_t *kdst = smem + lay.k_off + st * kTile * kKeyBytes;
+                uint8_t *ksdst = smem + lay.ks_off + st * kKsStageBytes;
+                const int R = p.rows_per_load;
+                for (int j = 0; j < kTile / R; ++j) {
+                    const int64_t pos = (int64_t)ti * kTile + j * R;
+                    bool ok = true;
+                    int64_t row = 0;
+                    if (pos < seq_len[b]) {
+                        row = row_of(p, b, pos, &ok);
+                        if (!ok) { flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX); row = 0; }
+                    }
+                    tma_load_2d_hint(kdst + j * R * kKeyBytes, &tmap_k, &bars->full[pp][s], 0, (int32_t)row,
+                                     stream_policy);
+                    tma_load_1d_hint(ksdst + ks_slot_offset(j * R, R), &tmap_ks, &bars->full[pp][s], (int32_t)row,
+                                     stream_policy);
+                }
+                ++issued;
+            }
+            for (int i = max(0, issued - S); i < issued; ++i)
+                mbar_wait(&bars->full[pp][i % S], (i / S) & 1, p.status);
+            if (pp == 0 && issued > 0) mbar_wait(&bars->q_full, 0, p.status);
+        }
+    } else if (warp < 2 * kPipes) {
+        // ---------------------------------------------------------- MMA issuer
+        const int pp = warp - kPipes;
+        const int n_p = pipe_count(pp);
+        if (lane == 0) {
+            const uint32_t idesc = umma_idesc_e4m3_f32(kTile, N);
+            for (int i = 0; i < n_p; ++i) {
+                const int s = i % S, st = pp * S + s, a = i % GE;
+                if (!mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status)) break;
+                if (i >= GE && !mbar_wait(&bars->tempty[pp][a], ((i / GE) & 1) ^ 1, p.status)) break;
+                if (i == 0 && !mbar_wait(&bars->q_full, 0, p.status)) break;
+                int b, ti;
+                locate(tile_of(pp, i), b, ti);
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + lay.k_off + st * kTile * kKeyBytes);
+                const uint32_t b_addr = smem_u32(smem + lay.q_off + b * N * kKeyBytes);
+                const uint32_t d = tmem_base + (uint32_t)((pp * GE + a) * N);
+#pragma unroll
+                for (int k = 0; k < kKeyBytes / 32; ++k)
+                    umma_f8(d, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
+                            k > 0 ? 1u : 0u);
+                umma_commit(&bars->empty[pp][s]);
+                umma_commit(&bars->tfull[pp][a]);
+            }
+            umma_commit(&bars->mma_done[pp]);
+            mbar_wait(&bars->mma_done[pp], 0, p.status);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - kEpiWarp0;
+        const int pp = ew / (kMaxGroups * kEpiWarps);
+        const int a = (ew / kEpiWarps) % kMaxGroups;
+        const int quarter = warp & 3;
+        const int gi = pp * kMaxGroups + a;          // group index: groups are in position order
+        const int gid = cta * kGroups + gi;          // the group's segment in every row's list
+        const int gbar = kGroupBar0 + gi;
+        const int row_in_tile = quarter * 32 + lane;
+        const int ng = a < GE ? group_count(pp, a) : 0;
+        const uint32_t lt = (1u << lane) - 1u;
+        float *coef = reinterpret_cast<float *>(smem + lay.epi_off) + ew * (17 * T);
+        int32_t *qp = reinterpret_cast<int32_t *>(coef + 16 * T);
+        uint32_t *xch = reinterpret_cast<uint32_t *>(smem + lay.xch_off) + gi * (2 * kEpiWarps * kMaxRows);
+        const uint32_t acc_col = (uint32_t)((pp * GE + a) * N);
+        uint32_t base[kMaxRows] = {0u, 0u, 0u, 0u};
+        uint32_t thr[kMaxRows] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+        bool ok = true, overflow = false;
+        int cur_b = -1;
+        for (int j = 0; j < ng || j == 0; ++j) {
+            const bool have = j < ng;
+            float sc[kMaxRows];
+            uint32_t vis = 0;
+            int b = 0;
+            int64_t pos = 0;
+            if (have && ok) {
+                const int i = j * GE + a, s = i % S, st = pp * S + s;
+                int ti;
+                locate(tile_of(pp, i), b, ti);
+                if (b != cur_b) {
+                    __syncwarp();
+                    for (int u = lane; u < 16 * T; u += 32)
+                        coef[u] = __ldg(p.w + (int64_t)b * 16 * T + u) * __ldg(p.q_scale + (int64_t)b * 16 * T + u);
+                    for (int u = lane; u < T; u += 32) qp[u] = __ldg(p.q_pos + b * T + u);
+                    __syncwarp();
+                    cur_b = b;
+                }
+                bool w_ok = mbar_wait(&bars->tfull[pp][a], (j & 1), p.status) &&
+                            mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status);
+                if (__all_sync(0xffffffffu, w_ok)) {
+                    tc_fence_after();
+                    const float ks = *reinterpret_cast<const float *>(smem + lay.ks_off + st * kKsStageBytes +
+                                                                      ks_slot_offset(row_in_tile, p.rows_per_load));
+                    pos = (int64_t)ti * kTile + row_in_tile;
+                    const int len = seq_len[b];
+                    float *out = p.scores + (int64_t)b * T * p.scores_stride + pos;
+#pragma unroll
+                    for (int t = 0; t < kMaxRows; ++t) {
+                        if (t < T) {
+                            float acc[16];
+                            tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc_col + (uint32_t)(16 * t),
+                                      acc);
+                            float sum = 0.f;
+#pragma unroll
+                            for (int h = 0; h < 16; ++h) sum = fmaf(coef[16 * t + h], fmaxf(acc[h], 0.f), sum);
+                            const bool visible = pos < len && pos <= qp[t];
+                            sc[t] = ks * sum;
+                            if (pos < len) out[(int64_t)t * p.scores_stride] = visible ? sc[t] : -INFINITY;
+                            if (visible) vis |= 1u << t;
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&bars->tempty[pp][a]);
+                        mbar_arrive(&bars->empty[pp][s]);
+                    }
+                    if (j == 0) {   // the sample: into the CTA's histogram of each row
+#pragma unroll
+                        for (int t = 0; t < kMaxRows; ++t)
+                            if (t < T)
+                                warp_hist_add(hist + (b * T + t) * kHistWords, sample_bin(float_order_key(sc[t])),
+                                              (vis >> t) & 1u);
+                    }
+                } else {
+                    ok = false;
+                }
+            }
+            if (j == 0) {
+                // ---- sample exchange: CTA histogram -> row histograms -> thresholds
+                named_bar_sync(gbar, 128);
+                uint32_t *flag = misc + 1 + gi;   // per group: 1 = flushes the CTA, 2 = also computes thresholds
+                if (quarter == 0 && lane == 0) {
+                    __threadfence_block();
+                    *flag = atomicAdd(misc, 1u) == kGroups - 1 ? 1u : 0u;
+                    __threadfence_block();
+                }
+                named_bar_sync(gbar, 128);
+                if (*flag) {
+                    const int tid = quarter * 32 + lane;
+                    for (int u = tid; u < rows * kHistWords; u += 128)
+                        if (hist[u]) atomicAdd(cp.sample_hist + u, hist[u]);
+                    __threadfence();
+                    named_bar_sync(gbar, 128);
+                    if (quarter == 0 && lane == 0) *flag = atomicAdd(ctl + kSampleArrive, 1u) == (uint32_t)ncta - 1 ? 2u : 1u;
+                    named_bar_sync(gbar, 128);
+                    if (*flag == 2u) {   // the last CTA: one warp per row
+                        __threadfence();
+                        if (quarter < rows) {
+                            const int r = quarter;
+                            const int64_t n = (int64_t)__ldg(p.q_pos + r) + 1;
+                            uint32_t t_r = 0xFFFFFFFFu;   // n <= top_k: every key is selected, nothing to capture
+                            uint32_t *h = cp.sample_hist + r * kHistWords;
+                            if (n > cp.K) {
+                                // the sample's visible keys: the histogram's total
+                                uint32_t tot = 0;
+                                for (int u = lane; u < kHistWords; u += 32) tot += __ldcg(h + u);
+#pragma unroll
+                                for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+                                const double want = (double)cp.oversample * cp.K * (double)tot / (double)n + 16.0;
+                                const uint32_t target = (uint32_t)min((double)tot, ceil(want));
+                                t_r = row_threshold(h, target);
+                            } else {
+                                for (int u = lane; u < kHistWords; u += 32) h[u] = 0;
+                            }
+                            if (lane == 0) ctl[kThr + r] = t_r;
+                        }
+                        __threadfence();
+                        named_bar_sync(gbar, 128);
+                        if (quarter == 0 && lane == 0) {
+                            ctl[kSampleArrive] = 0;
+                            __threadfence();
+                            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ctl + kReady), "r"(1u) : "memory");
+                        }
+                    }
+                }
+                // every group waits for the thresholds (one poller per group)
+                bool r_ok = true;
+                if (quarter == 0 && lane == 0) r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
+                ok = named_bar_and(gbar, 128, ok && r_ok);
+                if (ok) {
+#pragma unroll
+                    for (int r = 0; r < kMaxRows; ++r)
+                        if (r < rows) thr[r] = __ldcg(ctl + kThr + r);
+                }
+            }
+            // ---- candidates of this tile, in position order within the group
+            uint32_t cm[kMaxRows] = {0u, 0u, 0u, 0u};
+            if (have && ok) {
+#pragma unroll
+                for (int t = 0; t < kMaxRows; ++t) {
+                    if (t < T) {
+                        uint32_t th = 0xFFFFFFFFu;
+#pragma unroll
+                        for (int r = 0; r < kMaxRows; ++r)
+                            if (r == b * T + t) th = thr[r];
+                        const bool cand = ((vis >> t) & 1u) && float_order_key(sc[t]) >= th;
+                        cm[t] = __ballot_sync(0xffffffffu, cand);
+                        if (lane == 0) xch[(j & 1) * kEpiWarps * kMaxRows + quarter * kMaxRows + t] = __popc(cm[t]);
+                    }
+                }
+            }
+            ok = named_bar_and(gbar, 128, ok);
+            if (!ok) break;
+            if (have) {
+#pragma unroll
+                for (int t = 0; t < kMaxRows; ++t) {
+                    if (t < T) {
+                        const uint32_t *c4 = xch + (j & 1) * kEpiWarps * kMaxRows + t;
+                        uint32_t below = 0, tot = 0;
+#pragma unroll
+                        for (int q = 0; q < kEpiWarps; ++q) {
+                            const uint32_t v = c4[q * kMaxRows];
+                            tot += v;
+                            if (q < quarter) below += v;
+                        }
+                        const int r = b * T + t;
+                        uint32_t bs = 0;
+#pragma unroll
+                        for (int rr = 0; rr < kMaxRows; ++rr)
+                            if (rr == r) bs = base[rr];
+                        if ((cm[t] >> lane) & 1u) {
+                            const uint32_t at = bs + below + __popc(cm[t] & lt);
+                            if (at < (uint32_t)kSegCap)
+                                cp.lists[((int64_t)r * cp.NG + gid) * kSegCap + at] =
+                                    make_uint2(float_order_key(sc[t]), (uint32_t)pos);
+                            else
+                                overflow = true;
+                        }
+#pragma unroll
+                        for (int rr = 0; rr < kMaxRows; ++rr)
+                            if (rr == r) base[rr] += tot;
+                    }
+                }
+            }
+        }
+        if (__any_sync(0xffffffffu, overflow) && lane == 0) atomicOr(ctl + kOverflow, 1u);
+        if (quarter == 0 && lane == 0) {
+#pragma unroll
+            for (int r = 0; r < kMaxRows; ++r) {
+                if (r < rows) {
+                    cp.counts[(int64_t)r * cp.NG + gid] = base[r];
+                    if (base[r]) atomicAdd(ctl + kTotal + r, base[r]);
+                }
+            }
+        }
+    }
+    (void)any_tiles;
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kPipes) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, tmem_cols);
+    }
+    if (threadIdx.x == 0) {
+        for (int pp = 0; pp < kPipes; ++pp) {
+            for (int s = 0; s < S; ++s) {
+                mbar_inval(&bars->full[pp][s]);
+                mbar_inval(&bars->empty[pp][s]);
+            }
+            for (int a = 0; a < GE; ++a) {
+                mbar_inval(&bars->tfull[pp][a]);
+                mbar_inval(&bars->tempty[pp][a]);
+            }
+            mbar_inval(&bars->mma_done[pp]);
+        }
+        mbar_inval(&bars->q_full);
+    }
+    __syncthreads();
+}
+
+// The combine of one (row, KV group): the group's heads over all splits, with
+// the sink, by 32 threads per head (4 columns each) -- the same operations in
+// the same order as combine_row_cta, so the outputs are identical.
+__device__ void combine_group(const Params &cp, int bt, int g) {
+    const attn::Params &at = cp.at;
+    const int hpg = DSA_Q_HEADS / at.G, splits = at.splits;
+    const int t = threadIdx.x, hh = t >> 5, c4 = t & 31;
+    if (hh >= hpg) return;
+    const int h = g * hpg + hh;
+    const int64_t gw = (int64_t)bt * DSA_Q_HEADS + h;
+    const float *ml = at.part_ml + gw * splits * 2;
+    const float sk = cp.sink ? __ldg(cp.sink + h) * attn::kLog2e : -INFINITY;
+    float M = sk;
+    for (int j = 0; j < splits; ++j) M = fmaxf(M, __ldcg(ml + 2 * j));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float L = (cp.sink && M != -INFINITY) ? exp2f(sk - M) : 0.f;
+    for (int j = 0; j < splits; ++j) {
+        const float m = __ldcg(ml + 2 * j), l = __ldcg(ml + 2 * j + 1);
+        const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (w != 0.f) v = __ldcg(reinterpret_cast<const float4 *>(at.part_o + (gw * splits + j) * DSA_V_DIM) + c4);
+        acc[0] = __fadd_rn(acc[0], __fmul_rn(v.x, w));
+        acc[1] = __fadd_rn(acc[1], __fmul_rn(v.y, w));
+        acc[2] = __fadd_rn(acc[2], __fmul_rn(v.z, w));
+        acc[3] = __fadd_rn(acc[3], __fmul_rn(v.w, w));
+        L = __fadd_rn(L, w != 0.f ? __fmul_rn(l, w) : 0.f);
+    }
+    __nv_bfloat16 *o = cp.O + gw * DSA_V_DIM + c4 * 4;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) o[u] = __float2bfloat16_rn(L > 0.f ? acc[u] / L : 0.f);
+    if (cp.lse && c4 == 0) cp.lse[gw] = (L > 0.f) ? (M + log2f(L)) / attn::kLog2e : -INFINITY;
+}
+
+// Phase 2 (fast): the exact selection of row r from its candidates, into
+// `sel` (shared, top_k entries, -1 padded) and, by CTA c == 0, into the
+// output.  `work` is shared memory for the list.
+__device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *sel, uint8_t *work) {
+    constexpr int NT = kThreads;
+    const int K = cp.K, NG = cp.NG;
+    auto *sh = reinterpret_cast<topk::Shared<NT> *>(work);
+    uint32_t *off = reinterpret_cast<uint32_t *>(work + align128(sizeof(topk::Shared<NT>)));
+    uint32_t *lkey = off + ((NG + 1 + 31) & ~31);
+    uint32_t *lpos = lkey + kListCap;
+    int64_t n = (int64_t)__ldg(cp.ix.q_pos + r) + 1;
+    if (n > cp.ix.Lmax) n = cp.ix.Lmax;
+    if (n < 0) n = 0;
+    const int kr = (int)(n < K ? n : K);
+    if (n <= K) {
+        for (int j = threadIdx.x; j < K; j += NT) sel[j] = j < n ? j : -1;
+    } else {
+        // segment offsets (NG <= NT)
+        const uint32_t v = threadIdx.x < NG ? __ldcg(cp.counts + (int64_t)r * NG + threadIdx.x) : 0u;
+        uint32_t m;
+        const uint32_t incl = topk::block_scan<NT>(v, sh->warp_tmp, &m);
+        if (threadIdx.x < NG) off[threadIdx.x] = incl - v;
+        if (threadIdx.x == 0) off[NG] = m;
+        __syncthreads();
+        // the candidates, in position order
+        const uint2 *segs = cp.lists + (int64_t)r * NG * kSegCap;
+        for (uint32_t j0 = 0; j0 < m; j0 += 4 * NT) {
+            uint2 e[4];
+            uint32_t jj[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t j = j0 + u * NT + threadIdx.x;
+                jj[u] = j;
+                e[u] = make_uint2(0u, 0u);
+                if (j < m) {
+                    int lo = 0, hi = NG - 1;   // last segment starting at or before j
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (off[mid] <= j) lo = mid; else hi = mid - 1;
+                    }
+                    e[u] = __ldcg(segs + (int64_t)lo * kSegCap + (j - off[lo]));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (jj[u] < m) {
+                    lkey[jj[u]] = e[u].x;
+                    lpos[jj[u]] = e[u].y;
+                }
+        }
+        __syncthreads();
+        // exact radix select of the k-th largest key: 11 + 11 + 10 bits
+        uint32_t prefix = 0u, mask = 0u, Krem = (uint32_t)K;
+#pragma unroll 1
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+            const int nb = pass == 2 ? 1024 : 2048;
+            for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+            __syncthreads();
+            for (uint32_t j = threadIdx.x; j < m; j += NT) {
+                const uint32_t k = lkey[j];
+                if ((k & mask) == prefix) atomicAdd(&sh->hist[(k >> shift) & (uint32_t)(nb - 1)], 1u);
+            }
+            __syncthreads();
+            topk::find_threshold<NT>(sh, nb, Krem);
+            prefix |= (uint32_t)sh->bin << shift;
+            mask |= (uint32_t)(nb - 1) << shift;
+            Krem -= sh->above;
+            __syncthreads();
+        }
+        const uint32_t Tstar = prefix, ties = Krem;
+        // compaction in position order: each thread a contiguous run of the list
+        const uint32_t per_t = (m + NT - 1) / NT;
+        const uint32_t lo = min(m, threadIdx.x * per_t), hi = min(m, lo + per_t);
+        uint32_t g = 0, e = 0;
+        for (uint32_t j = lo; j < hi; ++j) {
+            g += lkey[j] > Tstar;
+            e += lkey[j] == Tstar;
+        }
+        uint32_t dummy;
+        const uint32_t packed = (g << 16) | e;
+        const uint32_t excl = topk::block_scan<NT>(packed, sh->warp_tmp, &dummy) - packed;
+        uint32_t gb = excl >> 16, eb = excl & 0xFFFFu;
+        for (uint32_t j = lo; j < hi; ++j) {
+            const uint32_t k = lkey[j];
+            if (k > Tstar) {
+                sel[gb + (eb < ties ? eb : ties)] = (int32_t)lpos[j];
+                ++gb;
+            } else if (k == Tstar) {
+                if (eb < ties) sel[gb + eb] = (int32_t)lpos[j];
+                ++eb;
+            }
+        }
+        for (int j = kr + threadIdx.x; j < K; j += NT) sel[j] = -1;
+    }
+    __syncthreads();
+    if (c == 0) {
+        int32_t *out = cp.tk.idx + (int64_t)r * K;
+        for (int j = threadIdx.x; j < K; j += NT) out[j] = sel[j];
+        if (threadIdx.x == 0) cp.tk.count[r] = kr;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
+                         const __grid_constant__ CUtensorMap tmap_q, const Params cp) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
+    __shared__ uint32_t sync_flag;
+    __shared__ int n_combine;
+    __shared__ int combine_g[DSA_Q_HEADS];
+    pdl_begin();
+    const uint32_t G = gridDim.x;
+    uint32_t *status = cp.ix.status;
+    uint32_t *ctl = cp.ctl;
+    const uint32_t status_at_entry = load_status(status);
+    if (threadIdx.x == 0) n_combine = 0;
+
+    // ---- phase 1: key stream, sample, candidates
+    run_indexer_capture(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G);
+    if (status_at_entry & kNeedsInitBit) {
+        if (threadIdx.x == 0) flag_timeout(status);
+        return;
+    }
+    if (!grid_sync(ctl + kGridArrive, 1 * G, cp.bar, status, &sync_flag)) return;
+
+    // the sample was good for every row? (the same answer in every CTA)
+    bool fast = __ldcg(ctl + kOverflow) == 0u;
+    for (int r = 0; r < cp.rows; ++r) {
+        const int64_t n = (int64_t)__ldg(cp.ix.q_pos + r) + 1;
+        const uint32_t m = __ldcg(ctl + kTotal + r);
+        if (n > cp.K && (m < (uint32_t)cp.K || m > (uint32_t)kListCap)) fast = false;
+    }
+    if (blockIdx.x == 0 && threadIdx.x < kMaxRows + 1) {   // read by nobody after phase 1
+        if (threadIdx.x == 0) ctl[kReady] = 0;
+        else ctl[kThr + threadIdx.x - 1] = 0;
+    }
+
+    const int rows = cp.rows, C = cp.C;
+    if (fast) {
+        // ---- phase 2 (fast): every CTA of a row selects from the row's candidates
+        if ((int)blockIdx.x < rows * C) {
+            const int r = blockIdx.x / C, c = blockIdx.x % C;
+            int32_t *sel = reinterpret_cast<int32_t *>(smem);
+            select_from_candidates(cp, r, c, sel, smem + kSelBytes);
+            // attention CTA units of this row, positions from shared memory
+            const int G_kv = cp.at.G, splits = cp.at.splits, nt = cp.at.n_teams;
+            if ((int)threadIdx.x < nt * 128) {
+                const attn::TeamSmem teams{smem + kSelBytes, (uint32_t)align128(sizeof(attn::Smem))};
+                for (int u = c; u < G_kv * splits; u += C) {
+                    const int g = u / splits, split = u % splits;
+                    attn::cta_unit(cp.at, teams, split, g, r, 1, kUnitBar, cp.sink, cp.O, cp.lse, sel);
+                    if (splits > 1 && threadIdx.x == 0) {   // the unit's partial is written and fenced
+                        const uint32_t done = atomicAdd(ctl + kCombine + r * DSA_Q_HEADS + g, 1u);
+                        if (done == (uint32_t)splits - 1) combine_g[atomicAdd(&n_combine, 1)] = g;
+                    }
+                }
+            }
+            __syncthreads();
+            // the last unit of a (row, KV group) combines its heads
+            for (int q = 0; q < n_combine; ++q) {
+                const int g = combine_g[q];
+                if (threadIdx.x == 0) __threadfence();
+                __syncthreads();
+                combine_group(cp, r, g);
+                if (threadIdx.x == 0) ctl[kCombine + r * DSA_Q_HEADS + g] = 0;
+            }
+        }
+    } else {
+        // ---- the general path (as the fused layer-step without the indexer histogram)
+        if ((int)blockIdx.x < rows * C) {
+            auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(smem);
+            uint32_t *cache = reinterpret_cast<uint32_t *>(smem + align128(sizeof(topk::Shared<kThreads>)));
+            topk::select_row<kThreads>(cp.tk, sh, cache, blockIdx.x / C, blockIdx.x % C, C, true);
+        }
+        if (!grid_sync(ctl + kGridArrive, 2 * G, cp.bar, status, &sync_flag)) return;
+        {
+            const int nt = cp.at.n_teams;
+            if ((int)threadIdx.x < nt * 128) {
+                const attn::TeamSmem teams{smem, (uint32_t)align128(sizeof(attn::Smem))};
+                const int G_kv = cp.at.G, splits = cp.at.splits;
+                const int units = rows * G_kv * splits;
+                for (int u = blockIdx.x; u < units; u += G) {
+                    const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
+                    attn::cta_unit(cp.at, teams, split, g, bt, 1, kUnitBar, cp.sink, cp.O, cp.lse);
+                }
+            } else if ((int)threadIdx.x >= kTeams * 128 && (int)blockIdx.x < rows * C && C > 1) {
+                constexpr int kFree = kThreads - kTeams * 128;
+                topk::clear_row_share(cp.tk, blockIdx.x / C, blockIdx.x % C, C, false, threadIdx.x - kTeams * 128,
+                                      kFree);
+            }
+        }
+        if (!grid_sync(ctl + kGridArrive, 3 * G, cp.bar, status, &sync_flag)) return;
+        if ((int)blockIdx.x < rows * C && blockIdx.x % C == 0) topk::reset_row_ctl(cp.tk, blockIdx.x / C, C);
+        if (cp.at.splits > 1)
+          for (int gw = blockIdx.x; gw < rows * DSA_Q_HEADS; gw += G)
+            attn::combine_row_cta<kThreads>(cp.at.part_o, cp.at.part_ml, gw, cp.at.splits, cp.sink, cp.O, cp.lse,
+                                            reinterpret_cast<float *>(smem));
+    }
+
+    // ---- the last CTA out resets the words read by everyone after phase 1
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(ctl + kGridExit, 1u) == G - 1) {
+            ctl[kGridArrive] = 0;
+            ctl[kOverflow] = 0;
+            for (int r = 0; r < kMaxRows; ++r) ctl[kTotal + r] = 0;
+            __threadfence();
+            ctl[kGridExit] = 0;
+        }
+    }
+}
+
+}  // namespace capture
+
+// --------------------------------------------------------------- host side
+static size_t capture_smem_budget() { return device_info().smem_optin - 256; }
+
+int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
+    using namespace capture;
+    const DeviceInfo &dev = device_info();
+    plan->ok = false;
+    const int rows = B * T;
+    if (dev.num_sms <= 0 || rows > kMaxRows || T > kMaxRows || Lmax < kMinContext) return DSA_OK;
+    const int grid = dev.num_sms;
+    if (grid * kGroups > kThreads) return DSA_OK;   // the segment offsets are scanned one per thread
+    // all CTAs must be resident together: one per SM (occupancy asked once per device)
+    static std::mutex mu;
+    static int per_sm_cache[64];
+    static bool known[64] = {};
+    int dev_id = -1;
+    cudaError_t e = cudaGetDevice(&dev_id);
+    if (e != cudaSuccess || dev_id < 0 || dev_id >= 64) return cuda_fail(e, "cudaGetDevice");
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!known[dev_id]) {
+            if (int rc = ensure_smem_limit((const void *)dsa_layer_capture_kernel, capture_smem_budget(),
+                                           "cudaFuncSetAttribute(capture)"))
+                return rc;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_cache[dev_id], dsa_layer_capture_kernel,
+                                                              kThreads, capture_smem_budget());
+            if (e != cudaSuccess) return cuda_fail(e, "occupancy of the capture kernel");
+            known[dev_id] = true;
+        }
+        if (per_sm_cache[dev_id] < 1) return DSA_OK;
+    }
+    // the shared-memory layouts must fit: phase 1 with at least 3 stages, phase 2's list and attention teams
+    if (Layout(3, T, B).total + 1024 > capture_smem_budget()) return DSA_OK;
+    const size_t ng = (size_t)grid * kGroups;
+    const size_t fast2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 +
+                                                  (size_t)2 * kListCap * 4,
+                                              kTeams * align128(sizeof(attn::Smem)));
+    if (fast2 + 1024 > capture_smem_budget()) return DSA_OK;
+    plan->grid = grid;
+    plan->rows = rows;
+    plan->C = std::max(1, grid / rows);
+    plan->NG = (int)ng;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = (off + bytes + 255) & ~size_t(255);
+        return at;
+    };
+    plan->ctl_off = take(kCtlWords * 4);
+    plan->hist_off = take((size_t)rows * kHistWords * 4);
+    plan->counts_off = take((size_t)rows * ng * 4);
+    plan->lists_off = take((size_t)rows * ng * kSegCap * 8);
+    plan->topk_off = take((size_t)rows * topk::scratch_words(plan->C, topk::kListCap, false) * 4);
+    plan->scratch_bytes = off;
+    plan->ok = true;
+    return DSA_OK;
+}
+
+int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
+                   int32_t *count, uint8_t *scratch, cudaStream_t stream, void *start_event) {
+    using namespace capture;
+    const size_t budget = capture_smem_budget();
+    IndexerLaunch L;
+    if (int rc = prepare_indexer(ia, 0, 0, nullptr, budget, &L)) return rc;   // tensor maps and parameters
+    // pipeline depth for this kernel's own layout (every row's query block resident, the sample histograms)
+    int S = indexer::kMaxStages;
+    while (S > 2 && Layout(S, ia.T, ia.B).total + 1024 > budget) --S;
+    const size_t smem1 = Layout(S, ia.T, ia.B).total + 1024;
+    const size_t ng = (size_t)plan.grid * kGroups;
+    const size_t smem2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 +
+                                                  (size_t)2 * kListCap * 4,
+                                              kTeams * align128(sizeof(attn::Smem))) +
+                         1024;
+    const size_t top_fixed = align128(sizeof(topk::Shared<kThreads>));
+    const size_t smem = std::max({smem1, smem2, top_fixed + 1024 + 4096});
+    if (smem > budget || S < 3) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "capture kernel shared memory does not fit");
+
+    Params cp;
+    cp.ix = L.p;
+    cp.ix.stages = S;
+    cp.ix.groups = indexer::kMaxGroups;
+    cp.ix.hist_rows = 0;
+    cp.ix.q_resident = 1;
+    cp.at = attn::make_params(aa);
+    cp.sink = aa.sink;
+    cp.O = aa.O;
+    cp.lse = aa.lse;
+    cp.ctl = reinterpret_cast<uint32_t *>(scratch + plan.ctl_off);
+    cp.sample_hist = reinterpret_cast<uint32_t *>(scratch + plan.hist_off);
+    cp.counts = reinterpret_cast<uint32_t *>(scratch + plan.counts_off);
+    cp.lists = reinterpret_cast<uint2 *>(scratch + plan.lists_off);
+    cp.bar = barrier_cfg();
+    cp.rows = plan.rows;
+    cp.K = top_k;
+    cp.C = plan.C;
+    cp.NG = plan.NG;
+    cp.oversample = 2.0f;
+    topk::Params &tp = cp.tk;
+    tp.scores = ia.scores;
+    tp.stride = ia.scores_stride;
+    tp.q_pos = ia.q_pos;
+    tp.rows = plan.rows;
+    tp.K = top_k;
+    tp.C = plan.C;
+    tp.idx = idx;
+    tp.count = count;
+    tp.scratch = reinterpret_cast<uint32_t *>(scratch + plan.topk_off);
+    tp.scratch_row_words = topk::scratch_words(plan.C, topk::kListCap, false);
+    tp.status = ia.status;
+    {
+        const int64_t avail = (int64_t)(smem - 1024 - top_fixed) / 4;
+        const int64_t chunk = ((ia.Lmax + plan.C - 1) / plan.C + 3) & ~int64_t(3);
+        const int64_t cand = std::min<int64_t>(topk::kCandCap, avail / 4) / kWarps * kWarps;
+        const int64_t rest = avail - 2 * cand;
+        int64_t list = std::min<int64_t>(topk::kListCap, std::max<int64_t>(0, (rest - chunk) / 2));
+        if (list < 1024) list = std::min<int64_t>(topk::kListCap, rest / 4);
+        tp.smem_list = (int)list;
+        tp.cand_cap = (int)cand;
+        tp.cache_keys = (int)(rest - 2 * list);
+    }
+    tp.list_cap = topk::kListCap;
+    tp.Lmax = ia.Lmax;
+    tp.bar = cp.bar;
+
+    if (int rc = ensure_smem_limit((const void *)dsa_layer_capture_kernel, smem, "cudaFuncSetAttribute(capture)"))
+        return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // phase 1's sample and the grid barrier wait on every CTA
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (start_event) {
+        e = cudaEventRecord(static_cast<cudaEvent_t>(start_event), stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    e = cudaLaunchKernelEx(&cfg, dsa_layer_capture_kernel, L.tmap_k, L.tmap_ks, L.tmap_q, cp);
+    if (e != cudaSuccess) return cuda_fail(e, "capture layer-step launch");
+    return DSA_OK;
+}
+
+}  // namespace dsa

@@ -21,15 +21,111 @@ __device__ __forceinline__ void flag_error(uint32_t *status, int code) {
     if (status) atomicOr(status, 1u << code);
 }
 
+// Bit 31 of the status word: a cross-CTA wait ran out, so the workspace's
+// self-cleaning scratch (barrier counters, histograms, lists) may hold a
+// partial state.  Kernels that use that scratch refuse to run on it (they set
+// the timeout bit again and return) until dsa_workspace_init zeroes it.
+constexpr uint32_t kNeedsInitBit = 1u << 31;
+
+__device__ __forceinline__ void flag_timeout(uint32_t *status) {
+    if (status) atomicOr(status, (1u << DSA_ERR_DEVICE_TIMEOUT) | kNeedsInitBit);
+}
+
+// Status word as seen at kernel entry (read through L2; a plain load issued
+// early, so that its latency overlaps the kernel's first phase).
+__device__ __forceinline__ uint32_t load_status(const uint32_t *status) {
+    return status ? __ldcg(status) : 0u;
+}
+
 // Time limit of every spin-wait in device code (nanoseconds of the global
 // timer): far beyond any legitimate wait in these kernels, short enough that a
 // broken wait ends the kernel with an error status instead of a hang.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// Cross-CTA barrier settings of one launch: the time limit of its waits and a
+// number of arrivals added to every barrier's target.  `extra` is 0 except
+// under the library's failure injection (dsa_debug_inject), where it makes
+// the first barrier wait for an arrival that never comes, so that the wait
+// runs out after `limit_ns` and the kernel takes its error path.
+struct BarrierCfg {
+    uint64_t limit_ns = kWaitLimitNs;
+    uint32_t extra = 0;
+};
+// The settings for a launch made now (host side; see dsa_debug_inject).
+BarrierCfg barrier_cfg();
+
+// Bounded wait of thread 0 of a CTA until *bar >= target (acquire); false and
+// the timeout status when the limit runs out.
+__device__ __forceinline__ bool spin_until_at_least(const uint32_t *bar, uint32_t target, uint64_t limit_ns,
+                                                    uint32_t *status) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+    if (v >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        __nanosleep(32);
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+        if (v >= target) return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            flag_timeout(status);
+            return false;
+        }
+    }
+}
+
+// Barrier of all CTAs of a (cooperatively launched) grid: thread 0 of each CTA
+// arrives on *bar and waits (bounded) for `target` arrivals; `flag` is a
+// shared word that carries the outcome to the CTA.  Returns false after a
+// timeout (recorded in the status word).
+__device__ __forceinline__ bool grid_sync(uint32_t *bar, uint32_t target, const BarrierCfg &cfg, uint32_t *status,
+                                          uint32_t *flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(bar, 1u);
+        const bool ok = spin_until_at_least(bar, target + cfg.extra, cfg.limit_ns, status);
+        __threadfence();
+        *flag = ok ? 1u : 0u;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
+// Named barrier of `n` threads (whole warps) with id `id` (1..15).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier that also returns, to every participating thread, whether
+// `pred` was true in all of them.
+__device__ __forceinline__ bool named_bar_and(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+// Programmatic dependent launch, at the start of every kernel of this
+// library: wait until the grid this one was chained after (if it was
+// launched as a programmatic dependent) has completed and its memory is
+// visible, then allow the next chained grid to be scheduled.  Both are no-ops
+// for a kernel launched in plain stream order.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -80,7 +176,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
-    flag_error(status, DSA_ERR_DEVICE_TIMEOUT);
+    flag_timeout(status);
     return false;
 }
 

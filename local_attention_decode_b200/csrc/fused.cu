@@ -22,6 +22,7 @@
 //            clear the selection scratch for the next call;
 //   phase 4  combine: one CTA per (query, head).
 #include <algorithm>
+#include <mutex>
 
 #include "attention_impl.cuh"
 #include "indexer_impl.cuh"
@@ -36,6 +37,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kTeams = 4;                     // attention teams of 4 warps (named barriers 1..4)
 constexpr int kMaxRows = 16;                  // B * T handled by the fused path
 constexpr int kMaxHistRows = 8;               // rows whose first histogram the indexer builds
+constexpr int kUnitBar = 9;                   // named barrier of the attention teams of a CTA unit
 
 static_assert(kTeams * 4 < kWarps, "the attention teams must leave warps free in the CTA");
 
@@ -47,36 +49,13 @@ struct Params {
     __nv_bfloat16 *O;
     float *lse;
     uint32_t *grid_bar;   // [0] arrivals, [1] exits
+    BarrierCfg bar;       // time limit (and injected extra arrivals) of the grid barriers
     int rows;             // B * T
     int C;                // CTAs per row in the selection phase
     int hist_ready;
 };
 
 __host__ __device__ constexpr size_t smem_align(size_t x) { return (x + 127) & ~size_t(127); }
-
-// Barrier of all CTAs of the grid (bounded spin).
-__device__ bool grid_sync(uint32_t *bar, uint32_t target, uint32_t *status, uint32_t *flag) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t ok = 1;
-        __threadfence();
-        atomicAdd(bar, 1u);
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(bar) < target) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                flag_error(status, DSA_ERR_DEVICE_TIMEOUT);
-                ok = 0;
-                break;
-            }
-            __nanosleep(32);
-        }
-        __threadfence();
-        *flag = ok;
-    }
-    __syncthreads();
-    return *flag != 0;
-}
-
 
 __global__ void __launch_bounds__(kThreads, 1)
 dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
@@ -87,12 +66,18 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     // aligned by an offset from the array itself, so the compiler keeps the shared address space
     uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     __shared__ uint32_t sync_flag;
+    pdl_begin();
     const uint32_t G = gridDim.x;
     uint32_t *status = fp.ix.status;
+    const uint32_t status_at_entry = load_status(status);
 
     // ---- phase 1: indexer
     indexer::run_indexer(&tmap_k, &tmap_ks, &tmap_q, fp.ix, smem, blockIdx.x, G);
-    if (!grid_sync(fp.grid_bar, 1 * G, status, &sync_flag)) return;
+    if (status_at_entry & kNeedsInitBit) {   // the cross-CTA scratch is not in its clean state
+        if (threadIdx.x == 0) flag_timeout(status);
+        return;
+    }
+    if (!grid_sync(fp.grid_bar, 1 * G, fp.bar, status, &sync_flag)) return;
 
     // ---- phase 2: selection (candidate runs when the indexer built the first histogram;
     //      the round-by-round path otherwise, or when the candidates would not fit)
@@ -104,33 +89,34 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         if (fp.hist_ready && fp.C > 1) done = topk::select_row_hist<kThreads>(fp.tk, sh, cache, row, c, fp.C);
         if (!done) topk::select_row<kThreads>(fp.tk, sh, cache, row, c, fp.C, true);
     }
-    if (!grid_sync(fp.grid_bar, 2 * G, status, &sync_flag)) return;
+    if (!grid_sync(fp.grid_bar, 2 * G, fp.bar, status, &sync_flag)) return;
 
-    // ---- phase 3: attention units
+    // ---- phase 3: attention, one CTA unit (n_teams teams of 64 keys) at a time
     {
-        const int team = warp_id() / 4;
-        if (team < kTeams) {
-            attn::Smem &sm = *reinterpret_cast<attn::Smem *>(smem + team * smem_align(sizeof(attn::Smem)));
+        const int nt = fp.at.n_teams;
+        if ((int)threadIdx.x < nt * 128) {
+            const attn::TeamSmem teams{smem, (uint32_t)smem_align(sizeof(attn::Smem))};
             const int G_kv = fp.at.G, splits = fp.at.splits;
             const int units = fp.rows * G_kv * splits;
-            for (int u = team * (int)G + (int)blockIdx.x; u < units; u += kTeams * (int)G) {
+            for (int u = blockIdx.x; u < units; u += G) {
                 const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
-                attn::attn_unit(fp.at, sm, split, g, bt, threadIdx.x & 127, 1 + team);
+                attn::cta_unit(fp.at, teams, split, g, bt, 1, kUnitBar, fp.sink, fp.O, fp.lse);
             }
-        } else if ((int)blockIdx.x < fp.rows * fp.C && (fp.C > 1 || fp.hist_ready)) {
+        } else if ((int)threadIdx.x >= kTeams * 128 && (int)blockIdx.x < fp.rows * fp.C && (fp.C > 1 || fp.hist_ready)) {
             // the warps outside the teams clear the selection scratch for the next call
             constexpr int kFree = kThreads - kTeams * 128;
             topk::clear_row_share(fp.tk, blockIdx.x / fp.C, blockIdx.x % fp.C, fp.C, fp.hist_ready != 0,
                                   threadIdx.x - kTeams * 128, kFree);
         }
     }
-    if (!grid_sync(fp.grid_bar, 3 * G, status, &sync_flag)) return;
+    if (!grid_sync(fp.grid_bar, 3 * G, fp.bar, status, &sync_flag)) return;
     if ((int)blockIdx.x < fp.rows * fp.C && blockIdx.x % fp.C == 0) topk::reset_row_ctl(fp.tk, blockIdx.x / fp.C, fp.C);
 
-    // ---- phase 4: combine, one CTA per (query, head)
-    for (int gw = blockIdx.x; gw < fp.rows * DSA_Q_HEADS; gw += G)
-        attn::combine_row_cta<kThreads>(fp.at.part_o, fp.at.part_ml, gw, fp.at.splits, fp.sink, fp.O, fp.lse,
-                                        reinterpret_cast<float *>(smem));
+    // ---- phase 4: combine of the units, one CTA per (query, head)
+    if (fp.at.splits > 1)
+        for (int gw = blockIdx.x; gw < fp.rows * DSA_Q_HEADS; gw += G)
+            attn::combine_row_cta<kThreads>(fp.at.part_o, fp.at.part_ml, gw, fp.at.splits, fp.sink, fp.O, fp.lse,
+                                            reinterpret_cast<float *>(smem));
 
     // ---- the last CTA out resets the grid barrier for the next call
     __syncthreads();
@@ -160,13 +146,27 @@ int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {
     if (dev.num_sms <= 0 || rows > kMaxRows) return DSA_OK;
     const int64_t max_tiles = (int64_t)B * ((Lmax + indexer::kTile - 1) / indexer::kTile);
     // all CTAs must be resident at once (the phases wait on each other): as many as fit
+    // (the occupancy query is made once per device)
+    static std::mutex mu;
+    static int per_sm_cache[64];
+    static bool known[64] = {};
+    int dev_id = -1;
+    cudaError_t e = cudaGetDevice(&dev_id);
+    if (e != cudaSuccess || dev_id < 0 || dev_id >= 64) return cuda_fail(e, "cudaGetDevice");
     int per_sm = 0;
-    cudaError_t e = cudaFuncSetAttribute(dsa_layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)fused_smem_budget());
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dsa_layer_fused_kernel, kThreads,
-                                                          fused_smem_budget());
-    if (e != cudaSuccess) return cuda_fail(e, "occupancy of the fused kernel");
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!known[dev_id]) {
+            if (int rc = ensure_smem_limit((const void *)dsa_layer_fused_kernel, fused_smem_budget(),
+                                           "cudaFuncSetAttribute(fused)"))
+                return rc;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_cache[dev_id], dsa_layer_fused_kernel, kThreads,
+                                                              fused_smem_budget());
+            if (e != cudaSuccess) return cuda_fail(e, "occupancy of the fused kernel");
+            known[dev_id] = true;
+        }
+        per_sm = per_sm_cache[dev_id];
+    }
     per_sm = std::min(per_sm, 1);
     if (per_sm < 1 || rows > per_sm * dev.num_sms) return DSA_OK;
     // every CTA takes part in every phase: at least one CTA per row for the selection
@@ -206,6 +206,7 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     fp.O = aa.O;
     fp.lse = aa.lse;
     fp.grid_bar = scratch;
+    fp.bar = barrier_cfg();
     fp.rows = plan.rows;
     fp.C = plan.C;
     fp.hist_ready = hist_rows > 0;
@@ -240,9 +241,10 @@ int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &a
     }
     tp.list_cap = topk::kListCap;
     tp.Lmax = ia.Lmax;
+    tp.bar = fp.bar;
 
-    cudaError_t e = cudaFuncSetAttribute(dsa_layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fused)");
+    if ((rc = ensure_smem_limit((const void *)dsa_layer_fused_kernel, smem, "cudaFuncSetAttribute(fused)"))) return rc;
+    cudaError_t e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.grid);
     cfg.blockDim = dim3(kThreads);

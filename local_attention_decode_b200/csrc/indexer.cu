@@ -4,6 +4,8 @@
 #include <algorithm>
 #include <cstdio>
 #include <cudaTypedefs.h>
+#include <cstring>
+#include <mutex>
 
 #include "indexer_impl.cuh"
 #include "kernels.h"
@@ -15,6 +17,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
                const __grid_constant__ CUtensorMap tmap_q, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    pdl_begin();
     // aligned by an offset from the array itself, so the compiler keeps the shared address space
     uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     run_indexer(&tmap_k, &tmap_ks, &tmap_q, p, smem, blockIdx.x, gridDim.x);
@@ -33,8 +36,42 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
+// Tensor-map encoding with a small cache: a decode loop calls the indexer with
+// the same buffers step after step, and the encoding is host work on the
+// critical path of every call.
+struct MapKey {
+    int device, dt, rank, swz;
+    const void *base;
+    uint64_t dims[2], strides[1];
+    uint32_t box[2];
+};
+
 static int make_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
                     const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz) {
+    static std::mutex mu;
+    static MapKey keys[32];
+    static CUtensorMap maps[32];
+    static int used = 0, next = 0;
+    MapKey k;
+    memset(&k, 0, sizeof k);
+    cudaGetDevice(&k.device);
+    k.dt = (int)dt;
+    k.rank = rank;
+    k.swz = (int)swz;
+    k.base = base;
+    for (int i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+    }
+    if (rank > 1) k.strides[0] = strides_bytes[0];
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (memcmp(&keys[i], &k, sizeof k) == 0) {
+                *map = maps[i];
+                return DSA_OK;
+            }
+    }
     auto enc = get_encode();
     if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     uint32_t estr[2] = {1, 1};
@@ -47,6 +84,10 @@ static int make_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, 
                     "tensor map encoding failed for %s (CUresult %d; base %p, dims %llu x %llu, box %u x %u)", what,
                     (int)r, base, (unsigned long long)dims[0], (unsigned long long)(rank > 1 ? dims[1] : 1),
                     box[0], rank > 1 ? box[1] : 1u);
+    std::lock_guard<std::mutex> lock(mu);
+    const int slot = used < 32 ? used++ : (next++ & 31);
+    keys[slot] = k;
+    maps[slot] = *map;
     return DSA_OK;
 }
 
@@ -129,10 +170,9 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream) {
     IndexerLaunch L;
     int rc = prepare_indexer(a, 0, 0, nullptr, device_info().smem_optin, &L);
     if (rc) return rc;
-    cudaError_t e = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer)");
-    indexer_kernel<<<L.grid, kThreads, L.smem, stream>>>(L.tmap_k, L.tmap_ks, L.tmap_q, L.p);
-    e = cudaGetLastError();
+    if ((rc = ensure_smem_limit((const void *)indexer_kernel, L.smem, "cudaFuncSetAttribute(indexer)"))) return rc;
+    cudaError_t e = launch_kernel(indexer_kernel, dim3(L.grid), dim3(kThreads), L.smem, stream, L.tmap_k, L.tmap_ks,
+                                  L.tmap_q, L.p);
     if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
     return DSA_OK;
 }

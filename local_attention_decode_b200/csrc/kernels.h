@@ -20,6 +20,37 @@ struct DeviceInfo {
 };
 const DeviceInfo &device_info();
 
+// Raises a kernel's dynamic shared memory limit to at least `bytes` on the
+// current device; the attribute call is made only when the cached limit is
+// lower (it is per device and per kernel, and costs a driver call).
+int ensure_smem_limit(const void *kernel, size_t bytes, const char *what);
+
+// Launches made from this host thread while a dsa_layer_chain call is
+// enqueueing carry the programmatic-stream-serialization attribute (each
+// kernel may be scheduled before the previous one ends; pdl_begin orders
+// their memory).
+bool pdl_launches();
+void set_pdl_launches(bool on);
+
+// A plain (non-cooperative) launch, chained when pdl_launches().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (pdl_launches()) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Sets the thread-local error message and returns `code`.
 int fail(int code, const char *fmt, ...);
 // Converts a CUDA runtime error into DSA_ERR_CUDA with a message.
@@ -68,8 +99,66 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
                 int top_k, int32_t *idx, int32_t *count, uint32_t *scratch, uint32_t *status,
                 cudaStream_t stream);
 
+// ------------------------------------------------------ index-K / index-Q producer
+struct ProduceArgs {
+    const __nv_bfloat16 *k_in;   // [B*T][128]
+    const __nv_bfloat16 *q_in;   // [B*T][16][128] or null
+    const float *ln_w, *ln_b;
+    float ln_eps;
+    int rope_dim;
+    double rope_base;
+    const dsa_kv_t *kv;
+    const int32_t *q_pos;
+    int B, T;
+    uint8_t *q8;
+    float *q_scale;
+    uint32_t *status;
+};
+int launch_index_produce(const ProduceArgs &a, cudaStream_t stream);
+
+// ------------------------------------------------------ indexer warm-up KL
+struct KlArgs {
+    const __nv_bfloat16 *Q;
+    const dsa_kv_t *kv;
+    const float *scores;
+    int64_t scores_stride;
+    const int32_t *q_pos;
+    int B, T;
+    int64_t Lmax;
+    float sm_scale;
+    float *kl_out;
+    float *target;
+    int64_t target_stride;
+    void *scratch;
+    uint32_t *status;
+};
+size_t kl_workspace_bytes(int B, int T, int64_t Lmax);
+int launch_indexer_kl(const KlArgs &a, cudaStream_t stream);
+
+// -------------------------------------------------- context-sharded decode
+int launch_shard_positions(const int32_t *q_pos, int rows, int64_t offset, int64_t len, int32_t *q_local,
+                           uint32_t *bad, cudaStream_t stream);
+int launch_shard_candidates(const float *scores, int64_t stride, const int32_t *idx, int K, int rows, int64_t offset,
+                            float *cand_score, int32_t *cand_pos, cudaStream_t stream);
+int launch_shard_merge(const float *cand_score, const int32_t *cand_pos, int N, int K, int rows, int64_t rank_offset,
+                       int64_t rank_len, int32_t *idx_out, int32_t *count_out, int32_t *local_idx,
+                       int32_t *local_count, cudaStream_t stream);
+int launch_shard_combine(const __nv_bfloat16 *O_all, const float *lse_all, int N, int rows, const float *sink,
+                         __nv_bfloat16 *O, float *lse, cudaStream_t stream);
+
 // ------------------------------------------------------------- attention
-constexpr int kAttnChunk = 64;   // keys per split
+constexpr int kAttnChunk = 64;   // keys per team chunk (one team of 4 warps)
+constexpr int kAttnMaxTeams = 4;
+// Team chunks per CTA unit, and CTA units per (query, KV head), for a key set
+// of at most max_keys keys: units of up to 256 keys.
+inline int attn_teams(int max_keys) {
+    const int c = (max_keys + kAttnChunk - 1) / kAttnChunk;
+    return c < kAttnMaxTeams ? (c > 0 ? c : 1) : kAttnMaxTeams;
+}
+inline int attn_splits(int max_keys) {
+    const int u = kAttnChunk * attn_teams(max_keys);
+    return (max_keys + u - 1) / u;
+}
 struct AttnArgs {
     const __nv_bfloat16 *Q;
     const dsa_kv_t *kv;
@@ -102,6 +191,23 @@ struct FusedPlan {
     size_t scratch_bytes = 0;   // grid barrier words + per-row selection scratch
 };
 int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan);
+
+// ------------------------------------------- layer-step with candidate capture
+// The fused layer-step for B * T <= 4 rows of long contexts (capture.cu): the
+// key stream samples the scores and keeps every key above a threshold in
+// position-ordered candidate lists, so the selection needs one grid barrier.
+struct CapturePlan {
+    bool ok = false;            // false: use the fused or the separate kernels
+    int grid = 0;
+    int rows = 0;
+    int C = 1;                  // CTAs per row
+    int NG = 0;                 // epilogue groups in the grid (segments of each row's list)
+    size_t ctl_off = 0, hist_off = 0, counts_off = 0, lists_off = 0, topk_off = 0;
+    size_t scratch_bytes = 0;   // all of the above (self-cleaning parts and overwritten parts)
+};
+int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan);
+int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
+                   int32_t *count, uint8_t *scratch, cudaStream_t stream, void *start_event = nullptr);
 int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
                  int32_t *count, uint32_t *scratch, cudaStream_t stream,
                  void *start_event = nullptr);

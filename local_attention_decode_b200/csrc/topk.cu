@@ -15,9 +15,11 @@ constexpr int kMaxCacheKeys = 32 * 1024;    // 128 KB of cached keys per CTA
 __global__ void __launch_bounds__(kThreads, 1)
 topk_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    pdl_begin();
+    const uint32_t status_at_entry = p.C > 1 ? load_status(p.status) : 0u;
     Shared<kThreads> *sh = reinterpret_cast<Shared<kThreads> *>(smem_raw);
     uint32_t *cache = reinterpret_cast<uint32_t *>(smem_raw + sizeof(Shared<kThreads>));
-    select_row<kThreads>(p, sh, cache, blockIdx.x / p.C, blockIdx.x % p.C, p.C);
+    select_row<kThreads>(p, sh, cache, blockIdx.x / p.C, blockIdx.x % p.C, p.C, false, status_at_entry);
 }
 
 }  // namespace topk
@@ -30,7 +32,10 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
     plan->Lmax = Lmax;
     int C = 1;
     if (dev.num_sms > 0 && Lmax > top_k) {
-        int co_resident = dev.num_sms;   // one CTA per SM is always co-resident at this size
+        // rows * C CTAs, at most one per SM: the cooperative launch below
+        // guarantees they are all resident together (their row barriers wait
+        // on one another)
+        int co_resident = dev.num_sms;
         C = (int)std::max<int64_t>(1, std::min<int64_t>(co_resident / std::max(1, plan->rows),
                                                        (Lmax + kMinChunk - 1) / kMinChunk));
     }
@@ -79,8 +84,9 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
     p.smem_list = plan.smem_list;
     p.cand_cap = plan.cand_cap;
     p.Lmax = plan.Lmax;
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(topk)");
+    p.bar = barrier_cfg();
+    if (int rc = ensure_smem_limit((const void *)topk_kernel, plan.smem, "cudaFuncSetAttribute(topk)")) return rc;
+    cudaError_t e;
     const unsigned grid = (unsigned)(plan.rows * plan.ctas_per_row);
     if (plan.ctas_per_row > 1) {
         // the CTAs of a row wait on one another: they must all be resident
@@ -96,8 +102,7 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, topk_kernel, p);
     } else {
-        topk_kernel<<<grid, kThreads, plan.smem, stream>>>(p);
-        e = cudaGetLastError();
+        e = launch_kernel(topk_kernel, dim3(grid), dim3(kThreads), plan.smem, stream, p);
     }
     if (e != cudaSuccess) return cuda_fail(e, "topk launch");
     return DSA_OK;

@@ -94,6 +94,7 @@ struct Params {
     int smem_list;         // list entries that fit in shared memory after the cache (<= list_cap)
     int cand_cap;          // candidate entries in shared memory after the list (a multiple of NT / 32)
     int64_t Lmax;
+    BarrierCfg bar;        // time limit (and injected extra arrivals) of the row barriers
 };
 
 template <int NT>
@@ -227,25 +228,17 @@ __device__ __forceinline__ uint32_t warp_sum_prefix(const uint32_t *a, int upto)
 }
 
 // Barrier among the C CTAs of a row: arrive, then wait (bounded) until
-// `target` arrivals have been counted.
+// `target` (+ the injected extra, normally 0) arrivals have been counted.
 template <int NT>
-__device__ bool row_barrier(Shared<NT> *sh, uint32_t *bar, uint32_t target, uint32_t *status) {
+__device__ bool row_barrier(Shared<NT> *sh, uint32_t *bar, uint32_t target, const BarrierCfg &cfg,
+                            uint32_t *status) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        uint32_t ok = 1;
         __threadfence();
         atomicAdd(bar, 1u);
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(bar) < target) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                flag_error(status, DSA_ERR_DEVICE_TIMEOUT);
-                ok = 0;
-                break;
-            }
-            __nanosleep(32);
-        }
+        const bool ok = spin_until_at_least(bar, target + cfg.extra, cfg.limit_ns, status);
         __threadfence();
-        sh->ok = ok;
+        sh->ok = ok ? 1u : 0u;
     }
     __syncthreads();
     return sh->ok != 0;
@@ -350,9 +343,12 @@ __device__ __forceinline__ void emit_slice(Shared<NT> *sh, int64_t len, int64_t 
 // 2 * p.smem_list list words, then 2 * p.cand_cap candidate words.
 // defer_clear: leave the row's scratch words for clear_row_share and
 // reset_row_ctl (called once every CTA of the row is past the selection).
+// status_at_entry: the status word as the kernel read it at entry; when it
+// says the scratch needs re-initialisation the row is not selected (the
+// timeout is flagged again) before any cross-CTA word is touched.
 template <int NT>
 __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int row, int c, int C,
-                           bool defer_clear = false) {
+                           bool defer_clear = false, uint32_t status_at_entry = 0u) {
     const int K = p.K;
     int64_t n = (int64_t)__ldg(p.q_pos + row) + 1;
     if (n > p.Lmax) {   // a position beyond the scores buffer: flag it, select within the buffer
@@ -420,13 +416,17 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     auto exchange_hist = [&](uint32_t *g, int nb) -> bool {
         for (int j = threadIdx.x; j < nb; j += NT)
             if (sh->hist[j]) atomicAdd(g + j, sh->hist[j]);
-        if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return false;
+        if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.bar, p.status)) return false;
         load_hist<NT>(sh, g, nb);
         return true;
     };
 
     // ---- digit 1
     slice_hist(0u, 0u, 21, kBins);
+    if (C > 1 && (status_at_entry & kNeedsInitBit)) {
+        if (threadIdx.x == 0) flag_timeout(p.status);
+        return;
+    }
     if (C > 1 && !exchange_hist(rs + kHist1, kBins)) return;
     find_threshold<NT>(sh, kBins, (uint32_t)K);
     uint32_t prefix = (uint32_t)sh->bin << 21, mask = 0xFFE00000u, Krem = (uint32_t)K - sh->above;
@@ -539,7 +539,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 });
             }
         }
-        if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
+        if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.bar, p.status)) return;
         m = __ldcg(ctl + 2);
         use_list = m <= (uint32_t)p.smem_list;
         if (use_list) {
@@ -649,7 +649,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
                 cnt[2 * c] = g;
                 cnt[2 * c + 1] = e;
             }
-            if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.status)) return;
+            if (!row_barrier<NT>(sh, ctl, ++barrier_no * C, p.bar, p.status)) return;
             uint32_t a = 0, e = 0;
             for (int j = threadIdx.x; j < c; j += NT) {
                 a += __ldcg(cnt + 2 * j);
@@ -790,7 +790,7 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
         }
     }
     for (int j = threadIdx.x; j < 1024; j += NT) sh->hist[j] = 0;   // for digit 2, filled while the list loads
-    if (!row_barrier<NT>(sh, ctl, (uint32_t)C, p.status)) return true;
+    if (!row_barrier<NT>(sh, ctl, (uint32_t)C, p.bar, p.status)) return true;
 
     // ---- the whole list into shared memory, with the digit-2 histogram of
     //      the keys in the threshold bin on the way

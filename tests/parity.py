@@ -83,10 +83,23 @@ def oracle_attention_rows(wl, b: int, t: int, positions: np.ndarray, sink, sm_sc
     return oracle.gqa_attention(bits16(wl.Q[b, t]), Ks, Vs, np.arange(len(positions), dtype=np.int32), s, sm_scale)
 
 
-def selection_is_valid(sel: np.ndarray, ref_scores: np.ndarray, k: int) -> bool:
-    """Every selected position's oracle score >= the oracle's k-th score minus 1e-3 relative."""
+def selection_agrees_outside_tie_band(sel: np.ndarray, ref_scores: np.ndarray, k: int) -> bool:
+    """A selection made from independently computed scores, checked against
+    the oracle's scores: the tie band is every position whose oracle score is
+    within 1e-3 relative of the oracle's k-th score (where rounding of the
+    GPU's fp32 scores may reorder keys).  Outside the band the selection must
+    equal the oracle's exactly -- every position above the band selected, none
+    below it -- so at most |band| positions can differ from the oracle's top-k,
+    and only inside the band."""
     n = ref_scores.shape[0]
     if n <= k:
         return np.array_equal(np.sort(sel), np.arange(n))
+    if len(np.unique(sel)) != len(sel) or len(sel) != k:
+        return False
     kth = np.partition(ref_scores, n - k)[n - k]
-    return bool(np.all(ref_scores[sel] >= kth - 1e-3 * abs(kth))) and len(np.unique(sel)) == len(sel) == k
+    tol = 1e-3 * abs(kth)
+    chosen = np.zeros(n, bool)
+    chosen[sel] = True
+    above = ref_scores > kth + tol
+    below = ref_scores < kth - tol
+    return bool(np.all(chosen[above]) and not np.any(chosen[below]))

@@ -106,3 +106,31 @@ def test_prefill_workspace_covers_every_block(dsa):
         dsa.DSA_ERR_UNSUPPORTED_SHAPE
     assert dsa._lib.dsa_workspace_size(dsa.OP_PREFILL, 1, 0, 8192, 2048, ctypes.byref(size)) == \
         dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_batched_contiguous_stride_rejected_on_the_host(dsa):
+    """B > 1 sequences in one contiguous index cache need seq_stride % 16 == 0
+    (the per-row scale copies start at b * seq_stride); the check happens on
+    the host, before any device memory is touched, so placeholder (never
+    dereferenced) 16-byte-aligned addresses are enough here."""
+    lib = dsa._lib
+    fake = ctypes.c_void_p(1 << 20)
+    kv = dsa.dsa_kv_t()
+    kv.k = kv.v = kv.index_k = kv.index_k_scale = fake
+    kv.num_kv_heads = 4
+    kv.seq_stride = 1001
+    kv.num_rows = 4096
+    rc = lib.dsa_layer_decode(fake, fake, fake, fake, ctypes.byref(kv), fake, 2, 1, 1000, 2048, None,
+                              ctypes.c_float(0.07), fake, None, None, None, fake, 1 << 20, None, None)
+    assert rc == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert b"seq_stride" in lib.dsa_last_error()
+    rc = lib.dsa_indexer_scores(fake, fake, fake, ctypes.byref(kv), fake, 2, 1, 1000, fake, 1000, fake, 1 << 20,
+                                None)
+    assert rc == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_debug_inject_arguments_checked_on_the_host(dsa):
+    lib = dsa._lib
+    assert lib.dsa_debug_inject(5, 2_000_000) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_debug_inject(dsa.INJECT_BARRIER_TIMEOUT, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_debug_inject(dsa.INJECT_NONE, 0) == dsa.DSA_OK

@@ -44,6 +44,12 @@ def _without_workspace(scores, q_pos, top_k):
     return idx, cnt
 
 
+def _many_rows_with_ties(g):
+    s = torch.randn((74, 1, 10000), generator=g, device=DEV)
+    s[3, 0] = torch.randint(0, 3, (10000,), generator=g, device=DEV).float()
+    return s.contiguous()
+
+
 def test_noalloc_topk_matches_workspace_topk_on_consecutive_calls():
     g = torch.Generator(device=DEV).manual_seed(1234)
     cases = [
@@ -52,6 +58,11 @@ def test_noalloc_topk_matches_workspace_topk_on_consecutive_calls():
         # four rows of a speculative block with heavy ties, then again with other data
         (torch.randint(0, 7, (1, 4, 70000), generator=g, device=DEV).float(), None, 2048),
         (torch.randn((2, 4, 50000), generator=g, device=DEV), "ragged", 2048),
+        # 74 rows of ~10,000 positions: two CTAs per row, and the fixed scratch
+        # of 74 rows leaves room for a candidate list of only 976 entries
+        # (shortened to fit the 2 MiB array); row 3 has so many tied scores that
+        # the list overflows and the selection exchanges every digit instead
+        (_many_rows_with_ties(g), None, 2048),
     ]
     for scores, pos_kind, k in cases:
         B, T, L = scores.shape
