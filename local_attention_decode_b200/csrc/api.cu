@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -272,6 +273,35 @@ static int plan_prefill(int NQ, int64_t Lmax, int top_k, WsPlan *full, WsPlan *t
     return DSA_OK;
 }
 
+// The whole dsa_prefill workspace: the per-block layout (plan_prefill) at
+// the start, then, when the tensor-core path applies, its region, then a
+// one-token layer-step layout for the tokens it hands back (offsets shifted,
+// the status word shared at offset 0).
+struct PrefillLayout {
+    WsPlan full, tail;        // the per-block path
+    PrefillPlan cap;          // the tensor-core path (cap.ok)
+    size_t cap_base = 0;
+    WsPlan redo;              // one token at a time
+    size_t total = 0;
+};
+
+static int plan_prefill_layout(int NQ, int64_t Lmax, int top_k, PrefillLayout *pl) {
+    int rc = plan_prefill(NQ, Lmax, top_k, &pl->full, &pl->tail);
+    if (rc) return rc;
+    pl->total = pl->full.total;
+    if ((rc = plan_prefill_capture(NQ, Lmax, top_k, &pl->cap))) return rc;
+    if (!pl->cap.ok) return DSA_OK;
+    pl->cap_base = align_up(pl->total, 256);
+    size_t end = pl->cap_base + pl->cap.total;
+    if ((rc = plan_workspace(DSA_OP_LAYER, 1, 1, Lmax, top_k, &pl->redo))) return rc;
+    const size_t base = align_up(end, 256) - kStatusBytes;
+    for (size_t *o : {&pl->redo.scores, &pl->redo.idx, &pl->redo.count, &pl->redo.topk, &pl->redo.part_o,
+                      &pl->redo.part_ml, &pl->redo.total})
+        *o += base;
+    pl->total = pl->redo.total;
+    return DSA_OK;
+}
+
 int dsa_workspace_size(int op, int B, int T, int64_t Lmax, int top_k, size_t *bytes) {
     if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
     if (op == DSA_OP_PREFILL) {
@@ -280,10 +310,10 @@ int dsa_workspace_size(int op, int B, int T, int64_t Lmax, int top_k, size_t *by
         if (Lmax < 1 || Lmax >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "Lmax outside [1, 2^31)");
         if (top_k < 1 || top_k > DSA_MAX_TOPK)
             return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k, DSA_MAX_TOPK);
-        WsPlan full, tail;
-        int rc = plan_prefill(T, Lmax, top_k, &full, &tail);
+        PrefillLayout pl;
+        int rc = plan_prefill_layout(T, Lmax, top_k, &pl);
         if (rc) return rc;
-        *bytes = full.total;
+        *bytes = pl.total;
         return DSA_OK;
     }
     int rc = check_common(B, T);
@@ -587,21 +617,41 @@ int dsa_prefill(const void *q8, const float *q_scale, const float *w, const void
     if (NQ < 1) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "NQ=%d < 1", NQ);
     int rc = check_layer_args(q8, q_scale, w, Q, kv, q_pos, 1, std::min(NQ, DSA_MAX_T), Lmax, top_k, sm_scale, O);
     if (rc) return rc;
-    WsPlan full, tail;
-    if ((rc = plan_prefill(NQ, Lmax, top_k, &full, &tail))) return rc;
-    if ((rc = check_ws(ws, ws_bytes, full))) return rc;
+    PrefillLayout pl;
+    if ((rc = plan_prefill_layout(NQ, Lmax, top_k, &pl))) return rc;
+    if (ws_bytes < pl.total)
+        return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, pl.total);
+    if ((rc = check_ws(ws, ws_bytes, pl.full))) return rc;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint8_t *q8b = static_cast<const uint8_t *>(q8);
+    const __nv_bfloat16 *Qb = static_cast<const __nv_bfloat16 *>(Q);
+    __nv_bfloat16 *Ob = static_cast<__nv_bfloat16 *>(O);
+    auto tokens = [&](int t0, int T, const WsPlan &wp) {
+        return layer_run(q8b + (size_t)t0 * DSA_INDEX_HEADS * DSA_INDEX_DIM, q_scale + (size_t)t0 * DSA_INDEX_HEADS,
+                         w + (size_t)t0 * DSA_INDEX_HEADS, Qb + (size_t)t0 * DSA_Q_HEADS * DSA_QK_DIM, kv, q_pos + t0, 1,
+                         T, Lmax, top_k, sink, sm_scale, Ob + (size_t)t0 * DSA_Q_HEADS * DSA_V_DIM,
+                         lse ? lse + (size_t)t0 * DSA_Q_HEADS : nullptr, idx_out ? idx_out + (size_t)t0 * top_k : nullptr,
+                         count_out ? count_out + t0 : nullptr, ws, wp, s, nullptr);
+    };
+    if (pl.cap.ok) {
+        // the tensor-core path: the indexer as one contraction over all tokens
+        PrefillArgs a{q8b, q_scale, w, Qb, kv, q_pos, Lmax, sink, sm_scale, Ob, lse, idx_out, count_out,
+                      at<uint32_t>(ws, 0)};
+        std::vector<int32_t> redo(NQ);
+        int n_redo = 0;
+        rc = run_prefill_capture(pl.cap, a, static_cast<uint8_t *>(ws) + pl.cap_base, s, redo.data(), &n_redo);
+        if (rc == DSA_OK) {
+            // the tokens whose candidates did not hold their selection: the decode layer-step, one by one
+            for (int i = 0; i < n_redo; ++i)
+                if ((rc = tokens(redo[i], 1, pl.redo))) return rc;
+            return DSA_OK;
+        }
+        if (rc != DSA_ERR_UNSUPPORTED_SHAPE) return rc;
+    }
     // one layer-step per block of DSA_MAX_T query tokens, on the one layout
     for (int t0 = 0; t0 < NQ; t0 += DSA_MAX_T) {
         const int T = std::min(DSA_MAX_T, NQ - t0);
-        rc = layer_run(static_cast<const uint8_t *>(q8) + (size_t)t0 * DSA_INDEX_HEADS * DSA_INDEX_DIM,
-                       q_scale + (size_t)t0 * DSA_INDEX_HEADS, w + (size_t)t0 * DSA_INDEX_HEADS,
-                       static_cast<const __nv_bfloat16 *>(Q) + (size_t)t0 * DSA_Q_HEADS * DSA_QK_DIM, kv, q_pos + t0,
-                       1, T, Lmax, top_k, sink, sm_scale,
-                       static_cast<__nv_bfloat16 *>(O) + (size_t)t0 * DSA_Q_HEADS * DSA_V_DIM,
-                       lse ? lse + (size_t)t0 * DSA_Q_HEADS : nullptr, idx_out ? idx_out + (size_t)t0 * top_k : nullptr,
-                       count_out ? count_out + t0 : nullptr, ws, T == DSA_MAX_T || T == NQ ? full : tail, s, nullptr);
-        if (rc) return rc;
+        if ((rc = tokens(t0, T, T == DSA_MAX_T || T == NQ ? pl.full : pl.tail))) return rc;
     }
     return DSA_OK;
 }

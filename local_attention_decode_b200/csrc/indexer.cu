@@ -46,8 +46,11 @@ struct MapKey {
     uint32_t box[2];
 };
 
-static int make_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
+}  // namespace indexer
+
+int make_tensor_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
                     const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz) {
+    using namespace indexer;
     static std::mutex mu;
     static MapKey keys[32];
     static CUtensorMap maps[32];
@@ -91,8 +94,6 @@ static int make_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, 
     return DSA_OK;
 }
 
-}  // namespace indexer
-
 int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uint32_t *hist_global,
                     size_t smem_budget, IndexerLaunch *out) {
     using namespace indexer;
@@ -106,14 +107,14 @@ int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uin
         uint64_t dims[2] = {(uint64_t)kKeyBytes, (uint64_t)kv->num_rows};
         uint64_t strides[1] = {(uint64_t)kKeyBytes};
         uint32_t box[2] = {(uint32_t)kKeyBytes, (uint32_t)R};
-        int rc = make_map("index keys", &out->tmap_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->index_k, dims, strides,
+        int rc = make_tensor_map("index keys", &out->tmap_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->index_k, dims, strides,
                           box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }
     {
         uint64_t dims[1] = {(uint64_t)kv->num_rows};
         uint32_t box[1] = {(uint32_t)R};
-        int rc = make_map("index key scales", &out->tmap_ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, kv->index_k_scale,
+        int rc = make_tensor_map("index key scales", &out->tmap_ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, kv->index_k_scale,
                           dims, nullptr, box, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc) return rc;
     }
@@ -121,7 +122,7 @@ int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uin
         uint64_t dims[2] = {(uint64_t)kKeyBytes, (uint64_t)a.B * T * 16};
         uint64_t strides[1] = {(uint64_t)kKeyBytes};
         uint32_t box[2] = {(uint32_t)kKeyBytes, (uint32_t)N};
-        int rc = make_map("index queries", &out->tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q8, dims, strides, box,
+        int rc = make_tensor_map("index queries", &out->tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q8, dims, strides, box,
                           CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     }

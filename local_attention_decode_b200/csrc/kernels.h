@@ -72,6 +72,9 @@ struct IndexerArgs {
 int launch_indexer(const IndexerArgs &a, cudaStream_t stream);
 
 namespace indexer { struct Params; }
+// Tiled tensor map (cached per device, base, shape and box; see indexer.cu).
+int make_tensor_map(const char *what, CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
+                    const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz);
 // Everything a launch of the indexer body needs: tensor maps, parameters,
 // dynamic shared memory and grid (one CTA per SM, two pipelines per CTA).  hist_rows > 0 adds each
 // CTA's histogram of the visible scores (see indexer::kHistWords) into hist_global.
@@ -97,7 +100,7 @@ struct TopkPlan {
 int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_scratch_bytes = SIZE_MAX);
 int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const int32_t *q_pos,
                 int top_k, int32_t *idx, int32_t *count, uint32_t *scratch, uint32_t *status,
-                cudaStream_t stream);
+                cudaStream_t stream, float *kth = nullptr);
 
 // ------------------------------------------------------ index-K / index-Q producer
 struct ProduceArgs {
@@ -134,6 +137,37 @@ struct KlArgs {
 };
 size_t kl_workspace_bytes(int B, int T, int64_t Lmax);
 int launch_indexer_kl(const KlArgs &a, cudaStream_t stream);
+
+// ------------------------------------------------ chunked prefill (prefill.cu)
+struct PrefillPlan {
+    bool ok = false;
+    int NQ = 0, K = 0, nblocks = 0, B_rep = 0, s = 0, max_ps = 0, cap = 0, attn_chunk = 0;
+    int64_t Lmax = 0, Ls_cap = 0;
+    TopkPlan tp;
+    size_t topk_scratch = 0, sample_table = 0, sample_pos = 0, sample_scores = 0, sample_idx = 0, sample_cnt = 0,
+           thr = 0, meta = 0, block_max = 0, cand_cnt = 0, cand = 0, idx = 0, count = 0, redo_n = 0, redo = 0,
+           part_o = 0, part_ml = 0, total = 0;
+};
+struct PrefillArgs {
+    const uint8_t *q8;
+    const float *q_scale, *w;
+    const __nv_bfloat16 *Q;
+    const dsa_kv_t *kv;
+    const int32_t *q_pos;
+    int64_t Lmax;
+    const float *sink;
+    float sm_scale;
+    __nv_bfloat16 *O;
+    float *lse;
+    int32_t *idx_out, *count_out;
+    uint32_t *status;
+};
+int plan_prefill_capture(int NQ, int64_t Lmax, int top_k, PrefillPlan *plan);
+// Runs the four stages; the tokens whose candidates did not hold their
+// selection (written with count 0) are listed in redo_host[0 .. *n_redo).
+// Synchronises the stream (to read that list).
+int run_prefill_capture(const PrefillPlan &plan, const PrefillArgs &a, uint8_t *ws, cudaStream_t s,
+                        int32_t *redo_host, int *n_redo);
 
 // -------------------------------------------------- context-sharded decode
 int launch_shard_positions(const int32_t *q_pos, int rows, int64_t offset, int64_t len, int32_t *q_local,

@@ -65,7 +65,7 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
 }
 
 int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const int32_t *q_pos, int top_k,
-                int32_t *idx, int32_t *count, uint32_t *scratch, uint32_t *status, cudaStream_t stream) {
+                int32_t *idx, int32_t *count, uint32_t *scratch, uint32_t *status, cudaStream_t stream, float *kth) {
     using namespace topk;
     Params p;
     p.scores = scores;
@@ -85,6 +85,7 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
     p.cand_cap = plan.cand_cap;
     p.Lmax = plan.Lmax;
     p.bar = barrier_cfg();
+    p.kth = kth;
     if (int rc = ensure_smem_limit((const void *)topk_kernel, plan.smem, "cudaFuncSetAttribute(topk)")) return rc;
     cudaError_t e;
     const unsigned grid = (unsigned)(plan.rows * plan.ctas_per_row);

@@ -95,6 +95,7 @@ struct Params {
     int cand_cap;          // candidate entries in shared memory after the list (a multiple of NT / 32)
     int64_t Lmax;
     BarrierCfg bar;        // time limit (and injected extra arrivals) of the row barriers
+    float *kth = nullptr;  // optional [rows]: the k-th largest visible score (-inf when n <= K)
 };
 
 template <int NT>
@@ -363,7 +364,10 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     if (n <= K) {   // every visible position is selected (same decision in all CTAs of the row)
         if (c == 0) {
             for (int j = threadIdx.x; j < K; j += NT) out[j] = j < n ? j : -1;
-            if (threadIdx.x == 0) p.count[row] = (int32_t)(n > 0 ? n : 0);
+            if (threadIdx.x == 0) {
+                p.count[row] = (int32_t)(n > 0 ? n : 0);
+                if (p.kth) p.kth[row] = -INFINITY;
+            }
         }
         return;
     }
@@ -581,6 +585,8 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     take_digit(1024, 0);
     const uint32_t Tstar = prefix;
     const uint32_t ties = Krem;   // keys equal to T* that are taken (>= 1)
+    if (p.kth && c == 0 && threadIdx.x == 0)   // the k-th largest score itself (the inverse of float_order_key)
+        p.kth[row] = __uint_as_float((Tstar & 0x80000000u) ? (Tstar & 0x7FFFFFFFu) : ~Tstar);
 
     // ---- this CTA's offset in the row's output
     uint32_t gt_before = 0, eq_before = 0;

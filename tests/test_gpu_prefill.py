@@ -82,3 +82,52 @@ def test_prefill_8k_queries_at_1m_context_sampled():
         assert np.array_equal(idx[t].cpu().numpy(), np.sort(ref_idx)), f"token {t}"
         ref_o, ref_l = oracle_attention_rows(wl, 0, t, idx[t].cpu().numpy(), wl.sink, SM)
         assert_attn_close(O[t], ref_o, lse[t], ref_l)
+
+
+def _decode_blocks(wl, Lmax, top_k=2048):
+    """The same tokens through dsa_layer_decode, 16 at a time."""
+    NQ = wl.T
+    O = torch.empty((NQ, 64, 128), dtype=torch.bfloat16, device=DEV)
+    idx = torch.empty((NQ, top_k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((NQ,), dtype=torch.int32, device=DEV)
+    for t0 in range(0, NQ, 16):
+        T = min(16, NQ - t0)
+        sl = slice(t0, t0 + T)
+        ws = dsa.alloc_workspace(dsa.OP_LAYER, 1, T, Lmax, top_k)
+        O2 = torch.empty((1, T, 64, 128), dtype=torch.bfloat16, device=DEV)
+        idx2 = torch.empty((1, T, top_k), dtype=torch.int32, device=DEV)
+        cnt2 = torch.empty((1, T), dtype=torch.int32, device=DEV)
+        dsa.dsa_layer_decode(wl.q8[:, sl].contiguous(), wl.q_scale[:, sl].contiguous(), wl.w[:, sl].contiguous(),
+                             wl.Q[:, sl].contiguous(), kv_for(wl), wl.q_pos[:, sl].contiguous(), Lmax, top_k,
+                             wl.sink, SM, O2, None, idx2, cnt2, ws)
+        O[sl], idx[sl], cnt[sl] = O2[0], idx2[0], cnt2[0]
+    return O, idx, cnt
+
+
+@pytest.mark.parametrize("L,NQ,page_size", [(100000, 64, 0), (70000, 96, 64), (40000, 80, 128)])
+def test_tensor_core_prefill_equals_decode_blocks(L, NQ, page_size):
+    """NQ a multiple of 16 (>= 64): the indexer runs as one contraction with the
+    candidate filter; every token's selection and output equal the decode
+    layer-step's bit for bit."""
+    wl = make_decode_workload(seed=170 + NQ, seq_lens=[L], T=NQ, device=DEV, page_size=page_size, n_needles=16,
+                              needle_mode="zipf")
+    O, lse, idx, cnt = run_prefill(wl)
+    O2, idx2, cnt2 = _decode_blocks(wl, L)
+    assert torch.equal(cnt, cnt2) and torch.equal(idx, idx2)
+    assert torch.equal(O.view(torch.int16), O2.view(torch.int16))
+    for t in (0, NQ // 2, NQ - 1):   # and the attention against the oracle over the selection
+        c = int(cnt[t])
+        ref_o, ref_l = oracle_attention_rows(wl, 0, t, idx[t, :c].cpu().numpy(), wl.sink, SM)
+        assert_attn_close(O[t], ref_o, lse[t], ref_l)
+
+
+def test_tensor_core_prefill_hands_tied_tokens_to_the_decode_path():
+    """Every score tied (zero index queries): the candidate lists overflow, every
+    token takes the decode layer-step, and the result is still exact."""
+    wl = make_decode_workload(seed=180, seq_lens=[30000], T=64, device=DEV, n_needles=2)
+    wl.q8 = torch.zeros_like(wl.q8)
+    O, lse, idx, cnt = run_prefill(wl)
+    O2, idx2, cnt2 = _decode_blocks(wl, 30000)
+    assert torch.equal(cnt, cnt2) and torch.equal(idx, idx2)
+    assert torch.equal(idx[0].cpu(), torch.arange(2048, dtype=torch.int32))
+    assert torch.equal(O.view(torch.int16), O2.view(torch.int16))
