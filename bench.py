@@ -490,8 +490,10 @@ PREFILL_METRIC = "chunked-prefill DSA layer (8,192 query tokens at 1M context) t
 
 def run_prefill(args, rank, world, local_rank):
     """One step = dsa_prefill over 8,192 query tokens at positions
-    1,040,384..1,048,575 of a 1,048,576-token cache (each causal), i.e. 512
-    fused layer-step launches of 16 tokens.  L2 flushed before each step."""
+    1,040,384..1,048,575 of a 1,048,576-token cache (each causal): the sample
+    thresholds, the fp8 contraction with the candidate filter on the tensor
+    cores, the per-token selection and the attention.  L2 flushed before each
+    step."""
     import torch
     import local_attention_decode_b200 as dsa
     from workloads import CONFIGS, make_decode_workload
@@ -546,7 +548,7 @@ def run_prefill(args, rank, world, local_rank):
         fp8_peak, fp8_kind = 2.0 * bf16, "measured bf16 x 2 (nominal fp8 : bf16 ratio)"
     except Exception:
         fp8_peak, fp8_kind = 2.0 * 1590.0, "fallback bf16 x 2"
-    key_bytes = -(-NQ // 16) * indexer_bytes(L, 16)          # keys streamed once per 16-token block
+    key_bytes = indexer_bytes(L, 0)                           # the keys streamed once by the contraction
     peak, peak_kind = measured_peaks()
     return {
         "metric": PREFILL_METRIC, "value": throughput(NQ, K, world, total_s), "unit": "tok/s", "n_gpus": world,
@@ -556,14 +558,16 @@ def run_prefill(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD_DESC["prefill_8k_1m"], "query_tokens": NQ, "context": L, "top_k": TOP_K,
                    "seed": cfg["seed"], "parallelism": f"replicas x{world}",
                    "l2": "flushed before each step outside the timed events"},
-        "roofline": {"kernel": "dsa_layer_fused_kernel x 512 (16-token blocks)", "bound": "tensor",
+        "roofline": {"kernel": "the whole dsa_prefill call (sample thresholds, prefill_capture_kernel contraction, "
+                               "per-token selection, attention); FLOPs of the indexer contraction only",
+                     "bound": "tensor",
                      "achieved": flops / step_s / 1e12, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": flops / step_s / 1e12 / fp8_peak, "peak_kind": fp8_kind, "traffic": None,
                      "algorithmic_flops_per_step": flops},
         "hbm_view": {"key_bytes_per_step": key_bytes, "achieved_GBps": key_bytes / step_s / 1e9, "peak": peak,
                      "frac": key_bytes / step_s / 1e9 / peak, "peak_kind": peak_kind},
         "e2e": None,
-        "gpu_launches": -(-NQ // 16) * K,
+        "gpu_launches": (6 + -(-NQ // 1024) * 2) * K,   # sample, indexer, selection, metadata, capture, select; attention + combine per 1,024 tokens
         "clocks": clocks,
     }
 
@@ -792,28 +796,53 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
         step()
     torch.cuda.synchronize(dev)
     K = args.steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    for i in range(K):
-        flush()
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    for w_ in (ws, ws_p):
-        st, _ = dsa.dsa_check_device_status(w_)
-        if st != dsa.DSA_OK:
-            raise RuntimeError(f"device status {st} in the end-to-end steps")
-    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
+
+    def timed(run):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            flush()
+            evs[i][0].record(stream)
+            run()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        return evs
+
+    eager = timed(step)
+    eager_ms = statistics.median([a.elapsed_time(b) for a, b in eager])
+    # the step captured once into a CUDA graph (copies, producer, cache writes,
+    # layer-step, copy back) and replayed: one launch per step from the host
+    graph_note = "captured once in a CUDA graph, replayed per step"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()   # one more warm-up on the capture stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize(dev)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        evs = timed(graph.replay)
+    except Exception as e:   # a launch that cannot be captured: the eager steps are the number
+        graph_note = f"eager (graph capture failed: {type(e).__name__}: {e})"
+        torch.cuda.synchronize(dev)
+        evs = timed(step)
+    for w_ in (ws, ws_p):    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
     import torch.distributed as dist
     world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
     return {"value": throughput(B * T, K, world, total_s), "unit": "tok/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K,
             "per_step": "1 pinned H2D copy of the token's raw inputs; dsa_index_produce (index key into the cache, "
                         "index query codes); 2 device copies of the K/V rows into the cache; dsa_layer_decode; "
-                        "1 D2H copy of O and the selection"}
+                        "1 D2H copy of O and the selection -- " + graph_note,
+            "ms_per_step_eager_median": eager_ms}
 
 
 # ------------------------------------------------------- CPU oracle timing

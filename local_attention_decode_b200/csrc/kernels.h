@@ -92,6 +92,7 @@ struct TopkPlan {
     int smem_list = 0;     // candidate-list entries that fit in shared memory
     int cand_cap = 0;      // per-warp candidate entries in shared memory, all warps together
     int64_t Lmax = 0;      // positions held by each scores row
+    bool var_c = false;    // CTAs per row follow the rows' lengths (ctas_per_row is then the most a row gets)
     size_t smem = 0;
     size_t scratch_bytes = 0;  // cross-CTA scratch (only when C > 1)
 };

@@ -11,6 +11,7 @@ namespace topk {
 constexpr int kThreads = 512;
 constexpr int kMinChunk = 4096;             // keys per CTA below which a row is not split further
 constexpr int kMaxCacheKeys = 32 * 1024;    // 128 KB of cached keys per CTA
+constexpr int kVarMinRows = 16;             // above this many rows, CTAs per row follow the rows' lengths
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_kernel(const Params p) {
@@ -19,6 +20,12 @@ topk_kernel(const Params p) {
     const uint32_t status_at_entry = p.C > 1 ? load_status(p.status) : 0u;
     Shared<kThreads> *sh = reinterpret_cast<Shared<kThreads> *>(smem_raw);
     uint32_t *cache = reinterpret_cast<uint32_t *>(smem_raw + sizeof(Shared<kThreads>));
+    if (p.var_c) {
+        int row, c, C;
+        row_of_cta<kThreads>(p, sh, &row, &c, &C);
+        if (row >= 0) select_row<kThreads>(p, sh, cache, row, c, C, false, status_at_entry);
+        return;
+    }
     select_row<kThreads>(p, sh, cache, blockIdx.x / p.C, blockIdx.x % p.C, p.C, false, status_at_entry);
 }
 
@@ -31,6 +38,7 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
     plan->threads = kThreads;
     plan->Lmax = Lmax;
     int C = 1;
+    plan->var_c = false;
     if (dev.num_sms > 0 && Lmax > top_k) {
         // rows * C CTAs, at most one per SM: the cooperative launch below
         // guarantees they are all resident together (their row barriers wait
@@ -38,8 +46,15 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
         int co_resident = dev.num_sms;
         C = (int)std::max<int64_t>(1, std::min<int64_t>(co_resident / std::max(1, plan->rows),
                                                        (Lmax + kMinChunk - 1) / kMinChunk));
+        // many rows of unequal length: CTAs in proportion to each row's length
+        // (decided on the device from the positions), up to grid - rows + 1 per row
+        if (plan->rows > kVarMinRows && plan->rows < co_resident && Lmax > 2 * kMinChunk) {
+            plan->var_c = true;
+            C = co_resident - plan->rows + 1;
+        }
     }
     int64_t chunk = ((Lmax + C - 1) / C + 3) & ~int64_t(3);
+    if (plan->var_c) chunk = kMaxCacheKeys;   // slices depend on the lengths: the most the cache holds
     plan->ctas_per_row = C;
     plan->cache_keys = (int)std::min<int64_t>(chunk, kMaxCacheKeys);
     plan->list_cap = 0;
@@ -86,9 +101,10 @@ int launch_topk(const TopkPlan &plan, const float *scores, int64_t stride, const
     p.Lmax = plan.Lmax;
     p.bar = barrier_cfg();
     p.kth = kth;
+    p.var_c = plan.var_c ? 1 : 0;
     if (int rc = ensure_smem_limit((const void *)topk_kernel, plan.smem, "cudaFuncSetAttribute(topk)")) return rc;
     cudaError_t e;
-    const unsigned grid = (unsigned)(plan.rows * plan.ctas_per_row);
+    const unsigned grid = plan.var_c ? (unsigned)device_info().num_sms : (unsigned)(plan.rows * plan.ctas_per_row);
     if (plan.ctas_per_row > 1) {
         // the CTAs of a row wait on one another: they must all be resident
         cudaLaunchConfig_t cfg = {};

@@ -96,7 +96,9 @@ struct Params {
     int64_t Lmax;
     BarrierCfg bar;        // time limit (and injected extra arrivals) of the row barriers
     float *kth = nullptr;  // optional [rows]: the k-th largest visible score (-inf when n <= K)
+    int var_c = 0;         // CTAs per row in proportion to the rows' lengths (see row_of_cta); C is then the largest
 };
+
 
 template <int NT>
 struct alignas(16) Shared {
@@ -111,6 +113,64 @@ struct alignas(16) Shared {
     uint32_t ok;
     uint32_t base;
 };
+
+// Length-proportional split of gridDim.x CTAs over the rows (rows <= grid):
+// row r gets 1 + floor(n_r * (grid - rows) / sum n) CTAs, n_r = its visible
+// keys.  Every CTA computes the same split and finds its (row, c, C_r); a CTA
+// past the last row gets row = -1.  All NT threads call it.
+template <int NT>
+__device__ void row_of_cta(const Params &p, Shared<NT> *sh, int *row, int *c, int *C) {
+    constexpr int NW = NT / 32;
+    const int rows = p.rows, G = gridDim.x;
+    // total visible keys
+    uint64_t tot = 0;
+    for (int r = threadIdx.x; r < rows; r += NT) {
+        int64_t n = (int64_t)__ldg(p.q_pos + r) + 1;
+        n = n > p.Lmax ? p.Lmax : (n < 0 ? 0 : n);
+        tot += (uint64_t)n;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    __shared__ uint64_t s_tot[NW];
+    __shared__ int s_row, s_c, s_C;
+    if (lane_id() == 0) s_tot[warp_id()] = tot;
+    if (threadIdx.x == 0) s_row = -1;
+    __syncthreads();
+    if (warp_id() == 0) {
+        uint64_t t = lane_id() < NW ? s_tot[lane_id()] : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        const uint64_t extra = (uint64_t)(G - rows);
+        // prefix of the per-row counts, 32 rows at a time
+        int base = 0;
+        for (int r0 = 0; r0 < rows; r0 += 32) {
+            const int r = r0 + lane_id();
+            int cr = 0;
+            if (r < rows) {
+                int64_t n = (int64_t)__ldg(p.q_pos + r) + 1;
+                n = n > p.Lmax ? p.Lmax : (n < 0 ? 0 : n);
+                cr = 1 + (t > 0 ? (int)((uint64_t)n * extra / t) : 0);
+            }
+            int incl = cr;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane_id() >= o) incl += u;
+            }
+            const int first = base + incl - cr;
+            if (r < rows && (int)blockIdx.x >= first && (int)blockIdx.x < first + cr) {
+                s_row = r;
+                s_c = (int)blockIdx.x - first;
+                s_C = cr;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncthreads();
+    *row = s_row;
+    *c = s_c;
+    *C = s_C;
+}
 
 // Inclusive block scan of one value per thread (all NT threads); returns the
 // inclusive prefix and writes the block total to *total.
