@@ -380,18 +380,29 @@ int dsa_shard_combine(const void *O_all, const float *lse_all, int n_ranks, int 
  * prefill chunk, or any block of queries over a shared cache): for each query
  * token t at position q_pos[t], exactly the decode layer-step -- indexer
  * scores over its visible keys 0..q_pos[t] (causal), the top_k selection, the
- * sparse GQA attention with the sink -- as dsa_layer_decode computes it.  The
- * queries run DSA_MAX_T at a time (one dsa_layer_decode per block, enqueued on
- * `stream`, reusing the workspace), so at most DSA_MAX_T x Lmax scores exist
- * at once, never the NQ x Lmax matrix.
+ * sparse GQA attention with the sink -- as dsa_layer_decode computes it, bit
+ * for bit ("What 'no full-attention layers' means": every DSA query keeps its
+ * own top 2,048 of the keys it may see).
  *   q8       e4m3 [NQ][16][128]      q_scale, w  f32 [NQ][16]
  *   Q        bf16 [NQ][64][192]      q_pos       int32 [NQ], each < Lmax
  *   kv       the sequence's caches (B = 1), as for dsa_layer_decode
  *   O        bf16 [NQ][64][128]      lse         f32 [NQ][64] or NULL
  *   idx_out  int32 [NQ][top_k] or NULL; count_out int32 [NQ] or NULL
- * Workspace: dsa_workspace_size(DSA_OP_PREFILL, 1, NQ, Lmax, top_k).
- * Errors as for dsa_layer_decode; a failing block stops the call (earlier
- * blocks stay enqueued).
+ * When NQ is a multiple of 16 (>= 64), the cache is contiguous or paged with
+ * pages of at most 256 positions, and Lmax >= 4,096, the indexer runs as one
+ * fp8 contraction of all NQ x 16 query heads against the keys on the tensor
+ * cores, keeping for each token only the keys above a threshold estimated
+ * from a sample of the keys (every 64th page), never the NQ x Lmax score
+ * matrix; each token's exact top_k is then taken from its candidates, and the
+ * attention runs over all tokens.  A token whose candidates turn out not to
+ * hold its selection (heavy ties, an unusual score distribution) is
+ * recomputed by the decode layer-step; this path reads that (usually empty)
+ * list back to the host, so the call synchronises `stream` once and cannot be
+ * captured in a CUDA graph.  Other shapes run DSA_MAX_T tokens at a time
+ * (one dsa_layer_decode per block, asynchronous).
+ * Workspace: dsa_workspace_size(DSA_OP_PREFILL, 1, NQ, Lmax, top_k) (about
+ * 1.4 GB for 8,192 tokens at 1,048,576 context: the sample's scores and the
+ * candidate lists).  Errors as for dsa_layer_decode.
  */
 int dsa_prefill(const void *q8, const float *q_scale, const float *w, const void *Q, const dsa_kv_t *kv,
                 const int32_t *q_pos, int NQ, int64_t Lmax, int top_k, const float *sink, float sm_scale,

@@ -832,7 +832,9 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
 }  // namespace capture
 
 // --------------------------------------------------------------- host side
-static size_t capture_smem_budget() { return device_info().smem_optin - 256; }
+// Largest dynamic shared memory of the capture kernel: the device's opt-in
+// maximum less room for the kernel's static shared memory (under 1 KB).
+static size_t capture_smem_budget() { return device_info().smem_optin - 1024; }
 
 int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
     using namespace capture;

@@ -135,7 +135,7 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
 // for its few bytes of static shared memory.
 static size_t fused_smem_budget() {
     // one CTA per SM; leave room for the kernel's few bytes of static shared memory
-    return device_info().smem_optin - 256;
+    return device_info().smem_optin - 1024;
 }
 
 int plan_fused(int B, int T, int64_t Lmax, int top_k, FusedPlan *plan) {

@@ -67,7 +67,8 @@ int plan_topk(int B, int T, int64_t Lmax, int top_k, TopkPlan *plan, size_t max_
         if (fixed > max_scratch_bytes) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "top-k scratch exceeds %zu bytes", max_scratch_bytes);
         cap = (int)std::min<size_t>(cap, (max_scratch_bytes - fixed) / ((size_t)plan->rows * 8));
         plan->list_cap = cap & ~3;
-        const size_t used = sizeof(Shared<kThreads>) + (size_t)plan->cache_keys * 4;
+        // room for the kernel's static shared memory (under 1 KB) stays free
+        const size_t used = sizeof(Shared<kThreads>) + (size_t)plan->cache_keys * 4 + 1024;
         size_t room = dev.smem_optin > used ? (dev.smem_optin - used) / 8 : 0;   // (key, position) pairs
         plan->smem_list = (int)std::min<size_t>({(size_t)plan->list_cap, (size_t)kSmemList, room});
         room -= plan->smem_list;

@@ -138,6 +138,28 @@ def test_topk_many_rows_ragged():
             assert np.all(idx[b, t, ref_cnt:].cpu().numpy() == -1)
 
 
+def test_topk_rows_of_very_different_lengths():
+    """More than 16 rows: the grid's CTAs go to the rows in proportion to their
+    lengths (one row of 250K keys next to rows of a few thousand)."""
+    B, T = 10, 4
+    L = 250000
+    g = torch.Generator(device=DEV).manual_seed(9)
+    scores = torch.randn((B, T, L), generator=g, device=DEV)
+    lens = np.exp(np.random.default_rng(9).uniform(np.log(3000), np.log(L), B * T)).astype(np.int64)
+    lens[0] = L
+    lens[1] = 2049
+    q_pos = torch.from_numpy(lens - 1).to(torch.int32).view(B, T).to(DEV)
+    for _ in range(2):   # run_topk also checks that the call leaves its workspace zeroed
+        idx, cnt = run_topk(scores, q_pos, 2048)
+    sc = scores.cpu().numpy()
+    for b in range(B):
+        for t in range(T):
+            n = int(q_pos[b, t]) + 1
+            ref_idx, ref_cnt = oracle.topk(sc[b, t, :n], 2048)
+            assert int(cnt[b, t]) == ref_cnt
+            assert np.array_equal(idx[b, t, :ref_cnt].cpu().numpy(), np.sort(ref_idx[:ref_cnt]))
+
+
 # ---------------------------------------------------------------- attention
 def _sparse_case(seed, seq_len, T, count_list, G=4, qk_std=None, page_size=0, sink=True):
     wl = make_decode_workload(seed=seed, seq_lens=[seq_len], T=T, G=G, device=DEV, qk_std=qk_std,
