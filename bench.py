@@ -614,6 +614,7 @@ def run_ours(args, rank, world, local_rank):
 
     K = args.steps
     fused = B * T <= FUSED_MAX_ROWS
+    paths0 = dsa.dsa_layer_path_counts(ws)
     # one fused kernel: only the events around it (no event records between its end and the last event)
     stage = [new_events(5) for _ in range(K)]
     if fused:
@@ -637,6 +638,7 @@ def run_ours(args, rank, world, local_rank):
         attn_ms = [stage[i][2].elapsed_time(stage[i][3]) for i in range(K)]
         comb_ms = [stage[i][3].elapsed_time(stage[i][4]) for i in range(K)]
     total_s = max_over_ranks(sum(step_ms) / 1e3, dev)
+    paths1 = dsa.dsa_layer_path_counts(ws)
     st, _ = dsa.dsa_check_device_status(ws)
     if st != dsa.DSA_OK:
         raise RuntimeError(f"device status {st} after the timed steps")
@@ -676,7 +678,8 @@ def run_ours(args, rank, world, local_rank):
     layer_bytes = ib + gathered_bytes(T, TOP_K)
     ind_avg_s = sum(ind_ms) / K2 / 1e3
     if fused:   # one kernel does the whole step: its roofline is the whole step's bytes
-        kern, kern_bytes, kern_avg_s = "dsa_layer_fused_kernel", layer_bytes, total_s / K
+        kern = "dsa_layer_capture_kernel" if paths1[0] + paths1[1] > paths0[0] + paths0[1] else "dsa_layer_fused_kernel"
+        kern_bytes, kern_avg_s = layer_bytes, total_s / K
     else:
         kern, kern_bytes, kern_avg_s = "indexer_kernel", ib, sum(idx_ms) / K / 1e3
     achieved = kern_bytes / kern_avg_s / 1e9
@@ -695,7 +698,10 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": decode_config(args.workload, world),
         "us_per_layer_step": total_s * 1e6 / K,
-        "path": "one fused cooperative kernel" if fused else "four kernels",
+        "path": ("one cooperative kernel" if fused else "four kernels"),
+        "timed_steps_by_path": {"one_barrier_fast": paths1[0] - paths0[0],
+                                "one_barrier_general": paths1[1] - paths0[1],
+                                "other": K - (paths1[0] - paths0[0]) - (paths1[1] - paths0[1])},
         "stage_us_median": ({"fused_layer_step": statistics.median(step_ms) * 1e3} if fused else {
             "indexer": statistics.median(idx_ms) * 1e3, "topk": statistics.median(topk_ms) * 1e3,
             "attention": statistics.median(attn_ms) * 1e3, "combine": statistics.median(comb_ms) * 1e3,

@@ -152,6 +152,17 @@ int dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
 #define DSA_STATUS_NEEDS_INIT 0x80000000u
 int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags);
 
+/* Synchronises `stream`, then reads two counters that the workspace header
+ * keeps since its last dsa_workspace_init: how many dsa_layer_decode calls
+ * (and dsa_layer_chain DSA steps) ran the one-barrier kernel for up to four
+ * long query rows on its fast path (*fast: the key stream's sampled threshold
+ * left between top_k and 16,384 candidates in every row, none lost) and on its
+ * general path (*general: a full selection over the stored scores).  Both
+ * give the same outputs; the counters say what the call cost.  Other paths
+ * count in neither.  Counters wrap at 2^32.  No page counterpart: an
+ * interface of this library. */
+int dsa_layer_path_counts(void *ws, void *stream, uint32_t *fast, uint32_t *general);
+
 /* Failure injection, for tests of the device-side failure path (no page
  * counterpart; an interface of this library).  While DSA_INJECT_BARRIER_TIMEOUT
  * is set (process-wide, for launches made from any host thread), every launch
@@ -166,6 +177,23 @@ int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags
 #define DSA_INJECT_NONE            0
 #define DSA_INJECT_BARRIER_TIMEOUT 1
 int dsa_debug_inject(int kind, int64_t wait_limit_ns);
+
+/* Phase trace of the one-barrier layer-step kernel (dsa_layer_decode and the
+ * DSA steps of dsa_layer_chain for up to four long query rows), for
+ * profiling; no page counterpart.  While a buffer is set (process-wide; NULL
+ * or words == 0 switches it off), every launch of that kernel made with a
+ * grid of at most words / DSA_TRACE_MARKS CTAs writes, per CTA c, the GPU's
+ * nanosecond clock (%globaltimer) into buf[c * DSA_TRACE_MARKS + i]:
+ *   i = 0 entry, 1 the sampled thresholds seen, 2 the key stream done (the
+ *   CTA's tiles scored and captured), 3 past the grid barrier, 4 the
+ *   selection done, 5 the attention units done, 6 exit.
+ * Marks a CTA does not reach (a CTA with no selection or attention work, the
+ * general path) are written as 0.  `buf` is device memory of the caller's,
+ * `words` its length in uint64 words; a launch with a grid too large for it
+ * writes nothing.  The buffer must outlive the launches made while it is
+ * set.  Returns DSA_ERR_INVALID_ARG for words < 0 or a NULL buf with words > 0. */
+#define DSA_TRACE_MARKS 8
+int dsa_trace_phases(uint64_t *buf, int64_t words);
 
 /*
  * dsa_indexer_scores -- lightning-indexer scores of every visible key

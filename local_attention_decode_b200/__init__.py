@@ -38,12 +38,14 @@ DSA_ERR_DEVICE_BAD_INDEX = 6
 OP_INDEXER, OP_TOPK, OP_SPARSE_ATTN, OP_SWA_ATTN, OP_LAYER, OP_PREFILL, OP_PRODUCE, OP_KL = range(8)
 STATUS_NEEDS_INIT = 0x80000000
 INJECT_NONE, INJECT_BARRIER_TIMEOUT = 0, 1
+TRACE_MARKS = 8   # phase marks per CTA of the one-barrier layer-step (dsa_trace_phases)
 
 EXPORTED = ("dsa_last_error", "dsa_get_dims", "dsa_workspace_size", "dsa_workspace_init",
             "dsa_check_device_status", "dsa_indexer_scores", "dsa_topk_select",
             "sparse_gqa_attn_decode", "swa_attn_decode", "dsa_layer_decode", "dsa_topk_select_noalloc",
             "dsa_prefill", "dsa_debug_inject", "dsa_index_produce", "dsa_layer_chain", "dsa_indexer_kl",
-            "dsa_shard_positions", "dsa_shard_candidates", "dsa_shard_merge", "dsa_shard_combine")
+            "dsa_shard_positions", "dsa_shard_candidates", "dsa_shard_merge", "dsa_shard_combine",
+            "dsa_layer_path_counts", "dsa_trace_phases")
 
 
 class DSAError(RuntimeError):
@@ -76,6 +78,8 @@ _lib.dsa_get_dims.argtypes = [P, I32]
 _lib.dsa_workspace_size.argtypes = [I32, I32, I32, I64, I32, ctypes.POINTER(ctypes.c_size_t)]
 _lib.dsa_workspace_init.argtypes = [P, SZ, P]
 _lib.dsa_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_uint32)]
+_lib.dsa_layer_path_counts.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]
+_lib.dsa_trace_phases.argtypes = [P, I64]
 _lib.dsa_indexer_scores.argtypes = [P, P, P, ctypes.POINTER(dsa_kv_t), P, I32, I32, I64, P, I64, P, SZ, P]
 _lib.dsa_topk_select.argtypes = [P, I64, P, I32, I32, I64, I32, P, P, P, SZ, P]
 _lib.sparse_gqa_attn_decode.argtypes = [P, ctypes.POINTER(dsa_kv_t), P, P, I32, I32, I32, P, F32, P, P, P, SZ, P]
@@ -148,6 +152,26 @@ def dsa_debug_inject(kind: int, wait_limit_ns: int = 0):
     the first cross-CTA barrier of the next launches run out after
     wait_limit_ns; INJECT_NONE turns it off."""
     _check(_lib.dsa_debug_inject(int(kind), int(wait_limit_ns)))
+
+
+def dsa_layer_path_counts(ws: torch.Tensor, stream=None):
+    """(fast, general): layer-steps the one-barrier kernel ran on each of its
+    paths since the workspace was zeroed; synchronises the stream."""
+    f = ctypes.c_uint32(0)
+    g = ctypes.c_uint32(0)
+    _check(_lib.dsa_layer_path_counts(_ptr(ws, torch.uint8, "ws"), _stream(stream), ctypes.byref(f), ctypes.byref(g)))
+    return f.value, g.value
+
+
+def dsa_trace_phases(buf):
+    """Set (a uint64 tensor on the device, viewed as int64 too) or clear
+    (None) the phase-trace buffer of the one-barrier layer-step kernel."""
+    if buf is None:
+        _check(_lib.dsa_trace_phases(None, 0))
+    else:
+        if buf.dtype not in (torch.int64, torch.uint64) or not buf.is_contiguous():
+            raise ValueError("trace buffer must be a contiguous 64-bit tensor")
+        _check(_lib.dsa_trace_phases(ctypes.c_void_p(buf.data_ptr()), buf.numel()))
 
 
 def dsa_check_device_status(ws: torch.Tensor, stream=None):

@@ -74,6 +74,14 @@ bool pdl_launches() { return g_pdl; }
 void set_pdl_launches(bool on) { g_pdl = on; }
 
 // Failure injection (dsa_debug_inject): process-wide, read at each launch.
+static std::atomic<uint64_t *> g_trace_buf{nullptr};
+static std::atomic<int64_t> g_trace_words{0};
+
+uint64_t *phase_trace(int grid) {
+    uint64_t *b = g_trace_buf.load();
+    return b && g_trace_words.load() >= (int64_t)grid * DSA_TRACE_MARKS ? b : nullptr;
+}
+
 static std::atomic<int> g_inject_kind{DSA_INJECT_NONE};
 static std::atomic<int64_t> g_inject_limit_ns{0};
 
@@ -349,6 +357,26 @@ int dsa_check_device_status(void *ws, void *stream, int *status, uint32_t *flags
     *status = (word & (1u << DSA_ERR_DEVICE_TIMEOUT))     ? DSA_ERR_DEVICE_TIMEOUT
               : (word & (1u << DSA_ERR_DEVICE_BAD_INDEX)) ? DSA_ERR_DEVICE_BAD_INDEX
                                                           : DSA_OK;
+    return DSA_OK;
+}
+
+int dsa_layer_path_counts(void *ws, void *stream, uint32_t *fast, uint32_t *general) {
+    if (!ws || !fast || !general) return fail(DSA_ERR_INVALID_ARG, "ws / fast / general is NULL");
+    uint32_t w[2] = {0u, 0u};
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess)
+        e = cudaMemcpy(w, static_cast<uint32_t *>(ws) + kPathCountWord, sizeof(w), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the path counters");
+    *fast = w[0];
+    *general = w[1];
+    return DSA_OK;
+}
+
+int dsa_trace_phases(uint64_t *buf, int64_t words) {
+    if (words < 0 || (!buf && words > 0)) return fail(DSA_ERR_INVALID_ARG, "trace buffer / words");
+    g_trace_buf.store(nullptr);
+    g_trace_words.store(buf ? words : 0);
+    g_trace_buf.store(words > 0 ? buf : nullptr);
     return DSA_OK;
 }
 

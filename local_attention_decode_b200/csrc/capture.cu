@@ -61,6 +61,7 @@ constexpr int kMaxRows = 4;                   // B * T on this path
 constexpr int kGroups = kPipes * kMaxGroups;  // epilogue groups per CTA
 constexpr int kBins = 2048;                   // sample histogram: bits 30..20 of the non-negative keys
 constexpr int kHistWords = kBins + 1;         // + the count of negative scores
+constexpr int kHistStride = kHistWords + 3;   // words between rows' histograms: rows start 16-byte aligned
 constexpr int kSegCap = 1024;                 // candidates one epilogue group may hold per row
 constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
 constexpr int kGroupBar0 = 5;                 // named barriers 5..8: the epilogue groups
@@ -92,9 +93,11 @@ struct Params {
     __nv_bfloat16 *O;
     float *lse;
     uint32_t *ctl;
-    uint32_t *sample_hist;    // [rows][kHistWords]
+    uint32_t *sample_hist;    // [rows][kHistStride]
     uint32_t *counts;         // [rows][NG]
     uint2 *lists;             // [rows][NG][kSegCap] (order key, position)
+    uint32_t *path_count;     // [2] calls that took the fast path / the general path
+    uint64_t *trace;          // [grid][DSA_TRACE_MARKS] phase marks, or NULL
     BarrierCfg bar;
     int rows, K, C, NG;
     float oversample;
@@ -116,7 +119,7 @@ struct Layout {
         tile_off = (len_off + 4 * (B + 1) + 15) & ~15u;
         epi_off = (tile_off + 4 * (B + 1) + 15) & ~15u;
         hist_off = epi_off + kGroups * kEpiWarps * (16 * T + T) * 4;
-        xch_off = hist_off + rows * kHistWords * 4;
+        xch_off = hist_off + rows * kHistStride * 4;
         misc_off = xch_off + kGroups * 2 * kEpiWarps * kMaxRows * 4;
         total = misc_off + 32;   // [0] groups sampled, [1 + g] group g's role in the sample exchange
     }
@@ -194,7 +197,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.tmem_off);
     int32_t *seq_len = reinterpret_cast<int32_t *>(smem + lay.len_off);
     int32_t *tile_pre = reinterpret_cast<int32_t *>(smem + lay.tile_off);
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [rows][kHistWords]
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [rows][kHistStride]
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags
     uint32_t *ctl = cp.ctl;
     const int warp = warp_id(), lane = lane_id();
@@ -214,7 +217,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         }
         seq_len[b] = mx + 1;
     }
-    for (int j = threadIdx.x; j < rows * kHistWords; j += blockDim.x) hist[j] = 0;
+    for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
     if (threadIdx.x < 8) misc[threadIdx.x] = 0;
     __syncthreads();
     if (warp == 0) {
@@ -430,7 +433,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
 #pragma unroll
                         for (int t = 0; t < kMaxRows; ++t)
                             if (t < T)
-                                warp_hist_add(hist + (b * T + t) * kHistWords, sample_bin(float_order_key(sc[t])),
+                                warp_hist_add(hist + (b * T + t) * kHistStride, sample_bin(float_order_key(sc[t])),
                                               (vis >> t) & 1u);
                     }
                 } else {
@@ -449,7 +452,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 named_bar_sync(gbar, 128);
                 if (*flag) {
                     const int tid = quarter * 32 + lane;
-                    for (int u = tid; u < rows * kHistWords; u += 128)
+                    for (int u = tid; u < rows * kHistStride; u += 128)
                         if (hist[u]) atomicAdd(cp.sample_hist + u, hist[u]);
                     __threadfence();
                     named_bar_sync(gbar, 128);
@@ -461,7 +464,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             const int r = quarter;
                             const int64_t n = (int64_t)__ldg(p.q_pos + r) + 1;
                             uint32_t t_r = 0xFFFFFFFFu;   // n <= top_k: every key is selected, nothing to capture
-                            uint32_t *h = cp.sample_hist + r * kHistWords;
+                            uint32_t *h = cp.sample_hist + r * kHistStride;
                             if (n > cp.K) {
                                 // the sample's visible keys: the histogram's total
                                 uint32_t tot = 0;
@@ -487,7 +490,10 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 }
                 // every group waits for the thresholds (one poller per group)
                 bool r_ok = true;
-                if (quarter == 0 && lane == 0) r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
+                if (quarter == 0 && lane == 0) {
+                    r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
+                    if (cp.trace && gi == 0) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
+                }
                 ok = named_bar_and(gbar, 128, ok && r_ok);
                 if (ok) {
 #pragma unroll
@@ -732,14 +738,24 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     uint32_t *ctl = cp.ctl;
     const uint32_t status_at_entry = load_status(status);
     if (threadIdx.x == 0) n_combine = 0;
+    uint64_t *trace = cp.trace ? cp.trace + blockIdx.x * DSA_TRACE_MARKS : nullptr;
+    auto mark = [&](int i) {
+        if (trace && threadIdx.x == 0) trace[i] = globaltimer_ns();
+    };
+    if (trace && threadIdx.x == 0) {
+        for (int i = 1; i < DSA_TRACE_MARKS; ++i) trace[i] = 0;
+        trace[0] = globaltimer_ns();
+    }
 
     // ---- phase 1: key stream, sample, candidates
     run_indexer_capture(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G);
+    mark(2);
     if (status_at_entry & kNeedsInitBit) {
         if (threadIdx.x == 0) flag_timeout(status);
         return;
     }
     if (!grid_sync(ctl + kGridArrive, 1 * G, cp.bar, status, &sync_flag)) return;
+    mark(3);
 
     // the sample was good for every row? (the same answer in every CTA)
     bool fast = __ldcg(ctl + kOverflow) == 0u;
@@ -749,8 +765,12 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
         if (n > cp.K && (m < (uint32_t)cp.K || m > (uint32_t)kListCap)) fast = false;
     }
     if (blockIdx.x == 0 && threadIdx.x < kMaxRows + 1) {   // read by nobody after phase 1
-        if (threadIdx.x == 0) ctl[kReady] = 0;
-        else ctl[kThr + threadIdx.x - 1] = 0;
+        if (threadIdx.x == 0) {
+            ctl[kReady] = 0;
+            atomicAdd(cp.path_count + (fast ? 0 : 1), 1u);
+        } else {
+            ctl[kThr + threadIdx.x - 1] = 0;
+        }
     }
 
     const int rows = cp.rows, C = cp.C;
@@ -760,6 +780,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
             const int r = blockIdx.x / C, c = blockIdx.x % C;
             int32_t *sel = reinterpret_cast<int32_t *>(smem);
             select_from_candidates(cp, r, c, sel, smem + kSelBytes);
+            mark(4);
             // attention CTA units of this row, positions from shared memory
             const int G_kv = cp.at.G, splits = cp.at.splits, nt = cp.at.n_teams;
             if ((int)threadIdx.x < nt * 128) {
@@ -774,6 +795,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
                 }
             }
             __syncthreads();
+            mark(5);
             // the last unit of a (row, KV group) combines its heads
             for (int q = 0; q < n_combine; ++q) {
                 const int g = combine_g[q];
@@ -817,6 +839,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
 
     // ---- the last CTA out resets the words read by everyone after phase 1
     __syncthreads();
+    mark(6);
     if (threadIdx.x == 0) {
         __threadfence();
         if (atomicAdd(ctl + kGridExit, 1u) == G - 1) {
@@ -882,7 +905,7 @@ int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
         return at;
     };
     plan->ctl_off = take(kCtlWords * 4);
-    plan->hist_off = take((size_t)rows * kHistWords * 4);
+    plan->hist_off = take((size_t)rows * kHistStride * 4);
     plan->counts_off = take((size_t)rows * ng * 4);
     plan->lists_off = take((size_t)rows * ng * kSegCap * 8);
     plan->topk_off = take((size_t)rows * topk::scratch_words(plan->C, topk::kListCap, false) * 4);
@@ -924,6 +947,8 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     cp.sample_hist = reinterpret_cast<uint32_t *>(scratch + plan.hist_off);
     cp.counts = reinterpret_cast<uint32_t *>(scratch + plan.counts_off);
     cp.lists = reinterpret_cast<uint2 *>(scratch + plan.lists_off);
+    cp.path_count = ia.status + kPathCountWord;
+    cp.trace = phase_trace(plan.grid);
     cp.bar = barrier_cfg();
     cp.rows = plan.rows;
     cp.K = top_k;

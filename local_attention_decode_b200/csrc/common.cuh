@@ -16,6 +16,9 @@ namespace dsa {
 // The first 256 bytes of every workspace hold a 32-bit status word: bit
 // (1 << code) is set for each kind of device-side error seen.
 constexpr size_t kStatusBytes = 256;
+// Words 1 and 2 of the workspace header: layer-steps the one-barrier kernel
+// ran on its fast path and on its general path (see dsa_layer_path_counts).
+constexpr int kPathCountWord = 1;
 
 __device__ __forceinline__ void flag_error(uint32_t *status, int code) {
     if (status) atomicOr(status, 1u << code);
@@ -60,6 +63,9 @@ struct BarrierCfg {
 };
 // The settings for a launch made now (host side; see dsa_debug_inject).
 BarrierCfg barrier_cfg();
+// The phase-trace buffer set by dsa_trace_phases when it holds `grid` CTAs'
+// marks, else NULL (host).
+uint64_t *phase_trace(int grid);
 
 // Bounded wait of thread 0 of a CTA until *bar >= target (acquire); false and
 // the timeout status when the limit runs out.

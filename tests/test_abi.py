@@ -134,3 +134,17 @@ def test_debug_inject_arguments_checked_on_the_host(dsa):
     assert lib.dsa_debug_inject(5, 2_000_000) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_debug_inject(dsa.INJECT_BARRIER_TIMEOUT, 0) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_debug_inject(dsa.INJECT_NONE, 0) == dsa.DSA_OK
+
+
+def test_trace_and_path_count_arguments_checked_on_the_host(dsa):
+    lib = dsa._lib
+    assert lib.dsa_trace_phases(None, -1) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_trace_phases(None, 8) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_trace_phases(None, 0) == dsa.DSA_OK            # switched off
+    fake = ctypes.c_void_p(1 << 20)                                # never dereferenced: only stored
+    assert lib.dsa_trace_phases(fake, 148 * dsa.TRACE_MARKS) == dsa.DSA_OK
+    assert lib.dsa_trace_phases(None, 0) == dsa.DSA_OK
+    out = ctypes.c_uint32(0)
+    assert lib.dsa_layer_path_counts(None, None, ctypes.byref(out), ctypes.byref(out)) == dsa.DSA_ERR_INVALID_ARG
+    m = re.search(r"#define DSA_TRACE_MARKS (\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == dsa.TRACE_MARKS

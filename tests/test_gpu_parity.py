@@ -228,7 +228,12 @@ def run_layer(wl, top_k=2048, sink=True, events=None):
                          wl.sink if sink else None, SM, O, lse, idx, cnt, ws)
     st, _ = dsa.dsa_check_device_status(ws)
     assert st == dsa.DSA_OK
+    LAST_PATHS[:] = dsa.dsa_layer_path_counts(ws)
     return O, lse, idx, cnt
+
+
+# (fast, general) path counts of the one-barrier kernel in the last run_layer call
+LAST_PATHS = [0, 0]
 
 
 def _check_layer(wl, O, lse, idx, cnt, top_k=2048, full_oracle=True, sink=True):
@@ -251,6 +256,8 @@ def _check_layer(wl, O, lse, idx, cnt, top_k=2048, full_oracle=True, sink=True):
 def test_layer_decode_matches_oracle(name):
     wl = make_decode_workload(device=DEV, **CONFIGS[name])
     O, lse, idx, cnt = run_layer(wl)
+    # up to four long rows: the one-barrier kernel, and its sample was good
+    assert LAST_PATHS == [1, 0]
     _check_layer(wl, O, lse, idx, cnt)
     # planted needles rank in the oracle's top-2048 and are selected
     sel = set(idx[0, 0].cpu().numpy().tolist())
@@ -369,6 +376,10 @@ def test_layer_decode_selection_fallbacks(weights):
         assert np.array_equal(idx[0, t].cpu().numpy(), np.sort(ref_idx))
     if weights == "zero_query":
         assert np.array_equal(idx[0, 0].cpu().numpy(), np.arange(2048))
+    if weights != "mixed":
+        # every key at or above the sampled threshold (all negative, or all
+        # tied): too many candidates, so the one-barrier kernel's general path
+        assert LAST_PATHS == [0, 1]
     _check_layer(wl, O, lse, idx, cnt)
 
 
@@ -388,6 +399,7 @@ def test_layer_decode_1m_context_sampled():
                                 np.array([len(sample) - 1], np.int32))
     assert_scores_close(scores[0][:, rows].cpu().numpy(), ref)
     O, lse, idx, cnt = run_layer(wl)
+    assert LAST_PATHS == [1, 0]   # the one-barrier kernel's fast path at 1M
     gpu_scores = scores[0, 0].cpu().numpy()
     ref_idx, ref_cnt = oracle.topk(gpu_scores, 2048)
     assert int(cnt[0, 0]) == 2048
