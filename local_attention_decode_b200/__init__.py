@@ -38,7 +38,7 @@ DSA_ERR_DEVICE_BAD_INDEX = 6
 OP_INDEXER, OP_TOPK, OP_SPARSE_ATTN, OP_SWA_ATTN, OP_LAYER, OP_PREFILL, OP_PRODUCE, OP_KL = range(8)
 STATUS_NEEDS_INIT = 0x80000000
 INJECT_NONE, INJECT_BARRIER_TIMEOUT = 0, 1
-TRACE_MARKS = 8   # phase marks per CTA of the one-barrier layer-step (dsa_trace_phases)
+TRACE_MARKS = 16   # phase marks per CTA of the one-barrier layer-step (dsa_trace_phases)
 
 EXPORTED = ("dsa_last_error", "dsa_get_dims", "dsa_workspace_size", "dsa_workspace_init",
             "dsa_check_device_status", "dsa_indexer_scores", "dsa_topk_select",

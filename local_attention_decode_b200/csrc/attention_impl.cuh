@@ -87,6 +87,10 @@ __device__ __forceinline__ void team_sync(int bar) {
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
+// 8-byte copy (both addresses 8-byte aligned), cached in L1 on the way
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -397,6 +401,20 @@ __device__ __forceinline__ void cta_unit(const Params &p, const TeamSmem &teams,
     cta_merge(p, teams, split, g, bt, t, sink, O, lse);
     if (p.splits > 1) __threadfence();   // the partial is visible before any later signal of this CTA
     cta_sync();
+}
+
+// One unit taken by a single team (p.n_teams == 1): chunk `split` of query bt
+// and KV head g, then the unit's partial (with one split: the output) written
+// by the same 128 threads, which synchronise on the named barrier `bar` only.
+// The teams of a CTA can so work on different units at once.
+__device__ __forceinline__ void team_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid, int bar,
+                                          const float *sink, __nv_bfloat16 *O, float *lse,
+                                          const int32_t *sel_smem = nullptr) {
+    attn_unit(p, sm, split, g, bt, tid, bar, sel_smem);
+    team_sync(bar);
+    cta_merge(p, TeamSmem{reinterpret_cast<uint8_t *>(&sm), 0u}, split, g, bt, tid, sink, O, lse);
+    if (p.splits > 1) __threadfence();   // the partial is visible before any later signal of this team
+    team_sync(bar);
 }
 
 // Merge of the splits of one (query, head) row gw by a whole CTA of NT

@@ -68,6 +68,8 @@ constexpr int kGroupBar0 = 5;                 // named barriers 5..8: the epilog
 constexpr int kUnitBar = 9;                   // named barrier of the attention teams of a CTA unit
 constexpr int kSelBytes = DSA_MAX_TOPK * 4;   // the selection, at the start of shared memory in phase 2
 constexpr int64_t kMinContext = 8192;         // shorter contexts take the fused layer-step
+// attention units per (row, KV head) for top_k <= DSA_MAX_TOPK
+constexpr int kMaxSplits = (DSA_MAX_TOPK + kAttnChunk - 1) / kAttnChunk;
 
 // control words at the start of the capture scratch
 enum {
@@ -120,7 +122,7 @@ struct Layout {
         epi_off = (tile_off + 4 * (B + 1) + 15) & ~15u;
         hist_off = epi_off + kGroups * kEpiWarps * (16 * T + T) * 4;
         xch_off = hist_off + rows * kHistStride * 4;
-        misc_off = xch_off + kGroups * 2 * kEpiWarps * kMaxRows * 4;
+        misc_off = xch_off + kGroups * 2 * (kEpiWarps * kMaxRows + 1) * 4;
         total = misc_off + 32;   // [0] groups sampled, [1 + g] group g's role in the sample exchange
     }
 };
@@ -309,6 +311,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                     for (int b = 0; b < B; ++b)
                         tma_load_2d(smem + lay.q_off + b * N * kKeyBytes, &tmap_q, &bars->q_full, 0, b * N);
                 }
+                if (i == 0 && pp == 0 && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 10] = globaltimer_ns();
                 mbar_arrive_expect_tx(&bars->full[pp][s], stage_tx);
                 int b, ti;
                 locate(tile_of(pp, i), b, ti);
@@ -357,6 +360,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             k > 0 ? 1u : 0u);
                 umma_commit(&bars->empty[pp][s]);
                 umma_commit(&bars->tfull[pp][a]);
+                if (i == 0 && pp == 0 && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 11] = globaltimer_ns();
             }
             umma_commit(&bars->mma_done[pp]);
             mbar_wait(&bars->mma_done[pp], 0, p.status);
@@ -375,15 +379,115 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         const uint32_t lt = (1u << lane) - 1u;
         float *coef = reinterpret_cast<float *>(smem + lay.epi_off) + ew * (17 * T);
         int32_t *qp = reinterpret_cast<int32_t *>(coef + 16 * T);
-        uint32_t *xch = reinterpret_cast<uint32_t *>(smem + lay.xch_off) + gi * (2 * kEpiWarps * kMaxRows);
+        // per group, twice (double-buffered): the four warps' candidate counts per query, the readiness poll
+        uint32_t *xch = reinterpret_cast<uint32_t *>(smem + lay.xch_off) + gi * (2 * (kEpiWarps * kMaxRows + 1));
         const uint32_t acc_col = (uint32_t)((pp * GE + a) * N);
         uint32_t base[kMaxRows] = {0u, 0u, 0u, 0u};
         uint32_t thr[kMaxRows] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-        bool ok = true, overflow = false;
+        bool ok = true, overflow = false, known = false;
         int cur_b = -1;
+        int pending = 0;   // the group's tiles 0 .. pending - 1 were scored before the thresholds were known
+        int slot = 0;      // half of the double-buffered exchange words that the next group barrier uses
+        const bool poller = quarter == 0 && lane == 0;
+
+        // The candidates of one tile to the group's segments, in position
+        // order: bit t of cbits says whether this thread's key is a candidate
+        // for query t of sequence b.  One group barrier exchanges the four
+        // warps' counts, and carries `okin` (AND over the group, returned) and
+        // the poller's `poll` (the thresholds' readiness, into *seen).
+        auto capture_tile = [&](int b, int64_t pos, const float (&sc)[kMaxRows], uint32_t cbits, bool okin,
+                                uint32_t poll, bool *seen) -> bool {
+            uint32_t *c = xch + slot * (kEpiWarps * kMaxRows + 1);
+            uint32_t cm[kMaxRows] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int t = 0; t < kMaxRows; ++t) {
+                if (t < T) {
+                    cm[t] = __ballot_sync(0xffffffffu, (cbits >> t) & 1u);
+                    if (lane == 0) c[quarter * kMaxRows + t] = __popc(cm[t]);
+                }
+            }
+            if (poller) c[kEpiWarps * kMaxRows] = poll;
+            const bool g_ok = named_bar_and(gbar, 128, okin);
+            *seen = c[kEpiWarps * kMaxRows] != 0u;
+            if (g_ok) {
+#pragma unroll
+                for (int t = 0; t < kMaxRows; ++t) {
+                    if (t < T) {
+                        uint32_t below = 0, tot = 0;
+#pragma unroll
+                        for (int q = 0; q < kEpiWarps; ++q) {
+                            const uint32_t v = c[q * kMaxRows + t];
+                            tot += v;
+                            if (q < quarter) below += v;
+                        }
+                        const int r = b * T + t;
+                        uint32_t bs = 0;
+#pragma unroll
+                        for (int rr = 0; rr < kMaxRows; ++rr)
+                            if (rr == r) bs = base[rr];
+                        if ((cm[t] >> lane) & 1u) {
+                            const uint32_t at = bs + below + __popc(cm[t] & lt);
+                            if (at < (uint32_t)kSegCap)
+                                cp.lists[((int64_t)r * cp.NG + gid) * kSegCap + at] =
+                                    make_uint2(float_order_key(sc[t]), (uint32_t)pos);
+                            else
+                                overflow = true;
+                        }
+#pragma unroll
+                        for (int rr = 0; rr < kMaxRows; ++rr)
+                            if (rr == r) base[rr] += tot;
+                    }
+                }
+            }
+            slot ^= 1;
+            return g_ok;
+        };
+        // Candidate bits of this thread's key for the queries of sequence b.
+        auto cand_bits = [&](int b, uint32_t vis, const float (&sc)[kMaxRows]) {
+            uint32_t bits = 0;
+#pragma unroll
+            for (int t = 0; t < kMaxRows; ++t) {
+                if (t < T) {
+                    uint32_t th = 0xFFFFFFFFu;
+#pragma unroll
+                    for (int r = 0; r < kMaxRows; ++r)
+                        if (r == b * T + t) th = thr[r];
+                    if (((vis >> t) & 1u) && float_order_key(sc[t]) >= th) bits |= 1u << t;
+                }
+            }
+            return bits;
+        };
+        // The thresholds are known: load them, then capture the pending
+        // tiles from their stored scores (this thread's own stores).
+        auto become_known = [&]() {
+            known = true;
+            if (poller && cp.trace && gi == 0) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
+#pragma unroll
+            for (int r = 0; r < kMaxRows; ++r)
+                if (r < rows) thr[r] = __ldcg(ctl + kThr + r);
+            for (int jj = 0; jj < pending && ok; ++jj) {
+                int bb, ti;
+                locate(tile_of(pp, jj * GE + a), bb, ti);
+                const int64_t ps = (int64_t)ti * kTile + row_in_tile;
+                const int len = seq_len[bb];
+                float s2[kMaxRows] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t v2 = 0;
+#pragma unroll
+                for (int t = 0; t < kMaxRows; ++t) {
+                    if (t < T && ps < len && ps <= (int64_t)__ldg(p.q_pos + bb * T + t)) {
+                        s2[t] = __ldcg(p.scores + ((int64_t)bb * T + t) * p.scores_stride + ps);
+                        v2 |= 1u << t;
+                    }
+                }
+                bool unused;
+                ok = capture_tile(bb, ps, s2, cand_bits(bb, v2, s2), ok, 0u, &unused);
+            }
+            pending = 0;
+        };
+
         for (int j = 0; j < ng || j == 0; ++j) {
             const bool have = j < ng;
-            float sc[kMaxRows];
+            float sc[kMaxRows] = {0.f, 0.f, 0.f, 0.f};
             uint32_t vis = 0;
             int b = 0;
             int64_t pos = 0;
@@ -402,6 +506,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 bool w_ok = mbar_wait(&bars->tfull[pp][a], (j & 1), p.status) &&
                             mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status);
                 if (__all_sync(0xffffffffu, w_ok)) {
+                    if (j == 0 && gi == 0 && poller && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 12] = globaltimer_ns();
                     tc_fence_after();
                     const float ks = *reinterpret_cast<const float *>(smem + lay.ks_off + st * kKsStageBytes +
                                                                       ks_slot_offset(row_in_tile, p.rows_per_load));
@@ -456,7 +561,10 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         if (hist[u]) atomicAdd(cp.sample_hist + u, hist[u]);
                     __threadfence();
                     named_bar_sync(gbar, 128);
-                    if (quarter == 0 && lane == 0) *flag = atomicAdd(ctl + kSampleArrive, 1u) == (uint32_t)ncta - 1 ? 2u : 1u;
+                    if (quarter == 0 && lane == 0) {
+                        *flag = atomicAdd(ctl + kSampleArrive, 1u) == (uint32_t)ncta - 1 ? 2u : 1u;
+                        if (cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 7] = globaltimer_ns();
+                    }
                     named_bar_sync(gbar, 128);
                     if (*flag == 2u) {   // the last CTA: one warp per row
                         __threadfence();
@@ -488,68 +596,26 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         }
                     }
                 }
-                // every group waits for the thresholds (one poller per group)
-                bool r_ok = true;
-                if (quarter == 0 && lane == 0) {
-                    r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
-                    if (cp.trace && gi == 0) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
-                }
-                ok = named_bar_and(gbar, 128, ok && r_ok);
-                if (ok) {
-#pragma unroll
-                    for (int r = 0; r < kMaxRows; ++r)
-                        if (r < rows) thr[r] = __ldcg(ctl + kThr + r);
-                }
             }
-            // ---- candidates of this tile, in position order within the group
-            uint32_t cm[kMaxRows] = {0u, 0u, 0u, 0u};
-            if (have && ok) {
-#pragma unroll
-                for (int t = 0; t < kMaxRows; ++t) {
-                    if (t < T) {
-                        uint32_t th = 0xFFFFFFFFu;
-#pragma unroll
-                        for (int r = 0; r < kMaxRows; ++r)
-                            if (r == b * T + t) th = thr[r];
-                        const bool cand = ((vis >> t) & 1u) && float_order_key(sc[t]) >= th;
-                        cm[t] = __ballot_sync(0xffffffffu, cand);
-                        if (lane == 0) xch[(j & 1) * kEpiWarps * kMaxRows + quarter * kMaxRows + t] = __popc(cm[t]);
-                    }
-                }
-            }
-            ok = named_bar_and(gbar, 128, ok);
+            // ---- this tile's candidates (deferred while the thresholds are unknown)
+            uint32_t poll = 0;
+            if (!known && poller) poll = ld_acquire_gpu(ctl + kReady) >= 1u ? 1u : 0u;
+            const bool was_known = known;
+            bool seen = false;
+            ok = capture_tile(b, pos, sc, (was_known && have && ok) ? cand_bits(b, vis, sc) : 0u, ok, poll, &seen);
             if (!ok) break;
-            if (have) {
-#pragma unroll
-                for (int t = 0; t < kMaxRows; ++t) {
-                    if (t < T) {
-                        const uint32_t *c4 = xch + (j & 1) * kEpiWarps * kMaxRows + t;
-                        uint32_t below = 0, tot = 0;
-#pragma unroll
-                        for (int q = 0; q < kEpiWarps; ++q) {
-                            const uint32_t v = c4[q * kMaxRows];
-                            tot += v;
-                            if (q < quarter) below += v;
-                        }
-                        const int r = b * T + t;
-                        uint32_t bs = 0;
-#pragma unroll
-                        for (int rr = 0; rr < kMaxRows; ++rr)
-                            if (rr == r) bs = base[rr];
-                        if ((cm[t] >> lane) & 1u) {
-                            const uint32_t at = bs + below + __popc(cm[t] & lt);
-                            if (at < (uint32_t)kSegCap)
-                                cp.lists[((int64_t)r * cp.NG + gid) * kSegCap + at] =
-                                    make_uint2(float_order_key(sc[t]), (uint32_t)pos);
-                            else
-                                overflow = true;
-                        }
-#pragma unroll
-                        for (int rr = 0; rr < kMaxRows; ++rr)
-                            if (rr == r) base[rr] += tot;
-                    }
-                }
+            if (!was_known) {
+                if (have) pending = j + 1;
+                if (seen) become_known();
+                if (!ok) break;
             }
+        }
+        // a short stream: the thresholds may come after the group's last tile
+        if (ok && !known) {
+            bool r_ok = true;
+            if (poller) r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
+            ok = named_bar_and(gbar, 128, r_ok);
+            if (ok) become_known();
         }
         if (__any_sync(0xffffffffu, overflow) && lane == 0) atomicOr(ctl + kOverflow, 1u);
         if (quarter == 0 && lane == 0) {
@@ -588,49 +654,81 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     __syncthreads();
 }
 
-// The combine of one (row, KV group): the group's heads over all splits, with
-// the sink, by 32 threads per head (4 columns each) -- the same operations in
-// the same order as combine_row_cta, so the outputs are identical.
-__device__ void combine_group(const Params &cp, int bt, int g) {
+// One slice of the combine of (row bt, KV group g), by the 128 threads of a
+// team (tid 0..127) once all `splits` units of that group have written their
+// partials: slice `piece` of the group's (head, column) outputs, head-major,
+// cut into `splits` near-equal slices.  The operations and their order are
+// those of combine_row_cta, so the outputs are identical:
+//   M = max(sink, m_j),  w_j = 2^(m_j - M) (0 for an empty split),
+//   O = sum_j (v_j w_j) / (2^(sink - M) + sum_j l_j w_j)   in order j = 0, 1, ...
+// `st` is team shared memory for the statistics of the slice's heads.
+__device__ void combine_piece(const Params &cp, int bt, int g, int piece, int tid, int bar, float *st) {
     const attn::Params &at = cp.at;
     const int hpg = DSA_Q_HEADS / at.G, splits = at.splits;
-    const int t = threadIdx.x, hh = t >> 5, c4 = t & 31;
-    if (hh >= hpg) return;
-    const int h = g * hpg + hh;
-    const int64_t gw = (int64_t)bt * DSA_Q_HEADS + h;
-    const float *ml = at.part_ml + gw * splits * 2;
-    const float sk = cp.sink ? __ldg(cp.sink + h) * attn::kLog2e : -INFINITY;
-    float M = sk;
-    for (int j = 0; j < splits; ++j) M = fmaxf(M, __ldcg(ml + 2 * j));
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    float L = (cp.sink && M != -INFINITY) ? exp2f(sk - M) : 0.f;
-    for (int j = 0; j < splits; ++j) {
-        const float m = __ldcg(ml + 2 * j), l = __ldcg(ml + 2 * j + 1);
-        const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (w != 0.f) v = __ldcg(reinterpret_cast<const float4 *>(at.part_o + (gw * splits + j) * DSA_V_DIM) + c4);
-        acc[0] = __fadd_rn(acc[0], __fmul_rn(v.x, w));
-        acc[1] = __fadd_rn(acc[1], __fmul_rn(v.y, w));
-        acc[2] = __fadd_rn(acc[2], __fmul_rn(v.z, w));
-        acc[3] = __fadd_rn(acc[3], __fmul_rn(v.w, w));
-        L = __fadd_rn(L, w != 0.f ? __fmul_rn(l, w) : 0.f);
+    const int E = hpg * DSA_V_DIM;
+    const int lo = (int)((int64_t)piece * E / splits), hi = (int)((int64_t)(piece + 1) * E / splits);
+    const int h_lo = lo / DSA_V_DIM, nh = (hi - 1) / DSA_V_DIM - h_lo + 1;
+    float *w = st;                            // [nh][splits] m_j, then the weights w_j
+    float *ls = st + hpg * kMaxSplits;        // [nh][splits] l_j
+    float *hs = ls + hpg * kMaxSplits;        // [nh][2]: M, L per head
+    // the heads' split statistics -> weights, M and the denominators
+    for (int i = tid; i < nh * splits; i += 128) {
+        const int hh = i / splits, j = i % splits;
+        const int64_t gw = (int64_t)bt * DSA_Q_HEADS + g * hpg + h_lo + hh;
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(at.part_ml) + gw * splits + j);
+        w[i] = ml.x;
+        ls[i] = ml.y;
     }
-    __nv_bfloat16 *o = cp.O + gw * DSA_V_DIM + c4 * 4;
+    attn::team_sync(bar);
+    if (tid < nh) {
+        const int h = g * hpg + h_lo + tid;
+        const float sk = cp.sink ? __ldg(cp.sink + h) * attn::kLog2e : -INFINITY;
+        float M = sk;
+        for (int j = 0; j < splits; ++j) M = fmaxf(M, w[tid * splits + j]);
+        float L = (cp.sink && M != -INFINITY) ? exp2f(sk - M) : 0.f;
+        for (int j = 0; j < splits; ++j) {
+            const float m = w[tid * splits + j];
+            const float wj = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
+            L = __fadd_rn(L, wj != 0.f ? __fmul_rn(ls[tid * splits + j], wj) : 0.f);
+            w[tid * splits + j] = wj;
+        }
+        hs[2 * tid] = M;
+        hs[2 * tid + 1] = L;
+    }
+    attn::team_sync(bar);
+    for (int e = lo + tid; e < hi; e += 128) {
+        const int hh = e / DSA_V_DIM - h_lo, col = e % DSA_V_DIM;
+        const int64_t gw = (int64_t)bt * DSA_Q_HEADS + g * hpg + h_lo + hh;
+        const float *po = at.part_o + gw * splits * DSA_V_DIM + col;
+        float v[kMaxSplits];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) o[u] = __float2bfloat16_rn(L > 0.f ? acc[u] / L : 0.f);
-    if (cp.lse && c4 == 0) cp.lse[gw] = (L > 0.f) ? (M + log2f(L)) / attn::kLog2e : -INFINITY;
+        for (int j = 0; j < kMaxSplits; ++j) v[j] = j < splits ? __ldcg(po + (int64_t)j * DSA_V_DIM) : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxSplits; ++j) {
+            if (j < splits) {
+                const float wj = w[hh * splits + j];
+                acc = __fadd_rn(acc, __fmul_rn(wj != 0.f ? v[j] : 0.f, wj));
+            }
+        }
+        const float M = hs[2 * hh], L = hs[2 * hh + 1];
+        cp.O[gw * DSA_V_DIM + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+        if (cp.lse && col == 0) cp.lse[gw] = (L > 0.f) ? (M + log2f(L)) / attn::kLog2e : -INFINITY;
+    }
+    attn::team_sync(bar);   // `st` may be reused
 }
 
 // Phase 2 (fast): the exact selection of row r from its candidates, into
 // `sel` (shared, top_k entries, -1 padded) and, by CTA c == 0, into the
-// output.  `work` is shared memory for the list.
-__device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *sel, uint8_t *work) {
-    constexpr int NT = kThreads;
+// output.  `work` is shared memory for the list.  Called by all threads.
+__device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *sel, uint8_t *work, uint64_t *trace) {
+    constexpr int NT = kThreads, NW = NT / 32;
     const int K = cp.K, NG = cp.NG;
+    const int lane = lane_id(), warp = warp_id();
+    const uint32_t lt = (1u << lane) - 1u;
     auto *sh = reinterpret_cast<topk::Shared<NT> *>(work);
     uint32_t *off = reinterpret_cast<uint32_t *>(work + align128(sizeof(topk::Shared<NT>)));
-    uint32_t *lkey = off + ((NG + 1 + 31) & ~31);
-    uint32_t *lpos = lkey + kListCap;
+    uint2 *list = reinterpret_cast<uint2 *>(off + ((NG + 1 + 31) & ~31));   // (order key, position)
     int64_t n = (int64_t)__ldg(cp.ix.q_pos + r) + 1;
     if (n > cp.ix.Lmax) n = cp.ix.Lmax;
     if (n < 0) n = 0;
@@ -645,33 +743,17 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         if (threadIdx.x < NG) off[threadIdx.x] = incl - v;
         if (threadIdx.x == 0) off[NG] = m;
         __syncthreads();
-        // the candidates, in position order
+        // the candidates, in position order: each warp copies whole segments,
+        // every copy in flight at once
         const uint2 *segs = cp.lists + (int64_t)r * NG * kSegCap;
-        for (uint32_t j0 = 0; j0 < m; j0 += 4 * NT) {
-            uint2 e[4];
-            uint32_t jj[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t j = j0 + u * NT + threadIdx.x;
-                jj[u] = j;
-                e[u] = make_uint2(0u, 0u);
-                if (j < m) {
-                    int lo = 0, hi = NG - 1;   // last segment starting at or before j
-                    while (lo < hi) {
-                        const int mid = (lo + hi + 1) >> 1;
-                        if (off[mid] <= j) lo = mid; else hi = mid - 1;
-                    }
-                    e[u] = __ldcg(segs + (int64_t)lo * kSegCap + (j - off[lo]));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (jj[u] < m) {
-                    lkey[jj[u]] = e[u].x;
-                    lpos[jj[u]] = e[u].y;
-                }
+        for (int sg = warp; sg < NG; sg += NW) {
+            const uint32_t o = off[sg], cnt = off[sg + 1] - o;
+            for (uint32_t i = lane; i < cnt; i += 32) attn::cp_async8(list + o + i, segs + (int64_t)sg * kSegCap + i);
         }
+        attn::cp_async_commit();
+        attn::cp_async_wait_all();
         __syncthreads();
+        if (trace && threadIdx.x == 0) trace[8] = globaltimer_ns();
         // exact radix select of the k-th largest key: 11 + 11 + 10 bits
         uint32_t prefix = 0u, mask = 0u, Krem = (uint32_t)K;
 #pragma unroll 1
@@ -680,10 +762,10 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             const int nb = pass == 2 ? 1024 : 2048;
             for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
             __syncthreads();
-            for (uint32_t j = threadIdx.x; j < m; j += NT) {
-                const uint32_t k = lkey[j];
-                if ((k & mask) == prefix) atomicAdd(&sh->hist[(k >> shift) & (uint32_t)(nb - 1)], 1u);
-            }
+            list_digit_hist<NT>(sh->hist, m, prefix, mask, shift, (uint32_t)nb, [&](uint32_t j, uint32_t &k) {
+                k = list[j].x;
+                return true;
+            });
             __syncthreads();
             topk::find_threshold<NT>(sh, nb, Krem);
             prefix |= (uint32_t)sh->bin << shift;
@@ -692,27 +774,40 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             __syncthreads();
         }
         const uint32_t Tstar = prefix, ties = Krem;
-        // compaction in position order: each thread a contiguous run of the list
-        const uint32_t per_t = (m + NT - 1) / NT;
-        const uint32_t lo = min(m, threadIdx.x * per_t), hi = min(m, lo + per_t);
-        uint32_t g = 0, e = 0;
-        for (uint32_t j = lo; j < hi; ++j) {
-            g += lkey[j] > Tstar;
-            e += lkey[j] == Tstar;
+        if (trace && threadIdx.x == 0) trace[9] = globaltimer_ns();
+        // compaction in position order, in 32-entry strips: each warp a run
+        // of whole strips; the keys above T* and the first `ties` keys equal
+        // to it, each at (keys above before it) + min(equal keys before it, ties)
+        const uint32_t strips = (m + 31) / 32, per_w = (strips + NW - 1) / NW;
+        const uint32_t s0 = min(strips, (uint32_t)warp * per_w), s1 = min(strips, s0 + per_w);
+        uint32_t gt = 0, eq = 0;
+        for (uint32_t q = s0; q < s1; ++q) {
+            const uint32_t j = q * 32 + lane;
+            const uint32_t k = j < m ? list[j].x : 0u;
+            gt += __popc(__ballot_sync(0xffffffffu, j < m && k > Tstar));
+            eq += __popc(__ballot_sync(0xffffffffu, j < m && k == Tstar));
         }
-        uint32_t dummy;
-        const uint32_t packed = (g << 16) | e;
-        const uint32_t excl = topk::block_scan<NT>(packed, sh->warp_tmp, &dummy) - packed;
-        uint32_t gb = excl >> 16, eb = excl & 0xFFFFu;
-        for (uint32_t j = lo; j < hi; ++j) {
-            const uint32_t k = lkey[j];
-            if (k > Tstar) {
-                sel[gb + (eb < ties ? eb : ties)] = (int32_t)lpos[j];
-                ++gb;
-            } else if (k == Tstar) {
-                if (eb < ties) sel[gb + eb] = (int32_t)lpos[j];
-                ++eb;
-            }
+        if (lane == 0) {
+            sh->warp_a[warp] = gt;
+            sh->warp_b[warp] = eq;
+        }
+        __syncthreads();
+        uint32_t gb = 0, eb = 0;
+        for (int w2 = 0; w2 < warp; ++w2) {
+            gb += sh->warp_a[w2];
+            eb += sh->warp_b[w2];
+        }
+        for (uint32_t q = s0; q < s1; ++q) {
+            const uint32_t j = q * 32 + lane;
+            const bool in = j < m;
+            const uint2 e = in ? list[j] : make_uint2(0u, 0u);
+            const uint32_t bg = __ballot_sync(0xffffffffu, in && e.x > Tstar);
+            const uint32_t be = __ballot_sync(0xffffffffu, in && e.x == Tstar);
+            const uint32_t g_before = gb + __popc(bg & lt), e_before = eb + __popc(be & lt);
+            if (in && e.x > Tstar) sel[g_before + (e_before < ties ? e_before : ties)] = (int32_t)e.y;
+            else if (in && e.x == Tstar && e_before < ties) sel[g_before + e_before] = (int32_t)e.y;
+            gb += __popc(bg);
+            eb += __popc(be);
         }
         for (int j = kr + threadIdx.x; j < K; j += NT) sel[j] = -1;
     }
@@ -730,14 +825,11 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     __shared__ uint32_t sync_flag;
-    __shared__ int n_combine;
-    __shared__ int combine_g[DSA_Q_HEADS];
     pdl_begin();
     const uint32_t G = gridDim.x;
     uint32_t *status = cp.ix.status;
     uint32_t *ctl = cp.ctl;
     const uint32_t status_at_entry = load_status(status);
-    if (threadIdx.x == 0) n_combine = 0;
     uint64_t *trace = cp.trace ? cp.trace + blockIdx.x * DSA_TRACE_MARKS : nullptr;
     auto mark = [&](int i) {
         if (trace && threadIdx.x == 0) trace[i] = globaltimer_ns();
@@ -774,35 +866,46 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     }
 
     const int rows = cp.rows, C = cp.C;
+    const int G_kv = cp.at.G, splits = cp.at.splits, nt = cp.at.n_teams;
+    const attn::TeamSmem teams{smem + (fast ? kSelBytes : 0), (uint32_t)align128(sizeof(attn::Smem))};
     if (fast) {
-        // ---- phase 2 (fast): every CTA of a row selects from the row's candidates
-        if ((int)blockIdx.x < rows * C) {
+        // ---- phase 2 (fast): the CTAs of a row that have attention units
+        //      select from the row's candidates, attend, then combine.  Unit
+        //      u of row r (KV head u / splits, 64-key chunk u % splits) is
+        //      taken by team u / C of the row's CTA u % C.
+        const int upr = G_kv * splits;   // units of a row (single teams; CTA units when nt > 1, then splits == 1)
+        if ((int)blockIdx.x < rows * C && (int)(blockIdx.x % C) < upr) {
             const int r = blockIdx.x / C, c = blockIdx.x % C;
             int32_t *sel = reinterpret_cast<int32_t *>(smem);
-            select_from_candidates(cp, r, c, sel, smem + kSelBytes);
+            select_from_candidates(cp, r, c, sel, smem + kSelBytes, trace);
             mark(4);
-            // attention CTA units of this row, positions from shared memory
-            const int G_kv = cp.at.G, splits = cp.at.splits, nt = cp.at.n_teams;
-            if ((int)threadIdx.x < nt * 128) {
-                const attn::TeamSmem teams{smem + kSelBytes, (uint32_t)align128(sizeof(attn::Smem))};
-                for (int u = c; u < G_kv * splits; u += C) {
-                    const int g = u / splits, split = u % splits;
-                    attn::cta_unit(cp.at, teams, split, g, r, 1, kUnitBar, cp.sink, cp.O, cp.lse, sel);
-                    if (splits > 1 && threadIdx.x == 0) {   // the unit's partial is written and fenced
-                        const uint32_t done = atomicAdd(ctl + kCombine + r * DSA_Q_HEADS + g, 1u);
-                        if (done == (uint32_t)splits - 1) combine_g[atomicAdd(&n_combine, 1)] = g;
+            if (nt == 1) {
+                const int tm = threadIdx.x >> 7, tid = threadIdx.x & 127;
+                if (tm < kTeams) {
+                    for (int u = c + tm * C; u < upr; u += kTeams * C) {
+                        const int g = u / splits, split = u % splits;
+                        attn::team_unit(cp.at, teams[tm], split, g, r, tid, 1 + tm, cp.sink, cp.O, cp.lse, sel);
+                        if (splits > 1 && tid == 0) atomicAdd(ctl + kCombine + r * DSA_Q_HEADS + g, 1u);
+                    }
+                    if (tm == 0) mark(5);
+                    // each unit's team then combines one slice of its KV head's
+                    // outputs, once every unit of that head has written its partial
+                    if (splits > 1) {
+                        for (int u = c + tm * C; u < upr; u += kTeams * C) {
+                            const int g = u / splits, split = u % splits;
+                            bool ok = true;
+                            if (tid == 0)
+                                ok = spin_until_at_least(ctl + kCombine + r * DSA_Q_HEADS + g, (uint32_t)splits,
+                                                         cp.bar.limit_ns, status);
+                            if (!named_bar_and(1 + tm, 128, ok)) break;
+                            combine_piece(cp, r, g, split, tid, 1 + tm, reinterpret_cast<float *>(&teams[tm]));
+                        }
                     }
                 }
-            }
-            __syncthreads();
-            mark(5);
-            // the last unit of a (row, KV group) combines its heads
-            for (int q = 0; q < n_combine; ++q) {
-                const int g = combine_g[q];
-                if (threadIdx.x == 0) __threadfence();
-                __syncthreads();
-                combine_group(cp, r, g);
-                if (threadIdx.x == 0) ctl[kCombine + r * DSA_Q_HEADS + g] = 0;
+            } else if ((int)threadIdx.x < nt * 128) {
+                // key sets of at most 256: one CTA unit per KV head, no combine
+                attn::cta_unit(cp.at, teams, 0, c, r, 1, kUnitBar, cp.sink, cp.O, cp.lse, sel);
+                mark(5);
             }
         }
     } else {
@@ -814,16 +917,22 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
         }
         if (!grid_sync(ctl + kGridArrive, 2 * G, cp.bar, status, &sync_flag)) return;
         {
-            const int nt = cp.at.n_teams;
-            if ((int)threadIdx.x < nt * 128) {
-                const attn::TeamSmem teams{smem, (uint32_t)align128(sizeof(attn::Smem))};
-                const int G_kv = cp.at.G, splits = cp.at.splits;
-                const int units = rows * G_kv * splits;
-                for (int u = blockIdx.x; u < units; u += G) {
-                    const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
-                    attn::cta_unit(cp.at, teams, split, g, bt, 1, kUnitBar, cp.sink, cp.O, cp.lse);
+            const int units = rows * G_kv * splits;
+            if ((int)threadIdx.x < kTeams * 128) {
+                if (nt == 1) {
+                    const int tm = threadIdx.x >> 7;
+                    for (int u = blockIdx.x + tm * G; u < units; u += kTeams * G) {
+                        const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
+                        attn::team_unit(cp.at, teams[tm], split, g, bt, threadIdx.x & 127, 1 + tm, cp.sink, cp.O,
+                                        cp.lse);
+                    }
+                } else if ((int)threadIdx.x < nt * 128) {
+                    for (int u = blockIdx.x; u < units; u += G) {
+                        const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
+                        attn::cta_unit(cp.at, teams, split, g, bt, 1, kUnitBar, cp.sink, cp.O, cp.lse);
+                    }
                 }
-            } else if ((int)threadIdx.x >= kTeams * 128 && (int)blockIdx.x < rows * C && C > 1) {
+            } else if ((int)blockIdx.x < rows * C && C > 1) {
                 constexpr int kFree = kThreads - kTeams * 128;
                 topk::clear_row_share(cp.tk, blockIdx.x / C, blockIdx.x % C, C, false, threadIdx.x - kTeams * 128,
                                       kFree);
@@ -831,10 +940,10 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
         }
         if (!grid_sync(ctl + kGridArrive, 3 * G, cp.bar, status, &sync_flag)) return;
         if ((int)blockIdx.x < rows * C && blockIdx.x % C == 0) topk::reset_row_ctl(cp.tk, blockIdx.x / C, C);
-        if (cp.at.splits > 1)
-          for (int gw = blockIdx.x; gw < rows * DSA_Q_HEADS; gw += G)
-            attn::combine_row_cta<kThreads>(cp.at.part_o, cp.at.part_ml, gw, cp.at.splits, cp.sink, cp.O, cp.lse,
-                                            reinterpret_cast<float *>(smem));
+        if (splits > 1)
+            for (int gw = blockIdx.x; gw < rows * DSA_Q_HEADS; gw += G)
+                attn::combine_row_cta<kThreads>(cp.at.part_o, cp.at.part_ml, gw, splits, cp.sink, cp.O, cp.lse,
+                                                reinterpret_cast<float *>(smem));
     }
 
     // ---- the last CTA out resets the words read by everyone after phase 1
@@ -846,6 +955,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
             ctl[kGridArrive] = 0;
             ctl[kOverflow] = 0;
             for (int r = 0; r < kMaxRows; ++r) ctl[kTotal + r] = 0;
+            for (int i = 0; i < rows * DSA_Q_HEADS; ++i) ctl[kCombine + i] = 0;
             __threadfence();
             ctl[kGridExit] = 0;
         }
@@ -940,6 +1050,7 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     cp.ix.hist_rows = 0;
     cp.ix.q_resident = 1;
     cp.at = attn::make_params(aa);
+    if (cp.at.splits > kMaxSplits) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "attention splits above the combine's bound");
     cp.sink = aa.sink;
     cp.O = aa.O;
     cp.lse = aa.lse;

@@ -306,9 +306,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 
 // ------------------------------------------------------------------ misc
-// Warp-level histogram increment: lanes with `active` add 1 to hist[bin].
-// When every active lane has the same bin (the common case for a narrow score
-// distribution) one atomic adds them all; otherwise each lane adds its own.
+// Warp-level histogram increment: lanes with `active` add 1 to hist[bin],
+// with one shared-memory atomic per distinct bin of the warp.  Keys that
+// agree on a digit (a narrow score range, a radix pass below a common prefix)
+// would otherwise serialise on one address, one atomic per key.  When every
+// active lane has the same bin one atomic adds them all; otherwise the lanes
+// of each bin find one another with match.any and their first lane adds.
 // All 32 lanes must call it.
 __device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool active) {
     const uint32_t amask = __ballot_sync(0xffffffffu, active);
@@ -318,7 +321,24 @@ __device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool
     if (bmin == bmax) {
         if ((threadIdx.x & 31) == (uint32_t)(__ffs(amask) - 1)) atomicAdd(&hist[bmin], (uint32_t)__popc(amask));
     } else if (active) {
-        atomicAdd(&hist[bin], 1u);
+        const uint32_t peers = __match_any_sync(amask, bin);
+        if ((threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+}
+
+// Histogram of the digit (key >> shift) & (nb - 1) of the keys of entries
+// j < m whose bits under `mask` equal `prefix`, added into hist by all NT
+// threads of the block (warp_hist_add; every warp walks whole 32-entry runs).
+// key_at(j, &k) stores entry j's key and returns whether the entry takes part.
+template <int NT, class KeyAt>
+__device__ __forceinline__ void list_digit_hist(uint32_t *hist, uint32_t m, uint32_t prefix, uint32_t mask, int shift,
+                                                uint32_t nb, KeyAt key_at) {
+    const uint32_t lane = threadIdx.x & 31u;
+    for (uint32_t jb = threadIdx.x & ~31u; jb < m; jb += NT) {
+        const uint32_t j = jb + lane;
+        uint32_t k = 0u;
+        const bool use = j < m && key_at(j, k);
+        warp_hist_add(hist, (k >> shift) & (nb - 1), use && (k & mask) == prefix);
     }
 }
 

@@ -91,16 +91,26 @@ dsa_layer_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     }
     if (!grid_sync(fp.grid_bar, 2 * G, fp.bar, status, &sync_flag)) return;
 
-    // ---- phase 3: attention, one CTA unit (n_teams teams of 64 keys) at a time
+    // ---- phase 3: attention units (one team each, the CTA's teams on four
+    //      units at once; or CTA units of n_teams merged teams)
     {
         const int nt = fp.at.n_teams;
-        if ((int)threadIdx.x < nt * 128) {
-            const attn::TeamSmem teams{smem, (uint32_t)smem_align(sizeof(attn::Smem))};
-            const int G_kv = fp.at.G, splits = fp.at.splits;
-            const int units = fp.rows * G_kv * splits;
-            for (int u = blockIdx.x; u < units; u += G) {
-                const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
-                attn::cta_unit(fp.at, teams, split, g, bt, 1, kUnitBar, fp.sink, fp.O, fp.lse);
+        const attn::TeamSmem teams{smem, (uint32_t)smem_align(sizeof(attn::Smem))};
+        const int G_kv = fp.at.G, splits = fp.at.splits;
+        const int units = fp.rows * G_kv * splits;
+        if ((int)threadIdx.x < kTeams * 128) {
+            if (nt == 1) {
+                const int tm = threadIdx.x >> 7;
+                for (int u = blockIdx.x + tm * G; u < units; u += kTeams * G) {
+                    const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
+                    attn::team_unit(fp.at, teams[tm], split, g, bt, threadIdx.x & 127, 1 + tm, fp.sink, fp.O,
+                                    fp.lse);
+                }
+            } else if ((int)threadIdx.x < nt * 128) {
+                for (int u = blockIdx.x; u < units; u += G) {
+                    const int split = u % splits, g = (u / splits) % G_kv, bt = u / (splits * G_kv);
+                    attn::cta_unit(fp.at, teams, split, g, bt, 1, kUnitBar, fp.sink, fp.O, fp.lse);
+                }
             }
         } else if ((int)threadIdx.x >= kTeams * 128 && (int)blockIdx.x < fp.rows * fp.C && (fp.C > 1 || fp.hist_ready)) {
             // the warps outside the teams clear the selection scratch for the next call

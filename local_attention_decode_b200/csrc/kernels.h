@@ -186,9 +186,15 @@ constexpr int kAttnChunk = 64;   // keys per team chunk (one team of 4 warps)
 constexpr int kAttnMaxTeams = 4;
 // Team chunks per CTA unit, and CTA units per (query, KV head), for a key set
 // of at most max_keys keys: units of up to 256 keys.
+// Teams of 64 keys per attention unit: up to kAttnMaxTeams teams merged in
+// one CTA unit for a key set of at most 256 (one unit per query and KV head,
+// no combine: the sliding window); a single team per unit above, so that a
+// top-k selection spreads over one unit per 64 keys (at most 32 for
+// DSA_MAX_TOPK) and every SM gathers a share.
 inline int attn_teams(int max_keys) {
     const int c = (max_keys + kAttnChunk - 1) / kAttnChunk;
-    return c < kAttnMaxTeams ? (c > 0 ? c : 1) : kAttnMaxTeams;
+    if (c > kAttnMaxTeams) return 1;
+    return c > 0 ? c : 1;
 }
 inline int attn_splits(int max_keys) {
     const int u = kAttnChunk * attn_teams(max_keys);

@@ -411,8 +411,7 @@ prefill_select_kernel(const uint32_t *cand_cnt, const uint2 *cand, int cap, cons
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0), nb = pass == 2 ? 1024 : 2048;
         for (int b = t; b < nb; b += NT) sh->hist[b] = 0;
         __syncthreads();
-        for (uint32_t j = t; j < m; j += NT)
-            if ((lkey[j] & mask) == prefix) atomicAdd(&sh->hist[(lkey[j] >> shift) & (nb - 1)], 1u);
+        list_digit_hist<NT>(sh->hist, m, prefix, mask, shift, (uint32_t)nb, [&](uint32_t j, uint32_t &k) { k = lkey[j]; return true; });
         __syncthreads();
         topk::find_threshold<NT>(sh, nb, Krem);
         prefix |= (uint32_t)sh->bin << shift;
@@ -437,10 +436,10 @@ prefill_select_kernel(const uint32_t *cand_cnt, const uint2 *cand, int cap, cons
             const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0), nb = pass == 2 ? 1024 : 2048;
             for (int b = t; b < nb; b += NT) sh->hist[b] = 0;
             __syncthreads();
-            for (uint32_t j = t; j < m; j += NT) {
-                const uint32_t v = ~lpos[j];
-                if (lkey[j] == Tstar && (v & pmask) == pprefix) atomicAdd(&sh->hist[(v >> shift) & (nb - 1)], 1u);
-            }
+            list_digit_hist<NT>(sh->hist, m, pprefix, pmask, shift, (uint32_t)nb, [&](uint32_t j, uint32_t &v) {
+                v = ~lpos[j];
+                return lkey[j] == Tstar;
+            });
             __syncthreads();
             topk::find_threshold<NT>(sh, nb, Kp);
             pprefix |= (uint32_t)sh->bin << shift;

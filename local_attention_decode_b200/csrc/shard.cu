@@ -79,8 +79,11 @@ merge_kernel(const float *cand_score, const int32_t *cand_pos, int N, int K, int
             const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0), nb = pass == 2 ? 1024 : 2048;
             for (int b = t; b < nb; b += kThreads) sh->hist[b] = 0;
             __syncthreads();
-            for (int i = t; i < n; i += kThreads)
-                if (pos[i] >= 0 && (key[i] & mask) == prefix) atomicAdd(&sh->hist[(key[i] >> shift) & (nb - 1)], 1u);
+            list_digit_hist<kThreads>(sh->hist, (uint32_t)n, prefix, mask, shift, (uint32_t)nb,
+                                      [&](uint32_t i, uint32_t &k) {
+                                          k = key[i];
+                                          return pos[i] >= 0;
+                                      });
             __syncthreads();
             topk::find_threshold<kThreads>(sh, nb, Krem);
             prefix |= (uint32_t)sh->bin << shift;

@@ -512,7 +512,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     warp_part<NT>(len, &wlo, &whi);
     uint32_t wc = 0;
     warp_walk(wlo, whi, cached, cache, key_at, [&](int64_t j, bool valid, uint32_t k) {
-        if (valid && (k & mask) == prefix) atomicAdd(&sh->hist[(k >> 10) & (kBins - 1)], 1u);
+        warp_hist_add(sh->hist, (k >> 10) & (kBins - 1), valid && (k & mask) == prefix);
         const bool cand = valid && k >= prefix;
         const uint32_t cm = __ballot_sync(0xffffffffu, cand);
         if (cand) {
@@ -633,10 +633,7 @@ __device__ void select_row(const Params &p, Shared<NT> *sh, uint32_t *cache, int
     if (use_list) {
         for (int j = threadIdx.x; j < 1024; j += NT) sh->hist[j] = 0;
         __syncthreads();
-        for (uint32_t j = threadIdx.x; j < m; j += NT) {
-            const uint32_t k = lkey[j];
-            if ((k & mask) == prefix) atomicAdd(&sh->hist[k & 1023u], 1u);
-        }
+        list_digit_hist<NT>(sh->hist, m, prefix, mask, 0, 1024u, [&](uint32_t j, uint32_t &k) { k = lkey[j]; return true; });
         __syncthreads();
     } else {
         slice_hist(prefix, mask, 0, 1024);
@@ -876,8 +873,8 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
                 if (j < m) {
                     lkey[j] = kv[u];
                     lpos[j] = pv[u];
-                    if ((kv[u] & mask) == prefix) atomicAdd(&sh->hist[(kv[u] >> 10) & 1023u], 1u);
                 }
+                warp_hist_add(sh->hist, (kv[u] >> 10) & 1023u, j < m && (kv[u] & mask) == prefix);
             }
         }
         __syncthreads();
@@ -889,14 +886,7 @@ __device__ bool select_row_hist(const Params &p, Shared<NT> *sh, uint32_t *cache
         if (r == 1) {
             for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
             __syncthreads();
-            for (uint32_t base = threadIdx.x; base < m; base += 4 * NT) {   // four loads in flight
-                uint32_t k4[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) k4[u] = base + u * NT < m ? lkey[base + u * NT] : ~prefix;
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if ((k4[u] & mask) == prefix) atomicAdd(&sh->hist[(k4[u] >> shift) & (uint32_t)(nb - 1)], 1u);
-            }
+            list_digit_hist<NT>(sh->hist, m, prefix, mask, shift, (uint32_t)nb, [&](uint32_t j, uint32_t &k) { k = lkey[j]; return true; });
             __syncthreads();
         }
         find_threshold<NT>(sh, nb, Krem);
