@@ -235,7 +235,7 @@ def read_stream_gbps(torch, dev, stream) -> float:
     return (1 << 30) / (best / 1e3) / 1e9
 
 
-def decode_config(workload: str, world: int) -> dict:
+def decode_config(workload: str, world: int, layers: int = 1) -> dict:
     """The `config` object of a decode workload's line (both arms)."""
     from workloads import CONFIGS
     cfg = CONFIGS[workload]
@@ -243,7 +243,10 @@ def decode_config(workload: str, world: int) -> dict:
         "workload": WORKLOAD_DESC[workload],
         "batch": len(cfg["seq_lens"]), "query_tokens": cfg["T"], "context": max(cfg["seq_lens"]), "top_k": TOP_K,
         "seed": cfg["seed"], "needles": cfg["n_needles"], "parallelism": f"replicas x{world}",
-        "l2": "flushed between steps outside the timed events (256 MB write, then 256 MB read so no dirty lines remain)",
+        "layers_in_rotation": layers,
+        "l2": (f"inputs larger than L2: {layers} layers' caches in rotation, steps back to back, no flush"
+               if layers > 1 else
+               "flushed between steps outside the timed events (256 MB write, then 256 MB read so no dirty lines remain)"),
     }
 
 
@@ -574,6 +577,14 @@ def run_prefill(args, rank, world, local_rank):
 
 # ------------------------------------------------------------------ ours
 def run_ours(args, rank, world, local_rank):
+    """The layer-step at the workload's configuration.  Timed: K steps issued
+    back to back, as a decode issues a model's DSA layers, each step on the
+    next of R layers' own caches (index keys, K, V and queries drawn with
+    their own seeds), so no step finds its keys in L2 -- the R caches hold
+    R x 2.7 GB at 1M context against a 126 MB L2.  The R steps are one CUDA
+    graph replayed K / R times: no host launch gaps.  Reported beside it: the
+    same step isolated (L2 flushed, events around the one call), and the
+    one-barrier kernel's phase trace."""
     import torch
     import local_attention_decode_b200 as dsa
     from workloads import CONFIGS, make_decode_workload
@@ -581,12 +592,19 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = CONFIGS[args.workload]
-    wl = make_decode_workload(device=dev, **cfg)
+    R = max(1, args.layers)
+    layers = []
+    for r in range(R):
+        c = dict(cfg)
+        c["seed"] = cfg["seed"] + 1000 * r
+        w_r = make_decode_workload(device=dev, **c)
+        kv_r = dsa.KV(k=w_r.K, v=w_r.V, index_k=w_r.k8, index_k_scale=w_r.k_scale, num_kv_heads=w_r.G,
+                      seq_stride=w_r.layout.seq_stride, num_rows=w_r.layout.num_rows)
+        layers.append((w_r, kv_r))
+    wl, kv = layers[0]
     B, T = wl.B, wl.T
     L = wl.layout.seq_lens[0]
     sm_scale = 1.0 / math.sqrt(192)
-    kv = dsa.KV(k=wl.K, v=wl.V, index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G,
-                seq_stride=wl.layout.seq_stride, num_rows=wl.layout.num_rows)
     O = torch.empty((B, T, 64, 128), dtype=torch.bfloat16, device=dev)
     idx = torch.empty((B, T, TOP_K), dtype=torch.int32, device=dev)
     cnt = torch.empty((B, T), dtype=torch.int32, device=dev)
@@ -600,68 +618,141 @@ def run_ours(args, rank, world, local_rank):
             e.record(stream)   # materialise the handle
         return evs
 
-    def step(events=None):
-        dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, L, TOP_K, wl.sink, sm_scale, O,
+    def step(i=0, events=None):
+        w_i, kv_i = layers[i % R]
+        dsa.dsa_layer_decode(w_i.q8, w_i.q_scale, w_i.w, w_i.Q, kv_i, w_i.q_pos, L, TOP_K, w_i.sink, sm_scale, O,
                              None, idx, cnt, ws, stage_events=events)
 
-    for _ in range(args.warmup):
-        flush()
-        step()
+    for i in range(args.warmup):
+        step(i)
     torch.cuda.synchronize(dev)
     st, _ = dsa.dsa_check_device_status(ws)
     if st != dsa.DSA_OK:
         raise RuntimeError(f"device status {st} after warm-up")
 
-    K = args.steps
+    # ---- the R layer-steps captured once into a CUDA graph
+    graph_note = f"{R} layers' steps in one CUDA graph, replayed"
+    graph = None
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(R):
+                step(i)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(R):
+                step(i)
+        torch.cuda.synchronize(dev)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+    except Exception as e:   # a launch that cannot be captured: eager launches
+        graph = None
+        graph_note = f"eager launches (graph capture failed: {type(e).__name__}: {e})"
+        torch.cuda.synchronize(dev)
+
+    K = max(R, args.steps // R * R)
     fused = B * T <= FUSED_MAX_ROWS
     paths0 = dsa.dsa_layer_path_counts(ws)
-    # one fused kernel: only the events around it (no event records between its end and the last event)
-    stage = [new_events(5) for _ in range(K)]
-    if fused:
-        stage = [[ev[0], None, None, None, ev[4]] for ev in stage]
-    torch.cuda.synchronize(dev)
+    t0, t1 = new_events(2)
     sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
     barrier(dev)
     torch.cuda.synchronize(dev)
     sampler.start()
-    for i in range(K):
-        flush()
-        step(stage[i])
+    t0.record(stream)
+    if graph is not None:
+        for _ in range(K // R):
+            graph.replay()
+    else:
+        for i in range(K):
+            step(i)
+    t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(dev)
     clocks = sampler.stop()
-
-    step_ms = [stage[i][0].elapsed_time(stage[i][4]) for i in range(K)]
-    if not fused:
-        idx_ms = [stage[i][0].elapsed_time(stage[i][1]) for i in range(K)]
-        topk_ms = [stage[i][1].elapsed_time(stage[i][2]) for i in range(K)]
-        attn_ms = [stage[i][2].elapsed_time(stage[i][3]) for i in range(K)]
-        comb_ms = [stage[i][3].elapsed_time(stage[i][4]) for i in range(K)]
-    total_s = max_over_ranks(sum(step_ms) / 1e3, dev)
+    total_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, dev)
     paths1 = dsa.dsa_layer_path_counts(ws)
     st, _ = dsa.dsa_check_device_status(ws)
     if st != dsa.DSA_OK:
         raise RuntimeError(f"device status {st} after the timed steps")
 
-    # the indexer on its own (dsa_indexer_scores), same inputs, for its HBM rate
+    # ---- the same step isolated: L2 flushed, events around the one call
+    K_iso = min(K, 100)
+    stage = [new_events(5) for _ in range(K_iso)]
+    if fused:
+        stage = [[ev[0], None, None, None, ev[4]] for ev in stage]
+    torch.cuda.synchronize(dev)
+    for i in range(K_iso):
+        flush()
+        step(0, stage[i])
+    torch.cuda.synchronize(dev)
+    iso_ms = [stage[i][0].elapsed_time(stage[i][4]) for i in range(K_iso)]
+    if not fused:
+        idx_ms = [stage[i][0].elapsed_time(stage[i][1]) for i in range(K_iso)]
+        topk_ms = [stage[i][1].elapsed_time(stage[i][2]) for i in range(K_iso)]
+        attn_ms = [stage[i][2].elapsed_time(stage[i][3]) for i in range(K_iso)]
+        comb_ms = [stage[i][3].elapsed_time(stage[i][4]) for i in range(K_iso)]
+
+    # ---- the one-barrier kernel's phases (trace marks; steps back to back, untimed)
+    phases = trace_phases(dsa, torch, dev, lambda i: step(i), R)
+
+    # ---- the indexer on its own (dsa_indexer_scores) over the R layers' caches, back to back
     idx_ws = dsa.alloc_workspace(dsa.OP_INDEXER, B, T, L, 1, device=dev)
     scores = torch.empty((B, T, L), dtype=torch.float32, device=dev)
-    ikv = dsa.KV(index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G, seq_stride=wl.layout.seq_stride,
-                 num_rows=wl.layout.num_rows)
-    K2 = min(K, 200)
-    iev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
-    for i in range(3 + K2):
-        flush()
-        # a bounded GPU sleep (outside the events) holds the stream while the
-        # host prepares the call, so the events see only the kernel
-        torch.cuda._sleep(200_000)
-        if i >= 3:
-            iev[i - 3][0].record(stream)
-        dsa.dsa_indexer_scores(wl.q8, wl.q_scale, wl.w, ikv, wl.q_pos, L, scores, idx_ws)
-        if i >= 3:
-            iev[i - 3][1].record(stream)
+    ikvs = [dsa.KV(index_k=w_r.k8, index_k_scale=w_r.k_scale, num_kv_heads=w_r.G, seq_stride=w_r.layout.seq_stride,
+                   num_rows=w_r.layout.num_rows) for w_r, _ in layers]
+
+    def ind(i):
+        w_i = layers[i % R][0]
+        dsa.dsa_indexer_scores(w_i.q8, w_i.q_scale, w_i.w, ikvs[i % R], w_i.q_pos, L, scores, idx_ws)
+
+    for i in range(R):
+        ind(i)
+    K2 = max(R, min(K, 400) // R * R)
+    igraph = None
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(R):
+                ind(i)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        igraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(igraph):
+            for i in range(R):
+                ind(i)
+        torch.cuda.synchronize(dev)
+        igraph.replay()
+    except Exception:
+        igraph = None
     torch.cuda.synchronize(dev)
-    ind_ms = [a.elapsed_time(b) for a, b in iev]
+    a_, b_ = new_events(2)
+    a_.record(stream)
+    if igraph is not None:
+        for _ in range(K2 // R):
+            igraph.replay()
+    else:
+        for i in range(K2):
+            ind(i)
+    b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ind_avg_s = a_.elapsed_time(b_) / 1e3 / K2
+    # and isolated (L2 flushed; a bounded GPU sleep outside the events holds the
+    # stream while the host prepares the call, so the events see only the kernel)
+    K3 = min(K2, 100)
+    iev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K3)]
+    for i in range(K3):
+        flush()
+        torch.cuda._sleep(200_000)
+        iev[i][0].record(stream)
+        ind(0)
+        iev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ind_iso_ms = [a.elapsed_time(b) for a, b in iev]
     del scores
 
     # ---- a read-only stream reference measured in this run (torch sum over 1 GiB):
@@ -676,12 +767,12 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = measured_peaks()
     ib = indexer_bytes(L, T)
     layer_bytes = ib + gathered_bytes(T, TOP_K)
-    ind_avg_s = sum(ind_ms) / K2 / 1e3
+    one_barrier = paths1[0] + paths1[1] > paths0[0] + paths0[1]
     if fused:   # one kernel does the whole step: its roofline is the whole step's bytes
-        kern = "dsa_layer_capture_kernel" if paths1[0] + paths1[1] > paths0[0] + paths0[1] else "dsa_layer_fused_kernel"
+        kern = "dsa_layer_capture_kernel" if one_barrier else "dsa_layer_fused_kernel"
         kern_bytes, kern_avg_s = layer_bytes, total_s / K
     else:
-        kern, kern_bytes, kern_avg_s = "indexer_kernel", ib, sum(idx_ms) / K / 1e3
+        kern, kern_bytes, kern_avg_s = "indexer_kernel", ib, ind_avg_s
     achieved = kern_bytes / kern_avg_s / 1e9
     line = {
         "metric": METRIC,
@@ -696,26 +787,32 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e4m3xe4m3->f32 indexer; bf16 attention, f32 softmax",
         "data": "synthetic",
-        "config": decode_config(args.workload, world),
+        "config": decode_config(args.workload, world, R),
         "us_per_layer_step": total_s * 1e6 / K,
+        "timing": f"{K} steps back to back over {R} layers' caches ({graph_note}); one event pair around them",
         "path": ("one cooperative kernel" if fused else "four kernels"),
         "timed_steps_by_path": {"one_barrier_fast": paths1[0] - paths0[0],
                                 "one_barrier_general": paths1[1] - paths0[1],
                                 "other": K - (paths1[0] - paths0[0]) - (paths1[1] - paths0[1])},
-        "stage_us_median": ({"fused_layer_step": statistics.median(step_ms) * 1e3} if fused else {
+        "isolated_step_us": {"median": statistics.median(iso_ms) * 1e3, "mean": statistics.fmean(iso_ms) * 1e3,
+                             "how": "L2 flushed before each step; events around the one call (launch included)"},
+        "stage_us_median": ({"layer_step_isolated": statistics.median(iso_ms) * 1e3} if fused else {
             "indexer": statistics.median(idx_ms) * 1e3, "topk": statistics.median(topk_ms) * 1e3,
             "attention": statistics.median(attn_ms) * 1e3, "combine": statistics.median(comb_ms) * 1e3,
         }),
+        "phase_us": phases,
         "indexer_standalone": {
-            "us_median": statistics.median(ind_ms) * 1e3, "us_mean": ind_avg_s * 1e6, "bytes": ib,
+            "us_mean": ind_avg_s * 1e6, "bytes": ib,
             "GBps": ib / ind_avg_s / 1e9, "frac_of_measured_peak": ib / ind_avg_s / 1e9 / peak,
             "frac_of_8TBps_nominal": ib / ind_avg_s / 1e9 / NOMINAL_HBM_GBS,
+            "how": f"{K2} launches back to back over the {R} layers' index caches, one event pair",
+            "isolated_us_median": statistics.median(ind_iso_ms) * 1e3,
         },
         "layer_step_byte_roofline_us": {
-            "bytes": ib + gathered_bytes(T, TOP_K),
-            "at_measured_peak": (ib + gathered_bytes(T, TOP_K)) / (peak * 1e9) * 1e6,
-            "at_8TBps_nominal": (ib + gathered_bytes(T, TOP_K)) / (NOMINAL_HBM_GBS * 1e9) * 1e6,
-            "at_read_stream": (ib + gathered_bytes(T, TOP_K)) / (read_gbs * 1e9) * 1e6,
+            "bytes": layer_bytes,
+            "at_measured_peak": layer_bytes / (peak * 1e9) * 1e6,
+            "at_8TBps_nominal": layer_bytes / (NOMINAL_HBM_GBS * 1e9) * 1e6,
+            "at_read_stream": layer_bytes / (read_gbs * 1e9) * 1e6,
         },
         "read_stream_reference": {"GBps": read_gbs, "how": "torch sum over 1 GiB fp32, best of 6, CUDA events",
                                   "layer_step_frac": kern_bytes / kern_avg_s / 1e9 / read_gbs if fused else None,
@@ -733,6 +830,35 @@ def run_ours(args, rank, world, local_rank):
         "_workload": wl,
     }
     return line
+
+
+def trace_phases(dsa, torch, dev, step, R, n=8):
+    """Median over n steps of each phase mark of the one-barrier layer-step
+    kernel, in us after the first CTA's entry, as the latest CTA reached it
+    (dsa_trace_phases); {} when that kernel did not run."""
+    import numpy as np
+    tr = torch.zeros(148 * 2 * dsa.TRACE_MARKS, dtype=torch.int64, device=dev)
+    names = {10: "first_key_tile_requested", 12: "first_tile_scored", 7: "sample_handed_in", 1: "thresholds_seen",
+             2: "key_stream_done", 3: "past_grid_barrier", 8: "candidates_in_smem", 9: "kth_key_found",
+             4: "selection_done", 5: "attention_units_done", 6: "exit"}
+    rows = []
+    dsa.dsa_trace_phases(tr)
+    try:
+        for i in range(n):
+            tr.zero_()
+            step(i)
+            torch.cuda.synchronize(dev)
+            m = tr.view(-1, dsa.TRACE_MARKS).cpu().numpy().astype(np.float64)
+            m = m[m[:, 0] > 0]
+            if len(m) == 0:
+                return {}
+            t0 = m[:, 0].min()
+            rows.append({k: (m[:, k][m[:, k] > 0].max() - t0) / 1e3 for k in names if (m[:, k] > 0).any()})
+    finally:
+        dsa.dsa_trace_phases(None)
+    out = {names[k]: float(np.median([r[k] for r in rows if k in r])) for k in names if any(k in r for r in rows)}
+    out["how"] = "latest CTA at each mark, us after the first CTA entered; median of 8 steps"
+    return out
 
 
 def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
@@ -840,7 +966,11 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
         graph_note = f"eager (graph capture failed: {type(e).__name__}: {e})"
         torch.cuda.synchronize(dev)
         evs = timed(step)
-    for w_ in (ws, ws_p):    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
+    for w_ in (ws, ws_p):
+        st, _ = dsa.dsa_check_device_status(w_)
+        if st != dsa.DSA_OK:
+            raise RuntimeError(f"device status {st} after the end-to-end steps")
+    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
     import torch.distributed as dist
     world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
     return {"value": throughput(B * T, K, world, total_s), "unit": "tok/s", "h2d_bytes_per_step": h2d,
@@ -964,7 +1094,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": decode_config(WORKLOAD, world),
+        "config": decode_config(WORKLOAD, world, args.layers),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": how,
                          "cpu_model": cpu_model(), "extrapolated": n != L},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -976,6 +1106,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--layers", type=int, default=4,
+                    help="layers' caches the timed decode steps rotate over (inputs larger than L2)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the ragged-mix and prefill lines that the default run adds as extra keys")

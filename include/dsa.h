@@ -189,7 +189,8 @@ int dsa_debug_inject(int kind, int64_t wait_limit_ns);
  *   selection done, 5 the attention units done, 6 exit, 7 the CTA's sample
  *   handed in, 8 the candidate list in shared memory, 9 the k-th key found
  *   (radix select done), 10 the first key tile requested, 11 its MMA issued,
- *   12 its scores in the epilogue; 13..15 unused.
+ *   12 its scores in the epilogue; 13 and 14 the SM's cycle counter
+ *   (clock64) at entry and at exit, for the clock rate; 15 unused.
  * Marks a CTA does not reach (a CTA with no selection or attention work, the
  * general path) are written as 0.  `buf` is device memory of the caller's,
  * `words` its length in uint64 words; a launch with a grid too large for it

@@ -12,7 +12,9 @@
 // selected keys; the sink column in the softmax).
 //
 // attn_unit: a team of 4 warps takes 64 keys of one KV head, gathers their K
-// and V rows into shared memory with 16-byte cp.async, and computes for the
+// and V rows (and the group's query rows) into shared memory with one bulk
+// copy per row on the TMA engine (a per-thread 16-byte copy path costs several
+// times more on this GPU), and computes for the
 // 64/G query heads of that group  S = Q K^T  and  O = softmax_partial(S) V  on
 // the tensor cores (mma.sync m16n8k16 bf16 -> fp32; the query heads of a group
 // form the 16-row M dimension).  Each warp owns 16 keys; the four warps merge
@@ -34,6 +36,7 @@ constexpr int kChunk = kAttnChunk;   // keys per CTA
 constexpr int kThreads = 128;
 constexpr int kQS = DSA_QK_DIM + 8;  // padded smem row stride of Q and K (elements)
 constexpr int kVS = DSA_V_DIM + 8;   // padded smem row stride of V
+constexpr int kOS = DSA_V_DIM + 8;   // padded row stride (floats) of the O exchange: rows 8 banks apart
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Params {
@@ -64,11 +67,14 @@ struct Smem {
     __nv_bfloat16 k[kChunk * kQS];
     __nv_bfloat16 v[kChunk * kVS];
     int64_t row[kChunk];
+    uint64_t bar[2];   // bulk-copy completion: [0] Q and K rows, [1] V rows
     float m[4][16];
     float l[4][16];
     float tm[16];   // the team's result: per head row, the max logit (log2 domain) ...
     float tl[16];   // ... and the sum of exp2(logit - max); its O is in the first 8 KB of k
 };
+
+static_assert(4 * 16 * kOS * 4 <= sizeof(Smem::k) + sizeof(Smem::v), "the O exchange fits in the K and V tiles");
 
 // The teams' shared memory of a CTA: team t at base + t * stride.
 struct TeamSmem {
@@ -167,6 +173,12 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     }
 
     // ---- positions -> cache rows (invalid ones are flagged and masked)
+    if (tid == 0) {   // the team's copy barriers, fresh for this unit
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        fence_mbar_init();
+    }
+    int64_t key_row_of_tid = -1;
     if (tid < kChunk) {
         int64_t row = -1;
         if (tid < nk) {
@@ -181,36 +193,44 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
             }
         }
         sm.row[tid] = row;
+        key_row_of_tid = row;
     }
-    // ---- Q rows of this head group (rows >= hpg are zero)
-    const __nv_bfloat16 *qg = p.Q + ((int64_t)bt * DSA_Q_HEADS + g * hpg) * DSA_QK_DIM;
-    for (int c = tid; c < 16 * (DSA_QK_DIM / 8); c += kThreads) {
-        int r = c / (DSA_QK_DIM / 8), col = (c % (DSA_QK_DIM / 8)) * 8;
-        __nv_bfloat16 *dst = sm.q + r * kQS + col;
-        if (r < hpg) cp_async16(dst, qg + (int64_t)r * DSA_QK_DIM + col);
-        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
+    fence_proxy_async_smem();   // this thread's earlier use of the tiles, before the copies overwrite them
     team_sync(bar);
-    // ---- gather K and V rows
+    // ---- one bulk copy per row: thread r < 64 its key's K and V rows (or
+    //      zeros), thread 64 + r query head r of the group (or zeros)
     const int G = p.G;
-    for (int c = tid; c < kChunk * (DSA_QK_DIM / 8); c += kThreads) {
-        int r = c / (DSA_QK_DIM / 8), col = (c % (DSA_QK_DIM / 8)) * 8;
-        __nv_bfloat16 *dst = sm.k + r * kQS + col;
-        int64_t row = sm.row[r];
-        if (row >= 0) cp_async16(dst, p.K + (row * G + g) * DSA_QK_DIM + col);
-        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+    if (tid < kChunk) {
+        __nv_bfloat16 *dk = sm.k + tid * kQS, *dv = sm.v + tid * kVS;
+        const int64_t row = key_row_of_tid;
+        if (row >= 0) {
+            mbar_expect_tx(&sm.bar[0], DSA_QK_DIM * 2);
+            bulk_load(dk, p.K + (row * G + g) * DSA_QK_DIM, DSA_QK_DIM * 2, &sm.bar[0]);
+            mbar_expect_tx(&sm.bar[1], DSA_V_DIM * 2);
+            bulk_load(dv, p.V + (row * G + g) * DSA_V_DIM, DSA_V_DIM * 2, &sm.bar[1]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < DSA_QK_DIM / 8; ++c) reinterpret_cast<uint4 *>(dk)[c] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int c = 0; c < DSA_V_DIM / 8; ++c) reinterpret_cast<uint4 *>(dv)[c] = make_uint4(0, 0, 0, 0);
+        }
+    } else if (tid < kChunk + 16) {
+        const int r = tid - kChunk;
+        __nv_bfloat16 *dq = sm.q + r * kQS;
+        if (r < hpg) {
+            mbar_expect_tx(&sm.bar[0], DSA_QK_DIM * 2);
+            bulk_load(dq, p.Q + ((int64_t)bt * DSA_Q_HEADS + g * hpg + r) * DSA_QK_DIM, DSA_QK_DIM * 2, &sm.bar[0]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < DSA_QK_DIM / 8; ++c) reinterpret_cast<uint4 *>(dq)[c] = make_uint4(0, 0, 0, 0);
+        }
     }
-    cp_async_commit();   // Q and K: the first group
-    for (int c = tid; c < kChunk * (DSA_V_DIM / 8); c += kThreads) {
-        int r = c / (DSA_V_DIM / 8), col = (c % (DSA_V_DIM / 8)) * 8;
-        __nv_bfloat16 *dst = sm.v + r * kVS + col;
-        int64_t row = sm.row[r];
-        if (row >= 0) cp_async16(dst, p.V + (row * G + g) * DSA_V_DIM + col);
-        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+    team_sync(bar);   // every expected byte is posted, and the zero rows are written
+    if (tid == 0) {
+        mbar_arrive(&sm.bar[0]);
+        mbar_arrive(&sm.bar[1]);
     }
-    cp_async_commit();   // V: the second group
-    cp_async_wait_group<1>();   // Q and K have landed; V may still be in flight
-    team_sync(bar);
+    mbar_wait(&sm.bar[0], 0, p.status);   // Q and K have landed; V may still be in flight
 
     // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8)
     const int key0 = warp * 16;
@@ -265,8 +285,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     float o[DSA_V_DIM / 8][4];
 #pragma unroll
     for (int nt = 0; nt < DSA_V_DIM / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-    cp_async_wait_group<0>();
-    team_sync(bar);
+    mbar_wait(&sm.bar[1], 0, p.status);
 #pragma unroll
     for (int dp = 0; dp < DSA_V_DIM / 16; ++dp) {
         uint32_t b0, b1, b2, b3;
@@ -284,7 +303,11 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
         sm.l[warp][g0 + 8] = lrow[1];
     }
     team_sync(bar);   // K/V tiles are no longer read: reuse them for the O exchange
-    float *so = reinterpret_cast<float *>(sm.k);   // [4 warps][16 rows][128]
+    if (tid == 0) {   // every thread of the team is past its waits
+        mbar_inval(&sm.bar[0]);
+        mbar_inval(&sm.bar[1]);
+    }
+    float *so = reinterpret_cast<float *>(sm.k);   // [4 warps][16 rows][kOS] (runs on into sm.v)
     float scale_row[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -295,15 +318,16 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
 #pragma unroll
     for (int nt = 0; nt < DSA_V_DIM / 8; ++nt) {
         const int col = nt * 8 + cq * 2;
-        float *d0 = so + (warp * 16 + g0) * DSA_V_DIM + col;
-        float *d1 = so + (warp * 16 + g0 + 8) * DSA_V_DIM + col;
+        float *d0 = so + (warp * 16 + g0) * kOS + col;
+        float *d1 = so + (warp * 16 + g0 + 8) * kOS + col;
         *reinterpret_cast<float2 *>(d0) = make_float2(o[nt][0] * scale_row[0], o[nt][1] * scale_row[0]);
         *reinterpret_cast<float2 *>(d1) = make_float2(o[nt][2] * scale_row[1], o[nt][3] * scale_row[1]);
     }
     team_sync(bar);
-    // each thread: one head row (tid / 8) and 16 columns; the four warps'
-    // scaled O summed in registers, then written over warp 0's slot
-    const int row = tid >> 3, c0 = (tid & 7) * 16;
+    // each thread: one head row (tid / 8) and four 4-column pieces 32 apart
+    // (eight threads read a row's 128 contiguous bytes at a time); the four
+    // warps' scaled O summed in registers, then written over warp 0's slot
+    const int row = tid >> 3, c0 = (tid & 7) * 4;
     float4 acc[4];
     float M = -INFINITY, L = 0.f;
     if (row < hpg) {
@@ -316,7 +340,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
             acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const float4 v = *reinterpret_cast<const float4 *>(so + (w * 16 + row) * DSA_V_DIM + c0 + 4 * c);
+                const float4 v = *reinterpret_cast<const float4 *>(so + (w * 16 + row) * kOS + c0 + 32 * c);
                 acc[c].x += v.x; acc[c].y += v.y; acc[c].z += v.z; acc[c].w += v.w;
             }
         }
@@ -324,7 +348,7 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     team_sync(bar);
     if (row < hpg) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) *reinterpret_cast<float4 *>(so + row * DSA_V_DIM + c0 + 4 * c) = acc[c];
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<float4 *>(so + row * kOS + c0 + 32 * c) = acc[c];
         if ((tid & 7) == 0) {
             sm.tm[row] = M;
             sm.tl[row] = L;
@@ -353,7 +377,7 @@ __device__ __forceinline__ void cta_merge(const Params &p, const TeamSmem &teams
             if (mt == -INFINITY) continue;
             const float w = exp2f(mt - M);
             const float4 v = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(teams[tm].k) +
-                                                               row * DSA_V_DIM + c);
+                                                               row * kOS + c);
             acc.x += v.x * w; acc.y += v.y * w; acc.z += v.z * w; acc.w += v.w * w;
             L += teams[tm].tl[row] * w;
         }

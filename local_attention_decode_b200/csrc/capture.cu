@@ -64,6 +64,8 @@ constexpr int kHistWords = kBins + 1;         // + the count of negative scores
 constexpr int kHistStride = kHistWords + 3;   // words between rows' histograms: rows start 16-byte aligned
 constexpr int kSegCap = 1024;                 // candidates one epilogue group may hold per row
 constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
+constexpr int kWide = 4096;                   // bins of the selection's first histogram
+constexpr int kSmall = 2048;                  // keys of T*'s bin taken aside for the remaining bits
 constexpr int kGroupBar0 = 5;                 // named barriers 5..8: the epilogue groups
 constexpr int kUnitBar = 9;                   // named barrier of the attention teams of a CTA unit
 constexpr int kSelBytes = DSA_MAX_TOPK * 4;   // the selection, at the start of shared memory in phase 2
@@ -133,11 +135,13 @@ __device__ __forceinline__ uint32_t sample_bin(uint32_t key) {
     return (key >> 31) ? ((key >> 20) & (kBins - 1)) : (uint32_t)kBins;
 }
 
-// The threshold of one row from its global sample histogram, by one warp:
-// the lower edge of the highest bin b whose count, with the bins above it,
-// reaches `target`; zero (take every key) when the sample's non-negative
-// scores do not reach it.  Zeroes the histogram for the next call.
-__device__ uint32_t row_threshold(uint32_t *hist, uint32_t target) {
+// The threshold of one row from its global sample histogram, by one warp.
+// The sample's visible keys (the histogram's total, tot) predict
+// oversample * K * tot / n + 16 of them at or above the row's threshold; the
+// threshold is the lower edge of the highest bin b whose count, with the bins
+// above it, reaches that target; zero (take every key) when the sample's
+// non-negative scores do not reach it.  Zeroes the histogram for the next call.
+__device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversample) {
     const int lane = lane_id();
     constexpr int kPer = kBins / 32;   // 64 bins per lane
     uint32_t s = 0;
@@ -147,12 +151,16 @@ __device__ uint32_t row_threshold(uint32_t *hist, uint32_t target) {
         const uint4 v = __ldcg(h4 + u);
         s += v.x + v.y + v.z + v.w;
     }
+    const uint32_t negative = __ldcg(hist + kBins);
     uint32_t incl = s;   // keys in this lane's bins and all higher ones
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
         if (lane + o < 32) incl += u;
     }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 0) + negative;
+    const double want = (double)oversample * K * (double)tot / (double)n + 16.0;
+    const uint32_t target = (uint32_t)min((double)tot, ceil(want));
     const uint32_t hit = __ballot_sync(0xffffffffu, incl >= target);
     uint32_t thr = 0;
     if (target > 0 && hit) {
@@ -193,7 +201,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     using namespace indexer;
     const indexer::Params &p = cp.ix;
     const CUtensorMap &tmap_k = *tmap_k_p, &tmap_ks = *tmap_ks_p, &tmap_q = *tmap_q_p;
-    const int S = p.stages, T = p.T, B = p.B, N = 16 * T, GE = p.groups, rows = B * T;
+    const int S = p.stages, T = p.T, B = p.B, N = 16 * T, GE = p.groups, AB = p.acc_bufs, rows = B * T;
     Layout lay(S, T, B);
     Bars *bars = reinterpret_cast<Bars *>(smem + lay.bar_off);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.tmem_off);
@@ -255,17 +263,18 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     };
 
     uint32_t tmem_cols = 32;
-    while (tmem_cols < (uint32_t)(kPipes * GE * N)) tmem_cols <<= 1;
+    while (tmem_cols < (uint32_t)(kPipes * GE * AB * N)) tmem_cols <<= 1;
     if (threadIdx.x == 0) {
         for (int pp = 0; pp < kPipes; ++pp) {
             for (int s = 0; s < S; ++s) {
                 mbar_init(&bars->full[pp][s], 1);
                 mbar_init(&bars->empty[pp][s], 1 + kEpiWarps);
             }
-            for (int a = 0; a < GE; ++a) {
-                mbar_init(&bars->tfull[pp][a], 1);
-                mbar_init(&bars->tempty[pp][a], kEpiWarps);
-            }
+            for (int a = 0; a < GE; ++a)
+                for (int u = 0; u < AB; ++u) {
+                    mbar_init(&bars->tfull[pp][a][u], 1);
+                    mbar_init(&bars->tempty[pp][a][u], kEpiWarps);
+                }
             mbar_init(&bars->mma_done[pp], 1);
         }
         mbar_init(&bars->q_full, 1);
@@ -345,21 +354,22 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
             const uint32_t idesc = umma_idesc_e4m3_f32(kTile, N);
             for (int i = 0; i < n_p; ++i) {
                 const int s = i % S, st = pp * S + s, a = i % GE;
+                const int jj = i / GE, u = jj % AB;   // the group's jj-th tile, its accumulator
                 if (!mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status)) break;
-                if (i >= GE && !mbar_wait(&bars->tempty[pp][a], ((i / GE) & 1) ^ 1, p.status)) break;
+                if (jj >= AB && !mbar_wait(&bars->tempty[pp][a][u], ((jj / AB) & 1) ^ 1, p.status)) break;
                 if (i == 0 && !mbar_wait(&bars->q_full, 0, p.status)) break;
                 int b, ti;
                 locate(tile_of(pp, i), b, ti);
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(smem + lay.k_off + st * kTile * kKeyBytes);
                 const uint32_t b_addr = smem_u32(smem + lay.q_off + b * N * kKeyBytes);
-                const uint32_t d = tmem_base + (uint32_t)((pp * GE + a) * N);
+                const uint32_t d = tmem_base + (uint32_t)(((pp * GE + a) * AB + u) * N);
 #pragma unroll
                 for (int k = 0; k < kKeyBytes / 32; ++k)
                     umma_f8(d, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
                             k > 0 ? 1u : 0u);
                 umma_commit(&bars->empty[pp][s]);
-                umma_commit(&bars->tfull[pp][a]);
+                umma_commit(&bars->tfull[pp][a][u]);
                 if (i == 0 && pp == 0 && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 11] = globaltimer_ns();
             }
             umma_commit(&bars->mma_done[pp]);
@@ -381,7 +391,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         int32_t *qp = reinterpret_cast<int32_t *>(coef + 16 * T);
         // per group, twice (double-buffered): the four warps' candidate counts per query, the readiness poll
         uint32_t *xch = reinterpret_cast<uint32_t *>(smem + lay.xch_off) + gi * (2 * (kEpiWarps * kMaxRows + 1));
-        const uint32_t acc_col = (uint32_t)((pp * GE + a) * N);
+        const uint32_t acc_col0 = (uint32_t)((pp * GE + a) * AB * N);
         uint32_t base[kMaxRows] = {0u, 0u, 0u, 0u};
         uint32_t thr[kMaxRows] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
         bool ok = true, overflow = false, known = false;
@@ -503,7 +513,9 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                     __syncwarp();
                     cur_b = b;
                 }
-                bool w_ok = mbar_wait(&bars->tfull[pp][a], (j & 1), p.status) &&
+                const int u = j % AB;
+                const uint32_t acc_col = acc_col0 + (uint32_t)(u * N);
+                bool w_ok = mbar_wait(&bars->tfull[pp][a][u], (j / AB) & 1, p.status) &&
                             mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status);
                 if (__all_sync(0xffffffffu, w_ok)) {
                     if (j == 0 && gi == 0 && poller && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 12] = globaltimer_ns();
@@ -531,7 +543,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(&bars->tempty[pp][a]);
+                        mbar_arrive(&bars->tempty[pp][a][u]);
                         mbar_arrive(&bars->empty[pp][s]);
                     }
                     if (j == 0) {   // the sample: into the CTA's histogram of each row
@@ -574,14 +586,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             uint32_t t_r = 0xFFFFFFFFu;   // n <= top_k: every key is selected, nothing to capture
                             uint32_t *h = cp.sample_hist + r * kHistStride;
                             if (n > cp.K) {
-                                // the sample's visible keys: the histogram's total
-                                uint32_t tot = 0;
-                                for (int u = lane; u < kHistWords; u += 32) tot += __ldcg(h + u);
-#pragma unroll
-                                for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-                                const double want = (double)cp.oversample * cp.K * (double)tot / (double)n + 16.0;
-                                const uint32_t target = (uint32_t)min((double)tot, ceil(want));
-                                t_r = row_threshold(h, target);
+                                t_r = row_threshold(h, n, cp.K, cp.oversample);
                             } else {
                                 for (int u = lane; u < kHistWords; u += 32) h[u] = 0;
                             }
@@ -599,7 +604,10 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
             }
             // ---- this tile's candidates (deferred while the thresholds are unknown)
             uint32_t poll = 0;
-            if (!known && poller) poll = ld_acquire_gpu(ctl + kReady) >= 1u ? 1u : 0u;
+            if (!known && poller && ld_relaxed_gpu(ctl + kReady) >= 1u) {
+                fence_acq_rel_gpu();   // the thresholds the flag publishes, before the group reads them
+                poll = 1u;
+            }
             const bool was_known = known;
             bool seen = false;
             ok = capture_tile(b, pos, sc, (was_known && have && ok) ? cand_bits(b, vis, sc) : 0u, ok, poll, &seen);
@@ -643,10 +651,11 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 mbar_inval(&bars->full[pp][s]);
                 mbar_inval(&bars->empty[pp][s]);
             }
-            for (int a = 0; a < GE; ++a) {
-                mbar_inval(&bars->tfull[pp][a]);
-                mbar_inval(&bars->tempty[pp][a]);
-            }
+            for (int a = 0; a < GE; ++a)
+                for (int u = 0; u < AB; ++u) {
+                    mbar_inval(&bars->tfull[pp][a][u]);
+                    mbar_inval(&bars->tempty[pp][a][u]);
+                }
             mbar_inval(&bars->mma_done[pp]);
         }
         mbar_inval(&bars->q_full);
@@ -728,7 +737,10 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
     const uint32_t lt = (1u << lane) - 1u;
     auto *sh = reinterpret_cast<topk::Shared<NT> *>(work);
     uint32_t *off = reinterpret_cast<uint32_t *>(work + align128(sizeof(topk::Shared<NT>)));
-    uint2 *list = reinterpret_cast<uint2 *>(off + ((NG + 1 + 31) & ~31));   // (order key, position)
+    uint64_t *copied = reinterpret_cast<uint64_t *>(off + ((NG + 1 + 31) & ~31));   // bulk-copy barrier
+    uint2 *list = reinterpret_cast<uint2 *>(copied + 2);   // (order key, position), 16-byte aligned
+    uint32_t *wide = reinterpret_cast<uint32_t *>(list + kListCap);   // [kWide] histogram
+    uint32_t *bin_keys = wide + kWide;                                // [kSmall] keys of T*'s bin
     int64_t n = (int64_t)__ldg(cp.ix.q_pos + r) + 1;
     if (n > cp.ix.Lmax) n = cp.ix.Lmax;
     if (n < 0) n = 0;
@@ -736,42 +748,157 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
     if (n <= K) {
         for (int j = threadIdx.x; j < K; j += NT) sel[j] = j < n ? j : -1;
     } else {
-        // segment offsets (NG <= NT)
-        const uint32_t v = threadIdx.x < NG ? __ldcg(cp.counts + (int64_t)r * NG + threadIdx.x) : 0u;
-        uint32_t m;
-        const uint32_t incl = topk::block_scan<NT>(v, sh->warp_tmp, &m);
-        if (threadIdx.x < NG) off[threadIdx.x] = incl - v;
-        if (threadIdx.x == 0) off[NG] = m;
-        __syncthreads();
-        // the candidates, in position order: each warp copies whole segments,
-        // every copy in flight at once
-        const uint2 *segs = cp.lists + (int64_t)r * NG * kSegCap;
-        for (int sg = warp; sg < NG; sg += NW) {
-            const uint32_t o = off[sg], cnt = off[sg + 1] - o;
-            for (uint32_t i = lane; i < cnt; i += 32) attn::cp_async8(list + o + i, segs + (int64_t)sg * kSegCap + i);
+        // the segments, in position order, each padded to an even length so
+        // that it moves as one 16-byte-multiple bulk copy; a pad slot gets
+        // the entry (key 0, position -1): below every candidate's key (the
+        // threshold's, or a finite score's), so it is never selected
+        if (threadIdx.x == 0) {
+            mbar_init(copied, 1);
+            fence_mbar_init();
         }
-        attn::cp_async_commit();
-        attn::cp_async_wait_all();
+        const uint32_t v = threadIdx.x < NG ? __ldcg(cp.counts + (int64_t)r * NG + threadIdx.x) : 0u;
+        const uint32_t vp = (v + 1u) & ~1u;
+        uint32_t m;   // entries, pads included
+        const uint32_t incl = topk::block_scan<NT>(vp, sh->warp_tmp, &m);
+        if (threadIdx.x < NG) off[threadIdx.x] = incl - vp;
+        if (threadIdx.x == 0) off[NG] = m;
+        fence_proxy_async_smem();   // earlier use of the list area, before the copies overwrite it
+        __syncthreads();
+        const uint2 *segs = cp.lists + (int64_t)r * NG * kSegCap;
+        if (threadIdx.x < NG && vp > 0) {
+            mbar_expect_tx(copied, vp * 8u);
+            bulk_load(list + (incl - vp), segs + (int64_t)threadIdx.x * kSegCap, vp * 8u, copied);
+        }
+        __syncthreads();   // every expected byte is posted
+        if (threadIdx.x == 0) mbar_arrive(copied);
+        mbar_wait(copied, 0, cp.ix.status);
+        if (threadIdx.x < NG && (v & 1u)) list[incl - 1] = make_uint2(0u, 0xFFFFFFFFu);
         __syncthreads();
         if (trace && threadIdx.x == 0) trace[8] = globaltimer_ns();
-        // exact radix select of the k-th largest key: 11 + 11 + 10 bits
-        uint32_t prefix = 0u, mask = 0u, Krem = (uint32_t)K;
-#pragma unroll 1
-        for (int pass = 0; pass < 3; ++pass) {
-            const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-            const int nb = pass == 2 ? 1024 : 2048;
-            for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+        // ---- the k-th largest key T*, exactly.  The candidates lie above one
+        //      threshold, so their keys share the high bits: a histogram of
+        //      the 12 bits below the common ones finds T*'s bin in one pass;
+        //      only that bin's keys (a handful) go on to the remaining bits.
+        auto is_key = [&](uint32_t j, uint32_t &k) {
+            const uint2 e = list[j];
+            k = e.x;
+            return e.y != 0xFFFFFFFFu;   // not a pad
+        };
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        for (uint32_t j = threadIdx.x; j < m; j += NT) {
+            uint32_t k;
+            if (is_key(j, k)) {
+                kmin = min(kmin, k);
+                kmax = max(kmax, k);
+            }
+        }
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0) {
+            sh->warp_a[warp] = kmin;
+            sh->warp_b[warp] = kmax;
+        }
+        for (int j = threadIdx.x; j < kWide; j += NT) wide[j] = 0;
+        __syncthreads();
+        for (int w2 = 0; w2 < NW; ++w2) {
+            kmin = min(kmin, sh->warp_a[w2]);
+            kmax = max(kmax, sh->warp_b[w2]);
+        }
+        const int top = kmin == kmax ? 0 : 31 - __clz(kmin ^ kmax);   // highest bit in which keys differ
+        const int shift = top > 11 ? top - 11 : 0;
+        const uint32_t hi_mask = top >= 31 ? 0u : ~((2u << top) - 1u);   // the bits every key shares
+        list_digit_hist<NT>(wide, m, kmin & hi_mask, hi_mask, shift, (uint32_t)kWide, is_key);
+        __syncthreads();
+        {   // the bin of the k-th largest key: 512 threads own 8 bins each, from the top
+            uint32_t s = 0;
+            if (threadIdx.x < kWide / 8)
+                for (int i = 0; i < 8; ++i) s += wide[kWide - 1 - 8 * (int)threadIdx.x - i];
+            uint32_t tot;
+            const uint32_t incl = topk::block_scan<NT>(s, sh->warp_tmp, &tot);
+            if (threadIdx.x < kWide / 8 && incl - s < (uint32_t)K && (uint32_t)K <= incl) {
+                uint32_t above = incl - s;
+                for (int i = 0; i < 8; ++i) {
+                    const int b = kWide - 1 - 8 * (int)threadIdx.x - i;
+                    if (above + wide[b] >= (uint32_t)K) {
+                        sh->bin = b;
+                        sh->above = above;
+                        break;
+                    }
+                    above += wide[b];
+                }
+            }
             __syncthreads();
-            list_digit_hist<NT>(sh->hist, m, prefix, mask, shift, (uint32_t)nb, [&](uint32_t j, uint32_t &k) {
-                k = list[j].x;
-                return true;
-            });
-            __syncthreads();
-            topk::find_threshold<NT>(sh, nb, Krem);
-            prefix |= (uint32_t)sh->bin << shift;
-            mask |= (uint32_t)(nb - 1) << shift;
-            Krem -= sh->above;
-            __syncthreads();
+        }
+        uint32_t prefix = (kmin & hi_mask) | ((uint32_t)sh->bin << shift);
+        uint32_t mask = hi_mask | ((uint32_t)(kWide - 1) << shift);
+        uint32_t Krem = (uint32_t)K - sh->above;
+        const uint32_t in_bin = wide[sh->bin];
+        __syncthreads();
+        if (shift > 0) {
+            // the keys of T*'s bin into a small buffer (any order), unless too many
+            const bool small = in_bin <= (uint32_t)kSmall;
+            if (small) {
+                if (threadIdx.x == 0) sh->total = 0;
+                __syncthreads();
+                for (uint32_t jb = threadIdx.x & ~31u; jb < m; jb += NT) {
+                    const uint32_t j = jb + lane;
+                    uint32_t k = 0u;
+                    const bool take = j < m && is_key(j, k) && (k & mask) == prefix;
+                    const uint32_t bits = __ballot_sync(0xffffffffu, take);
+                    uint32_t at = 0;
+                    if (lane == 0 && bits) at = atomicAdd(&sh->total, (uint32_t)__popc(bits));
+                    at = __shfl_sync(0xffffffffu, at, 0);
+                    if (take) bin_keys[at + __popc(bits & lt)] = k;
+                }
+                __syncthreads();
+            }
+            if (small && in_bin <= 32u) {
+                // a handful of keys: one warp ranks them; T* is the key with
+                // fewer than Krem keys above it and at least Krem at or above
+                if (warp == 0) {
+                    const bool valid = (uint32_t)lane < in_bin;
+                    const uint32_t mine = valid ? bin_keys[lane] : 0u;
+                    uint32_t gt = 0, ge = 0;
+                    for (uint32_t q = 0; q < in_bin; ++q) {
+                        const uint32_t o = __shfl_sync(0xffffffffu, mine, q);
+                        gt += o > mine;
+                        ge += o >= mine;
+                    }
+                    const uint32_t hit = __ballot_sync(0xffffffffu, valid && gt < Krem && Krem <= ge);
+                    const int src = hit ? __ffs(hit) - 1 : 0;
+                    const uint32_t t_key = __shfl_sync(0xffffffffu, mine, src);
+                    const uint32_t t_gt = __shfl_sync(0xffffffffu, gt, src);
+                    if (lane == 0) {
+                        sh->base = t_key;
+                        sh->above = t_gt;
+                    }
+                }
+                __syncthreads();
+                prefix = sh->base;
+                Krem -= sh->above;
+                __syncthreads();
+            } else
+            // the remaining bits, 11 at a time, over the bin's keys
+            for (int sh2 = shift; sh2 > 0;) {
+                const int w = sh2 > 11 ? 11 : sh2;
+                sh2 -= w;
+                const int nb = 1 << w;
+                for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+                __syncthreads();
+                if (small)
+                    list_digit_hist<NT>(sh->hist, in_bin, prefix, mask, sh2, (uint32_t)nb, [&](uint32_t j, uint32_t &k) {
+                        k = bin_keys[j];
+                        return true;
+                    });
+                else
+                    list_digit_hist<NT>(sh->hist, m, prefix, mask, sh2, (uint32_t)nb, is_key);
+                __syncthreads();
+                topk::find_threshold<NT>(sh, nb, Krem);
+                prefix |= (uint32_t)sh->bin << sh2;
+                mask |= (uint32_t)(nb - 1) << sh2;
+                Krem -= sh->above;
+                __syncthreads();
+            }
         }
         const uint32_t Tstar = prefix, ties = Krem;
         if (trace && threadIdx.x == 0) trace[9] = globaltimer_ns();
@@ -812,6 +939,7 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         for (int j = kr + threadIdx.x; j < K; j += NT) sel[j] = -1;
     }
     __syncthreads();
+    if (n > K && threadIdx.x == 0) mbar_inval(copied);
     if (c == 0) {
         int32_t *out = cp.tk.idx + (int64_t)r * K;
         for (int j = threadIdx.x; j < K; j += NT) out[j] = sel[j];
@@ -837,6 +965,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     if (trace && threadIdx.x == 0) {
         for (int i = 1; i < DSA_TRACE_MARKS; ++i) trace[i] = 0;
         trace[0] = globaltimer_ns();
+        trace[13] = clock64();
     }
 
     // ---- phase 1: key stream, sample, candidates
@@ -854,7 +983,8 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     for (int r = 0; r < cp.rows; ++r) {
         const int64_t n = (int64_t)__ldg(cp.ix.q_pos + r) + 1;
         const uint32_t m = __ldcg(ctl + kTotal + r);
-        if (n > cp.K && (m < (uint32_t)cp.K || m > (uint32_t)kListCap)) fast = false;
+        // the list in shared memory holds the candidates and up to one pad per segment
+        if (n > cp.K && (m < (uint32_t)cp.K || m + (uint32_t)cp.NG > (uint32_t)kListCap)) fast = false;
     }
     if (blockIdx.x == 0 && threadIdx.x < kMaxRows + 1) {   // read by nobody after phase 1
         if (threadIdx.x == 0) {
@@ -949,6 +1079,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     // ---- the last CTA out resets the words read by everyone after phase 1
     __syncthreads();
     mark(6);
+    if (trace && threadIdx.x == 0) trace[14] = clock64();
     if (threadIdx.x == 0) {
         __threadfence();
         if (atomicAdd(ctl + kGridExit, 1u) == G - 1) {
@@ -1000,8 +1131,8 @@ int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
     // the shared-memory layouts must fit: phase 1 with at least 3 stages, phase 2's list and attention teams
     if (Layout(3, T, B).total + 1024 > capture_smem_budget()) return DSA_OK;
     const size_t ng = (size_t)grid * kGroups;
-    const size_t fast2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 +
-                                                  (size_t)2 * kListCap * 4,
+    const size_t fast2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 + 16 +
+                                                  (size_t)2 * kListCap * 4 + (size_t)(kWide + kSmall) * 4,
                                               kTeams * align128(sizeof(attn::Smem)));
     if (fast2 + 1024 > capture_smem_budget()) return DSA_OK;
     plan->grid = grid;
@@ -1035,8 +1166,8 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     while (S > 2 && Layout(S, ia.T, ia.B).total + 1024 > budget) --S;
     const size_t smem1 = Layout(S, ia.T, ia.B).total + 1024;
     const size_t ng = (size_t)plan.grid * kGroups;
-    const size_t smem2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 +
-                                                  (size_t)2 * kListCap * 4,
+    const size_t smem2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 + 16 +
+                                                  (size_t)2 * kListCap * 4 + (size_t)(kWide + kSmall) * 4,
                                               kTeams * align128(sizeof(attn::Smem))) +
                          1024;
     const size_t top_fixed = align128(sizeof(topk::Shared<kThreads>));
@@ -1047,6 +1178,7 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     cp.ix = L.p;
     cp.ix.stages = S;
     cp.ix.groups = indexer::kMaxGroups;
+    cp.ix.acc_bufs = indexer::kAccBufs;   // 2 pipes * 2 groups * 2 * 16T <= 512 columns for T <= 4
     cp.ix.hist_rows = 0;
     cp.ix.q_resident = 1;
     cp.at = attn::make_params(aa);

@@ -223,6 +223,28 @@ __device__ __forceinline__ void tma_load_1d_hint(void *smem_dst, const CUtensorM
         : "memory");
 }
 
+// Bulk (TMA engine, untiled) copy of `bytes` from global to shared memory,
+// completing on `bar` (complete_tx); both addresses 16-byte aligned and bytes
+// a multiple of 16.  The barrier's transaction count must cover it
+// (mbar_expect_tx or mbar_arrive_expect_tx) before its phase can complete.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Raises the barrier's expected transaction bytes without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Orders this thread's earlier shared-memory accesses (generic proxy) before
+// later bulk copies (async proxy) into the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -306,13 +328,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 
 // ------------------------------------------------------------------ misc
-// Warp-level histogram increment: lanes with `active` add 1 to hist[bin],
-// with one shared-memory atomic per distinct bin of the warp.  Keys that
-// agree on a digit (a narrow score range, a radix pass below a common prefix)
-// would otherwise serialise on one address, one atomic per key.  When every
-// active lane has the same bin one atomic adds them all; otherwise the lanes
-// of each bin find one another with match.any and their first lane adds.
-// All 32 lanes must call it.
+// Warp-level histogram increment: lanes with `active` add 1 to hist[bin].
+// When every active lane has the same bin (keys that agree on a digit: a
+// narrow score range, a radix pass below a common prefix) one atomic adds them
+// all; otherwise each lane adds its own (grouping the lanes by bin with
+// match.any measured slower for spread bins).  All 32 lanes must call it.
 __device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool active) {
     const uint32_t amask = __ballot_sync(0xffffffffu, active);
     if (amask == 0) return;
@@ -321,8 +341,7 @@ __device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool
     if (bmin == bmax) {
         if ((threadIdx.x & 31) == (uint32_t)(__ffs(amask) - 1)) atomicAdd(&hist[bmin], (uint32_t)__popc(amask));
     } else if (active) {
-        const uint32_t peers = __match_any_sync(amask, bin);
-        if ((threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+        atomicAdd(&hist[bin], 1u);
     }
 }
 
@@ -344,6 +363,15 @@ __device__ __forceinline__ void list_digit_hist(uint32_t *hist, uint32_t m, uint
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// A relaxed load (no ordering): for polling a flag; follow a hit with
+// fence_acq_rel_gpu() before reading what the flag publishes.
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
     uint32_t v;

@@ -41,6 +41,8 @@ constexpr int kEpiWarps = 4;              // warps per epilogue group (one per T
 constexpr int kEpiWarp0 = 2 * kPipes;     // first epilogue warp
 constexpr int kThreads = 32 * (kEpiWarp0 + kPipes * kMaxGroups * kEpiWarps);   // 640
 constexpr int kMaxStages = 8;             // per pipeline
+constexpr int kAccBufs = 2;               // at most this many TMEM accumulators per epilogue group (two: the
+                                          // MMA of a group's next tile runs while its epilogue reads this one)
 constexpr int kKsStageBytes = 1024;       // key-scale slots of one stage
 // Score histogram for the selection: bits 30..20 of the order key of each
 // non-negative score (2048 bins, eight per octave), and one bin (2048) that
@@ -71,6 +73,7 @@ struct Params {
     int stages;          // per pipeline
     int rows_per_load;   // R: rows per TMA box (128, or the page size when pages are smaller)
     int groups;          // epilogue groups per pipeline (1..kMaxGroups)
+    int acc_bufs;        // TMEM accumulators per group (1..kAccBufs); kPipes * groups * acc_bufs * 16T <= 512
     // optional histogram of the visible scores (see kHistWords), added into
     // hist_global[row * hist_row_words + bin] for rows b * T + t < hist_rows;
     // hist_rows == 0 turns it off
@@ -85,8 +88,8 @@ struct Params {
 struct __align__(8) Bars {
     uint64_t full[kPipes][kMaxStages];
     uint64_t empty[kPipes][kMaxStages];
-    uint64_t tfull[kPipes][kMaxGroups];
-    uint64_t tempty[kPipes][kMaxGroups];
+    uint64_t tfull[kPipes][kMaxGroups][kAccBufs];
+    uint64_t tempty[kPipes][kMaxGroups][kAccBufs];
     uint64_t mma_done[kPipes];
     uint64_t q_full;
 };
@@ -136,7 +139,7 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
                                             const CUtensorMap *tmap_q_p, const Params &p, uint8_t *smem, int cta,
                                             int ncta) {
     const CUtensorMap &tmap_k = *tmap_k_p, &tmap_ks = *tmap_ks_p, &tmap_q = *tmap_q_p;
-    const int S = p.stages, T = p.T, B = p.B, N = 16 * T, GE = p.groups;
+    const int S = p.stages, T = p.T, B = p.B, N = 16 * T, GE = p.groups, AB = p.acc_bufs;
     Layout lay(S, T, B, p.hist_rows, p.q_resident != 0);
     Bars *bars = reinterpret_cast<Bars *>(smem + lay.bar_off);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.tmem_off);
@@ -196,17 +199,18 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
 
     // --- barriers and TMEM (GE accumulators of N columns per pipeline)
     uint32_t tmem_cols = 32;
-    while (tmem_cols < (uint32_t)(kPipes * GE * N)) tmem_cols <<= 1;
+    while (tmem_cols < (uint32_t)(kPipes * GE * AB * N)) tmem_cols <<= 1;
     if (threadIdx.x == 0) {
         for (int pp = 0; pp < kPipes; ++pp) {
             for (int s = 0; s < S; ++s) {
                 mbar_init(&bars->full[pp][s], 1);
                 mbar_init(&bars->empty[pp][s], 1 + kEpiWarps);
             }
-            for (int a = 0; a < GE; ++a) {
-                mbar_init(&bars->tfull[pp][a], 1);
-                mbar_init(&bars->tempty[pp][a], kEpiWarps);
-            }
+            for (int a = 0; a < GE; ++a)
+                for (int u = 0; u < AB; ++u) {
+                    mbar_init(&bars->tfull[pp][a][u], 1);
+                    mbar_init(&bars->tempty[pp][a][u], kEpiWarps);
+                }
             mbar_init(&bars->mma_done[pp], 1);
         }
         mbar_init(&bars->q_full, 1);
@@ -293,19 +297,20 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
             const uint32_t idesc = umma_idesc_e4m3_f32(kTile, N);
             for (int i = 0; i < n_p; ++i) {
                 const int s = i % S, st = stage_of(pp, s), a = i % GE;
+                const int jj = i / GE, u = jj % AB;   // the group's jj-th tile, its accumulator
                 if (!mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status)) break;
-                if (i >= GE && !mbar_wait(&bars->tempty[pp][a], ((i / GE) & 1) ^ 1, p.status)) break;
+                if (jj >= AB && !mbar_wait(&bars->tempty[pp][a][u], ((jj / AB) & 1) ^ 1, p.status)) break;
                 if (i == 0 && p.q_resident && !mbar_wait(&bars->q_full, 0, p.status)) break;
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(smem + lay.k_off + st * kTile * kKeyBytes);
                 const uint32_t b_addr = smem_u32(smem + lay.q_off + (p.q_resident ? 0 : st * N * kKeyBytes));
-                const uint32_t d = tmem_base + (uint32_t)((pp * GE + a) * N);
+                const uint32_t d = tmem_base + (uint32_t)(((pp * GE + a) * AB + u) * N);
 #pragma unroll
                 for (int k = 0; k < kKeyBytes / 32; ++k)
                     umma_f8(d, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
                             k > 0 ? 1u : 0u);
                 umma_commit(&bars->empty[pp][s]);
-                umma_commit(&bars->tfull[pp][a]);
+                umma_commit(&bars->tfull[pp][a][u]);
             }
             umma_commit(&bars->mma_done[pp]);
             mbar_wait(&bars->mma_done[pp], 0, p.status);
@@ -320,7 +325,7 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
         const int n_p = pipe_count(pp), g0 = pipe_begin(pp);
         float *coef = reinterpret_cast<float *>(smem + lay.epi_off) + ew * (17 * T);
         int32_t *qp = reinterpret_cast<int32_t *>(coef + 16 * T);
-        const uint32_t acc_col = (uint32_t)((pp * GE + a) * N);
+        const uint32_t acc_col0 = (uint32_t)((pp * GE + a) * AB * N);
         int cur_b = -1;
         for (int i = a; i < n_p && a < GE; i += GE) {
             const int s = i % S, st = stage_of(pp, s);
@@ -334,7 +339,9 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
                 __syncwarp();
                 cur_b = b;
             }
-            bool ok = mbar_wait(&bars->tfull[pp][a], (i / GE) & 1, p.status) &&
+            const int jj = i / GE, u = jj % AB;
+            const uint32_t acc_col = acc_col0 + (uint32_t)(u * N);
+            bool ok = mbar_wait(&bars->tfull[pp][a][u], (jj / AB) & 1, p.status) &&
                       mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
@@ -360,7 +367,7 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bars->tempty[pp][a]);
+                mbar_arrive(&bars->tempty[pp][a][u]);
                 mbar_arrive(&bars->empty[pp][s]);
             }
         }
@@ -379,10 +386,11 @@ __device__ __forceinline__ void run_indexer(const CUtensorMap *tmap_k_p, const C
                 mbar_inval(&bars->full[pp][s]);
                 mbar_inval(&bars->empty[pp][s]);
             }
-            for (int a = 0; a < GE; ++a) {
-                mbar_inval(&bars->tfull[pp][a]);
-                mbar_inval(&bars->tempty[pp][a]);
-            }
+            for (int a = 0; a < GE; ++a)
+                for (int u = 0; u < AB; ++u) {
+                    mbar_inval(&bars->tfull[pp][a][u]);
+                    mbar_inval(&bars->tempty[pp][a][u]);
+                }
             mbar_inval(&bars->mma_done[pp]);
         }
         mbar_inval(&bars->q_full);
