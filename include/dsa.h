@@ -185,12 +185,13 @@ int dsa_debug_inject(int kind, int64_t wait_limit_ns);
  * grid of at most words / DSA_TRACE_MARKS CTAs writes, per CTA c, the GPU's
  * nanosecond clock (%globaltimer) into buf[c * DSA_TRACE_MARKS + i]:
  *   i = 0 entry, 1 the sampled thresholds seen, 2 the key stream done (the
- *   CTA's tiles scored and captured), 3 past the grid barrier, 4 the
+ *   CTA's tiles scored), 3 past the grid barrier, 4 the
  *   selection done, 5 the attention units done, 6 exit, 7 the CTA's sample
  *   handed in, 8 the candidate list in shared memory, 9 the k-th key found
  *   (radix select done), 10 the first key tile requested, 11 its MMA issued,
  *   12 its scores in the epilogue; 13 and 14 the SM's cycle counter
- *   (clock64) at entry and at exit, for the clock rate; 15 unused.
+ *   (clock64) at entry and at exit, for the clock rate; 15 the CTA's
+ *   candidates captured (after its tiles, from their stored scores).
  * Marks a CTA does not reach (a CTA with no selection or attention work, the
  * general path) are written as 0.  `buf` is device memory of the caller's,
  * `words` its length in uint64 words; a launch with a grid too large for it

@@ -147,8 +147,14 @@ __device__ __forceinline__ bool key_row(const Params &p, int b, int64_t pos, int
 // memory (sm.tm, sm.tl, the first 16 x 128 floats of sm.k) for cta_merge.
 // sel_smem: the query's selection (-1 padded, the p.padded layout) already
 // in shared memory, read instead of p.idx.
+// direct: a single-team unit (p.n_teams == 1) writes its result itself --
+// the partial, or with one split the output -- with the arithmetic cta_merge
+// would apply to it (a one-team merge multiplies by 2^0 = 1 and adds to 0:
+// the same values), instead of leaving it in shared memory.
 __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, int g, int bt, int tid, int bar,
-                                          const int32_t *sel_smem = nullptr) {
+                                          const int32_t *sel_smem = nullptr, bool direct = false,
+                                          const float *sink = nullptr, __nv_bfloat16 *O = nullptr,
+                                          float *lse = nullptr) {
     const int b = bt / p.T;
     const int hpg = DSA_Q_HEADS / p.G;
     const int warp = tid >> 5, lane = tid & 31;
@@ -345,6 +351,39 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
             }
         }
     }
+    if (direct) {
+        if (row < hpg) {
+            const int64_t gw = (int64_t)bt * DSA_Q_HEADS + g * hpg + row;
+            if (p.splits == 1) {
+                const float sk = sink ? __ldg(sink + g * hpg + row) * kLog2e : -INFINITY;
+                const float M2 = fmaxf(M, sk);
+                float den = 0.f, w = 0.f;
+                if (M2 != -INFINITY) {
+                    w = (M == -INFINITY) ? 0.f : exp2f(M - M2);
+                    den = L * w + (sink ? exp2f(sk - M2) : 0.f);
+                }
+                const float f = den > 0.f ? w / den : 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    __nv_bfloat16 *o = O + gw * DSA_V_DIM + c0 + 32 * c;
+                    o[0] = __float2bfloat16_rn(acc[c].x * f);
+                    o[1] = __float2bfloat16_rn(acc[c].y * f);
+                    o[2] = __float2bfloat16_rn(acc[c].z * f);
+                    o[3] = __float2bfloat16_rn(acc[c].w * f);
+                }
+                if (lse && (tid & 7) == 0) lse[gw] = den > 0.f ? (M2 + log2f(den)) / kLog2e : -INFINITY;
+            } else {
+                float *po = p.part_o + (gw * p.splits + chunk) * DSA_V_DIM;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) *reinterpret_cast<float4 *>(po + c0 + 32 * c) = acc[c];
+                if ((tid & 7) == 0) {
+                    p.part_ml[(gw * p.splits + chunk) * 2 + 0] = M;
+                    p.part_ml[(gw * p.splits + chunk) * 2 + 1] = L;
+                }
+            }
+        }
+        return;
+    }
     team_sync(bar);
     if (row < hpg) {
 #pragma unroll
@@ -428,17 +467,17 @@ __device__ __forceinline__ void cta_unit(const Params &p, const TeamSmem &teams,
 }
 
 // One unit taken by a single team (p.n_teams == 1): chunk `split` of query bt
-// and KV head g, then the unit's partial (with one split: the output) written
-// by the same 128 threads, which synchronise on the named barrier `bar` only.
-// The teams of a CTA can so work on different units at once.
+// and KV head g, its partial (with one split: the output) written by the same
+// 128 threads, which synchronise on the named barrier `bar` only, so that the
+// teams of a CTA can work on different units at once.  On return the team's
+// stores are done and, with several splits, released by thread 0 (tid 0): a
+// flag that thread 0 then sets publishes the partial.
 __device__ __forceinline__ void team_unit(const Params &p, Smem &sm, int split, int g, int bt, int tid, int bar,
                                           const float *sink, __nv_bfloat16 *O, float *lse,
                                           const int32_t *sel_smem = nullptr) {
-    attn_unit(p, sm, split, g, bt, tid, bar, sel_smem);
-    team_sync(bar);
-    cta_merge(p, TeamSmem{reinterpret_cast<uint8_t *>(&sm), 0u}, split, g, bt, tid, sink, O, lse);
-    if (p.splits > 1) __threadfence();   // the partial is visible before any later signal of this team
-    team_sync(bar);
+    attn_unit(p, sm, split, g, bt, tid, bar, sel_smem, true, sink, O, lse);
+    team_sync(bar);   // every thread's stores are done ...
+    if (p.splits > 1 && tid == 0) __threadfence();   // ... and released, before thread 0 signals anything
 }
 
 // Merge of the splits of one (query, head) row gw by a whole CTA of NT

@@ -10,33 +10,33 @@
 // work that depends on every score is cut down to a short list that the key
 // stream itself produces.
 //
-// Phase 1, the key stream (one CTA per SM, two TMA -> tcgen05 pipelines, four
-// epilogue groups of four warps; indexer_impl.cuh has the machinery).  Each
-// epilogue group owns a contiguous range of key tiles, so that its output is
-// in position order:
-//   * its first tile is a sample: the scores' 8-bins-per-octave histogram
-//     goes into the CTA's shared histogram; when all four groups of a CTA have
-//     added theirs, one of them adds the CTA's histogram into the row's global
-//     one; the last CTA to do so turns each row's sample histogram into a
-//     score threshold -- a bin edge below which the sample predicts about
-//     `oversample` x top_k keys -- and publishes it;
-//   * every tile: keys with score >= threshold are appended, with their
-//     positions, to the group's segment of the row's candidate list, in
-//     position order (a ballot per warp, an exchange of counts among the
-//     group's four warps per tile).  Every score is also stored, as the
-//     standalone indexer stores it (the fallback below reads them).
+// Phase 1, the key stream (one CTA per SM, two TMA -> tcgen05 pipelines with
+// two TMEM accumulators per epilogue group, four epilogue groups of four
+// warps; indexer_impl.cuh has the machinery).  The epilogue scores and
+// stores as the standalone indexer does; besides, each group's first tile is
+// a sample: its 8-bins-per-octave histogram goes into the CTA's shared
+// histogram, the CTA's last group adds it into the row's global one, and the
+// last CTA to do so turns each row's histogram into a score threshold -- a
+// bin edge below which the sample predicts about `oversample` x top_k keys --
+// and publishes it.  When its tiles are done, a CTA takes its candidates from
+// its own stored scores (in L2): every visible key at or above the threshold,
+// with its position, in position order, into the CTA's segment of the row's
+// candidate list.
 // One grid barrier.  The segments' lengths tell whether the sample was good:
 // if every row holds at least top_k candidates (then the list holds every key
 // at or above the k-th largest score, since the threshold is below it) and no
 // segment overflowed, the fast path runs; otherwise the general path of the
 // fused layer-step does (the result is the same either way).
-// Phase 2 (fast), per CTA of a row: the row's candidates (a few thousand)
-// into shared memory in position order, an exact 11/11/10-bit radix select on
-// them, the selection compacted in position order into shared memory.  Its
-// attention units read the selection from there; the last unit of each KV
-// group of a row (a counter per group) combines that group's heads with the
-// sink, with the same arithmetic as the combine kernel.
+// Phase 2 (fast), per CTA of a row that has attention units: the row's
+// candidates (a few thousand) into shared memory in position order (one bulk
+// copy per segment), the exact k-th largest key (one wide histogram of the
+// bits below the keys' common ones, then the few keys of its bin), the
+// selection compacted in position order into shared memory.  Each team of the
+// CTA then runs a 64-key attention unit from there, and once every unit of
+// its (row, KV group) has written its partial, combines one slice of that
+// group's outputs with the sink, with the combine kernel's arithmetic.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "attention_impl.cuh"
@@ -62,7 +62,7 @@ constexpr int kGroups = kPipes * kMaxGroups;  // epilogue groups per CTA
 constexpr int kBins = 2048;                   // sample histogram: bits 30..20 of the non-negative keys
 constexpr int kHistWords = kBins + 1;         // + the count of negative scores
 constexpr int kHistStride = kHistWords + 3;   // words between rows' histograms: rows start 16-byte aligned
-constexpr int kSegCap = 1024;                 // candidates one epilogue group may hold per row
+constexpr int kSegCap = 1024;                 // candidates one CTA may hold per row
 constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
 constexpr int kWide = 4096;                   // bins of the selection's first histogram
 constexpr int kSmall = 2048;                  // keys of T*'s bin taken aside for the remaining bits
@@ -111,7 +111,7 @@ __host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~si
 
 // Shared memory of phase 1 (base aligned to 1024 bytes).
 struct Layout {
-    uint32_t k_off, q_off, ks_off, bar_off, tmem_off, len_off, tile_off, epi_off, hist_off, xch_off, misc_off, total;
+    uint32_t k_off, q_off, ks_off, bar_off, tmem_off, len_off, tile_off, epi_off, hist_off, misc_off, total;
     __host__ __device__ Layout(int S, int T, int B) {
         const int stages = kPipes * S, rows = B * T;
         k_off = 0;
@@ -123,9 +123,9 @@ struct Layout {
         tile_off = (len_off + 4 * (B + 1) + 15) & ~15u;
         epi_off = (tile_off + 4 * (B + 1) + 15) & ~15u;
         hist_off = epi_off + kGroups * kEpiWarps * (16 * T + T) * 4;
-        xch_off = hist_off + rows * kHistStride * 4;
-        misc_off = xch_off + kGroups * 2 * (kEpiWarps * kMaxRows + 1) * 4;
-        total = misc_off + 32;   // [0] groups sampled, [1 + g] group g's role in the sample exchange
+        misc_off = hist_off + rows * kHistStride * 4;
+        total = misc_off + 32 + 16;   // misc: [0] groups sampled, [1 + g] group g's role in the sample
+                                      // exchange; then the rows' query positions
     }
 };
 
@@ -196,12 +196,17 @@ __device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversa
 // Phase 1: the indexer over this CTA's tiles with sampling and candidate
 // capture (see the file comment).  All kThreads threads call it.  On return
 // nothing is in flight, TMEM is released and the mbarriers are invalidated.
+template <int TQ>
 __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorMap *tmap_ks_p,
                                     const CUtensorMap *tmap_q_p, const Params &cp, uint8_t *smem, int cta, int ncta) {
     using namespace indexer;
     const indexer::Params &p = cp.ix;
     const CUtensorMap &tmap_k = *tmap_k_p, &tmap_ks = *tmap_ks_p, &tmap_q = *tmap_q_p;
-    const int S = p.stages, T = p.T, B = p.B, N = 16 * T, GE = p.groups, AB = p.acc_bufs, rows = B * T;
+    // the query tokens per sequence are a compile-time constant: the per-query
+    // loops of the epilogue keep only the copies that run (a smaller loop body
+    // that stays in the instruction cache)
+    constexpr int T = TQ;
+    const int S = p.stages, B = p.B, N = 16 * T, GE = p.groups, AB = p.acc_bufs, rows = B * T;
     Layout lay(S, T, B);
     Bars *bars = reinterpret_cast<Bars *>(smem + lay.bar_off);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.tmem_off);
@@ -209,6 +214,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     int32_t *tile_pre = reinterpret_cast<int32_t *>(smem + lay.tile_off);
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [rows][kHistStride]
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags
+    int32_t *row_qpos = reinterpret_cast<int32_t *>(smem + lay.misc_off + 32);   // [rows] query positions
     uint32_t *ctl = cp.ctl;
     const int warp = warp_id(), lane = lane_id();
 
@@ -229,6 +235,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     }
     for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
     if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+    if (threadIdx.x < rows) row_qpos[threadIdx.x] = __ldg(p.q_pos + threadIdx.x);
     __syncthreads();
     if (warp == 0) {
         int carry = 0;
@@ -377,124 +384,23 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Scores only, as the standalone indexer: the candidates are taken
+        // from the stored scores after the stream, CTA by CTA.  The group's
+        // first tile is also the sample for the thresholds.
         const int ew = warp - kEpiWarp0;
         const int pp = ew / (kMaxGroups * kEpiWarps);
         const int a = (ew / kEpiWarps) % kMaxGroups;
         const int quarter = warp & 3;
-        const int gi = pp * kMaxGroups + a;          // group index: groups are in position order
-        const int gid = cta * kGroups + gi;          // the group's segment in every row's list
+        const int gi = pp * kMaxGroups + a;
         const int gbar = kGroupBar0 + gi;
         const int row_in_tile = quarter * 32 + lane;
         const int ng = a < GE ? group_count(pp, a) : 0;
-        const uint32_t lt = (1u << lane) - 1u;
         float *coef = reinterpret_cast<float *>(smem + lay.epi_off) + ew * (17 * T);
         int32_t *qp = reinterpret_cast<int32_t *>(coef + 16 * T);
-        // per group, twice (double-buffered): the four warps' candidate counts per query, the readiness poll
-        uint32_t *xch = reinterpret_cast<uint32_t *>(smem + lay.xch_off) + gi * (2 * (kEpiWarps * kMaxRows + 1));
         const uint32_t acc_col0 = (uint32_t)((pp * GE + a) * AB * N);
-        uint32_t base[kMaxRows] = {0u, 0u, 0u, 0u};
-        uint32_t thr[kMaxRows] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-        bool ok = true, overflow = false, known = false;
-        int cur_b = -1;
-        int pending = 0;   // the group's tiles 0 .. pending - 1 were scored before the thresholds were known
-        int slot = 0;      // half of the double-buffered exchange words that the next group barrier uses
         const bool poller = quarter == 0 && lane == 0;
-
-        // The candidates of one tile to the group's segments, in position
-        // order: bit t of cbits says whether this thread's key is a candidate
-        // for query t of sequence b.  One group barrier exchanges the four
-        // warps' counts, and carries `okin` (AND over the group, returned) and
-        // the poller's `poll` (the thresholds' readiness, into *seen).
-        auto capture_tile = [&](int b, int64_t pos, const float (&sc)[kMaxRows], uint32_t cbits, bool okin,
-                                uint32_t poll, bool *seen) -> bool {
-            uint32_t *c = xch + slot * (kEpiWarps * kMaxRows + 1);
-            uint32_t cm[kMaxRows] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int t = 0; t < kMaxRows; ++t) {
-                if (t < T) {
-                    cm[t] = __ballot_sync(0xffffffffu, (cbits >> t) & 1u);
-                    if (lane == 0) c[quarter * kMaxRows + t] = __popc(cm[t]);
-                }
-            }
-            if (poller) c[kEpiWarps * kMaxRows] = poll;
-            const bool g_ok = named_bar_and(gbar, 128, okin);
-            *seen = c[kEpiWarps * kMaxRows] != 0u;
-            if (g_ok) {
-#pragma unroll
-                for (int t = 0; t < kMaxRows; ++t) {
-                    if (t < T) {
-                        uint32_t below = 0, tot = 0;
-#pragma unroll
-                        for (int q = 0; q < kEpiWarps; ++q) {
-                            const uint32_t v = c[q * kMaxRows + t];
-                            tot += v;
-                            if (q < quarter) below += v;
-                        }
-                        const int r = b * T + t;
-                        uint32_t bs = 0;
-#pragma unroll
-                        for (int rr = 0; rr < kMaxRows; ++rr)
-                            if (rr == r) bs = base[rr];
-                        if ((cm[t] >> lane) & 1u) {
-                            const uint32_t at = bs + below + __popc(cm[t] & lt);
-                            if (at < (uint32_t)kSegCap)
-                                cp.lists[((int64_t)r * cp.NG + gid) * kSegCap + at] =
-                                    make_uint2(float_order_key(sc[t]), (uint32_t)pos);
-                            else
-                                overflow = true;
-                        }
-#pragma unroll
-                        for (int rr = 0; rr < kMaxRows; ++rr)
-                            if (rr == r) base[rr] += tot;
-                    }
-                }
-            }
-            slot ^= 1;
-            return g_ok;
-        };
-        // Candidate bits of this thread's key for the queries of sequence b.
-        auto cand_bits = [&](int b, uint32_t vis, const float (&sc)[kMaxRows]) {
-            uint32_t bits = 0;
-#pragma unroll
-            for (int t = 0; t < kMaxRows; ++t) {
-                if (t < T) {
-                    uint32_t th = 0xFFFFFFFFu;
-#pragma unroll
-                    for (int r = 0; r < kMaxRows; ++r)
-                        if (r == b * T + t) th = thr[r];
-                    if (((vis >> t) & 1u) && float_order_key(sc[t]) >= th) bits |= 1u << t;
-                }
-            }
-            return bits;
-        };
-        // The thresholds are known: load them, then capture the pending
-        // tiles from their stored scores (this thread's own stores).
-        auto become_known = [&]() {
-            known = true;
-            if (poller && cp.trace && gi == 0) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
-#pragma unroll
-            for (int r = 0; r < kMaxRows; ++r)
-                if (r < rows) thr[r] = __ldcg(ctl + kThr + r);
-            for (int jj = 0; jj < pending && ok; ++jj) {
-                int bb, ti;
-                locate(tile_of(pp, jj * GE + a), bb, ti);
-                const int64_t ps = (int64_t)ti * kTile + row_in_tile;
-                const int len = seq_len[bb];
-                float s2[kMaxRows] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t v2 = 0;
-#pragma unroll
-                for (int t = 0; t < kMaxRows; ++t) {
-                    if (t < T && ps < len && ps <= (int64_t)__ldg(p.q_pos + bb * T + t)) {
-                        s2[t] = __ldcg(p.scores + ((int64_t)bb * T + t) * p.scores_stride + ps);
-                        v2 |= 1u << t;
-                    }
-                }
-                bool unused;
-                ok = capture_tile(bb, ps, s2, cand_bits(bb, v2, s2), ok, 0u, &unused);
-            }
-            pending = 0;
-        };
-
+        bool ok = true;
+        int cur_b = -1;
         for (int j = 0; j < ng || j == 0; ++j) {
             const bool have = j < ng;
             float sc[kMaxRows] = {0.f, 0.f, 0.f, 0.f};
@@ -571,15 +477,14 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                     const int tid = quarter * 32 + lane;
                     for (int u = tid; u < rows * kHistStride; u += 128)
                         if (hist[u]) atomicAdd(cp.sample_hist + u, hist[u]);
-                    __threadfence();
-                    named_bar_sync(gbar, 128);
+                    named_bar_sync(gbar, 128);   // the group's adds, before its poller's release below
                     if (quarter == 0 && lane == 0) {
-                        *flag = atomicAdd(ctl + kSampleArrive, 1u) == (uint32_t)ncta - 1 ? 2u : 1u;
+                        // releases this CTA's adds; the last arrival acquires every CTA's
+                        *flag = atom_add_acq_rel_gpu(ctl + kSampleArrive, 1u) == (uint32_t)ncta - 1 ? 2u : 1u;
                         if (cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 7] = globaltimer_ns();
                     }
                     named_bar_sync(gbar, 128);
                     if (*flag == 2u) {   // the last CTA: one warp per row
-                        __threadfence();
                         if (quarter < rows) {
                             const int r = quarter;
                             const int64_t n = (int64_t)__ldg(p.q_pos + r) + 1;
@@ -592,46 +497,12 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             }
                             if (lane == 0) ctl[kThr + r] = t_r;
                         }
-                        __threadfence();
-                        named_bar_sync(gbar, 128);
+                        named_bar_sync(gbar, 128);   // the thresholds, before the release that publishes them
                         if (quarter == 0 && lane == 0) {
-                            ctl[kSampleArrive] = 0;
-                            __threadfence();
-                            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ctl + kReady), "r"(1u) : "memory");
+                            ctl[kSampleArrive] = 0;   // read by nobody until the next call
+                            st_release_gpu(ctl + kReady, 1u);
                         }
                     }
-                }
-            }
-            // ---- this tile's candidates (deferred while the thresholds are unknown)
-            uint32_t poll = 0;
-            if (!known && poller && ld_relaxed_gpu(ctl + kReady) >= 1u) {
-                fence_acq_rel_gpu();   // the thresholds the flag publishes, before the group reads them
-                poll = 1u;
-            }
-            const bool was_known = known;
-            bool seen = false;
-            ok = capture_tile(b, pos, sc, (was_known && have && ok) ? cand_bits(b, vis, sc) : 0u, ok, poll, &seen);
-            if (!ok) break;
-            if (!was_known) {
-                if (have) pending = j + 1;
-                if (seen) become_known();
-                if (!ok) break;
-            }
-        }
-        // a short stream: the thresholds may come after the group's last tile
-        if (ok && !known) {
-            bool r_ok = true;
-            if (poller) r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
-            ok = named_bar_and(gbar, 128, r_ok);
-            if (ok) become_known();
-        }
-        if (__any_sync(0xffffffffu, overflow) && lane == 0) atomicOr(ctl + kOverflow, 1u);
-        if (quarter == 0 && lane == 0) {
-#pragma unroll
-            for (int r = 0; r < kMaxRows; ++r) {
-                if (r < rows) {
-                    cp.counts[(int64_t)r * cp.NG + gid] = base[r];
-                    if (base[r]) atomicAdd(ctl + kTotal + r, base[r]);
                 }
             }
         }
@@ -661,6 +532,144 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         mbar_inval(&bars->q_full);
     }
     __syncthreads();
+    if (cp.trace && threadIdx.x == 0) cp.trace[cta * DSA_TRACE_MARKS + 2] = globaltimer_ns();
+
+    // ---- the CTA's candidates: every visible key of its tiles whose score
+    //      is at or above its row's threshold, in position order, into the
+    //      CTA's segment of the row's list (the scores are this CTA's own
+    //      stores, in L2).  Pair q = t * n_tiles + i is query t of tile i.
+    uint32_t *cnt = reinterpret_cast<uint32_t *>(smem);      // [P] candidates per pair
+    uint32_t *pref = cnt + kThreads;                          // [P] exclusive prefix of cnt
+    bool r_ok = true;
+    if (threadIdx.x == 0 && n_tiles > 0) r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
+    if (!__syncthreads_and(r_ok)) return;   // the timeout is in the status word; the grid barrier sees it
+    if (cp.trace && threadIdx.x == 0) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
+    uint32_t thr[kMaxRows];
+#pragma unroll
+    for (int r = 0; r < kMaxRows; ++r) thr[r] = r < rows ? __ldcg(ctl + kThr + r) : 0xFFFFFFFFu;
+    const int P = n_tiles * T;   // <= kThreads (plan_capture)
+    // Pairs are taken kQP per warp at a time with every score load in flight
+    // before the first ballot: lane l holds key 32 k + l of each pair's tile.
+    constexpr int kQP = 4;
+    static_assert(kTile / 32 == 4, "four 32-key strips per tile");
+    struct PairKeys {
+        uint32_t key[kQP][kTile / 32];
+        uint32_t cand;      // bit qq * 4 + k: key k of pair qq is a candidate
+        int r[kQP];
+        int64_t pos0[kQP];
+    };
+    auto load_pairs = [&](int q0, PairKeys &pk) {
+        pk.cand = 0;
+#pragma unroll
+        for (int qq = 0; qq < kQP; ++qq) {
+            const int q = q0 + qq * kWarps;
+            pk.r[qq] = 0;
+            pk.pos0[qq] = 0;
+#pragma unroll
+            for (int k = 0; k < kTile / 32; ++k) pk.key[qq][k] = 0u;
+            if (q < P) {
+                const int i = q % n_tiles, t = q / n_tiles;
+                int b, ti;
+                locate(t_begin + i, b, ti);
+                const int r = b * T + t;
+                pk.r[qq] = r;
+                pk.pos0[qq] = (int64_t)ti * kTile;
+                const int64_t lim = min((int64_t)seq_len[b] - 1, (int64_t)row_qpos[r]);   // last visible
+                const float *src = p.scores + (int64_t)r * p.scores_stride + pk.pos0[qq];
+#pragma unroll
+                for (int k = 0; k < kTile / 32; ++k) {
+                    const int64_t pos = pk.pos0[qq] + k * 32 + lane;
+                    if (pos <= lim) {
+                        pk.key[qq][k] = float_order_key(__ldcg(src + k * 32 + lane));
+                        pk.cand |= 1u << (qq * 4 + k);
+                    }
+                }
+            }
+        }
+        // visible -> candidate: at or above the row's threshold
+#pragma unroll
+        for (int qq = 0; qq < kQP; ++qq) {
+            uint32_t th = 0xFFFFFFFFu;
+#pragma unroll
+            for (int rr = 0; rr < kMaxRows; ++rr)
+                if (rr == pk.r[qq]) th = thr[rr];
+#pragma unroll
+            for (int k = 0; k < kTile / 32; ++k)
+                if (pk.key[qq][k] < th) pk.cand &= ~(1u << (qq * 4 + k));
+        }
+    };
+    const bool one_batch = P <= kWarps * kQP;   // then pass 2 reuses pass 1's keys
+    PairKeys kept;
+    for (int q0 = warp; q0 < P; q0 += kWarps * kQP) {
+        PairKeys pk;
+        load_pairs(q0, pk);
+        if (one_batch) kept = pk;
+#pragma unroll
+        for (int qq = 0; qq < kQP; ++qq) {
+            uint32_t c = 0;
+#pragma unroll
+            for (int k = 0; k < kTile / 32; ++k) c += __popc(__ballot_sync(0xffffffffu, (pk.cand >> (qq * 4 + k)) & 1u));
+            const int q = q0 + qq * kWarps;
+            if (lane == 0 && q < P) cnt[q] = c;
+        }
+    }
+    __syncthreads();
+    {
+        const uint32_t v = (int)threadIdx.x < P ? cnt[threadIdx.x] : 0u;
+        uint32_t total;
+        auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(pref + kThreads);
+        const uint32_t incl = topk::block_scan<kThreads>(v, sh->warp_tmp, &total);
+        if ((int)threadIdx.x < P) pref[threadIdx.x] = incl - v;
+    }
+    __syncthreads();
+    // the pairs of row r = b * T + t in this CTA: t * n_tiles + [i0, i1), the tiles of sequence b
+    auto row_span = [&](int r, int &q0, int &q1) {
+        const int b = r / T, t = r % T;
+        const int i0 = min(n_tiles, max(0, tile_pre[b] - t_begin));
+        const int i1 = min(n_tiles, max(0, tile_pre[b + 1] - t_begin));
+        q0 = t * n_tiles + i0;
+        q1 = t * n_tiles + i1;
+    };
+    bool overflow = false;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int q0 = warp; q0 < P; q0 += kWarps * kQP) {
+        PairKeys pk;
+        if (one_batch) pk = kept;
+        else load_pairs(q0, pk);   // again: the scores are in L2
+#pragma unroll
+        for (int qq = 0; qq < kQP; ++qq) {
+            const int q = q0 + qq * kWarps;
+            if (q < P) {   // warp-uniform
+                int rq0, rq1;
+                row_span(pk.r[qq], rq0, rq1);
+                uint32_t at = pref[q] - pref[rq0];
+#pragma unroll
+                for (int k = 0; k < kTile / 32; ++k) {
+                    const bool cand = (pk.cand >> (qq * 4 + k)) & 1u;
+                    const uint32_t bits = __ballot_sync(0xffffffffu, cand);
+                    if (cand) {
+                        const uint32_t slot = at + __popc(bits & lt);
+                        if (slot < (uint32_t)kSegCap)
+                            cp.lists[((int64_t)pk.r[qq] * cp.NG + cta) * kSegCap + slot] =
+                                make_uint2(pk.key[qq][k], (uint32_t)(pk.pos0[qq] + k * 32 + lane));
+                        else
+                            overflow = true;
+                    }
+                    at += __popc(bits);
+                }
+            }
+        }
+    }
+    if (__any_sync(0xffffffffu, overflow) && lane == 0) atomicOr(ctl + kOverflow, 1u);
+    if ((int)threadIdx.x < rows) {   // the row's count in this CTA
+        const int r = threadIdx.x;
+        int q0, q1;
+        row_span(r, q0, q1);
+        const uint32_t total = q1 > q0 ? pref[q1 - 1] + cnt[q1 - 1] - pref[q0] : 0u;
+        cp.counts[(int64_t)r * cp.NG + cta] = total;
+        if (total) atomicAdd(ctl + kTotal + r, total);
+        if (total > (uint32_t)kSegCap) atomicOr(ctl + kOverflow, 1u);
+    }
 }
 
 // One slice of the combine of (row bt, KV group g), by the 128 threads of a
@@ -947,6 +956,7 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
     }
 }
 
+template <int TQ>
 __global__ void __launch_bounds__(kThreads, 1)
 dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_ks,
                          const __grid_constant__ CUtensorMap tmap_q, const Params cp) {
@@ -969,8 +979,8 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     }
 
     // ---- phase 1: key stream, sample, candidates
-    run_indexer_capture(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G);
-    mark(2);
+    run_indexer_capture<TQ>(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G);
+    mark(15);
     if (status_at_entry & kNeedsInitBit) {
         if (threadIdx.x == 0) flag_timeout(status);
         return;
@@ -1093,6 +1103,22 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     }
 }
 
+// Whether the one-barrier kernel is launched as a programmatic dependent of
+// the previous kernel (on until a launch with both attributes is refused).
+static std::atomic<bool> g_pdl_capture{true};
+static bool pdl_capture_ok() { return g_pdl_capture.load(); }
+static void pdl_capture_off() { g_pdl_capture.store(false); }
+
+// The kernel for T query tokens per sequence (1..kMaxRows).
+static const void *capture_kernel_for(int T) {
+    switch (T) {
+        case 1: return (const void *)dsa_layer_capture_kernel<1>;
+        case 2: return (const void *)dsa_layer_capture_kernel<2>;
+        case 3: return (const void *)dsa_layer_capture_kernel<3>;
+        default: return (const void *)dsa_layer_capture_kernel<4>;
+    }
+}
+
 }  // namespace capture
 
 // --------------------------------------------------------------- host side
@@ -1107,7 +1133,12 @@ int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
     const int rows = B * T;
     if (dev.num_sms <= 0 || rows > kMaxRows || T > kMaxRows || Lmax < kMinContext) return DSA_OK;
     const int grid = dev.num_sms;
-    if (grid * kGroups > kThreads) return DSA_OK;   // the segment offsets are scanned one per thread
+    if (grid > kThreads) return DSA_OK;   // the segment offsets are scanned one per thread
+    // a CTA's (tile, query) pairs are counted one per thread after the stream
+    {
+        const int64_t tiles = (int64_t)B * ((Lmax + indexer::kTile - 1) / indexer::kTile);
+        if ((tiles + grid - 1) / grid * T > kThreads) return DSA_OK;
+    }
     // all CTAs must be resident together: one per SM (occupancy asked once per device)
     static std::mutex mu;
     static int per_sm_cache[64];
@@ -1118,19 +1149,23 @@ int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!known[dev_id]) {
-            if (int rc = ensure_smem_limit((const void *)dsa_layer_capture_kernel, capture_smem_budget(),
-                                           "cudaFuncSetAttribute(capture)"))
-                return rc;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_cache[dev_id], dsa_layer_capture_kernel,
-                                                              kThreads, capture_smem_budget());
-            if (e != cudaSuccess) return cuda_fail(e, "occupancy of the capture kernel");
+            // all CTAs of every instantiation must be resident together: the least occupancy
+            per_sm_cache[dev_id] = 1 << 30;
+            for (int t = 1; t <= kMaxRows; ++t) {
+                const void *k = capture_kernel_for(t);
+                if (int rc = ensure_smem_limit(k, capture_smem_budget(), "cudaFuncSetAttribute(capture)")) return rc;
+                int per_sm = 0;
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, capture_smem_budget());
+                if (e != cudaSuccess) return cuda_fail(e, "occupancy of the capture kernel");
+                per_sm_cache[dev_id] = std::min(per_sm_cache[dev_id], per_sm);
+            }
             known[dev_id] = true;
         }
         if (per_sm_cache[dev_id] < 1) return DSA_OK;
     }
     // the shared-memory layouts must fit: phase 1 with at least 3 stages, phase 2's list and attention teams
     if (Layout(3, T, B).total + 1024 > capture_smem_budget()) return DSA_OK;
-    const size_t ng = (size_t)grid * kGroups;
+    const size_t ng = (size_t)grid;   // one candidate segment per CTA and row
     const size_t fast2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 + 16 +
                                                   (size_t)2 * kListCap * 4 + (size_t)(kWide + kSmall) * 4,
                                               kTeams * align128(sizeof(attn::Smem)));
@@ -1165,7 +1200,7 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     int S = indexer::kMaxStages;
     while (S > 2 && Layout(S, ia.T, ia.B).total + 1024 > budget) --S;
     const size_t smem1 = Layout(S, ia.T, ia.B).total + 1024;
-    const size_t ng = (size_t)plan.grid * kGroups;
+    const size_t ng = (size_t)plan.grid;
     const size_t smem2 = kSelBytes + std::max(align128(sizeof(topk::Shared<kThreads>)) + ((ng + 1 + 31) & ~size_t(31)) * 4 + 16 +
                                                   (size_t)2 * kListCap * 4 + (size_t)(kWide + kSmall) * 4,
                                               kTeams * align128(sizeof(attn::Smem))) +
@@ -1225,24 +1260,39 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     tp.Lmax = ia.Lmax;
     tp.bar = cp.bar;
 
-    if (int rc = ensure_smem_limit((const void *)dsa_layer_capture_kernel, smem, "cudaFuncSetAttribute(capture)"))
-        return rc;
+    const void *kern = capture_kernel_for(ia.T);
+    if (int rc = ensure_smem_limit(kern, smem, "cudaFuncSetAttribute(capture)")) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;   // phase 1's sample and the grid barrier wait on every CTA
     attr[0].val.cooperative = 1;
+    // chained after the previous kernel of the stream (programmatic dependent
+    // launch): its launch overlaps that kernel's tail; the kernel's first
+    // instruction waits for that kernel's completion and memory
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_capture_ok() ? 2 : 1;
     cudaError_t e;
     if (start_event) {
         e = cudaEventRecord(static_cast<cudaEvent_t>(start_event), stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
-    e = cudaLaunchKernelEx(&cfg, dsa_layer_capture_kernel, L.tmap_k, L.tmap_ks, L.tmap_q, cp);
+    {
+        const CUtensorMap *mk = &L.tmap_k, *mks = &L.tmap_ks, *mq = &L.tmap_q;
+        void *args[] = {(void *)mk, (void *)mks, (void *)mq, (void *)&cp};
+        e = cudaLaunchKernelExC(&cfg, kern, args);
+        if (e != cudaSuccess && cfg.numAttrs == 2) {   // the driver refuses the pair: plain stream order from now on
+            (void)cudaGetLastError();
+            pdl_capture_off();
+            cfg.numAttrs = 1;
+            e = cudaLaunchKernelExC(&cfg, kern, args);
+        }
+    }
     if (e != cudaSuccess) return cuda_fail(e, "capture layer-step launch");
     return DSA_OK;
 }
