@@ -1109,6 +1109,9 @@ def main():
     ap.add_argument("--layers", type=int, default=4,
                     help="layers' caches the timed decode steps rotate over (inputs larger than L2)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--profile", type=int, default=0, metavar="N",
+                    help="no timing: N iterations of (L2 flush, dsa_indexer_scores, L2 flush, dsa_layer_decode) on "
+                         "the workload, for a profiler to attach to; prints the device status")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the ragged-mix and prefill lines that the default run adds as extra keys")
     ap.add_argument("--workload", choices=["tiny_8k", "verify_64k_t4", "ctx_1m", "ragged_b64_mix", "prefill_8k_1m",
@@ -1120,6 +1123,9 @@ def main():
         args.warmup = 3
     rank, world, local_rank = dist_env()
 
+    if args.profile > 0:
+        profile_run(args)
+        return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
@@ -1148,6 +1154,37 @@ def main():
     finally:
         if world > 1:
             dist.destroy_process_group()
+
+
+def profile_run(args):
+    """Untimed iterations of the indexer and the layer-step for ncu (one GPU):
+    each call after an L2 flush, so counters see a cold L2."""
+    import torch
+    import local_attention_decode_b200 as dsa
+    from workloads import CONFIGS, make_decode_workload
+    dev = torch.device("cuda", 0)
+    wl = make_decode_workload(device=dev, **CONFIGS[args.workload])
+    B, T = wl.B, wl.T
+    L = wl.layout.seq_lens[0]
+    kv = dsa.KV(k=wl.K, v=wl.V, index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G,
+                seq_stride=wl.layout.seq_stride, num_rows=wl.layout.num_rows)
+    ikv = dsa.KV(index_k=wl.k8, index_k_scale=wl.k_scale, num_kv_heads=wl.G, seq_stride=wl.layout.seq_stride,
+                 num_rows=wl.layout.num_rows)
+    O = torch.empty((B, T, 64, 128), dtype=torch.bfloat16, device=dev)
+    scores = torch.empty((B, T, L), dtype=torch.float32, device=dev)
+    ws = dsa.alloc_workspace(dsa.OP_LAYER, B, T, L, TOP_K, device=dev)
+    iws = dsa.alloc_workspace(dsa.OP_INDEXER, B, T, L, 1, device=dev)
+    flush = L2Flush(dev)
+    for _ in range(args.profile):
+        flush()
+        dsa.dsa_indexer_scores(wl.q8, wl.q_scale, wl.w, ikv, wl.q_pos, L, scores, iws)
+        flush()
+        dsa.dsa_layer_decode(wl.q8, wl.q_scale, wl.w, wl.Q, kv, wl.q_pos, L, TOP_K, wl.sink, 1.0 / math.sqrt(192), O,
+                             ws=ws)
+    torch.cuda.synchronize(dev)
+    print(json.dumps({"profile_iterations": args.profile, "workload": args.workload,
+                      "status": [dsa.dsa_check_device_status(w)[0] for w in (ws, iws)],
+                      "layer_step_paths": dsa.dsa_layer_path_counts(ws)}), flush=True)
 
 
 def secondary_lines(args, rank, world, local_rank):

@@ -153,7 +153,7 @@ static int check_index_stride(const dsa_kv_t *kv, int B) {
 
 // ------------------------------------------------------------ workspace plan
 struct WsPlan {
-    size_t status = 0, scores = 0, idx = 0, count = 0, topk = 0, part_o = 0, part_ml = 0, total = 0;
+    size_t status = 0, scores = 0, idx = 0, count = 0, topk = 0, part_o = 0, part_ml = 0, cap_data = 0, total = 0;
     TopkPlan tp;
     FusedPlan fp;
     CapturePlan cp;
@@ -197,6 +197,7 @@ static int plan_workspace(int op, int B, int T, int64_t Lmax, int top_k, WsPlan 
             // the self-cleaning selection scratch first: its offset does not depend on the shape
             w->topk = take(std::max({w->tp.scratch_bytes, w->fp.ok ? w->fp.scratch_bytes : 0,
                                      w->cp.ok ? w->cp.scratch_bytes : 0}));
+            w->cap_data = take(w->cp.ok ? w->cp.data_bytes : 0);
             w->scores = take((size_t)B * T * Lmax * 4);
             w->idx = take((size_t)B * T * top_k * 4);
             w->count = take((size_t)B * T * 4);
@@ -304,7 +305,7 @@ static int plan_prefill_layout(int NQ, int64_t Lmax, int top_k, PrefillLayout *p
     if ((rc = plan_workspace(DSA_OP_LAYER, 1, 1, Lmax, top_k, &pl->redo))) return rc;
     const size_t base = align_up(end, 256) - kStatusBytes;
     for (size_t *o : {&pl->redo.scores, &pl->redo.idx, &pl->redo.count, &pl->redo.topk, &pl->redo.part_o,
-                      &pl->redo.part_ml, &pl->redo.total})
+                      &pl->redo.part_ml, &pl->redo.cap_data, &pl->redo.total})
         *o += base;
     pl->total = pl->redo.total;
     return DSA_OK;
@@ -593,8 +594,8 @@ static int layer_run(const void *q8, const float *q_scale, const float *w, const
         a.status = status;
         a.padded = 1;   // the fused selection pads every idx row with -1
         if (wp.cp.ok)
-            rc = launch_capture(wp.cp, ia, a, top_k, idx, count, at<uint8_t>(ws, wp.topk), s,
-                                stage_events ? stage_events[0] : nullptr);
+            rc = launch_capture(wp.cp, ia, a, top_k, idx, count, at<uint8_t>(ws, wp.topk), at<uint8_t>(ws, wp.cap_data),
+                                s, stage_events ? stage_events[0] : nullptr);
         if (!wp.cp.ok || rc == DSA_ERR_UNSUPPORTED_SHAPE)
             rc = wp.fp.ok ? launch_fused(wp.fp, ia, a, top_k, idx, count, at<uint32_t>(ws, wp.topk), s,
                                          stage_events ? stage_events[0] : nullptr)

@@ -66,6 +66,10 @@ constexpr int kSegCap = 1024;                 // candidates one CTA may hold per
 constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
 constexpr int kWide = 4096;                   // bins of the selection's first histogram
 constexpr int kSmall = 2048;                  // keys of T*'s bin taken aside for the remaining bits
+// The candidates' histogram that the stream builds: bin (key - threshold) >>
+// kCandShift, kWide bins, the last one taking everything above (two octaves
+// of non-negative scores at 1/2048 octave).
+constexpr int kCandShift = 12;
 constexpr int kGroupBar0 = 5;                 // named barriers 5..8: the epilogue groups
 constexpr int kUnitBar = 9;                   // named barrier of the attention teams of a CTA unit
 constexpr int kSelBytes = DSA_MAX_TOPK * 4;   // the selection, at the start of shared memory in phase 2
@@ -99,6 +103,7 @@ struct Params {
     uint32_t *ctl;
     uint32_t *sample_hist;    // [rows][kHistStride]
     uint32_t *counts;         // [rows][NG]
+    uint32_t *cand_hist;      // [rows][kWide] the candidates' keys above the row's threshold (kCandShift)
     uint2 *lists;             // [rows][NG][kSegCap] (order key, position)
     uint32_t *path_count;     // [2] calls that took the fast path / the general path
     uint64_t *trace;          // [grid][DSA_TRACE_MARKS] phase marks, or NULL
@@ -654,6 +659,12 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                                 make_uint2(pk.key[qq][k], (uint32_t)(pk.pos0[qq] + k * 32 + lane));
                         else
                             overflow = true;
+                        uint32_t th = 0u;
+#pragma unroll
+                        for (int rr = 0; rr < kMaxRows; ++rr)
+                            if (rr == pk.r[qq]) th = thr[rr];
+                        const uint32_t bin = min((pk.key[qq][k] - th) >> kCandShift, (uint32_t)(kWide - 1));
+                        atomicAdd(cp.cand_hist + (int64_t)pk.r[qq] * kWide + bin, 1u);
                     }
                     at += __popc(bits);
                 }
@@ -778,47 +789,26 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             mbar_expect_tx(copied, vp * 8u);
             bulk_load(list + (incl - vp), segs + (int64_t)threadIdx.x * kSegCap, vp * 8u, copied);
         }
+        if (threadIdx.x == NT - 1) {   // and the stream's histogram of the row's candidates
+            mbar_expect_tx(copied, kWide * 4u);
+            bulk_load(wide, cp.cand_hist + (int64_t)r * kWide, kWide * 4u, copied);
+        }
         __syncthreads();   // every expected byte is posted
         if (threadIdx.x == 0) mbar_arrive(copied);
         mbar_wait(copied, 0, cp.ix.status);
         if (threadIdx.x < NG && (v & 1u)) list[incl - 1] = make_uint2(0u, 0xFFFFFFFFu);
         __syncthreads();
         if (trace && threadIdx.x == 0) trace[8] = globaltimer_ns();
-        // ---- the k-th largest key T*, exactly.  The candidates lie above one
-        //      threshold, so their keys share the high bits: a histogram of
-        //      the 12 bits below the common ones finds T*'s bin in one pass;
-        //      only that bin's keys (a handful) go on to the remaining bits.
+        // ---- the k-th largest key T*, exactly.
         auto is_key = [&](uint32_t j, uint32_t &k) {
             const uint2 e = list[j];
             k = e.x;
             return e.y != 0xFFFFFFFFu;   // not a pad
         };
-        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-        for (uint32_t j = threadIdx.x; j < m; j += NT) {
-            uint32_t k;
-            if (is_key(j, k)) {
-                kmin = min(kmin, k);
-                kmax = max(kmax, k);
-            }
-        }
-        kmin = __reduce_min_sync(0xffffffffu, kmin);
-        kmax = __reduce_max_sync(0xffffffffu, kmax);
-        if (lane == 0) {
-            sh->warp_a[warp] = kmin;
-            sh->warp_b[warp] = kmax;
-        }
-        for (int j = threadIdx.x; j < kWide; j += NT) wide[j] = 0;
-        __syncthreads();
-        for (int w2 = 0; w2 < NW; ++w2) {
-            kmin = min(kmin, sh->warp_a[w2]);
-            kmax = max(kmax, sh->warp_b[w2]);
-        }
-        const int top = kmin == kmax ? 0 : 31 - __clz(kmin ^ kmax);   // highest bit in which keys differ
-        const int shift = top > 11 ? top - 11 : 0;
-        const uint32_t hi_mask = top >= 31 ? 0u : ~((2u << top) - 1u);   // the bits every key shares
-        list_digit_hist<NT>(wide, m, kmin & hi_mask, hi_mask, shift, (uint32_t)kWide, is_key);
-        __syncthreads();
-        {   // the bin of the k-th largest key: 512 threads own 8 bins each, from the top
+        // The bin of `wide` (kWide bins, the top one holding the largest
+        // keys) that holds the K-th largest key, and the keys above it: 512
+        // threads own 8 bins each, from the top.
+        auto find_bin = [&]() {
             uint32_t s = 0;
             if (threadIdx.x < kWide / 8)
                 for (int i = 0; i < 8; ++i) s += wide[kWide - 1 - 8 * (int)threadIdx.x - i];
@@ -837,79 +827,139 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
                 }
             }
             __syncthreads();
-        }
-        uint32_t prefix = (kmin & hi_mask) | ((uint32_t)sh->bin << shift);
-        uint32_t mask = hi_mask | ((uint32_t)(kWide - 1) << shift);
-        uint32_t Krem = (uint32_t)K - sh->above;
-        const uint32_t in_bin = wide[sh->bin];
-        __syncthreads();
-        if (shift > 0) {
-            // the keys of T*'s bin into a small buffer (any order), unless too many
-            const bool small = in_bin <= (uint32_t)kSmall;
-            if (small) {
-                if (threadIdx.x == 0) sh->total = 0;
-                __syncthreads();
-                for (uint32_t jb = threadIdx.x & ~31u; jb < m; jb += NT) {
-                    const uint32_t j = jb + lane;
-                    uint32_t k = 0u;
-                    const bool take = j < m && is_key(j, k) && (k & mask) == prefix;
-                    const uint32_t bits = __ballot_sync(0xffffffffu, take);
-                    uint32_t at = 0;
-                    if (lane == 0 && bits) at = atomicAdd(&sh->total, (uint32_t)__popc(bits));
-                    at = __shfl_sync(0xffffffffu, at, 0);
-                    if (take) bin_keys[at + __popc(bits & lt)] = k;
+        };
+        // A handful of keys in bin_keys: one warp ranks them; T* is the key
+        // with fewer than Krem keys above it and at least Krem at or above.
+        auto rank_small = [&](uint32_t n_keys, uint32_t Krem_in, uint32_t &t_out, uint32_t &ties_out) {
+            if (warp == 0) {
+                const bool valid = (uint32_t)lane < n_keys;
+                const uint32_t mine = valid ? bin_keys[lane] : 0u;
+                uint32_t gt = 0, ge = 0;
+                for (uint32_t q = 0; q < n_keys; ++q) {
+                    const uint32_t o = __shfl_sync(0xffffffffu, mine, q);
+                    gt += o > mine;
+                    ge += o >= mine;
                 }
-                __syncthreads();
+                const uint32_t hit = __ballot_sync(0xffffffffu, valid && gt < Krem_in && Krem_in <= ge);
+                const int src = hit ? __ffs(hit) - 1 : 0;
+                const uint32_t t_key = __shfl_sync(0xffffffffu, mine, src);
+                const uint32_t t_gt = __shfl_sync(0xffffffffu, gt, src);
+                if (lane == 0) {
+                    sh->base = t_key;
+                    sh->above = t_gt;
+                }
             }
-            if (small && in_bin <= 32u) {
-                // a handful of keys: one warp ranks them; T* is the key with
-                // fewer than Krem keys above it and at least Krem at or above
-                if (warp == 0) {
-                    const bool valid = (uint32_t)lane < in_bin;
-                    const uint32_t mine = valid ? bin_keys[lane] : 0u;
-                    uint32_t gt = 0, ge = 0;
-                    for (uint32_t q = 0; q < in_bin; ++q) {
-                        const uint32_t o = __shfl_sync(0xffffffffu, mine, q);
-                        gt += o > mine;
-                        ge += o >= mine;
-                    }
-                    const uint32_t hit = __ballot_sync(0xffffffffu, valid && gt < Krem && Krem <= ge);
-                    const int src = hit ? __ffs(hit) - 1 : 0;
-                    const uint32_t t_key = __shfl_sync(0xffffffffu, mine, src);
-                    const uint32_t t_gt = __shfl_sync(0xffffffffu, gt, src);
-                    if (lane == 0) {
-                        sh->base = t_key;
-                        sh->above = t_gt;
-                    }
+            __syncthreads();
+            t_out = sh->base;
+            ties_out = Krem_in - sh->above;
+            __syncthreads();
+        };
+        // Gathers into bin_keys the keys k with pred(k) (any order); their count.
+        auto gather_keys = [&](auto pred) {
+            if (threadIdx.x == 0) sh->total = 0;
+            __syncthreads();
+            for (uint32_t jb = threadIdx.x & ~31u; jb < m; jb += NT) {
+                const uint32_t j = jb + lane;
+                uint32_t k = 0u;
+                const bool take = j < m && is_key(j, k) && pred(k);
+                const uint32_t bits = __ballot_sync(0xffffffffu, take);
+                uint32_t at = 0;
+                if (lane == 0 && bits) at = atomicAdd(&sh->total, (uint32_t)__popc(bits));
+                at = __shfl_sync(0xffffffffu, at, 0);
+                if (take && at + __popc(bits & lt) < (uint32_t)kSmall) bin_keys[at + __popc(bits & lt)] = k;
+            }
+            __syncthreads();
+            const uint32_t n_keys = sh->total;
+            __syncthreads();
+            return n_keys;
+        };
+        uint32_t Tstar = 0u, ties = 0u;
+        bool found = false;
+        {   // from the stream's histogram of the row's candidates above its threshold
+            const uint32_t thr_r = __ldcg(cp.ctl + kThr + r);
+            find_bin();
+            const int B = sh->bin;
+            const uint32_t Kb = (uint32_t)K - sh->above, in_b = wide[B];
+            __syncthreads();
+            if (B < kWide - 1 && in_b <= 32u) {   // not the catch-all bin, and a handful of keys
+                const uint32_t n_keys = gather_keys(
+                    [&](uint32_t k) { return k >= thr_r && ((k - thr_r) >> kCandShift) == (uint32_t)B; });
+                if (n_keys == in_b) {   // (always: the histogram counted exactly these keys)
+                    rank_small(n_keys, Kb, Tstar, ties);
+                    found = true;
                 }
-                __syncthreads();
-                prefix = sh->base;
-                Krem -= sh->above;
-                __syncthreads();
-            } else
-            // the remaining bits, 11 at a time, over the bin's keys
-            for (int sh2 = shift; sh2 > 0;) {
-                const int w = sh2 > 11 ? 11 : sh2;
-                sh2 -= w;
-                const int nb = 1 << w;
-                for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
-                __syncthreads();
-                if (small)
-                    list_digit_hist<NT>(sh->hist, in_bin, prefix, mask, sh2, (uint32_t)nb, [&](uint32_t j, uint32_t &k) {
-                        k = bin_keys[j];
-                        return true;
-                    });
-                else
-                    list_digit_hist<NT>(sh->hist, m, prefix, mask, sh2, (uint32_t)nb, is_key);
-                __syncthreads();
-                topk::find_threshold<NT>(sh, nb, Krem);
-                prefix |= (uint32_t)sh->bin << sh2;
-                mask |= (uint32_t)(nb - 1) << sh2;
-                Krem -= sh->above;
-                __syncthreads();
             }
         }
-        const uint32_t Tstar = prefix, ties = Krem;
+        if (!found) {   // the general search: the 12 bits below the keys' common high bits, then the rest
+            uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+            for (uint32_t j = threadIdx.x; j < m; j += NT) {
+                uint32_t k;
+                if (is_key(j, k)) {
+                    kmin = min(kmin, k);
+                    kmax = max(kmax, k);
+                }
+            }
+            kmin = __reduce_min_sync(0xffffffffu, kmin);
+            kmax = __reduce_max_sync(0xffffffffu, kmax);
+            if (lane == 0) {
+                sh->warp_a[warp] = kmin;
+                sh->warp_b[warp] = kmax;
+            }
+            __syncthreads();
+            for (int j = threadIdx.x; j < kWide; j += NT) wide[j] = 0;
+            __syncthreads();
+            for (int w2 = 0; w2 < NW; ++w2) {
+                kmin = min(kmin, sh->warp_a[w2]);
+                kmax = max(kmax, sh->warp_b[w2]);
+            }
+            const int top = kmin == kmax ? 0 : 31 - __clz(kmin ^ kmax);   // highest bit in which keys differ
+            const int shift = top > 11 ? top - 11 : 0;
+            const uint32_t hi_mask = top >= 31 ? 0u : ~((2u << top) - 1u);   // the bits every key shares
+            list_digit_hist<NT>(wide, m, kmin & hi_mask, hi_mask, shift, (uint32_t)kWide, is_key);
+            __syncthreads();
+            find_bin();
+            uint32_t prefix = (kmin & hi_mask) | ((uint32_t)sh->bin << shift);
+            uint32_t mask = hi_mask | ((uint32_t)(kWide - 1) << shift);
+            uint32_t Krem = (uint32_t)K - sh->above;
+            const uint32_t in_bin = wide[sh->bin];
+            __syncthreads();
+            if (shift > 0) {
+                // the keys of T*'s bin into a small buffer (any order), unless too many
+                const bool small = in_bin <= (uint32_t)kSmall;
+                if (small) gather_keys([&](uint32_t k) { return (k & mask) == prefix; });
+                if (small && in_bin <= 32u) {
+                    uint32_t t_key, t_ties;
+                    rank_small(in_bin, Krem, t_key, t_ties);
+                    prefix = t_key;
+                    Krem = t_ties;
+                } else {
+                    // the remaining bits, 11 at a time, over the bin's keys
+                    for (int sh2 = shift; sh2 > 0;) {
+                        const int w = sh2 > 11 ? 11 : sh2;
+                        sh2 -= w;
+                        const int nb = 1 << w;
+                        for (int j = threadIdx.x; j < nb; j += NT) sh->hist[j] = 0;
+                        __syncthreads();
+                        if (small)
+                            list_digit_hist<NT>(sh->hist, in_bin, prefix, mask, sh2, (uint32_t)nb,
+                                                [&](uint32_t j, uint32_t &k) {
+                                                    k = bin_keys[j];
+                                                    return true;
+                                                });
+                        else
+                            list_digit_hist<NT>(sh->hist, m, prefix, mask, sh2, (uint32_t)nb, is_key);
+                        __syncthreads();
+                        topk::find_threshold<NT>(sh, nb, Krem);
+                        prefix |= (uint32_t)sh->bin << sh2;
+                        mask |= (uint32_t)(nb - 1) << sh2;
+                        Krem -= sh->above;
+                        __syncthreads();
+                    }
+                }
+            }
+            Tstar = prefix;
+            ties = Krem;
+        }
         if (trace && threadIdx.x == 0) trace[9] = globaltimer_ns();
         // compaction in position order, in 32-entry strips: each warp a run
         // of whole strips; the keys above T* and the first `ties` keys equal
@@ -996,13 +1046,9 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
         // the list in shared memory holds the candidates and up to one pad per segment
         if (n > cp.K && (m < (uint32_t)cp.K || m + (uint32_t)cp.NG > (uint32_t)kListCap)) fast = false;
     }
-    if (blockIdx.x == 0 && threadIdx.x < kMaxRows + 1) {   // read by nobody after phase 1
-        if (threadIdx.x == 0) {
-            ctl[kReady] = 0;
-            atomicAdd(cp.path_count + (fast ? 0 : 1), 1u);
-        } else {
-            ctl[kThr + threadIdx.x - 1] = 0;
-        }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {   // read by nobody after phase 1
+        ctl[kReady] = 0;
+        atomicAdd(cp.path_count + (fast ? 0 : 1), 1u);
     }
 
     const int rows = cp.rows, C = cp.C;
@@ -1092,11 +1138,22 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     if (trace && threadIdx.x == 0) trace[14] = clock64();
     if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(ctl + kGridExit, 1u) == G - 1) {
+        sync_flag = atomicAdd(ctl + kGridExit, 1u) == G - 1 ? 1u : 0u;
+    }
+    __syncthreads();
+    if (sync_flag) {   // the last CTA out: every other CTA is done with these words
+        for (int i = threadIdx.x; i < rows * kWide; i += blockDim.x) cp.cand_hist[i] = 0;
+        if (threadIdx.x == 0) {
             ctl[kGridArrive] = 0;
             ctl[kOverflow] = 0;
-            for (int r = 0; r < kMaxRows; ++r) ctl[kTotal + r] = 0;
+            for (int r = 0; r < kMaxRows; ++r) {
+                ctl[kTotal + r] = 0;
+                ctl[kThr + r] = 0;
+            }
             for (int i = 0; i < rows * DSA_Q_HEADS; ++i) ctl[kCombine + i] = 0;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
             __threadfence();
             ctl[kGridExit] = 0;
         }
@@ -1182,16 +1239,19 @@ int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
     };
     plan->ctl_off = take(kCtlWords * 4);
     plan->hist_off = take((size_t)rows * kHistStride * 4);
+    plan->topk_off = take((size_t)rows * topk::scratch_words(plan->C, topk::kListCap, false) * 4);
+    plan->cand_hist_off = take((size_t)rows * kWide * 4);
+    plan->scratch_bytes = off;
+    off = 0;
     plan->counts_off = take((size_t)rows * ng * 4);
     plan->lists_off = take((size_t)rows * ng * kSegCap * 8);
-    plan->topk_off = take((size_t)rows * topk::scratch_words(plan->C, topk::kListCap, false) * 4);
-    plan->scratch_bytes = off;
+    plan->data_bytes = off;
     plan->ok = true;
     return DSA_OK;
 }
 
 int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
-                   int32_t *count, uint8_t *scratch, cudaStream_t stream, void *start_event) {
+                   int32_t *count, uint8_t *scratch, uint8_t *data, cudaStream_t stream, void *start_event) {
     using namespace capture;
     const size_t budget = capture_smem_budget();
     IndexerLaunch L;
@@ -1223,8 +1283,9 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     cp.lse = aa.lse;
     cp.ctl = reinterpret_cast<uint32_t *>(scratch + plan.ctl_off);
     cp.sample_hist = reinterpret_cast<uint32_t *>(scratch + plan.hist_off);
-    cp.counts = reinterpret_cast<uint32_t *>(scratch + plan.counts_off);
-    cp.lists = reinterpret_cast<uint2 *>(scratch + plan.lists_off);
+    cp.counts = reinterpret_cast<uint32_t *>(data + plan.counts_off);
+    cp.cand_hist = reinterpret_cast<uint32_t *>(scratch + plan.cand_hist_off);
+    cp.lists = reinterpret_cast<uint2 *>(data + plan.lists_off);
     cp.path_count = ia.status + kPathCountWord;
     cp.trace = phase_trace(plan.grid);
     cp.bar = barrier_cfg();

@@ -242,13 +242,20 @@ struct CapturePlan {
     int grid = 0;
     int rows = 0;
     int C = 1;                  // CTAs per row
-    int NG = 0;                 // epilogue groups in the grid (segments of each row's list)
-    size_t ctl_off = 0, hist_off = 0, counts_off = 0, lists_off = 0, topk_off = 0;
-    size_t scratch_bytes = 0;   // all of the above (self-cleaning parts and overwritten parts)
+    int NG = 0;                 // CTAs in the grid (segments of each row's list)
+    // self-cleaning scratch (zero between calls): control words, sample and
+    // candidate histograms, the fallback selection's scratch
+    size_t ctl_off = 0, hist_off = 0, topk_off = 0, cand_hist_off = 0;
+    size_t scratch_bytes = 0;
+    // overwritten by every call (never assumed zero): the candidate segments
+    // and their lengths, in a workspace region of their own
+    size_t counts_off = 0, lists_off = 0;
+    size_t data_bytes = 0;
 };
 int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan);
 int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
-                   int32_t *count, uint8_t *scratch, cudaStream_t stream, void *start_event = nullptr);
+                   int32_t *count, uint8_t *scratch, uint8_t *data, cudaStream_t stream,
+                   void *start_event = nullptr);
 int launch_fused(const FusedPlan &plan, const IndexerArgs &ia, const AttnArgs &aa, int top_k, int32_t *idx,
                  int32_t *count, uint32_t *scratch, cudaStream_t stream,
                  void *start_event = nullptr);

@@ -421,3 +421,30 @@ def test_bad_positions_are_flagged_not_faulted():
     ref_o, _ = oracle_attention_rows(wl, 0, 0, np.array([5]), wl.sink, SM)   # bad entries are skipped
     assert_attn_close(O[0, 0], ref_o)
     assert dsa.dsa_check_device_status(ws)[0] == dsa.DSA_OK   # reading clears the word
+
+
+def test_layer_decode_many_tied_top_keys():
+    """3,000 keys share the row's highest score (copies of its best key, at
+    twice its scale): the bin of the k-th largest key in the one-barrier
+    kernel's candidate histogram holds all of them, so its general search runs;
+    the selection is the 2,048 lowest positions of the tied keys, as the
+    oracle's top-k (ties to the lower position)."""
+    wl = make_decode_workload(seed=95, seq_lens=[20000], T=1, device=DEV, n_needles=0)
+    scores = run_indexer(wl)
+    best = int(torch.argmax(scores[0, 0]))
+    assert float(scores[0, 0, best]) > 0
+    g = torch.Generator().manual_seed(6)
+    tied = torch.randperm(20000, generator=g)[:3000].sort().values.to(DEV)
+    key, scale = wl.k8[best].clone(), wl.k_scale[best].clone() * 2
+    wl.k8[tied] = key
+    wl.k_scale[tied] = scale
+    O, lse, idx, cnt = run_layer(wl)
+    assert LAST_PATHS == [1, 0]   # the fast path: the general search is inside it
+    scores = run_indexer(wl)
+    ref_idx, ref_cnt = oracle.topk(scores[0, 0].cpu().numpy(), 2048)
+    assert int(cnt[0, 0]) == ref_cnt == 2048
+    got = idx[0, 0].cpu().numpy()
+    assert np.array_equal(got, np.sort(ref_idx))
+    assert np.array_equal(got, np.sort(tied.cpu().numpy())[:2048])
+    ref_o, ref_l = oracle_attention_rows(wl, 0, 0, got, wl.sink, SM)
+    assert_attn_close(O[0, 0], ref_o, lse[0, 0], ref_l)
