@@ -146,16 +146,22 @@ __device__ __forceinline__ uint32_t sample_bin(uint32_t key) {
 // threshold is the lower edge of the highest bin b whose count, with the bins
 // above it, reaches that target; zero (take every key) when the sample's
 // non-negative scores do not reach it.  Zeroes the histogram for the next call.
-__device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversample) {
+// `local` is shared memory of kBins words that the warp may overwrite: the
+// loaded histogram goes there, so the second level of the search reads it
+// from shared memory (one round trip to L2 in all).
+__device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversample, uint32_t *local) {
     const int lane = lane_id();
     constexpr int kPer = kBins / 32;   // 64 bins per lane
     uint32_t s = 0;
     const uint4 *h4 = reinterpret_cast<const uint4 *>(hist + lane * kPer);
+    uint4 *l4 = reinterpret_cast<uint4 *>(local + lane * kPer);
 #pragma unroll
     for (int u = 0; u < kPer / 4; ++u) {
         const uint4 v = __ldcg(h4 + u);
         s += v.x + v.y + v.z + v.w;
+        l4[u] = v;
     }
+    __syncwarp();
     const uint32_t negative = __ldcg(hist + kBins);
     uint32_t incl = s;   // keys in this lane's bins and all higher ones
 #pragma unroll
@@ -173,7 +179,7 @@ __device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversa
         const uint32_t above = __shfl_sync(0xffffffffu, incl - s, L);
         // that lane's 64 bins, two per lane, then the same search over them
         const uint32_t b0 = (uint32_t)(L * kPer + 2 * lane);
-        const uint32_t v0 = __ldcg(hist + b0), v1 = __ldcg(hist + b0 + 1);
+        const uint32_t v0 = local[b0], v1 = local[b0 + 1];
         const uint32_t t = v0 + v1;
         uint32_t inc2 = t;
 #pragma unroll
@@ -496,7 +502,9 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             uint32_t t_r = 0xFFFFFFFFu;   // n <= top_k: every key is selected, nothing to capture
                             uint32_t *h = cp.sample_hist + r * kHistStride;
                             if (n > cp.K) {
-                                t_r = row_threshold(h, n, cp.K, cp.oversample);
+                                // (the CTA's shared histogram of this row, already added in,
+                                // takes the loaded global one)
+                                t_r = row_threshold(h, n, cp.K, cp.oversample, hist + r * kHistStride);
                             } else {
                                 for (int u = lane; u < kHistWords; u += 32) h[u] = 0;
                             }

@@ -173,8 +173,9 @@ int launch_indexer(const IndexerArgs &a, cudaStream_t stream) {
     int rc = prepare_indexer(a, 0, 0, nullptr, device_info().smem_optin, &L);
     if (rc) return rc;
     if ((rc = ensure_smem_limit((const void *)indexer_kernel, L.smem, "cudaFuncSetAttribute(indexer)"))) return rc;
-    cudaError_t e = launch_kernel(indexer_kernel, dim3(L.grid), dim3(kThreads), L.smem, stream, L.tmap_k, L.tmap_ks,
-                                  L.tmap_q, L.p);
+    // launched as a programmatic dependent: back-to-back calls overlap the launch with the previous tail
+    cudaError_t e = launch_kernel_as(true, indexer_kernel, dim3(L.grid), dim3(kThreads), L.smem, stream, L.tmap_k,
+                                     L.tmap_ks, L.tmap_q, L.p);
     if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
     return DSA_OK;
 }

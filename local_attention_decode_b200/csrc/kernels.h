@@ -34,15 +34,26 @@ void set_pdl_launches(bool on);
 
 // A plain (non-cooperative) launch, chained when pdl_launches().
 template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel_as(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args... args);
+template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                           Args... args) {
+    return launch_kernel_as(pdl_launches(), kernel, grid, block, smem, stream, args...);
+}
+
+// As launch_kernel, with programmatic dependent launch when `pdl` (every
+// kernel of this library waits for its predecessor at its first instruction).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel_as(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    if (pdl_launches()) {
+    if (pdl) {
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
