@@ -839,9 +839,11 @@ def trace_phases(dsa, torch, dev, step, R, n=8):
     import numpy as np
     tr = torch.zeros(148 * 2 * dsa.TRACE_MARKS, dtype=torch.int64, device=dev)
     names = {10: "first_key_tile_requested", 12: "first_tile_scored", 7: "sample_handed_in", 1: "thresholds_seen",
-             2: "key_stream_done", 3: "past_grid_barrier", 8: "candidates_in_smem", 9: "kth_key_found",
+             2: "key_stream_done", 15: "candidates_captured", 3: "past_grid_barrier", 8: "candidates_in_smem",
+             9: "kth_key_found",
              4: "selection_done", 5: "attention_units_done", 6: "exit"}
-    rows = []
+    rows, mids, spans = [], [], {}
+    chain = [2, 15, 3, 8, 9, 4, 5, 6]
     dsa.dsa_trace_phases(tr)
     try:
         for i in range(n):
@@ -854,10 +856,22 @@ def trace_phases(dsa, torch, dev, step, R, n=8):
                 return {}
             t0 = m[:, 0].min()
             rows.append({k: (m[:, k][m[:, k] > 0].max() - t0) / 1e3 for k in names if (m[:, k] > 0).any()})
+            mids.append({k: (np.median(m[:, k][m[:, k] > 0]) - t0) / 1e3 for k in names if (m[:, k] > 0).any()})
+            # each CTA's own time between consecutive marks of the post-stream chain
+            for a_, b_ in zip(chain[:-1], chain[1:]):
+                ok = (m[:, a_] > 0) & (m[:, b_] > 0)
+                if ok.any():
+                    d = (m[ok, b_] - m[ok, a_]) / 1e3
+                    spans.setdefault((a_, b_), []).append((np.median(d), d.max()))
     finally:
         dsa.dsa_trace_phases(None)
     out = {names[k]: float(np.median([r[k] for r in rows if k in r])) for k in names if any(k in r for r in rows)}
     out["how"] = "latest CTA at each mark, us after the first CTA entered; median of 8 steps"
+    out["median_cta"] = {names[k]: round(float(np.median([r[k] for r in mids if k in r])), 3)
+                         for k in names if any(k in r for r in mids)}
+    out["per_cta_span_us"] = {f"{names[a_]}->{names[b_]}": {"median": round(float(np.median([x[0] for x in v])), 3),
+                                                           "max": round(float(np.median([x[1] for x in v])), 3)}
+                              for (a_, b_), v in spans.items()}
     return out
 
 

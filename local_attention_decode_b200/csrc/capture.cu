@@ -18,10 +18,13 @@
 // histogram, the CTA's last group adds it into the row's global one, and the
 // last CTA to do so turns each row's histogram into a score threshold -- a
 // bin edge below which the sample predicts about `oversample` x top_k keys --
-// and publishes it.  When its tiles are done, a CTA takes its candidates from
-// its own stored scores (in L2): every visible key at or above the threshold,
-// with its position, in position order, into the CTA's segment of the row's
-// candidate list.
+// and publishes it.  The thresholds arrive in the middle of the stream: one
+// warp per epilogue group polls for them between tiles, and from then on each
+// epilogue warp keeps, tile by tile, every visible key of its 32 rows at or
+// above its row's threshold in a short list of its own in shared memory (the
+// tiles it scored before, it takes again from its own stored scores).  When
+// its tiles are done, a CTA merges its warps' lists into its segment of the
+// row's candidate list, in position order.
 // One grid barrier.  The segments' lengths tell whether the sample was good:
 // if every row holds at least top_k candidates (then the list holds every key
 // at or above the k-th largest score, since the threshold is below it) and no
@@ -63,6 +66,8 @@ constexpr int kBins = 2048;                   // sample histogram: bits 30..20 o
 constexpr int kHistWords = kBins + 1;         // + the count of negative scores
 constexpr int kHistStride = kHistWords + 3;   // words between rows' histograms: rows start 16-byte aligned
 constexpr int kSegCap = 1024;                 // candidates one CTA may hold per row
+constexpr int kGroupCap = 256;                // candidates one epilogue group may hold per row
+constexpr int kMaxBacklog = 16;               // tiles per epilogue group whose keys wait in TMEM for the thresholds
 constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
 constexpr int kWide = 4096;                   // bins of the selection's first histogram
 constexpr int kSmall = 2048;                  // keys of T*'s bin taken aside for the remaining bits
@@ -87,10 +92,13 @@ enum {
     kThr = 8,                 // [kMaxRows] thresholds (order keys)
     kTotal = 12,              // [kMaxRows] candidates per row
     kCombine = 16,            // [kMaxRows][64] attention units done per (row, KV group)
+    kThrPacked = 272,         // [kMaxRows] 64-bit: (1 << 32) | threshold, once published
     kCtlWords = 512
 };
 
-static_assert(kCombine + kMaxRows * DSA_Q_HEADS <= kCtlWords, "control words");
+static_assert(kCombine + kMaxRows * DSA_Q_HEADS <= kThrPacked && kThrPacked + 2 * kMaxRows <= kCtlWords,
+              "control words");
+static_assert(kThrPacked % 2 == 0, "64-bit words");
 static_assert(kTeams * 4 < kWarps, "the attention teams must leave warps free in the CTA");
 
 struct Params {
@@ -116,7 +124,8 @@ __host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~si
 
 // Shared memory of phase 1 (base aligned to 1024 bytes).
 struct Layout {
-    uint32_t k_off, q_off, ks_off, bar_off, tmem_off, len_off, tile_off, epi_off, hist_off, misc_off, total;
+    uint32_t k_off, q_off, ks_off, bar_off, tmem_off, len_off, tile_off, epi_off, hist_off, misc_off, cap_off, poll_off,
+        total;
     __host__ __device__ Layout(int S, int T, int B) {
         const int stages = kPipes * S, rows = B * T;
         k_off = 0;
@@ -129,8 +138,13 @@ struct Layout {
         epi_off = (tile_off + 4 * (B + 1) + 15) & ~15u;
         hist_off = epi_off + kGroups * kEpiWarps * (16 * T + T) * 4;
         misc_off = hist_off + rows * kHistStride * 4;
-        total = misc_off + 32 + 16;   // misc: [0] groups sampled, [1 + g] group g's role in the sample
-                                      // exchange; then the rows' query positions
+        // misc: [0] groups sampled, [1 + g] group g's role in the sample
+        // exchange; then the rows' query positions
+        // [kMaxRows] thresholds, [kMaxRows] their flag; then per group: the
+        // warps' counts of a capture step, the lists' lengths, the decisions
+        cap_off = misc_off + 32 + 16;
+        poll_off = cap_off + 4 * (2 * kMaxRows + kGroups * (kEpiWarps * kMaxRows + 2 * kMaxRows + 2));
+        total = poll_off + kGroups * kMaxRows * 8;   // [group] the packed words, as the poller read them
     }
 };
 
@@ -143,9 +157,13 @@ __device__ __forceinline__ uint32_t sample_bin(uint32_t key) {
 // The threshold of one row from its global sample histogram, by one warp.
 // The sample's visible keys (the histogram's total, tot) predict
 // oversample * K * tot / n + 16 of them at or above the row's threshold; the
-// threshold is the lower edge of the highest bin b whose count, with the bins
-// above it, reaches that target; zero (take every key) when the sample's
-// non-negative scores do not reach it.  Zeroes the histogram for the next call.
+// threshold lies in the highest bin b whose count, with the bins above it,
+// reaches that target, where the part of b's count still needed would lie
+// above it were b's keys spread evenly over its key values; zero (take every
+// key) when the sample's non-negative scores do not reach the target.  Any
+// threshold gives the exact result (a short list takes the general path);
+// this one keeps the list near oversample x top_k.  Zeroes the histogram for
+// the next call.
 // `local` is shared memory of kBins words that the warp may overwrite: the
 // loaded histogram goes there, so the second level of the search reads it
 // from shared memory (one round trip to L2 in all).
@@ -190,11 +208,28 @@ __device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversa
         // bins b0 + 1 and b0 in descending order
         const uint32_t run1 = above + inc2 - t + v1;   // keys in bins >= b0 + 1
         const uint32_t run0 = run1 + v0;               // keys in bins >= b0
-        uint32_t mine = 0xFFFFFFFFu;
-        if (run1 >= target) mine = b0 + 1;
-        else if (run0 >= target) mine = b0;
-        uint32_t best = __reduce_max_sync(0xffffffffu, mine == 0xFFFFFFFFu ? 0u : mine + 1);
-        thr = best ? (0x80000000u | ((best - 1) << 20)) : 0u;
+        uint32_t mine = 0xFFFFFFFFu, m_above = 0, m_cnt = 0;
+        if (run1 >= target) {
+            mine = b0 + 1;
+            m_above = run1 - v1;
+            m_cnt = v1;
+        } else if (run0 >= target) {
+            mine = b0;
+            m_above = run0 - v0;
+            m_cnt = v0;
+        }
+        const uint32_t best = __reduce_max_sync(0xffffffffu, mine == 0xFFFFFFFFu ? 0u : mine + 1);
+        if (best) {
+            // inside bin best - 1: the keys above the bins over it fall short
+            // of the target by `need` (1 .. its count cb); the threshold is
+            // put where `need` of its cb keys would lie above it if they were
+            // spread evenly over the bin's 2^20 key values
+            const int owner = __ffs(__ballot_sync(0xffffffffu, mine + 1u == best)) - 1;
+            const uint32_t ab = __shfl_sync(0xffffffffu, m_above, owner);
+            const uint32_t cb = __shfl_sync(0xffffffffu, m_cnt, owner);
+            const uint32_t need = target - ab;
+            thr = (0x80000000u | ((best - 1) << 20)) + (uint32_t)(((uint64_t)(cb - need) << 20) / cb);
+        }
     }
     __syncwarp();
     uint4 *w4 = reinterpret_cast<uint4 *>(hist + lane * kPer);
@@ -206,10 +241,12 @@ __device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversa
 
 // Phase 1: the indexer over this CTA's tiles with sampling and candidate
 // capture (see the file comment).  All kThreads threads call it.  On return
-// nothing is in flight, TMEM is released and the mbarriers are invalidated.
+// nothing is in flight, TMEM is released and the mbarriers are invalidated;
+// keep[0 .. kMaxRows) holds the rows' thresholds if keep[kMaxRows] != 0.
 template <int TQ>
 __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorMap *tmap_ks_p,
-                                    const CUtensorMap *tmap_q_p, const Params &cp, uint8_t *smem, int cta, int ncta) {
+                                    const CUtensorMap *tmap_q_p, const Params &cp, uint8_t *smem, int cta, int ncta,
+                                    uint32_t *keep) {
     using namespace indexer;
     const indexer::Params &p = cp.ix;
     const CUtensorMap &tmap_k = *tmap_k_p, &tmap_ks = *tmap_ks_p, &tmap_q = *tmap_q_p;
@@ -226,8 +263,22 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [rows][kHistStride]
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags
     int32_t *row_qpos = reinterpret_cast<int32_t *>(smem + lay.misc_off + 32);   // [rows] query positions
+    uint32_t *thr_s = reinterpret_cast<uint32_t *>(smem + lay.cap_off);   // [kMaxRows] thresholds, then the flag
+    uint32_t *cx = thr_s + 2 * kMaxRows;               // [group][warp][kMaxRows] a capture step's counts
+    uint32_t *gc = cx + kGroups * kEpiWarps * kMaxRows;   // [group][kMaxRows][2] the lists' lengths
+    uint32_t *dec = gc + kGroups * kMaxRows * 2;       // [group][2] the thresholds are known (by tile parity)
+    constexpr int kCapWords = 2 * kMaxRows + kGroups * (kEpiWarps * kMaxRows + 2 * kMaxRows + 2);
+    // After the sample the histogram area holds the groups' candidate lists:
+    // row r's lists at hist + r * kHistStride, group g's at + g * kGroupCap
+    // entries (order key, position).  List 0 (from the front) takes the keys
+    // of the tiles scored before the thresholds were known, list 1 (from the
+    // back) those of the later tiles: all of list 0's positions come first.
+    auto glist = [&](int r, int g) { return reinterpret_cast<uint2 *>(hist + r * kHistStride) + g * kGroupCap; };
+    static_assert(kGroups * kGroupCap * 8 <= kHistStride * 4, "group lists in the histogram area");
+    static_assert(kGroups * kGroupCap <= kSegCap, "a CTA's group lists fit its segment");
     uint32_t *ctl = cp.ctl;
     const int warp = warp_id(), lane = lane_id();
+    const uint32_t lt = (1u << lane) - 1u;
 
     for (int b = threadIdx.x; b < B; b += blockDim.x) {
         int32_t mx = -1;
@@ -246,6 +297,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     }
     for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
     if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+    for (int j = threadIdx.x; j < kCapWords; j += blockDim.x) thr_s[j] = 0;
     if (threadIdx.x < rows) row_qpos[threadIdx.x] = __ldg(p.q_pos + threadIdx.x);
     __syncthreads();
     if (warp == 0) {
@@ -280,8 +332,13 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         return pipe_begin(pp) + a * (c / GE) + min(a, c % GE) + i / GE;
     };
 
+    // TMEM: the accumulators, then the backlog: the order keys of the first
+    // back_cap tiles of each epilogue group, kept until the thresholds come
+    // (column acc_cols + (group * back_cap + tile) * T + query, lane = key row)
+    const int acc_cols = kPipes * GE * AB * N;
+    const int back_cap = min(kMaxBacklog, (512 - acc_cols) / (kGroups * T));
     uint32_t tmem_cols = 32;
-    while (tmem_cols < (uint32_t)(kPipes * GE * AB * N)) tmem_cols <<= 1;
+    while (tmem_cols < (uint32_t)(acc_cols + kGroups * back_cap * T)) tmem_cols <<= 1;
     if (threadIdx.x == 0) {
         for (int pp = 0; pp < kPipes; ++pp) {
             for (int s = 0; s < S; ++s) {
@@ -322,6 +379,144 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     };
     const uint32_t stage_tx = kTile * kKeyBytes + kTile * 4;
     const bool any_tiles = pipe_count(0) + pipe_count(1) > 0;
+
+    // ---- candidates, by the epilogue groups: group g of the CTA (its four
+    //      warps, rows 32 q .. 32 q + 31 of each of the group's tiles for warp
+    //      q; the groups in position order) keeps its keys at or above their
+    //      row's threshold in its lists, in position order
+    const int ew_c = warp - kEpiWarp0;   // negative for the other warps
+    const int e_gi = ew_c >= 0 ? ew_c / kEpiWarps : 0;
+    const int e_pp = e_gi / kMaxGroups, e_a = e_gi % kMaxGroups;
+    const int e_q = warp & 3;
+    const int e_row = e_q * 32 + lane;   // the lane's row in each tile
+    const int e_bar = kGroupBar0 + e_gi;
+    const int e_ng = ew_c >= 0 && e_a < GE ? group_count(e_pp, e_a) : 0;
+    bool capturing = false;   // the group has the thresholds and takes its candidates
+    // One capture step, by the group's four warps together: of the tile rows
+    // of sequence b at position pos (one per lane), those with bit t of cand
+    // go with key[t] to the end of list li of row b * T + t.
+    auto group_take = [&](int b, int li, uint32_t cand, const uint32_t (&key)[kMaxRows], uint32_t pos) {
+        uint32_t *cxg = cx + e_gi * kEpiWarps * kMaxRows;
+        uint32_t bits[kMaxRows];
+#pragma unroll
+        for (int t = 0; t < kMaxRows; ++t) {
+            bits[t] = t < T ? __ballot_sync(0xffffffffu, (cand >> t) & 1u) : 0u;
+            if (t < T && lane == 0) cxg[e_q * kMaxRows + t] = __popc(bits[t]);
+        }
+        named_bar_sync(e_bar, 128);   // the four warps' counts
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            const int r = b * T + t;
+            if ((cand >> t) & 1u) {
+                uint32_t slot = gc[(e_gi * kMaxRows + r) * 2 + li] + __popc(bits[t] & lt);
+                for (int q2 = 0; q2 < e_q; ++q2) slot += cxg[q2 * kMaxRows + t];
+                if (slot < (uint32_t)kGroupCap)
+                    glist(r, e_gi)[li == 0 ? slot : kGroupCap - 1 - slot] = make_uint2(key[t], pos);
+                const uint32_t bin = min((key[t] - thr_s[r]) >> kCandShift, (uint32_t)(kWide - 1));
+                atomicAdd(cp.cand_hist + (int64_t)r * kWide + bin, 1u);
+            }
+        }
+        named_bar_sync(e_bar, 128);   // every warp has read the counts and lengths
+        if (e_q == 0 && lane == 0) {
+#pragma unroll
+            for (int t = 0; t < T; ++t)
+                gc[(e_gi * kMaxRows + b * T + t) * 2 + li] +=
+                    cxg[t] + cxg[kMaxRows + t] + cxg[2 * kMaxRows + t] + cxg[3 * kMaxRows + t];
+        }
+    };
+    // the group's tiles [j_begin, j_end) again, from the scores its own lanes
+    // stored (a lane reads back only its own stores), a few tiles' loads in
+    // flight at a time; into list 0
+    auto catch_up = [&](int j_begin, int j_end) {
+        constexpr int kB = T <= 2 ? 4 : 2;
+        for (int jb = j_begin; jb < j_end; jb += kB) {
+            float v[kB][T];
+            int32_t ps[kB];   // (positions below 2^31)
+            int bb[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                bb[u] = 0;
+                ps[u] = -1;
+                if (jb + u < j_end) {
+                    int ti;
+                    locate(tile_of(e_pp, (jb + u) * GE + e_a), bb[u], ti);
+                    ps[u] = ti * kTile + e_row;
+                    if (ps[u] >= seq_len[bb[u]]) ps[u] = -1;
+                }
+#pragma unroll
+                for (int t = 0; t < T; ++t)
+                    v[u][t] = ps[u] >= 0 ? p.scores[((int64_t)bb[u] * T + t) * p.scores_stride + ps[u]] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                if (jb + u < j_end) {   // uniform in the group
+                    uint32_t key[kMaxRows] = {0u, 0u, 0u, 0u}, cand = 0u;
+#pragma unroll
+                    for (int t = 0; t < T; ++t) {
+                        const int r = bb[u] * T + t;
+                        key[t] = float_order_key(v[u][t]);
+                        if (ps[u] >= 0 && ps[u] <= row_qpos[r] && key[t] >= thr_s[r]) cand |= 1u << t;
+                    }
+                    group_take(bb[u], 0, cand, key, (uint32_t)ps[u]);
+                }
+            }
+        }
+    };
+    // The group's backlog: its tiles [0, j_now), scored before the thresholds
+    // were known; the first back_cap of them from TMEM now, the rest (if any)
+    // from its own stored scores after the stream.
+    int glob_lo = 0, glob_hi = 0;
+    auto transition = [&](int j_now) {
+        capturing = true;
+        const int nb = min(j_now, back_cap);
+        for (int jj = 0; jj < nb; ++jj) {
+            int bb, ti;
+            locate(tile_of(e_pp, jj * GE + e_a), bb, ti);
+            const int ps = ti * kTile + e_row;
+            uint32_t key[kMaxRows] = {0u, 0u, 0u, 0u}, cand = 0u;
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                const int r = bb * T + t;
+                key[t] = tmem_ld1(tmem_base + ((uint32_t)(e_q * 32) << 16) +
+                                  (uint32_t)(acc_cols + (e_gi * back_cap + jj) * T + t));
+                if (ps < seq_len[bb] && ps <= row_qpos[r] && key[t] >= thr_s[r]) cand |= 1u << t;
+            }
+            group_take(bb, 0, cand, key, (uint32_t)ps);
+        }
+        glob_lo = nb;
+        glob_hi = j_now;
+    };
+    // the thresholds from their packed words (all rows published), into
+    // shared memory for the CTA's warps
+    const uint64_t *packed = reinterpret_cast<const uint64_t *>(ctl + kThrPacked);
+    auto all_published = [&](const uint64_t (&w)[kMaxRows]) {
+        bool ok = true;
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r)
+            if (r < rows) ok &= (w[r] >> 32) != 0u;
+        return ok;
+    };
+    auto wait_packed = [&](uint64_t (&w)[kMaxRows]) {   // bounded
+        const uint64_t t0 = globaltimer_ns();
+        for (;;) {
+#pragma unroll
+            for (int r = 0; r < kMaxRows; ++r) w[r] = r < rows ? ld_relaxed_gpu_u64(packed + r) : 0ull;
+            if (all_published(w)) return true;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                flag_timeout(p.status);
+                return false;
+            }
+            __nanosleep(64);
+        }
+    };
+    auto publish = [&](const uint64_t (&w)[kMaxRows]) {
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r)
+            if (r < rows) thr_s[r] = (uint32_t)w[r];
+        __threadfence_block();
+        *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows) = 1u;
+        if (cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
+    };
 
     if (warp < kPipes) {
         // ------------------------------------------------------------ producer
@@ -412,8 +607,11 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         const bool poller = quarter == 0 && lane == 0;
         bool ok = true;
         int cur_b = -1;
+        bool polling = false;   // the poller's read of the packed words is in flight
+        uint32_t *poll = reinterpret_cast<uint32_t *>(smem + lay.poll_off) + gi * 2 * kMaxRows;
         for (int j = 0; j < ng || j == 0; ++j) {
             const bool have = j < ng;
+            bool scored = false;
             float sc[kMaxRows] = {0.f, 0.f, 0.f, 0.f};
             uint32_t vis = 0;
             int b = 0;
@@ -435,6 +633,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 bool w_ok = mbar_wait(&bars->tfull[pp][a][u], (j / AB) & 1, p.status) &&
                             mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status);
                 if (__all_sync(0xffffffffu, w_ok)) {
+                    scored = true;
                     if (j == 0 && gi == 0 && poller && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 12] = globaltimer_ns();
                     tc_fence_after();
                     const float ks = *reinterpret_cast<const float *>(smem + lay.ks_off + st * kKsStageBytes +
@@ -456,6 +655,13 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             if (pos < len) out[(int64_t)t * p.scores_stride] = visible ? sc[t] : -INFINITY;
                             if (visible) vis |= 1u << t;
                         }
+                    }
+                    if (!capturing && j < back_cap) {   // the backlog's keys wait in TMEM
+#pragma unroll
+                        for (int t = 0; t < T; ++t)
+                            tmem_st1(tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                         (uint32_t)(acc_cols + (gi * back_cap + j) * T + t),
+                                     float_order_key(sc[t]));
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -508,7 +714,11 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                             } else {
                                 for (int u = lane; u < kHistWords; u += 32) h[u] = 0;
                             }
-                            if (lane == 0) ctl[kThr + r] = t_r;
+                            if (lane == 0) {
+                                ctl[kThr + r] = t_r;
+                                st_relaxed_gpu_u64(reinterpret_cast<uint64_t *>(ctl + kThrPacked) + r,
+                                                   (1ull << 32) | t_r);
+                            }
                         }
                         named_bar_sync(gbar, 128);   // the thresholds, before the release that publishes them
                         if (quarter == 0 && lane == 0) {
@@ -517,6 +727,60 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         }
                     }
                 }
+            }
+            // ---- this tile's candidates, once the CTA has the thresholds (never
+            //      at j == 0: they need this CTA's sample).  The poller copies
+            //      the packed words into shared memory asynchronously and looks
+            //      at the copy one tile later, so it never waits for it.
+            if (!capturing) {
+                if (poller) {
+                    if (polling) {
+                        attn::cp_async_wait_all();   // (long done)
+                        uint64_t w[kMaxRows];
+#pragma unroll
+                        for (int r = 0; r < kMaxRows; ++r)
+                            w[r] = (uint64_t)poll[2 * r] | ((uint64_t)poll[2 * r + 1] << 32);
+                        if (all_published(w)) publish(w);
+                        polling = false;
+                    }
+                    if (j + 1 < ng && *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows) == 0u) {
+                        for (int r2 = 0; r2 < rows; r2 += 2) attn::cp_async16(poll + 2 * r2, packed + r2);
+                        attn::cp_async_commit();
+                        polling = true;
+                    }
+                }
+                // one decision for the group's four warps (a slot per tile parity)
+                if (poller) dec[gi * 2 + (j & 1)] = *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows);
+                named_bar_sync(gbar, 128);
+                if (*reinterpret_cast<volatile uint32_t *>(dec + gi * 2 + (j & 1)) != 0u) {
+                    __threadfence_block();
+                    transition(j);   // the tiles before this one
+                }
+            }
+            if (capturing) {
+                uint32_t key[kMaxRows] = {0u, 0u, 0u, 0u}, cand = 0u;
+#pragma unroll
+                for (int t = 0; t < T; ++t) {
+                    key[t] = float_order_key(sc[t]);
+                    if (scored && ((vis >> t) & 1u) && key[t] >= thr_s[b * T + t]) cand |= 1u << t;
+                }
+                group_take(b, 1, cand, key, (uint32_t)pos);
+            }
+        }
+        if (polling) attn::cp_async_wait_all();
+        // ---- after the group's tiles: warps still without the thresholds wait
+        //      for them here, while their backlog is in TMEM
+        if (ng > 0) {
+            bool okw = true;
+            if (poller && *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows) == 0u) {
+                uint64_t w[kMaxRows];
+                okw = wait_packed(w);
+                if (okw) publish(w);
+            }
+            okw = named_bar_and(gbar, 128, okw);
+            if (okw && !capturing) {
+                __threadfence_block();
+                transition(ng);
             }
         }
     }
@@ -547,148 +811,51 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     __syncthreads();
     if (cp.trace && threadIdx.x == 0) cp.trace[cta * DSA_TRACE_MARKS + 2] = globaltimer_ns();
 
-    // ---- the CTA's candidates: every visible key of its tiles whose score
-    //      is at or above its row's threshold, in position order, into the
-    //      CTA's segment of the row's list (the scores are this CTA's own
-    //      stores, in L2).  Pair q = t * n_tiles + i is query t of tile i.
-    uint32_t *cnt = reinterpret_cast<uint32_t *>(smem);      // [P] candidates per pair
-    uint32_t *pref = cnt + kThreads;                          // [P] exclusive prefix of cnt
+    // ---- the CTA's candidates: the warps that did not see the thresholds
+    //      during the stream take theirs now; the warps' lists are merged
+    //      into the CTA's segment of each row's list, in position order
     bool r_ok = true;
-    if (threadIdx.x == 0 && n_tiles > 0) r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);
+    if (threadIdx.x == 0 && n_tiles > 0 && thr_s[kMaxRows] == 0u) {
+        r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);   // (acquire)
+        if (r_ok) {
+            for (int r = 0; r < rows; ++r) thr_s[r] = ld_relaxed_gpu(ctl + kThr + r);
+            thr_s[kMaxRows] = 1u;
+            if (cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
+        }
+    }
     if (!__syncthreads_and(r_ok)) return;   // the timeout is in the status word; the grid barrier sees it
-    if (cp.trace && threadIdx.x == 0) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
-    uint32_t thr[kMaxRows];
-#pragma unroll
-    for (int r = 0; r < kMaxRows; ++r) thr[r] = r < rows ? __ldcg(ctl + kThr + r) : 0xFFFFFFFFu;
-    const int P = n_tiles * T;   // <= kThreads (plan_capture)
-    // Pairs are taken kQP per warp at a time with every score load in flight
-    // before the first ballot: lane l holds key 32 k + l of each pair's tile.
-    constexpr int kQP = 4;
-    static_assert(kTile / 32 == 4, "four 32-key strips per tile");
-    struct PairKeys {
-        uint32_t key[kQP][kTile / 32];
-        uint32_t cand;      // bit qq * 4 + k: key k of pair qq is a candidate
-        int r[kQP];
-        int64_t pos0[kQP];
-    };
-    auto load_pairs = [&](int q0, PairKeys &pk) {
-        pk.cand = 0;
-#pragma unroll
-        for (int qq = 0; qq < kQP; ++qq) {
-            const int q = q0 + qq * kWarps;
-            pk.r[qq] = 0;
-            pk.pos0[qq] = 0;
-#pragma unroll
-            for (int k = 0; k < kTile / 32; ++k) pk.key[qq][k] = 0u;
-            if (q < P) {
-                const int i = q % n_tiles, t = q / n_tiles;
-                int b, ti;
-                locate(t_begin + i, b, ti);
-                const int r = b * T + t;
-                pk.r[qq] = r;
-                pk.pos0[qq] = (int64_t)ti * kTile;
-                const int64_t lim = min((int64_t)seq_len[b] - 1, (int64_t)row_qpos[r]);   // last visible
-                const float *src = p.scores + (int64_t)r * p.scores_stride + pk.pos0[qq];
-#pragma unroll
-                for (int k = 0; k < kTile / 32; ++k) {
-                    const int64_t pos = pk.pos0[qq] + k * 32 + lane;
-                    if (pos <= lim) {
-                        pk.key[qq][k] = float_order_key(__ldcg(src + k * 32 + lane));
-                        pk.cand |= 1u << (qq * 4 + k);
-                    }
-                }
-            }
-        }
-        // visible -> candidate: at or above the row's threshold
-#pragma unroll
-        for (int qq = 0; qq < kQP; ++qq) {
-            uint32_t th = 0xFFFFFFFFu;
-#pragma unroll
-            for (int rr = 0; rr < kMaxRows; ++rr)
-                if (rr == pk.r[qq]) th = thr[rr];
-#pragma unroll
-            for (int k = 0; k < kTile / 32; ++k)
-                if (pk.key[qq][k] < th) pk.cand &= ~(1u << (qq * 4 + k));
-        }
-    };
-    const bool one_batch = P <= kWarps * kQP;   // then pass 2 reuses pass 1's keys
-    PairKeys kept;
-    for (int q0 = warp; q0 < P; q0 += kWarps * kQP) {
-        PairKeys pk;
-        load_pairs(q0, pk);
-        if (one_batch) kept = pk;
-#pragma unroll
-        for (int qq = 0; qq < kQP; ++qq) {
-            uint32_t c = 0;
-#pragma unroll
-            for (int k = 0; k < kTile / 32; ++k) c += __popc(__ballot_sync(0xffffffffu, (pk.cand >> (qq * 4 + k)) & 1u));
-            const int q = q0 + qq * kWarps;
-            if (lane == 0 && q < P) cnt[q] = c;
-        }
-    }
+    if (ew_c >= 0 && glob_hi > glob_lo) catch_up(glob_lo, glob_hi);   // backlog tiles TMEM did not hold
     __syncthreads();
-    {
-        const uint32_t v = (int)threadIdx.x < P ? cnt[threadIdx.x] : 0u;
-        uint32_t total;
-        auto *sh = reinterpret_cast<topk::Shared<kThreads> *>(pref + kThreads);
-        const uint32_t incl = topk::block_scan<kThreads>(v, sh->warp_tmp, &total);
-        if ((int)threadIdx.x < P) pref[threadIdx.x] = incl - v;
-    }
-    __syncthreads();
-    // the pairs of row r = b * T + t in this CTA: t * n_tiles + [i0, i1), the tiles of sequence b
-    auto row_span = [&](int r, int &q0, int &q1) {
-        const int b = r / T, t = r % T;
-        const int i0 = min(n_tiles, max(0, tile_pre[b] - t_begin));
-        const int i1 = min(n_tiles, max(0, tile_pre[b + 1] - t_begin));
-        q0 = t * n_tiles + i0;
-        q1 = t * n_tiles + i1;
-    };
-    bool overflow = false;
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int q0 = warp; q0 < P; q0 += kWarps * kQP) {
-        PairKeys pk;
-        if (one_batch) pk = kept;
-        else load_pairs(q0, pk);   // again: the scores are in L2
-#pragma unroll
-        for (int qq = 0; qq < kQP; ++qq) {
-            const int q = q0 + qq * kWarps;
-            if (q < P) {   // warp-uniform
-                int rq0, rq1;
-                row_span(pk.r[qq], rq0, rq1);
-                uint32_t at = pref[q] - pref[rq0];
-#pragma unroll
-                for (int k = 0; k < kTile / 32; ++k) {
-                    const bool cand = (pk.cand >> (qq * 4 + k)) & 1u;
-                    const uint32_t bits = __ballot_sync(0xffffffffu, cand);
-                    if (cand) {
-                        const uint32_t slot = at + __popc(bits & lt);
-                        if (slot < (uint32_t)kSegCap)
-                            cp.lists[((int64_t)pk.r[qq] * cp.NG + cta) * kSegCap + slot] =
-                                make_uint2(pk.key[qq][k], (uint32_t)(pk.pos0[qq] + k * 32 + lane));
-                        else
-                            overflow = true;
-                        uint32_t th = 0u;
-#pragma unroll
-                        for (int rr = 0; rr < kMaxRows; ++rr)
-                            if (rr == pk.r[qq]) th = thr[rr];
-                        const uint32_t bin = min((pk.key[qq][k] - th) >> kCandShift, (uint32_t)(kWide - 1));
-                        atomicAdd(cp.cand_hist + (int64_t)pk.r[qq] * kWide + bin, 1u);
-                    }
-                    at += __popc(bits);
-                }
+    // the CTA's segment of row r: for each group in turn, its list 0, then
+    // its list 1 (stored from the back), by the group's four warps
+    if (ew_c >= 0) {
+        for (int r = 0; r < rows; ++r) {
+            uint32_t at = 0;
+            for (int g2 = 0; g2 < e_gi; ++g2) at += gc[(g2 * kMaxRows + r) * 2] + gc[(g2 * kMaxRows + r) * 2 + 1];
+            const uint32_t n0 = gc[(e_gi * kMaxRows + r) * 2], n1 = gc[(e_gi * kMaxRows + r) * 2 + 1];
+            if (at + n0 + n1 <= (uint32_t)kSegCap && n0 + n1 <= (uint32_t)kGroupCap) {
+                const uint2 *L = glist(r, e_gi);
+                uint2 *seg = cp.lists + ((int64_t)r * cp.NG + cta) * kSegCap + at;
+                for (uint32_t i = e_q * 32 + lane; i < n0 + n1; i += kEpiWarps * 32)
+                    seg[i] = i < n0 ? L[i] : L[kGroupCap - 1 - (i - n0)];
             }
         }
     }
-    if (__any_sync(0xffffffffu, overflow) && lane == 0) atomicOr(ctl + kOverflow, 1u);
     if ((int)threadIdx.x < rows) {   // the row's count in this CTA
         const int r = threadIdx.x;
-        int q0, q1;
-        row_span(r, q0, q1);
-        const uint32_t total = q1 > q0 ? pref[q1 - 1] + cnt[q1 - 1] - pref[q0] : 0u;
-        cp.counts[(int64_t)r * cp.NG + cta] = total;
-        if (total) atomicAdd(ctl + kTotal + r, total);
-        if (total > (uint32_t)kSegCap) atomicOr(ctl + kOverflow, 1u);
+        uint32_t total = 0;
+        bool over = false;
+        for (int g2 = 0; g2 < kGroups; ++g2) {
+            const uint32_t c = gc[(g2 * kMaxRows + r) * 2] + gc[(g2 * kMaxRows + r) * 2 + 1];
+            over |= c > (uint32_t)kGroupCap;
+            total += c;
+        }
+        over |= total > (uint32_t)kSegCap;
+        cp.counts[(int64_t)r * cp.NG + cta] = over ? 0u : total;
+        if (total && !over) atomicAdd(ctl + kTotal + r, total);
+        if (over) atomicOr(ctl + kOverflow, 1u);
     }
+    if ((int)threadIdx.x <= kMaxRows) keep[threadIdx.x] = thr_s[threadIdx.x];   // the thresholds and their flag
 }
 
 // One slice of the combine of (row bt, KV group g), by the 128 threads of a
@@ -717,20 +884,33 @@ __device__ void combine_piece(const Params &cp, int bt, int g, int piece, int ti
         ls[i] = ml.y;
     }
     attn::team_sync(bar);
-    if (tid < nh) {
-        const int h = g * hpg + h_lo + tid;
-        const float sk = cp.sink ? __ldg(cp.sink + h) * attn::kLog2e : -INFINITY;
-        float M = sk;
-        for (int j = 0; j < splits; ++j) M = fmaxf(M, w[tid * splits + j]);
-        float L = (cp.sink && M != -INFINITY) ? exp2f(sk - M) : 0.f;
-        for (int j = 0; j < splits; ++j) {
-            const float m = w[tid * splits + j];
+    {   // per head, one warp: split j on lane j; the max is exact in any
+        // order, and lane 0 sums the denominator's terms in split order
+        const int wq = tid >> 5, ln = tid & 31;
+        for (int hh = wq; hh < nh; hh += 4) {
+            const int h = g * hpg + h_lo + hh;
+            const float sk = cp.sink ? __ldg(cp.sink + h) * attn::kLog2e : -INFINITY;
+            const bool on = ln < splits;
+            const float m = on ? w[hh * splits + ln] : -INFINITY;
+            float M = m;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            M = fmaxf(M, sk);
             const float wj = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
-            L = __fadd_rn(L, wj != 0.f ? __fmul_rn(ls[tid * splits + j], wj) : 0.f);
-            w[tid * splits + j] = wj;
+            if (on) {
+                const float lj = ls[hh * splits + ln];
+                w[hh * splits + ln] = wj;
+                ls[hh * splits + ln] = wj != 0.f ? __fmul_rn(lj, wj) : 0.f;
+            }
+            __syncwarp();
+            if (ln == 0) {
+                float L = (cp.sink && M != -INFINITY) ? exp2f(sk - M) : 0.f;
+#pragma unroll 8
+                for (int j = 0; j < splits; ++j) L = __fadd_rn(L, ls[hh * splits + j]);
+                hs[2 * hh] = M;
+                hs[2 * hh + 1] = L;
+            }
         }
-        hs[2 * tid] = M;
-        hs[2 * tid + 1] = L;
     }
     attn::team_sync(bar);
     for (int e = lo + tid; e < hi; e += 128) {
@@ -757,8 +937,11 @@ __device__ void combine_piece(const Params &cp, int bt, int g, int piece, int ti
 
 // Phase 2 (fast): the exact selection of row r from its candidates, into
 // `sel` (shared, top_k entries, -1 padded) and, by CTA c == 0, into the
-// output.  `work` is shared memory for the list.  Called by all threads.
-__device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *sel, uint8_t *work, uint64_t *trace) {
+// output.  `work` is shared memory for the list.  Called by all threads;
+// thread t < NG passes the length of CTA t's segment of the row (seg_len),
+// and keep holds the thresholds kept from phase 1 (see run_indexer_capture).
+__device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *sel, uint8_t *work, uint64_t *trace,
+                                       uint32_t seg_len, const uint32_t *keep) {
     constexpr int NT = kThreads, NW = NT / 32;
     const int K = cp.K, NG = cp.NG;
     const int lane = lane_id(), warp = warp_id();
@@ -784,7 +967,7 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             mbar_init(copied, 1);
             fence_mbar_init();
         }
-        const uint32_t v = threadIdx.x < NG ? __ldcg(cp.counts + (int64_t)r * NG + threadIdx.x) : 0u;
+        const uint32_t v = (int)threadIdx.x < NG ? seg_len : 0u;
         const uint32_t vp = (v + 1u) & ~1u;
         uint32_t m;   // entries, pads included
         const uint32_t incl = topk::block_scan<NT>(vp, sh->warp_tmp, &m);
@@ -866,15 +1049,26 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         auto gather_keys = [&](auto pred) {
             if (threadIdx.x == 0) sh->total = 0;
             __syncthreads();
-            for (uint32_t jb = threadIdx.x & ~31u; jb < m; jb += NT) {
-                const uint32_t j = jb + lane;
-                uint32_t k = 0u;
-                const bool take = j < m && is_key(j, k) && pred(k);
-                const uint32_t bits = __ballot_sync(0xffffffffu, take);
-                uint32_t at = 0;
-                if (lane == 0 && bits) at = atomicAdd(&sh->total, (uint32_t)__popc(bits));
-                at = __shfl_sync(0xffffffffu, at, 0);
-                if (take && at + __popc(bits & lt) < (uint32_t)kSmall) bin_keys[at + __popc(bits & lt)] = k;
+            constexpr uint32_t kG = 4;   // strips whose loads are in flight together
+            for (uint32_t jb = threadIdx.x & ~31u; jb < m; jb += kG * NT) {
+                uint32_t kk[kG];
+                bool tk[kG];
+#pragma unroll
+                for (uint32_t u = 0; u < kG; ++u) {
+                    const uint32_t j = jb + u * NT + lane;
+                    kk[u] = 0u;
+                    tk[u] = j < m && is_key(j, kk[u]) && pred(kk[u]);
+                }
+#pragma unroll
+                for (uint32_t u = 0; u < kG; ++u) {
+                    const uint32_t bits = __ballot_sync(0xffffffffu, tk[u]);
+                    if (bits) {
+                        uint32_t at = 0;
+                        if (lane == 0) at = atomicAdd(&sh->total, (uint32_t)__popc(bits));
+                        at = __shfl_sync(0xffffffffu, at, 0) + __popc(bits & lt);
+                        if (tk[u] && at < (uint32_t)kSmall) bin_keys[at] = kk[u];
+                    }
+                }
             }
             __syncthreads();
             const uint32_t n_keys = sh->total;
@@ -884,7 +1078,7 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         uint32_t Tstar = 0u, ties = 0u;
         bool found = false;
         {   // from the stream's histogram of the row's candidates above its threshold
-            const uint32_t thr_r = __ldcg(cp.ctl + kThr + r);
+            const uint32_t thr_r = keep[kMaxRows] ? keep[r] : __ldcg(cp.ctl + kThr + r);
             find_bin();
             const int B = sh->bin;
             const uint32_t Kb = (uint32_t)K - sh->above, in_b = wide[B];
@@ -974,12 +1168,22 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         // to it, each at (keys above before it) + min(equal keys before it, ties)
         const uint32_t strips = (m + 31) / 32, per_w = (strips + NW - 1) / NW;
         const uint32_t s0 = min(strips, (uint32_t)warp * per_w), s1 = min(strips, s0 + per_w);
+        // (four strips' loads in flight at a time)
+        constexpr uint32_t kU = 4;
         uint32_t gt = 0, eq = 0;
-        for (uint32_t q = s0; q < s1; ++q) {
-            const uint32_t j = q * 32 + lane;
-            const uint32_t k = j < m ? list[j].x : 0u;
-            gt += __popc(__ballot_sync(0xffffffffu, j < m && k > Tstar));
-            eq += __popc(__ballot_sync(0xffffffffu, j < m && k == Tstar));
+        for (uint32_t q = s0; q < s1; q += kU) {
+            uint32_t k[kU];
+#pragma unroll
+            for (uint32_t u = 0; u < kU; ++u) {
+                const uint32_t j = (q + u) * 32 + lane;
+                k[u] = q + u < s1 && j < m ? list[j].x : 0u;
+            }
+#pragma unroll
+            for (uint32_t u = 0; u < kU; ++u) {
+                const bool in = q + u < s1 && (q + u) * 32 + lane < m;
+                gt += __popc(__ballot_sync(0xffffffffu, in && k[u] > Tstar));
+                eq += __popc(__ballot_sync(0xffffffffu, in && k[u] == Tstar));
+            }
         }
         if (lane == 0) {
             sh->warp_a[warp] = gt;
@@ -991,17 +1195,25 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             gb += sh->warp_a[w2];
             eb += sh->warp_b[w2];
         }
-        for (uint32_t q = s0; q < s1; ++q) {
-            const uint32_t j = q * 32 + lane;
-            const bool in = j < m;
-            const uint2 e = in ? list[j] : make_uint2(0u, 0u);
-            const uint32_t bg = __ballot_sync(0xffffffffu, in && e.x > Tstar);
-            const uint32_t be = __ballot_sync(0xffffffffu, in && e.x == Tstar);
-            const uint32_t g_before = gb + __popc(bg & lt), e_before = eb + __popc(be & lt);
-            if (in && e.x > Tstar) sel[g_before + (e_before < ties ? e_before : ties)] = (int32_t)e.y;
-            else if (in && e.x == Tstar && e_before < ties) sel[g_before + e_before] = (int32_t)e.y;
-            gb += __popc(bg);
-            eb += __popc(be);
+        for (uint32_t q = s0; q < s1; q += kU) {
+            uint2 ent[kU];
+#pragma unroll
+            for (uint32_t u = 0; u < kU; ++u) {
+                const uint32_t j = (q + u) * 32 + lane;
+                ent[u] = q + u < s1 && j < m ? list[j] : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (uint32_t u = 0; u < kU; ++u) {
+                const bool in = q + u < s1 && (q + u) * 32 + lane < m;
+                const uint2 e = ent[u];
+                const uint32_t bg = __ballot_sync(0xffffffffu, in && e.x > Tstar);
+                const uint32_t be = __ballot_sync(0xffffffffu, in && e.x == Tstar);
+                const uint32_t g_before = gb + __popc(bg & lt), e_before = eb + __popc(be & lt);
+                if (in && e.x > Tstar) sel[g_before + (e_before < ties ? e_before : ties)] = (int32_t)e.y;
+                else if (in && e.x == Tstar && e_before < ties) sel[g_before + e_before] = (int32_t)e.y;
+                gb += __popc(bg);
+                eb += __popc(be);
+            }
         }
         for (int j = kr + threadIdx.x; j < K; j += NT) sel[j] = -1;
     }
@@ -1021,6 +1233,8 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     __shared__ uint32_t sync_flag;
+    __shared__ uint32_t thr_keep[kMaxRows + 1];
+    if (threadIdx.x == 0) thr_keep[kMaxRows] = 0u;
     pdl_begin();
     const uint32_t G = gridDim.x;
     uint32_t *status = cp.ix.status;
@@ -1037,7 +1251,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     }
 
     // ---- phase 1: key stream, sample, candidates
-    run_indexer_capture<TQ>(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G);
+    run_indexer_capture<TQ>(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G, thr_keep);
     mark(15);
     if (status_at_entry & kNeedsInitBit) {
         if (threadIdx.x == 0) flag_timeout(status);
@@ -1046,7 +1260,13 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     if (!grid_sync(ctl + kGridArrive, 1 * G, cp.bar, status, &sync_flag)) return;
     mark(3);
 
-    // the sample was good for every row? (the same answer in every CTA)
+    const int rows = cp.rows, C = cp.C;
+    // this CTA's row's segment lengths, loaded together with the words that
+    // decide the path: the sample was good for every row? (the same answer
+    // in every CTA)
+    uint32_t seg_len = 0u;
+    if ((int)blockIdx.x < rows * C && (int)threadIdx.x < cp.NG)
+        seg_len = __ldcg(cp.counts + (int64_t)(blockIdx.x / C) * cp.NG + threadIdx.x);
     bool fast = __ldcg(ctl + kOverflow) == 0u;
     for (int r = 0; r < cp.rows; ++r) {
         const int64_t n = (int64_t)__ldg(cp.ix.q_pos + r) + 1;
@@ -1059,7 +1279,6 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
         atomicAdd(cp.path_count + (fast ? 0 : 1), 1u);
     }
 
-    const int rows = cp.rows, C = cp.C;
     const int G_kv = cp.at.G, splits = cp.at.splits, nt = cp.at.n_teams;
     const attn::TeamSmem teams{smem + (fast ? kSelBytes : 0), (uint32_t)align128(sizeof(attn::Smem))};
     if (fast) {
@@ -1071,7 +1290,7 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
         if ((int)blockIdx.x < rows * C && (int)(blockIdx.x % C) < upr) {
             const int r = blockIdx.x / C, c = blockIdx.x % C;
             int32_t *sel = reinterpret_cast<int32_t *>(smem);
-            select_from_candidates(cp, r, c, sel, smem + kSelBytes, trace);
+            select_from_candidates(cp, r, c, sel, smem + kSelBytes, trace, seg_len, thr_keep);
             mark(4);
             if (nt == 1) {
                 const int tm = threadIdx.x >> 7, tid = threadIdx.x & 127;
@@ -1157,6 +1376,8 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
             for (int r = 0; r < kMaxRows; ++r) {
                 ctl[kTotal + r] = 0;
                 ctl[kThr + r] = 0;
+                ctl[kThrPacked + 2 * r] = 0;
+                ctl[kThrPacked + 2 * r + 1] = 0;
             }
             for (int i = 0; i < rows * DSA_Q_HEADS; ++i) ctl[kCombine + i] = 0;
         }
@@ -1199,11 +1420,6 @@ int plan_capture(int B, int T, int64_t Lmax, int top_k, CapturePlan *plan) {
     if (dev.num_sms <= 0 || rows > kMaxRows || T > kMaxRows || Lmax < kMinContext) return DSA_OK;
     const int grid = dev.num_sms;
     if (grid > kThreads) return DSA_OK;   // the segment offsets are scanned one per thread
-    // a CTA's (tile, query) pairs are counted one per thread after the stream
-    {
-        const int64_t tiles = (int64_t)B * ((Lmax + indexer::kTile - 1) / indexer::kTile);
-        if ((tiles + grid - 1) / grid * T > kThreads) return DSA_OK;
-    }
     // all CTAs must be resident together: one per SM (occupancy asked once per device)
     static std::mutex mu;
     static int per_sm_cache[64];

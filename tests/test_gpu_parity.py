@@ -280,12 +280,17 @@ def test_layer_decode_is_deterministic():
                            y.view(torch.uint8) if y.dtype == torch.bfloat16 else y)
 
 
-@pytest.mark.parametrize("seq_lens,T,page_size", [([65536], 4, 0), ([3000, 9000], 2, 64), ([20000] * 5, 4, 0)])
+@pytest.mark.parametrize("seq_lens,T,page_size", [([65536], 4, 0), ([3000, 9000], 2, 64), ([20000] * 5, 4, 0),
+                                                   ([40000], 3, 0), ([12000, 30000, 9000, 20000], 1, 64)])
 def test_layer_decode_equals_separate_calls(seq_lens, T, page_size):
-    """dsa_layer_decode (one fused launch for B*T <= 16 rows, separate kernels
-    above) gives exactly what the three separate entry points give."""
+    """dsa_layer_decode (the one-barrier kernel for up to four long rows, one
+    fused launch for B*T <= 16 rows, separate kernels above) gives exactly
+    what the three separate entry points give: three and four query rows of
+    one sequence, and four sequences of one row each, take the one-barrier
+    kernel."""
     wl = make_decode_workload(seed=80, seq_lens=seq_lens, T=T, device=DEV, page_size=page_size, n_needles=8)
     O, lse, idx, cnt = run_layer(wl)
+    assert sum(LAST_PATHS) == (1 if wl.B * T <= 4 else 0)   # the one-barrier kernel ran once, or not at all
     Lmax = int(wl.q_pos.max()) + 1
     scores = run_indexer(wl, Lmax)
     idx2, cnt2 = run_topk(scores, wl.q_pos, 2048)
