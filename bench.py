@@ -760,7 +760,7 @@ def run_ours(args, rank, world, local_rank):
     read_gbs = read_stream_gbps(torch, dev, stream)
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush)
+    e2e = run_e2e(args, dsa, torch, layers, dev, stream, sm_scale, ws, flush)
 
     tokens = B * T
     value = throughput(tokens, K, world, total_s)
@@ -875,7 +875,7 @@ def trace_phases(dsa, torch, dev, step, R, n=8):
     return out
 
 
-def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
+def run_e2e(args, dsa, torch, layers, dev, stream, sm_scale, ws, flush):
     """Same metric through the public API with host buffers.  Per step, the new
     token's raw inputs -- its index query (16 heads) and index key before
     normalisation, RoPE and fp8 (bf16), the head weights, the backbone query,
@@ -883,7 +883,12 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
     from pinned memory; dsa_index_produce normalises, rotates and quantises the
     index key into the cache row and the index queries into their e4m3 codes;
     the K / V rows are written into the cache; the layer-step runs; the output
-    and the selection come back to the host in one copy."""
+    and the selection come back to the host in one copy.  The steps run back to
+    back over the layers' caches in rotation, as the headline's do (inputs
+    larger than L2), with every step's two copies inside the timed region; the
+    same step isolated (L2 flushed, events around it) is reported beside."""
+    wl = layers[0][0]
+    R = len(layers)
     B, T = wl.B, wl.T
     L = wl.layout.seq_lens[0]
     G = wl.G
@@ -929,70 +934,83 @@ def run_e2e(args, dsa, torch, wl, kv, dev, stream, sm_scale, ws, flush):
     h2d = off
     d2h = o_bytes + i_bytes
 
-    def step():
+    def step(i=0):
+        w_i, kv_i = layers[i % R]
         d_in.copy_(h_in, non_blocking=True)
-        dsa.dsa_index_produce(d_kin, d_qin, ln_w, ln_b, 1e-5, 42, 1e7, kv, d_pos, q8, qs, ws_p)
-        wl.K[row].copy_(d_K, non_blocking=True)
-        wl.V[row].copy_(d_V, non_blocking=True)
-        dsa.dsa_layer_decode(q8, qs, d_w, d_Q, kv, d_pos, L, TOP_K, wl.sink, sm_scale, O, None, idx, cnt, ws)
+        dsa.dsa_index_produce(d_kin, d_qin, ln_w, ln_b, 1e-5, 42, 1e7, kv_i, d_pos, q8, qs, ws_p)
+        w_i.K[row].copy_(d_K, non_blocking=True)
+        w_i.V[row].copy_(d_V, non_blocking=True)
+        dsa.dsa_layer_decode(q8, qs, d_w, d_Q, kv_i, d_pos, L, TOP_K, w_i.sink, sm_scale, O, None, idx, cnt, ws)
         h_out.copy_(d_out, non_blocking=True)
 
-    for _ in range(max(3, args.warmup)):
-        flush()
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i)
     torch.cuda.synchronize(dev)
-    K = args.steps
+    K = max(R, args.steps // R * R)
 
-    def timed(run):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-        barrier(dev)
-        torch.cuda.synchronize(dev)
-        for i in range(K):
-            flush()
-            evs[i][0].record(stream)
-            run()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(dev)
-        return evs
+    # the same step isolated: L2 flushed, events around the one step (eager)
+    K_iso = min(K, 50)
+    iso = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_iso)]
+    for i in range(K_iso):
+        flush()
+        iso[i][0].record(stream)
+        step(0)
+        iso[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    iso_ms = statistics.median([a.elapsed_time(b) for a, b in iso])
 
-    eager = timed(step)
-    eager_ms = statistics.median([a.elapsed_time(b) for a, b in eager])
-    # the step captured once into a CUDA graph (copies, producer, cache writes,
-    # layer-step, copy back) and replayed: one launch per step from the host
-    graph_note = "captured once in a CUDA graph, replayed per step"
+    # the R steps captured once into a CUDA graph (copies, producer, cache
+    # writes, layer-step, copy back), replayed K / R times back to back
+    graph_note = f"{R} layers' steps captured once in a CUDA graph, replayed back to back"
+    graph = None
     try:
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
-            step()   # one more warm-up on the capture stream
+            for i in range(R):
+                step(i)   # one more warm-up on the capture stream
         stream.wait_stream(side)
         torch.cuda.synchronize(dev)
         with torch.cuda.graph(graph):
-            step()
+            for i in range(R):
+                step(i)
         torch.cuda.synchronize(dev)
-        for _ in range(3):
+        for _ in range(2):
             graph.replay()
         torch.cuda.synchronize(dev)
-        evs = timed(graph.replay)
-    except Exception as e:   # a launch that cannot be captured: the eager steps are the number
-        graph_note = f"eager (graph capture failed: {type(e).__name__}: {e})"
+    except Exception as e:   # a launch that cannot be captured: eager steps
+        graph = None
+        graph_note = f"eager steps back to back (graph capture failed: {type(e).__name__}: {e})"
         torch.cuda.synchronize(dev)
-        evs = timed(step)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    if graph is not None:
+        for _ in range(K // R):
+            graph.replay()
+    else:
+        for i in range(K):
+            step(i)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
     for w_ in (ws, ws_p):
         st, _ = dsa.dsa_check_device_status(w_)
         if st != dsa.DSA_OK:
             raise RuntimeError(f"device status {st} after the end-to-end steps")
-    total_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / 1e3, dev)
+    total_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, dev)
     import torch.distributed as dist
     world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
     return {"value": throughput(B * T, K, world, total_s), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K,
+            "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K, "steps": K,
             "per_step": "1 pinned H2D copy of the token's raw inputs; dsa_index_produce (index key into the cache, "
                         "index query codes); 2 device copies of the K/V rows into the cache; dsa_layer_decode; "
                         "1 D2H copy of O and the selection -- " + graph_note,
-            "ms_per_step_eager_median": eager_ms}
+            "l2": f"inputs larger than L2: {R} layers' caches in rotation, no flush",
+            "ms_per_step_isolated_median": iso_ms,
+            "isolated": "L2 flushed before each step, events around the one eager step"}
 
 
 # ------------------------------------------------------- CPU oracle timing

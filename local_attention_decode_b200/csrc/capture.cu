@@ -66,7 +66,7 @@ constexpr int kBins = 2048;                   // sample histogram: bits 30..20 o
 constexpr int kHistWords = kBins + 1;         // + the count of negative scores
 constexpr int kHistStride = kHistWords + 3;   // words between rows' histograms: rows start 16-byte aligned
 constexpr int kSegCap = 1024;                 // candidates one CTA may hold per row
-constexpr int kGroupCap = 256;                // candidates one epilogue group may hold per row
+constexpr int kWarpCap = 64;                  // candidates one epilogue warp may hold per row
 constexpr int kMaxBacklog = 16;               // tiles per epilogue group whose keys wait in TMEM for the thresholds
 constexpr int kListCap = 16384;               // candidates of one row the selection takes into shared memory
 constexpr int kWide = 4096;                   // bins of the selection's first histogram
@@ -264,74 +264,22 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags
     int32_t *row_qpos = reinterpret_cast<int32_t *>(smem + lay.misc_off + 32);   // [rows] query positions
     uint32_t *thr_s = reinterpret_cast<uint32_t *>(smem + lay.cap_off);   // [kMaxRows] thresholds, then the flag
-    uint32_t *cx = thr_s + 2 * kMaxRows;               // [group][warp][kMaxRows] a capture step's counts
-    uint32_t *gc = cx + kGroups * kEpiWarps * kMaxRows;   // [group][kMaxRows][2] the lists' lengths
-    uint32_t *dec = gc + kGroups * kMaxRows * 2;       // [group][2] the thresholds are known (by tile parity)
-    constexpr int kCapWords = 2 * kMaxRows + kGroups * (kEpiWarps * kMaxRows + 2 * kMaxRows + 2);
-    // After the sample the histogram area holds the groups' candidate lists:
-    // row r's lists at hist + r * kHistStride, group g's at + g * kGroupCap
-    // entries (order key, position).  List 0 (from the front) takes the keys
-    // of the tiles scored before the thresholds were known, list 1 (from the
-    // back) those of the later tiles: all of list 0's positions come first.
-    auto glist = [&](int r, int g) { return reinterpret_cast<uint2 *>(hist + r * kHistStride) + g * kGroupCap; };
-    static_assert(kGroups * kGroupCap * 8 <= kHistStride * 4, "group lists in the histogram area");
-    static_assert(kGroups * kGroupCap <= kSegCap, "a CTA's group lists fit its segment");
+    uint32_t *wcs = thr_s + 2 * kMaxRows;              // [epilogue warp][kMaxRows] the warps' list lengths
+    constexpr int kCapWords = 2 * kMaxRows + kGroups * kEpiWarps * kMaxRows;
+    // After the sample the histogram area holds the epilogue warps' candidate
+    // lists: row r's at hist + r * kHistStride, epilogue warp w's at
+    // + w * kWarpCap entries (order key, position), each in position order.
+    auto wlist = [&](int r, int w) { return reinterpret_cast<uint2 *>(hist + r * kHistStride) + w * kWarpCap; };
+    static_assert(kGroups * kEpiWarps * kWarpCap * 8 <= kHistStride * 4, "warp lists in the histogram area");
+    static_assert(kGroups * kEpiWarps * kWarpCap <= kSegCap, "a CTA's warp lists fit its segment");
     uint32_t *ctl = cp.ctl;
     const int warp = warp_id(), lane = lane_id();
     const uint32_t lt = (1u << lane) - 1u;
 
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-        int32_t mx = -1;
-        bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            int32_t q = __ldg(p.q_pos + b * T + t);
-            if (q < 0) ok = false;
-            mx = max(mx, q);
-        }
-        const int64_t cap = p.block_table ? (int64_t)p.max_pages * p.page_size : p.seq_stride;
-        if (!ok || (int64_t)mx >= cap || (int64_t)mx >= p.Lmax) {
-            if (cta == 0) flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX);
-            mx = -1;
-        }
-        seq_len[b] = mx + 1;
-    }
-    for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
-    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
-    for (int j = threadIdx.x; j < kCapWords; j += blockDim.x) thr_s[j] = 0;
-    if (threadIdx.x < rows) row_qpos[threadIdx.x] = __ldg(p.q_pos + threadIdx.x);
-    __syncthreads();
-    if (warp == 0) {
-        int carry = 0;
-        for (int base = 0; base < B; base += 32) {
-            const int b = base + lane;
-            int v = b < B ? (seq_len[b] + kTile - 1) / kTile : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            if (b < B) tile_pre[b + 1] = carry + v;
-            carry += __shfl_sync(0xffffffffu, v, 31);
-        }
-        if (lane == 0) tile_pre[0] = 0;
-    }
-    __syncthreads();
-
-    const int total = tile_pre[B];
-    const int per = total / ncta, rem = total % ncta;
-    const int t_begin = cta * per + min(cta, rem);
-    const int n_tiles = per + (cta < rem ? 1 : 0);
-    const int half = (n_tiles + kPipes - 1) / kPipes;
-    auto pipe_begin = [&](int pp) { return t_begin + min(n_tiles, pp * half); };
-    auto pipe_count = [&](int pp) { return min(n_tiles, (pp + 1) * half) - min(n_tiles, pp * half); };
-    // group a of pipe pp owns a contiguous part of the pipe's tiles; the
-    // pipe's i-th tile is tile i / GE of group i % GE
-    auto group_count = [&](int pp, int a) { const int c = pipe_count(pp); return c / GE + (a < c % GE ? 1 : 0); };
-    auto tile_of = [&](int pp, int i) {
-        const int c = pipe_count(pp), a = i % GE;
-        return pipe_begin(pp) + a * (c / GE) + min(a, c % GE) + i / GE;
-    };
-
+    // The prologue has one block barrier: thread 0 reads the (at most
+    // kMaxRows) query positions, all loads in flight together, and builds the
+    // per-sequence tables and the mbarriers while warp kPipes allocates TMEM
+    // and the other threads clear the shared words.
     // TMEM: the accumulators, then the backlog: the order keys of the first
     // back_cap tiles of each epilogue group, kept until the thresholds come
     // (column acc_cols + (group * back_cap + tile) * T + query, lane = key row)
@@ -340,6 +288,10 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     uint32_t tmem_cols = 32;
     while (tmem_cols < (uint32_t)(acc_cols + kGroups * back_cap * T)) tmem_cols <<= 1;
     if (threadIdx.x == 0) {
+        int32_t qv[kMaxRows];
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r) qv[r] = r < rows ? __ldg(p.q_pos + r) : 0;
+        // (the barriers while the loads are in flight)
         for (int pp = 0; pp < kPipes; ++pp) {
             for (int s = 0; s < S; ++s) {
                 mbar_init(&bars->full[pp][s], 1);
@@ -357,15 +309,59 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_ks);
         prefetch_tmap(&tmap_q);
+        const int64_t cap = p.block_table ? (int64_t)p.max_pages * p.page_size : p.seq_stride;
+        int pre = 0;
+        tile_pre[0] = 0;
+#pragma unroll
+        for (int b = 0; b < kMaxRows / T; ++b) {   // (B * T <= kMaxRows)
+            if (b < B) {
+                int32_t mx = -1;
+                bool ok = true;
+#pragma unroll
+                for (int t = 0; t < T; ++t) {
+                    const int32_t q = qv[b * T + t];
+                    if (q < 0) ok = false;
+                    mx = max(mx, q);
+                }
+                if (!ok || (int64_t)mx >= cap || (int64_t)mx >= p.Lmax) {
+                    if (cta == 0) flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX);
+                    mx = -1;
+                }
+                seq_len[b] = mx + 1;
+                pre += (mx + 1 + kTile - 1) / kTile;
+                tile_pre[b + 1] = pre;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r)
+            if (r < rows) row_qpos[r] = qv[r];
     }
     if (warp == kPipes) {
         tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
     }
+    for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
+    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+    for (int j = threadIdx.x; j < kCapWords; j += blockDim.x) thr_s[j] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+
+    const int total = tile_pre[B];
+    const int per = total / ncta, rem = total % ncta;
+    const int t_begin = cta * per + min(cta, rem);
+    const int n_tiles = per + (cta < rem ? 1 : 0);
+    const int half = (n_tiles + kPipes - 1) / kPipes;
+    auto pipe_begin = [&](int pp) { return t_begin + min(n_tiles, pp * half); };
+    auto pipe_count = [&](int pp) { return min(n_tiles, (pp + 1) * half) - min(n_tiles, pp * half); };
+    // group a of pipe pp owns a contiguous part of the pipe's tiles; the
+    // pipe's i-th tile is tile i / GE of group i % GE
+    auto group_count = [&](int pp, int a) { const int c = pipe_count(pp); return c / GE + (a < c % GE ? 1 : 0); };
+    auto tile_of = [&](int pp, int i) {
+        const int c = pipe_count(pp), a = i % GE;
+        return pipe_begin(pp) + a * (c / GE) + min(a, c % GE) + i / GE;
+    };
 
     auto locate = [&](int g, int &b, int &ti) {
         int lo = 0, hi = B - 1;
@@ -380,94 +376,59 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     const uint32_t stage_tx = kTile * kKeyBytes + kTile * 4;
     const bool any_tiles = pipe_count(0) + pipe_count(1) > 0;
 
-    // ---- candidates, by the epilogue groups: group g of the CTA (its four
-    //      warps, rows 32 q .. 32 q + 31 of each of the group's tiles for warp
-    //      q; the groups in position order) keeps its keys at or above their
-    //      row's threshold in its lists, in position order
+    // ---- candidates, by each epilogue warp on its own: warp w of group g
+    //      (rows 32 q .. 32 q + 31 of each of the group's tiles, q = w & 3)
+    //      keeps the visible keys of its rows at or above their row's
+    //      threshold in a list of its own, in the order it scores its tiles --
+    //      position order, since a group's tiles are contiguous and
+    //      increasing.  No barrier between warps; after the stream the CTA
+    //      merges its warps' lists into its segment in position order.
     const int ew_c = warp - kEpiWarp0;   // negative for the other warps
     const int e_gi = ew_c >= 0 ? ew_c / kEpiWarps : 0;
     const int e_pp = e_gi / kMaxGroups, e_a = e_gi % kMaxGroups;
     const int e_q = warp & 3;
     const int e_row = e_q * 32 + lane;   // the lane's row in each tile
-    const int e_bar = kGroupBar0 + e_gi;
     const int e_ng = ew_c >= 0 && e_a < GE ? group_count(e_pp, e_a) : 0;
-    bool capturing = false;   // the group has the thresholds and takes its candidates
-    // One capture step, by the group's four warps together: of the tile rows
-    // of sequence b at position pos (one per lane), those with bit t of cand
-    // go with key[t] to the end of list li of row b * T + t.
-    auto group_take = [&](int b, int li, uint32_t cand, const uint32_t (&key)[kMaxRows], uint32_t pos) {
-        uint32_t *cxg = cx + e_gi * kEpiWarps * kMaxRows;
-        uint32_t bits[kMaxRows];
-#pragma unroll
-        for (int t = 0; t < kMaxRows; ++t) {
-            bits[t] = t < T ? __ballot_sync(0xffffffffu, (cand >> t) & 1u) : 0u;
-            if (t < T && lane == 0) cxg[e_q * kMaxRows + t] = __popc(bits[t]);
-        }
-        named_bar_sync(e_bar, 128);   // the four warps' counts
+    bool capturing = false;   // the warp has the thresholds and takes its candidates
+    uint32_t thr[kMaxRows] = {0u, 0u, 0u, 0u};   // the rows' thresholds, once known
+    uint32_t wc[kMaxRows] = {0u, 0u, 0u, 0u};    // the warp's list lengths (the same in every lane)
+    // Of the warp's rows of one tile of sequence b at position pos (one per
+    // lane), those with bit t of cand go with key[t] to the end of the warp's
+    // list of row b * T + t.
+    auto warp_take = [&](int b, uint32_t cand, const uint32_t (&key)[kMaxRows], uint32_t pos) {
 #pragma unroll
         for (int t = 0; t < T; ++t) {
+            const uint32_t bits = __ballot_sync(0xffffffffu, (cand >> t) & 1u);
+            if (bits == 0u) continue;
             const int r = b * T + t;
+            uint32_t n = 0u, th = 0u;
+#pragma unroll
+            for (int rr = 0; rr < kMaxRows; ++rr)
+                if (rr == r) {
+                    n = wc[rr];
+                    th = thr[rr];
+                }
             if ((cand >> t) & 1u) {
-                uint32_t slot = gc[(e_gi * kMaxRows + r) * 2 + li] + __popc(bits[t] & lt);
-                for (int q2 = 0; q2 < e_q; ++q2) slot += cxg[q2 * kMaxRows + t];
-                if (slot < (uint32_t)kGroupCap)
-                    glist(r, e_gi)[li == 0 ? slot : kGroupCap - 1 - slot] = make_uint2(key[t], pos);
-                const uint32_t bin = min((key[t] - thr_s[r]) >> kCandShift, (uint32_t)(kWide - 1));
+                const uint32_t slot = n + __popc(bits & lt);
+                if (slot < (uint32_t)kWarpCap) wlist(r, ew_c)[slot] = make_uint2(key[t], pos);
+                const uint32_t bin = min((key[t] - th) >> kCandShift, (uint32_t)(kWide - 1));
                 atomicAdd(cp.cand_hist + (int64_t)r * kWide + bin, 1u);
             }
-        }
-        named_bar_sync(e_bar, 128);   // every warp has read the counts and lengths
-        if (e_q == 0 && lane == 0) {
 #pragma unroll
-            for (int t = 0; t < T; ++t)
-                gc[(e_gi * kMaxRows + b * T + t) * 2 + li] +=
-                    cxg[t] + cxg[kMaxRows + t] + cxg[2 * kMaxRows + t] + cxg[3 * kMaxRows + t];
+            for (int rr = 0; rr < kMaxRows; ++rr)
+                if (rr == r) wc[rr] += __popc(bits);
         }
     };
-    // the group's tiles [j_begin, j_end) again, from the scores its own lanes
-    // stored (a lane reads back only its own stores), a few tiles' loads in
-    // flight at a time; into list 0
-    auto catch_up = [&](int j_begin, int j_end) {
-        constexpr int kB = T <= 2 ? 4 : 2;
-        for (int jb = j_begin; jb < j_end; jb += kB) {
-            float v[kB][T];
-            int32_t ps[kB];   // (positions below 2^31)
-            int bb[kB];
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                bb[u] = 0;
-                ps[u] = -1;
-                if (jb + u < j_end) {
-                    int ti;
-                    locate(tile_of(e_pp, (jb + u) * GE + e_a), bb[u], ti);
-                    ps[u] = ti * kTile + e_row;
-                    if (ps[u] >= seq_len[bb[u]]) ps[u] = -1;
-                }
-#pragma unroll
-                for (int t = 0; t < T; ++t)
-                    v[u][t] = ps[u] >= 0 ? p.scores[((int64_t)bb[u] * T + t) * p.scores_stride + ps[u]] : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                if (jb + u < j_end) {   // uniform in the group
-                    uint32_t key[kMaxRows] = {0u, 0u, 0u, 0u}, cand = 0u;
-#pragma unroll
-                    for (int t = 0; t < T; ++t) {
-                        const int r = bb[u] * T + t;
-                        key[t] = float_order_key(v[u][t]);
-                        if (ps[u] >= 0 && ps[u] <= row_qpos[r] && key[t] >= thr_s[r]) cand |= 1u << t;
-                    }
-                    group_take(bb[u], 0, cand, key, (uint32_t)ps[u]);
-                }
-            }
-        }
-    };
-    // The group's backlog: its tiles [0, j_now), scored before the thresholds
-    // were known; the first back_cap of them from TMEM now, the rest (if any)
-    // from its own stored scores after the stream.
-    int glob_lo = 0, glob_hi = 0;
+    // The warp's backlog: the group's tiles [0, j_now), scored before the
+    // thresholds were known; the first back_cap of them from TMEM, the rest
+    // from the scores this lane stored (a lane reads back only its own
+    // stores), a few tiles' loads in flight at a time.
     auto transition = [&](int j_now) {
         capturing = true;
+        __threadfence_block();   // the thresholds, after the flag that announced them
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r) thr[r] = r < rows ? thr_s[r] : 0u;
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");   // the backlog's keys are in TMEM
         const int nb = min(j_now, back_cap);
         for (int jj = 0; jj < nb; ++jj) {
             int bb, ti;
@@ -481,10 +442,41 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                                   (uint32_t)(acc_cols + (e_gi * back_cap + jj) * T + t));
                 if (ps < seq_len[bb] && ps <= row_qpos[r] && key[t] >= thr_s[r]) cand |= 1u << t;
             }
-            group_take(bb, 0, cand, key, (uint32_t)ps);
+            warp_take(bb, cand, key, (uint32_t)ps);
         }
-        glob_lo = nb;
-        glob_hi = j_now;
+        constexpr int kB = T <= 2 ? 4 : 2;
+        for (int jb = nb; jb < j_now; jb += kB) {
+            float v[kB][T];
+            int32_t ps[kB];   // (positions below 2^31)
+            int bb[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                bb[u] = 0;
+                ps[u] = -1;
+                if (jb + u < j_now) {
+                    int ti;
+                    locate(tile_of(e_pp, (jb + u) * GE + e_a), bb[u], ti);
+                    ps[u] = ti * kTile + e_row;
+                    if (ps[u] >= seq_len[bb[u]]) ps[u] = -1;
+                }
+#pragma unroll
+                for (int t = 0; t < T; ++t)
+                    v[u][t] = ps[u] >= 0 ? p.scores[((int64_t)bb[u] * T + t) * p.scores_stride + ps[u]] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                if (jb + u < j_now) {   // uniform in the warp
+                    uint32_t key[kMaxRows] = {0u, 0u, 0u, 0u}, cand = 0u;
+#pragma unroll
+                    for (int t = 0; t < T; ++t) {
+                        const int r = bb[u] * T + t;
+                        key[t] = float_order_key(v[u][t]);
+                        if (ps[u] >= 0 && ps[u] <= row_qpos[r] && key[t] >= thr_s[r]) cand |= 1u << t;
+                    }
+                    warp_take(bb[u], cand, key, (uint32_t)ps[u]);
+                }
+            }
+        }
     };
     // the thresholds from their packed words (all rows published), into
     // shared memory for the CTA's warps
@@ -728,10 +720,11 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                     }
                 }
             }
-            // ---- this tile's candidates, once the CTA has the thresholds (never
-            //      at j == 0: they need this CTA's sample).  The poller copies
-            //      the packed words into shared memory asynchronously and looks
-            //      at the copy one tile later, so it never waits for it.
+            // ---- this tile's candidates, once the warp has the thresholds.
+            //      Each group's poller copies the packed words into shared
+            //      memory asynchronously and looks at the copy one tile later,
+            //      so it never waits for it; every warp looks at the CTA's
+            //      flag once per tile and switches on its own.
             if (!capturing) {
                 if (poller) {
                     if (polling) {
@@ -749,39 +742,38 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         polling = true;
                     }
                 }
-                // one decision for the group's four warps (a slot per tile parity)
-                if (poller) dec[gi * 2 + (j & 1)] = *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows);
-                named_bar_sync(gbar, 128);
-                if (*reinterpret_cast<volatile uint32_t *>(dec + gi * 2 + (j & 1)) != 0u) {
-                    __threadfence_block();
-                    transition(j);   // the tiles before this one
-                }
+                uint32_t seen = lane == 0 ? *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows) : 0u;
+                if (__shfl_sync(0xffffffffu, seen, 0) != 0u) transition(j);   // the tiles before this one
             }
             if (capturing) {
                 uint32_t key[kMaxRows] = {0u, 0u, 0u, 0u}, cand = 0u;
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
                     key[t] = float_order_key(sc[t]);
-                    if (scored && ((vis >> t) & 1u) && key[t] >= thr_s[b * T + t]) cand |= 1u << t;
+                    uint32_t th = 0u;
+#pragma unroll
+                    for (int rr = 0; rr < kMaxRows; ++rr)
+                        if (rr == b * T + t) th = thr[rr];
+                    if (scored && ((vis >> t) & 1u) && key[t] >= th) cand |= 1u << t;
                 }
-                group_take(b, 1, cand, key, (uint32_t)pos);
+                warp_take(b, cand, key, (uint32_t)pos);
             }
         }
         if (polling) attn::cp_async_wait_all();
-        // ---- after the group's tiles: warps still without the thresholds wait
-        //      for them here, while their backlog is in TMEM
-        if (ng > 0) {
-            bool okw = true;
-            if (poller && *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows) == 0u) {
-                uint64_t w[kMaxRows];
-                okw = wait_packed(w);
-                if (okw) publish(w);
+        // ---- after the group's tiles: a warp still without the thresholds
+        //      waits for them here, while its backlog is in TMEM
+        if (ng > 0 && !capturing) {
+            uint32_t okw = 1u;
+            const uint32_t seen = lane == 0 ? *reinterpret_cast<volatile uint32_t *>(thr_s + kMaxRows) : 0u;
+            if (__shfl_sync(0xffffffffu, seen, 0) == 0u) {
+                if (lane == 0) {
+                    uint64_t w[kMaxRows];
+                    okw = wait_packed(w) ? 1u : 0u;
+                    if (okw) publish(w);
+                }
+                okw = __shfl_sync(0xffffffffu, okw, 0);
             }
-            okw = named_bar_and(gbar, 128, okw);
-            if (okw && !capturing) {
-                __threadfence_block();
-                transition(ng);
-            }
+            if (okw) transition(ng);
         }
     }
     (void)any_tiles;
@@ -811,9 +803,8 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     __syncthreads();
     if (cp.trace && threadIdx.x == 0) cp.trace[cta * DSA_TRACE_MARKS + 2] = globaltimer_ns();
 
-    // ---- the CTA's candidates: the warps that did not see the thresholds
-    //      during the stream take theirs now; the warps' lists are merged
-    //      into the CTA's segment of each row's list, in position order
+    // ---- the CTA's candidates: the warps' lists merged into the CTA's
+    //      segment of each row's list, in position order
     bool r_ok = true;
     if (threadIdx.x == 0 && n_tiles > 0 && thr_s[kMaxRows] == 0u) {
         r_ok = spin_until_at_least(ctl + kReady, 1u, kWaitLimitNs, p.status);   // (acquire)
@@ -823,37 +814,70 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
             if (cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 1] = globaltimer_ns();
         }
     }
+    if (ew_c >= 0 && lane == 0) {
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r) wcs[ew_c * kMaxRows + r] = wc[r];
+    }
     if (!__syncthreads_and(r_ok)) return;   // the timeout is in the status word; the grid barrier sees it
-    if (ew_c >= 0 && glob_hi > glob_lo) catch_up(glob_lo, glob_hi);   // backlog tiles TMEM did not hold
-    __syncthreads();
-    // the CTA's segment of row r: for each group in turn, its list 0, then
-    // its list 1 (stored from the back), by the group's four warps
+    // Each epilogue warp places its own list's entries: an entry's place in
+    // the segment is the length of the lists of the groups before its group
+    // (the groups' position ranges are disjoint and in group order) plus the
+    // entries of its group's four lists (which interleave within each tile)
+    // with a lower position.  The candidates' K and V rows (all KV heads) go
+    // on their way into L2 as well, while the grid meets: HBM is idle after
+    // the stream, and the selection's rows are among these.
+    constexpr int kLists = kGroups * kEpiWarps;
+    static_assert(kLists <= 32, "one list length per lane");
     if (ew_c >= 0) {
         for (int r = 0; r < rows; ++r) {
-            uint32_t at = 0;
-            for (int g2 = 0; g2 < e_gi; ++g2) at += gc[(g2 * kMaxRows + r) * 2] + gc[(g2 * kMaxRows + r) * 2 + 1];
-            const uint32_t n0 = gc[(e_gi * kMaxRows + r) * 2], n1 = gc[(e_gi * kMaxRows + r) * 2 + 1];
-            if (at + n0 + n1 <= (uint32_t)kSegCap && n0 + n1 <= (uint32_t)kGroupCap) {
-                const uint2 *L = glist(r, e_gi);
-                uint2 *seg = cp.lists + ((int64_t)r * cp.NG + cta) * kSegCap + at;
-                for (uint32_t i = e_q * 32 + lane; i < n0 + n1; i += kEpiWarps * 32)
-                    seg[i] = i < n0 ? L[i] : L[kGroupCap - 1 - (i - n0)];
+            const uint32_t c_l = lane < kLists ? wcs[lane * kMaxRows + r] : 0u;
+            const bool over = __any_sync(0xffffffffu, c_l > (uint32_t)kWarpCap);
+            uint32_t incl = c_l;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            const uint32_t total = __shfl_sync(0xffffffffu, incl, kLists - 1);
+            const uint32_t gbase = __shfl_sync(0xffffffffu, incl - c_l, e_gi * kEpiWarps);
+            uint32_t n4[kEpiWarps];
+#pragma unroll
+            for (int q2 = 0; q2 < kEpiWarps; ++q2) n4[q2] = __shfl_sync(0xffffffffu, c_l, e_gi * kEpiWarps + q2);
+            if (!over && total <= (uint32_t)kSegCap) {
+                uint2 *seg = cp.lists + ((int64_t)r * cp.NG + cta) * kSegCap;
+                uint32_t mine = 0;
+#pragma unroll
+                for (int q2 = 0; q2 < kEpiWarps; ++q2)
+                    if (q2 == e_q) mine = n4[q2];
+                for (uint32_t i = lane; i < mine; i += 32) {
+                    const uint2 ent = wlist(r, ew_c)[i];
+                    uint32_t rank = gbase + i;
+#pragma unroll
+                    for (int q2 = 0; q2 < kEpiWarps; ++q2) {
+                        if (q2 == e_q) continue;
+                        const uint2 *L2 = wlist(r, e_gi * kEpiWarps + q2);
+                        uint32_t lo = 0, hi = n4[q2];
+                        while (lo < hi) {
+                            const uint32_t mid = (lo + hi) >> 1;
+                            if (L2[mid].y < ent.y) lo = mid + 1; else hi = mid;
+                        }
+                        rank += lo;
+                    }
+                    seg[rank] = ent;
+                    int64_t krow;
+                    if (attn::key_row(cp.at, r / T, (int64_t)ent.y, &krow)) {
+                        bulk_prefetch_l2(cp.at.K + krow * cp.at.G * DSA_QK_DIM, (uint32_t)(cp.at.G * DSA_QK_DIM * 2));
+                        bulk_prefetch_l2(cp.at.V + krow * cp.at.G * DSA_V_DIM, (uint32_t)(cp.at.G * DSA_V_DIM * 2));
+                    }
+                }
+            }
+            if (ew_c == 0 && lane == 0) {   // the row's count in this CTA
+                const bool ov = over || total > (uint32_t)kSegCap;
+                cp.counts[(int64_t)r * cp.NG + cta] = ov ? 0u : total;
+                if (total && !ov) atomicAdd(ctl + kTotal + r, total);
+                if (ov) atomicOr(ctl + kOverflow, 1u);
             }
         }
-    }
-    if ((int)threadIdx.x < rows) {   // the row's count in this CTA
-        const int r = threadIdx.x;
-        uint32_t total = 0;
-        bool over = false;
-        for (int g2 = 0; g2 < kGroups; ++g2) {
-            const uint32_t c = gc[(g2 * kMaxRows + r) * 2] + gc[(g2 * kMaxRows + r) * 2 + 1];
-            over |= c > (uint32_t)kGroupCap;
-            total += c;
-        }
-        over |= total > (uint32_t)kSegCap;
-        cp.counts[(int64_t)r * cp.NG + cta] = over ? 0u : total;
-        if (total && !over) atomicAdd(ctl + kTotal + r, total);
-        if (over) atomicOr(ctl + kOverflow, 1u);
     }
     if ((int)threadIdx.x <= kMaxRows) keep[threadIdx.x] = thr_s[threadIdx.x];   // the thresholds and their flag
 }

@@ -94,10 +94,10 @@ __device__ __forceinline__ bool grid_sync(uint32_t *bar, uint32_t target, const 
                                           uint32_t *flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(bar, 1u);
+        // the release arrival covers the CTA's writes (ordered before it by the
+        // block barrier); the acquire load of the count covers everyone else's
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
         const bool ok = spin_until_at_least(bar, target + cfg.extra, cfg.limit_ns, status);
-        __threadfence();
         *flag = ok ? 1u : 0u;
     }
     __syncthreads();
@@ -231,6 +231,12 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
+}
+
+// Bulk prefetch of global [gsrc, gsrc + bytes) into L2 (no destination, no
+// completion to wait for); gsrc 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gsrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
 }
 
 // Raises the barrier's expected transaction bytes without arriving.
