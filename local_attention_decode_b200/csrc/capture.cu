@@ -115,6 +115,7 @@ struct Params {
     uint2 *lists;             // [rows][NG][kSegCap] (order key, position)
     uint32_t *path_count;     // [2] calls that took the fast path / the general path
     uint64_t *trace;          // [grid][DSA_TRACE_MARKS] phase marks, or NULL
+    const float *k_scale;     // the index keys' scales, [cache rows]
     BarrierCfg bar;
     int rows, K, C, NG;
     float oversample;
@@ -249,7 +250,8 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                                     uint32_t *keep) {
     using namespace indexer;
     const indexer::Params &p = cp.ix;
-    const CUtensorMap &tmap_k = *tmap_k_p, &tmap_ks = *tmap_ks_p, &tmap_q = *tmap_q_p;
+    const CUtensorMap &tmap_k = *tmap_k_p, &tmap_q = *tmap_q_p;
+    (void)tmap_ks_p;   // (the key scales are read from global memory by the epilogue)
     // the query tokens per sequence are a compile-time constant: the per-query
     // loops of the epilogue keep only the copies that run (a smaller loop body
     // that stays in the instruction cache)
@@ -295,7 +297,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         for (int pp = 0; pp < kPipes; ++pp) {
             for (int s = 0; s < S; ++s) {
                 mbar_init(&bars->full[pp][s], 1);
-                mbar_init(&bars->empty[pp][s], 1 + kEpiWarps);
+                mbar_init(&bars->empty[pp][s], 1);   // the MMA's commit: the epilogue never reads the stage
             }
             for (int a = 0; a < GE; ++a)
                 for (int u = 0; u < AB; ++u) {
@@ -307,7 +309,6 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         mbar_init(&bars->q_full, 1);
         fence_mbar_init();
         prefetch_tmap(&tmap_k);
-        prefetch_tmap(&tmap_ks);
         prefetch_tmap(&tmap_q);
         const int64_t cap = p.block_table ? (int64_t)p.max_pages * p.page_size : p.seq_stride;
         int pre = 0;
@@ -373,7 +374,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         while (b < B - 1 && tile_pre[b + 1] <= g) ++b;
         ti = g - tile_pre[b];
     };
-    const uint32_t stage_tx = kTile * kKeyBytes + kTile * 4;
+    const uint32_t stage_tx = kTile * kKeyBytes;   // (the key scales go to the epilogue from global memory)
     const bool any_tiles = pipe_count(0) + pipe_count(1) > 0;
 
     // ---- candidates, by each epilogue warp on its own: warp w of group g
@@ -530,7 +531,6 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 int b, ti;
                 locate(tile_of(pp, i), b, ti);
                 uint8_t *kdst = smem + lay.k_off + st * kTile * kKeyBytes;
-                uint8_t *ksdst = smem + lay.ks_off + st * kKsStageBytes;
                 const int R = p.rows_per_load;
                 for (int j = 0; j < kTile / R; ++j) {
                     const int64_t pos = (int64_t)ti * kTile + j * R;
@@ -541,8 +541,6 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         if (!ok) { flag_error(p.status, DSA_ERR_DEVICE_BAD_INDEX); row = 0; }
                     }
                     tma_load_2d_hint(kdst + j * R * kKeyBytes, &tmap_k, &bars->full[pp][s], 0, (int32_t)row,
-                                     stream_policy);
-                    tma_load_1d_hint(ksdst + ks_slot_offset(j * R, R), &tmap_ks, &bars->full[pp][s], (int32_t)row,
                                      stream_policy);
                 }
                 ++issued;
@@ -601,8 +599,27 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         int cur_b = -1;
         bool polling = false;   // the poller's read of the packed words is in flight
         uint32_t *poll = reinterpret_cast<uint32_t *>(smem + lay.poll_off) + gi * 2 * kMaxRows;
+        // This lane's key scale in the group's jn-th tile, loaded one tile
+        // ahead (0 past the group's tiles or the sequence).  The scales come
+        // from global memory, not through the stage, so a stage is free as
+        // soon as its MMA has read it: an epilogue group that is held up (the
+        // sample exchange, the thresholds) holds up only its own TMEM
+        // accumulators, not the pipeline's ring.
+        auto scale_of = [&](int jn) -> float {
+            if (jn >= ng) return 0.f;
+            int bb, ti2;
+            locate(tile_of(pp, jn * GE + a), bb, ti2);
+            const int64_t ps = (int64_t)ti2 * kTile + row_in_tile;
+            if (ps >= seq_len[bb]) return 0.f;
+            bool okr = true;
+            const int64_t row = row_of(p, bb, ps, &okr);
+            return okr ? __ldcs(cp.k_scale + row) : 0.f;
+        };
+        float ks_next = scale_of(0);
         for (int j = 0; j < ng || j == 0; ++j) {
             const bool have = j < ng;
+            const float ks = ks_next;
+            ks_next = scale_of(j + 1);
             bool scored = false;
             float sc[kMaxRows] = {0.f, 0.f, 0.f, 0.f};
             uint32_t vis = 0;
@@ -622,14 +639,13 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 }
                 const int u = j % AB;
                 const uint32_t acc_col = acc_col0 + (uint32_t)(u * N);
-                bool w_ok = mbar_wait(&bars->tfull[pp][a][u], (j / AB) & 1, p.status) &&
-                            mbar_wait(&bars->full[pp][s], (i / S) & 1, p.status);
+                const bool w_ok = mbar_wait(&bars->tfull[pp][a][u], (j / AB) & 1, p.status);
+                (void)s;
+                (void)st;
                 if (__all_sync(0xffffffffu, w_ok)) {
                     scored = true;
                     if (j == 0 && gi == 0 && poller && cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 12] = globaltimer_ns();
                     tc_fence_after();
-                    const float ks = *reinterpret_cast<const float *>(smem + lay.ks_off + st * kKsStageBytes +
-                                                                      ks_slot_offset(row_in_tile, p.rows_per_load));
                     pos = (int64_t)ti * kTile + row_in_tile;
                     const int len = seq_len[b];
                     float *out = p.scores + (int64_t)b * T * p.scores_stride + pos;
@@ -657,10 +673,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&bars->tempty[pp][a][u]);
-                        mbar_arrive(&bars->empty[pp][s]);
-                    }
+                    if (lane == 0) mbar_arrive(&bars->tempty[pp][a][u]);
                     if (j == 0) {   // the sample: into the CTA's histogram of each row
 #pragma unroll
                         for (int t = 0; t < kMaxRows; ++t)
@@ -1521,7 +1534,10 @@ int launch_capture(const CapturePlan &plan, const IndexerArgs &ia, const AttnArg
     cp.ix = L.p;
     cp.ix.stages = S;
     cp.ix.groups = indexer::kMaxGroups;
-    cp.ix.acc_bufs = indexer::kAccBufs;   // 2 pipes * 2 groups * 2 * 16T <= 512 columns for T <= 4
+    // TMEM accumulators per epilogue group: four for one query token (2 pipes
+    // * 2 groups * 4 * 16 = 256 columns, the backlog beside them), else two
+    cp.ix.acc_bufs = ia.T == 1 ? 4 : 2;
+    cp.k_scale = static_cast<const float *>(ia.kv->index_k_scale);
     cp.ix.hist_rows = 0;
     cp.ix.q_resident = 1;
     cp.at = attn::make_params(aa);

@@ -156,7 +156,7 @@ int prepare_indexer(const IndexerArgs &a, int hist_rows, int hist_row_words, uin
     p.stages = S;
     p.rows_per_load = R;
     p.groups = std::max(1, std::min(kMaxGroups, 512 / (kPipes * N)));
-    p.acc_bufs = std::max(1, std::min(kAccBufs, 512 / (kPipes * p.groups * N)));
+    p.acc_bufs = std::max(1, std::min(2, 512 / (kPipes * p.groups * N)));
     p.hist_rows = hist_rows;
     p.hist_row_words = hist_row_words;
     p.hist_global = hist_global;

@@ -41,8 +41,9 @@ constexpr int kEpiWarps = 4;              // warps per epilogue group (one per T
 constexpr int kEpiWarp0 = 2 * kPipes;     // first epilogue warp
 constexpr int kThreads = 32 * (kEpiWarp0 + kPipes * kMaxGroups * kEpiWarps);   // 640
 constexpr int kMaxStages = 8;             // per pipeline
-constexpr int kAccBufs = 2;               // at most this many TMEM accumulators per epilogue group (two: the
-                                          // MMA of a group's next tile runs while its epilogue reads this one)
+constexpr int kAccBufs = 4;               // at most this many TMEM accumulators per epilogue group (two or
+                                          // more: the MMA of a group's next tiles runs while its epilogue
+                                          // reads this one)
 constexpr int kKsStageBytes = 1024;       // key-scale slots of one stage
 // Score histogram for the selection: bits 30..20 of the order key of each
 // non-negative score (2048 bins, eight per octave), and one bin (2048) that
