@@ -140,7 +140,8 @@ struct Layout {
         hist_off = epi_off + kGroups * kEpiWarps * (16 * T + T) * 4;
         misc_off = hist_off + rows * kHistStride * 4;
         // misc: [0] groups sampled, [1 + g] group g's role in the sample
-        // exchange; then the rows' query positions
+        // exchange, [5] rows' thresholds published; then the rows' query
+        // positions
         // [kMaxRows] thresholds, [kMaxRows] their flag; then per group: the
         // warps' counts of a capture step, the lists' lengths, the decisions
         cap_off = misc_off + 32 + 16;
@@ -155,7 +156,9 @@ __device__ __forceinline__ uint32_t sample_bin(uint32_t key) {
     return (key >> 31) ? ((key >> 20) & (kBins - 1)) : (uint32_t)kBins;
 }
 
-// The threshold of one row from its global sample histogram, by one warp.
+// The threshold of one row from its sample histogram (every CTA's sample
+// added in), already copied into shared memory `local` (kHistWords words),
+// by one warp.
 // The sample's visible keys (the histogram's total, tot) predict
 // oversample * K * tot / n + 16 of them at or above the row's threshold; the
 // threshold lies in the highest bin b whose count, with the bins above it,
@@ -163,25 +166,18 @@ __device__ __forceinline__ uint32_t sample_bin(uint32_t key) {
 // above it were b's keys spread evenly over its key values; zero (take every
 // key) when the sample's non-negative scores do not reach the target.  Any
 // threshold gives the exact result (a short list takes the general path);
-// this one keeps the list near oversample x top_k.  Zeroes the histogram for
-// the next call.
-// `local` is shared memory of kBins words that the warp may overwrite: the
-// loaded histogram goes there, so the second level of the search reads it
-// from shared memory (one round trip to L2 in all).
-__device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversample, uint32_t *local) {
+// this one keeps the list near oversample x top_k.
+__device__ uint32_t row_threshold(const uint32_t *local, int64_t n, int K, float oversample) {
     const int lane = lane_id();
     constexpr int kPer = kBins / 32;   // 64 bins per lane
     uint32_t s = 0;
-    const uint4 *h4 = reinterpret_cast<const uint4 *>(hist + lane * kPer);
-    uint4 *l4 = reinterpret_cast<uint4 *>(local + lane * kPer);
+    const uint4 *l4 = reinterpret_cast<const uint4 *>(local + lane * kPer);
 #pragma unroll
     for (int u = 0; u < kPer / 4; ++u) {
-        const uint4 v = __ldcg(h4 + u);
+        const uint4 v = l4[u];
         s += v.x + v.y + v.z + v.w;
-        l4[u] = v;
     }
-    __syncwarp();
-    const uint32_t negative = __ldcg(hist + kBins);
+    const uint32_t negative = local[kBins];
     uint32_t incl = s;   // keys in this lane's bins and all higher ones
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -232,11 +228,6 @@ __device__ uint32_t row_threshold(uint32_t *hist, int64_t n, int K, float oversa
             thr = (0x80000000u | ((best - 1) << 20)) + (uint32_t)(((uint64_t)(cb - need) << 20) / cb);
         }
     }
-    __syncwarp();
-    uint4 *w4 = reinterpret_cast<uint4 *>(hist + lane * kPer);
-#pragma unroll
-    for (int u = 0; u < kPer / 4; ++u) w4[u] = make_uint4(0, 0, 0, 0);
-    if (lane == 0) hist[kBins] = 0;
     return thr;
 }
 
@@ -263,7 +254,8 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     int32_t *seq_len = reinterpret_cast<int32_t *>(smem + lay.len_off);
     int32_t *tile_pre = reinterpret_cast<int32_t *>(smem + lay.tile_off);
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist_off);   // [rows][kHistStride]
-    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc_off);   // [0] groups sampled, [1..4] group flags,
+                                                                          // [5] rows' thresholds published
     int32_t *row_qpos = reinterpret_cast<int32_t *>(smem + lay.misc_off + 32);   // [rows] query positions
     uint32_t *thr_s = reinterpret_cast<uint32_t *>(smem + lay.cap_off);   // [kMaxRows] thresholds, then the flag
     uint32_t *wcs = thr_s + 2 * kMaxRows;              // [epilogue warp][kMaxRows] the warps' list lengths
@@ -356,13 +348,10 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     const int half = (n_tiles + kPipes - 1) / kPipes;
     auto pipe_begin = [&](int pp) { return t_begin + min(n_tiles, pp * half); };
     auto pipe_count = [&](int pp) { return min(n_tiles, (pp + 1) * half) - min(n_tiles, pp * half); };
-    // group a of pipe pp owns a contiguous part of the pipe's tiles; the
-    // pipe's i-th tile is tile i / GE of group i % GE
+    // the pipe's tiles in order, its i-th tile to group i % GE (one
+    // sequential stream per pipeline)
     auto group_count = [&](int pp, int a) { const int c = pipe_count(pp); return c / GE + (a < c % GE ? 1 : 0); };
-    auto tile_of = [&](int pp, int i) {
-        const int c = pipe_count(pp), a = i % GE;
-        return pipe_begin(pp) + a * (c / GE) + min(a, c % GE) + i / GE;
-    };
+    auto tile_of = [&](int pp, int i) { return pipe_begin(pp) + i; };
 
     auto locate = [&](int g, int &b, int &ti) {
         int lo = 0, hi = B - 1;
@@ -381,8 +370,8 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     //      (rows 32 q .. 32 q + 31 of each of the group's tiles, q = w & 3)
     //      keeps the visible keys of its rows at or above their row's
     //      threshold in a list of its own, in the order it scores its tiles --
-    //      position order, since a group's tiles are contiguous and
-    //      increasing.  No barrier between warps; after the stream the CTA
+    //      position order, since a group's tiles come in increasing
+    //      position.  No barrier between warps; after the stream the CTA
     //      merges its warps' lists into its segment in position order.
     const int ew_c = warp - kEpiWarp0;   // negative for the other warps
     const int e_gi = ew_c >= 0 ? ew_c / kEpiWarps : 0;
@@ -616,8 +605,35 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
             return okr ? __ldcs(cp.k_scale + row) : 0.f;
         };
         float ks_next = scale_of(0);
+        int thr_row = -1;   // the row whose threshold this warp computes, once its histogram has arrived
+        // Row thr_row's threshold from the histogram copied into shared memory:
+        // published (kThr, the packed word), the global histogram cleared for
+        // the next call; the last row's warp resets the arrival count and
+        // releases kReady.
+        auto finish_threshold = [&]() {
+            attn::cp_async_wait_all();
+            __syncwarp();
+            const int r = thr_row;
+            thr_row = -1;
+            const int64_t n = (int64_t)row_qpos[r] + 1;
+            uint32_t t_r = 0xFFFFFFFFu;   // n <= top_k: every key is selected, nothing to capture
+            if (n > cp.K) t_r = row_threshold(hist + r * kHistStride, n, cp.K, cp.oversample);
+            uint4 *g4 = reinterpret_cast<uint4 *>(cp.sample_hist + r * kHistStride);
+            for (int u = lane; u < kHistStride / 4; u += 32) g4[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (lane == 0) {
+                ctl[kThr + r] = t_r;
+                st_relaxed_gpu_u64(reinterpret_cast<uint64_t *>(ctl + kThrPacked) + r, (1ull << 32) | t_r);
+                __threadfence();   // this row's words, before the count that the last row's warp reads
+                if (atomicAdd(misc + 5, 1u) == (uint32_t)rows - 1) {
+                    ctl[kSampleArrive] = 0;   // read by nobody until the next call
+                    st_release_gpu(ctl + kReady, 1u);
+                }
+            }
+            __syncwarp();
+        };
         for (int j = 0; j < ng || j == 0; ++j) {
             const bool have = j < ng;
+            if (thr_row >= 0) finish_threshold();
             const float ks = ks_next;
             ks_next = scale_of(j + 1);
             bool scored = false;
@@ -706,30 +722,16 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         if (cp.trace) cp.trace[cta * DSA_TRACE_MARKS + 7] = globaltimer_ns();
                     }
                     named_bar_sync(gbar, 128);
-                    if (*flag == 2u) {   // the last CTA: one warp per row
-                        if (quarter < rows) {
-                            const int r = quarter;
-                            const int64_t n = (int64_t)__ldg(p.q_pos + r) + 1;
-                            uint32_t t_r = 0xFFFFFFFFu;   // n <= top_k: every key is selected, nothing to capture
-                            uint32_t *h = cp.sample_hist + r * kHistStride;
-                            if (n > cp.K) {
-                                // (the CTA's shared histogram of this row, already added in,
-                                // takes the loaded global one)
-                                t_r = row_threshold(h, n, cp.K, cp.oversample, hist + r * kHistStride);
-                            } else {
-                                for (int u = lane; u < kHistWords; u += 32) h[u] = 0;
-                            }
-                            if (lane == 0) {
-                                ctl[kThr + r] = t_r;
-                                st_relaxed_gpu_u64(reinterpret_cast<uint64_t *>(ctl + kThrPacked) + r,
-                                                   (1ull << 32) | t_r);
-                            }
-                        }
-                        named_bar_sync(gbar, 128);   // the thresholds, before the release that publishes them
-                        if (quarter == 0 && lane == 0) {
-                            ctl[kSampleArrive] = 0;   // read by nobody until the next call
-                            st_release_gpu(ctl + kReady, 1u);
-                        }
+                    if (*flag == 2u && quarter < rows) {
+                        // the last CTA: warp r of the group copies row r's
+                        // histogram into shared memory (the CTA's own, already
+                        // added in, is free) and goes on with its tiles; it
+                        // computes the threshold from the copy a tile later
+                        const uint4 *src = reinterpret_cast<const uint4 *>(cp.sample_hist + quarter * kHistStride);
+                        uint4 *dst = reinterpret_cast<uint4 *>(hist + quarter * kHistStride);
+                        for (int u = lane; u < kHistStride / 4; u += 32) attn::cp_async16(dst + u, src + u);
+                        attn::cp_async_commit();
+                        thr_row = quarter;
                     }
                 }
             }
@@ -772,6 +774,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 warp_take(b, cand, key, (uint32_t)pos);
             }
         }
+        if (thr_row >= 0) finish_threshold();
         if (polling) attn::cp_async_wait_all();
         // ---- after the group's tiles: a warp still without the thresholds
         //      waits for them here, while its backlog is in TMEM
@@ -833,13 +836,14 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     }
     if (!__syncthreads_and(r_ok)) return;   // the timeout is in the status word; the grid barrier sees it
     // Each epilogue warp places its own list's entries: an entry's place in
-    // the segment is the length of the lists of the groups before its group
-    // (the groups' position ranges are disjoint and in group order) plus the
-    // entries of its group's four lists (which interleave within each tile)
-    // with a lower position.  The candidates' K and V rows (all KV heads) go
+    // the segment is the length of the lists of the pipelines before its
+    // pipeline (their position ranges are disjoint and in order) plus the
+    // entries of its pipeline's eight lists (which interleave: tiles by
+    // group, rows within a tile by warp) with a lower position.  The candidates' K and V rows (all KV heads) go
     // on their way into L2 as well, while the grid meets: HBM is idle after
     // the stream, and the selection's rows are among these.
     constexpr int kLists = kGroups * kEpiWarps;
+    constexpr int kPipeWarps = kMaxGroups * kEpiWarps;   // the epilogue warps of one pipeline
     static_assert(kLists <= 32, "one list length per lane");
     if (ew_c >= 0) {
         for (int r = 0; r < rows; ++r) {
@@ -852,24 +856,25 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                 if (lane >= o) incl += u;
             }
             const uint32_t total = __shfl_sync(0xffffffffu, incl, kLists - 1);
-            const uint32_t gbase = __shfl_sync(0xffffffffu, incl - c_l, e_gi * kEpiWarps);
-            uint32_t n4[kEpiWarps];
+            const int w0 = e_pp * kPipeWarps;   // the pipeline's first epilogue warp
+            const uint32_t pbase = __shfl_sync(0xffffffffu, incl - c_l, w0);
+            uint32_t nw[kPipeWarps];
 #pragma unroll
-            for (int q2 = 0; q2 < kEpiWarps; ++q2) n4[q2] = __shfl_sync(0xffffffffu, c_l, e_gi * kEpiWarps + q2);
+            for (int q2 = 0; q2 < kPipeWarps; ++q2) nw[q2] = __shfl_sync(0xffffffffu, c_l, w0 + q2);
             if (!over && total <= (uint32_t)kSegCap) {
                 uint2 *seg = cp.lists + ((int64_t)r * cp.NG + cta) * kSegCap;
                 uint32_t mine = 0;
 #pragma unroll
-                for (int q2 = 0; q2 < kEpiWarps; ++q2)
-                    if (q2 == e_q) mine = n4[q2];
+                for (int q2 = 0; q2 < kPipeWarps; ++q2)
+                    if (w0 + q2 == ew_c) mine = nw[q2];
                 for (uint32_t i = lane; i < mine; i += 32) {
                     const uint2 ent = wlist(r, ew_c)[i];
-                    uint32_t rank = gbase + i;
+                    uint32_t rank = pbase + i;
 #pragma unroll
-                    for (int q2 = 0; q2 < kEpiWarps; ++q2) {
-                        if (q2 == e_q) continue;
-                        const uint2 *L2 = wlist(r, e_gi * kEpiWarps + q2);
-                        uint32_t lo = 0, hi = n4[q2];
+                    for (int q2 = 0; q2 < kPipeWarps; ++q2) {
+                        if (w0 + q2 == ew_c) continue;
+                        const uint2 *L2 = wlist(r, w0 + q2);
+                        uint32_t lo = 0, hi = nw[q2];
                         while (lo < hi) {
                             const uint32_t mid = (lo + hi) >> 1;
                             if (L2[mid].y < ent.y) lo = mid + 1; else hi = mid;
