@@ -1006,8 +1006,15 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         // the entry (key 0, position -1): below every candidate's key (the
         // threshold's, or a finite score's), so it is never selected
         if (threadIdx.x == 0) {
+            // the stream's histogram of the row's candidates first, on its own
+            // barrier: the k-th key's bin is found from it while the
+            // segments are still on their way
             mbar_init(copied, 1);
+            mbar_init(copied + 1, 1);
             fence_mbar_init();
+            fence_proxy_async_smem();   // earlier use of the area, before the copy overwrites it
+            mbar_arrive_expect_tx(copied + 1, kWide * 4u);
+            bulk_load(wide, cp.cand_hist + (int64_t)r * kWide, kWide * 4u, copied + 1);
         }
         const uint32_t v = (int)threadIdx.x < NG ? seg_len : 0u;
         const uint32_t vp = (v + 1u) & ~1u;
@@ -1022,16 +1029,8 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             mbar_expect_tx(copied, vp * 8u);
             bulk_load(list + (incl - vp), segs + (int64_t)threadIdx.x * kSegCap, vp * 8u, copied);
         }
-        if (threadIdx.x == NT - 1) {   // and the stream's histogram of the row's candidates
-            mbar_expect_tx(copied, kWide * 4u);
-            bulk_load(wide, cp.cand_hist + (int64_t)r * kWide, kWide * 4u, copied);
-        }
         __syncthreads();   // every expected byte is posted
         if (threadIdx.x == 0) mbar_arrive(copied);
-        mbar_wait(copied, 0, cp.ix.status);
-        if (threadIdx.x < NG && (v & 1u)) list[incl - 1] = make_uint2(0u, 0xFFFFFFFFu);
-        __syncthreads();
-        if (trace && threadIdx.x == 0) trace[8] = globaltimer_ns();
         // ---- the k-th largest key T*, exactly.
         auto is_key = [&](uint32_t j, uint32_t &k) {
             const uint2 e = list[j];
@@ -1119,18 +1118,73 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         };
         uint32_t Tstar = 0u, ties = 0u;
         bool found = false;
+        // the compaction's layout: 32-entry strips, each warp a run of whole
+        // strips, four strips' loads in flight at a time
+        const uint32_t strips = (m + 31) / 32, per_w = (strips + NW - 1) / NW;
+        const uint32_t s0 = min(strips, (uint32_t)warp * per_w), s1 = min(strips, s0 + per_w);
+        constexpr uint32_t kU = 4;
+        bool counted = false;   // sh->warp_a / warp_b hold each warp's keys above T* / equal to it
         {   // from the stream's histogram of the row's candidates above its threshold
             const uint32_t thr_r = keep[kMaxRows] ? keep[r] : __ldcg(cp.ctl + kThr + r);
+            mbar_wait(copied + 1, 0, cp.ix.status);
             find_bin();
             const int B = sh->bin;
             const uint32_t Kb = (uint32_t)K - sh->above, in_b = wide[B];
+            // then the list
+            mbar_wait(copied, 0, cp.ix.status);
+            if (threadIdx.x < NG && (v & 1u)) list[incl - 1] = make_uint2(0u, 0xFFFFFFFFu);
             __syncthreads();
+            if (trace && threadIdx.x == 0) trace[8] = globaltimer_ns();
             if (B < kWide - 1 && in_b <= 32u) {   // not the catch-all bin, and a handful of keys
-                const uint32_t n_keys = gather_keys(
-                    [&](uint32_t k) { return k >= thr_r && ((k - thr_r) >> kCandShift) == (uint32_t)B; });
+                // one pass in the compaction's layout: bin B's keys aside, with
+                // their warp, and per warp the keys of the bins above B (all
+                // above T*, which lies in bin B)
+                if (threadIdx.x == 0) sh->total = 0;
+                __syncthreads();
+                uint32_t above = 0;
+                for (uint32_t q = s0; q < s1; q += kU) {
+                    uint2 ent[kU];
+#pragma unroll
+                    for (uint32_t u = 0; u < kU; ++u) {
+                        const uint32_t j = (q + u) * 32 + lane;
+                        ent[u] = q + u < s1 && j < m ? list[j] : make_uint2(0u, 0xFFFFFFFFu);
+                    }
+#pragma unroll
+                    for (uint32_t u = 0; u < kU; ++u) {
+                        const uint2 e = ent[u];
+                        const bool key = e.y != 0xFFFFFFFFu && e.x >= thr_r;   // not a pad
+                        const uint32_t d = (e.x - thr_r) >> kCandShift;
+                        const bool in_bin = key && d == (uint32_t)B;
+                        above += __popc(__ballot_sync(0xffffffffu, key && d > (uint32_t)B));
+                        const uint32_t bits = __ballot_sync(0xffffffffu, in_bin);
+                        if (bits) {
+                            uint32_t at = 0;
+                            if (lane == 0) at = atomicAdd(&sh->total, (uint32_t)__popc(bits));
+                            at = __shfl_sync(0xffffffffu, at, 0) + __popc(bits & lt);
+                            if (in_bin && at < 32u) {
+                                bin_keys[at] = e.x;
+                                bin_keys[kSmall / 2 + at] = (uint32_t)warp;
+                            }
+                        }
+                    }
+                }
+                if (lane == 0) sh->warp_a[warp] = above;
+                __syncthreads();
+                const uint32_t n_keys = sh->total;
                 if (n_keys == in_b) {   // (always: the histogram counted exactly these keys)
                     rank_small(n_keys, Kb, Tstar, ties);
                     found = true;
+                    if ((int)threadIdx.x < NW) {   // each warp's counts, with its keys of bin B
+                        uint32_t g2 = sh->warp_a[threadIdx.x], e2 = 0;
+                        for (uint32_t i = 0; i < n_keys; ++i)
+                            if (bin_keys[kSmall / 2 + i] == threadIdx.x) {
+                                g2 += bin_keys[i] > Tstar;
+                                e2 += bin_keys[i] == Tstar;
+                            }
+                        sh->warp_a[threadIdx.x] = g2;
+                        sh->warp_b[threadIdx.x] = e2;
+                    }
+                    counted = true;
                 }
             }
         }
@@ -1205,31 +1259,30 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             ties = Krem;
         }
         if (trace && threadIdx.x == 0) trace[9] = globaltimer_ns();
-        // compaction in position order, in 32-entry strips: each warp a run
-        // of whole strips; the keys above T* and the first `ties` keys equal
-        // to it, each at (keys above before it) + min(equal keys before it, ties)
-        const uint32_t strips = (m + 31) / 32, per_w = (strips + NW - 1) / NW;
-        const uint32_t s0 = min(strips, (uint32_t)warp * per_w), s1 = min(strips, s0 + per_w);
-        // (four strips' loads in flight at a time)
-        constexpr uint32_t kU = 4;
-        uint32_t gt = 0, eq = 0;
-        for (uint32_t q = s0; q < s1; q += kU) {
-            uint32_t k[kU];
+        // compaction in position order, in the strips: the keys above T* and
+        // the first `ties` keys equal to it, each at (keys above before it) +
+        // min(equal keys before it, ties); the per-warp counts first (unless
+        // the bin search took them), pads never counted
+        if (!counted) {
+            uint32_t gt = 0, eq = 0;
+            for (uint32_t q = s0; q < s1; q += kU) {
+                uint2 ent[kU];
 #pragma unroll
-            for (uint32_t u = 0; u < kU; ++u) {
-                const uint32_t j = (q + u) * 32 + lane;
-                k[u] = q + u < s1 && j < m ? list[j].x : 0u;
-            }
+                for (uint32_t u = 0; u < kU; ++u) {
+                    const uint32_t j = (q + u) * 32 + lane;
+                    ent[u] = q + u < s1 && j < m ? list[j] : make_uint2(0u, 0xFFFFFFFFu);
+                }
 #pragma unroll
-            for (uint32_t u = 0; u < kU; ++u) {
-                const bool in = q + u < s1 && (q + u) * 32 + lane < m;
-                gt += __popc(__ballot_sync(0xffffffffu, in && k[u] > Tstar));
-                eq += __popc(__ballot_sync(0xffffffffu, in && k[u] == Tstar));
+                for (uint32_t u = 0; u < kU; ++u) {
+                    const bool in = ent[u].y != 0xFFFFFFFFu;
+                    gt += __popc(__ballot_sync(0xffffffffu, in && ent[u].x > Tstar));
+                    eq += __popc(__ballot_sync(0xffffffffu, in && ent[u].x == Tstar));
+                }
             }
-        }
-        if (lane == 0) {
-            sh->warp_a[warp] = gt;
-            sh->warp_b[warp] = eq;
+            if (lane == 0) {
+                sh->warp_a[warp] = gt;
+                sh->warp_b[warp] = eq;
+            }
         }
         __syncthreads();
         uint32_t gb = 0, eb = 0;
@@ -1246,8 +1299,8 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
             }
 #pragma unroll
             for (uint32_t u = 0; u < kU; ++u) {
-                const bool in = q + u < s1 && (q + u) * 32 + lane < m;
                 const uint2 e = ent[u];
+                const bool in = q + u < s1 && (q + u) * 32 + lane < m && e.y != 0xFFFFFFFFu;
                 const uint32_t bg = __ballot_sync(0xffffffffu, in && e.x > Tstar);
                 const uint32_t be = __ballot_sync(0xffffffffu, in && e.x == Tstar);
                 const uint32_t g_before = gb + __popc(bg & lt), e_before = eb + __popc(be & lt);
@@ -1260,7 +1313,10 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         for (int j = kr + threadIdx.x; j < K; j += NT) sel[j] = -1;
     }
     __syncthreads();
-    if (n > K && threadIdx.x == 0) mbar_inval(copied);
+    if (n > K && threadIdx.x == 0) {
+        mbar_inval(copied);
+        mbar_inval(copied + 1);
+    }
     if (c == 0) {
         int32_t *out = cp.tk.idx + (int64_t)r * K;
         for (int j = threadIdx.x; j < K; j += NT) out[j] = sel[j];
