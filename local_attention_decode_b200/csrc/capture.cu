@@ -1461,12 +1461,12 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     __syncthreads();
     mark(6);
     if (trace && threadIdx.x == 0) trace[14] = clock64();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        sync_flag = atomicAdd(ctl + kGridExit, 1u) == G - 1 ? 1u : 0u;
-    }
+    if (threadIdx.x == 0)   // (release: this CTA is done with the words; acquire: the last one sees that)
+        sync_flag = atom_add_acq_rel_gpu(ctl + kGridExit, 1u) == G - 1 ? 1u : 0u;
     __syncthreads();
     if (sync_flag) {   // the last CTA out: every other CTA is done with these words
+        // (nobody in this launch reads them again; the next launch sees them
+        // after this one has completed)
         for (int i = threadIdx.x; i < rows * kWide; i += blockDim.x) cp.cand_hist[i] = 0;
         if (threadIdx.x == 0) {
             ctl[kGridArrive] = 0;
@@ -1478,10 +1478,6 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
                 ctl[kThrPacked + 2 * r + 1] = 0;
             }
             for (int i = 0; i < rows * DSA_Q_HEADS; ++i) ctl[kCombine + i] = 0;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            __threadfence();
             ctl[kGridExit] = 0;
         }
     }
