@@ -204,15 +204,22 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     fence_proxy_async_smem();   // this thread's earlier use of the tiles, before the copies overwrite them
     team_sync(bar);
     // ---- one bulk copy per row: thread r < 64 its key's K and V rows (or
-    //      zeros), thread 64 + r query head r of the group (or zeros)
+    //      zeros), thread 64 + r query head r of the group (or zeros).  The
+    //      expected bytes are posted once per warp, before the warp's copies
+    //      (one transaction-count update per warp and barrier, not one per
+    //      copy: updates of one mbarrier from many threads serialise)
     const int G = p.G;
     if (tid < kChunk) {
         __nv_bfloat16 *dk = sm.k + tid * kQS, *dv = sm.v + tid * kVS;
         const int64_t row = key_row_of_tid;
+        const uint32_t rows_w = __popc(__ballot_sync(0xffffffffu, row >= 0));   // (threads 0..63: whole warps)
+        if (lane == 0 && rows_w > 0) {
+            mbar_expect_tx(&sm.bar[0], rows_w * (DSA_QK_DIM * 2));
+            mbar_expect_tx(&sm.bar[1], rows_w * (DSA_V_DIM * 2));
+        }
+        __syncwarp();
         if (row >= 0) {
-            mbar_expect_tx(&sm.bar[0], DSA_QK_DIM * 2);
             bulk_load(dk, p.K + (row * G + g) * DSA_QK_DIM, DSA_QK_DIM * 2, &sm.bar[0]);
-            mbar_expect_tx(&sm.bar[1], DSA_V_DIM * 2);
             bulk_load(dv, p.V + (row * G + g) * DSA_V_DIM, DSA_V_DIM * 2, &sm.bar[1]);
         } else {
 #pragma unroll
@@ -223,8 +230,9 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     } else if (tid < kChunk + 16) {
         const int r = tid - kChunk;
         __nv_bfloat16 *dq = sm.q + r * kQS;
+        if (r == 0) mbar_expect_tx(&sm.bar[0], (uint32_t)hpg * (DSA_QK_DIM * 2));
+        __syncwarp(0x0000ffffu);   // (threads 64..79: lanes 0..15 of one warp)
         if (r < hpg) {
-            mbar_expect_tx(&sm.bar[0], DSA_QK_DIM * 2);
             bulk_load(dq, p.Q + ((int64_t)bt * DSA_Q_HEADS + g * hpg + r) * DSA_QK_DIM, DSA_QK_DIM * 2, &sm.bar[0]);
         } else {
 #pragma unroll

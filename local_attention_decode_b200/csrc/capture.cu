@@ -1025,10 +1025,16 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
         fence_proxy_async_smem();   // earlier use of the list area, before the copies overwrite it
         __syncthreads();
         const uint2 *segs = cp.lists + (int64_t)r * NG * kSegCap;
-        if (threadIdx.x < NG && vp > 0) {
-            mbar_expect_tx(copied, vp * 8u);
-            bulk_load(list + (incl - vp), segs + (int64_t)threadIdx.x * kSegCap, vp * 8u, copied);
+        {   // the expected bytes posted once per warp, before the warp's copies
+            // (updates of one mbarrier from many threads serialise)
+            uint32_t bytes_w = vp * 8u;   // (0 for threads past the segments)
+#pragma unroll
+            for (int o = 16; o; o >>= 1) bytes_w += __shfl_xor_sync(0xffffffffu, bytes_w, o);
+            if (lane == 0 && bytes_w > 0) mbar_expect_tx(copied, bytes_w);
+            __syncwarp();
         }
+        if (threadIdx.x < NG && vp > 0)
+            bulk_load(list + (incl - vp), segs + (int64_t)threadIdx.x * kSegCap, vp * 8u, copied);
         __syncthreads();   // every expected byte is posted
         if (threadIdx.x == 0) mbar_arrive(copied);
         // ---- the k-th largest key T*, exactly.
