@@ -12,9 +12,10 @@
 // selected keys; the sink column in the softmax).
 //
 // attn_unit: a team of 4 warps takes 64 keys of one KV head, gathers their K
-// and V rows (and the group's query rows) into shared memory with one bulk
-// copy per row on the TMA engine (a per-thread 16-byte copy path costs several
-// times more on this GPU), and computes for the
+// and V rows (and the group's query rows) into shared memory with 16-byte
+// asynchronous copies spread over the team's 128 threads (one bulk copy per
+// row on the TMA engine issues more slowly: about 12 ns per copy on this GPU,
+// 1.8 us for a unit's 144 rows), and computes for the
 // 64/G query heads of that group  S = Q K^T  and  O = softmax_partial(S) V  on
 // the tensor cores (mma.sync m16n8k16 bf16 -> fp32; the query heads of a group
 // form the 16-row M dimension).  Each warp owns 16 keys; the four warps merge
@@ -67,7 +68,6 @@ struct Smem {
     __nv_bfloat16 k[kChunk * kQS];
     __nv_bfloat16 v[kChunk * kVS];
     int64_t row[kChunk];
-    uint64_t bar[2];   // bulk-copy completion: [0] Q and K rows, [1] V rows
     float m[4][16];
     float l[4][16];
     float tm[16];   // the team's result: per head row, the max logit (log2 domain) ...
@@ -179,12 +179,6 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     }
 
     // ---- positions -> cache rows (invalid ones are flagged and masked)
-    if (tid == 0) {   // the team's copy barriers, fresh for this unit
-        mbar_init(&sm.bar[0], 1);
-        mbar_init(&sm.bar[1], 1);
-        fence_mbar_init();
-    }
-    int64_t key_row_of_tid = -1;
     if (tid < kChunk) {
         int64_t row = -1;
         if (tid < nk) {
@@ -199,52 +193,37 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
             }
         }
         sm.row[tid] = row;
-        key_row_of_tid = row;
     }
     fence_proxy_async_smem();   // this thread's earlier use of the tiles, before the copies overwrite them
     team_sync(bar);
-    // ---- one bulk copy per row: thread r < 64 its key's K and V rows (or
-    //      zeros), thread 64 + r query head r of the group (or zeros).  The
-    //      expected bytes are posted once per warp, before the warp's copies
-    //      (one transaction-count update per warp and barrier, not one per
-    //      copy: updates of one mbarrier from many threads serialise)
+    // ---- the rows into shared memory by 16-byte asynchronous copies spread
+    //      over the team's threads: K and Q in one group, V in the next
     const int G = p.G;
-    if (tid < kChunk) {
-        __nv_bfloat16 *dk = sm.k + tid * kQS, *dv = sm.v + tid * kVS;
-        const int64_t row = key_row_of_tid;
-        const uint32_t rows_w = __popc(__ballot_sync(0xffffffffu, row >= 0));   // (threads 0..63: whole warps)
-        if (lane == 0 && rows_w > 0) {
-            mbar_expect_tx(&sm.bar[0], rows_w * (DSA_QK_DIM * 2));
-            mbar_expect_tx(&sm.bar[1], rows_w * (DSA_V_DIM * 2));
-        }
-        __syncwarp();
-        if (row >= 0) {
-            bulk_load(dk, p.K + (row * G + g) * DSA_QK_DIM, DSA_QK_DIM * 2, &sm.bar[0]);
-            bulk_load(dv, p.V + (row * G + g) * DSA_V_DIM, DSA_V_DIM * 2, &sm.bar[1]);
-        } else {
-#pragma unroll
-            for (int c = 0; c < DSA_QK_DIM / 8; ++c) reinterpret_cast<uint4 *>(dk)[c] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int c = 0; c < DSA_V_DIM / 8; ++c) reinterpret_cast<uint4 *>(dv)[c] = make_uint4(0, 0, 0, 0);
-        }
-    } else if (tid < kChunk + 16) {
-        const int r = tid - kChunk;
-        __nv_bfloat16 *dq = sm.q + r * kQS;
-        if (r == 0) mbar_expect_tx(&sm.bar[0], (uint32_t)hpg * (DSA_QK_DIM * 2));
-        __syncwarp(0x0000ffffu);   // (threads 64..79: lanes 0..15 of one warp)
-        if (r < hpg) {
-            bulk_load(dq, p.Q + ((int64_t)bt * DSA_Q_HEADS + g * hpg + r) * DSA_QK_DIM, DSA_QK_DIM * 2, &sm.bar[0]);
-        } else {
-#pragma unroll
-            for (int c = 0; c < DSA_QK_DIM / 8; ++c) reinterpret_cast<uint4 *>(dq)[c] = make_uint4(0, 0, 0, 0);
-        }
+    constexpr int kKC = DSA_QK_DIM / 8, kVC = DSA_V_DIM / 8;   // 16-byte chunks per row
+    for (int c = tid; c < kChunk * kKC; c += 128) {
+        const int rr = c / kKC, cc = c % kKC;
+        const int64_t row = sm.row[rr];
+        __nv_bfloat16 *dst = sm.k + rr * kQS + cc * 8;
+        if (row >= 0) cp_async16(dst, p.K + (row * G + g) * DSA_QK_DIM + cc * 8);
+        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
-    team_sync(bar);   // every expected byte is posted, and the zero rows are written
-    if (tid == 0) {
-        mbar_arrive(&sm.bar[0]);
-        mbar_arrive(&sm.bar[1]);
+    for (int c = tid; c < 16 * kKC; c += 128) {
+        const int rr = c / kKC, cc = c % kKC;
+        __nv_bfloat16 *dst = sm.q + rr * kQS + cc * 8;
+        if (rr < hpg) cp_async16(dst, p.Q + ((int64_t)bt * DSA_Q_HEADS + g * hpg + rr) * DSA_QK_DIM + cc * 8);
+        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
-    mbar_wait(&sm.bar[0], 0, p.status);   // Q and K have landed; V may still be in flight
+    cp_async_commit();
+    for (int c = tid; c < kChunk * kVC; c += 128) {
+        const int rr = c / kVC, cc = c % kVC;
+        const int64_t row = sm.row[rr];
+        __nv_bfloat16 *dst = sm.v + rr * kVS + cc * 8;
+        if (row >= 0) cp_async16(dst, p.V + (row * G + g) * DSA_V_DIM + cc * 8);
+        else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_commit();
+    cp_async_wait_group<1>();   // this thread's Q and K chunks
+    team_sync(bar);             // and everyone's
 
     // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8)
     const int key0 = warp * 16;
@@ -299,7 +278,8 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
     float o[DSA_V_DIM / 8][4];
 #pragma unroll
     for (int nt = 0; nt < DSA_V_DIM / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-    mbar_wait(&sm.bar[1], 0, p.status);
+    cp_async_wait_group<0>();
+    team_sync(bar);
 #pragma unroll
     for (int dp = 0; dp < DSA_V_DIM / 16; ++dp) {
         uint32_t b0, b1, b2, b3;
@@ -317,10 +297,6 @@ __device__ __forceinline__ void attn_unit(const Params &p, Smem &sm, int chunk, 
         sm.l[warp][g0 + 8] = lrow[1];
     }
     team_sync(bar);   // K/V tiles are no longer read: reuse them for the O exchange
-    if (tid == 0) {   // every thread of the team is past its waits
-        mbar_inval(&sm.bar[0]);
-        mbar_inval(&sm.bar[1]);
-    }
     float *so = reinterpret_cast<float *>(sm.k);   // [4 warps][16 rows][kOS] (runs on into sm.v)
     float scale_row[2];
 #pragma unroll
