@@ -990,7 +990,7 @@ __device__ void select_from_candidates(const Params &cp, int r, int c, int32_t *
     const uint32_t lt = (1u << lane) - 1u;
     auto *sh = reinterpret_cast<topk::Shared<NT> *>(work);
     uint32_t *off = reinterpret_cast<uint32_t *>(work + align128(sizeof(topk::Shared<NT>)));
-    uint64_t *copied = reinterpret_cast<uint64_t *>(off + ((NG + 1 + 31) & ~31));   // bulk-copy barrier
+    uint64_t *copied = reinterpret_cast<uint64_t *>(off + ((NG + 1 + 31) & ~31));   // bulk-copy barriers
     uint2 *list = reinterpret_cast<uint2 *>(copied + 2);   // (order key, position), 16-byte aligned
     uint32_t *wide = reinterpret_cast<uint32_t *>(list + kListCap);   // [kWide] histogram
     uint32_t *bin_keys = wide + kWide;                                // [kSmall] keys of T*'s bin
@@ -1401,8 +1401,9 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
                 if (tm < kTeams) {
                     for (int u = c + tm * C; u < upr; u += kTeams * C) {
                         const int g = u / splits, split = u % splits;
-                        attn::team_unit(cp.at, teams[tm], split, g, r, tid, 1 + tm, cp.sink, cp.O, cp.lse, sel);
-                        if (splits > 1 && tid == 0) atomicAdd(ctl + kCombine + r * DSA_Q_HEADS + g, 1u);
+                        attn::attn_unit(cp.at, teams[tm], split, g, r, tid, 1 + tm, sel, true, cp.sink, cp.O, cp.lse);
+                        attn::team_sync(1 + tm);   // every thread's stores are done; the count releases them
+                        if (splits > 1 && tid == 0) red_release_gpu_add(ctl + kCombine + r * DSA_Q_HEADS + g, 1u);
                     }
                     if (tm == 0) mark(5);
                     // each unit's team then combines one slice of its KV head's

@@ -67,6 +67,13 @@ BarrierCfg barrier_cfg();
 // marks, else NULL (host).
 uint64_t *phase_trace(int grid);
 
+// Reduction with release semantics (no value returned, the thread does not
+// wait for it): the executing thread's earlier accesses, and those ordered
+// before them by a block barrier, are visible before the add.
+__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Bounded wait of thread 0 of a CTA until *bar >= target (acquire); false and
 // the timeout status when the limit runs out.
 __device__ __forceinline__ bool spin_until_at_least(const uint32_t *bar, uint32_t target, uint64_t limit_ns,
@@ -96,7 +103,7 @@ __device__ __forceinline__ bool grid_sync(uint32_t *bar, uint32_t target, const 
     if (threadIdx.x == 0) {
         // the release arrival covers the CTA's writes (ordered before it by the
         // block barrier); the acquire load of the count covers everyone else's
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+        red_release_gpu_add(bar, 1u);
         const bool ok = spin_until_at_least(bar, target + cfg.extra, cfg.limit_ns, status);
         *flag = ok ? 1u : 0u;
     }
