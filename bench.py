@@ -938,8 +938,7 @@ def run_e2e(args, dsa, torch, layers, dev, stream, sm_scale, ws, flush):
         w_i, kv_i = layers[i % R]
         d_in.copy_(h_in, non_blocking=True)
         dsa.dsa_index_produce(d_kin, d_qin, ln_w, ln_b, 1e-5, 42, 1e7, kv_i, d_pos, q8, qs, ws_p)
-        w_i.K[row].copy_(d_K, non_blocking=True)
-        w_i.V[row].copy_(d_V, non_blocking=True)
+        torch._foreach_copy_([w_i.K[row], w_i.V[row]], [d_K, d_V], non_blocking=True)   # (one launch)
         dsa.dsa_layer_decode(q8, qs, d_w, d_Q, kv_i, d_pos, L, TOP_K, w_i.sink, sm_scale, O, None, idx, cnt, ws)
         h_out.copy_(d_out, non_blocking=True)
 
@@ -1006,7 +1005,7 @@ def run_e2e(args, dsa, torch, layers, dev, stream, sm_scale, ws, flush):
     return {"value": throughput(B * T, K, world, total_s), "unit": "tok/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": total_s * 1e3 / K, "steps": K,
             "per_step": "1 pinned H2D copy of the token's raw inputs; dsa_index_produce (index key into the cache, "
-                        "index query codes); 2 device copies of the K/V rows into the cache; dsa_layer_decode; "
+                        "index query codes); the K/V rows copied into the cache (one launch); dsa_layer_decode; "
                         "1 D2H copy of O and the selection -- " + graph_note,
             "l2": f"inputs larger than L2: {R} layers' caches in rotation, no flush",
             "ms_per_step_isolated_median": iso_ms,

@@ -839,9 +839,7 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     // the segment is the length of the lists of the pipelines before its
     // pipeline (their position ranges are disjoint and in order) plus the
     // entries of its pipeline's eight lists (which interleave: tiles by
-    // group, rows within a tile by warp) with a lower position.  The candidates' K and V rows (all KV heads) go
-    // on their way into L2 as well, while the grid meets: HBM is idle after
-    // the stream, and the selection's rows are among these.
+    // group, rows within a tile by warp) with a lower position.
     constexpr int kLists = kGroups * kEpiWarps;
     constexpr int kPipeWarps = kMaxGroups * kEpiWarps;   // the epilogue warps of one pipeline
     static_assert(kLists <= 32, "one list length per lane");
@@ -882,11 +880,6 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
                         rank += lo;
                     }
                     seg[rank] = ent;
-                    int64_t krow;
-                    if (attn::key_row(cp.at, r / T, (int64_t)ent.y, &krow)) {
-                        bulk_prefetch_l2(cp.at.K + krow * cp.at.G * DSA_QK_DIM, (uint32_t)(cp.at.G * DSA_QK_DIM * 2));
-                        bulk_prefetch_l2(cp.at.V + krow * cp.at.G * DSA_V_DIM, (uint32_t)(cp.at.G * DSA_V_DIM * 2));
-                    }
                 }
             }
             if (ew_c == 0 && lane == 0) {   // the row's count in this CTA
@@ -917,6 +910,19 @@ __device__ void combine_piece(const Params &cp, int bt, int g, int piece, int ti
     float *w = st;                            // [nh][splits] m_j, then the weights w_j
     float *ls = st + hpg * kMaxSplits;        // [nh][splits] l_j
     float *hs = ls + hpg * kMaxSplits;        // [nh][2]: M, L per head
+    // this thread's first element's split values, loaded together with the
+    // statistics (one round trip to L2 for both)
+    float v0[kMaxSplits];
+    {
+        const int e = lo + tid;
+        if (e < hi) {
+            const int hh = e / DSA_V_DIM - h_lo, col = e % DSA_V_DIM;
+            const int64_t gw = (int64_t)bt * DSA_Q_HEADS + g * hpg + h_lo + hh;
+            const float *po = at.part_o + gw * splits * DSA_V_DIM + col;
+#pragma unroll
+            for (int j = 0; j < kMaxSplits; ++j) v0[j] = j < splits ? __ldcg(po + (int64_t)j * DSA_V_DIM) : 0.f;
+        }
+    }
     // the heads' split statistics -> weights, M and the denominators
     for (int i = tid; i < nh * splits; i += 128) {
         const int hh = i / splits, j = i % splits;
@@ -960,8 +966,13 @@ __device__ void combine_piece(const Params &cp, int bt, int g, int piece, int ti
         const int64_t gw = (int64_t)bt * DSA_Q_HEADS + g * hpg + h_lo + hh;
         const float *po = at.part_o + gw * splits * DSA_V_DIM + col;
         float v[kMaxSplits];
+        if (e == lo + tid) {
 #pragma unroll
-        for (int j = 0; j < kMaxSplits; ++j) v[j] = j < splits ? __ldcg(po + (int64_t)j * DSA_V_DIM) : 0.f;
+            for (int j = 0; j < kMaxSplits; ++j) v[j] = v0[j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < kMaxSplits; ++j) v[j] = j < splits ? __ldcg(po + (int64_t)j * DSA_V_DIM) : 0.f;
+        }
         float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < kMaxSplits; ++j) {
