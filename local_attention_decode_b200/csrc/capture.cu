@@ -235,10 +235,10 @@ __device__ uint32_t row_threshold(const uint32_t *local, int64_t n, int K, float
 // capture (see the file comment).  All kThreads threads call it.  On return
 // nothing is in flight, TMEM is released and the mbarriers are invalidated;
 // keep[0 .. kMaxRows) holds the rows' thresholds if keep[kMaxRows] != 0.
-template <int TQ>
+template <int TQ, class AfterWait>
 __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorMap *tmap_ks_p,
                                     const CUtensorMap *tmap_q_p, const Params &cp, uint8_t *smem, int cta, int ncta,
-                                    uint32_t *keep) {
+                                    uint32_t *keep, AfterWait &&after_wait) {
     using namespace indexer;
     const indexer::Params &p = cp.ix;
     const CUtensorMap &tmap_k = *tmap_k_p, &tmap_q = *tmap_q_p;
@@ -270,10 +270,11 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     const int warp = warp_id(), lane = lane_id();
     const uint32_t lt = (1u << lane) - 1u;
 
-    // The prologue has one block barrier: thread 0 reads the (at most
+    // The prologue has one block barrier: thread 0 builds the mbarriers while
+    // warp kPipes allocates TMEM and the other threads clear the shared words;
+    // then (after the dependent-launch wait) thread 0 reads the (at most
     // kMaxRows) query positions, all loads in flight together, and builds the
-    // per-sequence tables and the mbarriers while warp kPipes allocates TMEM
-    // and the other threads clear the shared words.
+    // per-sequence tables.
     // TMEM: the accumulators, then the backlog: the order keys of the first
     // back_cap tiles of each epilogue group, kept until the thresholds come
     // (column acc_cols + (group * back_cap + tile) * T + query, lane = key row)
@@ -282,10 +283,6 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     uint32_t tmem_cols = 32;
     while (tmem_cols < (uint32_t)(acc_cols + kGroups * back_cap * T)) tmem_cols <<= 1;
     if (threadIdx.x == 0) {
-        int32_t qv[kMaxRows];
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) qv[r] = r < rows ? __ldg(p.q_pos + r) : 0;
-        // (the barriers while the loads are in flight)
         for (int pp = 0; pp < kPipes; ++pp) {
             for (int s = 0; s < S; ++s) {
                 mbar_init(&bars->full[pp][s], 1);
@@ -302,6 +299,23 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         fence_mbar_init();
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_q);
+    }
+    if (warp == kPipes) {
+        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
+    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
+    for (int j = threadIdx.x; j < kCapWords; j += blockDim.x) thr_s[j] = 0;
+    // Everything above touches only this CTA's shared memory and TMEM: under
+    // a programmatic dependent launch it overlaps the previous grid's tail.
+    // From here on the kernel reads what that grid may have written.
+    pdl_wait();
+    after_wait();
+    if (threadIdx.x == 0) {
+        int32_t qv[kMaxRows];
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r) qv[r] = r < rows ? __ldg(p.q_pos + r) : 0;
         const int64_t cap = p.block_table ? (int64_t)p.max_pages * p.page_size : p.seq_stride;
         int pre = 0;
         tile_pre[0] = 0;
@@ -329,13 +343,6 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
         for (int r = 0; r < kMaxRows; ++r)
             if (r < rows) row_qpos[r] = qv[r];
     }
-    if (warp == kPipes) {
-        tmem_alloc(tmem_slot, tmem_cols);
-        tmem_relinquish();
-    }
-    for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
-    if (threadIdx.x < 8) misc[threadIdx.x] = 0;
-    for (int j = threadIdx.x; j < kCapWords; j += blockDim.x) thr_s[j] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1350,23 +1357,27 @@ dsa_layer_capture_kernel(const __grid_constant__ CUtensorMap tmap_k, const __gri
     __shared__ uint32_t sync_flag;
     __shared__ uint32_t thr_keep[kMaxRows + 1];
     if (threadIdx.x == 0) thr_keep[kMaxRows] = 0u;
-    pdl_begin();
+    pdl_launch_dependents();   // (the wait comes once the CTA's own set-up is done)
     const uint32_t G = gridDim.x;
     uint32_t *status = cp.ix.status;
     uint32_t *ctl = cp.ctl;
-    const uint32_t status_at_entry = load_status(status);
+    uint32_t status_at_entry = 0;
     uint64_t *trace = cp.trace ? cp.trace + blockIdx.x * DSA_TRACE_MARKS : nullptr;
     auto mark = [&](int i) {
         if (trace && threadIdx.x == 0) trace[i] = globaltimer_ns();
     };
-    if (trace && threadIdx.x == 0) {
-        for (int i = 1; i < DSA_TRACE_MARKS; ++i) trace[i] = 0;
-        trace[0] = globaltimer_ns();
-        trace[13] = clock64();
-    }
+    // run by every thread right after the dependent-launch wait
+    auto after_wait = [&]() {
+        status_at_entry = load_status(status);
+        if (trace && threadIdx.x == 0) {
+            for (int i = 1; i < DSA_TRACE_MARKS; ++i) trace[i] = 0;
+            trace[0] = globaltimer_ns();
+            trace[13] = clock64();
+        }
+    };
 
     // ---- phase 1: key stream, sample, candidates
-    run_indexer_capture<TQ>(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G, thr_keep);
+    run_indexer_capture<TQ>(&tmap_k, &tmap_ks, &tmap_q, cp, smem, blockIdx.x, G, thr_keep, after_wait);
     mark(15);
     if (status_at_entry & kNeedsInitBit) {
         if (threadIdx.x == 0) flag_timeout(status);
