@@ -307,9 +307,23 @@ __device__ void run_indexer_capture(const CUtensorMap *tmap_k_p, const CUtensorM
     for (int j = threadIdx.x; j < rows * kHistStride; j += blockDim.x) hist[j] = 0;
     if (threadIdx.x < 8) misc[threadIdx.x] = 0;
     for (int j = threadIdx.x; j < kCapWords; j += blockDim.x) thr_s[j] = 0;
-    // Everything above touches only this CTA's shared memory and TMEM: under
-    // a programmatic dependent launch it overlaps the previous grid's tail.
-    // From here on the kernel reads what that grid may have written.
+    // One sequence in a contiguous cache: the first two tiles each pipeline
+    // streams when the query sits at the last position the cache holds (a
+    // decode step), on their way into L2 -- a guess from the sizes alone, so
+    // it reads nothing the previous grid may be writing; a wrong guess only
+    // costs the prefetch.
+    if (B == 1 && p.block_table == nullptr && warp < kPipes && lane == 0) {
+        const int total_g = (int)((p.Lmax + kTile - 1) / kTile);
+        const int per_g = total_g / ncta, rem_g = total_g % ncta;
+        const int n_g = per_g + (cta < rem_g ? 1 : 0), half_g = (n_g + kPipes - 1) / kPipes;
+        const int first = cta * per_g + min(cta, rem_g) + min(n_g, warp * half_g);
+        const int cnt = min(n_g, (warp + 1) * half_g) - min(n_g, warp * half_g);
+        for (int i = 0; i < min(cnt, 2); ++i) tma_prefetch_2d(&tmap_k, 0, (first + i) * kTile);
+    }
+    // Everything above touches only this CTA's shared memory and TMEM (and
+    // the prefetch): under a programmatic dependent launch it overlaps the
+    // previous grid's tail. From here on the kernel reads what that grid may
+    // have written.
     pdl_wait();
     after_wait();
     if (threadIdx.x == 0) {
